@@ -1,0 +1,140 @@
+"""Seeded synthetic inputs for the SSD scan workloads.
+
+This module only draws random numbers; it holds none of the scan's arithmetic.
+Both the CUDA path's tests/benchmark and the oracle are fed from it.
+
+Distributions (the pages' workloads are HFT-style tick sequences of 256-1024
+steps with d_state 64/128 and chunk 256; the proprietary market data they
+train on is not available, so these draws stand in for it):
+
+  x, B, C  ~ N(0, 1)
+  dt_raw   ~ N(0, 1)
+  dt_bias  = softplus^-1(v), v ~ U[1e-3, 0.1]      (inverse-softplus init of
+             the dt bias, "MAMBA-2 Implementation Gaps", Gap 3)
+  A_h      = -u, u ~ U[1, 16]    (a negative scalar per head)
+  D_h      ~ N(0, 1)
+  init     ~ N(0, 0.1^2) where a workload carries an initial state
+
+Draw order is fixed: x, dt_raw, B, C, dt_bias, A, D, init.  Everything is drawn
+in fp32 on a CPU torch.Generator and then cast to the workload dtype, so the
+oracle can read the exact rounded values.
+"""
+from __future__ import annotations
+
+import dataclasses
+import math
+
+import torch
+
+
+@dataclasses.dataclass(frozen=True)
+class FwdConfig:
+    name: str
+    batch: int
+    seqlen: int
+    nheads: int
+    headdim: int
+    dstate: int
+    ngroups: int
+    chunk: int
+    dtype: torch.dtype
+    init_state: bool = False
+    return_final: bool = False
+
+    @property
+    def tokens(self) -> int:
+        return self.batch * self.seqlen
+
+
+@dataclasses.dataclass(frozen=True)
+class DecodeConfig:
+    name: str
+    batch: int
+    nheads: int
+    headdim: int
+    dstate: int
+    ngroups: int
+    steps: int
+    dtype: torch.dtype
+
+
+FWD_CONFIGS = {
+    "fwd_f32_small": FwdConfig("fwd_f32_small", 1, 256, 4, 16, 16, 1, 64, torch.float32),
+    "fwd_bf16_b4_L1024": FwdConfig("fwd_bf16_b4_L1024", 4, 1024, 24, 64, 64, 1, 256,
+                                   torch.bfloat16),
+    "fwd_bf16_b8_L4096_init": FwdConfig("fwd_bf16_b8_L4096_init", 8, 4096, 32, 64, 128, 1,
+                                        256, torch.bfloat16, init_state=True,
+                                        return_final=True),
+    "fwd_bf16_b1_L65536_G8": FwdConfig("fwd_bf16_b1_L65536_G8", 1, 65536, 80, 64, 128, 8,
+                                       256, torch.bfloat16),
+}
+DECODE_CONFIGS = {
+    "decode_b256_H80": DecodeConfig("decode_b256_H80", 256, 80, 64, 128, 8, 1024,
+                                    torch.bfloat16),
+}
+# the seed offset of each workload (seed = 1234 + offset)
+SEED_OFFSET = {"fwd_f32_small": 0, "fwd_bf16_b4_L1024": 1, "fwd_bf16_b8_L4096_init": 2,
+               "fwd_bf16_b1_L65536_G8": 3, "decode_b256_H80": 4}
+
+
+def _uniform(gen, shape, lo, hi):
+    return torch.rand(shape, generator=gen, dtype=torch.float32) * (hi - lo) + lo
+
+
+def _inv_softplus(v: torch.Tensor) -> torch.Tensor:
+    v64 = v.double()
+    return (v64 + torch.log(-torch.expm1(-v64))).float()
+
+
+def head_params(gen: torch.Generator, nheads: int):
+    """dt_bias, A, D per head (fp32), drawn in the fixed order."""
+    dt_bias = _inv_softplus(_uniform(gen, (nheads,), 1e-3, 0.1))
+    A = -_uniform(gen, (nheads,), 1.0, 16.0)
+    D = torch.randn((nheads,), generator=gen, dtype=torch.float32)
+    return dt_bias, A, D
+
+
+def make_fwd_inputs(batch, seqlen, nheads, headdim, dstate, ngroups, dtype,
+                    seed: int, init_state: bool = False) -> dict:
+    """CPU tensors for one forward call (x, dt, B, C in ``dtype``; A, D,
+    dt_bias, init_state fp32)."""
+    gen = torch.Generator().manual_seed(seed)
+    x = torch.randn((batch, seqlen, nheads, headdim), generator=gen).to(dtype)
+    dt = torch.randn((batch, seqlen, nheads), generator=gen).to(dtype)
+    B = torch.randn((batch, seqlen, ngroups, dstate), generator=gen).to(dtype)
+    C = torch.randn((batch, seqlen, ngroups, dstate), generator=gen).to(dtype)
+    dt_bias, A, D = head_params(gen, nheads)
+    init = None
+    if init_state:
+        init = torch.randn((batch, nheads, headdim, dstate), generator=gen) * 0.1
+    return dict(x=x, dt=dt, A=A, B=B, C=C, D=D, dt_bias=dt_bias, init_state=init)
+
+
+def make_config_inputs(cfg: FwdConfig, seed: int | None = None) -> dict:
+    if seed is None:
+        seed = 1234 + SEED_OFFSET.get(cfg.name, 0)
+    return make_fwd_inputs(cfg.batch, cfg.seqlen, cfg.nheads, cfg.headdim, cfg.dstate,
+                           cfg.ngroups, cfg.dtype, seed, cfg.init_state)
+
+
+def make_decode_params(batch, nheads, headdim, dstate, seed: int) -> dict:
+    """Initial fp32 state ~ N(0, 0.1^2) and the per-head parameters."""
+    gen = torch.Generator().manual_seed(seed)
+    dt_bias, A, D = head_params(gen, nheads)
+    state = torch.randn((batch, nheads, headdim, dstate), generator=gen) * 0.1
+    return dict(state=state, A=A, D=D, dt_bias=dt_bias)
+
+
+def make_decode_step(batch, nheads, headdim, dstate, ngroups, dtype, seed: int,
+                     step: int) -> dict:
+    """Inputs of one decode step (x, dt, B, C in ``dtype``)."""
+    gen = torch.Generator().manual_seed(seed * 1_000_003 + step)
+    x = torch.randn((batch, nheads, headdim), generator=gen).to(dtype)
+    dt = torch.randn((batch, nheads), generator=gen).to(dtype)
+    B = torch.randn((batch, ngroups, dstate), generator=gen).to(dtype)
+    C = torch.randn((batch, ngroups, dstate), generator=gen).to(dtype)
+    return dict(x=x, dt=dt, B=B, C=C)
+
+
+def nchunks(seqlen: int, chunk: int) -> int:
+    return int(math.ceil(seqlen / chunk))

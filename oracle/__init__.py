@@ -1,0 +1,154 @@
+"""fp64 CPU oracle for the Mamba-2 SSD selective scan (test infrastructure).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product path (the CUDA library and
+its Python binding) never imports, loads or calls it, and it shares no code
+with that path.  See ``ssd_oracle.c`` for what each function computes and which
+passage of the pages it follows.
+
+Arrays may be numpy arrays or CPU torch tensors of any float dtype; they are
+converted to contiguous float64 before the call, so a bf16 input reaches the
+oracle as its exact value.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import sys
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "ssd_oracle.c")
+_LIB_NAME = "liboracle.so"
+
+
+def build(mutant: int = 0, out_dir: str | None = None, force: bool = False) -> str:
+    """Compile ssd_oracle.c with gcc (fp64, OpenMP, no FMA contraction).
+
+    ``mutant`` > 0 builds a deliberately wrong variant for the pin-strength
+    test; those land in ``out_dir`` and never replace the real oracle.
+    """
+    out_dir = out_dir or _HERE
+    name = _LIB_NAME if mutant == 0 else f"liboracle_mut{mutant}.so"
+    out = os.path.join(out_dir, name)
+    if not force and os.path.exists(out) and os.path.getmtime(out) >= os.path.getmtime(_SRC):
+        return out
+    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp",
+           "-ffp-contract=off", "-fno-fast-math", f"-DORACLE_MUTANT={mutant}",
+           _SRC, "-o", out + ".tmp", "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(out + ".tmp", out)
+    return out
+
+
+_dp = ctypes.POINTER(ctypes.c_double)
+_i64 = ctypes.c_int64
+
+
+class Oracle:
+    """ctypes handle on one build of the oracle library."""
+
+    def __init__(self, path: str):
+        self.path = path
+        lib = ctypes.CDLL(path)
+        lib.oracle_softplus.restype = ctypes.c_double
+        lib.oracle_softplus.argtypes = [ctypes.c_double]
+        lib.oracle_num_threads.restype = ctypes.c_int
+        lib.oracle_ssd_fwd.restype = None
+        lib.oracle_ssd_fwd.argtypes = [_i64] * 6 + [_dp] * 10
+        lib.oracle_ssd_chunked.restype = None
+        lib.oracle_ssd_chunked.argtypes = [_i64] * 7 + [_dp] * 14
+        lib.oracle_state_update.restype = None
+        lib.oracle_state_update.argtypes = [_i64] * 5 + [_dp] * 9
+        self.lib = lib
+
+    # -- helpers ---------------------------------------------------------
+    @staticmethod
+    def _f64(a):
+        if a is None:
+            return None
+        if hasattr(a, "detach"):  # torch tensor
+            a = a.detach().to("cpu").double().numpy()
+        return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+    @staticmethod
+    def _ptr(a):
+        if a is None:
+            return None
+        return a.ctypes.data_as(_dp)
+
+    def num_threads(self) -> int:
+        return int(self.lib.oracle_num_threads())
+
+    def softplus(self, u: float) -> float:
+        return float(self.lib.oracle_softplus(float(u)))
+
+    # -- the recurrence --------------------------------------------------
+    def ssd_fwd(self, x, dt, A, B, C, D=None, dt_bias=None, init_state=None):
+        """Token-by-token recurrence.  Returns (y, final_state) as float64.
+
+        x [b,L,H,P], dt [b,L,H] (raw, before softplus), A [H], B/C [b,L,G,N],
+        D/dt_bias [H] or None, init_state [b,H,P,N] or None.
+        """
+        x, dt, A, B, C = (self._f64(t) for t in (x, dt, A, B, C))
+        D, dt_bias, init = self._f64(D), self._f64(dt_bias), self._f64(init_state)
+        b, L, H, P = x.shape
+        G, N = B.shape[2], B.shape[3]
+        y = np.zeros((b, L, H, P))
+        fin = np.zeros((b, H, P, N))
+        self.lib.oracle_ssd_fwd(b, L, H, P, N, G, *(self._ptr(t) for t in (
+            x, dt, A, B, C, D, dt_bias, init, y, fin)))
+        return y, fin
+
+    def ssd_chunked(self, x, dt, A, B, C, D=None, dt_bias=None, init_state=None,
+                    chunk: int = 256):
+        """Chunked restatement.  Returns a dict with dt, cumA [b,H,nc,Q],
+        S, Hin [b,nc,H,P,N], y [b,L,H,P] and final_state [b,H,P,N]."""
+        x, dt, A, B, C = (self._f64(t) for t in (x, dt, A, B, C))
+        D, dt_bias, init = self._f64(D), self._f64(dt_bias), self._f64(init_state)
+        b, L, H, P = x.shape
+        G, N = B.shape[2], B.shape[3]
+        Q = int(chunk)
+        nc = (L + Q - 1) // Q
+        out = {
+            "dt": np.zeros((b, H, nc, Q)), "cumA": np.zeros((b, H, nc, Q)),
+            "S": np.zeros((b, nc, H, P, N)), "Hin": np.zeros((b, nc, H, P, N)),
+            "y": np.zeros((b, L, H, P)), "final_state": np.zeros((b, H, P, N)),
+        }
+        self.lib.oracle_ssd_chunked(b, L, H, P, N, G, Q, *(self._ptr(t) for t in (
+            x, dt, A, B, C, D, dt_bias, init, out["dt"], out["cumA"], out["S"],
+            out["Hin"], out["y"], out["final_state"])))
+        return out
+
+    def state_update(self, state, x, dt, A, B, C, D=None, dt_bias=None):
+        """One decode step.  Returns (new_state, y) as float64; the input
+        state is not modified.  state [b,H,P,N], x [b,H,P], dt [b,H],
+        B/C [b,G,N]."""
+        st = self._f64(state).copy()
+        x, dt, A, B, C = (self._f64(t) for t in (x, dt, A, B, C))
+        D, dt_bias = self._f64(D), self._f64(dt_bias)
+        b, H, P, N = st.shape
+        G = B.shape[1]
+        y = np.zeros((b, H, P))
+        self.lib.oracle_state_update(b, H, P, N, G, *(self._ptr(t) for t in (
+            st, x, dt, A, B, C, D, dt_bias, y)))
+        return st, y
+
+
+_DEFAULT: Oracle | None = None
+
+
+def load(mutant: int = 0, out_dir: str | None = None) -> Oracle:
+    """Build (if stale) and load the oracle, or a numbered mutant of it."""
+    global _DEFAULT
+    if mutant == 0 and out_dir is None:
+        if _DEFAULT is None:
+            _DEFAULT = Oracle(build())
+        return _DEFAULT
+    return Oracle(build(mutant=mutant, out_dir=out_dir))
+
+
+if __name__ == "__main__":  # python -m oracle  -> build it
+    print(build(force="--force" in sys.argv))

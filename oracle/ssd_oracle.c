@@ -1,0 +1,284 @@
+/*
+ * ssd_oracle.c -- fp64 CPU oracle for the Mamba-2 SSD selective scan.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may link, load or
+ * call this file: only the tests, the smoke check and the benchmark's
+ * CPU-baseline leg use it.  It shares no code, header, table or helper with
+ * the CUDA library; its inputs arrive as plain double arrays.
+ *
+ * What it computes (sources are the five pages this project is built from):
+ *
+ *   dt_t  = softplus(dt_raw_t + dt_bias_h)
+ *           ("MAMBA-2 Reference Implementations Comparison", section 3.2
+ *            "Selective Scan Algorithm"; "MAMBA-2 Implementation Gaps",
+ *            Gap 3 "dt (Time Step) Parameter")
+ *   a_t   = exp(dt_t * A_h), A_h a scalar per head
+ *           (same passages; scalar-times-identity A per "MAMBA-2 Reference
+ *            Implementations Comparison", section 2.2)
+ *   h_t   = a_t * h_{t-1} + dt_t * x_t B_t^T      (Euler input, B * dt)
+ *   y_t   = C_t . h_t + D_h * x_t
+ *           (D skip: "MAMBA-2 Implementation Gaps", Gap 4)
+ *
+ * Layouts (row-major, innermost last):
+ *   x, y       [batch, seqlen, nheads, headdim]
+ *   dt_raw     [batch, seqlen, nheads]
+ *   B, C       [batch, seqlen, ngroups, dstate]
+ *   A, D, bias [nheads]
+ *   state      [batch, nheads, headdim, dstate]
+ * Head h reads group g = h / (nheads / ngroups).
+ *
+ * Functions:
+ *   oracle_ssd_fwd       the plain token-by-token recurrence (the definition)
+ *   oracle_ssd_chunked   the chunked restatement (local chunk states, carry
+ *                        of the last state across chunks, per-chunk output)
+ *                        that also returns each step's intermediates
+ *   oracle_state_update  one decode step on a carried state (the recurrence
+ *                        body applied once; the page "MAMBA-2 Reference
+ *                        Implementations Comparison", section 1.3, names the
+ *                        Mamba2Cache this state lives in)
+ *
+ * Pins (tests/, CPU only): the masked-attention (quadratic) dual form by brute
+ * force, the A = 0 cumulative-sum closed form, chunk-size invariance, split /
+ * resume, decode == forward, special cases (C = 0, x = 0, full decay, L = 1),
+ * causality, and a hand-derived half-decay example.
+ *
+ * ORACLE_MUTANT selects a deliberately wrong variant for the test that checks
+ * the pins catch plausible mistakes; the default build (0) is the oracle.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#ifndef ORACLE_MUTANT
+#define ORACLE_MUTANT 0
+#endif
+
+/* softplus(u) = log(1 + e^u), evaluated without overflow. */
+double oracle_softplus(double u) {
+#if ORACLE_MUTANT == 8
+    return exp(u);
+#else
+    return (u > 0.0 ? u : 0.0) + log1p(exp(-fabs(u)));
+#endif
+}
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+static double dt_of(const double* dt_raw, const double* dt_bias,
+                    int64_t i, int64_t h) {
+#if ORACLE_MUTANT == 5
+    (void)dt_bias; (void)h;
+    return oracle_softplus(dt_raw[i]);
+#else
+    return oracle_softplus(dt_raw[i] + (dt_bias ? dt_bias[h] : 0.0));
+#endif
+}
+
+static int64_t group_of(int64_t h, int64_t H, int64_t G) {
+#if ORACLE_MUTANT == 6
+    (void)H;
+    return h % G;
+#else
+    return h / (H / G);
+#endif
+}
+
+/* The recurrence, token by token.  init may be NULL (zero state); D and
+ * dt_bias may be NULL (zero); final_state may be NULL. */
+void oracle_ssd_fwd(int64_t batch, int64_t L, int64_t H, int64_t P,
+                    int64_t N, int64_t G,
+                    const double* x, const double* dt_raw, const double* A,
+                    const double* B, const double* C, const double* D,
+                    const double* dt_bias, const double* init,
+                    double* y, double* final_state) {
+    int64_t bh;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (bh = 0; bh < batch * H; ++bh) {
+        const int64_t b = bh / H, h = bh % H, g = group_of(h, H, G);
+        double* S = (double*)malloc(sizeof(double) * (size_t)(P * N));
+        const double Dh = D ? D[h] : 0.0;
+        if (init && ORACLE_MUTANT != 9)
+            memcpy(S, init + bh * P * N, sizeof(double) * (size_t)(P * N));
+        else
+            memset(S, 0, sizeof(double) * (size_t)(P * N));
+        for (int64_t t = 0; t < L; ++t) {
+            const int64_t it = (b * L + t) * H + h;
+            const double dt = dt_of(dt_raw, dt_bias, it, h);
+#if ORACLE_MUTANT == 4
+            const double a = exp(-dt * A[h]);
+#else
+            const double a = exp(dt * A[h]);
+#endif
+            const double* xt = x + it * P;
+            const double* Bt = B + ((b * L + t) * G + g) * N;
+            const double* Ct = C + ((b * L + t) * G + g) * N;
+#if ORACLE_MUTANT == 3
+            { const double* tmp = Bt; Bt = Ct; Ct = tmp; }
+#endif
+            double* yt = y + it * P;
+            for (int64_t p = 0; p < P; ++p) {
+                double* Sp = S + p * N;
+                double acc = 0.0;
+#if ORACLE_MUTANT == 2
+                for (int64_t n = 0; n < N; ++n) acc += Sp[n] * Ct[n];
+#endif
+                for (int64_t n = 0; n < N; ++n) {
+#if ORACLE_MUTANT == 7
+                    Sp[n] = a * Sp[n] + xt[p] * Bt[n];
+#else
+                    Sp[n] = a * Sp[n] + dt * xt[p] * Bt[n];
+#endif
+                }
+#if ORACLE_MUTANT != 2
+                for (int64_t n = 0; n < N; ++n) acc += Sp[n] * Ct[n];
+#endif
+#if ORACLE_MUTANT == 1
+                yt[p] = acc;
+#else
+                yt[p] = acc + Dh * xt[p];
+#endif
+            }
+        }
+        if (final_state)
+            memcpy(final_state + bh * P * N, S, sizeof(double) * (size_t)(P * N));
+        free(S);
+    }
+}
+
+/*
+ * The chunked restatement: the sequence is cut into chunks of Q tokens (the
+ * last one may be shorter) and processed in the three phases the SSD chunk
+ * scan describes ("MAMBA-2 Implementation Gaps", Gap 1: a local, parallel
+ * "diagonal block" per chunk, an inter-chunk carry of the last state, then the
+ * output), with dt and the in-chunk cumulative sum of dt * A made explicit.
+ *
+ * Outputs (any may be NULL except y):
+ *   dt_out, cumA_out  [batch, H, nc, Q]  (entries past a short tail are 0)
+ *   S_out             [batch, nc, H, P, N] local state of each chunk
+ *   Hin_out           [batch, nc, H, P, N] state entering each chunk
+ *   final_state       [batch, H, P, N]
+ */
+void oracle_ssd_chunked(int64_t batch, int64_t L, int64_t H, int64_t P,
+                        int64_t N, int64_t G, int64_t Q,
+                        const double* x, const double* dt_raw, const double* A,
+                        const double* B, const double* C, const double* D,
+                        const double* dt_bias, const double* init,
+                        double* dt_out, double* cumA_out, double* S_out,
+                        double* Hin_out, double* y, double* final_state) {
+    const int64_t nc = (L + Q - 1) / Q;
+    int64_t bh;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (bh = 0; bh < batch * H; ++bh) {
+        const int64_t b = bh / H, h = bh % H, g = group_of(h, H, G);
+        const double Dh = D ? D[h] : 0.0;
+        double* dt = (double*)calloc((size_t)Q, sizeof(double));
+        double* cumA = (double*)calloc((size_t)Q, sizeof(double));
+        double* S = (double*)malloc(sizeof(double) * (size_t)(P * N));
+        double* Hc = (double*)malloc(sizeof(double) * (size_t)(P * N));
+        if (init)
+            memcpy(Hc, init + bh * P * N, sizeof(double) * (size_t)(P * N));
+        else
+            memset(Hc, 0, sizeof(double) * (size_t)(P * N));
+        for (int64_t c = 0; c < nc; ++c) {
+            const int64_t t0 = c * Q;
+            const int64_t Lc = (L - t0 < Q) ? (L - t0) : Q;
+            /* step 1: dt and the inclusive in-chunk cumulative sum of dt*A */
+            double run = 0.0;
+            for (int64_t l = 0; l < Q; ++l) {
+                if (l < Lc) {
+                    dt[l] = dt_of(dt_raw, dt_bias, (b * L + t0 + l) * H + h, h);
+                    run += dt[l] * A[h];
+                    cumA[l] = run;
+                } else {
+                    dt[l] = 0.0;
+                    cumA[l] = 0.0;
+                }
+            }
+            if (dt_out)
+                memcpy(dt_out + (bh * nc + c) * Q, dt, sizeof(double) * (size_t)Q);
+            if (cumA_out)
+                memcpy(cumA_out + (bh * nc + c) * Q, cumA, sizeof(double) * (size_t)Q);
+            /* step 2: the chunk's local state, as if it started from zero */
+            memset(S, 0, sizeof(double) * (size_t)(P * N));
+            for (int64_t l = 0; l < Lc; ++l) {
+                const double w = exp(cumA[Lc - 1] - cumA[l]) * dt[l];
+                const double* xl = x + ((b * L + t0 + l) * H + h) * P;
+                const double* Bl = B + ((b * L + t0 + l) * G + g) * N;
+                for (int64_t p = 0; p < P; ++p)
+                    for (int64_t n = 0; n < N; ++n)
+                        S[p * N + n] += w * xl[p] * Bl[n];
+            }
+            if (S_out)
+                memcpy(S_out + ((b * nc + c) * H + h) * P * N, S,
+                       sizeof(double) * (size_t)(P * N));
+            if (Hin_out)
+                memcpy(Hin_out + ((b * nc + c) * H + h) * P * N, Hc,
+                       sizeof(double) * (size_t)(P * N));
+            /* step 4 (uses the state entering the chunk): the output */
+            for (int64_t l = 0; l < Lc; ++l) {
+                const double* Cl = C + ((b * L + t0 + l) * G + g) * N;
+                const double* xl = x + ((b * L + t0 + l) * H + h) * P;
+                double* yl = y + ((b * L + t0 + l) * H + h) * P;
+                const double carry = exp(cumA[l]);
+                for (int64_t p = 0; p < P; ++p) {
+                    double acc = 0.0;
+                    for (int64_t n = 0; n < N; ++n) acc += Cl[n] * Hc[p * N + n];
+                    yl[p] = carry * acc + Dh * xl[p];
+                }
+                for (int64_t j = 0; j <= l; ++j) {
+                    const double* Bj = B + ((b * L + t0 + j) * G + g) * N;
+                    const double* xj = x + ((b * L + t0 + j) * H + h) * P;
+                    double cb = 0.0;
+                    for (int64_t n = 0; n < N; ++n) cb += Cl[n] * Bj[n];
+                    const double m = exp(cumA[l] - cumA[j]) * cb * dt[j];
+                    for (int64_t p = 0; p < P; ++p) yl[p] += m * xj[p];
+                }
+            }
+            /* step 3: carry the state across the chunk boundary */
+            const double decay = exp(cumA[Lc - 1]);
+            for (int64_t i = 0; i < P * N; ++i) Hc[i] = decay * Hc[i] + S[i];
+        }
+        if (final_state)
+            memcpy(final_state + bh * P * N, Hc, sizeof(double) * (size_t)(P * N));
+        free(dt); free(cumA); free(S); free(Hc);
+    }
+}
+
+/* One decode step: state [batch, H, P, N] is updated in place and y [batch,
+ * H, P] receives the step's output.  x [batch, H, P], dt_raw [batch, H],
+ * B, C [batch, G, N]. */
+void oracle_state_update(int64_t batch, int64_t H, int64_t P, int64_t N,
+                         int64_t G, double* state,
+                         const double* x, const double* dt_raw,
+                         const double* A, const double* B, const double* C,
+                         const double* D, const double* dt_bias, double* y) {
+    int64_t bh;
+#pragma omp parallel for schedule(static)
+    for (bh = 0; bh < batch * H; ++bh) {
+        const int64_t b = bh / H, h = bh % H, g = group_of(h, H, G);
+        const double dt = dt_of(dt_raw, dt_bias, bh, h);
+        const double a = exp(dt * A[h]);
+        const double* xt = x + bh * P;
+        const double* Bt = B + (b * G + g) * N;
+        const double* Ct = C + (b * G + g) * N;
+        double* S = state + bh * P * N;
+        for (int64_t p = 0; p < P; ++p) {
+            double acc = 0.0;
+            for (int64_t n = 0; n < N; ++n) {
+                S[p * N + n] = a * S[p * N + n] + dt * xt[p] * Bt[n];
+                acc += S[p * N + n] * Ct[n];
+            }
+            y[bh * P + p] = acc + (D ? D[h] : 0.0) * xt[p];
+        }
+    }
+}

@@ -1,0 +1,231 @@
+"""Pins of the fp64 oracle to facts outside itself.
+
+Each ``pin_*`` takes an oracle handle and raises AssertionError when the oracle
+disagrees with something the pages or the mathematics fix independently:
+
+* the masked-attention (quadratic) dual form of SSD, written out by brute force
+  ("MAMBA-2 Reference Implementations Comparison", section 2.2: Y = diag(p) M
+  diag(q) X with M a 1-semiseparable causal mask when A is a scalar times the
+  identity);
+* the A = 0 closed form, where the state is a plain cumulative sum;
+* chunk-size invariance of the chunked restatement ("MAMBA-2 Implementation
+  Gaps", Gap 1: diagonal blocks + inter-chunk carry compute the same scan);
+* split / resume through the carried state, decode == forward;
+* special cases: C = 0, x = 0, full decay, L = 1, causality (the "no future
+  leakage" test of "MAMBA-2 Implementation Gaps", Testing Strategy);
+* softplus values fixed by its definition;
+* a half-decay example worked by hand (tests/golden/half_decay_by_hand.json).
+
+They are plain functions so that the mutant test can run every pin against
+deliberately wrong builds of the oracle and check that each one is caught.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _rand_case(seed, b=2, L=13, H=4, P=3, N=5, G=2, init=True, A_scale=1.0):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((b, L, H, P))
+    dt = rng.standard_normal((b, L, H))
+    B = rng.standard_normal((b, L, G, N))
+    C = rng.standard_normal((b, L, G, N))
+    A = -rng.uniform(0.2, 2.0, H) * A_scale
+    D = rng.standard_normal(H)
+    bias = rng.uniform(-1.0, 0.5, H)
+    h0 = 0.5 * rng.standard_normal((b, H, P, N)) if init else None
+    return dict(x=x, dt=dt, A=A, B=B, C=C, D=D, dt_bias=bias, init_state=h0)
+
+
+def _softplus_np(u):
+    return np.logaddexp(0.0, u)
+
+
+def quadratic_form(x, dt, A, B, C, D, dt_bias, init_state):
+    """y by the masked-attention dual: y_i = sum_{j<=i} L[i,j] (C_i.B_j) dt_j x_j
+    + exp(sum_{k<=i} dt_k A) C_i.h0 + D x_i, with L[i,j] = exp(sum_{k=j+1..i}
+    dt_k A).  Brute force, O(L^2), every decay product summed explicitly."""
+    b, L, H, P = x.shape
+    G = B.shape[2]
+    y = np.zeros_like(x)
+    for bi in range(b):
+        for h in range(H):
+            g = h // (H // G)
+            d = _softplus_np(dt[bi, :, h] + (dt_bias[h] if dt_bias is not None else 0.0))
+            for i in range(L):
+                for j in range(i + 1):
+                    seg = sum(d[k] * A[h] for k in range(j + 1, i + 1))
+                    m = math.exp(seg) * float(C[bi, i, g] @ B[bi, j, g]) * d[j]
+                    y[bi, i, h] += m * x[bi, j, h]
+                if init_state is not None:
+                    tot = sum(d[k] * A[h] for k in range(0, i + 1))
+                    y[bi, i, h] += math.exp(tot) * (init_state[bi, h] @ C[bi, i, g])
+                if D is not None:
+                    y[bi, i, h] += D[h] * x[bi, i, h]
+    return y
+
+
+def _close(a, b, rtol, what):
+    a = np.asarray(a)
+    b = np.asarray(b)
+    err = np.max(np.abs(a - b) / (1.0 + np.abs(b))) if a.size else 0.0
+    assert err <= rtol, f"{what}: max rel err {err:.3e} > {rtol:.1e}"
+
+
+def pin_softplus(orc):
+    assert abs(orc.softplus(0.0) - math.log(2.0)) < 1e-15, "softplus(0) != ln 2"
+    for u in (-30.0, -3.0, -0.5, 0.25, 2.0, 40.0):
+        # softplus(u) - softplus(-u) = u for every u
+        assert abs(orc.softplus(u) - orc.softplus(-u) - u) < 1e-12 * max(1.0, abs(u))
+        assert abs(orc.softplus(u) - math.log1p(math.exp(u))) <= 1e-14 * max(1.0, abs(u))
+
+
+def pin_quadratic_dual(orc):
+    for seed, G, init in ((0, 1, False), (1, 2, True), (2, 4, True)):
+        case = _rand_case(seed, G=G, init=init)
+        y, _ = orc.ssd_fwd(**case)
+        _close(y, quadratic_form(**case), 1e-12, f"quadratic dual (G={G}, init={init})")
+
+
+def pin_A_zero_cumsum(orc):
+    case = _rand_case(3)
+    case["A"] = np.zeros_like(case["A"])
+    y, fin = orc.ssd_fwd(**case)
+    x, B, C, h0 = case["x"], case["B"], case["C"], case["init_state"]
+    b, L, H, P = x.shape
+    G = B.shape[2]
+    for bi in range(b):
+        for h in range(H):
+            g = h // (H // G)
+            d = _softplus_np(case["dt"][bi, :, h] + case["dt_bias"][h])
+            inc = d[:, None, None] * x[bi, :, h, :, None] * B[bi, :, g, None, :]
+            states = h0[bi, h][None] + np.cumsum(inc, axis=0)
+            yref = np.einsum("lpn,ln->lp", states, C[bi, :, g]) + case["D"][h] * x[bi, :, h]
+            _close(y[bi, :, h], yref, 1e-12, "A=0 closed form (y)")
+            _close(fin[bi, h], states[-1], 1e-12, "A=0 closed form (final state)")
+
+
+def pin_chunk_invariance(orc):
+    case = _rand_case(4, L=37)
+    y, fin = orc.ssd_fwd(**case)
+    for Q in (1, 3, 16, 37, 64):
+        out = orc.ssd_chunked(**case, chunk=Q)
+        _close(out["y"], y, 1e-12, f"chunked Q={Q} y")
+        _close(out["final_state"], fin, 1e-12, f"chunked Q={Q} final")
+        # the state entering chunk c is the recurrence's state after token c*Q-1
+        nc = out["Hin"].shape[1]
+        for c in range(1, nc):
+            sub = {k: (v[:, : c * Q] if k in ("x", "dt", "B", "C") else v)
+                   for k, v in case.items()}
+            _, fc = orc.ssd_fwd(**sub)
+            _close(out["Hin"][:, c], fc, 1e-12, f"chunked Q={Q} state entering chunk {c}")
+
+
+def pin_split_resume(orc):
+    case = _rand_case(5, L=20)
+    y, fin = orc.ssd_fwd(**case)
+    for L1 in (1, 7, 19):
+        a = {k: (v[:, :L1] if k in ("x", "dt", "B", "C") else v) for k, v in case.items()}
+        y1, f1 = orc.ssd_fwd(**a)
+        bb = {k: (v[:, L1:] if k in ("x", "dt", "B", "C") else v) for k, v in case.items()}
+        bb["init_state"] = f1
+        y2, f2 = orc.ssd_fwd(**bb)
+        _close(np.concatenate([y1, y2], axis=1), y, 1e-12, f"split at {L1} (y)")
+        _close(f2, fin, 1e-12, f"split at {L1} (final)")
+
+
+def pin_decode_equals_forward(orc):
+    case = _rand_case(6, L=9)
+    y, fin = orc.ssd_fwd(**case)
+    st = case["init_state"].copy()
+    for t in range(case["x"].shape[1]):
+        st, yt = orc.state_update(st, case["x"][:, t], case["dt"][:, t], case["A"],
+                                  case["B"][:, t], case["C"][:, t], case["D"],
+                                  case["dt_bias"])
+        _close(yt, y[:, t], 1e-12, f"decode step {t} y")
+    _close(st, fin, 1e-12, "decode final state")
+
+
+def pin_special_cases(orc):
+    case = _rand_case(7)
+    # C = 0: the output is the skip term only, exactly
+    c0 = dict(case, C=np.zeros_like(case["C"]))
+    y, _ = orc.ssd_fwd(**c0)
+    assert np.array_equal(y, case["D"][None, None, :, None] * case["x"]), "C=0 => y = D x"
+    # x = 0 and zero initial state: everything stays zero
+    z = dict(case, x=np.zeros_like(case["x"]), init_state=None)
+    y, fin = orc.ssd_fwd(**z)
+    assert not y.any() and not fin.any(), "x=0, h0=0 => y=0, final=0"
+    # full decay (dt*A -> -inf, a = 0): each token sees only itself
+    m = dict(case, A=np.full_like(case["A"], -1e300))
+    y, _ = orc.ssd_fwd(**m)
+    x, B, C = case["x"], case["B"], case["C"]
+    H, G = x.shape[2], B.shape[2]
+    for h in range(H):
+        g = h // (H // G)
+        d = _softplus_np(case["dt"][:, :, h] + case["dt_bias"][h])
+        cb = np.einsum("bln,bln->bl", C[:, :, g], B[:, :, g])
+        ref = (d * cb)[..., None] * x[:, :, h] + case["D"][h] * x[:, :, h]
+        _close(y[:, :, h], ref, 1e-13, "memoryless (a=0)")
+    # L = 1, zero initial state, by hand: y = dt (C.B) x + D x
+    one = {k: (v[:, :1] if k in ("x", "dt", "B", "C") else v) for k, v in case.items()}
+    one["init_state"] = None
+    y, fin = orc.ssd_fwd(**one)
+    for h in range(H):
+        g = h // (H // G)
+        d = _softplus_np(one["dt"][:, 0, h] + one["dt_bias"][h])
+        cb = np.einsum("bn,bn->b", one["C"][:, 0, g], one["B"][:, 0, g])
+        ref = (d * cb)[:, None] * one["x"][:, 0, h] + one["D"][h] * one["x"][:, 0, h]
+        _close(y[:, 0, h], ref, 1e-14, "L=1 by hand")
+        reff = d[:, None, None] * one["x"][:, 0, h, :, None] * one["B"][:, 0, g, None, :]
+        _close(fin[:, h], reff, 1e-14, "L=1 final by hand")
+
+
+def pin_causality(orc):
+    case = _rand_case(8, L=16)
+    y, _ = orc.ssd_fwd(**case)
+    for t0 in (0, 5, 15):
+        pert = {k: v.copy() if isinstance(v, np.ndarray) else v for k, v in case.items()}
+        pert["x"][:, t0] += 1.0
+        pert["B"][:, t0] -= 0.5
+        pert["C"][:, t0] *= 2.0
+        pert["dt"][:, t0] += 0.3
+        y2, _ = orc.ssd_fwd(**pert)
+        assert np.array_equal(y2[:, :t0], y[:, :t0]), f"future leak into t<{t0}"
+        assert not np.array_equal(y2[:, t0], y[:, t0]), f"perturbation at {t0} had no effect"
+
+
+def pin_half_decay_by_hand(orc):
+    with open(os.path.join(GOLDEN, "half_decay_by_hand.json")) as f:
+        g = json.load(f)
+    lam = math.log(2.0)
+    inp = {k: np.array(v, dtype=np.float64) for k, v in g["inputs"].items()}
+    y, fin = orc.ssd_fwd(**inp)
+    ey = np.array(g["expected"]["y_coef_ln2"]) * lam + np.array(g["expected"]["y_coef_1"])
+    ef = (np.array(g["expected"]["final_coef_ln2"]) * lam
+          + np.array(g["expected"]["final_coef_1"]))
+    _close(y, ey, 1e-14, "hand-worked half-decay y")
+    _close(fin, ef, 1e-14, "hand-worked half-decay final state")
+
+
+def pin_golden_regression(orc):
+    """Stored outputs of the oracle itself (tests/golden/make_golden.py), so
+    that any later change to its arithmetic shows up here."""
+    with open(os.path.join(GOLDEN, "oracle_small.json")) as f:
+        g = json.load(f)
+    inp = {k: (np.array(v, dtype=np.float64) if v is not None else None)
+           for k, v in g["inputs"].items()}
+    y, fin = orc.ssd_fwd(**inp)
+    _close(y, np.array(g["y"]), 1e-13, "golden y")
+    _close(fin, np.array(g["final_state"]), 1e-13, "golden final")
+
+
+ALL_PINS = [pin_softplus, pin_quadratic_dual, pin_A_zero_cumsum, pin_chunk_invariance,
+            pin_split_resume, pin_decode_equals_forward, pin_special_cases, pin_causality,
+            pin_half_decay_by_hand]
