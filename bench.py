@@ -1,0 +1,524 @@
+#!/usr/bin/env python
+"""Throughput of the SSD scan forward (tokens/s) and of the decode state update
+(us/step) on B200, one JSON line on stdout (rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one ssd_fwd call (chunk_cumsum -> chunk_state -> state_passing ->
+chunk_scan) over one batch of the headline workload, bf16 in / fp32 accumulate,
+batch 4 x seqlen 1024, 24 heads x headdim 64, dstate 64, 1 group, chunk 256.
+Inputs are seeded synthetic data already resident in HBM; the working set
+(26 MB) fits in L2, so a 256 MB buffer is rewritten before every timed step
+(outside the timed events) to flush it.  Each step is timed with CUDA events on
+the launching stream; ms_per_step is the mean over the K timed steps, the max
+over ranks.  Under torchrun every rank runs its own independent batch (weak
+scaling, no collective on the data path).
+
+Also reported: the same metric end to end through the public API from pinned
+host buffers (`e2e`), the roofline position of the dominant kernel, the other
+workloads (seqlen 4096 with an initial state, seqlen 65536 with 8 groups, and
+1024 successive decode steps replayed from one CUDA graph), SM clocks sampled
+through NVML during the timed region, and the fp64 CPU oracle timed on a
+bounded sample of the same workload (`cpu_baseline`).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+HEADLINE = "fwd_bf16_b4_L1024"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "sm_max_mhz": 1965.0, "source": "fallback"}
+N_SM = 148
+FFMA_LANES_PER_SM = 128
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=HEADLINE)
+    ap.add_argument("--no-extra", action="store_true", help="skip the other workloads")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--flush-mb", type=int, default=256)
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        p["source"] = "measured"
+        return p
+    return dict(FALLBACK_PEAKS)
+
+
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    """Samples the SM clock and the clock-event (throttle) reasons through NVML
+    in a background thread while the timed region runs."""
+
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.period = period_s
+        self.samples = []
+        self.reason_bits = 0
+        self.ok = False
+        self.max_mhz = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            import torch
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            h = None
+            for i in range(pynvml.nvmlDeviceGetCount()):
+                hi = pynvml.nvmlDeviceGetHandleByIndex(i)
+                u = pynvml.nvmlDeviceGetUUID(hi)
+                u = u.decode() if isinstance(u, bytes) else u
+                if u.replace("GPU-", "") == uuid.replace("GPU-", ""):
+                    h = hi
+            if h is None:
+                h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.nvml, self.h = pynvml, h
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: the line says so
+            self.err = repr(e)
+        self._stop = threading.Event()
+        self._t = None
+
+    def _run(self):
+        n = self.nvml
+        while not self._stop.is_set():
+            try:
+                self.samples.append(n.nvmlDeviceGetClockInfo(self.h, n.NVML_CLOCK_SM))
+                self.reason_bits |= int(n.nvmlDeviceGetCurrentClocksEventReasons(self.h))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._t:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        reasons = [k for k, bit in self.REASONS.items() if self.reason_bits & bit]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+def algorithmic_cost(cfg, elt):
+    """Bytes (inputs read once, outputs written once) and FLOP (causal half of
+    the chunk-square terms) of each kernel of the forward, per launch."""
+    b, L, H, P, N, G, Q = (cfg.batch, cfg.seqlen, cfg.nheads, cfg.headdim, cfg.dstate,
+                           cfg.ngroups, cfg.chunk)
+    nc = -(-L // Q)
+    tok = b * L
+    x = tok * H * P * elt
+    bc = tok * G * N * elt
+    dtr = tok * H * elt
+    vec = b * H * nc * Q * 4
+    states = b * nc * H * P * N * 4
+    init = b * H * P * N * 4 if cfg.init_state else 0
+    fin = b * H * P * N * 4 if cfg.return_final else 0
+    causal = Q * (Q + 1) / 2
+    flops_state = 2.0 * tok * H * P * N
+    flops_scan = (2.0 * b * nc * G * causal * N      # C.B^T per group
+                  + 2.0 * b * nc * H * causal * P    # masked (C.B^T) x per head
+                  + 2.0 * tok * H * P * N)           # C . H_in per head
+    return {
+        "chunk_cumsum": (dtr + 2 * vec, 0.0),
+        "chunk_state": (x + bc + 2 * vec + states, flops_state),
+        "state_passing": (2 * states + b * H * nc * 4 + init + fin, 3.0 * states / 4),
+        "chunk_scan": (x + 2 * bc + 2 * vec + states + x, flops_scan),
+        "path": (x + 2 * bc + dtr + x + init + fin, flops_state + flops_scan),
+    }
+
+
+def main_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import mamba_ssd_scan_b200 as ssd
+    from mamba_ssd_scan_b200 import synthetic
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    ssd.load_library()
+    peaks = load_peaks()
+    cfg = synthetic.FWD_CONFIGS[args.workload]
+    seed = 1234 + synthetic.SEED_OFFSET[cfg.name] + 1000 * rank
+    inp = synthetic.make_config_inputs(cfg, seed)
+    d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
+    elt = d["x"].element_size()
+    stream = torch.cuda.current_stream()
+    flush_buf = torch.empty(args.flush_mb << 20, dtype=torch.uint8, device=dev)
+
+    def flush():
+        flush_buf.fill_(1)
+
+    y = torch.empty_like(d["x"])
+    fin = (torch.empty((cfg.batch, cfg.nheads, cfg.headdim, cfg.dstate), device=dev)
+           if cfg.return_final else None)
+    ws = torch.empty(ssd.ssd_fwd_workspace_size(cfg.batch, cfg.seqlen, cfg.nheads, cfg.headdim,
+                                                cfg.dstate, cfg.ngroups, cfg.chunk,
+                                                cfg.dtype), dtype=torch.uint8, device=dev)
+
+    def step():
+        ssd.ssd_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["dt_bias"], cfg.chunk,
+                    d["init_state"], y=y, final_state=fin, workspace=ws)
+
+    # ---- headline: K timed steps ----------------------------------------
+    for _ in range(args.warmup):
+        flush()
+        step()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    with clocks:
+        barrier()
+        torch.cuda.synchronize()
+        for k in range(args.steps):
+            flush()
+            ev[k][0].record(stream)
+            step()
+            ev[k][1].record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
+    ms = max_over_ranks(ms)
+    tokens = cfg.tokens
+    value = world * tokens / (ms * 1e-3)
+    launches_per_step = 4
+
+    # ---- per-kernel durations over the same kind of timed steps ---------
+    nc = -(-cfg.seqlen // cfg.chunk)
+    dt_sp = torch.empty((cfg.batch, cfg.nheads, nc, cfg.chunk), device=dev)
+    cumA = torch.empty_like(dt_sp)
+    states = torch.empty((cfg.batch, nc, cfg.nheads, cfg.headdim, cfg.dstate), device=dev)
+    names = ["chunk_cumsum", "chunk_state", "state_passing", "chunk_scan"]
+
+    def step_split(evs):
+        evs[0].record(stream)
+        ssd.ssd_chunk_cumsum(d["x"], d["dt"], d["A"], d["B"], d["C"], d["dt_bias"], cfg.chunk,
+                             dt_out=dt_sp, cumA_out=cumA)
+        evs[1].record(stream)
+        ssd.ssd_chunk_state(d["x"], d["dt"], d["A"], d["B"], d["C"], dt_sp, cumA, cfg.chunk,
+                            states=states)
+        evs[2].record(stream)
+        ssd.ssd_state_passing(d["x"], d["dt"], d["A"], d["B"], d["C"], cumA, states, cfg.chunk,
+                              init_state=d["init_state"], final_state=fin)
+        evs[3].record(stream)
+        ssd.ssd_chunk_scan(d["x"], d["dt"], d["A"], d["B"], d["C"], dt_sp, cumA, states,
+                           d["D"], cfg.chunk, y=y)
+        evs[4].record(stream)
+
+    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    for _ in range(args.warmup):
+        flush()
+        step_split([torch.cuda.Event() for _ in range(5)])
+    barrier()
+    torch.cuda.synchronize()
+    for k in range(args.steps):
+        flush()
+        step_split(kev[k])
+    torch.cuda.synchronize()
+    kms = {n: sum(e[i].elapsed_time(e[i + 1]) for e in kev) / args.steps
+           for i, n in enumerate(names)}
+    cost = algorithmic_cost(cfg, elt)
+    top = max(names, key=lambda n: kms[n])
+    roofline = roofline_entry(top, cost[top], kms[top], peaks, clocks.summary())
+
+    # ---- e2e through the public API from pinned host buffers ------------
+    e2e = None
+    if True:
+        host = {k: (v.pin_memory() if v is not None else None) for k, v in inp.items()}
+        y_host = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
+        h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
+        d2h = y_host.numel() * y_host.element_size()
+
+        def e2e_step():
+            dd = {k: (v.to(dev, non_blocking=True) if v is not None else None)
+                  for k, v in host.items()}
+            yy = ssd.ssd_fwd(dd["x"], dd["dt"], dd["A"], dd["B"], dd["C"], dd["D"],
+                             dd["dt_bias"], cfg.chunk, dd["init_state"], workspace=ws)
+            y_host.copy_(yy, non_blocking=True)
+
+        for _ in range(args.warmup):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ems = max_over_ranks(e0.elapsed_time(e1) / args.steps)
+        e2e = {"value": world * tokens / (ems * 1e-3), "unit": "tokens/s",
+               "ms_per_step": ems, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    # ---- other workloads (rank-local, reported for context) --------------
+    extra = {}
+    if not args.no_extra:
+        extra = other_workloads(ssd, synthetic, dev, flush, peaks, rank, world,
+                                barrier, max_over_ranks)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(cfg, inp, budget_s=12.0)
+
+    clk = clocks.summary()
+    line = {
+        "metric": "SSD fwd tokens/s",
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if cfg.dtype.__repr__().endswith("bfloat16") else "f32",
+        "data": "synthetic",
+        "config": {"workload": cfg.name, "batch": cfg.batch, "seqlen": cfg.seqlen,
+                   "nheads": cfg.nheads, "headdim": cfg.headdim, "dstate": cfg.dstate,
+                   "ngroups": cfg.ngroups, "chunk": cfg.chunk, "global_batch":
+                   cfg.batch * world, "parallelism": f"dp{world}" if world > 1 else "single",
+                   "l2": f"flushed ({args.flush_mb} MB write) before every timed step"},
+        "roofline": roofline,
+        "kernel_ms": kms,
+        "e2e": e2e,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": {k: clk[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
+        "cpu_baseline": cpu,
+        "workloads": extra,
+        "peaks_source": peaks.get("source"),
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def roofline_entry(name, cost, ms, peaks, clk):
+    nbytes, flops = cost
+    sec = ms * 1e-3
+    hbm = peaks["hbm_gbs"]
+    t_hbm = nbytes / (hbm * 1e9)
+    # the CUDA-core path executes its contractions as fp32 FFMA; its compute
+    # peak is 148 SMs x 128 FP32 lanes x 2 FLOP x SM clock
+    mhz = clk.get("sm_mhz") or peaks.get("sm_max_mhz", 1965.0)
+    alu_peak = N_SM * FFMA_LANES_PER_SM * 2 * mhz * 1e6 / 1e12  # TFLOP/s
+    t_alu = flops / (alu_peak * 1e12) if flops else 0.0
+    if t_alu > t_hbm:
+        ach = flops / sec / 1e12
+        return {"kernel": name, "bound": "alu", "achieved": ach, "peak": alu_peak,
+                "unit": "TFLOP/s", "frac": ach / alu_peak, "traffic": None,
+                "peak_note": f"FFMA: 148 SM x 128 lanes x 2 x {mhz:.0f} MHz (sampled)",
+                "algorithmic_bytes": nbytes, "algorithmic_flops": flops}
+    ach = nbytes / sec / 1e9
+    return {"kernel": name, "bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s",
+            "frac": ach / hbm, "traffic": None, "peak_note": f"{peaks.get('source')} copy BW",
+            "algorithmic_bytes": nbytes, "algorithmic_flops": flops}
+
+
+def other_workloads(ssd, synthetic, dev, flush, peaks, rank, world, barrier, max_over_ranks):
+    import torch
+    out = {}
+    stream = torch.cuda.current_stream()
+    for name, steps in (("fwd_bf16_b8_L4096_init", 10), ("fwd_bf16_b1_L65536_G8", 5)):
+        cfg = synthetic.FWD_CONFIGS[name]
+        inp = synthetic.make_config_inputs(cfg, 1234 + synthetic.SEED_OFFSET[name] + 1000 * rank)
+        d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
+        del inp
+        y = torch.empty_like(d["x"])
+        fin = torch.empty((cfg.batch, cfg.nheads, cfg.headdim, cfg.dstate), device=dev) \
+            if cfg.return_final else None
+        ws = torch.empty(ssd.ssd_fwd_workspace_size(cfg.batch, cfg.seqlen, cfg.nheads,
+                                                    cfg.headdim, cfg.dstate, cfg.ngroups,
+                                                    cfg.chunk, cfg.dtype),
+                         dtype=torch.uint8, device=dev)
+
+        def step():
+            ssd.ssd_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["dt_bias"],
+                        cfg.chunk, d["init_state"], y=y, final_state=fin, workspace=ws)
+
+        for _ in range(3):
+            step()
+        torch.cuda.synchronize()
+        tot = 0.0
+        for _ in range(steps):
+            flush()
+            a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            step()
+            b_.record(stream)
+            torch.cuda.synchronize()
+            tot += a.elapsed_time(b_)
+        ms = max_over_ranks(tot / steps)
+        nbytes = algorithmic_cost(cfg, 2)["path"][0]
+        out[name] = {"tokens_per_s": world * cfg.tokens / (ms * 1e-3), "ms": ms,
+                     "hbm_frac_of_path_bytes": nbytes / (ms * 1e-3) / (peaks["hbm_gbs"] * 1e9)}
+        del d, y, fin, ws
+        torch.cuda.empty_cache()
+
+    # decode: 1024 successive steps captured in one CUDA graph
+    cfg = synthetic.DECODE_CONFIGS["decode_b256_H80"]
+    seed = 1234 + synthetic.SEED_OFFSET[cfg.name] + 1000 * rank
+    prm = synthetic.make_decode_params(cfg.batch, cfg.nheads, cfg.headdim, cfg.dstate, seed)
+    state = prm["state"].to(dev)
+    A, D, bias = prm["A"].to(dev), prm["D"].to(dev), prm["dt_bias"].to(dev)
+    n_distinct = 16  # step inputs cycle through 16 distinct draws (3.7 MB each)
+    steps_in = [synthetic.make_decode_step(cfg.batch, cfg.nheads, cfg.headdim, cfg.dstate,
+                                           cfg.ngroups, cfg.dtype, seed, s)
+                for s in range(n_distinct)]
+    steps_in = [{k: v.to(dev) for k, v in s.items()} for s in steps_in]
+    ys = torch.empty((cfg.batch, cfg.nheads, cfg.headdim), dtype=cfg.dtype, device=dev)
+
+    def run(n):
+        for s in range(n):
+            si = steps_in[s % n_distinct]
+            ssd.ssd_state_update(state, si["x"], si["dt"], A, si["B"], si["C"], D, bias, y=ys)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        run(3)
+    torch.cuda.current_stream().wait_stream(side)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        run(cfg.steps)
+    g.replay()
+    torch.cuda.synchronize()
+    a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    g.replay()
+    b_.record(stream)
+    torch.cuda.synchronize()
+    us = max_over_ranks(a.elapsed_time(b_) * 1e3 / cfg.steps)
+    sbytes = cfg.batch * cfg.nheads * cfg.headdim * cfg.dstate * 4
+    step_bytes = 2 * sbytes + cfg.batch * (2 * cfg.nheads * cfg.headdim + cfg.nheads +
+                                           2 * cfg.ngroups * cfg.dstate) * 2
+    out[cfg.name] = {"us_per_step": us, "steps": cfg.steps, "graph": True,
+                     "achieved_gbs": step_bytes / (us * 1e-6) / 1e9,
+                     "hbm_frac": step_bytes / (us * 1e-6) / (peaks["hbm_gbs"] * 1e9),
+                     "bytes_per_step": step_bytes}
+    del g
+    return out
+
+
+def cpu_baseline(cfg, inp, budget_s=12.0):
+    """The fp64 oracle, as it stands, on a bounded sample of the workload:
+    whole batch rows (all heads, full sequence) until about budget_s of work."""
+    import oracle
+    orc = oracle.load()
+    t0 = time.perf_counter()
+    rows = 0
+    while rows < cfg.batch and time.perf_counter() - t0 < budget_s:
+        sub = {k: (v[rows:rows + 1] if (v is not None and k not in ("A", "D", "dt_bias"))
+                   else v) for k, v in inp.items()}
+        orc.ssd_fwd(**sub)
+        rows += 1
+    dt = time.perf_counter() - t0
+    return {"value": rows * cfg.seqlen / dt, "unit": "tokens/s", "cores": orc.num_threads(),
+            "kind": "oracle", "sample": f"{rows} of {cfg.batch} batch rows of {cfg.name} "
+                                        f"(all heads, full sequence), {dt:.1f} s"}
+
+
+# ---------------------------------------------------------------------------
+def main_reference(args):
+    """The reference arm: the fp64 CPU oracle on this arm's workload, each step a
+    bounded sample (one batch row, as many heads as host threads, full sequence)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import oracle
+    from mamba_ssd_scan_b200 import synthetic
+    cfg = synthetic.FWD_CONFIGS[args.workload]
+    inp = synthetic.make_config_inputs(cfg)
+    orc = oracle.load()
+    heads = min(cfg.nheads, orc.num_threads())
+    hpg = cfg.nheads // cfg.ngroups
+    gsel = [h // hpg for h in range(heads)]
+    sub = {"x": inp["x"][:1, :, :heads], "dt": inp["dt"][:1, :, :heads], "A": inp["A"][:heads],
+           "B": inp["B"][:1, :, gsel], "C": inp["C"][:1, :, gsel], "D": inp["D"][:heads],
+           "dt_bias": inp["dt_bias"][:heads],
+           "init_state": None if inp["init_state"] is None else inp["init_state"][:1, :heads]}
+    for _ in range(args.warmup):
+        orc.ssd_fwd(**sub)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        orc.ssd_fwd(**sub)
+    sec = (time.perf_counter() - t0) / args.steps
+    # one step covers heads/H of one batch row's tokens
+    tok_equiv = cfg.seqlen * heads / cfg.nheads
+    value = tok_equiv / sec
+    line = {"impl": "reference", "metric": "SSD fwd tokens/s", "value": value,
+            "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": cfg.name, "batch": cfg.batch, "seqlen": cfg.seqlen,
+                       "nheads": cfg.nheads, "headdim": cfg.headdim, "dstate": cfg.dstate,
+                       "ngroups": cfg.ngroups, "chunk": cfg.chunk},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": orc.num_threads(),
+                             "kind": "oracle",
+                             "sample": f"per step: batch row 0, heads 0-{heads - 1} of "
+                                       f"{cfg.nheads}, full sequence (token-equivalents = "
+                                       f"seqlen x {heads}/{cfg.nheads})"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    a = parse_args()
+    if a.impl == "reference":
+        main_reference(a)
+    else:
+        main_ours(a)

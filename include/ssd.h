@@ -1,0 +1,175 @@
+/*
+ * ssd.h -- C ABI of libssd_b200.so: the Mamba-2 SSD selective scan forward and
+ * the single-token decode state update, on NVIDIA B200 (sm_100a).
+ *
+ * The operation (pages: "MAMBA-2 Reference Implementations Comparison",
+ * section 2.2 "SSD Mathematical Formulation" and section 3.2 "Selective Scan
+ * Algorithm"; "MAMBA-2 Implementation Gaps", Gap 1 "SSD Algorithm", Gap 3
+ * "dt (Time Step) Parameter", Gap 4 "D (Skip Connection) Parameter"):
+ *
+ *   dt_t = softplus(dt_raw_t + dt_bias_h)          (no clamp)
+ *   h_t  = exp(dt_t * A_h) * h_{t-1} + dt_t * x_t B_t^T      h: [P x N]
+ *   y_t  = C_t . h_t + D_h * x_t                     (h_t after the update)
+ *
+ * with A_h a scalar per head (normally negative), B_t, C_t shared by the heads
+ * of a group (head h reads group h / (nheads / ngroups)).  The forward pass
+ * computes this chunkwise: chunk_cumsum -> chunk_state -> state_passing ->
+ * chunk_scan, the chunked SSD of "MAMBA-2 Implementation Gaps", Gap 1.
+ *
+ * Layouts: row-major, innermost index last, densely packed (no strides):
+ *   x, y          [batch, seqlen, nheads, headdim]     dtype
+ *   dt (raw)      [batch, seqlen, nheads]              dtype
+ *   B, C          [batch, seqlen, ngroups, dstate]     dtype
+ *   A, D, dt_bias [nheads]                             fp32
+ *   state         [batch, nheads, headdim, dstate]     fp32
+ * "dtype" is SSD_F32 (fp32) or SSD_BF16 (bfloat16); arithmetic is fp32 either
+ * way (bf16 operands enter the tensor cores, products accumulate in fp32) and y
+ * is rounded to dtype (round to nearest even).
+ *
+ * Ownership and memory: every pointer is a DEVICE pointer owned by the caller
+ * (cudaMalloc, a torch tensor, ...).  The library allocates no memory and keeps
+ * no state between calls other than per-device kernel attributes.  Scratch
+ * memory for ssd_fwd comes from the caller (ssd_fwd_workspace_size).
+ * x, B, C, y, init_state, final_state and workspace must be 16-byte aligned.
+ *
+ * Calling convention: calls are asynchronous on `stream` (a cudaStream_t passed
+ * as void*; NULL = the legacy default stream) and never synchronise the host.
+ * Arguments are validated before anything is launched; on an error nothing is
+ * launched and nothing is written.  There is no CPU fallback.
+ *
+ * Errors: SSD_ERR_INVALID_ARG for a NULL required pointer, a pointer the CUDA
+ * runtime does not know as device memory, a misaligned pointer, a size <= 0 or
+ * nheads % ngroups != 0, a too-small workspace; SSD_ERR_UNSUPPORTED for sizes
+ * outside the kernels' range (listed per call); SSD_ERR_CUDA when a launch
+ * fails (cudaGetLastError after the launch).
+ */
+#ifndef SSD_B200_H
+#define SSD_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SSD_OK = 0,
+    SSD_ERR_INVALID_ARG = 1,
+    SSD_ERR_UNSUPPORTED = 2,
+    SSD_ERR_CUDA = 3,
+    SSD_ERR_TIMEOUT = 4
+} ssd_status;
+
+typedef enum { SSD_F32 = 0, SSD_BF16 = 1 } ssd_dtype;
+
+/* Arguments of the forward scan and of its four steps.
+ *   chunk        Q, tokens per chunk; the last chunk may be shorter
+ *                (nc = ceil(seqlen / chunk) chunks).
+ *   D, dt_bias   may be NULL (= 0).
+ *   init_state   may be NULL (= zero state): the state before token 0.
+ *   y            output [batch, seqlen, nheads, headdim], dtype.
+ *   final_state  may be NULL: receives h after the last token, fp32.
+ * Supported: 1 <= chunk <= 256; dstate a multiple of 4, <= 256; headdim a
+ * multiple of 4; the tensor-core path (bf16, headdim in {32, 64, 128},
+ * dstate in {64, 128}, chunk 256) is chosen automatically, every other valid
+ * shape runs on the CUDA-core path. */
+typedef struct {
+    int64_t batch, seqlen, nheads, headdim, dstate, ngroups, chunk;
+    int32_t dtype;          /* ssd_dtype of x, dt, B, C and y */
+    int32_t flags;          /* SSD_FLAG_* below; 0 = defaults */
+    const void* x;
+    const void* dt;         /* raw dt, before bias and softplus */
+    const float* A;
+    const void* B;
+    const void* C;
+    const float* D;
+    const float* dt_bias;
+    const float* init_state;
+    void* y;
+    float* final_state;
+    void* workspace;        /* device scratch, >= ssd_fwd_workspace_size() */
+    size_t workspace_bytes;
+} ssd_fwd_args;
+
+/* flags */
+#define SSD_FLAG_CUDA_CORES 1   /* force the CUDA-core (FFMA) path */
+
+/* Bytes of device workspace ssd_fwd needs for these sizes (0 on invalid
+ * sizes).  Only sizes, dtype and flags are read; pointers may be NULL. */
+size_t ssd_fwd_workspace_size(const ssd_fwd_args* args);
+
+/* The whole forward scan: y (and final_state) from x, dt, A, B, C, D,
+ * dt_bias, init_state.  Stream-ordered; the workspace must not be shared with
+ * another call in flight. */
+ssd_status ssd_fwd(const ssd_fwd_args* args, void* stream);
+
+/* ---- the four steps of ssd_fwd, exported one by one -------------------- */
+/* Each reads the fields of `args` it needs and the intermediate buffers named
+ * in its signature (device, fp32, caller-owned, 16-byte aligned):
+ *   dt_out, cumA_out  [batch, nheads, nc, chunk]
+ *   states            [batch, nc, nheads, headdim, dstate]
+ */
+
+/* Step 1: dt = softplus(dt_raw + dt_bias) and the inclusive in-chunk
+ * cumulative sum of dt * A_h.  Entries past the end of a short last chunk hold
+ * dt = 0 and the chunk's last cumulative value. */
+ssd_status ssd_chunk_cumsum(const ssd_fwd_args* args, float* dt_out, float* cumA_out,
+                            void* stream);
+
+/* Step 2: each chunk's local state, as if the chunk started from zero:
+ * S_c[p,n] = sum_{l in c} exp(cumA[last] - cumA[l]) * dt[l] * x[l,p] * B[l,n]. */
+ssd_status ssd_chunk_state(const ssd_fwd_args* args, const float* dt, const float* cumA,
+                           float* states, void* stream);
+
+/* Step 3: in place over `states`: reads the local states S_c and replaces each
+ * with the state entering chunk c, H_{c-1} = exp(cumA_{c-1}[last]) H_{c-2} +
+ * S_{c-1} (H before chunk 0 = init_state or 0); writes final_state if given. */
+ssd_status ssd_state_passing(const ssd_fwd_args* args, const float* cumA, float* states,
+                             void* stream);
+
+/* Step 4: y[l,p] = sum_{j<=l in chunk} exp(cumA[l]-cumA[j]) (C_l.B_j) dt[j] x[j,p]
+ *                 + exp(cumA[l]) sum_n C_l[n] H_in[p,n] + D x[l,p],
+ * with H_in the state entering the chunk (states after step 3). */
+ssd_status ssd_chunk_scan(const ssd_fwd_args* args, const float* dt, const float* cumA,
+                          const float* states, void* stream);
+
+/* ---- decode ------------------------------------------------------------- */
+/* One token per sequence against a carried state (the SSM half of the
+ * Mamba2Cache the page "MAMBA-2 Reference Implementations Comparison",
+ * section 1.3, mentions):
+ *   dt = softplus(dt_raw + dt_bias_h);  a = exp(dt A_h)
+ *   state[p,n] <- a state[p,n] + dt x[p] B[n];   y[p] = sum_n state[p,n] C[n] + D x[p]
+ * Layouts: state [batch, nheads, headdim, dstate] fp32, updated in place;
+ *   x, y [batch, nheads, headdim] dtype; dt [batch, nheads] dtype;
+ *   B, C [batch, ngroups, dstate] dtype; A, D, dt_bias [nheads] fp32
+ *   (D, dt_bias may be NULL).
+ * Supported: dstate in {16, 32, 64, 128, 256}; headdim >= 1. */
+typedef struct {
+    int64_t batch, nheads, headdim, dstate, ngroups;
+    int32_t dtype;
+    int32_t flags;          /* reserved, 0 */
+    float* state;
+    const void* x;
+    const void* dt;
+    const float* A;
+    const void* B;
+    const void* C;
+    const float* D;
+    const float* dt_bias;
+    void* y;
+} ssd_state_update_args;
+
+ssd_status ssd_state_update(const ssd_state_update_args* args, void* stream);
+
+/* ---- misc --------------------------------------------------------------- */
+/* Static, human-readable name of a status code. */
+const char* ssd_status_string(ssd_status status);
+
+/* Library version string (static). */
+const char* ssd_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SSD_B200_H */

@@ -1,0 +1,257 @@
+"""Mamba-2 SSD selective scan on NVIDIA B200: Python binding of libssd_b200.so.
+
+The functions here carry the names of the C ABI in include/ssd.h and only
+marshal arguments: they read shapes and device pointers off torch tensors,
+allocate outputs/workspace with torch when the caller does not pass them, and
+call the library on the current torch CUDA stream.  Every step of the scan runs
+in the library's CUDA kernels; there is no CPU fallback, and a missing library
+raises immediately.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "SsdError", "ssd_fwd", "ssd_fwd_workspace_size", "ssd_chunk_cumsum", "ssd_chunk_state",
+    "ssd_state_passing", "ssd_chunk_scan", "ssd_state_update", "ssd_status_string",
+    "ssd_version", "lib_path", "load_library", "SSD_FLAG_CUDA_CORES",
+]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_LIB_FILE = os.path.join(_PKG, "libssd_b200.so")
+
+SSD_OK, SSD_ERR_INVALID_ARG, SSD_ERR_UNSUPPORTED, SSD_ERR_CUDA, SSD_ERR_TIMEOUT = range(5)
+SSD_F32, SSD_BF16 = 0, 1
+SSD_FLAG_CUDA_CORES = 1
+
+_i64, _i32, _vp, _sz = ctypes.c_int64, ctypes.c_int32, ctypes.c_void_p, ctypes.c_size_t
+
+
+class SsdFwdArgs(ctypes.Structure):
+    """Mirror of ssd_fwd_args."""
+    _fields_ = [("batch", _i64), ("seqlen", _i64), ("nheads", _i64), ("headdim", _i64),
+                ("dstate", _i64), ("ngroups", _i64), ("chunk", _i64), ("dtype", _i32),
+                ("flags", _i32), ("x", _vp), ("dt", _vp), ("A", _vp), ("B", _vp), ("C", _vp),
+                ("D", _vp), ("dt_bias", _vp), ("init_state", _vp), ("y", _vp),
+                ("final_state", _vp), ("workspace", _vp), ("workspace_bytes", _sz)]
+
+
+class SsdStateUpdateArgs(ctypes.Structure):
+    """Mirror of ssd_state_update_args."""
+    _fields_ = [("batch", _i64), ("nheads", _i64), ("headdim", _i64), ("dstate", _i64),
+                ("ngroups", _i64), ("dtype", _i32), ("flags", _i32), ("state", _vp),
+                ("x", _vp), ("dt", _vp), ("A", _vp), ("B", _vp), ("C", _vp), ("D", _vp),
+                ("dt_bias", _vp), ("y", _vp)]
+
+
+class SsdError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {ssd_status_string(status)}")
+
+
+_lib = None
+
+
+def lib_path() -> str:
+    return _LIB_FILE
+
+
+def load_library():
+    """Load libssd_b200.so (built by mamba_ssd_scan_b200.build); raises if absent."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_FILE):
+        raise RuntimeError(f"{_LIB_FILE} is missing: run `python -m mamba_ssd_scan_b200.build`")
+    lib = ctypes.CDLL(_LIB_FILE)
+    F = ctypes.POINTER(SsdFwdArgs)
+    lib.ssd_fwd_workspace_size.restype = _sz
+    lib.ssd_fwd_workspace_size.argtypes = [F]
+    lib.ssd_fwd.restype = ctypes.c_int
+    lib.ssd_fwd.argtypes = [F, _vp]
+    lib.ssd_chunk_cumsum.restype = ctypes.c_int
+    lib.ssd_chunk_cumsum.argtypes = [F, _vp, _vp, _vp]
+    lib.ssd_chunk_state.restype = ctypes.c_int
+    lib.ssd_chunk_state.argtypes = [F, _vp, _vp, _vp, _vp]
+    lib.ssd_state_passing.restype = ctypes.c_int
+    lib.ssd_state_passing.argtypes = [F, _vp, _vp, _vp]
+    lib.ssd_chunk_scan.restype = ctypes.c_int
+    lib.ssd_chunk_scan.argtypes = [F, _vp, _vp, _vp, _vp]
+    lib.ssd_state_update.restype = ctypes.c_int
+    lib.ssd_state_update.argtypes = [ctypes.POINTER(SsdStateUpdateArgs), _vp]
+    lib.ssd_status_string.restype = ctypes.c_char_p
+    lib.ssd_status_string.argtypes = [ctypes.c_int]
+    lib.ssd_version.restype = ctypes.c_char_p
+    lib.ssd_version.argtypes = []
+    _lib = lib
+    return lib
+
+
+def ssd_status_string(status: int) -> str:
+    return load_library().ssd_status_string(int(status)).decode()
+
+
+def ssd_version() -> str:
+    return load_library().ssd_version().decode()
+
+
+# ---------------------------------------------------------------------------
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return SSD_F32
+    if t.dtype == torch.bfloat16:
+        return SSD_BF16
+    raise TypeError(f"unsupported dtype {t.dtype} (float32 or bfloat16)")
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return t.data_ptr()
+
+
+def _stream_ptr(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _check(status: int, where: str):
+    if status != SSD_OK:
+        raise SsdError(status, where)
+
+
+def _fwd_args(x, dt, A, B, C, D, dt_bias, chunk, init_state, y, final_state, flags):
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    a = SsdFwdArgs()
+    a.batch, a.seqlen, a.nheads, a.headdim, a.dstate, a.ngroups, a.chunk = b, L, H, P, N, G, chunk
+    a.dtype = _dtype_code(x)
+    a.flags = int(flags)
+    for name, t in (("dt", dt), ("B", B), ("C", C)):
+        if t.dtype != x.dtype:
+            raise TypeError(f"{name} must have x's dtype {x.dtype}")
+    for name, t in (("A", A), ("D", D), ("dt_bias", dt_bias), ("init_state", init_state)):
+        if t is not None and t.dtype != torch.float32:
+            raise TypeError(f"{name} must be float32")
+    a.x, a.dt, a.A, a.B, a.C = _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C)
+    a.D, a.dt_bias, a.init_state = _ptr(D), _ptr(dt_bias), _ptr(init_state)
+    a.y, a.final_state = _ptr(y), _ptr(final_state)
+    return a
+
+
+def ssd_fwd_workspace_size(batch, seqlen, nheads, headdim, dstate, ngroups, chunk,
+                           dtype=torch.bfloat16, flags: int = 0) -> int:
+    a = SsdFwdArgs()
+    a.batch, a.seqlen, a.nheads, a.headdim, a.dstate, a.ngroups, a.chunk = (
+        batch, seqlen, nheads, headdim, dstate, ngroups, chunk)
+    a.dtype = SSD_BF16 if dtype == torch.bfloat16 else SSD_F32
+    a.flags = flags
+    return int(load_library().ssd_fwd_workspace_size(ctypes.byref(a)))
+
+
+def ssd_fwd(x, dt, A, B, C, D=None, dt_bias=None, chunk: int = 256, init_state=None, *,
+            return_final_state: bool = False, y=None, final_state=None, workspace=None,
+            flags: int = 0, stream=None):
+    """The SSD scan forward.  x [b,L,H,P], dt [b,L,H] (raw), B/C [b,L,G,N] in one
+    dtype (float32 or bfloat16); A, D, dt_bias [H] and init_state [b,H,P,N]
+    float32.  Returns y (and the final fp32 state when asked)."""
+    lib = load_library()
+    if y is None:
+        y = torch.empty_like(x)
+    if final_state is None and return_final_state:
+        final_state = torch.empty((x.shape[0], x.shape[2], x.shape[3], B.shape[3]),
+                                  dtype=torch.float32, device=x.device)
+    a = _fwd_args(x, dt, A, B, C, D, dt_bias, chunk, init_state, y, final_state, flags)
+    need = int(lib.ssd_fwd_workspace_size(ctypes.byref(a)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
+    a.workspace = workspace.data_ptr()
+    a.workspace_bytes = workspace.numel() * workspace.element_size()
+    _check(lib.ssd_fwd(ctypes.byref(a), _stream_ptr(stream)), "ssd_fwd")
+    if final_state is not None:
+        return y, final_state
+    return y
+
+
+def _intermediate_shapes(x, B, chunk):
+    b, L, H, P = x.shape
+    N = B.shape[3]
+    nc = (L + chunk - 1) // chunk
+    return (b, H, nc, chunk), (b, nc, H, P, N)
+
+
+def ssd_chunk_cumsum(x, dt, A, B, C, dt_bias=None, chunk: int = 256, *, dt_out=None,
+                     cumA_out=None, stream=None):
+    """Step 1: returns (dt, cumA), each [b, H, nc, chunk] float32."""
+    lib = load_library()
+    vshape, _ = _intermediate_shapes(x, B, chunk)
+    dt_out = dt_out if dt_out is not None else torch.empty(vshape, dtype=torch.float32,
+                                                           device=x.device)
+    cumA_out = cumA_out if cumA_out is not None else torch.empty_like(dt_out)
+    a = _fwd_args(x, dt, A, B, C, None, dt_bias, chunk, None, None, None, 0)
+    _check(lib.ssd_chunk_cumsum(ctypes.byref(a), _ptr(dt_out), _ptr(cumA_out),
+                                _stream_ptr(stream)), "ssd_chunk_cumsum")
+    return dt_out, cumA_out
+
+
+def ssd_chunk_state(x, dt, A, B, C, dt_sp, cumA, chunk: int = 256, *, states=None,
+                    stream=None):
+    """Step 2: returns the chunk-local states [b, nc, H, P, N] float32.
+    ``dt_sp``/``cumA`` are step 1's outputs."""
+    lib = load_library()
+    _, sshape = _intermediate_shapes(x, B, chunk)
+    states = states if states is not None else torch.empty(sshape, dtype=torch.float32,
+                                                           device=x.device)
+    a = _fwd_args(x, dt, A, B, C, None, None, chunk, None, None, None, 0)
+    _check(lib.ssd_chunk_state(ctypes.byref(a), _ptr(dt_sp), _ptr(cumA), _ptr(states),
+                               _stream_ptr(stream)), "ssd_chunk_state")
+    return states
+
+
+def ssd_state_passing(x, dt, A, B, C, cumA, states, chunk: int = 256, init_state=None,
+                      final_state=None, stream=None):
+    """Step 3, in place: ``states`` goes from chunk-local states to the states
+    entering each chunk.  Writes ``final_state`` if given.  Returns states."""
+    lib = load_library()
+    a = _fwd_args(x, dt, A, B, C, None, None, chunk, init_state, None, final_state, 0)
+    _check(lib.ssd_state_passing(ctypes.byref(a), _ptr(cumA), _ptr(states),
+                                 _stream_ptr(stream)), "ssd_state_passing")
+    return states
+
+
+def ssd_chunk_scan(x, dt, A, B, C, dt_sp, cumA, states, D=None, chunk: int = 256, *, y=None,
+                   stream=None):
+    """Step 4: y from the chunk's tokens and the states entering each chunk."""
+    lib = load_library()
+    y = y if y is not None else torch.empty_like(x)
+    a = _fwd_args(x, dt, A, B, C, D, None, chunk, None, y, None, 0)
+    _check(lib.ssd_chunk_scan(ctypes.byref(a), _ptr(dt_sp), _ptr(cumA), _ptr(states),
+                              _stream_ptr(stream)), "ssd_chunk_scan")
+    return y
+
+
+def ssd_state_update(state, x, dt, A, B, C, D=None, dt_bias=None, *, y=None, stream=None):
+    """One decode step, in place on ``state`` [b,H,P,N] float32.  x [b,H,P],
+    dt [b,H], B/C [b,G,N] in one dtype.  Returns y [b,H,P] in x's dtype."""
+    lib = load_library()
+    b, H, P, N = state.shape
+    G = B.shape[1]
+    if state.dtype != torch.float32:
+        raise TypeError("state must be float32")
+    y = y if y is not None else torch.empty_like(x)
+    a = SsdStateUpdateArgs()
+    a.batch, a.nheads, a.headdim, a.dstate, a.ngroups = b, H, P, N, G
+    a.dtype = _dtype_code(x)
+    a.flags = 0
+    a.state, a.x, a.dt, a.A, a.B, a.C = (_ptr(state), _ptr(x), _ptr(dt), _ptr(A), _ptr(B),
+                                         _ptr(C))
+    a.D, a.dt_bias, a.y = _ptr(D), _ptr(dt_bias), _ptr(y)
+    _check(lib.ssd_state_update(ctypes.byref(a), _stream_ptr(stream)), "ssd_state_update")
+    return y

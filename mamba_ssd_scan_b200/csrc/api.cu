@@ -1,0 +1,263 @@
+// api.cu -- the extern "C" entry points of libssd_b200.so (declared and
+// documented in include/ssd.h): argument validation, workspace carving and
+// kernel dispatch.  Nothing here allocates memory or synchronises the host.
+#include <stdint.h>
+#include <string.h>
+
+#include "internal.cuh"
+
+namespace {
+
+using ssd::DecodeParams;
+using ssd::FwdParams;
+
+constexpr size_t kAlign = 256;
+inline size_t round_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// true iff the CUDA runtime knows `p` as memory of the current device
+bool on_current_device(const void* p) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    if (a.type == cudaMemoryTypeManaged) return true;
+    return a.type == cudaMemoryTypeDevice && a.device == dev;
+}
+
+// A required (or optional when allow_null) device pointer, 16-byte aligned
+// when need_align.
+bool check_ptr(const void* p, bool allow_null, bool need_align) {
+    if (!p) return allow_null;
+    if (need_align && !aligned16(p)) return false;
+    return on_current_device(p);
+}
+
+struct WsLayout {
+    size_t dt, cumA, states, total;
+};
+
+WsLayout ws_layout(const ssd_fwd_args& a) {
+    const int64_t nc = (a.seqlen + a.chunk - 1) / a.chunk;
+    const size_t vec = (size_t)a.batch * a.nheads * nc * a.chunk * sizeof(float);
+    const size_t st = (size_t)a.batch * nc * a.nheads * a.headdim * a.dstate * sizeof(float);
+    WsLayout w;
+    w.dt = 0;
+    w.cumA = w.dt + round_up(vec);
+    w.states = w.cumA + round_up(vec);
+    w.total = w.states + round_up(st);
+    return w;
+}
+
+// Sizes and dtype only.
+ssd_status check_fwd_sizes(const ssd_fwd_args* a) {
+    if (!a) return SSD_ERR_INVALID_ARG;
+    if (a->batch <= 0 || a->seqlen <= 0 || a->nheads <= 0 || a->headdim <= 0 ||
+        a->dstate <= 0 || a->ngroups <= 0 || a->chunk <= 0)
+        return SSD_ERR_INVALID_ARG;
+    if (a->nheads % a->ngroups != 0) return SSD_ERR_INVALID_ARG;
+    if (a->dtype != SSD_F32 && a->dtype != SSD_BF16) return SSD_ERR_INVALID_ARG;
+    if (a->chunk > 256) return SSD_ERR_UNSUPPORTED;
+    if (a->dstate % 4 != 0 || a->dstate > 256) return SSD_ERR_UNSUPPORTED;
+    if (a->headdim % 4 != 0) return SSD_ERR_UNSUPPORTED;
+    const int64_t nc = (a->seqlen + a->chunk - 1) / a->chunk;
+    if (a->batch > 65535 || nc * a->nheads > 0x7fffffffLL) return SSD_ERR_UNSUPPORTED;
+    return SSD_OK;
+}
+
+// Pointers of the inputs every step may read.
+ssd_status check_fwd_inputs(const ssd_fwd_args* a) {
+    if (!check_ptr(a->x, false, true) || !check_ptr(a->dt, false, false) ||
+        !check_ptr(a->A, false, false) || !check_ptr(a->B, false, true) ||
+        !check_ptr(a->C, false, true) || !check_ptr(a->D, true, false) ||
+        !check_ptr(a->dt_bias, true, false) || !check_ptr(a->init_state, true, true))
+        return SSD_ERR_INVALID_ARG;
+    return SSD_OK;
+}
+
+FwdParams make_params(const ssd_fwd_args* a) {
+    FwdParams p;
+    p.batch = a->batch;
+    p.seqlen = a->seqlen;
+    p.nheads = a->nheads;
+    p.headdim = a->headdim;
+    p.dstate = a->dstate;
+    p.ngroups = a->ngroups;
+    p.chunk = a->chunk;
+    p.nchunks = (a->seqlen + a->chunk - 1) / a->chunk;
+    p.heads_per_group = a->nheads / a->ngroups;
+    p.x = a->x;
+    p.dt_raw = a->dt;
+    p.A = a->A;
+    p.B = a->B;
+    p.C = a->C;
+    p.D = a->D;
+    p.dt_bias = a->dt_bias;
+    p.init_state = a->init_state;
+    p.y = a->y;
+    p.final_state = a->final_state;
+    p.dt = p.cumA = p.states = nullptr;
+    return p;
+}
+
+ssd_status to_status(cudaError_t e) { return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA; }
+
+cudaError_t run_cumsum(const FwdParams& p, int dtype, cudaStream_t s) {
+    return dtype == SSD_BF16 ? ssd::launch_chunk_cumsum<__nv_bfloat16>(p, s)
+                             : ssd::launch_chunk_cumsum<float>(p, s);
+}
+cudaError_t run_chunk_state(const FwdParams& p, int dtype, cudaStream_t s) {
+    return dtype == SSD_BF16 ? ssd::launch_chunk_state_ffma<__nv_bfloat16>(p, s)
+                             : ssd::launch_chunk_state_ffma<float>(p, s);
+}
+cudaError_t run_chunk_scan(const FwdParams& p, int dtype, cudaStream_t s) {
+    return dtype == SSD_BF16 ? ssd::launch_chunk_scan_ffma<__nv_bfloat16>(p, s)
+                             : ssd::launch_chunk_scan_ffma<float>(p, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t ssd_fwd_workspace_size(const ssd_fwd_args* args) {
+    if (check_fwd_sizes(args) != SSD_OK) return 0;
+    return ws_layout(*args).total;
+}
+
+ssd_status ssd_fwd(const ssd_fwd_args* a, void* stream) {
+    ssd_status st = check_fwd_sizes(a);
+    if (st != SSD_OK) return st;
+    if ((st = check_fwd_inputs(a)) != SSD_OK) return st;
+    if (!check_ptr(a->y, false, true) || !check_ptr(a->final_state, true, true))
+        return SSD_ERR_INVALID_ARG;
+    const WsLayout w = ws_layout(*a);
+    if (!a->workspace || a->workspace_bytes < w.total || !check_ptr(a->workspace, false, true))
+        return SSD_ERR_INVALID_ARG;
+    FwdParams p = make_params(a);
+    char* ws = static_cast<char*>(a->workspace);
+    p.dt = reinterpret_cast<float*>(ws + w.dt);
+    p.cumA = reinterpret_cast<float*>(ws + w.cumA);
+    p.states = reinterpret_cast<float*>(ws + w.states);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = run_cumsum(p, a->dtype, s);
+    if (e == cudaSuccess) e = run_chunk_state(p, a->dtype, s);
+    if (e == cudaSuccess) e = ssd::launch_state_passing(p, s);
+    if (e == cudaSuccess) e = run_chunk_scan(p, a->dtype, s);
+    return to_status(e);
+}
+
+ssd_status ssd_chunk_cumsum(const ssd_fwd_args* a, float* dt_out, float* cumA_out,
+                            void* stream) {
+    ssd_status st = check_fwd_sizes(a);
+    if (st != SSD_OK) return st;
+    if (!check_ptr(a->dt, false, false) || !check_ptr(a->A, false, false) ||
+        !check_ptr(a->dt_bias, true, false) || !check_ptr(dt_out, false, true) ||
+        !check_ptr(cumA_out, false, true))
+        return SSD_ERR_INVALID_ARG;
+    FwdParams p = make_params(a);
+    p.dt = dt_out;
+    p.cumA = cumA_out;
+    return to_status(run_cumsum(p, a->dtype, static_cast<cudaStream_t>(stream)));
+}
+
+ssd_status ssd_chunk_state(const ssd_fwd_args* a, const float* dt, const float* cumA,
+                           float* states, void* stream) {
+    ssd_status st = check_fwd_sizes(a);
+    if (st != SSD_OK) return st;
+    if ((st = check_fwd_inputs(a)) != SSD_OK) return st;
+    if (!check_ptr(dt, false, true) || !check_ptr(cumA, false, true) ||
+        !check_ptr(states, false, true))
+        return SSD_ERR_INVALID_ARG;
+    FwdParams p = make_params(a);
+    p.dt = const_cast<float*>(dt);
+    p.cumA = const_cast<float*>(cumA);
+    p.states = states;
+    return to_status(run_chunk_state(p, a->dtype, static_cast<cudaStream_t>(stream)));
+}
+
+ssd_status ssd_state_passing(const ssd_fwd_args* a, const float* cumA, float* states,
+                             void* stream) {
+    ssd_status st = check_fwd_sizes(a);
+    if (st != SSD_OK) return st;
+    if (!check_ptr(cumA, false, true) || !check_ptr(states, false, true) ||
+        !check_ptr(a->init_state, true, true) || !check_ptr(a->final_state, true, true))
+        return SSD_ERR_INVALID_ARG;
+    FwdParams p = make_params(a);
+    p.cumA = const_cast<float*>(cumA);
+    p.states = states;
+    return to_status(ssd::launch_state_passing(p, static_cast<cudaStream_t>(stream)));
+}
+
+ssd_status ssd_chunk_scan(const ssd_fwd_args* a, const float* dt, const float* cumA,
+                          const float* states, void* stream) {
+    ssd_status st = check_fwd_sizes(a);
+    if (st != SSD_OK) return st;
+    if ((st = check_fwd_inputs(a)) != SSD_OK) return st;
+    if (!check_ptr(a->y, false, true) || !check_ptr(dt, false, true) ||
+        !check_ptr(cumA, false, true) || !check_ptr(states, false, true))
+        return SSD_ERR_INVALID_ARG;
+    FwdParams p = make_params(a);
+    p.dt = const_cast<float*>(dt);
+    p.cumA = const_cast<float*>(cumA);
+    p.states = const_cast<float*>(states);
+    return to_status(run_chunk_scan(p, a->dtype, static_cast<cudaStream_t>(stream)));
+}
+
+ssd_status ssd_state_update(const ssd_state_update_args* a, void* stream) {
+    if (!a) return SSD_ERR_INVALID_ARG;
+    if (a->batch <= 0 || a->nheads <= 0 || a->headdim <= 0 || a->dstate <= 0 ||
+        a->ngroups <= 0 || a->nheads % a->ngroups != 0)
+        return SSD_ERR_INVALID_ARG;
+    if (a->dtype != SSD_F32 && a->dtype != SSD_BF16) return SSD_ERR_INVALID_ARG;
+    if (a->dstate != 16 && a->dstate != 32 && a->dstate != 64 && a->dstate != 128 &&
+        a->dstate != 256)
+        return SSD_ERR_UNSUPPORTED;
+    if (!check_ptr(a->state, false, true) || !check_ptr(a->x, false, false) ||
+        !check_ptr(a->dt, false, false) || !check_ptr(a->A, false, false) ||
+        !check_ptr(a->B, false, true) || !check_ptr(a->C, false, true) ||
+        !check_ptr(a->D, true, false) || !check_ptr(a->dt_bias, true, false) ||
+        !check_ptr(a->y, false, false))
+        return SSD_ERR_INVALID_ARG;
+    DecodeParams p;
+    p.batch = a->batch;
+    p.nheads = a->nheads;
+    p.headdim = a->headdim;
+    p.dstate = a->dstate;
+    p.ngroups = a->ngroups;
+    p.heads_per_group = a->nheads / a->ngroups;
+    p.state = a->state;
+    p.x = a->x;
+    p.dt_raw = a->dt;
+    p.A = a->A;
+    p.B = a->B;
+    p.C = a->C;
+    p.D = a->D;
+    p.dt_bias = a->dt_bias;
+    p.y = a->y;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = a->dtype == SSD_BF16 ? ssd::launch_state_update<__nv_bfloat16>(p, s)
+                                         : ssd::launch_state_update<float>(p, s);
+    return to_status(e);
+}
+
+const char* ssd_status_string(ssd_status s) {
+    switch (s) {
+        case SSD_OK: return "SSD_OK";
+        case SSD_ERR_INVALID_ARG: return "SSD_ERR_INVALID_ARG";
+        case SSD_ERR_UNSUPPORTED: return "SSD_ERR_UNSUPPORTED";
+        case SSD_ERR_CUDA: return "SSD_ERR_CUDA";
+        case SSD_ERR_TIMEOUT: return "SSD_ERR_TIMEOUT";
+        default: return "SSD_ERR_UNKNOWN";
+    }
+}
+
+const char* ssd_version(void) { return "ssd_b200 0.1.0 (sm_100a)"; }
+
+}  // extern "C"

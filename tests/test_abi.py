@@ -1,0 +1,95 @@
+"""The C-ABI library loads, exports every function include/ssd.h declares, and
+rejects bad arguments before touching the GPU (CPU only: no compute calls)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ssd.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from mamba_ssd_scan_b200 import build
+    build.build()
+    import mamba_ssd_scan_b200 as m
+    return m.load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^[A-Za-z_][\w\s\*]*?\b(ssd_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_entry_points():
+    names = declared_functions()
+    for required in ("ssd_fwd", "ssd_fwd_workspace_size", "ssd_state_update",
+                     "ssd_status_string", "ssd_chunk_cumsum", "ssd_chunk_state",
+                     "ssd_state_passing", "ssd_chunk_scan"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    raw = ctypes.CDLL(os.path.join(ROOT, "mamba_ssd_scan_b200", "libssd_b200.so"))
+    missing = [n for n in declared_functions() if not hasattr(raw, n)]
+    assert not missing, f"declared but not exported: {missing}"
+
+
+def test_status_strings(lib):
+    import mamba_ssd_scan_b200 as m
+    assert m.ssd_status_string(0) == "SSD_OK"
+    assert m.ssd_status_string(2) == "SSD_ERR_UNSUPPORTED"
+    assert "sm_100a" in m.ssd_version()
+
+
+def _args(**kw):
+    import mamba_ssd_scan_b200 as m
+    a = m.SsdFwdArgs()
+    a.batch, a.seqlen, a.nheads, a.headdim, a.dstate, a.ngroups, a.chunk = 1, 512, 4, 64, 64, 1, 256
+    a.dtype = m.SSD_BF16
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+def test_workspace_size_is_host_only(lib):
+    a = _args()
+    # dt + cumA: 1*4*2*256 fp32 each; states 1*2*4*64*64 fp32; 256-byte rounding
+    assert lib.ssd_fwd_workspace_size(ctypes.byref(a)) == 8192 + 8192 + 131072
+    assert lib.ssd_fwd_workspace_size(None) == 0
+    assert lib.ssd_fwd_workspace_size(ctypes.byref(_args(nheads=3, ngroups=2))) == 0
+
+
+@pytest.mark.parametrize("bad,status", [
+    (dict(batch=0), 1), (dict(seqlen=-1), 1), (dict(nheads=6, ngroups=4), 1),
+    (dict(dtype=7), 1), (dict(chunk=512), 2), (dict(dstate=66), 2), (dict(dstate=512), 2),
+    (dict(headdim=6), 2),
+])
+def test_fwd_rejects_bad_sizes(lib, bad, status):
+    assert lib.ssd_fwd(ctypes.byref(_args(**bad)), None) == status
+
+
+def test_fwd_rejects_null_and_host_pointers(lib):
+    # null required pointers
+    assert lib.ssd_fwd(ctypes.byref(_args()), None) == 1
+    # host memory is never accepted as device memory
+    buf = ctypes.create_string_buffer(1 << 16)
+    p = ctypes.addressof(buf)
+    a = _args(x=p, dt=p, A=p, B=p, C=p, y=p, workspace=p, workspace_bytes=1 << 16)
+    assert lib.ssd_fwd(ctypes.byref(a), None) == 1
+    assert lib.ssd_fwd(None, None) == 1
+
+
+def test_state_update_rejects_bad_args(lib):
+    import mamba_ssd_scan_b200 as m
+    a = m.SsdStateUpdateArgs()
+    a.batch, a.nheads, a.headdim, a.dstate, a.ngroups, a.dtype = 2, 4, 64, 128, 1, m.SSD_BF16
+    assert lib.ssd_state_update(ctypes.byref(a), None) == 1  # null pointers
+    a.dstate = 48
+    assert lib.ssd_state_update(ctypes.byref(a), None) == 2
+    a.dstate, a.ngroups = 128, 3
+    assert lib.ssd_state_update(ctypes.byref(a), None) == 1

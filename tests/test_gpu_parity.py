@@ -1,0 +1,225 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle.
+
+Small cases are compared element by element over every output; the full-size
+workloads (the same launch configuration the benchmark times) are compared on
+sampled heads / batch rows, which the oracle computes one by one over the
+whole sequence.
+"""
+import numpy as np
+import pytest
+import torch
+
+import mamba_ssd_scan_b200 as ssd
+from mamba_ssd_scan_b200 import synthetic
+from tolerance import assert_close
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def dev(inp):
+    return {k: (v.to(DEV) if v is not None else None) for k, v in inp.items()}
+
+
+def oracle_heads(orc, inp, heads, batches=None):
+    """Oracle y[:, :, heads] and final_state[:, heads] for a subset of heads
+    (and batch rows): each chosen head gets its own group in a smaller problem,
+    so the oracle's threads run the chosen heads side by side."""
+    H, G = inp["x"].shape[2], inp["B"].shape[2]
+    hpg = H // G
+    bsel = slice(None) if batches is None else list(batches)
+    groups = [h // hpg for h in heads]
+    sub = dict(
+        x=inp["x"][bsel][:, :, heads], dt=inp["dt"][bsel][:, :, heads], A=inp["A"][heads],
+        B=inp["B"][bsel][:, :, groups], C=inp["C"][bsel][:, :, groups],
+        D=None if inp["D"] is None else inp["D"][heads],
+        dt_bias=None if inp["dt_bias"] is None else inp["dt_bias"][heads],
+        init_state=None if inp["init_state"] is None else inp["init_state"][bsel][:, heads])
+    return orc.ssd_fwd(**sub)
+
+
+def run_fwd(inp, chunk, flags=0):
+    d = dev(inp)
+    y, fin = ssd.ssd_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["dt_bias"], chunk,
+                         d["init_state"], return_final_state=True, flags=flags)
+    torch.cuda.synchronize()
+    return y, fin
+
+
+# ---------------------------------------------------------------------------
+# full, element-by-element comparisons on small and medium shapes
+CASES = [
+    # (b, L, H, P, N, G, Q, dtype, init)
+    (1, 256, 4, 16, 16, 1, 64, torch.float32, False),      # the small fp32 workload
+    (2, 600, 4, 64, 64, 2, 256, torch.float32, True),      # ragged last chunk (88 tokens)
+    (2, 600, 4, 64, 64, 2, 256, torch.bfloat16, True),
+    (1, 333, 6, 32, 128, 3, 128, torch.bfloat16, False),   # ragged, G=2 heads per group
+    (2, 200, 4, 64, 128, 4, 64, torch.bfloat16, True),     # G = H
+    (1, 1, 2, 16, 16, 1, 64, torch.float32, True),         # L = 1
+    (1, 97, 2, 8, 32, 1, 3, torch.float32, True),          # odd tiny chunk
+    (1, 130, 2, 128, 256, 1, 256, torch.bfloat16, True),   # headdim 128, dstate 256
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "b{}_L{}_H{}_P{}_N{}_G{}_Q{}_{}_{}".format(
+    *c[:7], str(c[7]).split(".")[-1], "init" if c[8] else "zero"))
+def test_fwd_full_compare(orc, case):
+    b, L, H, P, N, G, Q, dtype, init = case
+    inp = synthetic.make_fwd_inputs(b, L, H, P, N, G, dtype, seed=99 + L, init_state=init)
+    y, fin = run_fwd(inp, Q)
+    yo, fo = orc.ssd_fwd(**inp)
+    assert_close(y, yo, dtype, "y")
+    assert_close(fin, fo, dtype, "final_state")
+
+
+@pytest.mark.parametrize("drop", ["D", "dt_bias", "both"])
+def test_fwd_optional_inputs(orc, drop):
+    inp = synthetic.make_fwd_inputs(1, 300, 4, 64, 64, 1, torch.bfloat16, seed=5)
+    if drop in ("D", "both"):
+        inp["D"] = None
+    if drop in ("dt_bias", "both"):
+        inp["dt_bias"] = None
+    y, fin = run_fwd(inp, 256)
+    yo, fo = orc.ssd_fwd(**inp)
+    assert_close(y, yo, torch.bfloat16, "y")
+    assert_close(fin, fo, torch.bfloat16, "final_state")
+
+
+def test_fwd_chunk_size_invariance():
+    """Q in {64, 128, 256} compute the same scan (up to rounding)."""
+    inp = synthetic.make_fwd_inputs(2, 1000, 4, 64, 64, 1, torch.float32, seed=7,
+                                    init_state=True)
+    outs = [run_fwd(inp, Q) for Q in (64, 128, 256)]
+    for y, f in outs[1:]:
+        assert_close(y, outs[0][0], torch.float32, "y across chunk sizes")
+        assert_close(f, outs[0][1], torch.float32, "final across chunk sizes")
+
+
+# ---------------------------------------------------------------------------
+# each of the four steps against the oracle's chunked intermediates
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+@pytest.mark.parametrize("Q", [64, 256])
+def test_steps_against_chunked_oracle(orc, dtype, Q):
+    b, L, H, P, N, G = 2, 600, 4, 64, 64, 2
+    inp = synthetic.make_fwd_inputs(b, L, H, P, N, G, dtype, seed=11, init_state=True)
+    ref = orc.ssd_chunked(**inp, chunk=Q)
+    d = dev(inp)
+    dt_sp, cumA = ssd.ssd_chunk_cumsum(d["x"], d["dt"], d["A"], d["B"], d["C"], d["dt_bias"], Q)
+    nc = (L + Q - 1) // Q
+    valid = np.zeros((b, H, nc, Q), dtype=bool)
+    for c in range(nc):
+        valid[:, :, c, : min(Q, L - c * Q)] = True
+    torch.cuda.synchronize()
+    assert_close(dt_sp.cpu().numpy()[valid], ref["dt"][valid], torch.float32, "dt")
+    assert_close(cumA.cpu().numpy()[valid], ref["cumA"][valid], torch.float32, "cumA")
+    states = ssd.ssd_chunk_state(d["x"], d["dt"], d["A"], d["B"], d["C"], dt_sp, cumA, Q)
+    torch.cuda.synchronize()
+    assert_close(states, ref["S"], dtype, "chunk states")
+    fin = torch.empty((b, H, P, N), dtype=torch.float32, device=DEV)
+    ssd.ssd_state_passing(d["x"], d["dt"], d["A"], d["B"], d["C"], cumA, states, Q,
+                          init_state=d["init_state"], final_state=fin)
+    torch.cuda.synchronize()
+    assert_close(states, ref["Hin"], dtype, "states entering each chunk")
+    assert_close(fin, ref["final_state"], dtype, "final state")
+    y = ssd.ssd_chunk_scan(d["x"], d["dt"], d["A"], d["B"], d["C"], dt_sp, cumA, states,
+                           d["D"], Q)
+    torch.cuda.synchronize()
+    assert_close(y, ref["y"], dtype, "y")
+
+
+# ---------------------------------------------------------------------------
+# the named workloads at full size
+def test_workload_fwd_f32_small(orc):
+    cfg = synthetic.FWD_CONFIGS["fwd_f32_small"]
+    inp = synthetic.make_config_inputs(cfg)
+    y, fin = run_fwd(inp, cfg.chunk)
+    yo, fo = orc.ssd_fwd(**inp)
+    assert_close(y, yo, cfg.dtype, "y")
+    assert_close(fin, fo, cfg.dtype, "final")
+
+
+def test_workload_fwd_bf16_b4_L1024(orc):
+    cfg = synthetic.FWD_CONFIGS["fwd_bf16_b4_L1024"]
+    inp = synthetic.make_config_inputs(cfg)
+    y, fin = run_fwd(inp, cfg.chunk)
+    yo, fo = orc.ssd_fwd(**inp)
+    assert_close(y, yo, cfg.dtype, "y")
+    assert_close(fin, fo, cfg.dtype, "final")
+
+
+@pytest.mark.parametrize("name,heads,batches", [
+    ("fwd_bf16_b8_L4096_init", [0, 13, 31], [0, 7]),
+    ("fwd_bf16_b1_L65536_G8", [0, 9, 10, 47, 79], None),
+])
+def test_workload_sampled_heads(orc, name, heads, batches):
+    cfg = synthetic.FWD_CONFIGS[name]
+    inp = synthetic.make_config_inputs(cfg)
+    y, fin = run_fwd(inp, cfg.chunk)
+    yo, fo = oracle_heads(orc, inp, heads, batches)
+    bsel = slice(None) if batches is None else batches
+    assert_close(y.cpu()[bsel][:, :, heads], yo, cfg.dtype, "y (sampled heads)")
+    assert_close(fin.cpu()[bsel][:, heads], fo, cfg.dtype, "final (sampled heads)")
+
+
+# ---------------------------------------------------------------------------
+# decode
+@pytest.mark.parametrize("N", [16, 32, 64, 128, 256])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+def test_decode_small(orc, N, dtype):
+    b, H, P, G = 3, 4, 16, 2
+    prm = synthetic.make_decode_params(b, H, P, N, seed=3)
+    st_gpu = prm["state"].to(DEV)
+    st_ref = prm["state"].double().numpy()
+    for step in range(3):
+        s = synthetic.make_decode_step(b, H, P, N, G, dtype, seed=3, step=step)
+        y = ssd.ssd_state_update(st_gpu, s["x"].to(DEV), s["dt"].to(DEV), prm["A"].to(DEV),
+                                 s["B"].to(DEV), s["C"].to(DEV), prm["D"].to(DEV),
+                                 prm["dt_bias"].to(DEV))
+        st_ref, yo = orc.state_update(st_ref, s["x"], s["dt"], prm["A"], s["B"], s["C"],
+                                      prm["D"], prm["dt_bias"])
+        torch.cuda.synchronize()
+        assert_close(y, yo, dtype, f"y step {step}")
+        assert_close(st_gpu, st_ref, torch.float32 if dtype == torch.float32 else dtype,
+                     f"state step {step}")
+
+
+def test_decode_workload_1024_steps_sampled(orc):
+    """The decode workload at full size, 1024 successive steps; the oracle
+    follows batch rows 0 and 255 (all heads) through every step."""
+    cfg = synthetic.DECODE_CONFIGS["decode_b256_H80"]
+    seed = 1234 + synthetic.SEED_OFFSET[cfg.name]
+    prm = synthetic.make_decode_params(cfg.batch, cfg.nheads, cfg.headdim, cfg.dstate, seed)
+    rows = [0, cfg.batch - 1]
+    st_gpu = prm["state"].to(DEV)
+    st_ref = prm["state"][rows].double().numpy()
+    A, D, bias = prm["A"].to(DEV), prm["D"].to(DEV), prm["dt_bias"].to(DEV)
+    worst = 0.0
+    for step in range(cfg.steps):
+        s = synthetic.make_decode_step(cfg.batch, cfg.nheads, cfg.headdim, cfg.dstate,
+                                       cfg.ngroups, cfg.dtype, seed, step)
+        y = ssd.ssd_state_update(st_gpu, s["x"].to(DEV), s["dt"].to(DEV), A, s["B"].to(DEV),
+                                 s["C"].to(DEV), D, bias)
+        st_ref, yo = orc.state_update(st_ref, s["x"][rows], s["dt"][rows], prm["A"],
+                                      s["B"][rows], s["C"][rows], prm["D"], prm["dt_bias"])
+        if step % 128 == 0 or step == cfg.steps - 1:
+            assert_close(y.cpu()[rows], yo, cfg.dtype, f"y step {step}")
+    assert_close(st_gpu.cpu()[rows], st_ref, cfg.dtype, "state after 1024 steps")
+
+
+def test_decode_equals_forward_on_gpu():
+    """T decode steps from h0 give the same y and state as one forward call
+    over the same T tokens with init_state h0."""
+    b, T, H, P, N, G = 2, 12, 4, 64, 128, 2
+    inp = synthetic.make_fwd_inputs(b, T, H, P, N, G, torch.float32, seed=21, init_state=True)
+    y_f, fin_f = run_fwd(inp, 64)
+    d = dev(inp)
+    st = d["init_state"].clone()
+    ys = []
+    for t in range(T):
+        ys.append(ssd.ssd_state_update(st, d["x"][:, t].contiguous(), d["dt"][:, t].contiguous(),
+                                       d["A"], d["B"][:, t].contiguous(),
+                                       d["C"][:, t].contiguous(), d["D"], d["dt_bias"]))
+    torch.cuda.synchronize()
+    assert_close(torch.stack(ys, 1), y_f.cpu().double().numpy(), torch.float32, "y")
+    assert_close(st, fin_f.cpu().double().numpy(), torch.float32, "state")

@@ -1,0 +1,57 @@
+"""Agreement rules between the CUDA path and the fp64 oracle.
+
+fp32 inputs: every element |g - o| <= 1e-4 * max(1, |o|).
+bf16 inputs (fp32 accumulation): max |g - o| <= 2e-2 * max |o| over the
+tensor, and every element |g - o| <= 2e-2 * (|o| + rms(o)).
+These are the 1e-4 (fp32) and 2e-2 relative (bf16) bounds of the task; the
+per-element form for bf16 measures each error against the element's own size
+plus the tensor's rms, so near-zero outputs are not held to a relative bound
+that rounding of their (cancelling) terms cannot meet.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+FP32_TOL = 1e-4
+BF16_TOL = 2e-2
+
+
+def _np(a):
+    if isinstance(a, torch.Tensor):
+        return a.detach().to("cpu").double().numpy()
+    return np.asarray(a, dtype=np.float64)
+
+
+def report(gpu, ref):
+    g, o = _np(gpu), _np(ref)
+    d = np.abs(g - o)
+    i = int(np.argmax(d)) if d.size else 0
+    rel = d / np.maximum(np.abs(o), 1e-30)
+    return {"max_abs": float(d.max()) if d.size else 0.0,
+            "max_rel": float(rel.max()) if d.size else 0.0,
+            "argmax": np.unravel_index(i, d.shape) if d.size else (),
+            "ref_max": float(np.abs(o).max()) if d.size else 0.0}
+
+
+def assert_close(gpu, ref, dtype, what=""):
+    g, o = _np(gpu), _np(ref)
+    assert g.shape == o.shape, f"{what}: shape {g.shape} != {o.shape}"
+    assert np.all(np.isfinite(g)), f"{what}: non-finite values in the CUDA result"
+    d = np.abs(g - o)
+    if d.size == 0:
+        return
+    if dtype in (torch.float32, "f32"):
+        bound = FP32_TOL * np.maximum(1.0, np.abs(o))
+        bad = d > bound
+        assert not bad.any(), (f"{what}: {int(bad.sum())} elements beyond the fp32 bound; "
+                               f"{report(g, o)}")
+    else:
+        omax = np.abs(o).max()
+        rms = float(np.sqrt(np.mean(o * o)))
+        assert d.max() <= BF16_TOL * omax + 1e-30, (
+            f"{what}: max abs err {d.max():.3e} > 2e-2 * max|o| = {BF16_TOL * omax:.3e}; "
+            f"{report(g, o)}")
+        bad = d > BF16_TOL * (np.abs(o) + rms)
+        assert not bad.any(), (f"{what}: {int(bad.sum())} elements beyond 2e-2 * (|o| + rms); "
+                               f"{report(g, o)}")
