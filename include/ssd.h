@@ -71,9 +71,12 @@ typedef enum { SSD_F32 = 0, SSD_BF16 = 1 } ssd_dtype;
  *   y            output [batch, seqlen, nheads, headdim], dtype.
  *   final_state  may be NULL: receives h after the last token, fp32.
  * Supported: 1 <= chunk <= 256; dstate a multiple of 4, <= 256; headdim a
- * multiple of 4; the tensor-core path (bf16, headdim in {32, 64, 128},
- * dstate in {64, 128}, chunk 256) is chosen automatically, every other valid
- * shape runs on the CUDA-core path. */
+ * multiple of 4.  bf16 inputs run the contractions on the tensor cores
+ * (tcgen05) where the shape allows -- chunk_state: headdim in {32, 64, 128},
+ * dstate in {64, 128, 256}, 128/headdim dividing the heads per group;
+ * chunk_scan: headdim 64, dstate in {64, 128}, chunk in {128, 256} -- and on
+ * the CUDA cores (fp32 FFMA) otherwise; fp32 inputs always take the CUDA-core
+ * path (its exact fp32 arithmetic is what the 1e-4 agreement needs). */
 typedef struct {
     int64_t batch, seqlen, nheads, headdim, dstate, ngroups, chunk;
     int32_t dtype;          /* ssd_dtype of x, dt, B, C and y */
@@ -103,6 +106,12 @@ size_t ssd_fwd_workspace_size(const ssd_fwd_args* args);
  * dt_bias, init_state.  Stream-ordered; the workspace must not be shared with
  * another call in flight. */
 ssd_status ssd_fwd(const ssd_fwd_args* args, void* stream);
+
+/* Synchronises `stream` and returns the device status of the last ssd_fwd
+ * call that used this workspace: SSD_OK, or SSD_ERR_TIMEOUT when a kernel gave
+ * up on a bounded wait (it then stops early and its outputs are invalid).
+ * Each ssd_fwd call resets the status at its start. */
+ssd_status ssd_fwd_check_status(const ssd_fwd_args* args, void* stream);
 
 /* ---- the four steps of ssd_fwd, exported one by one -------------------- */
 /* Each reads the fields of `args` it needs and the intermediate buffers named

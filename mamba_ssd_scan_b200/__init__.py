@@ -15,7 +15,7 @@ import os
 import torch
 
 __all__ = [
-    "SsdError", "ssd_fwd", "ssd_fwd_workspace_size", "ssd_chunk_cumsum", "ssd_chunk_state",
+    "SsdError", "ssd_fwd", "ssd_fwd_workspace_size", "ssd_fwd_check_status", "ssd_chunk_cumsum", "ssd_chunk_state",
     "ssd_state_passing", "ssd_chunk_scan", "ssd_state_update", "ssd_status_string",
     "ssd_version", "lib_path", "load_library", "SSD_FLAG_CUDA_CORES",
 ]
@@ -73,6 +73,8 @@ def load_library():
     lib.ssd_fwd_workspace_size.argtypes = [F]
     lib.ssd_fwd.restype = ctypes.c_int
     lib.ssd_fwd.argtypes = [F, _vp]
+    lib.ssd_fwd_check_status.restype = ctypes.c_int
+    lib.ssd_fwd_check_status.argtypes = [F, _vp]
     lib.ssd_chunk_cumsum.restype = ctypes.c_int
     lib.ssd_chunk_cumsum.argtypes = [F, _vp, _vp, _vp]
     lib.ssd_chunk_state.restype = ctypes.c_int
@@ -178,6 +180,20 @@ def ssd_fwd(x, dt, A, B, C, D=None, dt_bias=None, chunk: int = 256, init_state=N
     if final_state is not None:
         return y, final_state
     return y
+
+
+def ssd_fwd_check_status(x, B, chunk: int, workspace, flags: int = 0, stream=None) -> int:
+    """Synchronise and return the device status of the last ssd_fwd call that
+    used ``workspace`` (SSD_OK = 0, SSD_ERR_TIMEOUT = 4)."""
+    b, L, H, P = x.shape
+    a = SsdFwdArgs()
+    a.batch, a.seqlen, a.nheads, a.headdim, a.dstate, a.ngroups, a.chunk = (
+        b, L, H, P, B.shape[3], B.shape[2], chunk)
+    a.dtype = _dtype_code(x)
+    a.flags = flags
+    a.workspace = workspace.data_ptr()
+    a.workspace_bytes = workspace.numel() * workspace.element_size()
+    return int(load_library().ssd_fwd_check_status(ctypes.byref(a), _stream_ptr(stream)))
 
 
 def _intermediate_shapes(x, B, chunk):

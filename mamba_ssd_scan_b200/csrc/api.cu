@@ -41,7 +41,7 @@ bool check_ptr(const void* p, bool allow_null, bool need_align) {
 }
 
 struct WsLayout {
-    size_t dt, cumA, states, total;
+    size_t status, dt, cumA, states, total;
 };
 
 WsLayout ws_layout(const ssd_fwd_args& a) {
@@ -49,7 +49,8 @@ WsLayout ws_layout(const ssd_fwd_args& a) {
     const size_t vec = (size_t)a.batch * a.nheads * nc * a.chunk * sizeof(float);
     const size_t st = (size_t)a.batch * nc * a.nheads * a.headdim * a.dstate * sizeof(float);
     WsLayout w;
-    w.dt = 0;
+    w.status = 0;
+    w.dt = w.status + kAlign;
     w.cumA = w.dt + round_up(vec);
     w.states = w.cumA + round_up(vec);
     w.total = w.states + round_up(st);
@@ -104,6 +105,7 @@ FwdParams make_params(const ssd_fwd_args* a) {
     p.y = a->y;
     p.final_state = a->final_state;
     p.dt = p.cumA = p.states = nullptr;
+    p.status = nullptr;
     return p;
 }
 
@@ -113,11 +115,20 @@ cudaError_t run_cumsum(const FwdParams& p, int dtype, cudaStream_t s) {
     return dtype == SSD_BF16 ? ssd::launch_chunk_cumsum<__nv_bfloat16>(p, s)
                              : ssd::launch_chunk_cumsum<float>(p, s);
 }
-cudaError_t run_chunk_state(const FwdParams& p, int dtype, cudaStream_t s) {
+// The tensor-core kernels take bf16 inputs in their shape range unless the
+// caller forces the CUDA-core path; everything else runs on the FFMA kernels.
+bool use_tc(int dtype, int flags) {
+    return dtype == SSD_BF16 && (flags & SSD_FLAG_CUDA_CORES) == 0;
+}
+cudaError_t run_chunk_state(const FwdParams& p, int dtype, int flags, cudaStream_t s) {
+    if (use_tc(dtype, flags) && ssd::chunk_state_tc_supported(p))
+        return ssd::launch_chunk_state_tc(p, s);
     return dtype == SSD_BF16 ? ssd::launch_chunk_state_ffma<__nv_bfloat16>(p, s)
                              : ssd::launch_chunk_state_ffma<float>(p, s);
 }
-cudaError_t run_chunk_scan(const FwdParams& p, int dtype, cudaStream_t s) {
+cudaError_t run_chunk_scan(const FwdParams& p, int dtype, int flags, cudaStream_t s) {
+    if (use_tc(dtype, flags) && ssd::chunk_scan_tc_supported(p))
+        return ssd::launch_chunk_scan_tc(p, s);
     return dtype == SSD_BF16 ? ssd::launch_chunk_scan_ffma<__nv_bfloat16>(p, s)
                              : ssd::launch_chunk_scan_ffma<float>(p, s);
 }
@@ -145,12 +156,28 @@ ssd_status ssd_fwd(const ssd_fwd_args* a, void* stream) {
     p.dt = reinterpret_cast<float*>(ws + w.dt);
     p.cumA = reinterpret_cast<float*>(ws + w.cumA);
     p.states = reinterpret_cast<float*>(ws + w.states);
+    p.status = reinterpret_cast<int*>(ws + w.status);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e = run_cumsum(p, a->dtype, s);
-    if (e == cudaSuccess) e = run_chunk_state(p, a->dtype, s);
+    if (e == cudaSuccess) e = run_chunk_state(p, a->dtype, a->flags, s);
     if (e == cudaSuccess) e = ssd::launch_state_passing(p, s);
-    if (e == cudaSuccess) e = run_chunk_scan(p, a->dtype, s);
+    if (e == cudaSuccess) e = run_chunk_scan(p, a->dtype, a->flags, s);
     return to_status(e);
+}
+
+ssd_status ssd_fwd_check_status(const ssd_fwd_args* a, void* stream) {
+    ssd_status st = check_fwd_sizes(a);
+    if (st != SSD_OK) return st;
+    const WsLayout w = ws_layout(*a);
+    if (!a->workspace || a->workspace_bytes < w.total || !check_ptr(a->workspace, false, true))
+        return SSD_ERR_INVALID_ARG;
+    int v = 0;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(&v, static_cast<char*>(a->workspace) + w.status, sizeof(int),
+                        cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return SSD_ERR_CUDA;
+    return v == 0 ? SSD_OK : static_cast<ssd_status>(v);
 }
 
 ssd_status ssd_chunk_cumsum(const ssd_fwd_args* a, float* dt_out, float* cumA_out,
@@ -179,7 +206,7 @@ ssd_status ssd_chunk_state(const ssd_fwd_args* a, const float* dt, const float* 
     p.dt = const_cast<float*>(dt);
     p.cumA = const_cast<float*>(cumA);
     p.states = states;
-    return to_status(run_chunk_state(p, a->dtype, static_cast<cudaStream_t>(stream)));
+    return to_status(run_chunk_state(p, a->dtype, a->flags, static_cast<cudaStream_t>(stream)));
 }
 
 ssd_status ssd_state_passing(const ssd_fwd_args* a, const float* cumA, float* states,
@@ -207,7 +234,7 @@ ssd_status ssd_chunk_scan(const ssd_fwd_args* a, const float* dt, const float* c
     p.dt = const_cast<float*>(dt);
     p.cumA = const_cast<float*>(cumA);
     p.states = const_cast<float*>(states);
-    return to_status(run_chunk_scan(p, a->dtype, static_cast<cudaStream_t>(stream)));
+    return to_status(run_chunk_scan(p, a->dtype, a->flags, static_cast<cudaStream_t>(stream)));
 }
 
 ssd_status ssd_state_update(const ssd_state_update_args* a, void* stream) {

@@ -22,6 +22,7 @@ __global__ void __launch_bounds__(256) chunk_cumsum_kernel(FwdParams p) {
     const int64_t Lc = (L - t0 < Q) ? (L - t0) : Q;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const T* dtr = static_cast<const T*>(p.dt_raw);
+    if (c == 0 && b == 0 && threadIdx.x == 0 && p.status) *p.status = 0;  // a new call
     for (int64_t h = warp; h < H; h += (blockDim.x >> 5)) {
         const float A = p.A[h];
         const float bias = p.dt_bias ? p.dt_bias[h] : 0.0f;

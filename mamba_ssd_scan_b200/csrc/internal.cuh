@@ -28,6 +28,7 @@ struct FwdParams {
     float* dt;      // [b, H, nc, Q]
     float* cumA;    // [b, H, nc, Q]
     float* states;  // [b, nc, H, P, N] fp32
+    int* status;    // device status word (SSD_ERR_TIMEOUT on a timed-out wait); may be null
 };
 
 struct DecodeParams {
@@ -63,5 +64,11 @@ template <typename T> cudaError_t launch_chunk_state_ffma(const FwdParams& p, cu
 cudaError_t launch_state_passing(const FwdParams& p, cudaStream_t s);
 template <typename T> cudaError_t launch_chunk_scan_ffma(const FwdParams& p, cudaStream_t s);
 template <typename T> cudaError_t launch_state_update(const DecodeParams& p, cudaStream_t s);
+
+// Tensor-core (tcgen05) variants for bf16 inputs, with their shape ranges.
+bool chunk_state_tc_supported(const FwdParams& p);
+cudaError_t launch_chunk_state_tc(const FwdParams& p, cudaStream_t s);
+bool chunk_scan_tc_supported(const FwdParams& p);
+cudaError_t launch_chunk_scan_tc(const FwdParams& p, cudaStream_t s);
 
 }  // namespace ssd

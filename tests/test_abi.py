@@ -29,7 +29,7 @@ def test_header_declares_entry_points():
     names = declared_functions()
     for required in ("ssd_fwd", "ssd_fwd_workspace_size", "ssd_state_update",
                      "ssd_status_string", "ssd_chunk_cumsum", "ssd_chunk_state",
-                     "ssd_state_passing", "ssd_chunk_scan"):
+                     "ssd_state_passing", "ssd_chunk_scan", "ssd_fwd_check_status"):
         assert required in names
 
 
@@ -58,8 +58,8 @@ def _args(**kw):
 
 def test_workspace_size_is_host_only(lib):
     a = _args()
-    # dt + cumA: 1*4*2*256 fp32 each; states 1*2*4*64*64 fp32; 256-byte rounding
-    assert lib.ssd_fwd_workspace_size(ctypes.byref(a)) == 8192 + 8192 + 131072
+    # status word (256 B) + dt + cumA: 1*4*2*256 fp32 each + states 1*2*4*64*64 fp32
+    assert lib.ssd_fwd_workspace_size(ctypes.byref(a)) == 256 + 8192 + 8192 + 131072
     assert lib.ssd_fwd_workspace_size(None) == 0
     assert lib.ssd_fwd_workspace_size(ctypes.byref(_args(nheads=3, ngroups=2))) == 0
 

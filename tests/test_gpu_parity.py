@@ -223,3 +223,30 @@ def test_decode_equals_forward_on_gpu():
     torch.cuda.synchronize()
     assert_close(torch.stack(ys, 1), y_f.cpu().double().numpy(), torch.float32, "y")
     assert_close(st, fin_f.cpu().double().numpy(), torch.float32, "state")
+
+
+# ---------------------------------------------------------------------------
+# the tensor-core path against the CUDA-core path and the oracle
+TC_CASES = [
+    # (b, L, H, P, N, G, Q)  -- shapes the tcgen05 kernels take
+    (2, 512, 4, 64, 64, 1, 256),
+    (1, 700, 6, 64, 128, 3, 256),     # ragged last chunk (188 tokens: second tile partial)
+    (1, 300, 4, 64, 128, 2, 128),     # chunk 128 (one tile), ragged
+    (2, 257, 2, 64, 64, 1, 256),      # last chunk of one token
+    (1, 384, 4, 128, 256, 1, 256),    # chunk_state on tensor cores, chunk_scan on CUDA cores
+    (1, 256, 8, 32, 64, 2, 256),      # headdim 32 (4 heads per chunk_state tile)
+]
+
+
+@pytest.mark.parametrize("case", TC_CASES, ids=lambda c: "b{}_L{}_H{}_P{}_N{}_G{}_Q{}".format(*c))
+def test_tensor_core_path(orc, case):
+    b, L, H, P, N, G, Q = case
+    inp = synthetic.make_fwd_inputs(b, L, H, P, N, G, torch.bfloat16, seed=L + N,
+                                    init_state=True)
+    y_tc, f_tc = run_fwd(inp, Q)
+    y_cc, f_cc = run_fwd(inp, Q, flags=ssd.SSD_FLAG_CUDA_CORES)
+    yo, fo = orc.ssd_fwd(**inp)
+    assert_close(y_tc, yo, torch.bfloat16, "tensor-core y")
+    assert_close(f_tc, fo, torch.bfloat16, "tensor-core final")
+    assert_close(y_cc, yo, torch.bfloat16, "CUDA-core y")
+    assert_close(f_cc, fo, torch.bfloat16, "CUDA-core final")
