@@ -270,7 +270,10 @@ def main_ours(args):
            for i, n in enumerate(names)}
     cost = algorithmic_cost(cfg, elt)
     top = max(names, key=lambda n: kms[n])
-    roofline = roofline_entry(top, cost[top], kms[top], peaks, clocks.summary())
+    tc = ssd.tensor_core_steps(cfg.batch, cfg.seqlen, cfg.nheads, cfg.headdim, cfg.dstate,
+                               cfg.ngroups, cfg.chunk, cfg.dtype)
+    roofline = roofline_entry(top, cost[top], kms[top], peaks, clocks.summary(),
+                              top in tc)
 
     # ---- e2e through the public API from pinned host buffers ------------
     e2e = None
@@ -346,26 +349,35 @@ def main_ours(args):
         dist.destroy_process_group()
 
 
-def roofline_entry(name, cost, ms, peaks, clk):
+def roofline_entry(name, cost, ms, peaks, clk, on_tensor_cores):
+    """Roofline position of one kernel: the larger of its HBM time (algorithmic
+    bytes / measured copy bandwidth) and its compute time (algorithmic FLOP /
+    the peak of the unit that executes them) names the bound."""
     nbytes, flops = cost
     sec = ms * 1e-3
     hbm = peaks["hbm_gbs"]
     t_hbm = nbytes / (hbm * 1e9)
-    # the CUDA-core path executes its contractions as fp32 FFMA; its compute
-    # peak is 148 SMs x 128 FP32 lanes x 2 FLOP x SM clock
-    mhz = clk.get("sm_mhz") or peaks.get("sm_max_mhz", 1965.0)
-    alu_peak = N_SM * FFMA_LANES_PER_SM * 2 * mhz * 1e6 / 1e12  # TFLOP/s
-    t_alu = flops / (alu_peak * 1e12) if flops else 0.0
-    if t_alu > t_hbm:
+    if on_tensor_cores:
+        # the kernel is timed inside short steps: the burst GEMM figure
+        cpeak, cunit = peaks["bf16_tflops"], "bf16 tensor (cuBLAS burst)"
+    else:
+        # fp32 FFMA: 148 SMs x 128 FP32 lanes x 2 FLOP x SM clock
+        mhz = clk.get("sm_mhz") or peaks.get("sm_max_mhz", 1965.0)
+        cpeak = N_SM * FFMA_LANES_PER_SM * 2 * mhz * 1e6 / 1e12
+        cunit = f"FFMA 148 SM x 128 lanes x 2 x {mhz:.0f} MHz"
+    t_cmp = flops / (cpeak * 1e12) if flops else 0.0
+    src = peaks.get("source")
+    if t_cmp > t_hbm:
         ach = flops / sec / 1e12
-        return {"kernel": name, "bound": "alu", "achieved": ach, "peak": alu_peak,
-                "unit": "TFLOP/s", "frac": ach / alu_peak, "traffic": None,
-                "peak_note": f"FFMA: 148 SM x 128 lanes x 2 x {mhz:.0f} MHz (sampled)",
+        return {"kernel": name, "bound": "tensor" if on_tensor_cores else "alu",
+                "achieved": ach, "peak": cpeak, "unit": "TFLOP/s", "frac": ach / cpeak,
+                "traffic": None, "peak_note": f"{cunit}, {src}",
                 "algorithmic_bytes": nbytes, "algorithmic_flops": flops}
     ach = nbytes / sec / 1e9
     return {"kernel": name, "bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s",
-            "frac": ach / hbm, "traffic": None, "peak_note": f"{peaks.get('source')} copy BW",
-            "algorithmic_bytes": nbytes, "algorithmic_flops": flops}
+            "frac": ach / hbm, "traffic": None, "peak_note": f"copy bandwidth, {src}",
+            "algorithmic_bytes": nbytes, "algorithmic_flops": flops,
+            "compute_frac": (flops / sec / 1e12) / cpeak if flops else 0.0}
 
 
 def other_workloads(ssd, synthetic, dev, flush, peaks, rank, world, barrier, max_over_ranks):

@@ -97,10 +97,19 @@ typedef struct {
 
 /* flags */
 #define SSD_FLAG_CUDA_CORES 1   /* force the CUDA-core (FFMA) path */
+#define SSD_FLAG_WHOLE_GROUPS 2 /* tensor-core chunk_scan: one CTA per whole group
+                                   of heads (fewest B/C reads, fewest CTAs) */
 
 /* Bytes of device workspace ssd_fwd needs for these sizes (0 on invalid
  * sizes).  Only sizes, dtype and flags are read; pointers may be NULL. */
 size_t ssd_fwd_workspace_size(const ssd_fwd_args* args);
+
+/* Which steps of ssd_fwd run on the tensor cores for these sizes, dtype and
+ * flags: bit 0 = chunk_state, bit 1 = chunk_scan (0 = all on CUDA cores, or
+ * invalid sizes).  Host-only; pointers are not read. */
+#define SSD_TC_CHUNK_STATE 1
+#define SSD_TC_CHUNK_SCAN 2
+int ssd_fwd_tensor_core_steps(const ssd_fwd_args* args);
 
 /* The whole forward scan: y (and final_state) from x, dt, A, B, C, D,
  * dt_bias, init_state.  Stream-ordered; the workspace must not be shared with

@@ -15,9 +15,10 @@ import os
 import torch
 
 __all__ = [
-    "SsdError", "ssd_fwd", "ssd_fwd_workspace_size", "ssd_fwd_check_status", "ssd_chunk_cumsum", "ssd_chunk_state",
+    "SsdError", "ssd_fwd", "ssd_fwd_workspace_size", "ssd_fwd_check_status",
+    "ssd_fwd_tensor_core_steps", "tensor_core_steps", "ssd_chunk_cumsum", "ssd_chunk_state",
     "ssd_state_passing", "ssd_chunk_scan", "ssd_state_update", "ssd_status_string",
-    "ssd_version", "lib_path", "load_library", "SSD_FLAG_CUDA_CORES",
+    "ssd_version", "lib_path", "load_library", "SSD_FLAG_CUDA_CORES", "SSD_FLAG_WHOLE_GROUPS",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -26,6 +27,7 @@ _LIB_FILE = os.path.join(_PKG, "libssd_b200.so")
 SSD_OK, SSD_ERR_INVALID_ARG, SSD_ERR_UNSUPPORTED, SSD_ERR_CUDA, SSD_ERR_TIMEOUT = range(5)
 SSD_F32, SSD_BF16 = 0, 1
 SSD_FLAG_CUDA_CORES = 1
+SSD_FLAG_WHOLE_GROUPS = 2
 
 _i64, _i32, _vp, _sz = ctypes.c_int64, ctypes.c_int32, ctypes.c_void_p, ctypes.c_size_t
 
@@ -73,6 +75,8 @@ def load_library():
     lib.ssd_fwd_workspace_size.argtypes = [F]
     lib.ssd_fwd.restype = ctypes.c_int
     lib.ssd_fwd.argtypes = [F, _vp]
+    lib.ssd_fwd_tensor_core_steps.restype = ctypes.c_int
+    lib.ssd_fwd_tensor_core_steps.argtypes = [F]
     lib.ssd_fwd_check_status.restype = ctypes.c_int
     lib.ssd_fwd_check_status.argtypes = [F, _vp]
     lib.ssd_chunk_cumsum.restype = ctypes.c_int
@@ -156,6 +160,26 @@ def ssd_fwd_workspace_size(batch, seqlen, nheads, headdim, dstate, ngroups, chun
     a.dtype = SSD_BF16 if dtype == torch.bfloat16 else SSD_F32
     a.flags = flags
     return int(load_library().ssd_fwd_workspace_size(ctypes.byref(a)))
+
+
+def ssd_fwd_tensor_core_steps(batch, seqlen, nheads, headdim, dstate, ngroups, chunk,
+                              dtype=torch.bfloat16, flags: int = 0) -> int:
+    """Bitmask of the ssd_fwd steps that run on the tensor cores for these sizes
+    (1 = chunk_state, 2 = chunk_scan)."""
+    a = SsdFwdArgs()
+    a.batch, a.seqlen, a.nheads, a.headdim, a.dstate, a.ngroups, a.chunk = (
+        batch, seqlen, nheads, headdim, dstate, ngroups, chunk)
+    a.dtype = SSD_BF16 if dtype == torch.bfloat16 else SSD_F32
+    a.flags = flags
+    return int(load_library().ssd_fwd_tensor_core_steps(ctypes.byref(a)))
+
+
+def tensor_core_steps(batch, seqlen, nheads, headdim, dstate, ngroups, chunk,
+                      dtype=torch.bfloat16, flags: int = 0) -> set:
+    """Names of the ssd_fwd steps that run on the tensor cores for these sizes."""
+    m = ssd_fwd_tensor_core_steps(batch, seqlen, nheads, headdim, dstate, ngroups, chunk,
+                                  dtype, flags)
+    return {n for bit, n in ((1, "chunk_state"), (2, "chunk_scan")) if m & bit}
 
 
 def ssd_fwd(x, dt, A, B, C, D=None, dt_bias=None, chunk: int = 256, init_state=None, *,

@@ -94,6 +94,7 @@ FwdParams make_params(const ssd_fwd_args* a) {
     p.chunk = a->chunk;
     p.nchunks = (a->seqlen + a->chunk - 1) / a->chunk;
     p.heads_per_group = a->nheads / a->ngroups;
+    p.flags = a->flags;
     p.x = a->x;
     p.dt_raw = a->dt;
     p.A = a->A;
@@ -140,6 +141,13 @@ extern "C" {
 size_t ssd_fwd_workspace_size(const ssd_fwd_args* args) {
     if (check_fwd_sizes(args) != SSD_OK) return 0;
     return ws_layout(*args).total;
+}
+
+int ssd_fwd_tensor_core_steps(const ssd_fwd_args* a) {
+    if (check_fwd_sizes(a) != SSD_OK || !use_tc(a->dtype, a->flags)) return 0;
+    const FwdParams p = make_params(a);
+    return (ssd::chunk_state_tc_supported(p) ? SSD_TC_CHUNK_STATE : 0) |
+           (ssd::chunk_scan_tc_supported(p) ? SSD_TC_CHUNK_SCAN : 0);
 }
 
 ssd_status ssd_fwd(const ssd_fwd_args* a, void* stream) {

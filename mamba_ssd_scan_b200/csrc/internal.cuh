@@ -14,6 +14,7 @@ namespace ssd {
 struct FwdParams {
     int64_t batch, seqlen, nheads, headdim, dstate, ngroups, chunk, nchunks;
     int64_t heads_per_group;
+    int32_t flags;         // SSD_FLAG_* of the call
     const void* x;
     const void* dt_raw;
     const float* A;

@@ -1,0 +1,48 @@
+// tma.cuh -- tensor-memory-accelerator (TMA) loads: the host builds a tiled
+// tensor map (cuTensorMapEncodeTiled, reached through the runtime's driver
+// entry point so the library does not link libcuda) and one thread per CTA
+// issues cp.async.bulk.tensor loads that complete on an mbarrier.  Loads only,
+// never with cluster multicast.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ssd {
+
+// 4-D bf16 tensor [d3][d2][d1][d0] (d0 innermost, dense), a box of
+// {64, 1, rows, 1} elements with the 128-byte swizzle: it lands in shared
+// memory as `rows` 128-byte rows in the SW128 layout.  Elements outside the
+// tensor read as zero.  Returns false if the encoder is unavailable or
+// rejects the arguments.
+bool make_tmap_bf16_4d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1,
+                       uint64_t d2, uint64_t d3, uint32_t rows);
+
+namespace tc {
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t mbar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
+                 :
+                 : "r"(mbar), "r"(bytes)
+                 : "memory");
+}
+
+// One box of a 4-D tensor map into shared memory; completes `bytes` on mbar.
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, uint32_t mbar,
+                                            int c0, int c1, int c2, int c3) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6}], [%2];"
+        :
+        : "r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(mbar), "r"(c0), "r"(c1), "r"(c2),
+          "r"(c3)
+        : "memory");
+}
+
+__device__ __forceinline__ void tma_prefetch_map(const CUtensorMap* map) {
+    asm volatile("prefetch.tensormap [%0];" : : "l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+}  // namespace tc
+}  // namespace ssd

@@ -39,6 +39,17 @@ def test_every_declared_symbol_is_exported(lib):
     assert not missing, f"declared but not exported: {missing}"
 
 
+def test_tensor_core_dispatch_query(lib):
+    import torch
+
+    import mamba_ssd_scan_b200 as m
+    assert m.tensor_core_steps(4, 1024, 24, 64, 64, 1, 256) == {"chunk_state", "chunk_scan"}
+    assert m.tensor_core_steps(4, 1024, 24, 64, 64, 1, 256, torch.float32) == set()
+    assert m.tensor_core_steps(4, 1024, 24, 64, 64, 1, 256, flags=m.SSD_FLAG_CUDA_CORES) == set()
+    assert m.tensor_core_steps(1, 512, 2, 128, 256, 1, 256) == {"chunk_state"}
+    assert m.tensor_core_steps(1, 512, 4, 64, 128, 4, 64) == set()  # 1 head per group, chunk 64
+
+
 def test_status_strings(lib):
     import mamba_ssd_scan_b200 as m
     assert m.ssd_status_string(0) == "SSD_OK"

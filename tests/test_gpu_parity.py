@@ -235,6 +235,7 @@ TC_CASES = [
     (2, 257, 2, 64, 64, 1, 256),      # last chunk of one token
     (1, 384, 4, 128, 256, 1, 256),    # chunk_state on tensor cores, chunk_scan on CUDA cores
     (1, 256, 8, 32, 64, 2, 256),      # headdim 32 (4 heads per chunk_state tile)
+    (2, 600, 12, 64, 128, 2, 256),    # 6 heads per group
 ]
 
 
@@ -244,9 +245,12 @@ def test_tensor_core_path(orc, case):
     inp = synthetic.make_fwd_inputs(b, L, H, P, N, G, torch.bfloat16, seed=L + N,
                                     init_state=True)
     y_tc, f_tc = run_fwd(inp, Q)
+    y_wg, f_wg = run_fwd(inp, Q, flags=ssd.SSD_FLAG_WHOLE_GROUPS)
     y_cc, f_cc = run_fwd(inp, Q, flags=ssd.SSD_FLAG_CUDA_CORES)
     yo, fo = orc.ssd_fwd(**inp)
     assert_close(y_tc, yo, torch.bfloat16, "tensor-core y")
     assert_close(f_tc, fo, torch.bfloat16, "tensor-core final")
+    assert_close(y_wg, yo, torch.bfloat16, "tensor-core y, whole groups per CTA")
+    assert torch.equal(f_wg, f_tc)  # the head blocking changes only chunk_scan
     assert_close(y_cc, yo, torch.bfloat16, "CUDA-core y")
     assert_close(f_cc, fo, torch.bfloat16, "CUDA-core final")
