@@ -141,7 +141,7 @@ def algorithmic_cost(cfg, elt):
     bc = tok * G * N * elt
     dtr = tok * H * elt
     vec = b * H * nc * Q * 4
-    states = b * nc * H * P * N * 4
+    states = b * nc * H * P * N * elt     # chunk states are kept in the input dtype
     init = b * H * P * N * 4 if cfg.init_state else 0
     fin = b * H * P * N * 4 if cfg.return_final else 0
     causal = Q * (Q + 1) / 2
@@ -238,7 +238,8 @@ def main_ours(args):
     nc = -(-cfg.seqlen // cfg.chunk)
     dt_sp = torch.empty((cfg.batch, cfg.nheads, nc, cfg.chunk), device=dev)
     cumA = torch.empty_like(dt_sp)
-    states = torch.empty((cfg.batch, nc, cfg.nheads, cfg.headdim, cfg.dstate), device=dev)
+    states = torch.empty((cfg.batch, nc, cfg.nheads, cfg.headdim, cfg.dstate), device=dev,
+                         dtype=cfg.dtype)
     names = ["chunk_cumsum", "chunk_state", "state_passing", "chunk_scan"]
 
     def step_split(evs):

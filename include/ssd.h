@@ -124,9 +124,11 @@ ssd_status ssd_fwd_check_status(const ssd_fwd_args* args, void* stream);
 
 /* ---- the four steps of ssd_fwd, exported one by one -------------------- */
 /* Each reads the fields of `args` it needs and the intermediate buffers named
- * in its signature (device, fp32, caller-owned, 16-byte aligned):
- *   dt_out, cumA_out  [batch, nheads, nc, chunk]
- *   states            [batch, nc, nheads, headdim, dstate]
+ * in its signature (device, caller-owned, 16-byte aligned):
+ *   dt_out, cumA_out  [batch, nheads, nc, chunk]                 fp32
+ *   states            [batch, nc, nheads, headdim, dstate]       in args->dtype
+ * (chunk states are stored in the input dtype -- bf16 for bf16 inputs -- and
+ * accumulated in fp32; the carry across chunks is fp32 in registers).
  */
 
 /* Step 1: dt = softplus(dt_raw + dt_bias) and the inclusive in-chunk
@@ -138,19 +140,19 @@ ssd_status ssd_chunk_cumsum(const ssd_fwd_args* args, float* dt_out, float* cumA
 /* Step 2: each chunk's local state, as if the chunk started from zero:
  * S_c[p,n] = sum_{l in c} exp(cumA[last] - cumA[l]) * dt[l] * x[l,p] * B[l,n]. */
 ssd_status ssd_chunk_state(const ssd_fwd_args* args, const float* dt, const float* cumA,
-                           float* states, void* stream);
+                           void* states, void* stream);
 
 /* Step 3: in place over `states`: reads the local states S_c and replaces each
  * with the state entering chunk c, H_{c-1} = exp(cumA_{c-1}[last]) H_{c-2} +
  * S_{c-1} (H before chunk 0 = init_state or 0); writes final_state if given. */
-ssd_status ssd_state_passing(const ssd_fwd_args* args, const float* cumA, float* states,
+ssd_status ssd_state_passing(const ssd_fwd_args* args, const float* cumA, void* states,
                              void* stream);
 
 /* Step 4: y[l,p] = sum_{j<=l in chunk} exp(cumA[l]-cumA[j]) (C_l.B_j) dt[j] x[j,p]
  *                 + exp(cumA[l]) sum_n C_l[n] H_in[p,n] + D x[l,p],
  * with H_in the state entering the chunk (states after step 3). */
 ssd_status ssd_chunk_scan(const ssd_fwd_args* args, const float* dt, const float* cumA,
-                          const float* states, void* stream);
+                          const void* states, void* stream);
 
 /* ---- decode ------------------------------------------------------------- */
 /* One token per sequence against a carried state (the SSM half of the

@@ -243,11 +243,11 @@ def ssd_chunk_cumsum(x, dt, A, B, C, dt_bias=None, chunk: int = 256, *, dt_out=N
 
 def ssd_chunk_state(x, dt, A, B, C, dt_sp, cumA, chunk: int = 256, *, states=None,
                     stream=None):
-    """Step 2: returns the chunk-local states [b, nc, H, P, N] float32.
+    """Step 2: returns the chunk-local states [b, nc, H, P, N] in x's dtype.
     ``dt_sp``/``cumA`` are step 1's outputs."""
     lib = load_library()
     _, sshape = _intermediate_shapes(x, B, chunk)
-    states = states if states is not None else torch.empty(sshape, dtype=torch.float32,
+    states = states if states is not None else torch.empty(sshape, dtype=x.dtype,
                                                            device=x.device)
     a = _fwd_args(x, dt, A, B, C, None, None, chunk, None, None, None, 0)
     _check(lib.ssd_chunk_state(ctypes.byref(a), _ptr(dt_sp), _ptr(cumA), _ptr(states),

@@ -47,7 +47,8 @@ struct WsLayout {
 WsLayout ws_layout(const ssd_fwd_args& a) {
     const int64_t nc = (a.seqlen + a.chunk - 1) / a.chunk;
     const size_t vec = (size_t)a.batch * a.nheads * nc * a.chunk * sizeof(float);
-    const size_t st = (size_t)a.batch * nc * a.nheads * a.headdim * a.dstate * sizeof(float);
+    const size_t elt = a.dtype == SSD_BF16 ? 2 : 4;  // chunk states are kept in the input dtype
+    const size_t st = (size_t)a.batch * nc * a.nheads * a.headdim * a.dstate * elt;
     WsLayout w;
     w.status = 0;
     w.dt = w.status + kAlign;
@@ -105,7 +106,8 @@ FwdParams make_params(const ssd_fwd_args* a) {
     p.init_state = a->init_state;
     p.y = a->y;
     p.final_state = a->final_state;
-    p.dt = p.cumA = p.states = nullptr;
+    p.dt = p.cumA = nullptr;
+    p.states = nullptr;
     p.status = nullptr;
     return p;
 }
@@ -120,6 +122,10 @@ cudaError_t run_cumsum(const FwdParams& p, int dtype, cudaStream_t s) {
 // caller forces the CUDA-core path; everything else runs on the FFMA kernels.
 bool use_tc(int dtype, int flags) {
     return dtype == SSD_BF16 && (flags & SSD_FLAG_CUDA_CORES) == 0;
+}
+cudaError_t run_state_passing(const FwdParams& p, int dtype, cudaStream_t s) {
+    return dtype == SSD_BF16 ? ssd::launch_state_passing<__nv_bfloat16>(p, s)
+                             : ssd::launch_state_passing<float>(p, s);
 }
 cudaError_t run_chunk_state(const FwdParams& p, int dtype, int flags, cudaStream_t s) {
     if (use_tc(dtype, flags) && ssd::chunk_state_tc_supported(p))
@@ -163,12 +169,12 @@ ssd_status ssd_fwd(const ssd_fwd_args* a, void* stream) {
     char* ws = static_cast<char*>(a->workspace);
     p.dt = reinterpret_cast<float*>(ws + w.dt);
     p.cumA = reinterpret_cast<float*>(ws + w.cumA);
-    p.states = reinterpret_cast<float*>(ws + w.states);
+    p.states = ws + w.states;
     p.status = reinterpret_cast<int*>(ws + w.status);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e = run_cumsum(p, a->dtype, s);
     if (e == cudaSuccess) e = run_chunk_state(p, a->dtype, a->flags, s);
-    if (e == cudaSuccess) e = ssd::launch_state_passing(p, s);
+    if (e == cudaSuccess) e = run_state_passing(p, a->dtype, s);
     if (e == cudaSuccess) e = run_chunk_scan(p, a->dtype, a->flags, s);
     return to_status(e);
 }
@@ -203,7 +209,7 @@ ssd_status ssd_chunk_cumsum(const ssd_fwd_args* a, float* dt_out, float* cumA_ou
 }
 
 ssd_status ssd_chunk_state(const ssd_fwd_args* a, const float* dt, const float* cumA,
-                           float* states, void* stream) {
+                           void* states, void* stream) {
     ssd_status st = check_fwd_sizes(a);
     if (st != SSD_OK) return st;
     if ((st = check_fwd_inputs(a)) != SSD_OK) return st;
@@ -217,7 +223,7 @@ ssd_status ssd_chunk_state(const ssd_fwd_args* a, const float* dt, const float* 
     return to_status(run_chunk_state(p, a->dtype, a->flags, static_cast<cudaStream_t>(stream)));
 }
 
-ssd_status ssd_state_passing(const ssd_fwd_args* a, const float* cumA, float* states,
+ssd_status ssd_state_passing(const ssd_fwd_args* a, const float* cumA, void* states,
                              void* stream) {
     ssd_status st = check_fwd_sizes(a);
     if (st != SSD_OK) return st;
@@ -227,11 +233,11 @@ ssd_status ssd_state_passing(const ssd_fwd_args* a, const float* cumA, float* st
     FwdParams p = make_params(a);
     p.cumA = const_cast<float*>(cumA);
     p.states = states;
-    return to_status(ssd::launch_state_passing(p, static_cast<cudaStream_t>(stream)));
+    return to_status(run_state_passing(p, a->dtype, static_cast<cudaStream_t>(stream)));
 }
 
 ssd_status ssd_chunk_scan(const ssd_fwd_args* a, const float* dt, const float* cumA,
-                          const float* states, void* stream) {
+                          const void* states, void* stream) {
     ssd_status st = check_fwd_sizes(a);
     if (st != SSD_OK) return st;
     if ((st = check_fwd_inputs(a)) != SSD_OK) return st;
@@ -241,7 +247,7 @@ ssd_status ssd_chunk_scan(const ssd_fwd_args* a, const float* dt, const float* c
     FwdParams p = make_params(a);
     p.dt = const_cast<float*>(dt);
     p.cumA = const_cast<float*>(cumA);
-    p.states = const_cast<float*>(states);
+    p.states = const_cast<void*>(states);
     return to_status(run_chunk_scan(p, a->dtype, a->flags, static_cast<cudaStream_t>(stream)));
 }
 

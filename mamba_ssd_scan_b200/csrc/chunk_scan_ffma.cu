@@ -41,7 +41,7 @@ __global__ void __launch_bounds__(256) chunk_scan_ffma_kernel(FwdParams p) {
     const T* x = static_cast<const T*>(p.x);
     const T* Bm = static_cast<const T*>(p.B);
     const T* Cm = static_cast<const T*>(p.C);
-    const float* Hin = p.states + ((b * nc + c) * H + h) * P * N;
+    const T* Hin = static_cast<const T*>(p.states) + ((b * nc + c) * H + h) * P * N;
     const int64_t SN = cs_stride(N);
 
     extern __shared__ float smem[];
@@ -67,7 +67,7 @@ __global__ void __launch_bounds__(256) chunk_scan_ffma_kernel(FwdParams p) {
         for (int i = tid; i < TJ * TPP; i += 256) {
             const int kk = i / TPP, pp = i % TPP;
             const int64_t n = n0 + kk, pi = p0 + pp;
-            Xs[kk * TPP + pp] = (n < N && pi < P) ? Hin[pi * N + n] : 0.0f;
+            Xs[kk * TPP + pp] = (n < N && pi < P) ? to_f32(Hin[pi * N + n]) : 0.0f;
         }
         __syncthreads();
         const int64_t kmax = (N - n0 < TJ) ? (N - n0) : TJ;

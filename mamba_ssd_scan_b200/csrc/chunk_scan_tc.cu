@@ -16,7 +16,8 @@
 // as a bf16 K-major operand to shared memory; the tensor core accumulates the
 // state term C_t H_in^T and Mk x into TMEM; the epilogue adds D x and stores y.
 // Each head's x tile arrives by TMA into one of two buffers while the previous
-// head computes.  Decays are never formed as exp(cumA_l) / exp(cumA_j): below
+// head computes; its state entering the chunk (bf16, as state passing left it)
+// arrives by TMA too.  Decays are never formed as exp(cumA_l) / exp(cumA_j): below
 // the 32x32 diagonal blocks the factor is split as exp(cumA_l - cumA_r) *
 // exp(cumA_r - cumA_j) with r the first row of the thread's 32-row block (both
 // factors <= 1, one table of the second per warp); only the diagonal blocks
@@ -135,33 +136,12 @@ __device__ __forceinline__ void epilogue(int t, uint32_t tmem, uint32_t xbase, c
     }
 }
 
-// The state entering chunk c for one head: fp32 in global -> bf16 K-major
-// [kb][p][64 n] SW128 operand (each step converts 8 consecutive fp32).
-template <int NST>
-__device__ __forceinline__ void load_hin(uint32_t hbase, const float* hin, int tid) {
-    constexpr int CPR = NST / 8;             // chunks per p row
-    constexpr int STEPS = PD * CPR / 256;    // per thread; all loads issued before any store
-    float4 a[STEPS], d[STEPS];
-#pragma unroll
-    for (int k = 0; k < STEPS; ++k) {
-        const int i = tid + 256 * k, pr = i / CPR, cc = i % CPR;
-        a[k] = __ldg(reinterpret_cast<const float4*>(hin + pr * NST + cc * 8));
-        d[k] = __ldg(reinterpret_cast<const float4*>(hin + pr * NST + cc * 8 + 4));
-    }
-#pragma unroll
-    for (int k = 0; k < STEPS; ++k) {
-        const int i = tid + 256 * k, pr = i / CPR, cc = i % CPR;
-        st_shared_v4(hbase + (cc >> 3) * (PD * 128) + sw128(pr, cc & 7),
-                     pack_bf16x2(a[k].x, a[k].y), pack_bf16x2(a[k].z, a[k].w),
-                     pack_bf16x2(d[k].x, d[k].y), pack_bf16x2(d[k].z, d[k].w));
-    }
-}
-
 template <int NST>
 __global__ void __launch_bounds__(256, 1)
     chunk_scan_tc_kernel(const __grid_constant__ FwdParams p, const __grid_constant__ CUtensorMap tm_c,
                          const __grid_constant__ CUtensorMap tm_b,
-                         const __grid_constant__ CUtensorMap tm_x, int hb_size) {
+                         const __grid_constant__ CUtensorMap tm_x,
+                         const __grid_constant__ CUtensorMap tm_h, int hb_size) {
     using T = ScanTile<NST>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -170,8 +150,8 @@ __global__ void __launch_bounds__(256, 1)
     float* dtv = reinterpret_cast<float*>(smem + T::DT_OFF);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + T::BAR_OFF);
     // barriers: 0 = C/B landed, 1 = CB done, 2/3 = x buffer 0/1 landed, 4 = tile-0 MMAs,
-    // 5 = tile-1 MMAs
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 6);
+    // 5 = tile-1 MMAs, 6 = H_in landed
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 7);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t H = p.nheads, L = p.seqlen, Q = p.chunk, nc = p.nchunks, G = p.ngroups;
@@ -189,11 +169,12 @@ __global__ void __launch_bounds__(256, 1)
 
     if (warp == 0) tmem_alloc(smem_u32(tmem_slot), 512);
     if (tid == 0) {
-        for (int i = 0; i < 6; ++i) mbar_init(bar(i), 1);
+        for (int i = 0; i < 7; ++i) mbar_init(bar(i), 1);
         fence_mbar_init();
         tma_prefetch_map(&tm_c);
         tma_prefetch_map(&tm_b);
         tma_prefetch_map(&tm_x);
+        tma_prefetch_map(&tm_h);
     }
     __syncthreads();
     if (tid == 0) {
@@ -207,11 +188,14 @@ __global__ void __launch_bounds__(256, 1)
             mbar_expect_tx(bar(2 + i), box);
             tma_load_4d(sX + i * T::X_BYTES, &tm_x, bar(2 + i), 0, (int)(hfirst + i), (int)t0, (int)b);
         }
+        mbar_expect_tx(bar(6), T::H_BYTES);
+        for (int kb = 0; kb < NST / 64; ++kb)
+            tma_load_4d(sH + kb * (PD * 128), &tm_h, bar(6), kb * 64, 0, (int)hfirst,
+                        (int)(b * nc + c));
     }
-    // first head's state and decays
+    // first head's decays
     {
         const int64_t vbase = ((b * H + hfirst) * nc + c) * Q;
-        load_hin<NST>(sH, p.states + ((b * nc + c) * H + hfirst) * PD * NST, tid);
         for (int i = tid; i < QMAX; i += 256) {
             cum[i] = (i < Q) ? p.cumA[vbase + i] : 0.0f;
             dtv[i] = (i < Q) ? p.dt[vbase + i] : 0.0f;
@@ -249,7 +233,9 @@ __global__ void __launch_bounds__(256, 1)
         const int xb = i & 1;
         const uint32_t xbase = sX + xb * T::X_BYTES;
         // every thread observes the x tile's arrival (the epilogue reads it too)
-        ok = !__syncthreads_or(!mbar_wait(bar(2 + xb), (i >> 1) & 1));
+        // and the state's
+        ok = !__syncthreads_or(!mbar_wait(bar(2 + xb), (i >> 1) & 1) ||
+                               !mbar_wait(bar(6), i & 1));
         if (!ok) break;
         for (int t = 0; t < ntiles; ++t) {
             // CUDA cores: the decay mask of tile t
@@ -285,23 +271,30 @@ __global__ void __launch_bounds__(256, 1)
             __syncthreads();
         }
         if (!ok) break;
-        // the next head's state and decays; its x is already on the way
+        // the next head's decays; its x is already on the way
         if (i + 1 < hb_size) {
             const int64_t vbase = ((b * H + h + 1) * nc + c) * Q;
-            load_hin<NST>(sH, p.states + ((b * nc + c) * H + h + 1) * PD * NST, tid);
             for (int k = tid; k < QMAX; k += 256) {
                 cum[k] = (k < Q) ? p.cumA[vbase + k] : 0.0f;
                 dtv[k] = (k < Q) ? p.dt[vbase + k] : 0.0f;
             }
-            fence_smem_async();
         }
         fence_before_sync();
         __syncthreads();
         fence_after_sync();
-        // x buffer xb is free again: fetch head i + 2 into it
-        if (tid == 0 && i + 2 < hb_size) {
-            mbar_expect_tx(bar(2 + xb), static_cast<uint32_t>(Q) * 128);
-            tma_load_4d(xbase, &tm_x, bar(2 + xb), 0, (int)(h + 2), (int)t0, (int)b);
+        if (tid == 0) {
+            // every MMA of this head is done: its H_in buffer takes the next head's
+            // state, its x buffer head i + 2's x
+            if (i + 1 < hb_size) {
+                mbar_expect_tx(bar(6), T::H_BYTES);
+                for (int kb = 0; kb < NST / 64; ++kb)
+                    tma_load_4d(sH + kb * (PD * 128), &tm_h, bar(6), kb * 64, 0, (int)(h + 1),
+                                (int)(b * nc + c));
+            }
+            if (i + 2 < hb_size) {
+                mbar_expect_tx(bar(2 + xb), static_cast<uint32_t>(Q) * 128);
+                tma_load_4d(xbase, &tm_x, bar(2 + xb), 0, (int)(h + 2), (int)t0, (int)b);
+            }
         }
     }
     if (!ok && tid == 0 && p.status) atomicExch(p.status, static_cast<int>(SSD_ERR_TIMEOUT));
@@ -327,11 +320,12 @@ int heads_per_cta(const FwdParams& p) {
 template <int NST>
 cudaError_t launch_n(const FwdParams& p, cudaStream_t s) {
     using T = ScanTile<NST>;
-    CUtensorMap tc_, tb_, tx_;
+    CUtensorMap tc_, tb_, tx_, th_;
     const uint32_t rows = static_cast<uint32_t>(p.chunk);
-    if (!make_tmap_bf16_4d(&tc_, p.C, NST, p.ngroups, p.seqlen, p.batch, rows) ||
-        !make_tmap_bf16_4d(&tb_, p.B, NST, p.ngroups, p.seqlen, p.batch, rows) ||
-        !make_tmap_bf16_4d(&tx_, p.x, PD, p.nheads, p.seqlen, p.batch, rows))
+    if (!make_tmap_bf16_4d(&tc_, p.C, NST, p.ngroups, p.seqlen, p.batch, 1, rows) ||
+        !make_tmap_bf16_4d(&tb_, p.B, NST, p.ngroups, p.seqlen, p.batch, 1, rows) ||
+        !make_tmap_bf16_4d(&tx_, p.x, PD, p.nheads, p.seqlen, p.batch, 1, rows) ||
+        !make_tmap_bf16_4d(&th_, p.states, NST, PD, p.nheads, p.batch * p.nchunks, PD, 1))
         return cudaErrorInvalidValue;
     auto kern = chunk_scan_tc_kernel<NST>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, T::SMEM);
@@ -339,7 +333,7 @@ cudaError_t launch_n(const FwdParams& p, cudaStream_t s) {
     const int hb = heads_per_cta(p);
     dim3 grid(static_cast<unsigned>(p.nchunks * p.ngroups * (p.heads_per_group / hb)),
               static_cast<unsigned>(p.batch));
-    kern<<<grid, 256, T::SMEM, s>>>(p, tc_, tb_, tx_, hb);
+    kern<<<grid, 256, T::SMEM, s>>>(p, tc_, tb_, tx_, th_, hb);
     return cudaGetLastError();
 }
 

@@ -1,7 +1,8 @@
 // chunk_state_ffma.cu -- step 2 of the chunked SSD forward on CUDA cores
 // (fp32 FFMA): every chunk's local state, as if the chunk started from zero,
 //   S_c[p,n] = sum_{l in c} exp(cumA[last] - cumA[l]) dt[l] x[l,p] B[l,n]
-// (the "diagonal block: local state" of "MAMBA-2 Implementation Gaps", Gap 1).
+// (the "diagonal block: local state" of "MAMBA-2 Implementation Gaps", Gap 1),
+// accumulated in fp32 and stored in the input dtype.
 //
 // This is the exact-fp32 path (fp32 inputs need 1e-4 agreement, beyond what
 // TF32 tensor cores give) and the fallback for shapes outside the tensor-core
@@ -72,13 +73,14 @@ __global__ void __launch_bounds__(256) chunk_state_ffma_kernel(FwdParams p) {
         }
         __syncthreads();
     }
-    float* out = p.states + ((b * nc + c) * H + h) * P * N;
+    T* out = static_cast<T*>(p.states) + ((b * nc + c) * H + h) * P * N;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const int64_t pi = p0 + ty * 4 + i, nj = n0 + tx * 4;
-        if (pi < P && nj < N)
-            *reinterpret_cast<float4*>(out + pi * N + nj) =
-                make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+        if (pi < P && nj < N) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) out[pi * N + nj + j] = from_f32<T>(acc[i][j]);
+        }
     }
 }
 

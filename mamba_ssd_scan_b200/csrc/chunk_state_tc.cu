@@ -12,8 +12,8 @@
 // 256 threads load (16-byte vector loads, the decay weight folded into x while
 // staging) while the tensor core consumes the other stage; one thread issues
 // the MMAs and commits each stage to its mbarrier.  The epilogue moves the
-// fp32 accumulator from TMEM to the states buffer, one row of dstate per
-// thread.
+// fp32 accumulator from TMEM to the states buffer (bf16, the input dtype), one
+// row of dstate per thread.
 #include "internal.cuh"
 #include "tcgen05.cuh"
 
@@ -147,17 +147,21 @@ __global__ void __launch_bounds__(256, 1) chunk_state_tc_kernel(FwdParams p) {
         // warp w reads TMEM lanes 32*(w%4).. (rows m), warpgroup w/4 half the columns
         const int m = 32 * (warp & 3) + lane;
         const int64_t hh = m / PD, pp = m % PD;
-        float* out = p.states + (((b * nc + c) * H + h0 + hh) * PD + pp) * NST;
+        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.states) +
+                             (((b * nc + c) * H + h0 + hh) * PD + pp) * NST;
         constexpr int HALF = NST / 2;
         const int cbeg = (warp >> 2) * HALF;
 #pragma unroll
         for (int col = 0; col < HALF; col += 32) {
             float v[32];
             tmem_ld32(tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + cbeg + col, v);
-            float4* o = reinterpret_cast<float4*>(out + cbeg + col);
+            uint4* o = reinterpret_cast<uint4*>(out + cbeg + col);
 #pragma unroll
-            for (int q = 0; q < 8; ++q)
-                o[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+            for (int q = 0; q < 4; ++q)
+                o[q] = make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]),
+                                  pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                                  pack_bf16x2(v[8 * q + 4], v[8 * q + 5]),
+                                  pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
         }
     } else if (tid == 0 && p.status) {
         atomicExch(p.status, static_cast<int>(SSD_ERR_TIMEOUT));

@@ -28,7 +28,7 @@ struct FwdParams {
     // intermediates (workspace)
     float* dt;      // [b, H, nc, Q]
     float* cumA;    // [b, H, nc, Q]
-    float* states;  // [b, nc, H, P, N] fp32
+    void* states;   // [b, nc, H, P, N] in the input dtype (local states, then states entering each chunk)
     int* status;    // device status word (SSD_ERR_TIMEOUT on a timed-out wait); may be null
 };
 
@@ -62,7 +62,7 @@ __device__ __forceinline__ float softplus_f32(float u) {
 // Launchers (one per kernel family).  Each returns cudaGetLastError().
 template <typename T> cudaError_t launch_chunk_cumsum(const FwdParams& p, cudaStream_t s);
 template <typename T> cudaError_t launch_chunk_state_ffma(const FwdParams& p, cudaStream_t s);
-cudaError_t launch_state_passing(const FwdParams& p, cudaStream_t s);
+template <typename T> cudaError_t launch_state_passing(const FwdParams& p, cudaStream_t s);
 template <typename T> cudaError_t launch_chunk_scan_ffma(const FwdParams& p, cudaStream_t s);
 template <typename T> cudaError_t launch_state_update(const DecodeParams& p, cudaStream_t s);
 

@@ -6,11 +6,12 @@
 //   H_{-1} = init (or 0);   H_c = exp(cumA_c[last]) H_{c-1} + S_c
 //
 // Sequential over chunks, parallel over batch x heads x headdim x dstate: each
-// thread carries 4 consecutive state elements (one 16-byte vector) in
-// registers.  In place over `states`: slot c receives H_{c-1}, the state that
-// enters chunk c; the final state H_{nc-1} goes to final_state.  The loads of
-// the next chunks' S do not depend on the carry, so they are issued ahead of
-// the multiply-adds (UNROLL chunks at a time) to keep enough bytes in flight.
+// thread carries one 16-byte vector of state elements (4 fp32 or 8 bf16) in
+// fp32 registers.  In place over `states` (stored in the input dtype): slot c
+// receives H_{c-1}, the state that enters chunk c; the final state H_{nc-1}
+// goes to final_state in fp32.  The loads of the next chunks' S do not depend
+// on the carry, so UNROLL chunks are loaded before their multiply-adds to keep
+// enough bytes in flight.
 #include "internal.cuh"
 
 namespace ssd {
@@ -18,55 +19,103 @@ namespace {
 
 constexpr int UNROLL = 4;
 
+template <typename T> struct Pack;
+template <> struct Pack<float> {
+    static constexpr int E = 4;
+    static __device__ __forceinline__ void unpack(uint4 v, float (&f)[4]) {
+        f[0] = __uint_as_float(v.x); f[1] = __uint_as_float(v.y);
+        f[2] = __uint_as_float(v.z); f[3] = __uint_as_float(v.w);
+    }
+    static __device__ __forceinline__ uint4 pack(const float (&f)[4]) {
+        return make_uint4(__float_as_uint(f[0]), __float_as_uint(f[1]), __float_as_uint(f[2]),
+                          __float_as_uint(f[3]));
+    }
+};
+template <> struct Pack<__nv_bfloat16> {
+    static constexpr int E = 8;
+    static __device__ __forceinline__ void unpack(uint4 v, float (&f)[8]) {
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 t = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
+            f[2 * i] = t.x;
+            f[2 * i + 1] = t.y;
+        }
+    }
+    static __device__ __forceinline__ uint4 pack(const float (&f)[8]) {
+        uint32_t w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const __nv_bfloat162 t = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+            w[i] = *reinterpret_cast<const uint32_t*>(&t);
+        }
+        return make_uint4(w[0], w[1], w[2], w[3]);
+    }
+};
+
+template <typename T>
 __global__ void __launch_bounds__(256) state_passing_kernel(FwdParams p) {
+    constexpr int E = Pack<T>::E;
     const int64_t H = p.nheads, nc = p.nchunks, Q = p.chunk;
-    const int64_t vecs_per_head = p.headdim * p.dstate / 4;
+    const int64_t vecs_per_head = p.headdim * p.dstate / E;
     const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (e >= p.batch * H * vecs_per_head) return;
     const int64_t bh = e / vecs_per_head, off = e % vecs_per_head;
     const int64_t b = bh / H, h = bh % H;
-    float4 carry = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (p.init_state) carry = reinterpret_cast<const float4*>(p.init_state)[e];
-    float4* st = reinterpret_cast<float4*>(p.states);
+    float carry[E];
+    if (p.init_state) {
+        const float4* ip = reinterpret_cast<const float4*>(p.init_state + e * E);
+#pragma unroll
+        for (int k = 0; k < E / 4; ++k) {
+            const float4 v = ip[k];
+            carry[4 * k] = v.x; carry[4 * k + 1] = v.y; carry[4 * k + 2] = v.z; carry[4 * k + 3] = v.w;
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < E; ++k) carry[k] = 0.0f;
+    }
+    uint4* base = reinterpret_cast<uint4*>(p.states) + (b * nc * H + h) * vecs_per_head + off;
+    const int64_t cstride = H * vecs_per_head;  // vectors between consecutive chunks
     const float* cs = p.cumA + (b * H + h) * nc * Q + (Q - 1);
-    const int64_t cstride = H * vecs_per_head;  // float4s between consecutive chunks
-    float4* base = st + (b * nc * H + h) * vecs_per_head + off;
-    int64_t c = 0;
-    for (; c + UNROLL <= nc; c += UNROLL) {
-        float4 s[UNROLL];
+    for (int64_t c = 0; c < nc; c += UNROLL) {
+        uint4 s[UNROLL];
         float a[UNROLL];
 #pragma unroll
         for (int u = 0; u < UNROLL; ++u) {
-            s[u] = base[(c + u) * cstride];
-            a[u] = expf(cs[(c + u) * Q]);
+            if (c + u < nc) {
+                s[u] = base[(c + u) * cstride];
+                a[u] = expf(cs[(c + u) * Q]);
+            }
         }
 #pragma unroll
         for (int u = 0; u < UNROLL; ++u) {
-            base[(c + u) * cstride] = carry;
-            carry.x = fmaf(a[u], carry.x, s[u].x);
-            carry.y = fmaf(a[u], carry.y, s[u].y);
-            carry.z = fmaf(a[u], carry.z, s[u].z);
-            carry.w = fmaf(a[u], carry.w, s[u].w);
+            if (c + u < nc) {
+                float sv[E];
+                Pack<T>::unpack(s[u], sv);
+                base[(c + u) * cstride] = Pack<T>::pack(carry);
+#pragma unroll
+                for (int k = 0; k < E; ++k) carry[k] = fmaf(a[u], carry[k], sv[k]);
+            }
         }
     }
-    for (; c < nc; ++c) {
-        const float4 s = base[c * cstride];
-        const float a = expf(cs[c * Q]);
-        base[c * cstride] = carry;
-        carry.x = fmaf(a, carry.x, s.x);
-        carry.y = fmaf(a, carry.y, s.y);
-        carry.z = fmaf(a, carry.z, s.z);
-        carry.w = fmaf(a, carry.w, s.w);
+    if (p.final_state) {
+        float4* fp = reinterpret_cast<float4*>(p.final_state + e * E);
+#pragma unroll
+        for (int k = 0; k < E / 4; ++k)
+            fp[k] = make_float4(carry[4 * k], carry[4 * k + 1], carry[4 * k + 2], carry[4 * k + 3]);
     }
-    if (p.final_state) reinterpret_cast<float4*>(p.final_state)[e] = carry;
 }
 
 }  // namespace
 
+template <typename T>
 cudaError_t launch_state_passing(const FwdParams& p, cudaStream_t s) {
-    const int64_t n = p.batch * p.nheads * p.headdim * p.dstate / 4;
-    state_passing_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(p);
+    const int64_t n = p.batch * p.nheads * p.headdim * p.dstate / Pack<T>::E;
+    state_passing_kernel<T><<<(unsigned)((n + 255) / 256), 256, 0, s>>>(p);
     return cudaGetLastError();
 }
+
+template cudaError_t launch_state_passing<float>(const FwdParams&, cudaStream_t);
+template cudaError_t launch_state_passing<__nv_bfloat16>(const FwdParams&, cudaStream_t);
 
 }  // namespace ssd

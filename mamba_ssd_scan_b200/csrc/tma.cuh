@@ -12,12 +12,12 @@
 namespace ssd {
 
 // 4-D bf16 tensor [d3][d2][d1][d0] (d0 innermost, dense), a box of
-// {64, 1, rows, 1} elements with the 128-byte swizzle: it lands in shared
-// memory as `rows` 128-byte rows in the SW128 layout.  Elements outside the
-// tensor read as zero.  Returns false if the encoder is unavailable or
+// {64, box1, box2, 1} elements with the 128-byte swizzle: it lands in shared
+// memory as box1 * box2 128-byte rows in the SW128 layout.  Elements outside
+// the tensor read as zero.  Returns false if the encoder is unavailable or
 // rejects the arguments.
 bool make_tmap_bf16_4d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1,
-                       uint64_t d2, uint64_t d3, uint32_t rows);
+                       uint64_t d2, uint64_t d3, uint32_t box1, uint32_t box2);
 
 namespace tc {
 

@@ -27,12 +27,12 @@ EncodeTiledFn encoder() {
 }  // namespace
 
 bool make_tmap_bf16_4d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1,
-                       uint64_t d2, uint64_t d3, uint32_t rows) {
+                       uint64_t d2, uint64_t d3, uint32_t box1, uint32_t box2) {
     EncodeTiledFn fn = encoder();
-    if (!fn || rows == 0 || rows > 256 || d0 < 64) return false;
+    if (!fn || box1 == 0 || box1 > 256 || box2 == 0 || box2 > 256 || d0 < 64) return false;
     const cuuint64_t dims[4] = {d0, d1, d2, d3};
     const cuuint64_t strides[3] = {d0 * 2, d0 * d1 * 2, d0 * d1 * d2 * 2};
-    const cuuint32_t box[4] = {64, 1, rows, 1};
+    const cuuint32_t box[4] = {64, box1, box2, 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
               box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,

@@ -69,8 +69,8 @@ def _args(**kw):
 
 def test_workspace_size_is_host_only(lib):
     a = _args()
-    # status word (256 B) + dt + cumA: 1*4*2*256 fp32 each + states 1*2*4*64*64 fp32
-    assert lib.ssd_fwd_workspace_size(ctypes.byref(a)) == 256 + 8192 + 8192 + 131072
+    # status word (256 B) + dt + cumA: 1*4*2*256 fp32 each + states 1*2*4*64*64 bf16
+    assert lib.ssd_fwd_workspace_size(ctypes.byref(a)) == 256 + 8192 + 8192 + 65536
     assert lib.ssd_fwd_workspace_size(None) == 0
     assert lib.ssd_fwd_workspace_size(ctypes.byref(_args(nheads=3, ngroups=2))) == 0
 
