@@ -416,8 +416,10 @@ def other_workloads(ssd, synthetic, dev, flush, peaks, rank, world, barrier, max
             tot += a.elapsed_time(b_)
         ms = max_over_ranks(tot / steps)
         nbytes = algorithmic_cost(cfg, 2)["path"][0]
+        kms = split_kernel_ms(ssd, cfg, d, y, fin, dev, flush, steps)
         out[name] = {"tokens_per_s": world * cfg.tokens / (ms * 1e-3), "ms": ms,
-                     "hbm_frac_of_path_bytes": nbytes / (ms * 1e-3) / (peaks["hbm_gbs"] * 1e9)}
+                     "hbm_frac_of_path_bytes": nbytes / (ms * 1e-3) / (peaks["hbm_gbs"] * 1e9),
+                     "kernel_ms": kms}
         del d, y, fin, ws
         torch.cuda.empty_cache()
 
@@ -464,6 +466,42 @@ def other_workloads(ssd, synthetic, dev, flush, peaks, rank, world, barrier, max
                      "bytes_per_step": step_bytes}
     del g
     return out
+
+
+def split_kernel_ms(ssd, cfg, d, y, fin, dev, flush, steps):
+    """Mean duration of each of the four steps (CUDA events between the step
+    entry points, which launch the same kernels ssd_fwd does)."""
+    import torch
+    stream = torch.cuda.current_stream()
+    nc = -(-cfg.seqlen // cfg.chunk)
+    dt_sp = torch.empty((cfg.batch, cfg.nheads, nc, cfg.chunk), device=dev)
+    cumA = torch.empty_like(dt_sp)
+    states = torch.empty((cfg.batch, nc, cfg.nheads, cfg.headdim, cfg.dstate), device=dev,
+                         dtype=cfg.dtype)
+    names = ["chunk_cumsum", "chunk_state", "state_passing", "chunk_scan"]
+    tot = dict.fromkeys(names, 0.0)
+    for it in range(steps + 2):
+        flush()
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+        ev[0].record(stream)
+        ssd.ssd_chunk_cumsum(d["x"], d["dt"], d["A"], d["B"], d["C"], d["dt_bias"], cfg.chunk,
+                             dt_out=dt_sp, cumA_out=cumA)
+        ev[1].record(stream)
+        ssd.ssd_chunk_state(d["x"], d["dt"], d["A"], d["B"], d["C"], dt_sp, cumA, cfg.chunk,
+                            states=states)
+        ev[2].record(stream)
+        ssd.ssd_state_passing(d["x"], d["dt"], d["A"], d["B"], d["C"], cumA, states, cfg.chunk,
+                              init_state=d["init_state"], final_state=fin)
+        ev[3].record(stream)
+        ssd.ssd_chunk_scan(d["x"], d["dt"], d["A"], d["B"], d["C"], dt_sp, cumA, states,
+                           d["D"], cfg.chunk, y=y)
+        ev[4].record(stream)
+        torch.cuda.synchronize()
+        if it >= 2:
+            for i, n in enumerate(names):
+                tot[n] += ev[i].elapsed_time(ev[i + 1])
+    del dt_sp, cumA, states
+    return {n: tot[n] / steps for n in names}
 
 
 def cpu_baseline(cfg, inp, budget_s=12.0):

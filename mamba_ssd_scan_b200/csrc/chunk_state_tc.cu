@@ -6,71 +6,94 @@
 // TMEM):
 //   D[m, n] = sum_l A[m, l] B[l, n],  m = (head, p) over 128/P heads of one
 //   group (M = 128), n = 0..dstate-1 (N = dstate), K = the chunk's tokens.
-// Both operands are MN-major: A is the weighted x rows as they sit in memory
-// (for a token, the 128/P heads' P values are contiguous), B is the group's B
-// rows.  Tokens stream through a 2-stage shared-memory ring of 64 tokens; all
-// 256 threads load (16-byte vector loads, the decay weight folded into x while
-// staging) while the tensor core consumes the other stage; one thread issues
-// the MMAs and commits each stage to its mbarrier.  The epilogue moves the
-// fp32 accumulator from TMEM to the states buffer (bf16, the input dtype), one
-// row of dstate per thread.
+// Both operands are MN-major and arrive by TMA exactly as they sit in memory:
+// A is x viewed as 64-element units (for a token, the 128/P heads' P values
+// are two contiguous units), B the group's B rows.  The chunk streams in as
+// four 64-token quarters, each on its own mbarrier; the CUDA cores fold the
+// decay weight into a quarter of x in place (bf16 -> fp32 -> bf16) while the
+// tensor core multiplies the previous quarter.  The epilogue moves the fp32
+// accumulator from TMEM to the states buffer in the input dtype (bf16), one row
+// of dstate per thread.
 #include "internal.cuh"
 #include "tcgen05.cuh"
+#include "tma.cuh"
 
 namespace ssd {
 namespace {
 
 using namespace tc;
 
-constexpr int KT = 64;      // tokens per stage
-constexpr int NSTAGE = 2;
+constexpr int KT = 64;      // tokens per quarter
+constexpr int NQ = 4;       // quarters (chunk <= 256)
 constexpr int QMAX = 256;
 
 template <int NST, int PD>
 struct StateTile {
-    static constexpr int HPC = 128 / PD;               // heads per CTA
-    static constexpr int A_BYTES = 2 * KT * 128;       // 2 blocks of 64 rows (m) x 64 tokens
-    static constexpr int B_BYTES = (NST / 64) * KT * 128;
-    static constexpr int STAGE = A_BYTES + B_BYTES;
-    static constexpr int TMEM_COLS = NST;              // 64, 128 or 256 (powers of two)
-    static constexpr int W_OFF = NSTAGE * STAGE;       // decay weights [HPC][QMAX] fp32
+    static constexpr int HPC = 128 / PD;                 // heads per CTA
+    static constexpr int A_BLK = QMAX * 128;             // one 64-wide m block, all tokens
+    static constexpr int A_BYTES = 2 * A_BLK;
+    static constexpr int B_BLK = QMAX * 128;             // one 64-wide n block, all tokens
+    static constexpr int B_BYTES = (NST / 64) * B_BLK;
+    static constexpr int TMEM_COLS = NST;                // 64, 128 or 256
+    static constexpr int W_OFF = A_BYTES + B_BYTES;      // decay weights [HPC][QMAX] fp32
     static constexpr int BAR_OFF = W_OFF + HPC * QMAX * 4;
-    static constexpr int SMEM = BAR_OFF + 64 + 1024;   // + alignment slack
+    static constexpr int SMEM = BAR_OFF + 128 + 1024;    // + alignment slack
+    static_assert(SMEM <= 232448, "shared memory budget");
 };
 
 __device__ __forceinline__ uint4 scale_bf16x8(uint4 v, float w) {
     uint32_t in[4] = {v.x, v.y, v.z, v.w}, out[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162*>(&in[i]);
-        const float2 f = __bfloat1622float2(h);
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&in[i]));
         out[i] = pack_bf16x2(f.x * w, f.y * w);
     }
     return make_uint4(out[0], out[1], out[2], out[3]);
 }
 
 template <int NST, int PD>
-__global__ void __launch_bounds__(256, 1) chunk_state_tc_kernel(FwdParams p) {
+__global__ void __launch_bounds__(256, 1)
+    chunk_state_tc_kernel(const __grid_constant__ FwdParams p,
+                          const __grid_constant__ CUtensorMap tm_x,
+                          const __grid_constant__ CUtensorMap tm_b) {
     using T = StateTile<NST, PD>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
     float* wtab = reinterpret_cast<float*>(smem + T::W_OFF);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + T::BAR_OFF);
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NSTAGE);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + T::BAR_OFF);  // NQ loads + 1 MMA
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NQ + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int64_t H = p.nheads, L = p.seqlen, Q = p.chunk, nc = p.nchunks, G = p.ngroups;
+    const int64_t H = p.nheads, L = p.seqlen, Q = p.chunk, nc = p.nchunks;
     const int64_t hblocks = H / T::HPC;
     const int64_t c = blockIdx.x / hblocks, h0 = (blockIdx.x % hblocks) * T::HPC;
     const int64_t b = blockIdx.y, g = h0 / p.heads_per_group;
     const int64_t t0 = c * Q;
     const int Lc = static_cast<int>((L - t0 < Q) ? (L - t0) : Q);
+    const int nq = (Lc + KT - 1) / KT;
+    const uint32_t sA = smem_u32(smem), sB = sA + T::A_BYTES;
+    auto bar = [&](int i) { return smem_u32(&bars[i]); };
 
     if (warp == 0) tmem_alloc(smem_u32(tmem_slot), T::TMEM_COLS);
     if (tid == 0) {
-        for (int s = 0; s < NSTAGE; ++s) mbar_init(smem_u32(&bars[s]), 1);
+        for (int i = 0; i <= NQ; ++i) mbar_init(bar(i), 1);
         fence_mbar_init();
+        tma_prefetch_map(&tm_x);
+        tma_prefetch_map(&tm_b);
+    }
+    __syncthreads();
+    if (tid == 0) {
+        const int unit0 = static_cast<int>(h0 * PD / 64);  // x in 64-element units
+        for (int q = 0; q < nq; ++q) {
+            mbar_expect_tx(bar(q), (2 + NST / 64) * KT * 128);
+            for (int blk = 0; blk < 2; ++blk)
+                tma_load_4d(sA + blk * T::A_BLK + q * KT * 128, &tm_x, bar(q), 0, unit0 + blk,
+                            static_cast<int>(t0 + q * KT), static_cast<int>(b));
+            for (int nb = 0; nb < NST / 64; ++nb)
+                tma_load_4d(sB + nb * T::B_BLK + q * KT * 128, &tm_b, bar(q), nb * 64,
+                            static_cast<int>(g), static_cast<int>(t0 + q * KT), static_cast<int>(b));
+        }
     }
     for (int i = tid; i < T::HPC * QMAX; i += 256) {
         const int hh = i / QMAX, l = i % QMAX;
@@ -86,43 +109,22 @@ __global__ void __launch_bounds__(256, 1) chunk_state_tc_kernel(FwdParams p) {
     fence_after_sync();
     const uint32_t tmem = *tmem_slot;
 
-    const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(p.x);
-    const __nv_bfloat16* Bm = static_cast<const __nv_bfloat16*>(p.B);
-    const int nkt = (Lc + KT - 1) / KT;
     constexpr uint32_t idesc = idesc_bf16(128, NST, true, true);
     bool ok = true;
-    for (int kt = 0; kt < nkt; ++kt) {
-        const int s = kt % NSTAGE;
-        uint8_t* As = smem + s * T::STAGE;
-        uint8_t* Bs = As + T::A_BYTES;
-        if (kt >= NSTAGE) {  // wait until the MMAs that read this stage are done
-            const bool w = mbar_wait(smem_u32(&bars[s]), ((kt / NSTAGE) - 1) & 1);
-            if (__syncthreads_or(!w)) {
-                ok = false;
-                break;
-            }
-        }
-        // A: 64 token rows x 16 chunks (two 64-wide m blocks)
-#pragma unroll 4
-        for (int i = tid; i < KT * 16; i += 256) {
-            const int r = i >> 4, cc = i & 15, blk = cc >> 3, ch = cc & 7;
-            const int l = kt * KT + r;
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (l < Lc) {
-                const int m = blk * 64 + ch * 8;
-                v = ldg16(x + ((b * L + t0 + l) * H + h0) * PD + m);
-                v = scale_bf16x8(v, wtab[(m / PD) * QMAX + l]);
-            }
-            st_shared_v4(smem_u32(As) + blk * (KT * 128) + sw128(r, ch), v.x, v.y, v.z, v.w);
-        }
-        // B: 64 token rows x NST/8 chunks
-#pragma unroll 4
-        for (int i = tid; i < KT * (NST / 8); i += 256) {
-            const int r = i / (NST / 8), cc = i % (NST / 8), blk = cc >> 3, ch = cc & 7;
-            const int l = kt * KT + r;
-            uint4 v = make_uint4(0u, 0u, 0u, 0u);
-            if (l < Lc) v = ldg16(Bm + ((b * L + t0 + l) * G + g) * NST + cc * 8);
-            st_shared_v4(smem_u32(Bs) + blk * (KT * 128) + sw128(r, ch), v.x, v.y, v.z, v.w);
+    for (int q = 0; q < nq && ok; ++q) {
+        ok = !__syncthreads_or(!mbar_wait(bar(q), 0));
+        if (!ok) break;
+        // fold the decay weights into this quarter of x: 2 blocks x 64 rows x 8 chunks
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int i = tid + 256 * k;
+            const int blk = i >> 9, r = (i >> 3) & 63, ch = i & 7;
+            const int l = q * KT + r;
+            const uint32_t addr = sA + blk * T::A_BLK + sw128(l, ch);
+            const int hh = (blk * 64 + ch * 8) / PD;
+            const uint4 v = ld_shared_v4(addr);
+            const uint4 o = scale_bf16x8(v, wtab[hh * QMAX + l]);
+            st_shared_v4(addr, o.x, o.y, o.z, o.w);
         }
         fence_smem_async();
         __syncthreads();
@@ -130,18 +132,14 @@ __global__ void __launch_bounds__(256, 1) chunk_state_tc_kernel(FwdParams p) {
             fence_after_sync();
 #pragma unroll
             for (int k = 0; k < KT / 16; ++k) {
-                const uint64_t ad = desc_sw128(smem_u32(As) + k * 2048, KT * 128, 1024);
-                const uint64_t bd = desc_sw128(smem_u32(Bs) + k * 2048, KT * 128, 1024);
-                mma_bf16(tmem, ad, bd, idesc, (kt > 0 || k > 0) ? 1u : 0u);
+                const uint32_t off = (q * KT + k * 16) * 128;
+                mma_bf16(tmem, desc_sw128(sA + off, T::A_BLK, 1024),
+                         desc_sw128(sB + off, T::B_BLK, 1024), idesc, (q > 0 || k > 0) ? 1u : 0u);
             }
-            mma_commit(smem_u32(&bars[s]));
+            if (q == nq - 1) mma_commit(bar(NQ));
         }
     }
-    if (ok) {
-        const int last = nkt - 1;
-        const bool w = mbar_wait(smem_u32(&bars[last % NSTAGE]), (last / NSTAGE) & 1);
-        if (__syncthreads_or(!w)) ok = false;
-    }
+    if (ok) ok = !__syncthreads_or(!mbar_wait(bar(NQ), 0));
     fence_after_sync();
     if (ok) {
         // warp w reads TMEM lanes 32*(w%4).. (rows m), warpgroup w/4 half the columns
@@ -157,11 +155,11 @@ __global__ void __launch_bounds__(256, 1) chunk_state_tc_kernel(FwdParams p) {
             tmem_ld32(tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + cbeg + col, v);
             uint4* o = reinterpret_cast<uint4*>(out + cbeg + col);
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-                o[q] = make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]),
-                                  pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
-                                  pack_bf16x2(v[8 * q + 4], v[8 * q + 5]),
-                                  pack_bf16x2(v[8 * q + 6], v[8 * q + 7]));
+            for (int k = 0; k < 4; ++k)
+                o[k] = make_uint4(pack_bf16x2(v[8 * k], v[8 * k + 1]),
+                                  pack_bf16x2(v[8 * k + 2], v[8 * k + 3]),
+                                  pack_bf16x2(v[8 * k + 4], v[8 * k + 5]),
+                                  pack_bf16x2(v[8 * k + 6], v[8 * k + 7]));
         }
     } else if (tid == 0 && p.status) {
         atomicExch(p.status, static_cast<int>(SSD_ERR_TIMEOUT));
@@ -177,11 +175,15 @@ __global__ void __launch_bounds__(256, 1) chunk_state_tc_kernel(FwdParams p) {
 template <int NST, int PD>
 cudaError_t launch_nd(const FwdParams& p, cudaStream_t s) {
     using T = StateTile<NST, PD>;
+    CUtensorMap tx_, tb_;
+    if (!make_tmap_bf16_4d(&tx_, p.x, 64, p.nheads * PD / 64, p.seqlen, p.batch, 1, KT) ||
+        !make_tmap_bf16_4d(&tb_, p.B, NST, p.ngroups, p.seqlen, p.batch, 1, KT))
+        return cudaErrorInvalidValue;
     auto kern = chunk_state_tc_kernel<NST, PD>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, T::SMEM);
     if (e != cudaSuccess) return e;
     dim3 grid(static_cast<unsigned>(p.nchunks * (p.nheads / T::HPC)), static_cast<unsigned>(p.batch));
-    kern<<<grid, 256, T::SMEM, s>>>(p);
+    kern<<<grid, 256, T::SMEM, s>>>(p, tx_, tb_);
     return cudaGetLastError();
 }
 
