@@ -113,8 +113,7 @@ __device__ __forceinline__ void epilogue(int t, uint32_t tmem, uint32_t xbase, c
     const int pc = 32 * (warp >> 2);
     const uint32_t lane_addr = static_cast<uint32_t>(32 * (warp & 3)) << 16;
     float vi[32], vs[32];
-    tmem_ld32(tmem + lane_addr + IN_COL + pc, vi);
-    tmem_ld32(tmem + lane_addr + ST_COL + pc, vs);
+    tmem_ld32x2(tmem + lane_addr + IN_COL + pc, vi, tmem + lane_addr + ST_COL + pc, vs);
     if (l >= Lc) return;
     const float sc = __expf(cum[l]);
     const float Dh = p.D ? p.D[h] : 0.0f;
@@ -233,20 +232,27 @@ __global__ void __launch_bounds__(256, 1)
         const int xb = i & 1;
         const uint32_t xbase = sX + xb * T::X_BYTES;
         // every thread observes the x tile's arrival (the epilogue reads it too)
-        // and the state's
-        ok = !__syncthreads_or(!mbar_wait(bar(2 + xb), (i >> 1) & 1) ||
-                               !mbar_wait(bar(6), i & 1));
+        ok = !__syncthreads_or(!mbar_wait(bar(2 + xb), (i >> 1) & 1));
         if (!ok) break;
+        // the next head's decays, into registers now, into shared memory at the end
+        float cum_next = 0.0f, dt_next = 0.0f;
+        if (i + 1 < hb_size && tid < Q) {
+            const int64_t vbase = ((b * H + h + 1) * nc + c) * Q;
+            cum_next = p.cumA[vbase + tid];
+            dt_next = p.dt[vbase + tid];
+        }
         for (int t = 0; t < ntiles; ++t) {
             // CUDA cores: the decay mask of tile t
             build_mask(t, tmem, sM, cum, dtv, stab, warp, lane);
             fence_smem_async();
             fence_before_sync();
             __syncthreads();
-            // tensor core: state term and Mk x of tile t
+            // tensor core: state term and Mk x of tile t (the state has to have landed)
+            bool mine = true;
             if (tid == 0) {
                 fence_after_sync();
-                {
+                if (t == 0) mine = mbar_wait(bar(6), i & 1);
+                if (mine) {
                     for (int k = 0; k < NST / 16; ++k) {
                         const uint32_t ko = (k >> 2) * T::KB_BYTES + (k & 3) * 32;
                         const uint32_t kh = (k >> 2) * (PD * 128) + (k & 3) * 32;
@@ -263,7 +269,8 @@ __global__ void __launch_bounds__(256, 1)
                     mma_commit(bar(4 + t));
                 }
             }
-            ok = !__syncthreads_or(!mbar_wait(bar(4 + t), i & 1));
+            ok = !__syncthreads_or(!mine);
+            if (ok) ok = !__syncthreads_or(!mbar_wait(bar(4 + t), i & 1));
             fence_after_sync();
             if (!ok) break;
             epilogue(t, tmem, xbase, cum, p, b, t0, h, Lc, warp, lane);
@@ -271,13 +278,10 @@ __global__ void __launch_bounds__(256, 1)
             __syncthreads();
         }
         if (!ok) break;
-        // the next head's decays; its x is already on the way
+        // the next head's decays; its x and state are already on the way
         if (i + 1 < hb_size) {
-            const int64_t vbase = ((b * H + h + 1) * nc + c) * Q;
-            for (int k = tid; k < QMAX; k += 256) {
-                cum[k] = (k < Q) ? p.cumA[vbase + k] : 0.0f;
-                dtv[k] = (k < Q) ? p.dt[vbase + k] : 0.0f;
-            }
+            cum[tid] = cum_next;
+            dtv[tid] = dt_next;
         }
         fence_before_sync();
         __syncthreads();

@@ -8,12 +8,15 @@
 //   group (M = 128), n = 0..dstate-1 (N = dstate), K = the chunk's tokens.
 // Both operands are MN-major and arrive by TMA exactly as they sit in memory:
 // A is x viewed as 64-element units (for a token, the 128/P heads' P values
-// are two contiguous units), B the group's B rows.  The chunk streams in as
-// four 64-token quarters, each on its own mbarrier; the CUDA cores fold the
-// decay weight into a quarter of x in place (bf16 -> fp32 -> bf16) while the
-// tensor core multiplies the previous quarter.  The epilogue moves the fp32
-// accumulator from TMEM to the states buffer in the input dtype (bf16), one row
-// of dstate per thread.
+// are two contiguous units), B the group's B rows.  The chunk streams through
+// a two-slot ring of 64-token quarters (load and free mbarriers per slot); the
+// CUDA cores fold the decay weight into a quarter of x in place (bf16 -> fp32
+// -> bf16) while the tensor core multiplies the previous one, and the next
+// quarter's TMA is issued as soon as its slot's MMAs have completed.  With
+// 64 KB of shared memory (dstate 128) three CTAs share an SM, so one CTA's
+// loads overlap another's MMAs and epilogue.  The epilogue moves the fp32
+// accumulator from TMEM to the states buffer in the input dtype (bf16), one
+// row of dstate per thread.
 #include "internal.cuh"
 #include "tcgen05.cuh"
 #include "tma.cuh"
@@ -24,18 +27,19 @@ namespace {
 using namespace tc;
 
 constexpr int KT = 64;      // tokens per quarter
-constexpr int NQ = 4;       // quarters (chunk <= 256)
+constexpr int NSLOT = 2;    // ring slots
 constexpr int QMAX = 256;
 
 template <int NST, int PD>
 struct StateTile {
     static constexpr int HPC = 128 / PD;                 // heads per CTA
-    static constexpr int A_BLK = QMAX * 128;             // one 64-wide m block, all tokens
+    static constexpr int A_BLK = KT * 128;               // one 64-wide m block of a quarter
     static constexpr int A_BYTES = 2 * A_BLK;
-    static constexpr int B_BLK = QMAX * 128;             // one 64-wide n block, all tokens
+    static constexpr int B_BLK = KT * 128;               // one 64-wide n block of a quarter
     static constexpr int B_BYTES = (NST / 64) * B_BLK;
+    static constexpr int SLOT = A_BYTES + B_BYTES;
     static constexpr int TMEM_COLS = NST;                // 64, 128 or 256
-    static constexpr int W_OFF = A_BYTES + B_BYTES;      // decay weights [HPC][QMAX] fp32
+    static constexpr int W_OFF = NSLOT * SLOT;           // decay weights [HPC][QMAX] fp32
     static constexpr int BAR_OFF = W_OFF + HPC * QMAX * 4;
     static constexpr int SMEM = BAR_OFF + 128 + 1024;    // + alignment slack
     static_assert(SMEM <= 232448, "shared memory budget");
@@ -61,8 +65,8 @@ __global__ void __launch_bounds__(256, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
     float* wtab = reinterpret_cast<float*>(smem + T::W_OFF);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + T::BAR_OFF);  // NQ loads + 1 MMA
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NQ + 1);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + T::BAR_OFF);  // load[2], free[2]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * NSLOT);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t H = p.nheads, L = p.seqlen, Q = p.chunk, nc = p.nchunks;
@@ -72,29 +76,31 @@ __global__ void __launch_bounds__(256, 1)
     const int64_t t0 = c * Q;
     const int Lc = static_cast<int>((L - t0 < Q) ? (L - t0) : Q);
     const int nq = (Lc + KT - 1) / KT;
-    const uint32_t sA = smem_u32(smem), sB = sA + T::A_BYTES;
-    auto bar = [&](int i) { return smem_u32(&bars[i]); };
+    const uint32_t s0 = smem_u32(smem);
+    auto bar = [&](int i) { return smem_u32(&bars[i]); };  // 0,1 = loaded; 2,3 = free
+    const int unit0 = static_cast<int>(h0 * PD / 64);     // x in 64-element units
+    // quarter q -> slot q % 2: A blocks then B blocks
+    auto issue = [&](int q) {
+        const uint32_t sl = s0 + (q & 1) * T::SLOT;
+        mbar_expect_tx(bar(q & 1), T::SLOT);
+        for (int blk = 0; blk < 2; ++blk)
+            tma_load_4d(sl + blk * T::A_BLK, &tm_x, bar(q & 1), 0, unit0 + blk,
+                        static_cast<int>(t0 + q * KT), static_cast<int>(b));
+        for (int nb = 0; nb < NST / 64; ++nb)
+            tma_load_4d(sl + T::A_BYTES + nb * T::B_BLK, &tm_b, bar(q & 1), nb * 64,
+                        static_cast<int>(g), static_cast<int>(t0 + q * KT), static_cast<int>(b));
+    };
 
     if (warp == 0) tmem_alloc(smem_u32(tmem_slot), T::TMEM_COLS);
     if (tid == 0) {
-        for (int i = 0; i <= NQ; ++i) mbar_init(bar(i), 1);
+        for (int i = 0; i < 2 * NSLOT; ++i) mbar_init(bar(i), 1);
         fence_mbar_init();
         tma_prefetch_map(&tm_x);
         tma_prefetch_map(&tm_b);
     }
     __syncthreads();
-    if (tid == 0) {
-        const int unit0 = static_cast<int>(h0 * PD / 64);  // x in 64-element units
-        for (int q = 0; q < nq; ++q) {
-            mbar_expect_tx(bar(q), (2 + NST / 64) * KT * 128);
-            for (int blk = 0; blk < 2; ++blk)
-                tma_load_4d(sA + blk * T::A_BLK + q * KT * 128, &tm_x, bar(q), 0, unit0 + blk,
-                            static_cast<int>(t0 + q * KT), static_cast<int>(b));
-            for (int nb = 0; nb < NST / 64; ++nb)
-                tma_load_4d(sB + nb * T::B_BLK + q * KT * 128, &tm_b, bar(q), nb * 64,
-                            static_cast<int>(g), static_cast<int>(t0 + q * KT), static_cast<int>(b));
-        }
-    }
+    if (tid == 0)
+        for (int q = 0; q < nq && q < NSLOT; ++q) issue(q);
     for (int i = tid; i < T::HPC * QMAX; i += 256) {
         const int hh = i / QMAX, l = i % QMAX;
         float w = 0.0f;
@@ -110,20 +116,21 @@ __global__ void __launch_bounds__(256, 1)
     const uint32_t tmem = *tmem_slot;
 
     constexpr uint32_t idesc = idesc_bf16(128, NST, true, true);
-    bool ok = true;
+    bool ok = true, mine = true;  // mine: thread 0's refill waits
     for (int q = 0; q < nq && ok; ++q) {
-        ok = !__syncthreads_or(!mbar_wait(bar(q), 0));
+        const int sl = q & 1, use = q >> 1;
+        const uint32_t sA = s0 + sl * T::SLOT, sB = sA + T::A_BYTES;
+        ok = !__syncthreads_or(!(mine && mbar_wait(bar(sl), use & 1)));
         if (!ok) break;
         // fold the decay weights into this quarter of x: 2 blocks x 64 rows x 8 chunks
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             const int i = tid + 256 * k;
             const int blk = i >> 9, r = (i >> 3) & 63, ch = i & 7;
-            const int l = q * KT + r;
-            const uint32_t addr = sA + blk * T::A_BLK + sw128(l, ch);
+            const uint32_t addr = sA + blk * T::A_BLK + sw128(r, ch);
             const int hh = (blk * 64 + ch * 8) / PD;
             const uint4 v = ld_shared_v4(addr);
-            const uint4 o = scale_bf16x8(v, wtab[hh * QMAX + l]);
+            const uint4 o = scale_bf16x8(v, wtab[hh * QMAX + q * KT + r]);
             st_shared_v4(addr, o.x, o.y, o.z, o.w);
         }
         fence_smem_async();
@@ -131,15 +138,18 @@ __global__ void __launch_bounds__(256, 1)
         if (tid == 0) {
             fence_after_sync();
 #pragma unroll
-            for (int k = 0; k < KT / 16; ++k) {
-                const uint32_t off = (q * KT + k * 16) * 128;
-                mma_bf16(tmem, desc_sw128(sA + off, T::A_BLK, 1024),
-                         desc_sw128(sB + off, T::B_BLK, 1024), idesc, (q > 0 || k > 0) ? 1u : 0u);
+            for (int k = 0; k < KT / 16; ++k)
+                mma_bf16(tmem, desc_sw128(sA + k * 2048, T::A_BLK, 1024),
+                         desc_sw128(sB + k * 2048, T::B_BLK, 1024), idesc,
+                         (q > 0 || k > 0) ? 1u : 0u);
+            mma_commit(bar(2 + sl));
+            if (q + NSLOT < nq) {  // refill this slot once its MMAs are done
+                mine = mbar_wait(bar(2 + sl), use & 1);
+                if (mine) issue(q + NSLOT);
             }
-            if (q == nq - 1) mma_commit(bar(NQ));
         }
     }
-    if (ok) ok = !__syncthreads_or(!mbar_wait(bar(NQ), 0));
+    if (ok) ok = !__syncthreads_or(!mbar_wait(bar(2 + ((nq - 1) & 1)), ((nq - 1) >> 1) & 1));
     fence_after_sync();
     if (ok) {
         // warp w reads TMEM lanes 32*(w%4).. (rows m), warpgroup w/4 half the columns
