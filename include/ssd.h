@@ -186,6 +186,10 @@ ssd_status ssd_state_update(const ssd_state_update_args* args, void* stream);
 /* Static, human-readable name of a status code. */
 const char* ssd_status_string(ssd_status status);
 
+/* Name of the last CUDA error behind an SSD_ERR_CUDA returned to this host
+ * thread (static string; "no CUDA error" if none). */
+const char* ssd_last_cuda_error(void);
+
 /* Library version string (static). */
 const char* ssd_version(void);
 

@@ -52,7 +52,10 @@ class SsdStateUpdateArgs(ctypes.Structure):
 class SsdError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {ssd_status_string(status)}")
+        msg = f"{where}: {ssd_status_string(status)}"
+        if status == SSD_ERR_CUDA:
+            msg += f" ({load_library().ssd_last_cuda_error().decode()})"
+        super().__init__(msg)
 
 
 _lib = None
@@ -91,6 +94,8 @@ def load_library():
     lib.ssd_state_update.argtypes = [ctypes.POINTER(SsdStateUpdateArgs), _vp]
     lib.ssd_status_string.restype = ctypes.c_char_p
     lib.ssd_status_string.argtypes = [ctypes.c_int]
+    lib.ssd_last_cuda_error.restype = ctypes.c_char_p
+    lib.ssd_last_cuda_error.argtypes = []
     lib.ssd_version.restype = ctypes.c_char_p
     lib.ssd_version.argtypes = []
     _lib = lib

@@ -112,7 +112,14 @@ FwdParams make_params(const ssd_fwd_args* a) {
     return p;
 }
 
-ssd_status to_status(cudaError_t e) { return e == cudaSuccess ? SSD_OK : SSD_ERR_CUDA; }
+// the last CUDA error a call of this library saw, per host thread
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+
+ssd_status to_status(cudaError_t e) {
+    if (e == cudaSuccess) return SSD_OK;
+    g_last_cuda_error = e;
+    return SSD_ERR_CUDA;
+}
 
 cudaError_t run_cumsum(const FwdParams& p, int dtype, cudaStream_t s) {
     return dtype == SSD_BF16 ? ssd::launch_chunk_cumsum<__nv_bfloat16>(p, s)
@@ -297,6 +304,10 @@ const char* ssd_status_string(ssd_status s) {
         case SSD_ERR_TIMEOUT: return "SSD_ERR_TIMEOUT";
         default: return "SSD_ERR_UNKNOWN";
     }
+}
+
+const char* ssd_last_cuda_error(void) {
+    return g_last_cuda_error == cudaSuccess ? "no CUDA error" : cudaGetErrorString(g_last_cuda_error);
 }
 
 const char* ssd_version(void) { return "ssd_b200 0.1.0 (sm_100a)"; }

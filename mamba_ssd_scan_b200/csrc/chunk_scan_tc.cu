@@ -9,23 +9,35 @@
 // off-diagonal contribution ("MAMBA-2 Implementation Gaps", Gap 1) and the D
 // skip (Gap 4).
 //
-// One CTA serves a block of heads that share a group's B and C: TMA brings the
-// chunk's C and B rows once, tcgen05.mma computes CB = C B^T once into TMEM
-// (K = dstate), and then each head reuses it.  Per head and per 128-row output
-// tile t, the CUDA cores read CB back, apply the causal decay mask and write Mk
-// as a bf16 K-major operand to shared memory; the tensor core accumulates the
-// state term C_t H_in^T and Mk x into TMEM; the epilogue adds D x and stores y.
-// Each head's x tile arrives by TMA into one of two buffers while the previous
-// head computes; its state entering the chunk (bf16, as state passing left it)
-// arrives by TMA too.  Decays are never formed as exp(cumA_l) / exp(cumA_j): below
-// the 32x32 diagonal blocks the factor is split as exp(cumA_l - cumA_r) *
-// exp(cumA_r - cumA_j) with r the first row of the thread's 32-row block (both
-// factors <= 1, one table of the second per warp); only the diagonal blocks
-// take one exp per element.
+// One CTA serves a block of heads that share a group's B and C.  TMA brings
+// the chunk's C and B rows once and tcgen05.mma computes CB = C B^T for the two
+// 128-row output tiles once; the CB rows are then repacked in TMEM as fp16
+// pairs (192 columns instead of 384), each row scaled by a power of two that
+// keeps it inside fp16's range, so that both tiles' accumulators fit beside
+// them at ~2^-11 relative rounding.  The CTA is warp-specialised and its roles
+// hand work to each other through mbarriers:
 //
-// TMEM (512 columns): CB of tile 1 [0,256) and of tile 0 [256,384) stay for
-// every head; [384,448) and [448,512) hold the state and intra-chunk
-// accumulators of the tile in flight.
+//   warps 0-7  "mask": per head and tile, read CB back, apply the causal decay
+//              mask and write Mk as a bf16 K-major operand to shared memory
+//              (one buffer per tile, refilled as soon as its MMA is done); two
+//              warps share each 32-row block, taking alternate column groups;
+//   warps 8-11 "epilogue": per head and tile, read the state and intra-chunk
+//              accumulators, add D x and store y (bf16);
+//   warp 12    "control": one lane issues every TMA load (C, B once; x and
+//              H_in per head) and every MMA (CB once; per head and tile the
+//              state term C_t H_in^T and Mk x).
+//
+// so the tensor core, the mask arithmetic and the epilogue of different tiles
+// and heads run at the same time.  Decays are never formed as exp(cumA_l) /
+// exp(cumA_j): below the 32x32 diagonal blocks the factor is split as
+// exp(cumA_l - cumA_r) * exp(cumA_r - cumA_j), r the first row of the 32-row
+// block (both factors <= 1), and only the diagonal blocks take one exp per
+// element.  Every wait is bounded; a timed-out role raises a shared abort flag
+// that the others observe, and the CTA still frees its TMEM.
+//
+// TMEM columns: [0,64) tile 0's CB and [64,192) tile 1's CB as packed fp16
+// pairs (tile 1's fp32 CB sits in [128,384) until packed); [192,256)/[256,320)
+// tile 0's state/intra accumulators; [320,384)/[384,448) tile 1's.
 #include "internal.cuh"
 #include "tcgen05.cuh"
 #include "tma.cuh"
@@ -37,106 +49,112 @@ using namespace tc;
 
 constexpr int QMAX = 256;
 constexpr int PD = 64;
-constexpr uint32_t ST_COL = 384, IN_COL = 448;
+constexpr int NTHREADS = 416;  // 8 mask warps, 4 epilogue warps, 1 control warp
+constexpr int NMASK = 256;
+constexpr uint32_t CB0P = 0, CB1P = 64, CB1F = 128;
+__device__ __forceinline__ uint32_t st_col(int t) { return t == 0 ? 192u : 320u; }
+__device__ __forceinline__ uint32_t in_col(int t) { return t == 0 ? 256u : 384u; }
 
 template <int NST>
 struct ScanTile {
-    static constexpr int KB_BYTES = QMAX * 128;                    // one 64-wide K block, 256 rows
+    static constexpr int KB_BYTES = QMAX * 128;              // 64-wide K block of C or B
     static constexpr int C_OFF = 0;
     static constexpr int C_BYTES = (NST / 64) * KB_BYTES;
-    static constexpr int B_OFF = C_OFF + C_BYTES;
-    static constexpr int MASK_BYTES = 4 * 128 * 128;               // [4 kb][128 rows][128 B]
-    static constexpr int B_BYTES = C_BYTES > MASK_BYTES ? C_BYTES : MASK_BYTES;
-    static constexpr int X_OFF = B_OFF + B_BYTES;
-    static constexpr int X_BYTES = QMAX * 128;                     // MN-major [j][64 p]
-    static constexpr int H_OFF = X_OFF + 2 * X_BYTES;              // two x buffers
-    static constexpr int H_BYTES = (NST / 64) * PD * 128;          // K-major [kb][p][64 n]
-    static constexpr int CUM_OFF = H_OFF + H_BYTES;
+    static constexpr int B_OFF = C_OFF + C_BYTES;            // B, later tile 1's mask
+    static constexpr int MK1_BYTES = 4 * 128 * 128;
+    static constexpr int B_BYTES = C_BYTES > MK1_BYTES ? C_BYTES : MK1_BYTES;
+    static constexpr int MK0_OFF = B_OFF + B_BYTES;          // tile 0's mask
+    static constexpr int MK0_BYTES = 2 * 128 * 128;
+    static constexpr int X_OFF = MK0_OFF + MK0_BYTES;
+    static constexpr int X_BYTES = QMAX * 128;
+    static constexpr int H_OFF = X_OFF + X_BYTES;
+    static constexpr int H_BYTES = (NST / 64) * PD * 128;
+    static constexpr int CUM_OFF = H_OFF + H_BYTES;          // mask warps: log2e * cumA, dt
     static constexpr int DT_OFF = CUM_OFF + QMAX * 4;
-    static constexpr int STAB_OFF = DT_OFF + QMAX * 4;             // 8 warps x QMAX fp32
+    static constexpr int RINV_OFF = DT_OFF + QMAX * 4;       // per-row CB scale, 2 tiles
+    static constexpr int STAB_OFF = RINV_OFF + 2 * 128 * 4;  // 8 mask warps x QMAX
     static constexpr int BAR_OFF = STAB_OFF + 8 * QMAX * 4;
-    static constexpr int SMEM = BAR_OFF + 128 + 1024;
+    static constexpr int SMEM = BAR_OFF + 32 * 8 + 1024;
     static_assert(SMEM <= 232448, "shared memory budget");
 };
 
-__device__ __forceinline__ uint32_t cb_col(int t) { return t == 0 ? 256u : 0u; }
+enum : int {
+    B_CB_LOAD = 0, B_CB_DONE, B_CB_PACKED, B_X_FULL, B_H_FULL, B_H_FREE, B_X_FREE,
+    B_MK_FULL, B_MK_EMPTY = B_MK_FULL + 2, B_ACC_FULL = B_MK_EMPTY + 2,
+    B_ACC_EMPTY = B_ACC_FULL + 2, B_COUNT = B_ACC_EMPTY + 2
+};
 
-// Mk for the 128 rows of tile t, column groups of 32 split over the two
-// warpgroups; written as bf16 into the K-major mask operand.
-__device__ __forceinline__ void build_mask(int t, uint32_t tmem, uint32_t mbase, const float* cum,
-                                           const float* dtv, float* stab, int warp, int lane) {
-    const int rb = 32 * (warp & 3);             // tile-local row block
-    const int lb = 128 * t + rb;                // chunk row of the block's first row
-    const int l = lb + lane;                    // this thread's chunk row
-    const float cl = cum[l];
-    // per-warp table: s[j] = exp(cum[lb] - cum[j]) dt[j], j < lb
-    for (int j = lane; j < lb; j += 32) stab[j] = __expf(cum[lb] - cum[j]) * dtv[j];
+// Bounded wait that also gives up when another role has aborted.
+__device__ __forceinline__ bool wait_bar(uint32_t mbar, uint32_t parity, volatile int* abort) {
+    for (uint32_t i = 0; i < kSpinLimit; ++i) {
+        if (mbar_try_wait(mbar, parity)) return true;
+        if ((i & 63) == 63 && *abort) return false;
+    }
+    *abort = 1;
+    return false;
+}
+
+__device__ __forceinline__ void unpack_f16x32(const uint32_t (&r)[16], float (&v)[32]) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&r[i]));
+        v[2 * i] = f.x;
+        v[2 * i + 1] = f.y;
+    }
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    const __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// Mask warp: rows 128 t + 32 qd + lane of tile t (qd = TMEM lane quarter),
+// column groups of 32 with index = hf (mod 2).  cum2 holds log2(e) * cumA, so
+// every decay is one exp2; rinv undoes the row's CB scale.
+__device__ __forceinline__ void build_mask(int t, uint32_t tmem, uint32_t mbase, const float* cum2,
+                                           const float* dtv, float* stab, float rinv, int qd,
+                                           int hf, int lane) {
+    const int lb = 128 * t + 32 * qd;           // chunk row of the block's first row
+    const int l = lb + lane;
+    const float cl = cum2[l];
+    for (int j = lane; j < lb; j += 32) stab[j] = exp2f(cum2[lb] - cum2[j]) * dtv[j];
     __syncwarp();
-    const float rl = __expf(cl - cum[lb]);
-    const int ngroups = 4 * (t + 1);            // 32-wide column groups in [0, 128(t+1))
-    const int half = ngroups / 2;
-    const int gbeg = (warp >> 2) * half;
-    const uint32_t lane_addr = static_cast<uint32_t>(rb) << 16;
-    for (int gi = gbeg; gi < gbeg + half; ++gi) {
+    const float rl = exp2f(cl - cum2[lb]) * rinv;
+    const uint32_t cbase = tmem + (static_cast<uint32_t>(32 * qd) << 16) + (t == 0 ? CB0P : CB1P);
+    const uint32_t row = 32 * qd + lane;
+    const int ngroups = 4 * (t + 1);
+    for (int gi = hf; gi < ngroups; gi += 2) {
         const int j0 = 32 * gi;
+        const uint32_t dst = mbase + (j0 >> 6) * (128 * 128);
+        const int c0 = (j0 & 63) >> 3;
+        if (j0 > lb) {  // above the diagonal: zeros
+#pragma unroll
+            for (int i = 0; i < 4; ++i) st_shared_v4(dst + sw128(row, c0 + i), 0u, 0u, 0u, 0u);
+            continue;
+        }
+        uint32_t r[16];
         float v[32];
+        tmem_ld16(cbase + j0 / 2, r);
+        unpack_f16x32(r, v);
         if (j0 + 32 <= lb) {
-            tmem_ld32(tmem + lane_addr + cb_col(t) + j0, v);
 #pragma unroll
             for (int q = 0; q < 32; ++q) v[q] *= rl * stab[j0 + q];
-        } else if (j0 == lb) {
-            tmem_ld32(tmem + lane_addr + cb_col(t) + j0, v);
-#pragma unroll
-            for (int q = 0; q < 32; ++q)
-                v[q] = (q <= lane) ? v[q] * __expf(cl - cum[j0 + q]) * dtv[j0 + q] : 0.0f;
         } else {
 #pragma unroll
-            for (int q = 0; q < 32; ++q) v[q] = 0.0f;
+            for (int q = 0; q < 32; ++q)
+                v[q] = (q <= lane) ? v[q] * rinv * exp2f(cl - cum2[j0 + q]) * dtv[j0 + q] : 0.0f;
         }
-        const int kb = j0 >> 6, c0 = (j0 & 63) >> 3;
 #pragma unroll
         for (int i = 0; i < 4; ++i)
-            st_shared_v4(mbase + kb * (128 * 128) + sw128(rb + lane, c0 + i),
-                         pack_bf16x2(v[8 * i + 0], v[8 * i + 1]),
+            st_shared_v4(dst + sw128(row, c0 + i), pack_bf16x2(v[8 * i + 0], v[8 * i + 1]),
                          pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
                          pack_bf16x2(v[8 * i + 4], v[8 * i + 5]),
                          pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
     }
 }
 
-// y rows of tile t: warp w%4 -> rows, warpgroup -> 32 of the 64 p columns
-__device__ __forceinline__ void epilogue(int t, uint32_t tmem, uint32_t xbase, const float* cum,
-                                         const FwdParams& p, int64_t b, int64_t t0, int64_t h,
-                                         int Lc, int warp, int lane) {
-    const int r = 32 * (warp & 3) + lane;
-    const int l = 128 * t + r;
-    const int pc = 32 * (warp >> 2);
-    const uint32_t lane_addr = static_cast<uint32_t>(32 * (warp & 3)) << 16;
-    float vi[32], vs[32];
-    tmem_ld32x2(tmem + lane_addr + IN_COL + pc, vi, tmem + lane_addr + ST_COL + pc, vs);
-    if (l >= Lc) return;
-    const float sc = __expf(cum[l]);
-    const float Dh = p.D ? p.D[h] : 0.0f;
-    __nv_bfloat16* y = static_cast<__nv_bfloat16*>(p.y) +
-                       ((b * p.seqlen + t0 + l) * p.nheads + h) * PD + pc;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const uint4 xv = ld_shared_v4(xbase + sw128(l, (pc >> 3) + i));
-        const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
-        uint32_t o[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const float2 xf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xw[k]));
-            const int q = 8 * i + 2 * k;
-            o[k] = pack_bf16x2(vi[q] + sc * vs[q] + Dh * xf.x,
-                               vi[q + 1] + sc * vs[q + 1] + Dh * xf.y);
-        }
-        reinterpret_cast<uint4*>(y)[i] = make_uint4(o[0], o[1], o[2], o[3]);
-    }
-}
-
 template <int NST>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(NTHREADS, 1)
     chunk_scan_tc_kernel(const __grid_constant__ FwdParams p, const __grid_constant__ CUtensorMap tm_c,
                          const __grid_constant__ CUtensorMap tm_b,
                          const __grid_constant__ CUtensorMap tm_x,
@@ -145,12 +163,10 @@ __global__ void __launch_bounds__(256, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                ~static_cast<uintptr_t>(1023));
-    float* cum = reinterpret_cast<float*>(smem + T::CUM_OFF);
-    float* dtv = reinterpret_cast<float*>(smem + T::DT_OFF);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + T::BAR_OFF);
-    // barriers: 0 = C/B landed, 1 = CB done, 2/3 = x buffer 0/1 landed, 4 = tile-0 MMAs,
-    // 5 = tile-1 MMAs, 6 = H_in landed
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 7);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + B_COUNT);
+    volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    auto bar = [&](int i) { return smem_u32(&bars[i]); };
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t H = p.nheads, L = p.seqlen, Q = p.chunk, nc = p.nchunks, G = p.ngroups;
@@ -160,150 +176,229 @@ __global__ void __launch_bounds__(256, 1)
     const int64_t t0 = c * Q;
     const int Lc = static_cast<int>((L - t0 < Q) ? (L - t0) : Q);
     const int ntiles = (Lc + 127) / 128;
-    float* stab = reinterpret_cast<float*>(smem + T::STAB_OFF) + warp * QMAX;
     const uint32_t sC = smem_u32(smem + T::C_OFF), sB = smem_u32(smem + T::B_OFF);
+    const uint32_t sM0 = smem_u32(smem + T::MK0_OFF), sM1 = sB;
     const uint32_t sX = smem_u32(smem + T::X_OFF), sH = smem_u32(smem + T::H_OFF);
-    const uint32_t sM = sB;  // the mask operand reuses B's space once CB is done
-    auto bar = [&](int i) { return smem_u32(&bars[i]); };
 
     if (warp == 0) tmem_alloc(smem_u32(tmem_slot), 512);
     if (tid == 0) {
-        for (int i = 0; i < 7; ++i) mbar_init(bar(i), 1);
+        for (int i = 0; i < B_COUNT; ++i) {
+            uint32_t count = 1;
+            if (i == B_CB_PACKED || i == B_ACC_EMPTY || i == B_ACC_EMPTY + 1) count = 128;
+            if (i == B_MK_FULL || i == B_MK_FULL + 1) count = NMASK;
+            mbar_init(bar(i), count);
+        }
+        *abort = 0;
         fence_mbar_init();
-        tma_prefetch_map(&tm_c);
-        tma_prefetch_map(&tm_b);
-        tma_prefetch_map(&tm_x);
-        tma_prefetch_map(&tm_h);
     }
-    __syncthreads();
-    if (tid == 0) {
-        const uint32_t box = static_cast<uint32_t>(Q) * 128;
-        mbar_expect_tx(bar(0), 2 * (NST / 64) * box);
-        for (int kb = 0; kb < NST / 64; ++kb) {
-            tma_load_4d(sC + kb * T::KB_BYTES, &tm_c, bar(0), kb * 64, (int)g, (int)t0, (int)b);
-            tma_load_4d(sB + kb * T::KB_BYTES, &tm_b, bar(0), kb * 64, (int)g, (int)t0, (int)b);
-        }
-        for (int i = 0; i < 2 && i < hb_size; ++i) {
-            mbar_expect_tx(bar(2 + i), box);
-            tma_load_4d(sX + i * T::X_BYTES, &tm_x, bar(2 + i), 0, (int)(hfirst + i), (int)t0, (int)b);
-        }
-        mbar_expect_tx(bar(6), T::H_BYTES);
-        for (int kb = 0; kb < NST / 64; ++kb)
-            tma_load_4d(sH + kb * (PD * 128), &tm_h, bar(6), kb * 64, 0, (int)hfirst,
-                        (int)(b * nc + c));
-    }
-    // first head's decays
-    {
-        const int64_t vbase = ((b * H + hfirst) * nc + c) * Q;
-        for (int i = tid; i < QMAX; i += 256) {
-            cum[i] = (i < Q) ? p.cumA[vbase + i] : 0.0f;
-            dtv[i] = (i < Q) ? p.dt[vbase + i] : 0.0f;
-        }
-    }
-    fence_smem_async();
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
     const uint32_t tmem = *tmem_slot;
 
-    bool mine = true;
-    if (tid == 0) {
-        mine = mbar_wait(bar(0), 0);
-        if (mine) {
-            fence_after_sync();
-            for (int t = 0; t < ntiles; ++t) {
-                const uint32_t id = t == 0 ? idesc_bf16(128, 128, false, false)
-                                           : idesc_bf16(128, 256, false, false);
-                for (int k = 0; k < NST / 16; ++k) {
-                    const uint32_t ko = (k >> 2) * T::KB_BYTES + (k & 3) * 32;
-                    mma_bf16(tmem + cb_col(t), desc_sw128(sC + ko + t * 128 * 128, 16, 1024),
-                             desc_sw128(sB + ko, 16, 1024), id, k > 0 ? 1u : 0u);
-                }
+    if (warp == 12) {
+        // ------------------------------ control ------------------------------
+        if (lane == 0) {
+            const uint32_t box = static_cast<uint32_t>(Q) * 128;
+            auto load_x = [&](int64_t h) {
+                mbar_expect_tx(bar(B_X_FULL), box);
+                tma_load_4d(sX, &tm_x, bar(B_X_FULL), 0, (int)h, (int)t0, (int)b);
+            };
+            auto load_h = [&](int64_t h) {
+                mbar_expect_tx(bar(B_H_FULL), T::H_BYTES);
+                for (int kb = 0; kb < NST / 64; ++kb)
+                    tma_load_4d(sH + kb * (PD * 128), &tm_h, bar(B_H_FULL), kb * 64, 0, (int)h,
+                                (int)(b * nc + c));
+            };
+            tma_prefetch_map(&tm_c);
+            tma_prefetch_map(&tm_b);
+            tma_prefetch_map(&tm_x);
+            tma_prefetch_map(&tm_h);
+            mbar_expect_tx(bar(B_CB_LOAD), 2 * (NST / 64) * box);
+            for (int kb = 0; kb < NST / 64; ++kb) {
+                tma_load_4d(sC + kb * T::KB_BYTES, &tm_c, bar(B_CB_LOAD), kb * 64, (int)g,
+                            (int)t0, (int)b);
+                tma_load_4d(sB + kb * T::KB_BYTES, &tm_b, bar(B_CB_LOAD), kb * 64, (int)g,
+                            (int)t0, (int)b);
             }
-            mma_commit(bar(1));
-        }
-    }
-    bool ok = !__syncthreads_or(!mine);
-    if (ok) ok = !__syncthreads_or(!mbar_wait(bar(1), 0));
-    fence_after_sync();
-
-    for (int i = 0; ok && i < hb_size; ++i) {
-        const int64_t h = hfirst + i;
-        const int xb = i & 1;
-        const uint32_t xbase = sX + xb * T::X_BYTES;
-        // every thread observes the x tile's arrival (the epilogue reads it too)
-        ok = !__syncthreads_or(!mbar_wait(bar(2 + xb), (i >> 1) & 1));
-        if (!ok) break;
-        // the next head's decays, into registers now, into shared memory at the end
-        float cum_next = 0.0f, dt_next = 0.0f;
-        if (i + 1 < hb_size && tid < Q) {
-            const int64_t vbase = ((b * H + h + 1) * nc + c) * Q;
-            cum_next = p.cumA[vbase + tid];
-            dt_next = p.dt[vbase + tid];
-        }
-        for (int t = 0; t < ntiles; ++t) {
-            // CUDA cores: the decay mask of tile t
-            build_mask(t, tmem, sM, cum, dtv, stab, warp, lane);
-            fence_smem_async();
-            fence_before_sync();
-            __syncthreads();
-            // tensor core: state term and Mk x of tile t (the state has to have landed)
-            bool mine = true;
-            if (tid == 0) {
+            load_x(hfirst);
+            load_h(hfirst);
+            bool ok = wait_bar(bar(B_CB_LOAD), 0, abort);
+            if (ok) {
                 fence_after_sync();
-                if (t == 0) mine = mbar_wait(bar(6), i & 1);
-                if (mine) {
+                for (int t = 0; t < ntiles; ++t) {
+                    const uint32_t id = idesc_bf16(128, 128 * (t + 1), false, false);
+                    for (int k = 0; k < NST / 16; ++k) {
+                        const uint32_t ko = (k >> 2) * T::KB_BYTES + (k & 3) * 32;
+                        mma_bf16(tmem + (t == 0 ? 0u : CB1F),
+                                 desc_sw128(sC + ko + t * 128 * 128, 16, 1024),
+                                 desc_sw128(sB + ko, 16, 1024), id, k > 0 ? 1u : 0u);
+                    }
+                }
+                mma_commit(bar(B_CB_DONE));
+                ok = wait_bar(bar(B_CB_PACKED), 0, abort);  // CB packed: accumulators free
+                fence_after_sync();
+            }
+            for (int i = 0; ok && i < hb_size; ++i) {
+                const uint32_t ph = i & 1;
+                ok = wait_bar(bar(B_H_FULL), ph, abort);
+                for (int t = 0; ok && t < ntiles; ++t) {
+                    // state term of tile t, once the epilogue has drained its accumulators
+                    if (i > 0) ok = wait_bar(bar(B_ACC_EMPTY + t), (i - 1) & 1, abort);
+                    if (!ok) break;
+                    fence_after_sync();
                     for (int k = 0; k < NST / 16; ++k) {
                         const uint32_t ko = (k >> 2) * T::KB_BYTES + (k & 3) * 32;
                         const uint32_t kh = (k >> 2) * (PD * 128) + (k & 3) * 32;
-                        mma_bf16(tmem + ST_COL, desc_sw128(sC + ko + t * 128 * 128, 16, 1024),
+                        mma_bf16(tmem + st_col(t), desc_sw128(sC + ko + t * 128 * 128, 16, 1024),
                                  desc_sw128(sH + kh, 16, 1024), idesc_bf16(128, PD, false, false),
                                  k > 0 ? 1u : 0u);
                     }
-                    for (int k = 0; k < 8 * (t + 1); ++k) {
-                        mma_bf16(tmem + IN_COL,
+                    if (t == ntiles - 1) mma_commit(bar(B_H_FREE));
+                    // intra-chunk term of tile t, once its mask (and the head's x) is in
+                    ok = wait_bar(bar(B_MK_FULL + t), ph, abort);
+                    if (ok && t == 0) ok = wait_bar(bar(B_X_FULL), ph, abort);
+                    if (!ok) break;
+                    fence_after_sync();
+                    const uint32_t sM = t == 0 ? sM0 : sM1;
+                    for (int k = 0; k < 8 * (t + 1); ++k)
+                        mma_bf16(tmem + in_col(t),
                                  desc_sw128(sM + (k >> 2) * (128 * 128) + (k & 3) * 32, 16, 1024),
-                                 desc_sw128(xbase + k * 2048, QMAX * 128, 1024),
+                                 desc_sw128(sX + k * 2048, QMAX * 128, 1024),
                                  idesc_bf16(128, PD, false, true), k > 0 ? 1u : 0u);
-                    }
-                    mma_commit(bar(4 + t));
+                    mma_commit(bar(B_ACC_FULL + t));
+                    mma_commit(bar(B_MK_EMPTY + t));
+                }
+                if (!ok) break;
+                mma_commit(bar(B_X_FREE));
+                if (i + 1 < hb_size) {  // refill the state and x buffers for the next head
+                    ok = wait_bar(bar(B_H_FREE), ph, abort);
+                    if (ok) load_h(hfirst + i + 1);
+                    if (ok) ok = wait_bar(bar(B_X_FREE), ph, abort);
+                    if (ok) load_x(hfirst + i + 1);
                 }
             }
-            ok = !__syncthreads_or(!mine);
-            if (ok) ok = !__syncthreads_or(!mbar_wait(bar(4 + t), i & 1));
+            if (!ok) *abort = 1;
+        }
+    } else if (warp < 8) {
+        // -------------------------------- mask -------------------------------
+        const int qd = warp & 3, hf = warp >> 2;
+        float* cum2 = reinterpret_cast<float*>(smem + T::CUM_OFF);
+        float* dtv = reinterpret_cast<float*>(smem + T::DT_OFF);
+        float* rinv_s = reinterpret_cast<float*>(smem + T::RINV_OFF);
+        float* stab = reinterpret_cast<float*>(smem + T::STAB_OFF) + warp * QMAX;
+        const uint32_t lanes = static_cast<uint32_t>(32 * qd) << 16;
+        bool ok = wait_bar(bar(B_CB_DONE), 0, abort);
+        if (ok && hf == 0) {
             fence_after_sync();
-            if (!ok) break;
-            epilogue(t, tmem, xbase, cum, p, b, t0, h, Lc, warp, lane);
-            fence_before_sync();
-            __syncthreads();
-        }
-        if (!ok) break;
-        // the next head's decays; its x and state are already on the way
-        if (i + 1 < hb_size) {
-            cum[tid] = cum_next;
-            dtv[tid] = dt_next;
-        }
-        fence_before_sync();
-        __syncthreads();
-        fence_after_sync();
-        if (tid == 0) {
-            // every MMA of this head is done: its H_in buffer takes the next head's
-            // state, its x buffer head i + 2's x
-            if (i + 1 < hb_size) {
-                mbar_expect_tx(bar(6), T::H_BYTES);
-                for (int kb = 0; kb < NST / 64; ++kb)
-                    tma_load_4d(sH + kb * (PD * 128), &tm_h, bar(6), kb * 64, 0, (int)(h + 1),
-                                (int)(b * nc + c));
+            // repack CB as fp16 pairs with a per-row power-of-two scale:
+            // tile 0 [0,128) -> [0,64), tile 1 [128,384) -> [64,192)
+            for (int t = 0; t < ntiles; ++t) {
+                const uint32_t src = t == 0 ? 0u : CB1F, dst = t == 0 ? CB0P : CB1P;
+                float mx = 0.0f;
+                for (int k = 0; k < 4 * (t + 1); ++k) {
+                    float v[32];
+                    tmem_ld32(tmem + lanes + src + 32 * k, v);
+#pragma unroll
+                    for (int q = 0; q < 32; ++q) mx = fmaxf(mx, fabsf(v[q]));
+                }
+                // 2^e with the row's largest |CB| * 2^-e below 2^15
+                const int e2 = max(0, ((__float_as_int(mx) >> 23) & 255) - 127 - 14 + 1);
+                const float sc = __int_as_float((127 - e2) << 23);
+                rinv_s[t * 128 + 32 * qd + lane] = __int_as_float((127 + e2) << 23);
+                for (int k = 0; k < 4 * (t + 1); ++k) {
+                    float v[32];
+                    uint32_t r[16];
+                    tmem_ld32(tmem + lanes + src + 32 * k, v);
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) r[q] = pack_f16x2(v[2 * q] * sc, v[2 * q + 1] * sc);
+                    tmem_st16(tmem + lanes + dst + 16 * k, r);
+                }
+                tmem_wait_st();
             }
-            if (i + 2 < hb_size) {
-                mbar_expect_tx(bar(2 + xb), static_cast<uint32_t>(Q) * 128);
-                tma_load_4d(xbase, &tm_x, bar(2 + xb), 0, (int)(h + 2), (int)t0, (int)b);
+            fence_before_sync();
+            mbar_arrive(bar(B_CB_PACKED));
+        }
+        if (ok && hf == 1) ok = wait_bar(bar(B_CB_PACKED), 0, abort);
+        fence_after_sync();
+        const float rinv0 = ok ? rinv_s[32 * qd + lane] : 1.0f;
+        const float rinv1 = (ok && ntiles == 2) ? rinv_s[128 + 32 * qd + lane] : 1.0f;
+        for (int i = 0; ok && i < hb_size; ++i) {
+            const int64_t vbase = ((b * H + hfirst + i) * nc + c) * Q;
+            named_sync(1, NMASK);  // every mask warp is done with the previous head's decays
+            {
+                const int k = tid;  // 256 mask threads, 256 entries
+                cum2[k] = (k < Q) ? p.cumA[vbase + k] * 1.4426950408889634f : 0.0f;
+                dtv[k] = (k < Q) ? p.dt[vbase + k] : 0.0f;
+            }
+            named_sync(1, NMASK);
+            for (int t = 0; t < ntiles; ++t) {
+                if (i > 0) ok = wait_bar(bar(B_MK_EMPTY + t), (i - 1) & 1, abort);
+                if (!ok) break;
+                build_mask(t, tmem, t == 0 ? sM0 : sM1, cum2, dtv, stab, t == 0 ? rinv0 : rinv1,
+                           qd, hf, lane);
+                fence_smem_async();
+                mbar_arrive(bar(B_MK_FULL + t));
+            }
+        }
+    } else {
+        // ------------------------------ epilogue -----------------------------
+        const int q = warp & 3;
+        const uint32_t lanes = static_cast<uint32_t>(32 * q) << 16;
+        bool ok = true;
+        for (int i = 0; ok && i < hb_size; ++i) {
+            const int64_t h = hfirst + i;
+            const int64_t vbase = ((b * H + h) * nc + c) * Q;
+            const float D = p.D ? p.D[h] : 0.0f;
+            for (int t = 0; t < ntiles; ++t) {
+                const int l = 128 * t + 32 * q + lane;
+                const bool valid = l < Lc;
+                const float sc = valid ? __expf(p.cumA[vbase + l]) : 0.0f;
+                const __nv_bfloat16* xr = static_cast<const __nv_bfloat16*>(p.x) +
+                                          ((b * L + t0 + l) * H + h) * PD;
+                __nv_bfloat16* yr =
+                    static_cast<__nv_bfloat16*>(p.y) + ((b * L + t0 + l) * H + h) * PD;
+                // x for the D skip, fetched before the accumulators are ready
+                uint4 xv[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) xv[k] = valid ? ldg16(xr + 8 * k) : make_uint4(0u, 0u, 0u, 0u);
+                ok = wait_bar(bar(B_ACC_FULL + t), i & 1, abort);
+                if (!ok) break;
+                fence_after_sync();
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    float vi[32], vs[32];
+                    tmem_ld32x2(tmem + lanes + in_col(t) + 32 * half, vi,
+                                tmem + lanes + st_col(t) + 32 * half, vs);
+                    if (half == 1) {  // both accumulators read: let the next head's MMAs in
+                        fence_before_sync();
+                        mbar_arrive(bar(B_ACC_EMPTY + t));
+                    }
+                    if (valid) {
+#pragma unroll
+                        for (int k4 = 0; k4 < 4; ++k4) {
+                            const uint4 xq = xv[4 * half + k4];
+                            const uint32_t xw[4] = {xq.x, xq.y, xq.z, xq.w};
+                            uint32_t o[4];
+#pragma unroll
+                            for (int k = 0; k < 4; ++k) {
+                                const float2 xf = __bfloat1622float2(
+                                    *reinterpret_cast<const __nv_bfloat162*>(&xw[k]));
+                                const int e = 8 * k4 + 2 * k;
+                                o[k] = pack_bf16x2(vi[e] + sc * vs[e] + D * xf.x,
+                                                   vi[e + 1] + sc * vs[e + 1] + D * xf.y);
+                            }
+                            reinterpret_cast<uint4*>(yr + 32 * half)[k4] =
+                                make_uint4(o[0], o[1], o[2], o[3]);
+                        }
+                    }
+                }
             }
         }
     }
-    if (!ok && tid == 0 && p.status) atomicExch(p.status, static_cast<int>(SSD_ERR_TIMEOUT));
     fence_before_sync();
     __syncthreads();
+    if (*abort && tid == 0 && p.status) atomicExch(p.status, static_cast<int>(SSD_ERR_TIMEOUT));
     if (warp == 0) {
         fence_after_sync();
         tmem_dealloc(tmem, 512);
@@ -337,7 +432,7 @@ cudaError_t launch_n(const FwdParams& p, cudaStream_t s) {
     const int hb = heads_per_cta(p);
     dim3 grid(static_cast<unsigned>(p.nchunks * p.ngroups * (p.heads_per_group / hb)),
               static_cast<unsigned>(p.batch));
-    kern<<<grid, 256, T::SMEM, s>>>(p, tc_, tb_, tx_, th_, hb);
+    kern<<<grid, NTHREADS, T::SMEM, s>>>(p, tc_, tb_, tx_, th_, hb);
     return cudaGetLastError();
 }
 

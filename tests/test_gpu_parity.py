@@ -11,7 +11,7 @@ import torch
 
 import mamba_ssd_scan_b200 as ssd
 from mamba_ssd_scan_b200 import synthetic
-from tolerance import assert_close
+from tolerance import assert_close, report
 
 pytestmark = pytest.mark.gpu
 
@@ -158,6 +158,7 @@ def test_workload_sampled_heads(orc, name, heads, batches):
     y, fin = run_fwd(inp, cfg.chunk)
     yo, fo = oracle_heads(orc, inp, heads, batches)
     bsel = slice(None) if batches is None else batches
+    print(name, "y", report(y.cpu()[bsel][:, :, heads], yo))
     assert_close(y.cpu()[bsel][:, :, heads], yo, cfg.dtype, "y (sampled heads)")
     assert_close(fin.cpu()[bsel][:, heads], fo, cfg.dtype, "final (sampled heads)")
 
