@@ -51,6 +51,23 @@ def _compile(src: str, obj: str, verbose_ptxas: bool) -> str:
     return r.stderr
 
 
+def build_trace() -> str:
+    """A separate build with -DSSD_TRACE (kernel timelines), to _build/; never
+    the library the package loads."""
+    out_dir = os.path.join(BUILD, "trace")
+    os.makedirs(out_dir, exist_ok=True)
+    objs = []
+    for src in sorted(glob.glob(os.path.join(CSRC, "*.cu"))):
+        obj = os.path.join(out_dir, os.path.basename(src)[:-3] + ".o")
+        cmd = [nvcc()] + NVCC_FLAGS + ["-DSSD_TRACE", "-c", src, "-o", obj]
+        subprocess.run(cmd, check=True)
+        objs.append(obj)
+    lib = os.path.join(out_dir, "libssd_b200_trace.so")
+    subprocess.run([nvcc()] + ARCH + ["-shared", "-Xcompiler", "-fPIC", "-cudart", "static"] +
+                   objs + ["-o", lib], check=True)
+    return lib
+
+
 def build(force: bool = False, verbose_ptxas: bool = False) -> str:
     os.makedirs(BUILD, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
@@ -81,4 +98,7 @@ def build(force: bool = False, verbose_ptxas: bool = False) -> str:
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose_ptxas="--verbose-ptxas" in sys.argv))
+    if "--trace" in sys.argv:
+        print(build_trace())
+    else:
+        print(build(force="--force" in sys.argv, verbose_ptxas="--verbose-ptxas" in sys.argv))

@@ -49,7 +49,7 @@ using namespace tc;
 
 constexpr int QMAX = 256;
 constexpr int PD = 64;
-constexpr int NTHREADS = 416;  // 8 mask warps, 4 epilogue warps, 1 control warp
+constexpr int NTHREADS = 288;  // 8 worker warps, 1 control warp
 constexpr int NMASK = 256;
 constexpr uint32_t CB0P = 0, CB1P = 64, CB1F = 128;
 __device__ __forceinline__ uint32_t st_col(int t) { return t == 0 ? 192u : 320u; }
@@ -78,17 +78,45 @@ struct ScanTile {
     static_assert(SMEM <= 232448, "shared memory budget");
 };
 
+// Optional timeline of the first CTAs (builds with -DSSD_TRACE only): each role
+// stamps the SM cycle counter at its hand-offs; ssd_scan_trace_copy() reads it
+// back.
+#ifdef SSD_TRACE
+__device__ unsigned long long g_scan_trace[8][256];
+#define SCAN_TRACE(slot)                                                              \
+    do {                                                                              \
+        if (blockIdx.x < 8 && blockIdx.y == 0 && (slot) < 256) {                      \
+            g_scan_trace[blockIdx.x][(slot)] = clock64();                             \
+        }                                                                             \
+    } while (0)
+// SM-clock stamps of warp 0 inside the mask routine, head 1 only
+#define MASK_CLOCK(slot)                                                              \
+    do {                                                                              \
+        if (blockIdx.x < 8 && blockIdx.y == 0 && threadIdx.x == 0)                    \
+            g_scan_trace[blockIdx.x][(slot)] = clock64();                             \
+    } while (0)
+#else
+#define SCAN_TRACE(slot) \
+    do {                 \
+    } while (0)
+#define MASK_CLOCK(slot) \
+    do {                 \
+    } while (0)
+#endif
+
 enum : int {
     B_CB_LOAD = 0, B_CB_DONE, B_CB_PACKED, B_X_FULL, B_H_FULL, B_H_FREE, B_X_FREE,
     B_MK_FULL, B_MK_EMPTY = B_MK_FULL + 2, B_ACC_FULL = B_MK_EMPTY + 2,
     B_ACC_EMPTY = B_ACC_FULL + 2, B_COUNT = B_ACC_EMPTY + 2
 };
 
-// Bounded wait that also gives up when another role has aborted.
+// Bounded wait that also gives up when another role has aborted.  It spins on
+// the non-blocking probe: a suspending try_wait wakes up late (~1 us), which
+// on the hand-offs of this pipeline costs more than the spin.
 __device__ __forceinline__ bool wait_bar(uint32_t mbar, uint32_t parity, volatile int* abort) {
-    for (uint32_t i = 0; i < kSpinLimit; ++i) {
-        if (mbar_try_wait(mbar, parity)) return true;
-        if ((i & 63) == 63 && *abort) return false;
+    for (uint32_t i = 0; i < 4 * kSpinLimit; ++i) {
+        if (mbar_test_wait(mbar, parity)) return true;
+        if ((i & 255) == 255 && *abort) return false;
     }
     *abort = 1;
     return false;
@@ -109,40 +137,57 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
 }
 
 // Mask warp: rows 128 t + 32 qd + lane of tile t (qd = TMEM lane quarter),
-// column groups of 32 with index = hf (mod 2).  cum2 holds log2(e) * cumA, so
-// every decay is one exp2; rinv undoes the row's CB scale.
-__device__ __forceinline__ void build_mask(int t, uint32_t tmem, uint32_t mbase, const float* cum2,
+// column groups of 32 with index = hf (mod 2): 2 groups in tile 0, 4 in tile
+// 1.  The warp's TMEM reads are issued together and waited for once; the
+// per-block decay table is filled while they are in flight.  cum2 holds
+// log2(e) * cumA, so every decay is one exp2; rinv undoes the row's CB scale.
+template <int TT>
+__device__ __forceinline__ void build_mask(uint32_t tmem, uint32_t mbase, const float* cum2,
                                            const float* dtv, float* stab, float rinv, int qd,
                                            int hf, int lane) {
-    const int lb = 128 * t + 32 * qd;           // chunk row of the block's first row
+    constexpr int NG = 2 * (TT + 1);            // this warp's groups
+    const int lb = 128 * TT + 32 * qd;          // chunk row of the block's first row
     const int l = lb + lane;
+    const uint32_t cbase = tmem + (static_cast<uint32_t>(32 * qd) << 16) + (TT == 0 ? CB0P : CB1P);
+    uint32_t addr[NG];
+    uint32_t raw[NG][16];
+#pragma unroll
+    for (int k = 0; k < NG; ++k) addr[k] = cbase + 16 * (hf + 2 * k);   // j0 / 2
+    MASK_CLOCK(200 + 10 * TT);
+    if constexpr (NG == 2) tmem_ld16x2(addr, raw);
+    else tmem_ld16x4(addr, raw);
+    MASK_CLOCK(201 + 10 * TT);
     const float cl = cum2[l];
-    for (int j = lane; j < lb; j += 32) stab[j] = exp2f(cum2[lb] - cum2[j]) * dtv[j];
+    for (int j = lane; j < lb; j += 32) stab[j] = ex2(cum2[lb] - cum2[j]) * dtv[j];
     __syncwarp();
-    const float rl = exp2f(cl - cum2[lb]) * rinv;
-    const uint32_t cbase = tmem + (static_cast<uint32_t>(32 * qd) << 16) + (t == 0 ? CB0P : CB1P);
+    const float rl = ex2(cl - cum2[lb]) * rinv;
+    MASK_CLOCK(202 + 10 * TT);
     const uint32_t row = 32 * qd + lane;
-    const int ngroups = 4 * (t + 1);
-    for (int gi = hf; gi < ngroups; gi += 2) {
-        const int j0 = 32 * gi;
+#pragma unroll
+    for (int k = 0; k < NG; ++k) {
+        const int j0 = 32 * (hf + 2 * k);
         const uint32_t dst = mbase + (j0 >> 6) * (128 * 128);
         const int c0 = (j0 & 63) >> 3;
+        float v[32];
         if (j0 > lb) {  // above the diagonal: zeros
 #pragma unroll
-            for (int i = 0; i < 4; ++i) st_shared_v4(dst + sw128(row, c0 + i), 0u, 0u, 0u, 0u);
-            continue;
-        }
-        uint32_t r[16];
-        float v[32];
-        tmem_ld16(cbase + j0 / 2, r);
-        unpack_f16x32(r, v);
-        if (j0 + 32 <= lb) {
-#pragma unroll
-            for (int q = 0; q < 32; ++q) v[q] *= rl * stab[j0 + q];
+            for (int q = 0; q < 32; ++q) v[q] = 0.0f;
         } else {
+            unpack_f16x32(raw[k], v);
+            if (j0 + 32 <= lb) {
 #pragma unroll
-            for (int q = 0; q < 32; ++q)
-                v[q] = (q <= lane) ? v[q] * rinv * exp2f(cl - cum2[j0 + q]) * dtv[j0 + q] : 0.0f;
+                for (int q = 0; q < 32; ++q) v[q] *= rl * stab[j0 + q];
+            } else {
+                // the diagonal block: one exp2 per element, computed for every
+                // lane (exponent clamped at 0, so the entries above the diagonal
+                // stay finite) and then selected -- no divergent branches
+#pragma unroll
+                for (int q = 0; q < 32; ++q) {
+                    const float e = ex2(fminf(cl - cum2[j0 + q], 0.0f)) * dtv[j0 + q];
+                    const float m = v[q] * rinv * e;
+                    v[q] = (q <= lane) ? m : 0.0f;
+                }
+            }
         }
 #pragma unroll
         for (int i = 0; i < 4; ++i)
@@ -150,6 +195,7 @@ __device__ __forceinline__ void build_mask(int t, uint32_t tmem, uint32_t mbase,
                          pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
                          pack_bf16x2(v[8 * i + 4], v[8 * i + 5]),
                          pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
+        MASK_CLOCK(203 + 10 * TT + k);
     }
 }
 
@@ -184,8 +230,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (tid == 0) {
         for (int i = 0; i < B_COUNT; ++i) {
             uint32_t count = 1;
-            if (i == B_CB_PACKED || i == B_ACC_EMPTY || i == B_ACC_EMPTY + 1) count = 128;
-            if (i == B_MK_FULL || i == B_MK_FULL + 1) count = NMASK;
+            if (i == B_CB_PACKED) count = 128;
+            if (i == B_MK_FULL || i == B_MK_FULL + 1 || i == B_ACC_EMPTY || i == B_ACC_EMPTY + 1)
+                count = NMASK;
             mbar_init(bar(i), count);
         }
         *abort = 0;
@@ -196,7 +243,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     fence_after_sync();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == 12) {
+    if (warp == 8) {
         // ------------------------------ control ------------------------------
         if (lane == 0) {
             const uint32_t box = static_cast<uint32_t>(Q) * 128;
@@ -221,9 +268,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 tma_load_4d(sB + kb * T::KB_BYTES, &tm_b, bar(B_CB_LOAD), kb * 64, (int)g,
                             (int)t0, (int)b);
             }
+            SCAN_TRACE(0);
             load_x(hfirst);
             load_h(hfirst);
             bool ok = wait_bar(bar(B_CB_LOAD), 0, abort);
+            SCAN_TRACE(1);
             if (ok) {
                 fence_after_sync();
                 for (int t = 0; t < ntiles; ++t) {
@@ -237,11 +286,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 }
                 mma_commit(bar(B_CB_DONE));
                 ok = wait_bar(bar(B_CB_PACKED), 0, abort);  // CB packed: accumulators free
+                SCAN_TRACE(2);
                 fence_after_sync();
             }
             for (int i = 0; ok && i < hb_size; ++i) {
                 const uint32_t ph = i & 1;
                 ok = wait_bar(bar(B_H_FULL), ph, abort);
+                SCAN_TRACE(8 + 8 * i);
                 for (int t = 0; ok && t < ntiles; ++t) {
                     // state term of tile t, once the epilogue has drained its accumulators
                     if (i > 0) ok = wait_bar(bar(B_ACC_EMPTY + t), (i - 1) & 1, abort);
@@ -255,8 +306,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                                  k > 0 ? 1u : 0u);
                     }
                     if (t == ntiles - 1) mma_commit(bar(B_H_FREE));
+                    SCAN_TRACE(9 + 8 * i + 3 * t);
                     // intra-chunk term of tile t, once its mask (and the head's x) is in
                     ok = wait_bar(bar(B_MK_FULL + t), ph, abort);
+                    SCAN_TRACE(10 + 8 * i + 3 * t);
                     if (ok && t == 0) ok = wait_bar(bar(B_X_FULL), ph, abort);
                     if (!ok) break;
                     fence_after_sync();
@@ -268,6 +321,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                                  idesc_bf16(128, PD, false, true), k > 0 ? 1u : 0u);
                     mma_commit(bar(B_ACC_FULL + t));
                     mma_commit(bar(B_MK_EMPTY + t));
+                    SCAN_TRACE(11 + 8 * i + 3 * t);
+#ifdef SSD_TRACE
+                    if (t == 0 && i < 8) {  // latency of this tile's MMAs and commit
+                        wait_bar(bar(B_MK_EMPTY), ph, abort);
+                        SCAN_TRACE(176 + i);
+                    }
+#endif
                 }
                 if (!ok) break;
                 mma_commit(bar(B_X_FREE));
@@ -275,13 +335,14 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     ok = wait_bar(bar(B_H_FREE), ph, abort);
                     if (ok) load_h(hfirst + i + 1);
                     if (ok) ok = wait_bar(bar(B_X_FREE), ph, abort);
+                    SCAN_TRACE(15 + 8 * i);
                     if (ok) load_x(hfirst + i + 1);
                 }
             }
             if (!ok) *abort = 1;
         }
-    } else if (warp < 8) {
-        // -------------------------------- mask -------------------------------
+    } else {
+        // ------------------------------ workers ------------------------------
         const int qd = warp & 3, hf = warp >> 2;
         float* cum2 = reinterpret_cast<float*>(smem + T::CUM_OFF);
         float* dtv = reinterpret_cast<float*>(smem + T::DT_OFF);
@@ -318,81 +379,108 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             fence_before_sync();
             mbar_arrive(bar(B_CB_PACKED));
+            if (warp == 0 && lane == 0) SCAN_TRACE(80);
         }
         if (ok && hf == 1) ok = wait_bar(bar(B_CB_PACKED), 0, abort);
         fence_after_sync();
         const float rinv0 = ok ? rinv_s[32 * qd + lane] : 1.0f;
         const float rinv1 = (ok && ntiles == 2) ? rinv_s[128 + 32 * qd + lane] : 1.0f;
-        for (int i = 0; ok && i < hb_size; ++i) {
-            const int64_t vbase = ((b * H + hfirst + i) * nc + c) * Q;
-            named_sync(1, NMASK);  // every mask warp is done with the previous head's decays
-            {
-                const int k = tid;  // 256 mask threads, 256 entries
-                cum2[k] = (k < Q) ? p.cumA[vbase + k] * 1.4426950408889634f : 0.0f;
-                dtv[k] = (k < Q) ? p.dt[vbase + k] : 0.0f;
-            }
-            named_sync(1, NMASK);
-            for (int t = 0; t < ntiles; ++t) {
-                if (i > 0) ok = wait_bar(bar(B_MK_EMPTY + t), (i - 1) & 1, abort);
-                if (!ok) break;
-                build_mask(t, tmem, t == 0 ? sM0 : sM1, cum2, dtv, stab, t == 0 ? rinv0 : rinv1,
-                           qd, hf, lane);
-                fence_smem_async();
-                mbar_arrive(bar(B_MK_FULL + t));
-            }
-        }
-    } else {
-        // ------------------------------ epilogue -----------------------------
-        const int q = warp & 3;
-        const uint32_t lanes = static_cast<uint32_t>(32 * q) << 16;
-        bool ok = true;
-        for (int i = 0; ok && i < hb_size; ++i) {
+
+        // The epilogue of head i, tile t, for this warp's rows and 32 p columns, in
+        // two halves: its global loads (x for the D skip, exp(cumA) of the row, D)
+        // are issued before the tile's mask is built, so that they have landed
+        // by the time this thread waits on an mbarrier again (an acquire wait
+        // also waits for the thread's outstanding loads).
+        struct EpiIn {
+            uint4 xv[4];
+            float sc, D;
+            int64_t rowoff;
+            bool valid;
+        };
+        auto epi_load = [&](int i, int t, EpiIn& e) {
             const int64_t h = hfirst + i;
+            const int l = 128 * t + 32 * qd + lane;
+            e.valid = l < Lc;
             const int64_t vbase = ((b * H + h) * nc + c) * Q;
-            const float D = p.D ? p.D[h] : 0.0f;
-            for (int t = 0; t < ntiles; ++t) {
-                const int l = 128 * t + 32 * q + lane;
-                const bool valid = l < Lc;
-                const float sc = valid ? __expf(p.cumA[vbase + l]) : 0.0f;
-                const __nv_bfloat16* xr = static_cast<const __nv_bfloat16*>(p.x) +
-                                          ((b * L + t0 + l) * H + h) * PD;
-                __nv_bfloat16* yr =
-                    static_cast<__nv_bfloat16*>(p.y) + ((b * L + t0 + l) * H + h) * PD;
-                // x for the D skip, fetched before the accumulators are ready
-                uint4 xv[8];
+            e.sc = e.valid ? p.cumA[vbase + l] : 0.0f;
+            e.D = p.D ? p.D[h] : 0.0f;
+            e.rowoff = ((b * L + t0 + l) * H + h) * PD + 32 * hf;
 #pragma unroll
-                for (int k = 0; k < 8; ++k) xv[k] = valid ? ldg16(xr + 8 * k) : make_uint4(0u, 0u, 0u, 0u);
-                ok = wait_bar(bar(B_ACC_FULL + t), i & 1, abort);
-                if (!ok) break;
-                fence_after_sync();
+            for (int k = 0; k < 4; ++k)
+                e.xv[k] = e.valid ? ldg16(static_cast<const __nv_bfloat16*>(p.x) + e.rowoff + 8 * k)
+                                  : make_uint4(0u, 0u, 0u, 0u);
+        };
+        auto epi_finish = [&](int i, int t, const EpiIn& e) -> bool {
+            if (!wait_bar(bar(B_ACC_FULL + t), i & 1, abort)) return false;
+            if (warp == 0 && lane == 0) SCAN_TRACE(140 + 4 * i + 2 * t);
+            fence_after_sync();
+            float vi[32], vs[32];
+            tmem_ld32x2(tmem + lanes + in_col(t) + 32 * hf, vi, tmem + lanes + st_col(t) + 32 * hf, vs);
+            fence_before_sync();
+            mbar_arrive(bar(B_ACC_EMPTY + t));
+            if (e.valid) {
+                const float sc = ex2(e.sc * 1.4426950408889634f);
+                __nv_bfloat16* yr = static_cast<__nv_bfloat16*>(p.y) + e.rowoff;
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    float vi[32], vs[32];
-                    tmem_ld32x2(tmem + lanes + in_col(t) + 32 * half, vi,
-                                tmem + lanes + st_col(t) + 32 * half, vs);
-                    if (half == 1) {  // both accumulators read: let the next head's MMAs in
-                        fence_before_sync();
-                        mbar_arrive(bar(B_ACC_EMPTY + t));
+                for (int k4 = 0; k4 < 4; ++k4) {
+                    const uint32_t xw[4] = {e.xv[k4].x, e.xv[k4].y, e.xv[k4].z, e.xv[k4].w};
+                    uint32_t o[4];
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const float2 xf =
+                            __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xw[k]));
+                        const int q = 8 * k4 + 2 * k;
+                        o[k] = pack_bf16x2(vi[q] + sc * vs[q] + e.D * xf.x,
+                                           vi[q + 1] + sc * vs[q + 1] + e.D * xf.y);
                     }
-                    if (valid) {
-#pragma unroll
-                        for (int k4 = 0; k4 < 4; ++k4) {
-                            const uint4 xq = xv[4 * half + k4];
-                            const uint32_t xw[4] = {xq.x, xq.y, xq.z, xq.w};
-                            uint32_t o[4];
-#pragma unroll
-                            for (int k = 0; k < 4; ++k) {
-                                const float2 xf = __bfloat1622float2(
-                                    *reinterpret_cast<const __nv_bfloat162*>(&xw[k]));
-                                const int e = 8 * k4 + 2 * k;
-                                o[k] = pack_bf16x2(vi[e] + sc * vs[e] + D * xf.x,
-                                                   vi[e + 1] + sc * vs[e + 1] + D * xf.y);
-                            }
-                            reinterpret_cast<uint4*>(yr + 32 * half)[k4] =
-                                make_uint4(o[0], o[1], o[2], o[3]);
-                        }
-                    }
+                    reinterpret_cast<uint4*>(yr)[k4] = make_uint4(o[0], o[1], o[2], o[3]);
                 }
+            }
+            if (warp == 0 && lane == 0) SCAN_TRACE(141 + 4 * i + 2 * t);
+            return true;
+        };
+
+        // this head's decays travel in registers one head ahead (256 worker
+        // threads, one entry each)
+        float cum_r = 0.0f, dt_r = 0.0f;
+        if (tid < Q) {
+            const int64_t vbase = ((b * H + hfirst) * nc + c) * Q;
+            cum_r = p.cumA[vbase + tid];
+            dt_r = p.dt[vbase + tid];
+        }
+        // Every worker runs every iteration and reaches both named barriers even
+        // after a failed wait (the work is skipped), so no worker is left waiting
+        // at a barrier another one has abandoned.  Iteration i builds head i's
+        // masks and drains head i-1's accumulators, tile by tile.
+        for (int i = 0; i <= hb_size; ++i) {
+            const bool mask_now = i < hb_size, epi_now = i > 0;
+            if (mask_now) {
+                named_sync(1, NMASK);  // every worker is done with the previous head's decays
+                cum2[tid] = cum_r * 1.4426950408889634f;
+                dtv[tid] = dt_r;
+                named_sync(1, NMASK);
+                if (warp == 0 && lane == 0) SCAN_TRACE(82 + 5 * i);
+            }
+            for (int t = 0; t < ntiles; ++t) {
+                if (mask_now && ok && i > 0) ok = wait_bar(bar(B_MK_EMPTY + t), (i - 1) & 1, abort);
+                if (warp == 0 && lane == 0) SCAN_TRACE(83 + 5 * i + 2 * t);
+                EpiIn e;
+                if (epi_now && ok) epi_load(i - 1, t, e);
+                if (t == 0 && i + 1 < hb_size && tid < Q) {  // next head's decays
+                    const int64_t vbase = ((b * H + hfirst + i + 1) * nc + c) * Q;
+                    cum_r = p.cumA[vbase + tid];
+                    dt_r = p.dt[vbase + tid];
+                }
+                if (mask_now && ok) {
+                    if (t == 0)
+                        build_mask<0>(tmem, sM0, cum2, dtv, stab, rinv0, qd, hf, lane);
+                    else
+                        build_mask<1>(tmem, sM1, cum2, dtv, stab, rinv1, qd, hf, lane);
+                    fence_smem_async();
+                    mbar_arrive(bar(B_MK_FULL + t));
+                    if (warp == 0 && lane == 0) SCAN_TRACE(84 + 5 * i + 2 * t);
+                }
+                if (epi_now && ok) ok = epi_finish(i - 1, t, e);
             }
         }
     }
@@ -437,6 +525,12 @@ cudaError_t launch_n(const FwdParams& p, cudaStream_t s) {
 }
 
 }  // namespace
+
+#ifdef SSD_TRACE
+extern "C" int ssd_scan_trace_copy(void* dst) {
+    return cudaMemcpyFromSymbol(dst, g_scan_trace, sizeof(g_scan_trace)) == cudaSuccess ? 0 : 1;
+}
+#endif
 
 bool chunk_scan_tc_supported(const FwdParams& p) {
     return p.headdim == PD && (p.dstate == 64 || p.dstate == 128) &&
