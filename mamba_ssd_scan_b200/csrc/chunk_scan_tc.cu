@@ -17,18 +17,21 @@
 // them at ~2^-11 relative rounding.  The CTA is warp-specialised and its roles
 // hand work to each other through mbarriers:
 //
-//   warps 0-7  "mask": per head and tile, read CB back, apply the causal decay
-//              mask and write Mk as a bf16 K-major operand to shared memory
-//              (one buffer per tile, refilled as soon as its MMA is done); two
-//              warps share each 32-row block, taking alternate column groups;
-//   warps 8-11 "epilogue": per head and tile, read the state and intra-chunk
-//              accumulators, add D x and store y (bf16);
-//   warp 12    "control": one lane issues every TMA load (C, B once; x and
+//   warps 0-7  "workers": per head and tile, read CB back, apply the causal
+//              decay mask (with D on the diagonal, so the MMA also forms D x)
+//              and write Mk as a bf16 K-major operand to shared memory (one
+//              buffer per tile, refilled as soon as its MMA is done); then
+//              drain the previous head's accumulators for the same tile
+//              (y = intra + exp(cumA) * state, bf16).  Two warps share each
+//              32-row block, taking alternate column groups and p halves;
+//   warp 8     "control": one lane issues every TMA load (C, B once; x and
 //              H_in per head) and every MMA (CB once; per head and tile the
-//              state term C_t H_in^T and Mk x).
+//              state term C_t H_in^T and Mk x);
+//   warp 9     "loader": stages each head's decays and D in shared memory
+//              (two buffers), so the workers never wait on a global load.
 //
-// so the tensor core, the mask arithmetic and the epilogue of different tiles
-// and heads run at the same time.  Decays are never formed as exp(cumA_l) /
+// The tensor core thus works on head i while the CUDA cores finish head i-1
+// and prepare the next tile.  Decays are never formed as exp(cumA_l) /
 // exp(cumA_j): below the 32x32 diagonal blocks the factor is split as
 // exp(cumA_l - cumA_r) * exp(cumA_r - cumA_j), r the first row of the 32-row
 // block (both factors <= 1), and only the diagonal blocks take one exp per
@@ -49,7 +52,7 @@ using namespace tc;
 
 constexpr int QMAX = 256;
 constexpr int PD = 64;
-constexpr int NTHREADS = 288;  // 8 worker warps, 1 control warp
+constexpr int NTHREADS = 320;  // 8 worker warps, 1 control warp, 1 loader warp
 constexpr int NMASK = 256;
 constexpr uint32_t CB0P = 0, CB1P = 64, CB1F = 128;
 __device__ __forceinline__ uint32_t st_col(int t) { return t == 0 ? 192u : 320u; }
@@ -69,9 +72,11 @@ struct ScanTile {
     static constexpr int X_BYTES = QMAX * 128;
     static constexpr int H_OFF = X_OFF + X_BYTES;
     static constexpr int H_BYTES = (NST / 64) * PD * 128;
-    static constexpr int CUM_OFF = H_OFF + H_BYTES;          // mask warps: log2e * cumA, dt
-    static constexpr int DT_OFF = CUM_OFF + QMAX * 4;
-    static constexpr int RINV_OFF = DT_OFF + QMAX * 4;       // per-row CB scale, 2 tiles
+    // per-head decays, two buffers filled by the loader warp:
+    // [log2e * cumA (QMAX) | dt (QMAX) | D, padding (4)] fp32
+    static constexpr int DEC_FLOATS = 2 * QMAX + 4;
+    static constexpr int DEC_OFF = H_OFF + H_BYTES;
+    static constexpr int RINV_OFF = DEC_OFF + 2 * DEC_FLOATS * 4;  // per-row CB scale, 2 tiles
     static constexpr int STAB_OFF = RINV_OFF + 2 * 128 * 4;  // 8 mask warps x QMAX
     static constexpr int BAR_OFF = STAB_OFF + 8 * QMAX * 4;
     static constexpr int SMEM = BAR_OFF + 32 * 8 + 1024;
@@ -107,7 +112,8 @@ __device__ unsigned long long g_scan_trace[8][256];
 enum : int {
     B_CB_LOAD = 0, B_CB_DONE, B_CB_PACKED, B_X_FULL, B_H_FULL, B_H_FREE, B_X_FREE,
     B_MK_FULL, B_MK_EMPTY = B_MK_FULL + 2, B_ACC_FULL = B_MK_EMPTY + 2,
-    B_ACC_EMPTY = B_ACC_FULL + 2, B_COUNT = B_ACC_EMPTY + 2
+    B_ACC_EMPTY = B_ACC_FULL + 2, B_DEC_FULL = B_ACC_EMPTY + 2, B_DEC_FREE = B_DEC_FULL + 2,
+    B_COUNT = B_DEC_FREE + 2
 };
 
 // Bounded wait that also gives up when another role has aborted.  It spins on
@@ -141,10 +147,12 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
 // 1.  The warp's TMEM reads are issued together and waited for once; the
 // per-block decay table is filled while they are in flight.  cum2 holds
 // log2(e) * cumA, so every decay is one exp2; rinv undoes the row's CB scale.
+// The skip weight D is added to the diagonal (j = l), so the MMA also forms
+// D x and the epilogue needs no x.
 template <int TT>
 __device__ __forceinline__ void build_mask(uint32_t tmem, uint32_t mbase, const float* cum2,
-                                           const float* dtv, float* stab, float rinv, int qd,
-                                           int hf, int lane) {
+                                           const float* dtv, float* stab, float rinv, float Dh,
+                                           int qd, int hf, int lane) {
     constexpr int NG = 2 * (TT + 1);            // this warp's groups
     const int lb = 128 * TT + 32 * qd;          // chunk row of the block's first row
     const int l = lb + lane;
@@ -184,7 +192,7 @@ __device__ __forceinline__ void build_mask(uint32_t tmem, uint32_t mbase, const 
 #pragma unroll
                 for (int q = 0; q < 32; ++q) {
                     const float e = ex2(fminf(cl - cum2[j0 + q], 0.0f)) * dtv[j0 + q];
-                    const float m = v[q] * rinv * e;
+                    const float m = v[q] * rinv * e + (q == lane ? Dh : 0.0f);
                     v[q] = (q <= lane) ? m : 0.0f;
                 }
             }
@@ -231,8 +239,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int i = 0; i < B_COUNT; ++i) {
             uint32_t count = 1;
             if (i == B_CB_PACKED) count = 128;
-            if (i == B_MK_FULL || i == B_MK_FULL + 1 || i == B_ACC_EMPTY || i == B_ACC_EMPTY + 1)
+            if (i == B_MK_FULL || i == B_MK_FULL + 1 || i == B_ACC_EMPTY || i == B_ACC_EMPTY + 1 ||
+                i == B_DEC_FREE || i == B_DEC_FREE + 1)
                 count = NMASK;
+            if (i == B_DEC_FULL || i == B_DEC_FULL + 1) count = 32;
             mbar_init(bar(i), count);
         }
         *abort = 0;
@@ -341,11 +351,37 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             if (!ok) *abort = 1;
         }
+    } else if (warp == 9) {
+        // ------------------------------- loader ------------------------------
+        // Stages each head's decays (log2e * cumA, dt) and D into the two
+        // shared buffers, so the workers never wait on a global load.
+        bool ok = true;
+        for (int i = 0; ok && i < hb_size; ++i) {
+            const int bsel = i & 1;
+            if (i >= 2) ok = wait_bar(bar(B_DEC_FREE + bsel), ((i - 2) >> 1) & 1, abort);
+            if (!ok) break;
+            float* dec = reinterpret_cast<float*>(smem + T::DEC_OFF) + bsel * T::DEC_FLOATS;
+            const int64_t h = hfirst + i;
+            const int64_t vbase = ((b * H + h) * nc + c) * Q;
+            float cv[QMAX / 32], dv[QMAX / 32];
+#pragma unroll
+            for (int k = 0; k < QMAX / 32; ++k) {
+                const int j = lane + 32 * k;
+                cv[k] = j < Q ? p.cumA[vbase + j] : 0.0f;
+                dv[k] = j < Q ? p.dt[vbase + j] : 0.0f;
+            }
+#pragma unroll
+            for (int k = 0; k < QMAX / 32; ++k) {
+                dec[lane + 32 * k] = cv[k] * 1.4426950408889634f;
+                dec[QMAX + lane + 32 * k] = dv[k];
+            }
+            if (lane == 0) dec[2 * QMAX] = p.D ? p.D[h] : 0.0f;
+            mbar_arrive(bar(B_DEC_FULL + bsel));
+        }
+        if (!ok) *abort = 1;
     } else {
         // ------------------------------ workers ------------------------------
         const int qd = warp & 3, hf = warp >> 2;
-        float* cum2 = reinterpret_cast<float*>(smem + T::CUM_OFF);
-        float* dtv = reinterpret_cast<float*>(smem + T::DT_OFF);
         float* rinv_s = reinterpret_cast<float*>(smem + T::RINV_OFF);
         float* stab = reinterpret_cast<float*>(smem + T::STAB_OFF) + warp * QMAX;
         const uint32_t lanes = static_cast<uint32_t>(32 * qd) << 16;
@@ -386,31 +422,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const float rinv0 = ok ? rinv_s[32 * qd + lane] : 1.0f;
         const float rinv1 = (ok && ntiles == 2) ? rinv_s[128 + 32 * qd + lane] : 1.0f;
 
-        // The epilogue of head i, tile t, for this warp's rows and 32 p columns, in
-        // two halves: its global loads (x for the D skip, exp(cumA) of the row, D)
-        // are issued before the tile's mask is built, so that they have landed
-        // by the time this thread waits on an mbarrier again (an acquire wait
-        // also waits for the thread's outstanding loads).
-        struct EpiIn {
-            uint4 xv[4];
-            float sc, D;
-            int64_t rowoff;
-            bool valid;
-        };
-        auto epi_load = [&](int i, int t, EpiIn& e) {
+        // The epilogue of head i, tile t, for this warp's rows and 32 p columns.
+        // D x came through the mask diagonal and log2e * cumA of the row was kept
+        // from the mask phase, so nothing here waits on a global load.
+        auto epilogue = [&](int i, int t, float cl2) -> bool {
             const int64_t h = hfirst + i;
             const int l = 128 * t + 32 * qd + lane;
-            e.valid = l < Lc;
-            const int64_t vbase = ((b * H + h) * nc + c) * Q;
-            e.sc = e.valid ? p.cumA[vbase + l] : 0.0f;
-            e.D = p.D ? p.D[h] : 0.0f;
-            e.rowoff = ((b * L + t0 + l) * H + h) * PD + 32 * hf;
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-                e.xv[k] = e.valid ? ldg16(static_cast<const __nv_bfloat16*>(p.x) + e.rowoff + 8 * k)
-                                  : make_uint4(0u, 0u, 0u, 0u);
-        };
-        auto epi_finish = [&](int i, int t, const EpiIn& e) -> bool {
             if (!wait_bar(bar(B_ACC_FULL + t), i & 1, abort)) return false;
             if (warp == 0 && lane == 0) SCAN_TRACE(140 + 4 * i + 2 * t);
             fence_after_sync();
@@ -418,20 +435,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             tmem_ld32x2(tmem + lanes + in_col(t) + 32 * hf, vi, tmem + lanes + st_col(t) + 32 * hf, vs);
             fence_before_sync();
             mbar_arrive(bar(B_ACC_EMPTY + t));
-            if (e.valid) {
-                const float sc = ex2(e.sc * 1.4426950408889634f);
-                __nv_bfloat16* yr = static_cast<__nv_bfloat16*>(p.y) + e.rowoff;
+            if (l < Lc) {
+                const float sc = ex2(cl2);
+                __nv_bfloat16* yr = static_cast<__nv_bfloat16*>(p.y) +
+                                    ((b * L + t0 + l) * H + h) * PD + 32 * hf;
 #pragma unroll
                 for (int k4 = 0; k4 < 4; ++k4) {
-                    const uint32_t xw[4] = {e.xv[k4].x, e.xv[k4].y, e.xv[k4].z, e.xv[k4].w};
                     uint32_t o[4];
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
-                        const float2 xf =
-                            __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xw[k]));
-                        const int q = 8 * k4 + 2 * k;
-                        o[k] = pack_bf16x2(vi[q] + sc * vs[q] + e.D * xf.x,
-                                           vi[q + 1] + sc * vs[q + 1] + e.D * xf.y);
+                        const int e = 8 * k4 + 2 * k;
+                        o[k] = pack_bf16x2(fmaf(sc, vs[e], vi[e]), fmaf(sc, vs[e + 1], vi[e + 1]));
                     }
                     reinterpret_cast<uint4*>(yr)[k4] = make_uint4(o[0], o[1], o[2], o[3]);
                 }
@@ -440,48 +454,44 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             return true;
         };
 
-        // this head's decays travel in registers one head ahead (256 worker
-        // threads, one entry each)
-        float cum_r = 0.0f, dt_r = 0.0f;
-        if (tid < Q) {
-            const int64_t vbase = ((b * H + hfirst) * nc + c) * Q;
-            cum_r = p.cumA[vbase + tid];
-            dt_r = p.dt[vbase + tid];
-        }
-        // Every worker runs every iteration and reaches both named barriers even
-        // after a failed wait (the work is skipped), so no worker is left waiting
-        // at a barrier another one has abandoned.  Iteration i builds head i's
-        // masks and drains head i-1's accumulators, tile by tile.
+        // Iteration i builds head i's masks and drains head i-1's accumulators,
+        // tile by tile, so the tensor core works on one head while the CUDA cores
+        // finish the previous one.
+        float cl_prev[2] = {0.0f, 0.0f};
         for (int i = 0; i <= hb_size; ++i) {
             const bool mask_now = i < hb_size, epi_now = i > 0;
-            if (mask_now) {
-                named_sync(1, NMASK);  // every worker is done with the previous head's decays
-                cum2[tid] = cum_r * 1.4426950408889634f;
-                dtv[tid] = dt_r;
-                named_sync(1, NMASK);
+            const int bsel = i & 1;
+            const float* dec = reinterpret_cast<const float*>(smem + T::DEC_OFF) + bsel * T::DEC_FLOATS;
+            float cl_cur[2] = {0.0f, 0.0f};
+            float Dh = 0.0f;
+            if (mask_now && ok) {
+                ok = wait_bar(bar(B_DEC_FULL + bsel), (i >> 1) & 1, abort);
                 if (warp == 0 && lane == 0) SCAN_TRACE(82 + 5 * i);
+                if (ok) {
+                    cl_cur[0] = dec[32 * qd + lane];
+                    cl_cur[1] = dec[128 + 32 * qd + lane];
+                    Dh = dec[2 * QMAX];
+                }
             }
             for (int t = 0; t < ntiles; ++t) {
-                if (mask_now && ok && i > 0) ok = wait_bar(bar(B_MK_EMPTY + t), (i - 1) & 1, abort);
-                if (warp == 0 && lane == 0) SCAN_TRACE(83 + 5 * i + 2 * t);
-                EpiIn e;
-                if (epi_now && ok) epi_load(i - 1, t, e);
-                if (t == 0 && i + 1 < hb_size && tid < Q) {  // next head's decays
-                    const int64_t vbase = ((b * H + hfirst + i + 1) * nc + c) * Q;
-                    cum_r = p.cumA[vbase + tid];
-                    dt_r = p.dt[vbase + tid];
-                }
                 if (mask_now && ok) {
-                    if (t == 0)
-                        build_mask<0>(tmem, sM0, cum2, dtv, stab, rinv0, qd, hf, lane);
-                    else
-                        build_mask<1>(tmem, sM1, cum2, dtv, stab, rinv1, qd, hf, lane);
-                    fence_smem_async();
-                    mbar_arrive(bar(B_MK_FULL + t));
+                    if (i > 0) ok = wait_bar(bar(B_MK_EMPTY + t), (i - 1) & 1, abort);
+                    if (warp == 0 && lane == 0) SCAN_TRACE(83 + 5 * i + 2 * t);
+                    if (ok) {
+                        if (t == 0)
+                            build_mask<0>(tmem, sM0, dec, dec + QMAX, stab, rinv0, Dh, qd, hf, lane);
+                        else
+                            build_mask<1>(tmem, sM1, dec, dec + QMAX, stab, rinv1, Dh, qd, hf, lane);
+                        fence_smem_async();
+                        mbar_arrive(bar(B_MK_FULL + t));
+                    }
                     if (warp == 0 && lane == 0) SCAN_TRACE(84 + 5 * i + 2 * t);
                 }
-                if (epi_now && ok) ok = epi_finish(i - 1, t, e);
+                if (epi_now && ok) ok = epilogue(i - 1, t, cl_prev[t]);
             }
+            if (mask_now && ok) mbar_arrive(bar(B_DEC_FREE + bsel));  // this head's decays are used
+            cl_prev[0] = cl_cur[0];
+            cl_prev[1] = cl_cur[1];
         }
     }
     fence_before_sync();
