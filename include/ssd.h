@@ -116,6 +116,30 @@ int ssd_fwd_tensor_core_steps(const ssd_fwd_args* args);
  * another call in flight. */
 ssd_status ssd_fwd(const ssd_fwd_args* args, void* stream);
 
+/* ssd_fwd for callers that cannot allocate device memory (there is no
+ * counterpart on the pages: this is a deployment variant).  Some callers only
+ * hold the input and output buffers their host application hands them --
+ * plugins and runtime extensions with no access to an allocator, or
+ * latency-critical code that must not risk a cudaMalloc's device-wide
+ * synchronisation.  This entry point ignores args->workspace and
+ * args->workspace_bytes and takes the scratch from a buffer of
+ * SSD_NO_ALLOC_SCRATCH_BYTES compiled into the library (every GPU that loads
+ * the library holds it until the process exits).  It calls no cudaMalloc,
+ * cudaFree or other allocating routine.
+ *   - Sizes whose ssd_fwd_workspace_size() exceeds the buffer are rejected
+ *     with SSD_ERR_UNSUPPORTED before anything is launched.
+ *   - The first call on each device looks up the buffer's device address
+ *     (cudaGetSymbolAddress, that device current) and caches it; make that
+ *     first call before any stream capture on the device.
+ *   - All calls share the one buffer: calls that can overlap on the GPU (on
+ *     different streams without ordering between them, or from different host
+ *     threads) race and give wrong results; serialise them.  The buffer keeps
+ *     the last call's contents; every call writes each scratch entry before it
+ *     reads it, so nothing needs clearing between calls.
+ * Everything else (arguments, layouts, errors, asynchrony) is as ssd_fwd. */
+#define SSD_NO_ALLOC_SCRATCH_BYTES (16u << 20)
+ssd_status ssd_fwd_no_alloc(const ssd_fwd_args* args, void* stream);
+
 /* Synchronises `stream` and returns the device status of the last ssd_fwd
  * call that used this workspace: SSD_OK, or SSD_ERR_TIMEOUT when a kernel gave
  * up on a bounded wait (it then stops early and its outputs are invalid).

@@ -15,7 +15,7 @@ import os
 import torch
 
 __all__ = [
-    "SsdError", "ssd_fwd", "ssd_fwd_workspace_size", "ssd_fwd_check_status",
+    "SsdError", "ssd_fwd", "ssd_fwd_workspace_size", "ssd_fwd_check_status", "ssd_fwd_no_alloc",
     "ssd_fwd_tensor_core_steps", "tensor_core_steps", "ssd_chunk_cumsum", "ssd_chunk_state",
     "ssd_state_passing", "ssd_chunk_scan", "ssd_state_update", "ssd_status_string",
     "ssd_version", "lib_path", "load_library", "SSD_FLAG_CUDA_CORES", "SSD_FLAG_WHOLE_GROUPS",
@@ -80,6 +80,8 @@ def load_library():
     lib.ssd_fwd.argtypes = [F, _vp]
     lib.ssd_fwd_tensor_core_steps.restype = ctypes.c_int
     lib.ssd_fwd_tensor_core_steps.argtypes = [F]
+    lib.ssd_fwd_no_alloc.restype = ctypes.c_int
+    lib.ssd_fwd_no_alloc.argtypes = [F, _vp]
     lib.ssd_fwd_check_status.restype = ctypes.c_int
     lib.ssd_fwd_check_status.argtypes = [F, _vp]
     lib.ssd_chunk_cumsum.restype = ctypes.c_int
@@ -208,6 +210,26 @@ def ssd_fwd(x, dt, A, B, C, D=None, dt_bias=None, chunk: int = 256, init_state=N
     _check(lib.ssd_fwd(ctypes.byref(a), _stream_ptr(stream)), "ssd_fwd")
     if final_state is not None:
         return y, final_state
+    return y
+
+
+SSD_NO_ALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def ssd_fwd_no_alloc(x, dt, A, B, C, D=None, dt_bias=None, chunk: int = 256, init_state=None,
+                     *, y, final_state=None, flags: int = 0, stream=None):
+    """ssd_fwd without a workspace, for callers that cannot allocate: the
+    scratch comes from a fixed buffer inside the library (see ssd_fwd_no_alloc
+    in include/ssd.h).  ``y`` (and ``final_state``, if wanted) are caller-owned
+    outputs; calls that can overlap on the GPU race and must be serialised."""
+    lib = load_library()
+    a = _fwd_args(x, dt, A, B, C, D, dt_bias, chunk, init_state, y, final_state, flags)
+    need = int(lib.ssd_fwd_workspace_size(ctypes.byref(a)))
+    if need > SSD_NO_ALLOC_SCRATCH_BYTES:
+        raise SsdError(SSD_ERR_UNSUPPORTED,
+                       f"ssd_fwd_no_alloc: these sizes need {need} bytes of scratch, more than "
+                       f"the built-in {SSD_NO_ALLOC_SCRATCH_BYTES}")
+    _check(lib.ssd_fwd_no_alloc(ctypes.byref(a), _stream_ptr(stream)), "ssd_fwd_no_alloc")
     return y
 
 
