@@ -41,6 +41,8 @@
 // TMEM columns: [0,64) tile 0's CB and [64,192) tile 1's CB as packed fp16
 // pairs (tile 1's fp32 CB sits in [128,384) until packed); [192,256)/[256,320)
 // tile 0's state/intra accumulators; [320,384)/[384,448) tile 1's.
+#include <stdlib.h>
+
 #include "internal.cuh"
 #include "tcgen05.cuh"
 #include "tma.cuh"
@@ -503,15 +505,45 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
 }
 
-// heads per CTA: the largest divisor of the heads per group that still leaves
-// at least two CTAs per SM of work (or every head of the group, when asked)
-int heads_per_cta(const FwdParams& p) {
+// Heads per CTA: each CTA pays a fixed set-up (C and B loads, CB, its repack)
+// and then pipelines its heads, so with w waves of CTAs over the SMs the
+// kernel takes about w * (setup + heads * per_head).  The divisor of the heads
+// per group that minimises this, up to 12 heads, is used (or every head of the
+// group, when asked).  The two costs are the measured ones (about 5 and 4.5
+// us); beyond about a dozen heads per CTA the measured time rises again.
+int heads_per_cta(const FwdParams& p, int num_sms) {
     if (p.flags & SSD_FLAG_WHOLE_GROUPS) return static_cast<int>(p.heads_per_group);
+    // tuning override: SSD_SCAN_HEADS_PER_CTA=d (used when d divides the heads per group)
+    static const int forced = [] {
+        const char* e = getenv("SSD_SCAN_HEADS_PER_CTA");
+        return e ? atoi(e) : 0;
+    }();
+    if (forced > 0 && p.heads_per_group % forced == 0) return forced;
     const int64_t units = p.batch * p.nchunks * p.ngroups;
+    const double setup = 5.0, per_head = 4.5;
     int best = 1;
-    for (int d = 1; d <= p.heads_per_group; ++d)
-        if (p.heads_per_group % d == 0 && units * (p.heads_per_group / d) >= 2 * 148) best = d;
+    double best_t = 0.0;
+    for (int d = 1; d <= p.heads_per_group && d <= 12; ++d) {
+        if (p.heads_per_group % d) continue;
+        const int64_t ctas = units * (p.heads_per_group / d);
+        const int64_t waves = (ctas + num_sms - 1) / num_sms;
+        const double t = static_cast<double>(waves) * (setup + per_head * d);
+        if (d == 1 || t < best_t) {
+            best = d;
+            best_t = t;
+        }
+    }
     return best;
+}
+
+int sm_count() {
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+        cudaGetLastError();
+        n = 148;
+    }
+    return n;
 }
 
 template <int NST>
@@ -527,7 +559,7 @@ cudaError_t launch_n(const FwdParams& p, cudaStream_t s) {
     auto kern = chunk_scan_tc_kernel<NST>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, T::SMEM);
     if (e != cudaSuccess) return e;
-    const int hb = heads_per_cta(p);
+    const int hb = heads_per_cta(p, sm_count());
     dim3 grid(static_cast<unsigned>(p.nchunks * p.ngroups * (p.heads_per_group / hb)),
               static_cast<unsigned>(p.batch));
     kern<<<grid, NTHREADS, T::SMEM, s>>>(p, tc_, tb_, tx_, th_, hb);
