@@ -158,6 +158,37 @@ def algorithmic_cost(cfg, elt):
     }
 
 
+# ---------------------------------------------------------------------------
+# multi-rank plumbing (weak scaling: every rank runs its own independent batch)
+def rank_env():
+    """(rank, world size, local rank) from the torchrun environment."""
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def rank_seed(base: int, rank: int) -> int:
+    """Each rank draws its own batch (independent problems, no data-path
+    collective)."""
+    return base + 1000 * rank
+
+
+def max_over_ranks(v: float, world: int, device) -> float:
+    """The step time of the job: the slowest rank's."""
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank: float, world: int, ms_max: float) -> float:
+    """Whole-job units per second: all ranks' units over the slowest rank's
+    time."""
+    return world * units_per_rank / (ms_max * 1e-3)
+
+
 def main_ours(args):
     import torch
     import torch.distributed as dist
@@ -165,9 +196,7 @@ def main_ours(args):
     import mamba_ssd_scan_b200 as ssd
     from mamba_ssd_scan_b200 import synthetic
 
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, world, local = rank_env()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
@@ -179,17 +208,13 @@ def main_ours(args):
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def ranks_max(v: float) -> float:
+        return max_over_ranks(v, world, dev)
 
     ssd.load_library()
     peaks = load_peaks()
     cfg = synthetic.FWD_CONFIGS[args.workload]
-    seed = 1234 + synthetic.SEED_OFFSET[cfg.name] + 1000 * rank
+    seed = rank_seed(1234 + synthetic.SEED_OFFSET[cfg.name], rank)
     inp = synthetic.make_config_inputs(cfg, seed)
     d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
     elt = d["x"].element_size()
@@ -229,9 +254,9 @@ def main_ours(args):
         torch.cuda.synchronize()
         barrier()
     ms = sum(a.elapsed_time(b) for a, b in ev) / args.steps
-    ms = max_over_ranks(ms)
+    ms = ranks_max(ms)
     tokens = cfg.tokens
-    value = world * tokens / (ms * 1e-3)
+    value = job_throughput(tokens, world, ms)
     launches_per_step = 4
 
     # ---- per-kernel durations over the same kind of timed steps ---------
@@ -301,15 +326,15 @@ def main_ours(args):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        ems = max_over_ranks(e0.elapsed_time(e1) / args.steps)
-        e2e = {"value": world * tokens / (ems * 1e-3), "unit": "tokens/s",
+        ems = ranks_max(e0.elapsed_time(e1) / args.steps)
+        e2e = {"value": job_throughput(tokens, world, ems), "unit": "tokens/s",
                "ms_per_step": ems, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     # ---- other workloads (rank-local, reported for context) --------------
     extra = {}
     if not args.no_extra:
         extra = other_workloads(ssd, synthetic, dev, flush, peaks, rank, world,
-                                barrier, max_over_ranks)
+                                barrier, ranks_max)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -350,6 +375,33 @@ def main_ours(args):
         dist.destroy_process_group()
 
 
+KERNEL_SOURCES = {
+    "chunk_scan": ["chunk_scan_tc.cu", "tcgen05.cuh", "tma.cuh", "internal.cuh"],
+    "chunk_state": ["chunk_state_tc.cu", "tcgen05.cuh", "tma.cuh", "internal.cuh"],
+}
+
+
+def measured_traffic(kernel: str):
+    """DRAM bytes per launch of `kernel` from profiles/dram_traffic.md, or None
+    when it was not measured or its source has changed since."""
+    import hashlib
+    srcs = KERNEL_SOURCES.get(kernel)
+    path = os.path.join(ROOT, "profiles", "dram_traffic.md")
+    if not srcs or not os.path.exists(path):
+        return None
+    h = hashlib.sha256()
+    for f in srcs:
+        with open(os.path.join(ROOT, "mamba_ssd_scan_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    digest = h.hexdigest()[:16]
+    with open(path) as fh:
+        for line in fh:
+            cells = [c.strip() for c in line.strip().strip("|").split("|")]
+            if len(cells) >= 4 and cells[0] == kernel and cells[1] == digest:
+                return int(cells[2]) + int(cells[3])
+    return None
+
+
 def roofline_entry(name, cost, ms, peaks, clk, on_tensor_cores):
     """Roofline position of one kernel: the larger of its HBM time (algorithmic
     bytes / measured copy bandwidth) and its compute time (algorithmic FLOP /
@@ -376,18 +428,18 @@ def roofline_entry(name, cost, ms, peaks, clk, on_tensor_cores):
                 "algorithmic_bytes": nbytes, "algorithmic_flops": flops}
     ach = nbytes / sec / 1e9
     return {"kernel": name, "bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s",
-            "frac": ach / hbm, "traffic": None, "peak_note": f"copy bandwidth, {src}",
+            "frac": ach / hbm, "traffic": measured_traffic(name), "peak_note": f"copy bandwidth, {src}",
             "algorithmic_bytes": nbytes, "algorithmic_flops": flops,
             "compute_frac": (flops / sec / 1e12) / cpeak if flops else 0.0}
 
 
-def other_workloads(ssd, synthetic, dev, flush, peaks, rank, world, barrier, max_over_ranks):
+def other_workloads(ssd, synthetic, dev, flush, peaks, rank, world, barrier, ranks_max):
     import torch
     out = {}
     stream = torch.cuda.current_stream()
     for name, steps in (("fwd_bf16_b8_L4096_init", 10), ("fwd_bf16_b1_L65536_G8", 5)):
         cfg = synthetic.FWD_CONFIGS[name]
-        inp = synthetic.make_config_inputs(cfg, 1234 + synthetic.SEED_OFFSET[name] + 1000 * rank)
+        inp = synthetic.make_config_inputs(cfg, rank_seed(1234 + synthetic.SEED_OFFSET[name], rank))
         d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
         del inp
         y = torch.empty_like(d["x"])
@@ -414,10 +466,10 @@ def other_workloads(ssd, synthetic, dev, flush, peaks, rank, world, barrier, max
             b_.record(stream)
             torch.cuda.synchronize()
             tot += a.elapsed_time(b_)
-        ms = max_over_ranks(tot / steps)
+        ms = ranks_max(tot / steps)
         nbytes = algorithmic_cost(cfg, 2)["path"][0]
         kms = split_kernel_ms(ssd, cfg, d, y, fin, dev, flush, steps)
-        out[name] = {"tokens_per_s": world * cfg.tokens / (ms * 1e-3), "ms": ms,
+        out[name] = {"tokens_per_s": job_throughput(cfg.tokens, world, ms), "ms": ms,
                      "hbm_frac_of_path_bytes": nbytes / (ms * 1e-3) / (peaks["hbm_gbs"] * 1e9),
                      "kernel_ms": kms}
         del d, y, fin, ws
@@ -425,7 +477,7 @@ def other_workloads(ssd, synthetic, dev, flush, peaks, rank, world, barrier, max
 
     # decode: 1024 successive steps captured in one CUDA graph
     cfg = synthetic.DECODE_CONFIGS["decode_b256_H80"]
-    seed = 1234 + synthetic.SEED_OFFSET[cfg.name] + 1000 * rank
+    seed = rank_seed(1234 + synthetic.SEED_OFFSET[cfg.name], rank)
     prm = synthetic.make_decode_params(cfg.batch, cfg.nheads, cfg.headdim, cfg.dstate, seed)
     state = prm["state"].to(dev)
     A, D, bias = prm["A"].to(dev), prm["D"].to(dev), prm["dt_bias"].to(dev)
@@ -456,7 +508,7 @@ def other_workloads(ssd, synthetic, dev, flush, peaks, rank, world, barrier, max
     g.replay()
     b_.record(stream)
     torch.cuda.synchronize()
-    us = max_over_ranks(a.elapsed_time(b_) * 1e3 / cfg.steps)
+    us = ranks_max(a.elapsed_time(b_) * 1e3 / cfg.steps)
     sbytes = cfg.batch * cfg.nheads * cfg.headdim * cfg.dstate * 4
     step_bytes = 2 * sbytes + cfg.batch * (2 * cfg.nheads * cfg.headdim + cfg.nheads +
                                            2 * cfg.ngroups * cfg.dstate) * 2

@@ -118,13 +118,17 @@ enum : int {
     B_COUNT = B_DEC_FREE + 2
 };
 
-// Bounded wait that also gives up when another role has aborted.  It spins on
-// the non-blocking probe: a suspending try_wait wakes up late (~1 us), which
-// on the hand-offs of this pipeline costs more than the spin.
+// Bounded wait that also gives up when another role has aborted: a few
+// non-blocking probes first (most hand-offs are already complete), then
+// probes that may suspend the thread for a short, bounded time, so a waiting
+// warp gives its issue slots to the worker sharing its scheduler without the
+// late wake-up of an unbounded suspend.
 __device__ __forceinline__ bool wait_bar(uint32_t mbar, uint32_t parity, volatile int* abort) {
-    for (uint32_t i = 0; i < 4 * kSpinLimit; ++i) {
+    for (int i = 0; i < 8; ++i)
         if (mbar_test_wait(mbar, parity)) return true;
-        if ((i & 255) == 255 && *abort) return false;
+    for (uint32_t i = 0; i < kSpinLimit; ++i) {
+        if (mbar_try_wait_hint(mbar, parity, 100)) return true;
+        if ((i & 63) == 63 && *abort) return false;
     }
     *abort = 1;
     return false;

@@ -97,6 +97,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t mbar, uint32_t parity) {
     return ok != 0;
 }
 
+// Like mbar_try_wait, with a hint (ns) of how long the thread may be suspended
+// before the probe returns.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint32_t mbar, uint32_t parity, uint32_t ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(mbar), "r"(parity), "r"(ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Non-blocking probe of the same condition (never suspends the thread).
 __device__ __forceinline__ bool mbar_test_wait(uint32_t mbar, uint32_t parity) {
     uint32_t ok;
