@@ -267,7 +267,10 @@ def main_ours(args):
     ms = ranks_max(ms)
     tokens = cfg.tokens
     value = job_throughput(tokens, world, ms)
-    launches_per_step = 4
+    tc = ssd.tensor_core_steps(cfg.batch, cfg.seqlen, cfg.nheads, cfg.headdim, cfg.dstate,
+                               cfg.ngroups, cfg.chunk, cfg.dtype)
+    # ssd_fwd folds step 1 into the tensor-core chunk_state
+    launches_per_step = 3 if "chunk_state" in tc else 4
 
     # ---- per-kernel durations over the same kind of timed steps ---------
     nc = -(-cfg.seqlen // cfg.chunk)
@@ -307,10 +310,8 @@ def main_ours(args):
            for i, n in enumerate(names)}
     cost = algorithmic_cost(cfg, elt)
     top = max(names, key=lambda n: kms[n])
-    tc = ssd.tensor_core_steps(cfg.batch, cfg.seqlen, cfg.nheads, cfg.headdim, cfg.dstate,
-                               cfg.ngroups, cfg.chunk, cfg.dtype)
     roofline = roofline_entry(top, cost[top], kms[top], peaks, clocks.summary(),
-                              top in tc)
+                              top in tc, cfg.name)
 
     # ---- e2e through the public API from pinned host buffers ------------
     e2e = None
@@ -392,9 +393,10 @@ KERNEL_SOURCES = {
 }
 
 
-def measured_traffic(kernel: str):
-    """DRAM bytes per launch of `kernel` from profiles/dram_traffic.md, or None
-    when it was not measured or its source has changed since."""
+def measured_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` on `workload` from
+    profiles/dram_traffic.md, or None when that pair was not measured or the
+    kernel's source has changed since."""
     import hashlib
     srcs = KERNEL_SOURCES.get(kernel)
     path = os.path.join(ROOT, "profiles", "dram_traffic.md")
@@ -408,12 +410,13 @@ def measured_traffic(kernel: str):
     with open(path) as fh:
         for line in fh:
             cells = [c.strip() for c in line.strip().strip("|").split("|")]
-            if len(cells) >= 4 and cells[0] == kernel and cells[1] == digest:
-                return int(cells[2]) + int(cells[3])
+            if (len(cells) >= 5 and cells[0] == workload and cells[1] == kernel
+                    and cells[2] == digest):
+                return int(cells[3]) + int(cells[4])
     return None
 
 
-def roofline_entry(name, cost, ms, peaks, clk, on_tensor_cores):
+def roofline_entry(name, cost, ms, peaks, clk, on_tensor_cores, workload):
     """Roofline position of one kernel: the larger of its HBM time (algorithmic
     bytes / measured copy bandwidth) and its compute time (algorithmic FLOP /
     the peak of the unit that executes them) names the bound."""
@@ -439,7 +442,7 @@ def roofline_entry(name, cost, ms, peaks, clk, on_tensor_cores):
                 "algorithmic_bytes": nbytes, "algorithmic_flops": flops}
     ach = nbytes / sec / 1e9
     return {"kernel": name, "bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s",
-            "frac": ach / hbm, "traffic": measured_traffic(name), "peak_note": f"copy bandwidth, {src}",
+            "frac": ach / hbm, "traffic": measured_traffic(name, workload), "peak_note": f"copy bandwidth, {src}",
             "algorithmic_bytes": nbytes, "algorithmic_flops": flops,
             "compute_frac": (flops / sec / 1e12) / cpeak if flops else 0.0}
 

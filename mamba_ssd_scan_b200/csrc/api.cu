@@ -96,6 +96,8 @@ FwdParams make_params(const ssd_fwd_args* a) {
     p.nchunks = (a->seqlen + a->chunk - 1) / a->chunk;
     p.heads_per_group = a->nheads / a->ngroups;
     p.flags = a->flags;
+    p.pdl = 0;
+    p.fuse_cumsum = 0;
     p.x = a->x;
     p.dt_raw = a->dt;
     p.A = a->A;
@@ -179,8 +181,21 @@ ssd_status ssd_fwd(const ssd_fwd_args* a, void* stream) {
     p.states = ws + w.states;
     p.status = reinterpret_cast<int*>(ws + w.status);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = run_cumsum(p, a->dtype, s);
+    // The first kernel is a plain launch (it waits for all earlier work on
+    // the stream); the later ones go out with programmatic dependent launch,
+    // so their set-up overlaps the previous kernel's tail.  The tensor-core
+    // chunk_state forms dt and cumA itself, which saves step 1's launch.
+    cudaError_t e = cudaSuccess;
+    const bool fused = use_tc(a->dtype, a->flags) && ssd::chunk_state_tc_supported(p);
+    if (!fused) {
+        e = run_cumsum(p, a->dtype, s);
+        p.pdl = 1;
+    } else {
+        p.fuse_cumsum = 1;
+    }
     if (e == cudaSuccess) e = run_chunk_state(p, a->dtype, a->flags, s);
+    p.pdl = 1;
+    p.fuse_cumsum = 0;
     if (e == cudaSuccess) e = run_state_passing(p, a->dtype, s);
     if (e == cudaSuccess) e = run_chunk_scan(p, a->dtype, a->flags, s);
     return to_status(e);

@@ -27,6 +27,7 @@ __host__ __device__ inline int64_t cs_stride(int64_t N) { return N + 4; }  // pa
 
 template <typename T>
 __global__ void __launch_bounds__(256) chunk_scan_ffma_kernel(FwdParams p) {
+    grid_dep_wait();  // dt, cumA and the carried states come from steps 1-3
     const int64_t H = p.nheads, P = p.headdim, N = p.dstate, G = p.ngroups;
     const int64_t L = p.seqlen, Q = p.chunk, nc = p.nchunks;
     const int64_t ntile_p = (P + TPP - 1) / TPP;
@@ -175,8 +176,7 @@ cudaError_t launch_chunk_scan_ffma(const FwdParams& p, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     const unsigned tiles = (unsigned)(((p.chunk + TL - 1) / TL) * ((p.headdim + TPP - 1) / TPP));
     dim3 grid((unsigned)(p.nchunks * p.nheads), tiles, (unsigned)p.batch);
-    chunk_scan_ffma_kernel<T><<<grid, 256, smem, s>>>(p);
-    return cudaGetLastError();
+    return launch_kernel(chunk_scan_ffma_kernel<T>, grid, dim3(256), smem, s, p.pdl != 0, p);
 }
 
 template cudaError_t launch_chunk_scan_ffma<float>(const FwdParams&, cudaStream_t);

@@ -17,30 +17,45 @@
 // them at ~2^-11 relative rounding.  The CTA is warp-specialised and its roles
 // hand work to each other through mbarriers:
 //
-//   warps 0-7  "workers": per head and tile, read CB back, apply the causal
-//              decay mask (with D on the diagonal, so the MMA also forms D x)
-//              and write Mk as a bf16 K-major operand to shared memory (one
-//              buffer per tile, refilled as soon as its MMA is done); then
-//              drain the previous head's accumulators for the same tile
-//              (y = intra + exp(cumA) * state, bf16).  Two warps share each
-//              32-row block, taking alternate column groups and p halves;
-//   warp 8     "control": one lane issues every TMA load (C, B once; x and
+//   warps 0-15 "workers": per head and tile, read CB back, apply the causal
+//              decay mask below the diagonal and write Mk as a bf16 K-major
+//              operand to shared memory (one buffer per tile, refilled as soon
+//              as its MMA is done); then drain the previous head's accumulators
+//              for the same tile (y = f * intra + exp(cumA) * state, plus the
+//              diagonal term (C_l . B_l dt_l + D) x_l in fp32, bf16 out).  The
+//              four warps of a TMEM lane quarter share its 32 rows and take
+//              one column group in four (and a quarter of the p columns in
+//              the epilogue);
+//   warp 16    "control": one lane issues every TMA load (C, B once; x and
 //              H_in per head) and every MMA (CB once; per head and tile the
 //              state term C_t H_in^T and Mk x);
-//   warp 9     "loader": stages each head's decays and D in shared memory
-//              (two buffers), so the workers never wait on a global load.
+//   warp 17    "loader": stages each head's decays and D in shared memory
+//              (two buffers), so the mask phase never waits on a global load.
 //
-// The tensor core thus works on head i while the CUDA cores finish head i-1
-// and prepare the next tile.  Decays are never formed as exp(cumA_l) /
-// exp(cumA_j): below the 32x32 diagonal blocks the factor is split as
-// exp(cumA_l - cumA_r) * exp(cumA_r - cumA_j), r the first row of the 32-row
-// block (both factors <= 1), and only the diagonal blocks take one exp per
-// element.  Every wait is bounded; a timed-out role raises a shared abort flag
-// that the others observe, and the CTA still frees its TMEM.
+// Balance.  A warp only reaches the TMEM lanes of its quarter (warp % 4),
+// which is also the scheduler it issues on, and a causal row's work grows
+// with its index.  Tile 0's 32-row blocks are therefore stored in reverse
+// order (lane quarter q holds chunk rows 32 (3 - q) ...), so quarter q holds
+// row blocks 3 - q and 4 + q: nine column groups per quarter and head.
 //
-// TMEM columns: [0,64) tile 0's CB and [64,192) tile 1's CB as packed fp16
-// pairs (tile 1's fp32 CB sits in [128,384) until packed); [192,256)/[256,320)
-// tile 0's state/intra accumulators; [320,384)/[384,448) tile 1's.
+// Decay factors.  For the 32-row block starting at row lb, with a reference
+// value M inside the block's cumA range, exp(cumA_l - cumA_j) is split as
+// exp(cumA_l - M) * exp(M - cumA_j): the first factor goes to the epilogue
+// (one multiply per output element), the second is computed once per column
+// by one lane, so each mask element costs one multiply.  M is the midpoint of
+// the block's cumA range, so neither factor exceeds 2^(span / 2), span the
+// block's log2 decay; blocks whose span exceeds kFastSpan (where such factors
+// would leave fp32 or bf16 range) use M = cumA_lb and one exp2 per diagonal
+// element instead, which is exact for any decay.  Every wait is bounded; a
+// timed-out role raises a shared abort flag that the others observe, and the
+// CTA still frees its TMEM.
+//
+// TMEM columns: [0,64) tile 0's CB and [128,256) tile 1's CB as packed fp16
+// pairs (the fp32 CB sits in [0,128) and [256,512) until packed; the two tiles
+// are packed at the same time, so their source and destination columns never
+// overlap); [64,128) the workers' stash of the head's x rows (diagonal term);
+// [256,320)/[320,384) tile 0's state/intra accumulators, [384,448)/[448,512)
+// tile 1's.
 #include <stdlib.h>
 
 #include "internal.cuh"
@@ -54,11 +69,22 @@ using namespace tc;
 
 constexpr int QMAX = 256;
 constexpr int PD = 64;
-constexpr int NTHREADS = 320;  // 8 worker warps, 1 control warp, 1 loader warp
-constexpr int NMASK = 256;
-constexpr uint32_t CB0P = 0, CB1P = 64, CB1F = 128;
-__device__ __forceinline__ uint32_t st_col(int t) { return t == 0 ? 192u : 320u; }
-__device__ __forceinline__ uint32_t in_col(int t) { return t == 0 ? 256u : 384u; }
+constexpr int NWORK = 16;                        // worker warps
+constexpr int CTRL_WARP = NWORK, LOAD_WARP = NWORK + 1;
+constexpr int NTHREADS = (NWORK + 2) * 32;
+constexpr int NMASK = NWORK * 32;
+constexpr uint32_t CB0P = 0, CB1P = 128, CB1F = 256;
+// largest log2 decay span of a 32-row block that takes the factored path:
+// factors stay within 2^90, so masked entries (|CB| scaled below 2^15) and
+// their 256-term sums stay far inside fp32 and bf16 range
+constexpr float kFastSpan = 180.0f;
+constexpr float kMaxExp = 96.0f;
+__device__ __forceinline__ uint32_t st_col(int t) { return t == 0 ? 256u : 384u; }
+__device__ __forceinline__ uint32_t in_col(int t) { return t == 0 ? 320u : 448u; }
+// TMEM columns of worker hf's stash of tile t's x rows (16 bf16 per lane)
+__device__ __forceinline__ uint32_t stash_col(int t, int hf) { return 64u + 32u * t + 8u * hf; }
+// first chunk row of the 32-row block that TMEM lane quarter qd holds in tile t
+__device__ __forceinline__ int block_row(int t, int qd) { return t == 0 ? 32 * (3 - qd) : 128 + 32 * qd; }
 
 template <int NST>
 struct ScanTile {
@@ -79,34 +105,26 @@ struct ScanTile {
     static constexpr int DEC_FLOATS = 2 * QMAX + 4;
     static constexpr int DEC_OFF = H_OFF + H_BYTES;
     static constexpr int RINV_OFF = DEC_OFF + 2 * DEC_FLOATS * 4;  // per-row CB scale, 2 tiles
-    static constexpr int STAB_OFF = RINV_OFF + 2 * 128 * 4;  // 8 mask warps x QMAX
-    static constexpr int BAR_OFF = STAB_OFF + 8 * QMAX * 4;
+    static constexpr int CBD_OFF = RINV_OFF + 2 * 128 * 4;   // per-row C_l . B_l, 2 tiles
+    static constexpr int CTAB_OFF = CBD_OFF + 2 * 128 * 4;   // per worker warp: 32 column factors
+    static constexpr int BAR_OFF = CTAB_OFF + NWORK * 32 * 4;
     static constexpr int SMEM = BAR_OFF + 32 * 8 + 1024;
     static_assert(SMEM <= 232448, "shared memory budget");
 };
 
 // Optional timeline of the first CTAs (builds with -DSSD_TRACE only): each role
-// stamps the SM cycle counter at its hand-offs; ssd_scan_trace_copy() reads it
-// back.
+// stamps the SM cycle counter at its hand-offs into shared memory (a global
+// store before an mbarrier arrive would delay the arrive until the store is
+// acknowledged); the CTA copies the stamps out when it ends and
+// ssd_scan_trace_copy() reads them back.
 #ifdef SSD_TRACE
 __device__ unsigned long long g_scan_trace[8][256];
 #define SCAN_TRACE(slot)                                                              \
     do {                                                                              \
-        if (blockIdx.x < 8 && blockIdx.y == 0 && (slot) < 256) {                      \
-            g_scan_trace[blockIdx.x][(slot)] = clock64();                             \
-        }                                                                             \
-    } while (0)
-// SM-clock stamps of warp 0 inside the mask routine, head 1 only
-#define MASK_CLOCK(slot)                                                              \
-    do {                                                                              \
-        if (blockIdx.x < 8 && blockIdx.y == 0 && threadIdx.x == 0)                    \
-            g_scan_trace[blockIdx.x][(slot)] = clock64();                             \
+        if ((slot) < 256) s_trace[(slot)] = clock64();                                \
     } while (0)
 #else
 #define SCAN_TRACE(slot) \
-    do {                 \
-    } while (0)
-#define MASK_CLOCK(slot) \
     do {                 \
     } while (0)
 #endif
@@ -121,7 +139,7 @@ enum : int {
 // Bounded wait that also gives up when another role has aborted: a few
 // non-blocking probes first (most hand-offs are already complete), then
 // probes that may suspend the thread for a short, bounded time, so a waiting
-// warp gives its issue slots to the worker sharing its scheduler without the
+// warp gives its issue slots to the workers sharing its scheduler without the
 // late wake-up of an unbounded suspend.
 __device__ __forceinline__ bool wait_bar(uint32_t mbar, uint32_t parity, volatile int* abort) {
     for (int i = 0; i < 8; ++i)
@@ -148,68 +166,135 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
     return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-// Mask warp: rows 128 t + 32 qd + lane of tile t (qd = TMEM lane quarter),
-// column groups of 32 with index = hf (mod 2): 2 groups in tile 0, 4 in tile
-// 1.  The warp's TMEM reads are issued together and waited for once; the
-// per-block decay table is filled while they are in flight.  cum2 holds
-// log2(e) * cumA, so every decay is one exp2; rinv undoes the row's CB scale.
-// The skip weight D is added to the diagonal (j = l), so the MMA also forms
-// D x and the epilogue needs no x.
-template <int TT>
-__device__ __forceinline__ void build_mask(uint32_t tmem, uint32_t mbase, const float* cum2,
-                                           const float* dtv, float* stab, float rinv, float Dh,
-                                           int qd, int hf, int lane) {
-    constexpr int NG = 2 * (TT + 1);            // this warp's groups
-    const int lb = 128 * TT + 32 * qd;          // chunk row of the block's first row
-    const int l = lb + lane;
-    const uint32_t cbase = tmem + (static_cast<uint32_t>(32 * qd) << 16) + (TT == 0 ? CB0P : CB1P);
-    uint32_t addr[NG];
-    uint32_t raw[NG][16];
+// 32 masked values of one row -> bf16, into the K-major SW128 operand
+__device__ __forceinline__ void store_group(uint32_t mbase, uint32_t row, int j0, const float (&v)[32]) {
+    const uint32_t dst = mbase + (j0 >> 6) * (128 * 128);
+    const int c0 = (j0 & 63) >> 3;
 #pragma unroll
-    for (int k = 0; k < NG; ++k) addr[k] = cbase + 16 * (hf + 2 * k);   // j0 / 2
-    MASK_CLOCK(200 + 10 * TT);
-    if constexpr (NG == 2) tmem_ld16x2(addr, raw);
-    else tmem_ld16x4(addr, raw);
-    MASK_CLOCK(201 + 10 * TT);
-    const float cl = cum2[l];
-    for (int j = lane; j < lb; j += 32) stab[j] = ex2(cum2[lb] - cum2[j]) * dtv[j];
-    __syncwarp();
-    const float rl = ex2(cl - cum2[lb]) * rinv;
-    MASK_CLOCK(202 + 10 * TT);
+    for (int i = 0; i < 4; ++i)
+        st_shared_v4(dst + sw128(row, c0 + i), pack_bf16x2(v[8 * i + 0], v[8 * i + 1]),
+                     pack_bf16x2(v[8 * i + 2], v[8 * i + 3]), pack_bf16x2(v[8 * i + 4], v[8 * i + 5]),
+                     pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
+}
+
+__device__ __forceinline__ void store_zero_group(uint32_t mbase, uint32_t row, int j0) {
+    const uint32_t dst = mbase + (j0 >> 6) * (128 * 128);
+    const int c0 = (j0 & 63) >> 3;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) st_shared_v4(dst + sw128(row, c0 + i), 0u, 0u, 0u, 0u);
+}
+
+// Mask warp for tile TT: rows block_row(TT, qd) + lane (TMEM lane 32 qd + lane),
+// column groups hf + 4 k (k <= TT) of 32 columns.  Groups above the diagonal
+// block are zeros; they are written for the first head only (nothing else
+// writes there).  cum2 holds log2(e) * cumA, so every decay is one exp2.  The
+// diagonal entry (j = l, decay 1) is left out of the operand: the epilogue
+// adds (C_l . B_l dt_l + D) x_l in fp32, so the term that is often the row's
+// largest, and the D skip, are not rounded to bf16.  cbd is the row's C_l . B_l
+// (fp32, saved when CB was packed).  Returns the row's epilogue factor f
+// (y_intra = f * accumulator) in .x and that diagonal weight in .y.
+template <int TT>
+__device__ __forceinline__ float2 build_mask(uint32_t tmem, uint32_t mbase, const float* cum2,
+                                             const float* dtv, float* ctab, float rinv, float cbd,
+                                             float Dh, int qd, int hf, int lane, int Lc, bool first) {
+    constexpr int NG = TT + 1;
+    const int lb = block_row(TT, qd);
+    const int rb = lb >> 5;
+    const int l = lb + lane;
     const uint32_t row = 32 * qd + lane;
+    const uint32_t cbase = tmem + (static_cast<uint32_t>(32 * qd) << 16) + (TT == 0 ? CB0P : CB1P);
+
+    // the block's log2 decay span picks the path (warp-uniform)
+    const int last = max(lb, min(lb + 31, Lc - 1));
+    const float c_first = cum2[lb], c_last = cum2[last];
+    const bool fast = (c_first - c_last) <= kFastSpan;
+    const float ref = fast ? 0.5f * (c_first + c_last) : c_first;
+    const float cl = cum2[l];
+    const float f = fast ? rinv * ex2(cl - ref) : rinv;
+    const float w = fmaf(cbd, dtv[l], Dh);
+
 #pragma unroll
     for (int k = 0; k < NG; ++k) {
-        const int j0 = 32 * (hf + 2 * k);
-        const uint32_t dst = mbase + (j0 >> 6) * (128 * 128);
-        const int c0 = (j0 & 63) >> 3;
+        const int g = hf + 4 * k;
+        const int j0 = 32 * g;
+        if (g > rb) {  // above the diagonal block: zeros, kept from the first head
+            if (first) store_zero_group(mbase, row, j0);
+            continue;
+        }
+        uint32_t raw[16];
+        tmem_ld16(cbase + 16 * g, raw);
+        // this lane's column factor, shared with the warp through its table
+        const float cj = ex2(fminf(ref - cum2[j0 + lane], kMaxExp)) * dtv[j0 + lane];
+        __syncwarp();
+        ctab[lane] = cj;
+        __syncwarp();
+        const float4* ct = reinterpret_cast<const float4*>(ctab);
         float v[32];
-        if (j0 > lb) {  // above the diagonal: zeros
+        unpack_f16x32(raw, v);
+        if (g < rb) {  // below the diagonal block
+            if (fast) {
 #pragma unroll
-            for (int q = 0; q < 32; ++q) v[q] = 0.0f;
-        } else {
-            unpack_f16x32(raw[k], v);
-            if (j0 + 32 <= lb) {
-#pragma unroll
-                for (int q = 0; q < 32; ++q) v[q] *= rl * stab[j0 + q];
+                for (int i = 0; i < 8; ++i) {
+                    const float4 c = ct[i];
+                    v[4 * i + 0] *= c.x;
+                    v[4 * i + 1] *= c.y;
+                    v[4 * i + 2] *= c.z;
+                    v[4 * i + 3] *= c.w;
+                }
             } else {
-                // the diagonal block: one exp2 per element, computed for every
-                // lane (exponent clamped at 0, so the entries above the diagonal
-                // stay finite) and then selected -- no divergent branches
+                const float r = ex2(cl - c_first);
 #pragma unroll
-                for (int q = 0; q < 32; ++q) {
-                    const float e = ex2(fminf(cl - cum2[j0 + q], 0.0f)) * dtv[j0 + q];
-                    const float m = v[q] * rinv * e + (q == lane ? Dh : 0.0f);
-                    v[q] = (q <= lane) ? m : 0.0f;
+                for (int i = 0; i < 8; ++i) {
+                    const float4 c = ct[i];
+                    v[4 * i + 0] *= r * c.x;
+                    v[4 * i + 1] *= r * c.y;
+                    v[4 * i + 2] *= r * c.z;
+                    v[4 * i + 3] *= r * c.w;
                 }
             }
-        }
+        } else if (fast) {  // the diagonal block, factored; j = l left to the epilogue
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-            st_shared_v4(dst + sw128(row, c0 + i), pack_bf16x2(v[8 * i + 0], v[8 * i + 1]),
-                         pack_bf16x2(v[8 * i + 2], v[8 * i + 3]),
-                         pack_bf16x2(v[8 * i + 4], v[8 * i + 5]),
-                         pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
-        MASK_CLOCK(203 + 10 * TT + k);
+            for (int i = 0; i < 8; ++i) {
+                const float4 c = ct[i];
+                const float cc[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int q = 4 * i + e;
+                    v[q] = (q < lane) ? v[q] * cc[e] : 0.0f;
+                }
+            }
+        } else {  // the diagonal block of a steep block: one exp2 per element
+#pragma unroll
+            for (int q = 0; q < 32; ++q) {
+                const float e = ex2(fminf(cl - cum2[j0 + q], 0.0f)) * dtv[j0 + q];
+                v[q] = (q < lane) ? v[q] * e : 0.0f;
+            }
+        }
+        store_group(mbase, row, j0, v);
+    }
+    return make_float2(f, w);
+}
+
+// Per-head MMAs, issued by the control thread.  Descriptors are built once;
+// each K step only advances their start-address field (address / 16).
+// State term of one tile: C_t (K-major, NST wide) x H_in^T (K-major).
+template <int NST>
+__device__ __forceinline__ void issue_state(uint32_t d_tmem, uint64_t dA, uint64_t dB) {
+#pragma unroll
+    for (int k = 0; k < NST / 16; ++k) {
+        const uint32_t ka = ((k >> 2) * (QMAX * 128) + (k & 3) * 32) >> 4;
+        const uint32_t kb = ((k >> 2) * (PD * 128) + (k & 3) * 32) >> 4;
+        mma_bf16(d_tmem, dA + ka, dB + kb, idesc_bf16(128, PD, false, false), k > 0 ? 1u : 0u);
+    }
+}
+// Intra-chunk term of one tile: Mk_t (K-major, KS * 16 wide) x x (MN-major).
+template <int KS>
+__device__ __forceinline__ void issue_intra(uint32_t d_tmem, uint64_t dA, uint64_t dB) {
+#pragma unroll
+    for (int k = 0; k < KS; ++k) {
+        const uint32_t ka = ((k >> 2) * (128 * 128) + (k & 3) * 32) >> 4;
+        const uint32_t kb = (k * 2048) >> 4;
+        mma_bf16(d_tmem, dA + ka, dB + kb, idesc_bf16(128, PD, false, true), k > 0 ? 1u : 0u);
     }
 }
 
@@ -244,7 +329,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (tid == 0) {
         for (int i = 0; i < B_COUNT; ++i) {
             uint32_t count = 1;
-            if (i == B_CB_PACKED) count = 128;
+            if (i == B_CB_PACKED) count = 256;  // the packing warps (two per lane quarter)
             if (i == B_MK_FULL || i == B_MK_FULL + 1 || i == B_ACC_EMPTY || i == B_ACC_EMPTY + 1 ||
                 i == B_DEC_FREE || i == B_DEC_FREE + 1)
                 count = NMASK;
@@ -258,8 +343,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     __syncthreads();
     fence_after_sync();
     const uint32_t tmem = *tmem_slot;
+#ifdef SSD_TRACE
+    __shared__ unsigned long long s_trace[256];
+    for (int k = tid; k < 256; k += NTHREADS) s_trace[k] = 0;
+    __syncthreads();
+#endif
 
-    if (warp == 8) {
+    if (warp == CTRL_WARP) {
         // ------------------------------ control ------------------------------
         if (lane == 0) {
             const uint32_t box = static_cast<uint32_t>(Q) * 128;
@@ -273,19 +363,31 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     tma_load_4d(sH + kb * (PD * 128), &tm_h, bar(B_H_FULL), kb * 64, 0, (int)h,
                                 (int)(b * nc + c));
             };
+            auto prefetch_head = [&](int64_t h) {
+                tma_prefetch_l2_4d(&tm_x, 0, (int)h, (int)t0, (int)b);
+                for (int kb = 0; kb < NST / 64; ++kb)
+                    tma_prefetch_l2_4d(&tm_h, kb * 64, 0, (int)h, (int)(b * nc + c));
+            };
             tma_prefetch_map(&tm_c);
             tma_prefetch_map(&tm_b);
             tma_prefetch_map(&tm_x);
             tma_prefetch_map(&tm_h);
-            mbar_expect_tx(bar(B_CB_LOAD), 2 * (NST / 64) * box);
+            // C in 32-row blocks, each stored where its TMEM lane quarter
+            // expects it (tile 0's blocks reversed); B in chunk order
+            mbar_expect_tx(bar(B_CB_LOAD), (NST / 64) * (ntiles * 128 * 128 + box));
             for (int kb = 0; kb < NST / 64; ++kb) {
-                tma_load_4d(sC + kb * T::KB_BYTES, &tm_c, bar(B_CB_LOAD), kb * 64, (int)g,
-                            (int)t0, (int)b);
+                for (int t = 0; t < ntiles; ++t)
+                    for (int q = 0; q < 4; ++q)
+                        tma_load_4d(sC + kb * T::KB_BYTES + (128 * t + 32 * q) * 128, &tm_c,
+                                    bar(B_CB_LOAD), kb * 64, (int)g, (int)(t0 + block_row(t, q)),
+                                    (int)b);
                 tma_load_4d(sB + kb * T::KB_BYTES, &tm_b, bar(B_CB_LOAD), kb * 64, (int)g,
                             (int)t0, (int)b);
             }
             SCAN_TRACE(0);
             load_x(hfirst);
+            // C, B and x are inputs; the carried states come from step 3
+            grid_dep_wait();
             load_h(hfirst);
             bool ok = wait_bar(bar(B_CB_LOAD), 0, abort);
             SCAN_TRACE(1);
@@ -305,8 +407,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 SCAN_TRACE(2);
                 fence_after_sync();
             }
+            const uint64_t dC0 = desc_sw128(sC, 16, 1024), dC1 = desc_sw128(sC + 128 * 128, 16, 1024);
+            const uint64_t dH = desc_sw128(sH, 16, 1024), dX = desc_sw128(sX, QMAX * 128, 1024);
+            const uint64_t dM0 = desc_sw128(sM0, 16, 1024), dM1 = desc_sw128(sM1, 16, 1024);
             for (int i = 0; ok && i < hb_size; ++i) {
                 const uint32_t ph = i & 1;
+                if (i + 1 < hb_size) prefetch_head(hfirst + i + 1);  // next head's x, H_in into L2
                 ok = wait_bar(bar(B_H_FULL), ph, abort);
                 SCAN_TRACE(8 + 8 * i);
                 for (int t = 0; ok && t < ntiles; ++t) {
@@ -314,13 +420,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     if (i > 0) ok = wait_bar(bar(B_ACC_EMPTY + t), (i - 1) & 1, abort);
                     if (!ok) break;
                     fence_after_sync();
-                    for (int k = 0; k < NST / 16; ++k) {
-                        const uint32_t ko = (k >> 2) * T::KB_BYTES + (k & 3) * 32;
-                        const uint32_t kh = (k >> 2) * (PD * 128) + (k & 3) * 32;
-                        mma_bf16(tmem + st_col(t), desc_sw128(sC + ko + t * 128 * 128, 16, 1024),
-                                 desc_sw128(sH + kh, 16, 1024), idesc_bf16(128, PD, false, false),
-                                 k > 0 ? 1u : 0u);
-                    }
+                    issue_state<NST>(tmem + st_col(t), t == 0 ? dC0 : dC1, dH);
                     if (t == ntiles - 1) mma_commit(bar(B_H_FREE));
                     SCAN_TRACE(9 + 8 * i + 3 * t);
                     // intra-chunk term of tile t, once its mask (and the head's x) is in
@@ -329,21 +429,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     if (ok && t == 0) ok = wait_bar(bar(B_X_FULL), ph, abort);
                     if (!ok) break;
                     fence_after_sync();
-                    const uint32_t sM = t == 0 ? sM0 : sM1;
-                    for (int k = 0; k < 8 * (t + 1); ++k)
-                        mma_bf16(tmem + in_col(t),
-                                 desc_sw128(sM + (k >> 2) * (128 * 128) + (k & 3) * 32, 16, 1024),
-                                 desc_sw128(sX + k * 2048, QMAX * 128, 1024),
-                                 idesc_bf16(128, PD, false, true), k > 0 ? 1u : 0u);
+                    if (t == 0) issue_intra<8>(tmem + in_col(0), dM0, dX);
+                    else issue_intra<16>(tmem + in_col(1), dM1, dX);
                     mma_commit(bar(B_ACC_FULL + t));
                     mma_commit(bar(B_MK_EMPTY + t));
                     SCAN_TRACE(11 + 8 * i + 3 * t);
-#ifdef SSD_TRACE
-                    if (t == 0 && i < 8) {  // latency of this tile's MMAs and commit
-                        wait_bar(bar(B_MK_EMPTY), ph, abort);
-                        SCAN_TRACE(176 + i);
-                    }
-#endif
                 }
                 if (!ok) break;
                 mma_commit(bar(B_X_FREE));
@@ -357,11 +447,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             if (!ok) *abort = 1;
         }
-    } else if (warp == 9) {
+    } else if (warp == LOAD_WARP) {
         // ------------------------------- loader ------------------------------
         // Stages each head's decays (log2e * cumA, dt) and D into the two
-        // shared buffers, so the workers never wait on a global load.
+        // shared buffers.  Slots past the chunk's last token get that token's
+        // cumA and dt = 0, so every factor formed from them is finite.
         bool ok = true;
+        grid_dep_wait();  // dt and cumA come from steps 1-2
         for (int i = 0; ok && i < hb_size; ++i) {
             const int bsel = i & 1;
             if (i >= 2) ok = wait_bar(bar(B_DEC_FREE + bsel), ((i - 2) >> 1) & 1, abort);
@@ -369,12 +461,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             float* dec = reinterpret_cast<float*>(smem + T::DEC_OFF) + bsel * T::DEC_FLOATS;
             const int64_t h = hfirst + i;
             const int64_t vbase = ((b * H + h) * nc + c) * Q;
+            const float c_end = p.cumA[vbase + Lc - 1];
             float cv[QMAX / 32], dv[QMAX / 32];
 #pragma unroll
             for (int k = 0; k < QMAX / 32; ++k) {
                 const int j = lane + 32 * k;
-                cv[k] = j < Q ? p.cumA[vbase + j] : 0.0f;
-                dv[k] = j < Q ? p.dt[vbase + j] : 0.0f;
+                cv[k] = j < Lc ? p.cumA[vbase + j] : c_end;
+                dv[k] = j < Lc ? p.dt[vbase + j] : 0.0f;
             }
 #pragma unroll
             for (int k = 0; k < QMAX / 32; ++k) {
@@ -389,22 +482,30 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // ------------------------------ workers ------------------------------
         const int qd = warp & 3, hf = warp >> 2;
         float* rinv_s = reinterpret_cast<float*>(smem + T::RINV_OFF);
-        float* stab = reinterpret_cast<float*>(smem + T::STAB_OFF) + warp * QMAX;
+        float* cbd_s = reinterpret_cast<float*>(smem + T::CBD_OFF);
+        float* ctab = reinterpret_cast<float*>(smem + T::CTAB_OFF) + warp * 32;
         const uint32_t lanes = static_cast<uint32_t>(32 * qd) << 16;
         bool ok = wait_bar(bar(B_CB_DONE), 0, abort);
-        if (ok && hf == 0) {
-            fence_after_sync();
-            // repack CB as fp16 pairs with a per-row power-of-two scale:
-            // tile 0 [0,128) -> [0,64), tile 1 [128,384) -> [64,192)
-            for (int t = 0; t < ntiles; ++t) {
+        if (hf < 2) {
+            // repack tile hf's CB as fp16 pairs with a per-row power-of-two
+            // scale: tile 0 [0,128) -> [0,64), tile 1 [256,512) -> [128,256)
+            const int t = hf;
+            if (ok && t < ntiles) {
+                fence_after_sync();
                 const uint32_t src = t == 0 ? 0u : CB1F, dst = t == 0 ? CB0P : CB1P;
-                float mx = 0.0f;
+                const int rb = block_row(t, qd) >> 5;  // the 32 columns holding this row's diagonal
+                float mx = 0.0f, dg = 0.0f;
                 for (int k = 0; k < 4 * (t + 1); ++k) {
                     float v[32];
                     tmem_ld32(tmem + lanes + src + 32 * k, v);
 #pragma unroll
                     for (int q = 0; q < 32; ++q) mx = fmaxf(mx, fabsf(v[q]));
+                    if (k == rb) {
+#pragma unroll
+                        for (int q = 0; q < 32; ++q) dg = (q == lane) ? v[q] : dg;
+                    }
                 }
+                cbd_s[t * 128 + 32 * qd + lane] = dg;
                 // 2^e with the row's largest |CB| * 2^-e below 2^15
                 const int e2 = max(0, ((__float_as_int(mx) >> 23) & 255) - 127 - 14 + 1);
                 const float sc = __int_as_float((127 - e2) << 23);
@@ -423,35 +524,46 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             mbar_arrive(bar(B_CB_PACKED));
             if (warp == 0 && lane == 0) SCAN_TRACE(80);
         }
-        if (ok && hf == 1) ok = wait_bar(bar(B_CB_PACKED), 0, abort);
+        if (ok) ok = wait_bar(bar(B_CB_PACKED), 0, abort);
         fence_after_sync();
         const float rinv0 = ok ? rinv_s[32 * qd + lane] : 1.0f;
         const float rinv1 = (ok && ntiles == 2) ? rinv_s[128 + 32 * qd + lane] : 1.0f;
+        const float cbd0 = ok ? cbd_s[32 * qd + lane] : 0.0f;
+        const float cbd1 = (ok && ntiles == 2) ? cbd_s[128 + 32 * qd + lane] : 0.0f;
 
-        // The epilogue of head i, tile t, for this warp's rows and 32 p columns.
-        // D x came through the mask diagonal and log2e * cumA of the row was kept
-        // from the mask phase, so nothing here waits on a global load.
-        auto epilogue = [&](int i, int t, float cl2) -> bool {
+        // The epilogue of head i, tile t, for this warp's rows and 16 p
+        // columns: y = f * intra + 2^cl * state + w x_l, w the diagonal weight
+        // (C_l . B_l dt_l + D).  x_l was stashed in TMEM while the head's x
+        // tile was resident, so the worker loop never waits on a global load.
+        auto epilogue = [&](int i, int t, float cl2, float2 fw) -> bool {
             const int64_t h = hfirst + i;
-            const int l = 128 * t + 32 * qd + lane;
+            const int l = block_row(t, qd) + lane;
             if (!wait_bar(bar(B_ACC_FULL + t), i & 1, abort)) return false;
             if (warp == 0 && lane == 0) SCAN_TRACE(140 + 4 * i + 2 * t);
+            const int64_t off = ((b * L + t0 + l) * H + h) * PD + 16 * hf;
             fence_after_sync();
-            float vi[32], vs[32];
-            tmem_ld32x2(tmem + lanes + in_col(t) + 32 * hf, vi, tmem + lanes + st_col(t) + 32 * hf, vs);
+            const uint32_t a[2] = {tmem + lanes + in_col(t) + 16 * hf, tmem + lanes + st_col(t) + 16 * hf};
+            uint32_t r[2][16], xw[8];
+            tmem_ld8(tmem + lanes + stash_col(t, hf), xw);
+            tmem_ld16x2(a, r);
             fence_before_sync();
             mbar_arrive(bar(B_ACC_EMPTY + t));
             if (l < Lc) {
-                const float sc = ex2(cl2);
-                __nv_bfloat16* yr = static_cast<__nv_bfloat16*>(p.y) +
-                                    ((b * L + t0 + l) * H + h) * PD + 32 * hf;
+                const float s = ex2(cl2);
+                __nv_bfloat16* yr = static_cast<__nv_bfloat16*>(p.y) + off;
 #pragma unroll
-                for (int k4 = 0; k4 < 4; ++k4) {
+                for (int k4 = 0; k4 < 2; ++k4) {
                     uint32_t o[4];
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
                         const int e = 8 * k4 + 2 * k;
-                        o[k] = pack_bf16x2(fmaf(sc, vs[e], vi[e]), fmaf(sc, vs[e + 1], vi[e + 1]));
+                        const float2 xf =
+                            __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xw[4 * k4 + k]));
+                        const float y0 = fmaf(fw.y, xf.x, fmaf(s, __uint_as_float(r[1][e]),
+                                                              fw.x * __uint_as_float(r[0][e])));
+                        const float y1 = fmaf(fw.y, xf.y, fmaf(s, __uint_as_float(r[1][e + 1]),
+                                                              fw.x * __uint_as_float(r[0][e + 1])));
+                        o[k] = pack_bf16x2(y0, y1);
                     }
                     reinterpret_cast<uint4*>(yr)[k4] = make_uint4(o[0], o[1], o[2], o[3]);
                 }
@@ -460,48 +572,87 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             return true;
         };
 
-        // Iteration i builds head i's masks and drains head i-1's accumulators,
-        // tile by tile, so the tensor core works on one head while the CUDA cores
-        // finish the previous one.
+        // This warp's x rows of the resident x tile -> TMEM, for the diagonal
+        // term of the head's epilogue (x is overwritten by the next head once
+        // the last tile's MMA is done, which waits for this warp's mask).
+        auto stash_x = [&]() {
+            for (int t = 0; t < ntiles; ++t) {
+                const int l = block_row(t, qd) + lane;
+                const uint4 v0 = ld_shared_v4(sX + sw128(l, 2 * hf));
+                const uint4 v1 = ld_shared_v4(sX + sw128(l, 2 * hf + 1));
+                const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+                tmem_st8(tmem + lanes + stash_col(t, hf), w);
+            }
+            tmem_wait_st();
+        };
+
+        // Iteration i builds head i's tile-0 mask, drains head i-1's
+        // accumulators, stashes head i's x rows and builds its tile-1 mask, so
+        // the tensor core works on one head while the CUDA cores finish the
+        // previous one.
         float cl_prev[2] = {0.0f, 0.0f};
+        float2 fw_prev[2] = {make_float2(1.0f, 0.0f), make_float2(1.0f, 0.0f)};
         for (int i = 0; i <= hb_size; ++i) {
             const bool mask_now = i < hb_size, epi_now = i > 0;
             const int bsel = i & 1;
             const float* dec = reinterpret_cast<const float*>(smem + T::DEC_OFF) + bsel * T::DEC_FLOATS;
             float cl_cur[2] = {0.0f, 0.0f};
+            float2 fw_cur[2] = {make_float2(1.0f, 0.0f), make_float2(1.0f, 0.0f)};
             float Dh = 0.0f;
             if (mask_now && ok) {
                 ok = wait_bar(bar(B_DEC_FULL + bsel), (i >> 1) & 1, abort);
                 if (warp == 0 && lane == 0) SCAN_TRACE(82 + 5 * i);
                 if (ok) {
-                    cl_cur[0] = dec[32 * qd + lane];
-                    cl_cur[1] = dec[128 + 32 * qd + lane];
+                    cl_cur[0] = dec[block_row(0, qd) + lane];
+                    cl_cur[1] = dec[block_row(1, qd) + lane];
                     Dh = dec[2 * QMAX];
                 }
             }
-            for (int t = 0; t < ntiles; ++t) {
-                if (mask_now && ok) {
-                    if (i > 0) ok = wait_bar(bar(B_MK_EMPTY + t), (i - 1) & 1, abort);
-                    if (warp == 0 && lane == 0) SCAN_TRACE(83 + 5 * i + 2 * t);
-                    if (ok) {
-                        if (t == 0)
-                            build_mask<0>(tmem, sM0, dec, dec + QMAX, stab, rinv0, Dh, qd, hf, lane);
-                        else
-                            build_mask<1>(tmem, sM1, dec, dec + QMAX, stab, rinv1, Dh, qd, hf, lane);
-                        fence_smem_async();
-                        mbar_arrive(bar(B_MK_FULL + t));
-                    }
-                    if (warp == 0 && lane == 0) SCAN_TRACE(84 + 5 * i + 2 * t);
+            if (mask_now && ok) {
+                if (i > 0) ok = wait_bar(bar(B_MK_EMPTY), (i - 1) & 1, abort);
+                if (warp == 0 && lane == 0) SCAN_TRACE(83 + 5 * i);
+                if (ok) {
+                    fw_cur[0] = build_mask<0>(tmem, sM0, dec, dec + QMAX, ctab, rinv0, cbd0, Dh, qd,
+                                              hf, lane, Lc, i == 0);
+                    fence_smem_async();
+                    // the last tile's mask is released only after the x stash
+                    if (ntiles == 2) mbar_arrive(bar(B_MK_FULL));
                 }
-                if (epi_now && ok) ok = epilogue(i - 1, t, cl_prev[t]);
+                if (warp == 0 && lane == 0) SCAN_TRACE(84 + 5 * i);
+            }
+            for (int t = 0; t < ntiles; ++t)
+                if (epi_now && ok) ok = epilogue(i - 1, t, cl_prev[t], fw_prev[t]);
+            if (mask_now && ok) {
+                ok = wait_bar(bar(B_X_FULL), i & 1, abort);
+                if (warp == 0 && lane == 0) SCAN_TRACE(200 + 2 * i);
+                if (ok) stash_x();
+                if (warp == 0 && lane == 0) SCAN_TRACE(201 + 2 * i);
+                if (ok && ntiles == 1) mbar_arrive(bar(B_MK_FULL));
+            }
+            if (mask_now && ok && ntiles == 2) {
+                if (i > 0) ok = wait_bar(bar(B_MK_EMPTY + 1), (i - 1) & 1, abort);
+                if (warp == 0 && lane == 0) SCAN_TRACE(85 + 5 * i);
+                if (ok) {
+                    fw_cur[1] = build_mask<1>(tmem, sM1, dec, dec + QMAX, ctab, rinv1, cbd1, Dh, qd,
+                                              hf, lane, Lc, i == 0);
+                    fence_smem_async();
+                    mbar_arrive(bar(B_MK_FULL + 1));
+                }
+                if (warp == 0 && lane == 0) SCAN_TRACE(86 + 5 * i);
             }
             if (mask_now && ok) mbar_arrive(bar(B_DEC_FREE + bsel));  // this head's decays are used
             cl_prev[0] = cl_cur[0];
             cl_prev[1] = cl_cur[1];
+            fw_prev[0] = fw_cur[0];
+            fw_prev[1] = fw_cur[1];
         }
     }
     fence_before_sync();
     __syncthreads();
+#ifdef SSD_TRACE
+    if (blockIdx.x < 8 && blockIdx.y == 0)
+        for (int k = tid; k < 256; k += NTHREADS) g_scan_trace[blockIdx.x][k] = s_trace[k];
+#endif
     if (*abort && tid == 0 && p.status) atomicExch(p.status, static_cast<int>(SSD_ERR_TIMEOUT));
     if (warp == 0) {
         fence_after_sync();
@@ -513,8 +664,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 // and then pipelines its heads, so with w waves of CTAs over the SMs the
 // kernel takes about w * (setup + heads * per_head).  The divisor of the heads
 // per group that minimises this, up to 12 heads, is used (or every head of the
-// group, when asked).  The two costs are the measured ones (about 5 and 4.5
-// us); beyond about a dozen heads per CTA the measured time rises again.
+// group, when asked).  The two costs are the measured ones (in microseconds);
+// beyond about a dozen heads per CTA the measured time rises again.
 int heads_per_cta(const FwdParams& p, int num_sms) {
     if (p.flags & SSD_FLAG_WHOLE_GROUPS) return static_cast<int>(p.heads_per_group);
     // tuning override: SSD_SCAN_HEADS_PER_CTA=d (used when d divides the heads per group)
@@ -555,7 +706,7 @@ cudaError_t launch_n(const FwdParams& p, cudaStream_t s) {
     using T = ScanTile<NST>;
     CUtensorMap tc_, tb_, tx_, th_;
     const uint32_t rows = static_cast<uint32_t>(p.chunk);
-    if (!make_tmap_bf16_4d(&tc_, p.C, NST, p.ngroups, p.seqlen, p.batch, 1, rows) ||
+    if (!make_tmap_bf16_4d(&tc_, p.C, NST, p.ngroups, p.seqlen, p.batch, 1, 32) ||
         !make_tmap_bf16_4d(&tb_, p.B, NST, p.ngroups, p.seqlen, p.batch, 1, rows) ||
         !make_tmap_bf16_4d(&tx_, p.x, PD, p.nheads, p.seqlen, p.batch, 1, rows) ||
         !make_tmap_bf16_4d(&th_, p.states, NST, PD, p.nheads, p.batch * p.nchunks, PD, 1))
@@ -566,8 +717,7 @@ cudaError_t launch_n(const FwdParams& p, cudaStream_t s) {
     const int hb = heads_per_cta(p, sm_count());
     dim3 grid(static_cast<unsigned>(p.nchunks * p.ngroups * (p.heads_per_group / hb)),
               static_cast<unsigned>(p.batch));
-    kern<<<grid, NTHREADS, T::SMEM, s>>>(p, tc_, tb_, tx_, th_, hb);
-    return cudaGetLastError();
+    return launch_kernel(kern, grid, dim3(NTHREADS), T::SMEM, s, p.pdl != 0, p, tc_, tb_, tx_, th_, hb);
 }
 
 }  // namespace

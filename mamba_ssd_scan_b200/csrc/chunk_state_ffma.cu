@@ -18,6 +18,8 @@ constexpr int TP = 64, TN = 64, TK = 32;
 
 template <typename T>
 __global__ void __launch_bounds__(256) chunk_state_ffma_kernel(FwdParams p) {
+    grid_dep_wait();  // dt and cumA come from step 1
+    grid_dep_launch();
     const int64_t H = p.nheads, P = p.headdim, N = p.dstate, G = p.ngroups;
     const int64_t L = p.seqlen, Q = p.chunk, nc = p.nchunks;
     const int64_t ntile_n = (N + TN - 1) / TN;
@@ -90,8 +92,7 @@ template <typename T>
 cudaError_t launch_chunk_state_ffma(const FwdParams& p, cudaStream_t s) {
     const unsigned tiles = (unsigned)(((p.headdim + TP - 1) / TP) * ((p.dstate + TN - 1) / TN));
     dim3 grid((unsigned)(p.nchunks * p.nheads), tiles, (unsigned)p.batch);
-    chunk_state_ffma_kernel<T><<<grid, 256, 0, s>>>(p);
-    return cudaGetLastError();
+    return launch_kernel(chunk_state_ffma_kernel<T>, grid, dim3(256), 0, s, p.pdl != 0, p);
 }
 
 template cudaError_t launch_chunk_state_ffma<float>(const FwdParams&, cudaStream_t);

@@ -16,7 +16,9 @@
 // 64 KB of shared memory (dstate 128) three CTAs share an SM, so one CTA's
 // loads overlap another's MMAs and epilogue.  The epilogue moves the fp32
 // accumulator from TMEM to the states buffer in the input dtype (bf16), one
-// row of dstate per thread.
+// row of dstate per thread.  When the forward call fuses step 1, the first
+// 128/P warps first form dt and cumA of the CTA's heads with the same warp
+// scan as step 1 and store them for steps 3 and 4.
 #include "internal.cuh"
 #include "tcgen05.cuh"
 #include "tma.cuh"
@@ -101,6 +103,18 @@ __global__ void __launch_bounds__(256, 1)
     __syncthreads();
     if (tid == 0)
         for (int q = 0; q < nq && q < NSLOT; ++q) issue(q);
+    // x and B are inputs; dt and cumA are formed here (step 1 fused, one warp
+    // per head) or come from step 1
+    grid_dep_wait();
+    if (p.fuse_cumsum) {
+        if (warp < T::HPC) {
+            const int64_t off = ((b * H + h0 + warp) * nc + c) * Q;
+            chunk_cumsum_warp<__nv_bfloat16>(p, b, c, h0 + warp, p.dt + off, p.cumA + off, lane);
+        }
+        if (blockIdx.x == 0 && blockIdx.y == 0 && tid == 0 && p.status) *p.status = 0;  // a new call
+        __syncthreads();
+    }
+    grid_dep_launch();
     for (int i = tid; i < T::HPC * QMAX; i += 256) {
         const int hh = i / QMAX, l = i % QMAX;
         float w = 0.0f;
@@ -193,8 +207,7 @@ cudaError_t launch_nd(const FwdParams& p, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, T::SMEM);
     if (e != cudaSuccess) return e;
     dim3 grid(static_cast<unsigned>(p.nchunks * (p.nheads / T::HPC)), static_cast<unsigned>(p.batch));
-    kern<<<grid, 256, T::SMEM, s>>>(p, tx_, tb_);
-    return cudaGetLastError();
+    return launch_kernel(kern, grid, dim3(256), T::SMEM, s, p.pdl != 0, p, tx_, tb_);
 }
 
 }  // namespace

@@ -15,6 +15,11 @@ struct FwdParams {
     int64_t batch, seqlen, nheads, headdim, dstate, ngroups, chunk, nchunks;
     int64_t heads_per_group;
     int32_t flags;         // SSD_FLAG_* of the call
+    // launch plumbing (not a user flag): the kernels after the first of a call
+    // go out with programmatic dependent launch, and the tensor-core
+    // chunk_state forms dt and cumA itself (fusing step 1)
+    int32_t pdl;
+    int32_t fuse_cumsum;
     const void* x;
     const void* dt_raw;
     const float* A;
@@ -57,6 +62,81 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
 // softplus(u) = log(1 + e^u) without overflow.
 __device__ __forceinline__ float softplus_f32(float u) {
     return fmaxf(u, 0.0f) + log1pf(expf(-fabsf(u)));
+}
+
+// Programmatic dependent launch.  A kernel launched with pdl set may start
+// while the previous kernel of the stream is still running; it must call
+// grid_dep_wait() before it reads or writes anything that kernel (or an
+// earlier one of the same call) produces.  grid_dep_launch() lets the next
+// kernel start its own prologue early.  Both are no-ops for plain launches.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                          bool pdl, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
+// dt = softplus(dt_raw + dt_bias) and the inclusive in-chunk cumulative sum of
+// dt * A for one (batch, chunk, head), by one warp: each lane loads its
+// tokens of every 32-token segment first, then the warp scans the segments in
+// order with shuffles and a running carry.  Entries past the end of a short
+// last chunk hold dt = 0 and the last cumulative value, so cumA[Q-1] is the
+// chunk's total log-decay.  Writes both to dt_out / cum_out (Q entries).
+// "MAMBA-2 Reference Implementations Comparison", section 3.2 (softplus
+// discretisation of dt and the exp(A dt) decays whose exponents this sums).
+template <typename T>
+__device__ __forceinline__ void chunk_cumsum_warp(const FwdParams& p, int64_t b, int64_t c, int64_t h,
+                                                  float* dt_out, float* cum_out, int lane) {
+    constexpr int MAXSEG = 8;  // chunk <= 256 tokens
+    const int64_t Q = p.chunk, H = p.nheads, L = p.seqlen;
+    const int64_t t0 = c * Q;
+    const int64_t Lc = (L - t0 < Q) ? (L - t0) : Q;
+    const int nseg = static_cast<int>((Q + 31) / 32);
+    const T* dtr = static_cast<const T*>(p.dt_raw) + (b * L + t0) * H + h;
+    const float A = p.A[h];
+    const float bias = p.dt_bias ? p.dt_bias[h] : 0.0f;
+    float u[MAXSEG];
+#pragma unroll
+    for (int s = 0; s < MAXSEG; ++s) {
+        const int64_t l = s * 32 + lane;
+        u[s] = (s < nseg && l < Lc) ? to_f32(dtr[l * H]) : 0.0f;
+    }
+    float carry = 0.0f;
+#pragma unroll
+    for (int s = 0; s < MAXSEG; ++s) {
+        if (s >= nseg) break;
+        const int64_t l = s * 32 + lane;
+        float dt = 0.0f, v = 0.0f;
+        if (l < Lc) {
+            dt = softplus_f32(u[s] + bias);
+            v = dt * A;
+        }
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float n = __shfl_up_sync(0xffffffffu, v, o);
+            if (lane >= o) v += n;
+        }
+        v += carry;
+        if (l < Q) {
+            dt_out[l] = dt;
+            cum_out[l] = v;
+        }
+        carry = __shfl_sync(0xffffffffu, v, 31);
+    }
 }
 
 // Launchers (one per kernel family).  Each returns cudaGetLastError().

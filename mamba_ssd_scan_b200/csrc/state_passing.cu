@@ -55,6 +55,8 @@ template <> struct Pack<__nv_bfloat16> {
 
 template <typename T>
 __global__ void __launch_bounds__(256) state_passing_kernel(FwdParams p) {
+    grid_dep_wait();  // the local states and cumA come from the previous steps
+    grid_dep_launch();
     constexpr int E = Pack<T>::E;
     const int64_t H = p.nheads, nc = p.nchunks, Q = p.chunk;
     const int64_t vecs_per_head = p.headdim * p.dstate / E;
@@ -111,8 +113,8 @@ __global__ void __launch_bounds__(256) state_passing_kernel(FwdParams p) {
 template <typename T>
 cudaError_t launch_state_passing(const FwdParams& p, cudaStream_t s) {
     const int64_t n = p.batch * p.nheads * p.headdim * p.dstate / Pack<T>::E;
-    state_passing_kernel<T><<<(unsigned)((n + 255) / 256), 256, 0, s>>>(p);
-    return cudaGetLastError();
+    return launch_kernel(state_passing_kernel<T>, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s,
+                         p.pdl != 0, p);
 }
 
 template cudaError_t launch_state_passing<float>(const FwdParams&, cudaStream_t);

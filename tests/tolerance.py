@@ -30,12 +30,15 @@ def report(gpu, ref):
     rel = d / np.maximum(np.abs(o), 1e-30)
     rms = float(np.sqrt(np.mean(o * o))) if d.size else 0.0
     # worst element against the bf16 element-wise bound (1.0 = at the bound)
-    margin = float((d / (BF16_TOL * (np.abs(o) + rms) + 1e-300)).max()) if d.size else 0.0
+    ratio = d / (BF16_TOL * (np.abs(o) + rms) + 1e-300)
+    w = int(np.argmax(ratio)) if d.size else 0
     return {"max_abs": float(d.max()) if d.size else 0.0,
             "max_rel": float(rel.max()) if d.size else 0.0,
             "argmax": np.unravel_index(i, d.shape) if d.size else (),
             "ref_max": float(np.abs(o).max()) if d.size else 0.0,
-            "ref_rms": rms, "worst_vs_bf16_bound": margin}
+            "ref_rms": rms, "worst_vs_bf16_bound": float(ratio.max()) if d.size else 0.0,
+            "worst_at": np.unravel_index(w, d.shape) if d.size else (),
+            "worst_gpu_ref": (float(g.flat[w]), float(o.flat[w])) if d.size else ()}
 
 
 def assert_close(gpu, ref, dtype, what=""):
