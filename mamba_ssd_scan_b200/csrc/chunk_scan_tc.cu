@@ -22,7 +22,8 @@
 //              operand to shared memory (one buffer per tile, refilled as soon
 //              as its MMA is done); then drain the previous head's accumulators
 //              for the same tile (y = f * intra + exp(cumA) * state, plus the
-//              diagonal term (C_l . B_l dt_l + D) x_l in fp32, bf16 out).  The
+//              diagonal term (C_l . B_l dt_l + D) x_l in fp32, bf16 staged
+//              for the storer).  The
 //              four warps of a TMEM lane quarter share its 32 rows and take
 //              one column group in four (and a quarter of the p columns in
 //              the epilogue);
@@ -30,7 +31,10 @@
 //              H_in per head) and every MMA (CB once; per head and tile the
 //              state term C_t H_in^T and Mk x);
 //   warp 17    "loader": stages each head's decays and D in shared memory
-//              (two buffers), so the mask phase never waits on a global load.
+//              (two buffers), so the mask phase never waits on a global load;
+//   warp 18    "storer": the workers stage each head's y tile in shared memory
+//              and one lane writes it out with a TMA store, so no worker
+//              holds a global store when it next signals an mbarrier.
 //
 // Balance.  A warp only reaches the TMEM lanes of its quarter (warp % 4),
 // which is also the scheduler it issues on, and a causal row's work grows
@@ -70,8 +74,8 @@ using namespace tc;
 constexpr int QMAX = 256;
 constexpr int PD = 64;
 constexpr int NWORK = 16;                        // worker warps
-constexpr int CTRL_WARP = NWORK, LOAD_WARP = NWORK + 1;
-constexpr int NTHREADS = (NWORK + 2) * 32;
+constexpr int CTRL_WARP = NWORK, LOAD_WARP = NWORK + 1, STORE_WARP = NWORK + 2;
+constexpr int NTHREADS = (NWORK + 3) * 32;
 constexpr int NMASK = NWORK * 32;
 constexpr uint32_t CB0P = 0, CB1P = 128, CB1F = 256;
 // largest log2 decay span of a 32-row block that takes the factored path:
@@ -133,7 +137,7 @@ enum : int {
     B_CB_LOAD = 0, B_CB_DONE, B_CB_PACKED, B_X_FULL, B_H_FULL, B_H_FREE, B_X_FREE,
     B_MK_FULL, B_MK_EMPTY = B_MK_FULL + 2, B_ACC_FULL = B_MK_EMPTY + 2,
     B_ACC_EMPTY = B_ACC_FULL + 2, B_DEC_FULL = B_ACC_EMPTY + 2, B_DEC_FREE = B_DEC_FULL + 2,
-    B_COUNT = B_DEC_FREE + 2
+    B_Y_STAGED = B_DEC_FREE + 2, B_Y_READ, B_COUNT
 };
 
 // Bounded wait that also gives up when another role has aborted: a few
@@ -303,7 +307,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     chunk_scan_tc_kernel(const __grid_constant__ FwdParams p, const __grid_constant__ CUtensorMap tm_c,
                          const __grid_constant__ CUtensorMap tm_b,
                          const __grid_constant__ CUtensorMap tm_x,
-                         const __grid_constant__ CUtensorMap tm_h, int hb_size) {
+                         const __grid_constant__ CUtensorMap tm_h,
+                         const __grid_constant__ CUtensorMap tm_y, int hb_size) {
     using T = ScanTile<NST>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -324,6 +329,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t sC = smem_u32(smem + T::C_OFF), sB = smem_u32(smem + T::B_OFF);
     const uint32_t sM0 = smem_u32(smem + T::MK0_OFF), sM1 = sB;
     const uint32_t sX = smem_u32(smem + T::X_OFF), sH = smem_u32(smem + T::H_OFF);
+    // y of one head is staged in tile 1's mask buffer, in its K columns
+    // 0-127 (rewritten for every head, never a zero group), between the MMA
+    // that read that buffer and the next mask, and leaves by TMA
+    const uint32_t sY = sM1;
 
     if (warp == 0) tmem_alloc(smem_u32(tmem_slot), 512);
     if (tid == 0) {
@@ -331,7 +340,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             uint32_t count = 1;
             if (i == B_CB_PACKED) count = 256;  // the packing warps (two per lane quarter)
             if (i == B_MK_FULL || i == B_MK_FULL + 1 || i == B_ACC_EMPTY || i == B_ACC_EMPTY + 1 ||
-                i == B_DEC_FREE || i == B_DEC_FREE + 1)
+                i == B_DEC_FREE || i == B_DEC_FREE + 1 || i == B_Y_STAGED)
                 count = NMASK;
             if (i == B_DEC_FULL || i == B_DEC_FULL + 1) count = 32;
             mbar_init(bar(i), count);
@@ -478,6 +487,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             mbar_arrive(bar(B_DEC_FULL + bsel));
         }
         if (!ok) *abort = 1;
+    } else if (warp == STORE_WARP) {
+        // ------------------------------- storer ------------------------------
+        // Each head's staged y tile goes out as one TMA store; the workers
+        // may overwrite the staging buffer once the store has read it.
+        if (lane == 0) {
+            tma_prefetch_map(&tm_y);
+            for (int k = 0; k < hb_size; ++k) {
+                if (!wait_bar(bar(B_Y_STAGED), k & 1, abort)) break;
+                tma_store_4d(&tm_y, sY, 0, (int)(hfirst + k), (int)t0, (int)b);
+                bulk_commit_group();
+                bulk_wait_read_all();
+                mbar_arrive(bar(B_Y_READ));
+            }
+            bulk_wait_all();
+        }
     } else {
         // ------------------------------ workers ------------------------------
         const int qd = warp & 3, hf = warp >> 2;
@@ -536,11 +560,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // (C_l . B_l dt_l + D).  x_l was stashed in TMEM while the head's x
         // tile was resident, so the worker loop never waits on a global load.
         auto epilogue = [&](int i, int t, float cl2, float2 fw) -> bool {
-            const int64_t h = hfirst + i;
             const int l = block_row(t, qd) + lane;
             if (!wait_bar(bar(B_ACC_FULL + t), i & 1, abort)) return false;
             if (warp == 0 && lane == 0) SCAN_TRACE(140 + 4 * i + 2 * t);
-            const int64_t off = ((b * L + t0 + l) * H + h) * PD + 16 * hf;
             fence_after_sync();
             const uint32_t a[2] = {tmem + lanes + in_col(t) + 16 * hf, tmem + lanes + st_col(t) + 16 * hf};
             uint32_t r[2][16], xw[8];
@@ -550,7 +572,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             mbar_arrive(bar(B_ACC_EMPTY + t));
             if (l < Lc) {
                 const float s = ex2(cl2);
-                __nv_bfloat16* yr = static_cast<__nv_bfloat16*>(p.y) + off;
 #pragma unroll
                 for (int k4 = 0; k4 < 2; ++k4) {
                     uint32_t o[4];
@@ -565,7 +586,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                                                               fw.x * __uint_as_float(r[0][e + 1])));
                         o[k] = pack_bf16x2(y0, y1);
                     }
-                    reinterpret_cast<uint4*>(yr)[k4] = make_uint4(o[0], o[1], o[2], o[3]);
+                    st_shared_v4(sY + sw128(l, 2 * hf + k4), o[0], o[1], o[2], o[3]);
                 }
             }
             if (warp == 0 && lane == 0) SCAN_TRACE(141 + 4 * i + 2 * t);
@@ -620,8 +641,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 }
                 if (warp == 0 && lane == 0) SCAN_TRACE(84 + 5 * i);
             }
-            for (int t = 0; t < ntiles; ++t)
-                if (epi_now && ok) ok = epilogue(i - 1, t, cl_prev[t], fw_prev[t]);
+            if (epi_now && ok) {
+                // the staging buffer is free once tile 1's MMA of head i-1 is
+                // done with it and the store of head i-2 has read it
+                if (ntiles == 2) ok = wait_bar(bar(B_MK_EMPTY + 1), (i - 1) & 1, abort);
+                else if (i >= 2) ok = wait_bar(bar(B_Y_READ), (i - 2) & 1, abort);
+                for (int t = 0; t < ntiles; ++t)
+                    if (ok) ok = epilogue(i - 1, t, cl_prev[t], fw_prev[t]);
+                if (ok) {
+                    fence_smem_async();
+                    mbar_arrive(bar(B_Y_STAGED));
+                }
+            }
             if (mask_now && ok) {
                 ok = wait_bar(bar(B_X_FULL), i & 1, abort);
                 if (warp == 0 && lane == 0) SCAN_TRACE(200 + 2 * i);
@@ -630,7 +661,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (ok && ntiles == 1) mbar_arrive(bar(B_MK_FULL));
             }
             if (mask_now && ok && ntiles == 2) {
-                if (i > 0) ok = wait_bar(bar(B_MK_EMPTY + 1), (i - 1) & 1, abort);
+                if (i > 0) ok = wait_bar(bar(B_Y_READ), (i - 1) & 1, abort);  // staged y stored
                 if (warp == 0 && lane == 0) SCAN_TRACE(85 + 5 * i);
                 if (ok) {
                     fw_cur[1] = build_mask<1>(tmem, sM1, dec, dec + QMAX, ctab, rinv1, cbd1, Dh, qd,
@@ -704,12 +735,13 @@ int sm_count() {
 template <int NST>
 cudaError_t launch_n(const FwdParams& p, cudaStream_t s) {
     using T = ScanTile<NST>;
-    CUtensorMap tc_, tb_, tx_, th_;
+    CUtensorMap tc_, tb_, tx_, th_, ty_;
     const uint32_t rows = static_cast<uint32_t>(p.chunk);
     if (!make_tmap_bf16_4d(&tc_, p.C, NST, p.ngroups, p.seqlen, p.batch, 1, 32) ||
         !make_tmap_bf16_4d(&tb_, p.B, NST, p.ngroups, p.seqlen, p.batch, 1, rows) ||
         !make_tmap_bf16_4d(&tx_, p.x, PD, p.nheads, p.seqlen, p.batch, 1, rows) ||
-        !make_tmap_bf16_4d(&th_, p.states, NST, PD, p.nheads, p.batch * p.nchunks, PD, 1))
+        !make_tmap_bf16_4d(&th_, p.states, NST, PD, p.nheads, p.batch * p.nchunks, PD, 1) ||
+        !make_tmap_bf16_4d(&ty_, p.y, PD, p.nheads, p.seqlen, p.batch, 1, rows))
         return cudaErrorInvalidValue;
     auto kern = chunk_scan_tc_kernel<NST>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, T::SMEM);
@@ -717,7 +749,7 @@ cudaError_t launch_n(const FwdParams& p, cudaStream_t s) {
     const int hb = heads_per_cta(p, sm_count());
     dim3 grid(static_cast<unsigned>(p.nchunks * p.ngroups * (p.heads_per_group / hb)),
               static_cast<unsigned>(p.batch));
-    return launch_kernel(kern, grid, dim3(NTHREADS), T::SMEM, s, p.pdl != 0, p, tc_, tb_, tx_, th_, hb);
+    return launch_kernel(kern, grid, dim3(NTHREADS), T::SMEM, s, p.pdl != 0, p, tc_, tb_, tx_, th_, ty_, hb);
 }
 
 }  // namespace

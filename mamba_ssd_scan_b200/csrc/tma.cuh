@@ -1,8 +1,8 @@
 // tma.cuh -- tensor-memory-accelerator (TMA) loads: the host builds a tiled
 // tensor map (cuTensorMapEncodeTiled, reached through the runtime's driver
 // entry point so the library does not link libcuda) and one thread per CTA
-// issues cp.async.bulk.tensor loads that complete on an mbarrier.  Loads only,
-// never with cluster multicast.
+// issues cp.async.bulk.tensor loads that complete on an mbarrier (and bulk
+// stores tracked by bulk async groups).  Never with cluster multicast.
 #pragma once
 
 #include <cuda.h>
@@ -38,6 +38,28 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map
         : "r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(mbar), "r"(c0), "r"(c1), "r"(c2),
           "r"(c3)
         : "memory");
+}
+
+// One box from shared memory to a 4-D tensor in global memory (bulk async
+// group of the issuing thread; elements outside the tensor are not written).
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, uint32_t src, int c0, int c1,
+                                             int c2, int c3) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];"
+        :
+        : "l"(reinterpret_cast<uint64_t>(map)), "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+        : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() {
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Wait until the bulk groups of this thread have finished reading shared memory.
+__device__ __forceinline__ void bulk_wait_read_all() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Wait until the bulk groups of this thread have completed.
+__device__ __forceinline__ void bulk_wait_all() {
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 // Bring one box of a 4-D tensor map into L2 only (no shared memory, no
