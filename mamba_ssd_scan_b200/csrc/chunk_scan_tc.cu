@@ -170,6 +170,16 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
     return *reinterpret_cast<const uint32_t*>(&v);
 }
 
+// 32 bf16 values of one row (16 packed pairs) into the K-major SW128 operand
+__device__ __forceinline__ void store_group_packed(uint32_t mbase, uint32_t row, int j0,
+                                                   const uint32_t (&o)[16]) {
+    const uint32_t dst = mbase + (j0 >> 6) * (128 * 128);
+    const int c0 = (j0 & 63) >> 3;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        st_shared_v4(dst + sw128(row, c0 + i), o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+}
+
 // 32 masked values of one row -> bf16, into the K-major SW128 operand
 __device__ __forceinline__ void store_group(uint32_t mbase, uint32_t row, int j0, const float (&v)[32]) {
     const uint32_t dst = mbase + (j0 >> 6) * (128 * 128);
@@ -233,28 +243,32 @@ __device__ __forceinline__ float2 build_mask(uint32_t tmem, uint32_t mbase, cons
         ctab[lane] = cj;
         __syncwarp();
         const float4* ct = reinterpret_cast<const float4*>(ctab);
+        if (g < rb && fast) {  // below the diagonal block: packed fp32x2 products
+            uint32_t o[16];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float4 c = ct[i];
+                const float2 a0 = __half22float2(*reinterpret_cast<const __half2*>(&raw[2 * i]));
+                const float2 a1 = __half22float2(*reinterpret_cast<const __half2*>(&raw[2 * i + 1]));
+                const float2 m0 = __fmul2_rn(a0, make_float2(c.x, c.y));
+                const float2 m1 = __fmul2_rn(a1, make_float2(c.z, c.w));
+                o[2 * i] = pack_bf16x2(m0.x, m0.y);
+                o[2 * i + 1] = pack_bf16x2(m1.x, m1.y);
+            }
+            store_group_packed(mbase, row, j0, o);
+            continue;
+        }
         float v[32];
         unpack_f16x32(raw, v);
-        if (g < rb) {  // below the diagonal block
-            if (fast) {
+        if (g < rb) {  // below the diagonal block, steep row block
+            const float r = ex2(cl - c_first);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float4 c = ct[i];
-                    v[4 * i + 0] *= c.x;
-                    v[4 * i + 1] *= c.y;
-                    v[4 * i + 2] *= c.z;
-                    v[4 * i + 3] *= c.w;
-                }
-            } else {
-                const float r = ex2(cl - c_first);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float4 c = ct[i];
-                    v[4 * i + 0] *= r * c.x;
-                    v[4 * i + 1] *= r * c.y;
-                    v[4 * i + 2] *= r * c.z;
-                    v[4 * i + 3] *= r * c.w;
-                }
+            for (int i = 0; i < 8; ++i) {
+                const float4 c = ct[i];
+                v[4 * i + 0] *= r * c.x;
+                v[4 * i + 1] *= r * c.y;
+                v[4 * i + 2] *= r * c.z;
+                v[4 * i + 3] *= r * c.w;
             }
         } else if (fast) {  // the diagonal block, factored; j = l left to the epilogue
 #pragma unroll
@@ -572,6 +586,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             mbar_arrive(bar(B_ACC_EMPTY + t));
             if (l < Lc) {
                 const float s = ex2(cl2);
+                const float2 f2 = make_float2(fw.x, fw.x), s2 = make_float2(s, s);
+                const float2 w2 = make_float2(fw.y, fw.y);
 #pragma unroll
                 for (int k4 = 0; k4 < 2; ++k4) {
                     uint32_t o[4];
@@ -580,11 +596,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         const int e = 8 * k4 + 2 * k;
                         const float2 xf =
                             __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xw[4 * k4 + k]));
-                        const float y0 = fmaf(fw.y, xf.x, fmaf(s, __uint_as_float(r[1][e]),
-                                                              fw.x * __uint_as_float(r[0][e])));
-                        const float y1 = fmaf(fw.y, xf.y, fmaf(s, __uint_as_float(r[1][e + 1]),
-                                                              fw.x * __uint_as_float(r[0][e + 1])));
-                        o[k] = pack_bf16x2(y0, y1);
+                        const float2 vi = make_float2(__uint_as_float(r[0][e]), __uint_as_float(r[0][e + 1]));
+                        const float2 vs = make_float2(__uint_as_float(r[1][e]), __uint_as_float(r[1][e + 1]));
+                        const float2 yv = __ffma2_rn(w2, xf, __ffma2_rn(s2, vs, __fmul2_rn(f2, vi)));
+                        o[k] = pack_bf16x2(yv.x, yv.y);
                     }
                     st_shared_v4(sY + sw128(l, 2 * hf + k4), o[0], o[1], o[2], o[3]);
                 }
@@ -694,9 +709,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 // Heads per CTA: each CTA pays a fixed set-up (C and B loads, CB, its repack)
 // and then pipelines its heads, so with w waves of CTAs over the SMs the
 // kernel takes about w * (setup + heads * per_head).  The divisor of the heads
-// per group that minimises this, up to 12 heads, is used (or every head of the
-// group, when asked).  The two costs are the measured ones (in microseconds);
-// beyond about a dozen heads per CTA the measured time rises again.
+// per group that minimises this, up to 32 heads, is used (or every head of the
+// group, when asked).  The two costs are the measured ones (in microseconds;
+// the set-up includes filling and draining the head pipeline).
 int heads_per_cta(const FwdParams& p, int num_sms) {
     if (p.flags & SSD_FLAG_WHOLE_GROUPS) return static_cast<int>(p.heads_per_group);
     // tuning override: SSD_SCAN_HEADS_PER_CTA=d (used when d divides the heads per group)
@@ -706,10 +721,10 @@ int heads_per_cta(const FwdParams& p, int num_sms) {
     }();
     if (forced > 0 && p.heads_per_group % forced == 0) return forced;
     const int64_t units = p.batch * p.nchunks * p.ngroups;
-    const double setup = 5.0, per_head = 4.5;
+    const double setup = 9.0, per_head = 4.0;
     int best = 1;
     double best_t = 0.0;
-    for (int d = 1; d <= p.heads_per_group && d <= 12; ++d) {
+    for (int d = 1; d <= p.heads_per_group && d <= 32; ++d) {
         if (p.heads_per_group % d) continue;
         const int64_t ctas = units * (p.heads_per_group / d);
         const int64_t waves = (ctas + num_sms - 1) / num_sms;
