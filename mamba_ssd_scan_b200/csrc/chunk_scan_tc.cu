@@ -137,7 +137,7 @@ enum : int {
     B_CB_LOAD = 0, B_CB_DONE, B_CB_PACKED, B_X_FULL, B_H_FULL, B_H_FREE, B_X_FREE,
     B_MK_FULL, B_MK_EMPTY = B_MK_FULL + 2, B_ACC_FULL = B_MK_EMPTY + 2,
     B_ACC_EMPTY = B_ACC_FULL + 2, B_DEC_FULL = B_ACC_EMPTY + 2, B_DEC_FREE = B_DEC_FULL + 2,
-    B_Y_STAGED = B_DEC_FREE + 2, B_Y_READ, B_COUNT
+    B_Y_STAGED = B_DEC_FREE + 2, B_Y_READ, B_MK1A_FULL, B_COUNT
 };
 
 // Bounded wait that also gives up when another role has aborted: a few
@@ -205,92 +205,99 @@ __device__ __forceinline__ void store_zero_group(uint32_t mbase, uint32_t row, i
 // diagonal entry (j = l, decay 1) is left out of the operand: the epilogue
 // adds (C_l . B_l dt_l + D) x_l in fp32, so the term that is often the row's
 // largest, and the D skip, are not rounded to bf16.  cbd is the row's C_l . B_l
-// (fp32, saved when CB was packed).  Returns the row's epilogue factor f
-// (y_intra = f * accumulator) in .x and that diagonal weight in .y.
+// (fp32, saved when CB was packed).
+struct RowPlan {
+    float ref, cl, c_first;
+    float f, w;      // the row's epilogue factor and diagonal weight
+    bool fast;       // factored decays (warp-uniform)
+    int rb;          // 32-row block index of the rows
+    uint32_t row;    // TMEM lane = Mk row
+    uint32_t cbase;  // TMEM address of the rows' packed CB
+};
+
 template <int TT>
-__device__ __forceinline__ float2 build_mask(uint32_t tmem, uint32_t mbase, const float* cum2,
-                                             const float* dtv, float* ctab, float rinv, float cbd,
-                                             float Dh, int qd, int hf, int lane, int Lc, bool first) {
-    constexpr int NG = TT + 1;
+__device__ __forceinline__ RowPlan plan_rows(uint32_t tmem, const float* cum2, const float* dtv,
+                                             float rinv, float cbd, float Dh, int qd, int lane,
+                                             int Lc) {
+    RowPlan r;
     const int lb = block_row(TT, qd);
-    const int rb = lb >> 5;
-    const int l = lb + lane;
-    const uint32_t row = 32 * qd + lane;
-    const uint32_t cbase = tmem + (static_cast<uint32_t>(32 * qd) << 16) + (TT == 0 ? CB0P : CB1P);
-
-    // the block's log2 decay span picks the path (warp-uniform)
+    r.rb = lb >> 5;
+    r.row = 32 * qd + lane;
+    r.cbase = tmem + (static_cast<uint32_t>(32 * qd) << 16) + (TT == 0 ? CB0P : CB1P);
+    // the block's log2 decay span picks the path
     const int last = max(lb, min(lb + 31, Lc - 1));
-    const float c_first = cum2[lb], c_last = cum2[last];
-    const bool fast = (c_first - c_last) <= kFastSpan;
-    const float ref = fast ? 0.5f * (c_first + c_last) : c_first;
-    const float cl = cum2[l];
-    const float f = fast ? rinv * ex2(cl - ref) : rinv;
-    const float w = fmaf(cbd, dtv[l], Dh);
+    r.c_first = cum2[lb];
+    const float c_last = cum2[last];
+    r.fast = (r.c_first - c_last) <= kFastSpan;
+    r.ref = r.fast ? 0.5f * (r.c_first + c_last) : r.c_first;
+    r.cl = cum2[lb + lane];
+    r.f = r.fast ? rinv * ex2(r.cl - r.ref) : rinv;
+    r.w = fmaf(cbd, dtv[lb + lane], Dh);
+    return r;
+}
 
-#pragma unroll
-    for (int k = 0; k < NG; ++k) {
-        const int g = hf + 4 * k;
-        const int j0 = 32 * g;
-        if (g > rb) {  // above the diagonal block: zeros, kept from the first head
-            if (first) store_zero_group(mbase, row, j0);
-            continue;
-        }
-        uint32_t raw[16];
-        tmem_ld16(cbase + 16 * g, raw);
-        // this lane's column factor, shared with the warp through its table
-        const float cj = ex2(fminf(ref - cum2[j0 + lane], kMaxExp)) * dtv[j0 + lane];
-        __syncwarp();
-        ctab[lane] = cj;
-        __syncwarp();
-        const float4* ct = reinterpret_cast<const float4*>(ctab);
-        if (g < rb && fast) {  // below the diagonal block: packed fp32x2 products
-            uint32_t o[16];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float4 c = ct[i];
-                const float2 a0 = __half22float2(*reinterpret_cast<const __half2*>(&raw[2 * i]));
-                const float2 a1 = __half22float2(*reinterpret_cast<const __half2*>(&raw[2 * i + 1]));
-                const float2 m0 = __fmul2_rn(a0, make_float2(c.x, c.y));
-                const float2 m1 = __fmul2_rn(a1, make_float2(c.z, c.w));
-                o[2 * i] = pack_bf16x2(m0.x, m0.y);
-                o[2 * i + 1] = pack_bf16x2(m1.x, m1.y);
-            }
-            store_group_packed(mbase, row, j0, o);
-            continue;
-        }
-        float v[32];
-        unpack_f16x32(raw, v);
-        if (g < rb) {  // below the diagonal block, steep row block
-            const float r = ex2(cl - c_first);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float4 c = ct[i];
-                v[4 * i + 0] *= r * c.x;
-                v[4 * i + 1] *= r * c.y;
-                v[4 * i + 2] *= r * c.z;
-                v[4 * i + 3] *= r * c.w;
-            }
-        } else if (fast) {  // the diagonal block, factored; j = l left to the epilogue
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float4 c = ct[i];
-                const float cc[4] = {c.x, c.y, c.z, c.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int q = 4 * i + e;
-                    v[q] = (q < lane) ? v[q] * cc[e] : 0.0f;
-                }
-            }
-        } else {  // the diagonal block of a steep block: one exp2 per element
-#pragma unroll
-            for (int q = 0; q < 32; ++q) {
-                const float e = ex2(fminf(cl - cum2[j0 + q], 0.0f)) * dtv[j0 + q];
-                v[q] = (q < lane) ? v[q] * e : 0.0f;
-            }
-        }
-        store_group(mbase, row, j0, v);
+// One 32-column group g of the plan's rows.
+__device__ __forceinline__ void mask_group(const RowPlan& r, int g, uint32_t mbase, const float* cum2,
+                                           const float* dtv, float* ctab, int lane, bool first) {
+    const int j0 = 32 * g;
+    if (g > r.rb) {  // above the diagonal block: zeros, kept from the first head
+        if (first) store_zero_group(mbase, r.row, j0);
+        return;
     }
-    return make_float2(f, w);
+    uint32_t raw[16];
+    tmem_ld16(r.cbase + 16 * g, raw);
+    // this lane's column factor, shared with the warp through its table
+    const float cj = ex2(fminf(r.ref - cum2[j0 + lane], kMaxExp)) * dtv[j0 + lane];
+    __syncwarp();
+    ctab[lane] = cj;
+    __syncwarp();
+    const float4* ct = reinterpret_cast<const float4*>(ctab);
+    if (g < r.rb && r.fast) {  // below the diagonal block: packed fp32x2 products
+        uint32_t o[16];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float4 c = ct[i];
+            const float2 a0 = __half22float2(*reinterpret_cast<const __half2*>(&raw[2 * i]));
+            const float2 a1 = __half22float2(*reinterpret_cast<const __half2*>(&raw[2 * i + 1]));
+            const float2 m0 = __fmul2_rn(a0, make_float2(c.x, c.y));
+            const float2 m1 = __fmul2_rn(a1, make_float2(c.z, c.w));
+            o[2 * i] = pack_bf16x2(m0.x, m0.y);
+            o[2 * i + 1] = pack_bf16x2(m1.x, m1.y);
+        }
+        store_group_packed(mbase, r.row, j0, o);
+        return;
+    }
+    float v[32];
+    unpack_f16x32(raw, v);
+    if (g < r.rb) {  // below the diagonal block, steep row block
+        const float rr = ex2(r.cl - r.c_first);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float4 c = ct[i];
+            v[4 * i + 0] *= rr * c.x;
+            v[4 * i + 1] *= rr * c.y;
+            v[4 * i + 2] *= rr * c.z;
+            v[4 * i + 3] *= rr * c.w;
+        }
+    } else if (r.fast) {  // the diagonal block, factored; j = l left to the epilogue
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float4 c = ct[i];
+            const float cc[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int q = 4 * i + e;
+                v[q] = (q < lane) ? v[q] * cc[e] : 0.0f;
+            }
+        }
+    } else {  // the diagonal block of a steep block: one exp2 per element
+#pragma unroll
+        for (int q = 0; q < 32; ++q) {
+            const float e = ex2(fminf(r.cl - cum2[j0 + q], 0.0f)) * dtv[j0 + q];
+            v[q] = (q < lane) ? v[q] * e : 0.0f;
+        }
+    }
+    store_group(mbase, r.row, j0, v);
 }
 
 // Per-head MMAs, issued by the control thread.  Descriptors are built once;
@@ -305,14 +312,16 @@ __device__ __forceinline__ void issue_state(uint32_t d_tmem, uint64_t dA, uint64
         mma_bf16(d_tmem, dA + ka, dB + kb, idesc_bf16(128, PD, false, false), k > 0 ? 1u : 0u);
     }
 }
-// Intra-chunk term of one tile: Mk_t (K-major, KS * 16 wide) x x (MN-major).
-template <int KS>
+// Intra-chunk term of one tile: Mk_t (K-major) x x (MN-major), K steps
+// [K0, K1) of 16; FRESH: the first of them overwrites the accumulator.
+template <int K0, int K1, bool FRESH>
 __device__ __forceinline__ void issue_intra(uint32_t d_tmem, uint64_t dA, uint64_t dB) {
 #pragma unroll
-    for (int k = 0; k < KS; ++k) {
+    for (int k = K0; k < K1; ++k) {
         const uint32_t ka = ((k >> 2) * (128 * 128) + (k & 3) * 32) >> 4;
         const uint32_t kb = (k * 2048) >> 4;
-        mma_bf16(d_tmem, dA + ka, dB + kb, idesc_bf16(128, PD, false, true), k > 0 ? 1u : 0u);
+        mma_bf16(d_tmem, dA + ka, dB + kb, idesc_bf16(128, PD, false, true),
+                 (FRESH && k == K0) ? 0u : 1u);
     }
 }
 
@@ -354,7 +363,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             uint32_t count = 1;
             if (i == B_CB_PACKED) count = 256;  // the packing warps (two per lane quarter)
             if (i == B_MK_FULL || i == B_MK_FULL + 1 || i == B_ACC_EMPTY || i == B_ACC_EMPTY + 1 ||
-                i == B_DEC_FREE || i == B_DEC_FREE + 1 || i == B_Y_STAGED)
+                i == B_DEC_FREE || i == B_DEC_FREE + 1 || i == B_Y_STAGED || i == B_MK1A_FULL)
                 count = NMASK;
             if (i == B_DEC_FULL || i == B_DEC_FULL + 1) count = 32;
             mbar_init(bar(i), count);
@@ -452,8 +461,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     if (ok && t == 0) ok = wait_bar(bar(B_X_FULL), ph, abort);
                     if (!ok) break;
                     fence_after_sync();
-                    if (t == 0) issue_intra<8>(tmem + in_col(0), dM0, dX);
-                    else issue_intra<16>(tmem + in_col(1), dM1, dX);
+                    if (t == 0) {
+                        issue_intra<0, 8, true>(tmem + in_col(0), dM0, dX);
+                    } else {
+                        // tile 1's mask arrives in two halves: K columns
+                        // 128-255 first, then 0-127
+                        issue_intra<8, 16, true>(tmem + in_col(1), dM1, dX);
+                        ok = wait_bar(bar(B_MK1A_FULL), ph, abort);
+                        if (!ok) break;
+                        fence_after_sync();
+                        issue_intra<0, 8, false>(tmem + in_col(1), dM1, dX);
+                    }
                     mma_commit(bar(B_ACC_FULL + t));
                     mma_commit(bar(B_MK_EMPTY + t));
                     SCAN_TRACE(11 + 8 * i + 3 * t);
@@ -648,10 +666,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (i > 0) ok = wait_bar(bar(B_MK_EMPTY), (i - 1) & 1, abort);
                 if (warp == 0 && lane == 0) SCAN_TRACE(83 + 5 * i);
                 if (ok) {
-                    fw_cur[0] = build_mask<0>(tmem, sM0, dec, dec + QMAX, ctab, rinv0, cbd0, Dh, qd,
-                                              hf, lane, Lc, i == 0);
+                    const RowPlan r0 = plan_rows<0>(tmem, dec, dec + QMAX, rinv0, cbd0, Dh, qd, lane, Lc);
+                    mask_group(r0, hf, sM0, dec, dec + QMAX, ctab, lane, i == 0);
+                    fw_cur[0] = make_float2(r0.f, r0.w);
                     fence_smem_async();
-                    // the last tile's mask is released only after the x stash
+                    // a single tile's mask is released only after the x stash
                     if (ntiles == 2) mbar_arrive(bar(B_MK_FULL));
                 }
                 if (warp == 0 && lane == 0) SCAN_TRACE(84 + 5 * i);
@@ -668,6 +687,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     mbar_arrive(bar(B_Y_STAGED));
                 }
             }
+            RowPlan r1;
+            if (mask_now && ok && ntiles == 2) {
+                // tile 1, K columns 128-255 (clear of the y staging area)
+                r1 = plan_rows<1>(tmem, dec, dec + QMAX, rinv1, cbd1, Dh, qd, lane, Lc);
+                mask_group(r1, hf + 4, sM1, dec, dec + QMAX, ctab, lane, i == 0);
+                fw_cur[1] = make_float2(r1.f, r1.w);
+                fence_smem_async();
+                mbar_arrive(bar(B_MK_FULL + 1));
+                if (warp == 0 && lane == 0 && i < 16) SCAN_TRACE(240 + i);
+            }
             if (mask_now && ok) {
                 ok = wait_bar(bar(B_X_FULL), i & 1, abort);
                 if (warp == 0 && lane == 0) SCAN_TRACE(200 + 2 * i);
@@ -676,13 +705,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (ok && ntiles == 1) mbar_arrive(bar(B_MK_FULL));
             }
             if (mask_now && ok && ntiles == 2) {
-                if (i > 0) ok = wait_bar(bar(B_Y_READ), (i - 1) & 1, abort);  // staged y stored
+                // tile 1, K columns 0-127, once the staged y has been stored
+                if (i > 0) ok = wait_bar(bar(B_Y_READ), (i - 1) & 1, abort);
                 if (warp == 0 && lane == 0) SCAN_TRACE(85 + 5 * i);
                 if (ok) {
-                    fw_cur[1] = build_mask<1>(tmem, sM1, dec, dec + QMAX, ctab, rinv1, cbd1, Dh, qd,
-                                              hf, lane, Lc, i == 0);
+                    mask_group(r1, hf, sM1, dec, dec + QMAX, ctab, lane, i == 0);
                     fence_smem_async();
-                    mbar_arrive(bar(B_MK_FULL + 1));
+                    mbar_arrive(bar(B_MK1A_FULL));
                 }
                 if (warp == 0 && lane == 0) SCAN_TRACE(86 + 5 * i);
             }
