@@ -390,6 +390,8 @@ def main_ours(args):
 KERNEL_SOURCES = {
     "chunk_scan": ["chunk_scan_tc.cu", "tcgen05.cuh", "tma.cuh", "internal.cuh"],
     "chunk_state": ["chunk_state_tc.cu", "tcgen05.cuh", "tma.cuh", "internal.cuh"],
+    "state_passing": ["state_passing.cu", "internal.cuh"],
+    "chunk_cumsum": ["chunk_cumsum.cu", "internal.cuh"],
 }
 
 
