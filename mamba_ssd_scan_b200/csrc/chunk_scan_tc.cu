@@ -110,7 +110,8 @@ struct ScanTile {
     static constexpr int DEC_OFF = H_OFF + H_BYTES;
     static constexpr int RINV_OFF = DEC_OFF + 2 * DEC_FLOATS * 4;  // per-row CB scale, 2 tiles
     static constexpr int CBD_OFF = RINV_OFF + 2 * 128 * 4;   // per-row C_l . B_l, 2 tiles
-    static constexpr int CTAB_OFF = CBD_OFF + 2 * 128 * 4;   // per worker warp: 32 column factors
+    static constexpr int NORM_OFF = CBD_OFF + 2 * 128 * 4;   // |C_r|^2 per row, max |B_j|^2 partials
+    static constexpr int CTAB_OFF = NORM_OFF + (256 + 8) * 4;  // per worker warp: 32 column factors
     static constexpr int BAR_OFF = CTAB_OFF + NWORK * 32 * 4;
     static constexpr int SMEM = BAR_OFF + 32 * 8 + 1024;
     static_assert(SMEM <= 232448, "shared memory budget");
@@ -361,7 +362,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     if (tid == 0) {
         for (int i = 0; i < B_COUNT; ++i) {
             uint32_t count = 1;
-            if (i == B_CB_PACKED) count = 256;  // the packing warps (two per lane quarter)
+            if (i == B_CB_PACKED) count = NMASK;
             if (i == B_MK_FULL || i == B_MK_FULL + 1 || i == B_ACC_EMPTY || i == B_ACC_EMPTY + 1 ||
                 i == B_DEC_FREE || i == B_DEC_FREE + 1 || i == B_Y_STAGED || i == B_MK1A_FULL)
                 count = NMASK;
@@ -541,45 +542,102 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         float* cbd_s = reinterpret_cast<float*>(smem + T::CBD_OFF);
         float* ctab = reinterpret_cast<float*>(smem + T::CTAB_OFF) + warp * 32;
         const uint32_t lanes = static_cast<uint32_t>(32 * qd) << 16;
-        bool ok = wait_bar(bar(B_CB_DONE), 0, abort);
-        if (hf < 2) {
-            // repack tile hf's CB as fp16 pairs with a per-row power-of-two
-            // scale: tile 0 [0,128) -> [0,64), tile 1 [256,512) -> [128,256)
-            const int t = hf;
-            if (ok && t < ntiles) {
-                fence_after_sync();
-                const uint32_t src = t == 0 ? 0u : CB1F, dst = t == 0 ? CB0P : CB1P;
-                const int rb = block_row(t, qd) >> 5;  // the 32 columns holding this row's diagonal
-                float mx = 0.0f, dg = 0.0f;
-                for (int k = 0; k < 4 * (t + 1); ++k) {
-                    float v[32];
-                    tmem_ld32(tmem + lanes + src + 32 * k, v);
+        // CB is repacked as fp16 pairs with a power-of-two scale per row,
+        // chosen from |C_l . B_j| <= |C_l| max_j |B_j| (norms of the C and B
+        // rows in shared memory, taken while the CB MMA runs) so that the
+        // packed row stays below 2^15.  All sixteen workers repack in one pass:
+        // tile 1's fp32 [256,512) -> [128,256); tile 0's [0,128) -> [0,64) in
+        // place, loaded by every warp before any warp stores.
+        float* cn_s = reinterpret_cast<float*>(smem + T::NORM_OFF);
+        float* bn_s = cn_s + 256;
+        bool ok = wait_bar(bar(B_CB_LOAD), 0, abort);
+        if (ok) {
+            const int r = 32 * (warp & 7) + lane;           // warps 0-7: C rows, 8-15: B rows
+            const bool is_c = warp < 8;
+            const bool valid = is_c ? r < 128 * ntiles : r < Q;
+            const uint32_t base = (is_c ? sC : sB) + r * 128;
+            float ss = 0.0f;
+            if (valid) {
 #pragma unroll
-                    for (int q = 0; q < 32; ++q) mx = fmaxf(mx, fabsf(v[q]));
-                    if (k == rb) {
+                for (int kb = 0; kb < NST / 64; ++kb)
+#pragma unroll
+                    for (int c16 = 0; c16 < 8; ++c16) {  // the row's 128 bytes, rotated by lane
+                        const uint4 v = ld_shared_v4(base + kb * T::KB_BYTES + ((c16 + lane) & 7) * 16);
+                        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[e]));
+                            ss = fmaf(f.x, f.x, fmaf(f.y, f.y, ss));
+                        }
+                    }
+            }
+            if (is_c) {
+                cn_s[r] = ss;
+            } else {
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) ss = fmaxf(ss, __shfl_xor_sync(0xffffffffu, ss, o));
+                if (lane == 0) bn_s[warp - 8] = ss;
+            }
+        }
+        named_sync(1, NMASK);
+        float sc_t[2] = {1.0f, 1.0f};
+        if (ok) {
+            float bmax = 0.0f;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) bmax = fmaxf(bmax, bn_s[k]);
+            for (int t = 0; t < ntiles; ++t) {
+                const int rr = 128 * t + 32 * qd + lane;    // TMEM lane = C row in shared memory
+                const float bound = sqrtf(cn_s[rr] * bmax);
+                // 2^e with bound * 2^-e below 2^14 (fp16 holds up to 65504)
+                const int e2 = max(0, ((__float_as_int(bound) >> 23) & 255) - 127 - 13 + 1);
+                sc_t[t] = __int_as_float((127 - e2) << 23);
+                if (hf == 0) rinv_s[rr] = __int_as_float((127 + e2) << 23);
+            }
+        }
+        if (ok) ok = wait_bar(bar(B_CB_DONE), 0, abort);
+        uint32_t r0[16];
+        if (ok) {
+            fence_after_sync();
+            if (ntiles == 2) {
+                const int rb1 = block_row(1, qd) >> 5;
+#pragma unroll
+                for (int k = 0; k < 2; ++k) {
+                    const int kk = hf + 4 * k;
+                    float v[32];
+                    uint32_t r1[16];
+                    tmem_ld32(tmem + lanes + CB1F + 32 * kk, v);
+                    if (kk == rb1) {
+                        float dg = 0.0f;
 #pragma unroll
                         for (int q = 0; q < 32; ++q) dg = (q == lane) ? v[q] : dg;
+                        cbd_s[128 + 32 * qd + lane] = dg;
                     }
-                }
-                cbd_s[t * 128 + 32 * qd + lane] = dg;
-                // 2^e with the row's largest |CB| * 2^-e below 2^15
-                const int e2 = max(0, ((__float_as_int(mx) >> 23) & 255) - 127 - 14 + 1);
-                const float sc = __int_as_float((127 - e2) << 23);
-                rinv_s[t * 128 + 32 * qd + lane] = __int_as_float((127 + e2) << 23);
-                for (int k = 0; k < 4 * (t + 1); ++k) {
-                    float v[32];
-                    uint32_t r[16];
-                    tmem_ld32(tmem + lanes + src + 32 * k, v);
 #pragma unroll
-                    for (int q = 0; q < 16; ++q) r[q] = pack_f16x2(v[2 * q] * sc, v[2 * q + 1] * sc);
-                    tmem_st16(tmem + lanes + dst + 16 * k, r);
+                    for (int q = 0; q < 16; ++q) r1[q] = pack_f16x2(v[2 * q] * sc_t[1], v[2 * q + 1] * sc_t[1]);
+                    tmem_st16(tmem + lanes + CB1P + 16 * kk, r1);
                 }
-                tmem_wait_st();
             }
-            fence_before_sync();
-            mbar_arrive(bar(B_CB_PACKED));
-            if (warp == 0 && lane == 0) SCAN_TRACE(80);
+            float v[32];
+            tmem_ld32(tmem + lanes + 32 * hf, v);
+            if (hf == (block_row(0, qd) >> 5)) {
+                float dg = 0.0f;
+#pragma unroll
+                for (int q = 0; q < 32; ++q) dg = (q == lane) ? v[q] : dg;
+                cbd_s[32 * qd + lane] = dg;
+            }
+#pragma unroll
+            for (int q = 0; q < 16; ++q) r0[q] = pack_f16x2(v[2 * q] * sc_t[0], v[2 * q + 1] * sc_t[0]);
         }
+        fence_before_sync();
+        named_sync(2, NMASK);  // every warp has read its part of tile 0's fp32 CB
+        fence_after_sync();
+        if (ok) {
+            tmem_st16(tmem + lanes + CB0P + 16 * hf, r0);
+            tmem_wait_st();
+        }
+        fence_before_sync();
+        mbar_arrive(bar(B_CB_PACKED));
+        if (warp == 0 && lane == 0) SCAN_TRACE(80);
         if (ok) ok = wait_bar(bar(B_CB_PACKED), 0, abort);
         fence_after_sync();
         const float rinv0 = ok ? rinv_s[32 * qd + lane] : 1.0f;
