@@ -9,12 +9,14 @@
 // Both operands are MN-major and arrive by TMA exactly as they sit in memory:
 // A is x viewed as 64-element units (for a token, the 128/P heads' P values
 // are two contiguous units), B the group's B rows.  The chunk streams through
-// a two-slot ring of 64-token quarters (load and free mbarriers per slot); the
-// CUDA cores fold the decay weight into a quarter of x in place (bf16 -> fp32
-// -> bf16) while the tensor core multiplies the previous one, and the next
-// quarter's TMA is issued as soon as its slot's MMAs have completed.  With
-// 64 KB of shared memory (dstate 128) three CTAs share an SM, so one CTA's
-// loads overlap another's MMAs and epilogue.  The epilogue moves the fp32
+// a two-slot ring of 64-token quarters.  Warps 0-7 fold the decay weight into
+// a quarter of x in place (bf16 -> fp32 -> bf16) as soon as it has landed;
+// one lane of warp 8 issues the quarter's MMAs once it is scaled and refills
+// the slot by TMA as soon as those MMAs are done, so loads stay in flight
+// while the previous quarter is scaled and multiplied (mbarriers per slot:
+// loaded, scaled, free).  With 64 KB of shared memory (dstate 128) three CTAs
+// share an SM, so one CTA's loads overlap another's MMAs and epilogue.  The
+// epilogue moves the fp32
 // accumulator from TMEM to the states buffer in the input dtype (bf16), one
 // row of dstate per thread.  When the forward call fuses step 1, the first
 // 128/P warps first form dt and cumA of the CTA's heads with the same warp
@@ -31,6 +33,9 @@ using namespace tc;
 constexpr int KT = 64;      // tokens per quarter
 constexpr int NSLOT = 2;    // ring slots
 constexpr int QMAX = 256;
+constexpr int NSCALE = 256;             // scaler / epilogue threads (warps 0-7)
+constexpr int NTHR = NSCALE + 32;       // + the control warp
+enum : int { B_LOADED = 0, B_SCALED = NSLOT, B_FREE = 2 * NSLOT, B_DONE = 3 * NSLOT, B_NBARS };
 
 template <int NST, int PD>
 struct StateTile {
@@ -43,7 +48,7 @@ struct StateTile {
     static constexpr int TMEM_COLS = NST;                // 64, 128 or 256
     static constexpr int W_OFF = NSLOT * SLOT;           // decay weights [HPC][QMAX] fp32
     static constexpr int BAR_OFF = W_OFF + HPC * QMAX * 4;
-    static constexpr int SMEM = BAR_OFF + 128 + 1024;    // + alignment slack
+    static constexpr int SMEM = BAR_OFF + B_NBARS * 8 + 16 + 1024;  // + alignment slack
     static_assert(SMEM <= 232448, "shared memory budget");
 };
 
@@ -57,18 +62,28 @@ __device__ __forceinline__ uint4 scale_bf16x8(uint4 v, float w) {
     return make_uint4(out[0], out[1], out[2], out[3]);
 }
 
+// Bounded mbarrier wait that also gives up when another role has aborted.
+__device__ __forceinline__ bool wait_or_abort(uint32_t mbar, uint32_t parity, volatile int* abort) {
+    for (uint32_t i = 0; i < kSpinLimit; ++i) {
+        if (mbar_try_wait_hint(mbar, parity, 200)) return true;
+        if ((i & 63) == 63 && *abort) return false;
+    }
+    *abort = 1;
+    return false;
+}
+
 template <int NST, int PD>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(NTHR, NST == 256 ? 2 : 3)  // CTAs per SM that fit
     chunk_state_tc_kernel(const __grid_constant__ FwdParams p,
                           const __grid_constant__ CUtensorMap tm_x,
                           const __grid_constant__ CUtensorMap tm_b) {
     using T = StateTile<NST, PD>;
     extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                               ~static_cast<uintptr_t>(1023));
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     float* wtab = reinterpret_cast<float*>(smem + T::W_OFF);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + T::BAR_OFF);  // load[2], free[2]
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * NSLOT);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + T::BAR_OFF);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + B_NBARS);
+    volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t H = p.nheads, L = p.seqlen, Q = p.chunk, nc = p.nchunks;
@@ -79,117 +94,130 @@ __global__ void __launch_bounds__(256, 1)
     const int Lc = static_cast<int>((L - t0 < Q) ? (L - t0) : Q);
     const int nq = (Lc + KT - 1) / KT;
     const uint32_t s0 = smem_u32(smem);
-    auto bar = [&](int i) { return smem_u32(&bars[i]); };  // 0,1 = loaded; 2,3 = free
+    auto bar = [&](int i) { return smem_u32(&bars[i]); };
     const int unit0 = static_cast<int>(h0 * PD / 64);     // x in 64-element units
-    // quarter q -> slot q % 2: A blocks then B blocks
+    // quarter q -> slot q % NSLOT: A blocks then B blocks
     auto issue = [&](int q) {
-        const uint32_t sl = s0 + (q & 1) * T::SLOT;
-        mbar_expect_tx(bar(q & 1), T::SLOT);
+        const int sl = q % NSLOT;
+        const uint32_t sa = s0 + sl * T::SLOT;
+        mbar_expect_tx(bar(B_LOADED + sl), T::SLOT);
         for (int blk = 0; blk < 2; ++blk)
-            tma_load_4d(sl + blk * T::A_BLK, &tm_x, bar(q & 1), 0, unit0 + blk,
+            tma_load_4d(sa + blk * T::A_BLK, &tm_x, bar(B_LOADED + sl), 0, unit0 + blk,
                         static_cast<int>(t0 + q * KT), static_cast<int>(b));
         for (int nb = 0; nb < NST / 64; ++nb)
-            tma_load_4d(sl + T::A_BYTES + nb * T::B_BLK, &tm_b, bar(q & 1), nb * 64,
+            tma_load_4d(sa + T::A_BYTES + nb * T::B_BLK, &tm_b, bar(B_LOADED + sl), nb * 64,
                         static_cast<int>(g), static_cast<int>(t0 + q * KT), static_cast<int>(b));
     };
 
     if (warp == 0) tmem_alloc(smem_u32(tmem_slot), T::TMEM_COLS);
     if (tid == 0) {
-        for (int i = 0; i < 2 * NSLOT; ++i) mbar_init(bar(i), 1);
+        for (int i = 0; i < B_NBARS; ++i)
+            mbar_init(bar(i), (i >= B_SCALED && i < B_SCALED + NSLOT) ? NSCALE : 1u);
+        *abort = 0;
         fence_mbar_init();
-        tma_prefetch_map(&tm_x);
-        tma_prefetch_map(&tm_b);
-    }
-    __syncthreads();
-    if (tid == 0)
-        for (int q = 0; q < nq && q < NSLOT; ++q) issue(q);
-    // x and B are inputs; dt and cumA are formed here (step 1 fused, one warp
-    // per head) or come from step 1
-    grid_dep_wait();
-    if (p.fuse_cumsum) {
-        if (warp < T::HPC) {
-            const int64_t off = ((b * H + h0 + warp) * nc + c) * Q;
-            chunk_cumsum_warp<__nv_bfloat16>(p, b, c, h0 + warp, p.dt + off, p.cumA + off, lane);
-        }
-        if (blockIdx.x == 0 && blockIdx.y == 0 && tid == 0 && p.status) *p.status = 0;  // a new call
-        __syncthreads();
-    }
-    grid_dep_launch();
-    for (int i = tid; i < T::HPC * QMAX; i += 256) {
-        const int hh = i / QMAX, l = i % QMAX;
-        float w = 0.0f;
-        if (l < Lc) {
-            const int64_t base = ((b * H + h0 + hh) * nc + c) * Q;
-            w = expf(p.cumA[base + Q - 1] - p.cumA[base + l]) * p.dt[base + l];
-        }
-        wtab[i] = w;
     }
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
     const uint32_t tmem = *tmem_slot;
 
-    constexpr uint32_t idesc = idesc_bf16(128, NST, true, true);
-    bool ok = true, mine = true;  // mine: thread 0's refill waits
-    for (int q = 0; q < nq && ok; ++q) {
-        const int sl = q & 1, use = q >> 1;
-        const uint32_t sA = s0 + sl * T::SLOT, sB = sA + T::A_BYTES;
-        ok = !__syncthreads_or(!(mine && mbar_wait(bar(sl), use & 1)));
-        if (!ok) break;
-        // fold the decay weights into this quarter of x: 2 blocks x 64 rows x 8 chunks
+    if (warp == NSCALE / 32) {
+        // ----- control: TMA ring producer and MMA issuer (one lane) -----
+        if (lane == 0) {
+            tma_prefetch_map(&tm_x);
+            tma_prefetch_map(&tm_b);
+            for (int q = 0; q < nq && q < NSLOT; ++q) issue(q);  // x and B are inputs
+            constexpr uint32_t idesc = idesc_bf16(128, NST, true, true);
+            bool ok = true;
+            for (int q = 0; ok && q < nq; ++q) {
+                const int sl = q % NSLOT, use = q / NSLOT;
+                const uint32_t sa = s0 + sl * T::SLOT, sb = sa + T::A_BYTES;
+                ok = wait_or_abort(bar(B_SCALED + sl), use & 1, abort);
+                if (!ok) break;
+                fence_after_sync();
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int i = tid + 256 * k;
-            const int blk = i >> 9, r = (i >> 3) & 63, ch = i & 7;
-            const uint32_t addr = sA + blk * T::A_BLK + sw128(r, ch);
-            const int hh = (blk * 64 + ch * 8) / PD;
-            const uint4 v = ld_shared_v4(addr);
-            const uint4 o = scale_bf16x8(v, wtab[hh * QMAX + q * KT + r]);
-            st_shared_v4(addr, o.x, o.y, o.z, o.w);
+                for (int k = 0; k < KT / 16; ++k)
+                    mma_bf16(tmem, desc_sw128(sa + k * 2048, T::A_BLK, 1024),
+                             desc_sw128(sb + k * 2048, T::B_BLK, 1024), idesc,
+                             (q > 0 || k > 0) ? 1u : 0u);
+                mma_commit(bar(B_FREE + sl));
+                if (q + NSLOT < nq) {  // refill this slot once its MMAs are done
+                    ok = wait_or_abort(bar(B_FREE + sl), use & 1, abort);
+                    if (ok) issue(q + NSLOT);
+                }
+            }
+            if (ok) mma_commit(bar(B_DONE));
+            else *abort = 1;
         }
-        fence_smem_async();
-        __syncthreads();
-        if (tid == 0) {
-            fence_after_sync();
+    } else {
+        // ----- scalers (warps 0-7): decay weights, x scaling, epilogue -----
+        grid_dep_wait();  // dt and cumA are formed here (step 1 fused) or come from step 1
+        if (p.fuse_cumsum) {
+            if (warp < T::HPC) {
+                const int64_t off = ((b * H + h0 + warp) * nc + c) * Q;
+                chunk_cumsum_warp<__nv_bfloat16>(p, b, c, h0 + warp, p.dt + off, p.cumA + off, lane);
+            }
+            if (blockIdx.x == 0 && blockIdx.y == 0 && tid == 0 && p.status) *p.status = 0;  // a new call
+            named_sync(1, NSCALE);
+        }
+        grid_dep_launch();
+        for (int i = tid; i < T::HPC * QMAX; i += NSCALE) {
+            const int hh = i / QMAX, l = i % QMAX;
+            float w = 0.0f;
+            if (l < Lc) {
+                const int64_t base = ((b * H + h0 + hh) * nc + c) * Q;
+                w = expf(p.cumA[base + Q - 1] - p.cumA[base + l]) * p.dt[base + l];
+            }
+            wtab[i] = w;
+        }
+        named_sync(1, NSCALE);
+        bool ok = true;
+        for (int q = 0; q < nq; ++q) {
+            const int sl = q % NSLOT, use = q / NSLOT;
+            const uint32_t sa = s0 + sl * T::SLOT;
+            ok = wait_or_abort(bar(B_LOADED + sl), use & 1, abort);
+            if (!ok) break;
+            // fold the decay weights into this quarter of x: 2 blocks x 64 rows x 8 chunks
 #pragma unroll
-            for (int k = 0; k < KT / 16; ++k)
-                mma_bf16(tmem, desc_sw128(sA + k * 2048, T::A_BLK, 1024),
-                         desc_sw128(sB + k * 2048, T::B_BLK, 1024), idesc,
-                         (q > 0 || k > 0) ? 1u : 0u);
-            mma_commit(bar(2 + sl));
-            if (q + NSLOT < nq) {  // refill this slot once its MMAs are done
-                mine = mbar_wait(bar(2 + sl), use & 1);
-                if (mine) issue(q + NSLOT);
+            for (int k = 0; k < 4; ++k) {
+                const int i = tid + NSCALE * k;
+                const int blk = i >> 9, r = (i >> 3) & 63, ch = i & 7;
+                const uint32_t addr = sa + blk * T::A_BLK + sw128(r, ch);
+                const int hh = (blk * 64 + ch * 8) / PD;
+                const uint4 v = ld_shared_v4(addr);
+                const uint4 o = scale_bf16x8(v, wtab[hh * QMAX + q * KT + r]);
+                st_shared_v4(addr, o.x, o.y, o.z, o.w);
+            }
+            fence_smem_async();
+            mbar_arrive(bar(B_SCALED + sl));
+        }
+        if (ok) ok = wait_or_abort(bar(B_DONE), 0, abort);
+        fence_after_sync();
+        if (ok) {
+            // warp w reads TMEM lanes 32*(w%4).. (rows m), warpgroup w/4 half the columns
+            const int m = 32 * (warp & 3) + lane;
+            const int64_t hh = m / PD, pp = m % PD;
+            __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.states) +
+                                 (((b * nc + c) * H + h0 + hh) * PD + pp) * NST;
+            constexpr int HALF = NST / 2;
+            const int cbeg = (warp >> 2) * HALF;
+#pragma unroll
+            for (int col = 0; col < HALF; col += 32) {
+                float v[32];
+                tmem_ld32(tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + cbeg + col, v);
+                uint4* o = reinterpret_cast<uint4*>(out + cbeg + col);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    o[k] = make_uint4(pack_bf16x2(v[8 * k], v[8 * k + 1]),
+                                      pack_bf16x2(v[8 * k + 2], v[8 * k + 3]),
+                                      pack_bf16x2(v[8 * k + 4], v[8 * k + 5]),
+                                      pack_bf16x2(v[8 * k + 6], v[8 * k + 7]));
             }
         }
     }
-    if (ok) ok = !__syncthreads_or(!mbar_wait(bar(2 + ((nq - 1) & 1)), ((nq - 1) >> 1) & 1));
-    fence_after_sync();
-    if (ok) {
-        // warp w reads TMEM lanes 32*(w%4).. (rows m), warpgroup w/4 half the columns
-        const int m = 32 * (warp & 3) + lane;
-        const int64_t hh = m / PD, pp = m % PD;
-        __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.states) +
-                             (((b * nc + c) * H + h0 + hh) * PD + pp) * NST;
-        constexpr int HALF = NST / 2;
-        const int cbeg = (warp >> 2) * HALF;
-#pragma unroll
-        for (int col = 0; col < HALF; col += 32) {
-            float v[32];
-            tmem_ld32(tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + cbeg + col, v);
-            uint4* o = reinterpret_cast<uint4*>(out + cbeg + col);
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-                o[k] = make_uint4(pack_bf16x2(v[8 * k], v[8 * k + 1]),
-                                  pack_bf16x2(v[8 * k + 2], v[8 * k + 3]),
-                                  pack_bf16x2(v[8 * k + 4], v[8 * k + 5]),
-                                  pack_bf16x2(v[8 * k + 6], v[8 * k + 7]));
-        }
-    } else if (tid == 0 && p.status) {
-        atomicExch(p.status, static_cast<int>(SSD_ERR_TIMEOUT));
-    }
     fence_before_sync();
     __syncthreads();
+    if (*abort && tid == 0 && p.status) atomicExch(p.status, static_cast<int>(SSD_ERR_TIMEOUT));
     if (warp == 0) {
         fence_after_sync();
         tmem_dealloc(tmem, T::TMEM_COLS);
@@ -207,7 +235,7 @@ cudaError_t launch_nd(const FwdParams& p, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, T::SMEM);
     if (e != cudaSuccess) return e;
     dim3 grid(static_cast<unsigned>(p.nchunks * (p.nheads / T::HPC)), static_cast<unsigned>(p.batch));
-    return launch_kernel(kern, grid, dim3(256), T::SMEM, s, p.pdl != 0, p, tx_, tb_);
+    return launch_kernel(kern, grid, dim3(NTHR), T::SMEM, s, p.pdl != 0, p, tx_, tb_);
 }
 
 }  // namespace
