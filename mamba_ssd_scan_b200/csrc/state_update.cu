@@ -7,12 +7,15 @@
 //   h[p,n] <- a h[p,n] + dt x[p] B[n];   y[p] = sum_n h[p,n] C[n] + D_h x[p]
 //
 // Bandwidth-bound: the state is read once and written once, in place.  One
-// CTA owns one (batch, head) state tile [P x N]; a state row is spread over
-// TPR lanes holding 4 V consecutive floats each, a warp covers RPW rows per
-// pass, and every thread issues the 16-byte loads of all its passes (up to
-// MAXPASS) before any arithmetic, so an SM keeps ~128 KB of state reads in
-// flight.  The state stream is marked evict-first (ld/st .cs) so it does not
-// push B/C/x out of L2.  dt, the decay and B/C are computed or loaded once per
+// CTA of four warps owns one (batch, head) state tile [P x N]; a state row is
+// spread over TPR lanes holding 4 V consecutive floats each, a warp covers
+// RPW rows per pass, and every thread issues the 16-byte loads of MAXPASS
+// passes before their arithmetic.  Four passes keep the kernel at 55
+// registers, so many small CTAs share an SM and one CTA's loads overlap
+// another's stores (measured: 4 passes x 128 threads streams at the copy
+// bandwidth; 8 passes x 256 threads, at 86 registers, reached 74% of it).
+// The state stream is marked evict-first (ld/st .cs) so it does not push
+// B/C/x out of L2.  dt, the decay and B/C are computed or loaded once per
 // thread, and the C-dot of each row is reduced with xor shuffles inside its
 // lane group.
 #include "internal.cuh"
@@ -36,14 +39,15 @@ template <> struct Vec4<__nv_bfloat16> {
     }
 };
 
-constexpr int MAXPASS = 8;
+constexpr int MAXPASS = 4;
+constexpr int NTHREADS = 128;
 
 template <typename T, int N>
-__global__ void __launch_bounds__(256) state_update_kernel(DecodeParams p) {
+__global__ void __launch_bounds__(NTHREADS) state_update_kernel(DecodeParams p) {
     constexpr int TPR = (N / 4 < 32) ? N / 4 : 32;  // threads per state row
     constexpr int V = N / (4 * TPR);                // float4s per thread per row
     constexpr int RPW = 32 / TPR;                   // rows per warp per pass
-    constexpr int RPP = 8 * RPW;                    // rows per CTA pass
+    constexpr int RPP = (NTHREADS / 32) * RPW;      // rows per CTA pass
     static_assert(TPR * V * 4 == N && RPW * TPR == 32, "bad tiling");
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -112,7 +116,7 @@ __global__ void __launch_bounds__(256) state_update_kernel(DecodeParams p) {
 
 template <typename T, int N>
 cudaError_t launch_n(const DecodeParams& p, cudaStream_t s) {
-    state_update_kernel<T, N><<<static_cast<unsigned>(p.batch * p.nheads), 256, 0, s>>>(p);
+    state_update_kernel<T, N><<<static_cast<unsigned>(p.batch * p.nheads), NTHREADS, 0, s>>>(p);
     return cudaGetLastError();
 }
 
