@@ -478,10 +478,75 @@ def roofline_entry(name, cost, ms, peaks, clk, on_tensor_cores, workload):
             "compute_frac": (flops / sec / 1e12) / cpeak if flops else 0.0}
 
 
+def launch_timing(ssd, synthetic, dev, flush, name, rank, steps=200):
+    """Per-step device time of a small workload three ways: L2 flushed before
+    each step, warm (back to back), and replayed from a CUDA graph holding one
+    step (launch latency left out)."""
+    import torch
+    cfg = synthetic.FWD_CONFIGS[name]
+    inp = synthetic.make_config_inputs(cfg, rank_seed(1234 + synthetic.SEED_OFFSET[name], rank))
+    d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
+    y = torch.empty_like(d["x"])
+    fin = (torch.empty((cfg.batch, cfg.nheads, cfg.headdim, cfg.dstate), device=dev)
+           if cfg.return_final else None)
+    ws = torch.empty(ssd.ssd_fwd_workspace_size(cfg.batch, cfg.seqlen, cfg.nheads, cfg.headdim,
+                                                cfg.dstate, cfg.ngroups, cfg.chunk, cfg.dtype),
+                     dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        ssd.ssd_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["dt_bias"], cfg.chunk,
+                    d["init_state"], y=y, final_state=fin, workspace=ws)
+
+    def timed(with_flush):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)]
+        torch.cuda.synchronize()
+        gpu_head_start(0.2 * steps)
+        for a, b_ in evs:
+            if with_flush:
+                flush()
+            a.record(stream)
+            step()
+            b_.record(stream)
+        torch.cuda.synchronize()
+        return sum(a.elapsed_time(b_) for a, b_ in evs) / steps * 1e3
+
+    for _ in range(3):
+        step()
+    res = {"flushed_us": timed(True), "warm_us": timed(False)}
+    try:
+        side = torch.cuda.Stream()
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            step()
+        stream.wait_stream(side)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step()
+        g.replay()
+        torch.cuda.synchronize()
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(steps):
+            g.replay()
+        b_.record(stream)
+        torch.cuda.synchronize()
+        res["graph_us"] = a.elapsed_time(b_) / steps * 1e3
+        del g
+    except Exception as e:  # reported, not fatal
+        res["graph_error"] = repr(e)[:200]
+    res["tokens_per_s_warm"] = cfg.tokens / (res["warm_us"] * 1e-6)
+    return res
+
+
 def other_workloads(ssd, synthetic, dev, flush, peaks, rank, world, barrier, ranks_max):
     import torch
     out = {}
     stream = torch.cuda.current_stream()
+    # launch-latency view of the two small workloads
+    for name in ("fwd_f32_small", "fwd_bf16_b4_L1024"):
+        out[name + "_launch"] = launch_timing(ssd, synthetic, dev, flush, name, rank)
     for name, steps in (("fwd_bf16_b8_L4096_init", 10), ("fwd_bf16_b1_L65536_G8", 5)):
         cfg = synthetic.FWD_CONFIGS[name]
         inp = synthetic.make_config_inputs(cfg, rank_seed(1234 + synthetic.SEED_OFFSET[name], rank))
@@ -607,21 +672,51 @@ def split_kernel_ms(ssd, cfg, d, y, fin, dev, flush, steps):
 def cpu_baseline(cfg, inp, budget_s=12.0):
     """The fp64 oracle, as it stands, on a bounded sample of the workload:
     whole batch rows (all heads, full sequence), cycling over the batch, until
-    about budget_s seconds of work have been done."""
+    about budget_s seconds of work have been done, on all host threads; then
+    a shorter sample on one thread, and a few decode steps of the decode
+    workload on all threads."""
     import oracle
+    from mamba_ssd_scan_b200 import synthetic
     orc = oracle.load()
+    threads = orc.num_threads()
+
+    def fwd_rate(budget):
+        t0 = time.perf_counter()
+        rows = 0
+        while time.perf_counter() - t0 < budget:
+            r = rows % cfg.batch
+            sub = {k: (v[r:r + 1] if (v is not None and k not in ("A", "D", "dt_bias"))
+                       else v) for k, v in inp.items()}
+            orc.ssd_fwd(**sub)
+            rows += 1
+        return rows, time.perf_counter() - t0
+
+    rows, dt = fwd_rate(budget_s)
+    out = {"value": rows * cfg.seqlen / dt, "unit": "tokens/s", "cores": threads,
+           "kind": "oracle", "sample": f"{rows} batch rows of {cfg.name} (all heads, full "
+                                       f"sequence each), {dt:.1f} s"}
+    orc.set_num_threads(1)
+    rows1, dt1 = fwd_rate(budget_s / 4)
+    orc.set_num_threads(threads)
+    out["one_core"] = {"value": rows1 * cfg.seqlen / dt1, "unit": "tokens/s",
+                       "sample": f"{rows1} batch rows, {dt1:.1f} s"}
+    # decode: a few steps on 8 of the 256 batch rows (the rows are independent),
+    # scaled to the whole batch
+    dcfg = synthetic.DECODE_CONFIGS["decode_b256_H80"]
+    rows_d = 8
+    prm = synthetic.make_decode_params(dcfg.batch, dcfg.nheads, dcfg.headdim, dcfg.dstate, 1)
+    st = prm["state"][:rows_d].double().numpy().copy()
+    steps_in = [synthetic.make_decode_step(dcfg.batch, dcfg.nheads, dcfg.headdim, dcfg.dstate,
+                                           dcfg.ngroups, dcfg.dtype, 1, s_) for s_ in range(4)]
     t0 = time.perf_counter()
-    rows = 0
-    while time.perf_counter() - t0 < budget_s:
-        r = rows % cfg.batch
-        sub = {k: (v[r:r + 1] if (v is not None and k not in ("A", "D", "dt_bias"))
-                   else v) for k, v in inp.items()}
-        orc.ssd_fwd(**sub)
-        rows += 1
-    dt = time.perf_counter() - t0
-    return {"value": rows * cfg.seqlen / dt, "unit": "tokens/s", "cores": orc.num_threads(),
-            "kind": "oracle", "sample": f"{rows} batch rows of {cfg.name} (all heads, full "
-                                        f"sequence each), {dt:.1f} s"}
+    for si in steps_in:
+        st, _ = orc.state_update(st, si["x"][:rows_d], si["dt"][:rows_d], prm["A"],
+                                 si["B"][:rows_d], si["C"][:rows_d], prm["D"], prm["dt_bias"])
+    per_step = (time.perf_counter() - t0) / len(steps_in) * dcfg.batch / rows_d
+    out["decode"] = {"us_per_step": per_step * 1e6, "workload": dcfg.name, "cores": threads,
+                     "sample": f"{len(steps_in)} steps on {rows_d} of {dcfg.batch} batch rows, "
+                               f"scaled to the whole batch"}
+    return out
 
 
 # ---------------------------------------------------------------------------

@@ -56,6 +56,8 @@ class Oracle:
         lib.oracle_softplus.restype = ctypes.c_double
         lib.oracle_softplus.argtypes = [ctypes.c_double]
         lib.oracle_num_threads.restype = ctypes.c_int
+        lib.oracle_set_num_threads.restype = None
+        lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
         lib.oracle_ssd_fwd.restype = None
         lib.oracle_ssd_fwd.argtypes = [_i64] * 6 + [_dp] * 10
         lib.oracle_ssd_chunked.restype = None
@@ -81,6 +83,9 @@ class Oracle:
 
     def num_threads(self) -> int:
         return int(self.lib.oracle_num_threads())
+
+    def set_num_threads(self, n: int) -> None:
+        self.lib.oracle_set_num_threads(int(n))
 
     def softplus(self, u: float) -> float:
         return float(self.lib.oracle_softplus(float(u)))

@@ -74,6 +74,16 @@ int oracle_num_threads(void) {
 #endif
 }
 
+/* Threads for the following calls (timing on one core or all of them); no
+ * effect on the arithmetic. */
+void oracle_set_num_threads(int n) {
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
 static double dt_of(const double* dt_raw, const double* dt_bias,
                     int64_t i, int64_t h) {
 #if ORACLE_MUTANT == 5
