@@ -70,6 +70,12 @@ typedef enum { SSD_F32 = 0, SSD_BF16 = 1 } ssd_dtype;
  *   init_state   may be NULL (= zero state): the state before token 0.
  *   y            output [batch, seqlen, nheads, headdim], dtype.
  *   final_state  may be NULL: receives h after the last token, fp32.
+ *   z            may be NULL: the output gate, [batch, seqlen, nheads,
+ *                headdim] in dtype; when given, y = (C h + D x) silu(z),
+ *                silu(z) = z / (1 + e^-z) (the output gating of the page
+ *                "MAMBA-2 Reference Implementations Comparison", sections 3
+ *                and 6.1), applied in the kernel that writes y.  The gate does
+ *                not touch the carried state.
  * Supported: 1 <= chunk <= 256; dstate a multiple of 4, <= 256; headdim a
  * multiple of 4.  bf16 inputs run the contractions on the tensor cores
  * (tcgen05) where the shape allows -- chunk_state: headdim in {32, 64, 128},
@@ -93,6 +99,7 @@ typedef struct {
     float* final_state;
     void* workspace;        /* device scratch, >= ssd_fwd_workspace_size() */
     size_t workspace_bytes;
+    const void* z;          /* optional output gate (see above); NULL = none */
 } ssd_fwd_args;
 
 /* flags */
@@ -187,7 +194,8 @@ ssd_status ssd_chunk_scan(const ssd_fwd_args* args, const float* dt, const float
  * Layouts: state [batch, nheads, headdim, dstate] fp32, updated in place;
  *   x, y [batch, nheads, headdim] dtype; dt [batch, nheads] dtype;
  *   B, C [batch, ngroups, dstate] dtype; A, D, dt_bias [nheads] fp32
- *   (D, dt_bias may be NULL).
+ *   (D, dt_bias may be NULL); z may be NULL, else the output gate
+ *   [batch, nheads, headdim] dtype: y = (sum_n state C + D x) silu(z).
  * Supported: dstate in {16, 32, 64, 128, 256}; headdim >= 1. */
 typedef struct {
     int64_t batch, nheads, headdim, dstate, ngroups;
@@ -202,6 +210,7 @@ typedef struct {
     const float* D;
     const float* dt_bias;
     void* y;
+    const void* z;          /* optional output gate; NULL = none */
 } ssd_state_update_args;
 
 ssd_status ssd_state_update(const ssd_state_update_args* args, void* stream);

@@ -38,7 +38,8 @@ class SsdFwdArgs(ctypes.Structure):
                 ("dstate", _i64), ("ngroups", _i64), ("chunk", _i64), ("dtype", _i32),
                 ("flags", _i32), ("x", _vp), ("dt", _vp), ("A", _vp), ("B", _vp), ("C", _vp),
                 ("D", _vp), ("dt_bias", _vp), ("init_state", _vp), ("y", _vp),
-                ("final_state", _vp), ("workspace", _vp), ("workspace_bytes", _sz)]
+                ("final_state", _vp), ("workspace", _vp), ("workspace_bytes", _sz),
+                ("z", _vp)]
 
 
 class SsdStateUpdateArgs(ctypes.Structure):
@@ -46,7 +47,7 @@ class SsdStateUpdateArgs(ctypes.Structure):
     _fields_ = [("batch", _i64), ("nheads", _i64), ("headdim", _i64), ("dstate", _i64),
                 ("ngroups", _i64), ("dtype", _i32), ("flags", _i32), ("state", _vp),
                 ("x", _vp), ("dt", _vp), ("A", _vp), ("B", _vp), ("C", _vp), ("D", _vp),
-                ("dt_bias", _vp), ("y", _vp)]
+                ("dt_bias", _vp), ("y", _vp), ("z", _vp)]
 
 
 class SsdError(RuntimeError):
@@ -140,22 +141,25 @@ def _check(status: int, where: str):
         raise SsdError(status, where)
 
 
-def _fwd_args(x, dt, A, B, C, D, dt_bias, chunk, init_state, y, final_state, flags):
+def _fwd_args(x, dt, A, B, C, D, dt_bias, chunk, init_state, y, final_state, flags, z=None):
     b, L, H, P = x.shape
     G, N = B.shape[2], B.shape[3]
     a = SsdFwdArgs()
     a.batch, a.seqlen, a.nheads, a.headdim, a.dstate, a.ngroups, a.chunk = b, L, H, P, N, G, chunk
     a.dtype = _dtype_code(x)
     a.flags = int(flags)
-    for name, t in (("dt", dt), ("B", B), ("C", C)):
-        if t.dtype != x.dtype:
+    for name, t in (("dt", dt), ("B", B), ("C", C), ("z", z)):
+        if t is not None and t.dtype != x.dtype:
             raise TypeError(f"{name} must have x's dtype {x.dtype}")
+    if z is not None and tuple(z.shape) != tuple(x.shape):
+        raise ValueError("z must have x's shape")
     for name, t in (("A", A), ("D", D), ("dt_bias", dt_bias), ("init_state", init_state)):
         if t is not None and t.dtype != torch.float32:
             raise TypeError(f"{name} must be float32")
     a.x, a.dt, a.A, a.B, a.C = _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C)
     a.D, a.dt_bias, a.init_state = _ptr(D), _ptr(dt_bias), _ptr(init_state)
     a.y, a.final_state = _ptr(y), _ptr(final_state)
+    a.z = _ptr(z)
     return a
 
 
@@ -191,17 +195,18 @@ def tensor_core_steps(batch, seqlen, nheads, headdim, dstate, ngroups, chunk,
 
 def ssd_fwd(x, dt, A, B, C, D=None, dt_bias=None, chunk: int = 256, init_state=None, *,
             return_final_state: bool = False, y=None, final_state=None, workspace=None,
-            flags: int = 0, stream=None):
+            flags: int = 0, stream=None, z=None):
     """The SSD scan forward.  x [b,L,H,P], dt [b,L,H] (raw), B/C [b,L,G,N] in one
     dtype (float32 or bfloat16); A, D, dt_bias [H] and init_state [b,H,P,N]
-    float32.  Returns y (and the final fp32 state when asked)."""
+    float32; z (optional output gate, x's shape and dtype): y *= silu(z).
+    Returns y (and the final fp32 state when asked)."""
     lib = load_library()
     if y is None:
         y = torch.empty_like(x)
     if final_state is None and return_final_state:
         final_state = torch.empty((x.shape[0], x.shape[2], x.shape[3], B.shape[3]),
                                   dtype=torch.float32, device=x.device)
-    a = _fwd_args(x, dt, A, B, C, D, dt_bias, chunk, init_state, y, final_state, flags)
+    a = _fwd_args(x, dt, A, B, C, D, dt_bias, chunk, init_state, y, final_state, flags, z)
     need = int(lib.ssd_fwd_workspace_size(ctypes.byref(a)))
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=x.device)
@@ -217,13 +222,13 @@ SSD_NO_ALLOC_SCRATCH_BYTES = 16 << 20
 
 
 def ssd_fwd_no_alloc(x, dt, A, B, C, D=None, dt_bias=None, chunk: int = 256, init_state=None,
-                     *, y, final_state=None, flags: int = 0, stream=None):
+                     *, y, final_state=None, flags: int = 0, stream=None, z=None):
     """ssd_fwd without a workspace, for callers that cannot allocate: the
     scratch comes from a fixed buffer inside the library (see ssd_fwd_no_alloc
     in include/ssd.h).  ``y`` (and ``final_state``, if wanted) are caller-owned
     outputs; calls that can overlap on the GPU race and must be serialised."""
     lib = load_library()
-    a = _fwd_args(x, dt, A, B, C, D, dt_bias, chunk, init_state, y, final_state, flags)
+    a = _fwd_args(x, dt, A, B, C, D, dt_bias, chunk, init_state, y, final_state, flags, z)
     need = int(lib.ssd_fwd_workspace_size(ctypes.byref(a)))
     if need > SSD_NO_ALLOC_SCRATCH_BYTES:
         raise SsdError(SSD_ERR_UNSUPPORTED,
@@ -294,19 +299,22 @@ def ssd_state_passing(x, dt, A, B, C, cumA, states, chunk: int = 256, init_state
 
 
 def ssd_chunk_scan(x, dt, A, B, C, dt_sp, cumA, states, D=None, chunk: int = 256, *, y=None,
-                   stream=None):
-    """Step 4: y from the chunk's tokens and the states entering each chunk."""
+                   stream=None, z=None):
+    """Step 4: y from the chunk's tokens and the states entering each chunk
+    (times silu(z) when the gate z is given)."""
     lib = load_library()
     y = y if y is not None else torch.empty_like(x)
-    a = _fwd_args(x, dt, A, B, C, D, None, chunk, None, y, None, 0)
+    a = _fwd_args(x, dt, A, B, C, D, None, chunk, None, y, None, 0, z)
     _check(lib.ssd_chunk_scan(ctypes.byref(a), _ptr(dt_sp), _ptr(cumA), _ptr(states),
                               _stream_ptr(stream)), "ssd_chunk_scan")
     return y
 
 
-def ssd_state_update(state, x, dt, A, B, C, D=None, dt_bias=None, *, y=None, stream=None):
+def ssd_state_update(state, x, dt, A, B, C, D=None, dt_bias=None, *, y=None, stream=None,
+                     z=None):
     """One decode step, in place on ``state`` [b,H,P,N] float32.  x [b,H,P],
-    dt [b,H], B/C [b,G,N] in one dtype.  Returns y [b,H,P] in x's dtype."""
+    dt [b,H], B/C [b,G,N] in one dtype; z (optional output gate, x's shape and
+    dtype).  Returns y [b,H,P] in x's dtype."""
     lib = load_library()
     b, H, P, N = state.shape
     G = B.shape[1]
@@ -319,6 +327,8 @@ def ssd_state_update(state, x, dt, A, B, C, D=None, dt_bias=None, *, y=None, str
     a.flags = 0
     a.state, a.x, a.dt, a.A, a.B, a.C = (_ptr(state), _ptr(x), _ptr(dt), _ptr(A), _ptr(B),
                                          _ptr(C))
-    a.D, a.dt_bias, a.y = _ptr(D), _ptr(dt_bias), _ptr(y)
+    if z is not None and (z.dtype != x.dtype or tuple(z.shape) != tuple(x.shape)):
+        raise TypeError("z must have x's shape and dtype")
+    a.D, a.dt_bias, a.y, a.z = _ptr(D), _ptr(dt_bias), _ptr(y), _ptr(z)
     _check(lib.ssd_state_update(ctypes.byref(a), _stream_ptr(stream)), "ssd_state_update")
     return y

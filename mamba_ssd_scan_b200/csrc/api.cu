@@ -79,7 +79,8 @@ ssd_status check_fwd_inputs(const ssd_fwd_args* a) {
     if (!check_ptr(a->x, false, true) || !check_ptr(a->dt, false, false) ||
         !check_ptr(a->A, false, false) || !check_ptr(a->B, false, true) ||
         !check_ptr(a->C, false, true) || !check_ptr(a->D, true, false) ||
-        !check_ptr(a->dt_bias, true, false) || !check_ptr(a->init_state, true, true))
+        !check_ptr(a->dt_bias, true, false) || !check_ptr(a->init_state, true, true) ||
+        !check_ptr(a->z, true, true))
         return SSD_ERR_INVALID_ARG;
     return SSD_OK;
 }
@@ -108,6 +109,7 @@ FwdParams make_params(const ssd_fwd_args* a) {
     p.init_state = a->init_state;
     p.y = a->y;
     p.final_state = a->final_state;
+    p.z = a->z;
     p.dt = p.cumA = nullptr;
     p.states = nullptr;
     p.status = nullptr;
@@ -286,7 +288,7 @@ ssd_status ssd_state_update(const ssd_state_update_args* a, void* stream) {
         !check_ptr(a->dt, false, false) || !check_ptr(a->A, false, false) ||
         !check_ptr(a->B, false, true) || !check_ptr(a->C, false, true) ||
         !check_ptr(a->D, true, false) || !check_ptr(a->dt_bias, true, false) ||
-        !check_ptr(a->y, false, false))
+        !check_ptr(a->y, false, false) || !check_ptr(a->z, true, false))
         return SSD_ERR_INVALID_ARG;
     DecodeParams p;
     p.batch = a->batch;
@@ -304,6 +306,7 @@ ssd_status ssd_state_update(const ssd_state_update_args* a, void* stream) {
     p.D = a->D;
     p.dt_bias = a->dt_bias;
     p.y = a->y;
+    p.z = a->z;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e = a->dtype == SSD_BF16 ? ssd::launch_state_update<__nv_bfloat16>(p, s)
                                          : ssd::launch_state_update<float>(p, s);

@@ -144,9 +144,10 @@ __global__ void __launch_bounds__(256) chunk_scan_ffma_kernel(FwdParams p) {
         __syncthreads();
     }
 
-    // epilogue: + D x, round to the output type
+    // epilogue: + D x, the optional output gate, round to the output type
     const float Dh = p.D ? p.D[h] : 0.0f;
     T* y = static_cast<T*>(p.y);
+    const T* zg = static_cast<const T*>(p.z);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const int64_t l = l0 + ty * 4 + i;
@@ -156,7 +157,8 @@ __global__ void __launch_bounds__(256) chunk_scan_ffma_kernel(FwdParams p) {
             const int64_t pi = p0 + tx * 4 + j;
             if (pi >= P) continue;
             const int64_t o = ((b * L + t0 + l) * H + h) * P + pi;
-            y[o] = from_f32<T>(acc[i][j] + Dh * to_f32(x[o]));
+            const float v = acc[i][j] + Dh * to_f32(x[o]);
+            y[o] = from_f32<T>(zg ? v * silu_f32(to_f32(zg[o])) : v);
         }
     }
 }

@@ -326,13 +326,14 @@ __device__ __forceinline__ void issue_intra(uint32_t d_tmem, uint64_t dA, uint64
     }
 }
 
-template <int NST>
+template <int NST, bool GATED>
 __global__ void __launch_bounds__(NTHREADS, 1)
     chunk_scan_tc_kernel(const __grid_constant__ FwdParams p, const __grid_constant__ CUtensorMap tm_c,
                          const __grid_constant__ CUtensorMap tm_b,
                          const __grid_constant__ CUtensorMap tm_x,
                          const __grid_constant__ CUtensorMap tm_h,
-                         const __grid_constant__ CUtensorMap tm_y, int hb_size) {
+                         const __grid_constant__ CUtensorMap tm_y,
+                         const __grid_constant__ CUtensorMap tm_z, int hb_size) {
     using T = ScanTile<NST>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -350,6 +351,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int64_t t0 = c * Q;
     const int Lc = static_cast<int>((L - t0 < Q) ? (L - t0) : Q);
     const int ntiles = (Lc + 127) / 128;
+    constexpr bool gated = GATED;  // y *= silu(z): a separate instantiation
     const uint32_t sC = smem_u32(smem + T::C_OFF), sB = smem_u32(smem + T::B_OFF);
     const uint32_t sM0 = smem_u32(smem + T::MK0_OFF), sM1 = sB;
     const uint32_t sX = smem_u32(smem + T::X_OFF), sH = smem_u32(smem + T::H_OFF);
@@ -398,6 +400,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             };
             auto prefetch_head = [&](int64_t h) {
                 tma_prefetch_l2_4d(&tm_x, 0, (int)h, (int)t0, (int)b);
+                if (gated) tma_prefetch_l2_4d(&tm_z, 0, (int)h, (int)t0, (int)b);
                 for (int kb = 0; kb < NST / 64; ++kb)
                     tma_prefetch_l2_4d(&tm_h, kb * 64, 0, (int)h, (int)(b * nc + c));
             };
@@ -418,6 +421,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                             (int)t0, (int)b);
             }
             SCAN_TRACE(0);
+            if (gated) tma_prefetch_l2_4d(&tm_z, 0, (int)hfirst, (int)t0, (int)b);
             load_x(hfirst);
             // C, B and x are inputs; the carried states come from step 3
             grid_dep_wait();
@@ -661,6 +665,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             fence_before_sync();
             mbar_arrive(bar(B_ACC_EMPTY + t));
             if (l < Lc) {
+                // optional output gate: y *= silu(z), z read after the
+                // accumulators are released (no load is in flight at an arrive)
+                uint32_t zw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+                if constexpr (gated) {
+                    const uint4* zr = reinterpret_cast<const uint4*>(
+                        static_cast<const __nv_bfloat16*>(p.z) + ((b * L + t0 + l) * H + hfirst + i) * PD +
+                        16 * hf);
+                    const uint4 z0 = ldg16(zr), z1 = ldg16(zr + 1);
+                    zw[0] = z0.x; zw[1] = z0.y; zw[2] = z0.z; zw[3] = z0.w;
+                    zw[4] = z1.x; zw[5] = z1.y; zw[6] = z1.z; zw[7] = z1.w;
+                }
                 const float s = ex2(cl2);
                 const float2 f2 = make_float2(fw.x, fw.x), s2 = make_float2(s, s);
                 const float2 w2 = make_float2(fw.y, fw.y);
@@ -674,7 +689,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                             __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xw[4 * k4 + k]));
                         const float2 vi = make_float2(__uint_as_float(r[0][e]), __uint_as_float(r[0][e + 1]));
                         const float2 vs = make_float2(__uint_as_float(r[1][e]), __uint_as_float(r[1][e + 1]));
-                        const float2 yv = __ffma2_rn(w2, xf, __ffma2_rn(s2, vs, __fmul2_rn(f2, vi)));
+                        float2 yv = __ffma2_rn(w2, xf, __ffma2_rn(s2, vs, __fmul2_rn(f2, vi)));
+                        if constexpr (gated) {
+                            const float2 zf =
+                                __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&zw[4 * k4 + k]));
+                            yv.x *= silu_f32(zf.x);
+                            yv.y *= silu_f32(zf.y);
+                        }
                         o[k] = pack_bf16x2(yv.x, yv.y);
                     }
                     st_shared_v4(sY + sw128(l, 2 * hf + k4), o[0], o[1], o[2], o[3]);
@@ -837,21 +858,22 @@ int sm_count() {
 template <int NST>
 cudaError_t launch_n(const FwdParams& p, cudaStream_t s) {
     using T = ScanTile<NST>;
-    CUtensorMap tc_, tb_, tx_, th_, ty_;
+    CUtensorMap tc_, tb_, tx_, th_, ty_, tz_;
     const uint32_t rows = static_cast<uint32_t>(p.chunk);
     if (!make_tmap_bf16_4d(&tc_, p.C, NST, p.ngroups, p.seqlen, p.batch, 1, 32) ||
         !make_tmap_bf16_4d(&tb_, p.B, NST, p.ngroups, p.seqlen, p.batch, 1, rows) ||
         !make_tmap_bf16_4d(&tx_, p.x, PD, p.nheads, p.seqlen, p.batch, 1, rows) ||
         !make_tmap_bf16_4d(&th_, p.states, NST, PD, p.nheads, p.batch * p.nchunks, PD, 1) ||
-        !make_tmap_bf16_4d(&ty_, p.y, PD, p.nheads, p.seqlen, p.batch, 1, rows))
+        !make_tmap_bf16_4d(&ty_, p.y, PD, p.nheads, p.seqlen, p.batch, 1, rows) ||
+        !make_tmap_bf16_4d(&tz_, p.z ? p.z : p.x, PD, p.nheads, p.seqlen, p.batch, 1, rows))
         return cudaErrorInvalidValue;
-    auto kern = chunk_scan_tc_kernel<NST>;
+    auto kern = p.z ? chunk_scan_tc_kernel<NST, true> : chunk_scan_tc_kernel<NST, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, T::SMEM);
     if (e != cudaSuccess) return e;
     const int hb = heads_per_cta(p, sm_count());
     dim3 grid(static_cast<unsigned>(p.nchunks * p.ngroups * (p.heads_per_group / hb)),
               static_cast<unsigned>(p.batch));
-    return launch_kernel(kern, grid, dim3(NTHREADS), T::SMEM, s, p.pdl != 0, p, tc_, tb_, tx_, th_, ty_, hb);
+    return launch_kernel(kern, grid, dim3(NTHREADS), T::SMEM, s, p.pdl != 0, p, tc_, tb_, tx_, th_, ty_, tz_, hb);
 }
 
 }  // namespace

@@ -30,6 +30,7 @@ struct FwdParams {
     const float* init_state;  // may be null
     void* y;
     float* final_state;    // may be null
+    const void* z;         // output gate [b, L, H, P] (y *= silu(z)); may be null
     // intermediates (workspace)
     float* dt;      // [b, H, nc, Q]
     float* cumA;    // [b, H, nc, Q]
@@ -48,6 +49,7 @@ struct DecodeParams {
     const float* D;
     const float* dt_bias;
     void* y;
+    const void* z;         // output gate [b, H, P]; may be null
 };
 
 // Element loads/stores for the two supported input types.
@@ -58,6 +60,9 @@ template <> __device__ __forceinline__ float from_f32<float>(float v) { return v
 template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) {
     return __float2bfloat16_rn(v);
 }
+
+// silu(z) = z / (1 + e^-z), the output gate's activation.
+__device__ __forceinline__ float silu_f32(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
 
 // softplus(u) = log(1 + e^u) without overflow.
 __device__ __forceinline__ float softplus_f32(float u) {

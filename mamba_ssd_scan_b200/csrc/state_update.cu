@@ -69,6 +69,7 @@ __global__ void __launch_bounds__(NTHREADS) state_update_kernel(DecodeParams p) 
     }
     const T* xg = static_cast<const T*>(p.x) + bh * P;
     T* yg = static_cast<T*>(p.y) + bh * P;
+    const T* zg = p.z ? static_cast<const T*>(p.z) + bh * P : nullptr;  // output gate
     float* st = p.state + bh * P * N;
 
     for (int64_t p0 = 0; p0 < P; p0 += MAXPASS * RPP) {
@@ -108,7 +109,10 @@ __global__ void __launch_bounds__(NTHREADS) state_update_kernel(DecodeParams p) 
                 float4* sp = reinterpret_cast<float4*>(st + row * N) + tl * V;
 #pragma unroll
                 for (int v = 0; v < V; ++v) __stcs(sp + v, s[ps][v]);
-                if (tl == 0) yg[row] = from_f32<T>(acc + Dh * xv[ps]);
+                if (tl == 0) {
+                    const float v = acc + Dh * xv[ps];
+                    yg[row] = from_f32<T>(zg ? v * silu_f32(to_f32(zg[row])) : v);
+                }
             }
         }
     }

@@ -136,5 +136,12 @@ def make_decode_step(batch, nheads, headdim, dstate, ngroups, dtype, seed: int,
     return dict(x=x, dt=dt, B=B, C=C)
 
 
+def make_gate(shape, dtype, seed: int) -> torch.Tensor:
+    """The optional output gate z ~ N(0, 1), of x's shape (drawn from its own
+    generator, so the other inputs of a seed are unchanged)."""
+    gen = torch.Generator().manual_seed(seed + 7919)
+    return torch.randn(tuple(shape), generator=gen, dtype=torch.float32).to(dtype)
+
+
 def nchunks(seqlen: int, chunk: int) -> int:
     return int(math.ceil(seqlen / chunk))

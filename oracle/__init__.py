@@ -64,6 +64,8 @@ class Oracle:
         lib.oracle_ssd_chunked.argtypes = [_i64] * 7 + [_dp] * 14
         lib.oracle_state_update.restype = None
         lib.oracle_state_update.argtypes = [_i64] * 5 + [_dp] * 9
+        lib.oracle_gate.restype = None
+        lib.oracle_gate.argtypes = [_dp, _dp, _i64]
         self.lib = lib
 
     # -- helpers ---------------------------------------------------------
@@ -91,11 +93,20 @@ class Oracle:
         return float(self.lib.oracle_softplus(float(u)))
 
     # -- the recurrence --------------------------------------------------
-    def ssd_fwd(self, x, dt, A, B, C, D=None, dt_bias=None, init_state=None):
+    def gate(self, y, z):
+        """y * silu(z) (float64, new array), the output gate after the scan."""
+        out = np.ascontiguousarray(y, dtype=np.float64).copy()
+        zz = self._f64(z)
+        assert zz.shape == out.shape
+        self.lib.oracle_gate(self._ptr(out), self._ptr(zz), out.size)
+        return out
+
+    def ssd_fwd(self, x, dt, A, B, C, D=None, dt_bias=None, init_state=None, z=None):
         """Token-by-token recurrence.  Returns (y, final_state) as float64.
 
         x [b,L,H,P], dt [b,L,H] (raw, before softplus), A [H], B/C [b,L,G,N],
-        D/dt_bias [H] or None, init_state [b,H,P,N] or None.
+        D/dt_bias [H] or None, init_state [b,H,P,N] or None, z (the output
+        gate, shaped like x) or None.
         """
         x, dt, A, B, C = (self._f64(t) for t in (x, dt, A, B, C))
         D, dt_bias, init = self._f64(D), self._f64(dt_bias), self._f64(init_state)
@@ -105,10 +116,12 @@ class Oracle:
         fin = np.zeros((b, H, P, N))
         self.lib.oracle_ssd_fwd(b, L, H, P, N, G, *(self._ptr(t) for t in (
             x, dt, A, B, C, D, dt_bias, init, y, fin)))
+        if z is not None:
+            y = self.gate(y, z)
         return y, fin
 
     def ssd_chunked(self, x, dt, A, B, C, D=None, dt_bias=None, init_state=None,
-                    chunk: int = 256):
+                    chunk: int = 256, z=None):
         """Chunked restatement.  Returns a dict with dt, cumA [b,H,nc,Q],
         S, Hin [b,nc,H,P,N], y [b,L,H,P] and final_state [b,H,P,N]."""
         x, dt, A, B, C = (self._f64(t) for t in (x, dt, A, B, C))
@@ -125,9 +138,11 @@ class Oracle:
         self.lib.oracle_ssd_chunked(b, L, H, P, N, G, Q, *(self._ptr(t) for t in (
             x, dt, A, B, C, D, dt_bias, init, out["dt"], out["cumA"], out["S"],
             out["Hin"], out["y"], out["final_state"])))
+        if z is not None:
+            out["y"] = self.gate(out["y"], z)
         return out
 
-    def state_update(self, state, x, dt, A, B, C, D=None, dt_bias=None):
+    def state_update(self, state, x, dt, A, B, C, D=None, dt_bias=None, z=None):
         """One decode step.  Returns (new_state, y) as float64; the input
         state is not modified.  state [b,H,P,N], x [b,H,P], dt [b,H],
         B/C [b,G,N]."""
@@ -139,6 +154,8 @@ class Oracle:
         y = np.zeros((b, H, P))
         self.lib.oracle_state_update(b, H, P, N, G, *(self._ptr(t) for t in (
             st, x, dt, A, B, C, D, dt_bias, y)))
+        if z is not None:
+            y = self.gate(y, z)
         return st, y
 
 

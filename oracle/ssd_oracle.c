@@ -103,6 +103,22 @@ static int64_t group_of(int64_t h, int64_t H, int64_t G) {
 #endif
 }
 
+/* The output gate applied after the scan, y <- y * silu(z) with
+ * silu(z) = z * sigmoid(z) = z / (1 + e^-z) ("MAMBA-2 Reference
+ * Implementations Comparison", section 3 (the forward listing) and section 6.1
+ * item 5, output gating).  n elements, in place on y. */
+void oracle_gate(double* y, const double* z, int64_t n) {
+    int64_t i;
+#pragma omp parallel for schedule(static)
+    for (i = 0; i < n; ++i) {
+#if ORACLE_MUTANT == 10
+        y[i] = y[i] / (1.0 + exp(-z[i]));
+#else
+        y[i] = y[i] * (z[i] / (1.0 + exp(-z[i])));
+#endif
+    }
+}
+
 /* The recurrence, token by token.  init may be NULL (zero state); D and
  * dt_bias may be NULL (zero); final_state may be NULL. */
 void oracle_ssd_fwd(int64_t batch, int64_t L, int64_t H, int64_t P,

@@ -226,6 +226,29 @@ def pin_golden_regression(orc):
     _close(fin, np.array(g["final_state"]), 1e-13, "golden final")
 
 
+def pin_gate(orc):
+    """The output gate y * silu(z) ("MAMBA-2 Reference Implementations
+    Comparison", sections 3 and 6.1) against values fixed without its
+    formula: silu(0) = 0; sigmoid(ln 3) = 3/4, so silu(ln 3) = (3/4) ln 3;
+    silu(z) - silu(-z) = z for every z (z sigmoid(z) + z sigmoid(-z) = z);
+    silu(40) = 40 to double precision; and the gated forward is the ungated
+    forward times the gate, the same for the decode step."""
+    rng = np.random.default_rng(7)
+    y = rng.standard_normal((3, 5, 2, 4))
+    _close(orc.gate(y, np.zeros_like(y)), np.zeros_like(y), 0.0, "silu(0)")
+    ln3 = np.log(3.0)
+    _close(orc.gate(y, np.full_like(y, ln3)), y * 0.75 * ln3, 1e-15, "silu(ln 3)")
+    z = rng.standard_normal(y.shape) * 4.0
+    _close(orc.gate(y, z) - orc.gate(y, -z), y * z, 1e-12, "silu odd part")
+    _close(orc.gate(y, np.full_like(y, 40.0)), 40.0 * y, 1e-15, "silu(40)")
+    c = _rand_case(11)
+    zz = rng.standard_normal(c["x"].shape)
+    y0, f0 = orc.ssd_fwd(**c)
+    y1, f1 = orc.ssd_fwd(**c, z=zz)
+    _close(y1, y0 * zz / (1.0 + np.exp(-zz)), 1e-13, "gated forward")
+    _close(f1, f0, 0.0, "the gate leaves the state alone")
+
+
 ALL_PINS = [pin_softplus, pin_quadratic_dual, pin_A_zero_cumsum, pin_chunk_invariance,
             pin_split_resume, pin_decode_equals_forward, pin_special_cases, pin_causality,
-            pin_half_decay_by_hand]
+            pin_half_decay_by_hand, pin_gate]

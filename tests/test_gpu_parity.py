@@ -255,3 +255,67 @@ def test_tensor_core_path(orc, case):
     assert torch.equal(f_wg, f_tc)  # the head blocking changes only chunk_scan
     assert_close(y_cc, yo, torch.bfloat16, "CUDA-core y")
     assert_close(f_cc, fo, torch.bfloat16, "CUDA-core final")
+
+
+# ---------------------------------------------------------------------------
+# the optional output gate y * silu(z)
+GATE_CASES = [
+    # (b, L, H, P, N, G, Q, dtype, flags)
+    (1, 256, 4, 16, 16, 1, 64, torch.float32, 0),          # CUDA-core path
+    (2, 600, 4, 64, 64, 2, 256, torch.bfloat16, 0),        # tensor cores, ragged tail
+    (1, 1024, 8, 64, 128, 1, 256, torch.bfloat16, 0),      # tensor cores, dstate 128
+    (2, 600, 4, 64, 64, 2, 256, torch.bfloat16, ssd.SSD_FLAG_CUDA_CORES),
+]
+
+
+@pytest.mark.parametrize("case", GATE_CASES, ids=lambda c: "b{}_L{}_H{}_P{}_N{}_G{}_Q{}_{}_f{}".format(
+    *c[:7], str(c[7]).split(".")[-1], c[8]))
+def test_gated_fwd(orc, case):
+    b, L, H, P, N, G, Q, dtype, flags = case
+    inp = synthetic.make_fwd_inputs(b, L, H, P, N, G, dtype, seed=31 + L, init_state=True)
+    z = synthetic.make_gate(inp["x"].shape, dtype, seed=31 + L)
+    d = dev(inp)
+    y, fin = ssd.ssd_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["dt_bias"], Q,
+                         d["init_state"], return_final_state=True, flags=flags, z=z.to(DEV))
+    torch.cuda.synchronize()
+    yo, fo = orc.ssd_fwd(**inp, z=z)
+    assert_close(y, yo, dtype, "gated y")
+    assert_close(fin, fo, dtype, "final_state (gate leaves it alone)")
+
+
+def test_gated_scan_step(orc):
+    b, L, H, P, N, G, Q = 2, 600, 4, 64, 64, 2, 256
+    inp = synthetic.make_fwd_inputs(b, L, H, P, N, G, torch.bfloat16, seed=77, init_state=True)
+    z = synthetic.make_gate(inp["x"].shape, torch.bfloat16, seed=77)
+    d = dev(inp)
+    nc = synthetic.nchunks(L, Q)
+    dt_sp = torch.empty((b, H, nc, Q), device=DEV)
+    cumA = torch.empty_like(dt_sp)
+    states = torch.empty((b, nc, H, P, N), device=DEV, dtype=torch.bfloat16)
+    ssd.ssd_chunk_cumsum(d["x"], d["dt"], d["A"], d["B"], d["C"], d["dt_bias"], Q,
+                         dt_out=dt_sp, cumA_out=cumA)
+    ssd.ssd_chunk_state(d["x"], d["dt"], d["A"], d["B"], d["C"], dt_sp, cumA, Q, states=states)
+    ssd.ssd_state_passing(d["x"], d["dt"], d["A"], d["B"], d["C"], cumA, states, Q,
+                          init_state=d["init_state"])
+    y = ssd.ssd_chunk_scan(d["x"], d["dt"], d["A"], d["B"], d["C"], dt_sp, cumA, states, d["D"],
+                           Q, z=z.to(DEV))
+    torch.cuda.synchronize()
+    yo = orc.ssd_chunked(**inp, chunk=Q, z=z)["y"]
+    assert_close(y, yo, torch.bfloat16, "gated y from the scan step")
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+def test_gated_decode(orc, dtype):
+    b, H, P, N, G = 4, 8, 64, 128, 2
+    prm = synthetic.make_decode_params(b, H, P, N, seed=5)
+    step = synthetic.make_decode_step(b, H, P, N, G, dtype, 5, 0)
+    z = synthetic.make_gate(step["x"].shape, dtype, seed=5)
+    state = prm["state"].to(DEV)
+    y = ssd.ssd_state_update(state, step["x"].to(DEV), step["dt"].to(DEV), prm["A"].to(DEV),
+                             step["B"].to(DEV), step["C"].to(DEV), prm["D"].to(DEV),
+                             prm["dt_bias"].to(DEV), z=z.to(DEV))
+    torch.cuda.synchronize()
+    so, yo = orc.state_update(prm["state"], step["x"], step["dt"], prm["A"], step["B"], step["C"],
+                              prm["D"], prm["dt_bias"], z=z)
+    assert_close(y, yo, dtype, "gated decode y")
+    assert_close(state, so, torch.float32, "decode state")
