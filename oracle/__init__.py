@@ -66,6 +66,10 @@ class Oracle:
         lib.oracle_state_update.argtypes = [_i64] * 5 + [_dp] * 9
         lib.oracle_gate.restype = None
         lib.oracle_gate.argtypes = [_dp, _dp, _i64]
+        lib.oracle_causal_conv1d.restype = None
+        lib.oracle_causal_conv1d.argtypes = [_i64] * 4 + [_dp] * 4 + [ctypes.c_int] + [_dp] * 2
+        lib.oracle_conv1d_update.restype = None
+        lib.oracle_conv1d_update.argtypes = [_i64] * 3 + [_dp] * 4 + [ctypes.c_int, _dp]
         self.lib = lib
 
     # -- helpers ---------------------------------------------------------
@@ -158,6 +162,33 @@ class Oracle:
             y = self.gate(y, z)
         return st, y
 
+
+    def causal_conv1d(self, x, w, bias=None, init_state=None, act: bool = True):
+        """Causal depthwise conv1d (+ SiLU when act).  x [b,L,C], w [C,K],
+        bias [C] or None, init_state [b,C,K-1] or None (zeros).  Returns
+        (y [b,L,C], final_state [b,C,K-1]) as float64."""
+        x, w = self._f64(x), self._f64(w)
+        bias, init = self._f64(bias), self._f64(init_state)
+        b, L, Cn = x.shape
+        K = w.shape[1]
+        y = np.zeros((b, L, Cn))
+        fin = np.zeros((b, Cn, max(K - 1, 1)))
+        self.lib.oracle_causal_conv1d(b, L, Cn, K, self._ptr(x), self._ptr(w), self._ptr(bias),
+                                      self._ptr(init), int(bool(act)), self._ptr(y),
+                                      self._ptr(fin) if K > 1 else None)
+        return y, fin[:, :, :K - 1]
+
+    def conv1d_update(self, state, x, w, bias=None, act: bool = True):
+        """One decode step of the convolution.  state [b,C,K-1] (not modified),
+        x [b,C].  Returns (new_state, y [b,C]) as float64."""
+        st = np.ascontiguousarray(self._f64(state)).copy()
+        x, w, bias = self._f64(x), self._f64(w), self._f64(bias)
+        b, Cn = x.shape
+        K = w.shape[1]
+        y = np.zeros((b, Cn))
+        self.lib.oracle_conv1d_update(b, Cn, K, self._ptr(st), self._ptr(x), self._ptr(w),
+                                      self._ptr(bias), int(bool(act)), self._ptr(y))
+        return st, y
 
 _DEFAULT: Oracle | None = None
 

@@ -19,6 +19,10 @@
  *   y_t   = C_t . h_t + D_h * x_t
  *           (D skip: "MAMBA-2 Implementation Gaps", Gap 4)
  *
+ * and, around the scan, the output gate y * silu(z) (oracle_gate) and the causal
+ * depthwise convolution before it with its decode step (oracle_causal_conv1d,
+ * oracle_conv1d_update).
+ *
  * Layouts (row-major, innermost last):
  *   x, y       [batch, seqlen, nheads, headdim]
  *   dt_raw     [batch, seqlen, nheads]
@@ -306,5 +310,79 @@ void oracle_state_update(int64_t batch, int64_t H, int64_t P, int64_t N,
             }
             y[bh * P + p] = acc + (D ? D[h] : 0.0) * xt[p];
         }
+    }
+}
+
+/*
+ * Causal depthwise convolution over time with an optional SiLU, the layer the
+ * page "MAMBA-2 Implementation Gaps" (Gap 2, "Convolution Layer") puts before
+ * the scan: a Conv1d with one filter per channel, kernel width K, padding K-1
+ * and the output cut to the sequence length, so
+ *
+ *   out[t, c] = bias[c] + sum_{k=0}^{K-1} w[c, k] * xin[t - (K-1) + k, c]
+ *   y[t, c]   = silu(out[t, c])  (or out when act == 0)
+ *
+ * where xin[i] = x[i] for i >= 0 and, for -(K-1) <= i < 0, the carried
+ * inputs before token 0: init[c, K-1+i] (oldest first), zero when init is
+ * NULL.  final (may be NULL) receives the last K-1 entries of xin, the state
+ * the next call (or a decode step) continues from.
+ * x, y [batch, L, Cn]; w [Cn, K]; bias [Cn] or NULL; init, final [batch, Cn, K-1].
+ */
+static double conv_in(const double* x, const double* init, int64_t L, int64_t Cn,
+                      int64_t K, int64_t b, int64_t c, int64_t i) {
+    if (i >= 0) return x[(b * L + i) * Cn + c];
+#if ORACLE_MUTANT == 13
+    (void)init;
+    return 0.0;
+#else
+    return init ? init[(b * Cn + c) * (K - 1) + (K - 1 + i)] : 0.0;
+#endif
+}
+
+void oracle_causal_conv1d(int64_t batch, int64_t L, int64_t Cn, int64_t K,
+                          const double* x, const double* w, const double* bias,
+                          const double* init, int act, double* y, double* final) {
+    int64_t bc;
+#pragma omp parallel for schedule(static)
+    for (bc = 0; bc < batch * Cn; ++bc) {
+        const int64_t b = bc / Cn, c = bc % Cn;
+        for (int64_t t = 0; t < L; ++t) {
+            double acc = bias ? bias[c] : 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+#if ORACLE_MUTANT == 11
+                const int64_t i = t - k;                 /* kernel reversed */
+#elif ORACLE_MUTANT == 12
+                const int64_t i = t - (K - 1) + k + 1;   /* one token ahead */
+                if (i >= L) continue;
+#else
+                const int64_t i = t - (K - 1) + k;
+#endif
+                acc += w[c * K + k] * conv_in(x, init, L, Cn, K, b, c, i);
+            }
+            y[(b * L + t) * Cn + c] = act ? acc / (1.0 + exp(-acc)) : acc;
+        }
+        if (final)
+            for (int64_t j = 0; j < K - 1; ++j)
+                final[(b * Cn + c) * (K - 1) + j] = conv_in(x, init, L, Cn, K, b, c, L - (K - 1) + j);
+    }
+}
+
+/* One decode step of the same convolution: state [batch, Cn, K-1] holds the
+ * previous K-1 inputs (oldest first) and is shifted in place to end with
+ * x [batch, Cn]; y [batch, Cn] receives the step's output. */
+void oracle_conv1d_update(int64_t batch, int64_t Cn, int64_t K, double* state,
+                          const double* x, const double* w, const double* bias,
+                          int act, double* y) {
+    int64_t bc;
+#pragma omp parallel for schedule(static)
+    for (bc = 0; bc < batch * Cn; ++bc) {
+        const int64_t c = bc % Cn;
+        double* s = state + bc * (K - 1);
+        double acc = bias ? bias[c] : 0.0;
+        for (int64_t k = 0; k < K - 1; ++k) acc += w[c * K + k] * s[k];
+        acc += w[c * K + K - 1] * x[bc];
+        for (int64_t k = 0; k + 1 < K - 1; ++k) s[k] = s[k + 1];
+        if (K > 1) s[K - 2] = x[bc];
+        y[bc] = act ? acc / (1.0 + exp(-acc)) : acc;
     }
 }

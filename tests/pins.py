@@ -249,6 +249,50 @@ def pin_gate(orc):
     _close(f1, f0, 0.0, "the gate leaves the state alone")
 
 
+def pin_conv1d(orc):
+    """The causal depthwise convolution ("MAMBA-2 Implementation Gaps", Gap 2:
+    Conv1d, groups = channels, padding K - 1, output cut to the sequence)
+    against: numpy's full convolution with the kernel reversed (a Conv1d is a
+    cross-correlation), its first L outputs; the impulse response (a one-hot
+    input at t0 gives w[K-1-j] at t0 + j); split / resume through the carried
+    state; decode steps equal to the forward; and the SiLU through the
+    identity silu(u) - silu(-u) = u (the convolution is linear in x, bias and
+    the carried inputs)."""
+    rng = np.random.default_rng(13)
+    b, L, Cn, K = 2, 21, 5, 4
+    x = rng.standard_normal((b, L, Cn))
+    w = rng.standard_normal((Cn, K))
+    bias = rng.standard_normal(Cn)
+    y, fin = orc.causal_conv1d(x, w, bias, act=False)
+    ref = np.stack([np.stack([np.convolve(x[i, :, c], w[c][::-1])[:L] + bias[c]
+                              for c in range(Cn)], -1) for i in range(b)])
+    _close(y, ref, 1e-13, "conv1d vs numpy convolve")
+    _close(fin, np.transpose(x[:, L - (K - 1):, :], (0, 2, 1)), 0.0, "carried inputs")
+    imp = np.zeros((1, L, Cn))
+    imp[0, 7, :] = 1.0
+    yi, _ = orc.causal_conv1d(imp, w, None, act=False)
+    for j in range(K):
+        _close(yi[0, 7 + j, :], w[:, K - 1 - j], 0.0, f"impulse response tap {j}")
+    _close(yi[0, :7, :], np.zeros((7, Cn)), 0.0, "causality")
+    init = rng.standard_normal((b, Cn, K - 1))
+    ya, fa = orc.causal_conv1d(x, w, bias, init, act=True)
+    L1 = 9
+    y1, f1 = orc.causal_conv1d(x[:, :L1], w, bias, init, act=True)
+    y2, f2 = orc.causal_conv1d(x[:, L1:], w, bias, f1, act=True)
+    _close(np.concatenate([y1, y2], 1), ya, 1e-14, "conv1d split / resume")
+    _close(f2, fa, 0.0, "conv1d final state after resume")
+    st = init.copy()
+    ys = []
+    for t in range(L):
+        st, yt = orc.conv1d_update(st, x[:, t], w, bias, act=True)
+        ys.append(yt)
+    _close(np.stack(ys, 1), ya, 1e-14, "conv1d decode = forward")
+    _close(st, fa, 0.0, "conv1d decode state = forward final state")
+    yn, _ = orc.causal_conv1d(-x, w, -bias, -init, act=True)
+    yl, _ = orc.causal_conv1d(x, w, bias, init, act=False)
+    _close(ya - yn, yl, 1e-13, "silu(u) - silu(-u) = u")
+
+
 ALL_PINS = [pin_softplus, pin_quadratic_dual, pin_A_zero_cumsum, pin_chunk_invariance,
             pin_split_resume, pin_decode_equals_forward, pin_special_cases, pin_causality,
-            pin_half_decay_by_hand, pin_gate]
+            pin_half_decay_by_hand, pin_gate, pin_conv1d]

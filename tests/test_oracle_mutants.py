@@ -5,14 +5,16 @@ Mutants: 1 drops the D skip; 2 reads y from the state before the update;
 3 swaps the roles of B and C; 4 flips the sign of the decay exponent; 5 drops
 dt_bias; 6 maps heads to groups round-robin instead of contiguously; 7 drops dt
 from the input term; 8 replaces softplus by exp; 9 ignores the initial state;
-10 gates with sigmoid(z) instead of silu(z).
+10 gates with sigmoid(z) instead of silu(z); 11 reverses the convolution
+kernel; 12 shifts the convolution one token ahead; 13 ignores the carried
+convolution inputs.
 """
 import pytest
 
 import oracle
 import pins
 
-MUTANTS = list(range(1, 11))
+MUTANTS = list(range(1, 14))
 
 
 @pytest.fixture(scope="module")
