@@ -215,6 +215,51 @@ typedef struct {
 
 ssd_status ssd_state_update(const ssd_state_update_args* args, void* stream);
 
+/* ---- causal depthwise convolution (before the scan) ---------------------- */
+/* The layer the page "MAMBA-2 Implementation Gaps" (Gap 2, "Convolution
+ * Layer") puts in front of the scan: a Conv1d with one filter per channel,
+ * kernel width K, causal padding K - 1 and the output cut to the sequence
+ * length, then SiLU:
+ *   out[t, c] = bias[c] + sum_{k<K} w[c, k] xin[t - (K-1) + k, c];  y = silu(out)
+ * where xin extends x backwards with the carried inputs (init_state).
+ * Layouts: x, y [batch, seqlen, channels] dtype; weight [channels, width]
+ *   fp32; bias [channels] fp32 or NULL; init_state, final_state [batch,
+ *   channels, width - 1] fp32, the inputs before token 0 / the last width - 1
+ *   inputs, oldest first; NULL = zeros / not returned.
+ * Supported: 1 <= width <= 8; channels a multiple of 8 (bf16) or 4 (fp32);
+ *   x and y 16-byte aligned.  Errors as for ssd_fwd. */
+typedef struct {
+    int64_t batch, seqlen, channels, width;
+    int32_t dtype;
+    int32_t activation;     /* 1 = SiLU, 0 = none */
+    const void* x;
+    const float* weight;
+    const float* bias;
+    const float* init_state;
+    void* y;
+    float* final_state;
+} ssd_conv1d_args;
+
+ssd_status ssd_causal_conv1d(const ssd_conv1d_args* args, void* stream);
+
+/* One decode step of the same convolution (its half of the Mamba2Cache):
+ * state [batch, channels, width - 1] fp32 holds the previous width - 1 inputs,
+ * oldest first, and is shifted in place to end with x;
+ *   y[c] = silu(bias[c] + sum_{k<width-1} w[c, k] state[c, k] + w[c, width-1] x[c]).
+ * x, y [batch, channels] dtype.  Supported: 1 <= width <= 8. */
+typedef struct {
+    int64_t batch, channels, width;
+    int32_t dtype;
+    int32_t activation;     /* 1 = SiLU, 0 = none */
+    float* state;
+    const void* x;
+    const float* weight;
+    const float* bias;
+    void* y;
+} ssd_conv1d_update_args;
+
+ssd_status ssd_conv1d_update(const ssd_conv1d_update_args* args, void* stream);
+
 /* ---- misc --------------------------------------------------------------- */
 /* Static, human-readable name of a status code. */
 const char* ssd_status_string(ssd_status status);

@@ -50,6 +50,20 @@ class SsdStateUpdateArgs(ctypes.Structure):
                 ("dt_bias", _vp), ("y", _vp), ("z", _vp)]
 
 
+class SsdConv1dArgs(ctypes.Structure):
+    """Mirror of ssd_conv1d_args."""
+    _fields_ = [("batch", _i64), ("seqlen", _i64), ("channels", _i64), ("width", _i64),
+                ("dtype", _i32), ("activation", _i32), ("x", _vp), ("weight", _vp),
+                ("bias", _vp), ("init_state", _vp), ("y", _vp), ("final_state", _vp)]
+
+
+class SsdConv1dUpdateArgs(ctypes.Structure):
+    """Mirror of ssd_conv1d_update_args."""
+    _fields_ = [("batch", _i64), ("channels", _i64), ("width", _i64), ("dtype", _i32),
+                ("activation", _i32), ("state", _vp), ("x", _vp), ("weight", _vp),
+                ("bias", _vp), ("y", _vp)]
+
+
 class SsdError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
@@ -331,4 +345,51 @@ def ssd_state_update(state, x, dt, A, B, C, D=None, dt_bias=None, *, y=None, str
         raise TypeError("z must have x's shape and dtype")
     a.D, a.dt_bias, a.y, a.z = _ptr(D), _ptr(dt_bias), _ptr(y), _ptr(z)
     _check(lib.ssd_state_update(ctypes.byref(a), _stream_ptr(stream)), "ssd_state_update")
+    return y
+
+
+def ssd_causal_conv1d(x, weight, bias=None, init_state=None, *, activation: bool = True,
+                      y=None, final_state=None, return_final_state: bool = False, stream=None):
+    """Causal depthwise conv1d (+ SiLU) in front of the scan.  x [b,L,C] float32
+    or bfloat16; weight [C,K] float32; bias [C] float32 or None; init_state
+    [b,C,K-1] float32 or None.  Returns y (and the final [b,C,K-1] state when
+    asked)."""
+    lib = load_library()
+    b, L, Cn = x.shape
+    K = weight.shape[1]
+    for name, t in (("weight", weight), ("bias", bias), ("init_state", init_state),
+                    ("final_state", final_state)):
+        if t is not None and t.dtype != torch.float32:
+            raise TypeError(f"{name} must be float32")
+    y = y if y is not None else torch.empty_like(x)
+    if final_state is None and return_final_state and K > 1:
+        final_state = torch.empty((b, Cn, K - 1), dtype=torch.float32, device=x.device)
+    a = SsdConv1dArgs()
+    a.batch, a.seqlen, a.channels, a.width = b, L, Cn, K
+    a.dtype = _dtype_code(x)
+    a.activation = 1 if activation else 0
+    a.x, a.weight, a.bias, a.init_state = _ptr(x), _ptr(weight), _ptr(bias), _ptr(init_state)
+    a.y, a.final_state = _ptr(y), _ptr(final_state)
+    _check(lib.ssd_causal_conv1d(ctypes.byref(a), _stream_ptr(stream)), "ssd_causal_conv1d")
+    if return_final_state:
+        return y, final_state
+    return y
+
+
+def ssd_conv1d_update(state, x, weight, bias=None, *, activation: bool = True, y=None,
+                      stream=None):
+    """One decode step of the convolution, in place on ``state`` [b,C,K-1]
+    float32.  x [b,C].  Returns y [b,C] in x's dtype."""
+    lib = load_library()
+    b, Cn = x.shape
+    K = weight.shape[1]
+    if state is not None and state.dtype != torch.float32:
+        raise TypeError("state must be float32")
+    y = y if y is not None else torch.empty_like(x)
+    a = SsdConv1dUpdateArgs()
+    a.batch, a.channels, a.width = b, Cn, K
+    a.dtype = _dtype_code(x)
+    a.activation = 1 if activation else 0
+    a.state, a.x, a.weight, a.bias, a.y = _ptr(state), _ptr(x), _ptr(weight), _ptr(bias), _ptr(y)
+    _check(lib.ssd_conv1d_update(ctypes.byref(a), _stream_ptr(stream)), "ssd_conv1d_update")
     return y

@@ -275,6 +275,62 @@ ssd_status ssd_chunk_scan(const ssd_fwd_args* a, const float* dt, const float* c
     return to_status(run_chunk_scan(p, a->dtype, a->flags, static_cast<cudaStream_t>(stream)));
 }
 
+ssd_status ssd_causal_conv1d(const ssd_conv1d_args* a, void* stream) {
+    if (!a) return SSD_ERR_INVALID_ARG;
+    if (a->batch <= 0 || a->seqlen <= 0 || a->channels <= 0 || a->width <= 0)
+        return SSD_ERR_INVALID_ARG;
+    if (a->dtype != SSD_F32 && a->dtype != SSD_BF16) return SSD_ERR_INVALID_ARG;
+    if (a->width > 8 || a->channels % (a->dtype == SSD_BF16 ? 8 : 4) != 0)
+        return SSD_ERR_UNSUPPORTED;
+    if (!check_ptr(a->x, false, true) || !check_ptr(a->weight, false, false) ||
+        !check_ptr(a->bias, true, false) || !check_ptr(a->init_state, true, false) ||
+        !check_ptr(a->y, false, true) || !check_ptr(a->final_state, true, false))
+        return SSD_ERR_INVALID_ARG;
+    ssd::ConvParams p;
+    p.batch = a->batch;
+    p.seqlen = a->seqlen;
+    p.channels = a->channels;
+    p.width = a->width;
+    p.activation = a->activation ? 1 : 0;
+    p.x = a->x;
+    p.weight = a->weight;
+    p.bias = a->bias;
+    p.init_state = a->init_state;
+    p.y = a->y;
+    p.final_state = a->final_state;
+    p.update_state = nullptr;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return to_status(a->dtype == SSD_BF16 ? ssd::launch_conv1d<__nv_bfloat16>(p, false, s)
+                                          : ssd::launch_conv1d<float>(p, false, s));
+}
+
+ssd_status ssd_conv1d_update(const ssd_conv1d_update_args* a, void* stream) {
+    if (!a) return SSD_ERR_INVALID_ARG;
+    if (a->batch <= 0 || a->channels <= 0 || a->width <= 0) return SSD_ERR_INVALID_ARG;
+    if (a->dtype != SSD_F32 && a->dtype != SSD_BF16) return SSD_ERR_INVALID_ARG;
+    if (a->width > 8) return SSD_ERR_UNSUPPORTED;
+    if (!check_ptr(a->state, a->width == 1, false) || !check_ptr(a->x, false, false) ||
+        !check_ptr(a->weight, false, false) || !check_ptr(a->bias, true, false) ||
+        !check_ptr(a->y, false, false))
+        return SSD_ERR_INVALID_ARG;
+    ssd::ConvParams p;
+    p.batch = a->batch;
+    p.seqlen = 1;
+    p.channels = a->channels;
+    p.width = a->width;
+    p.activation = a->activation ? 1 : 0;
+    p.x = a->x;
+    p.weight = a->weight;
+    p.bias = a->bias;
+    p.init_state = nullptr;
+    p.y = a->y;
+    p.final_state = nullptr;
+    p.update_state = a->state;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return to_status(a->dtype == SSD_BF16 ? ssd::launch_conv1d<__nv_bfloat16>(p, true, s)
+                                          : ssd::launch_conv1d<float>(p, true, s));
+}
+
 ssd_status ssd_state_update(const ssd_state_update_args* a, void* stream) {
     if (!a) return SSD_ERR_INVALID_ARG;
     if (a->batch <= 0 || a->nheads <= 0 || a->headdim <= 0 || a->dstate <= 0 ||

@@ -52,6 +52,19 @@ struct DecodeParams {
     const void* z;         // output gate [b, H, P]; may be null
 };
 
+// The causal depthwise convolution (forward and decode step).
+struct ConvParams {
+    int64_t batch, seqlen, channels, width;
+    int32_t activation;            // 1 = SiLU
+    const void* x;                 // [b, L, C] (forward) or [b, C] (decode)
+    const float* weight;           // [C, width]
+    const float* bias;             // [C]; may be null
+    const float* init_state;       // [b, C, width-1]; may be null (forward)
+    void* y;
+    float* final_state;            // [b, C, width-1]; may be null (forward)
+    float* update_state;           // [b, C, width-1], in place (decode)
+};
+
 // Element loads/stores for the two supported input types.
 __device__ __forceinline__ float to_f32(float v) { return v; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }
@@ -150,6 +163,7 @@ template <typename T> cudaError_t launch_chunk_state_ffma(const FwdParams& p, cu
 template <typename T> cudaError_t launch_state_passing(const FwdParams& p, cudaStream_t s);
 template <typename T> cudaError_t launch_chunk_scan_ffma(const FwdParams& p, cudaStream_t s);
 template <typename T> cudaError_t launch_state_update(const DecodeParams& p, cudaStream_t s);
+template <typename T> cudaError_t launch_conv1d(const ConvParams& p, bool update, cudaStream_t s);
 
 // Tensor-core (tcgen05) variants for bf16 inputs, with their shape ranges.
 bool chunk_state_tc_supported(const FwdParams& p);

@@ -143,5 +143,19 @@ def make_gate(shape, dtype, seed: int) -> torch.Tensor:
     return torch.randn(tuple(shape), generator=gen, dtype=torch.float32).to(dtype)
 
 
+def make_conv_inputs(batch, seqlen, channels, width, dtype, seed: int,
+                     init_state: bool = True) -> dict:
+    """Inputs of the causal depthwise convolution: x ~ N(0, 1) [b, L, C] in
+    dtype, weight ~ N(0, 1/width) [C, width], bias ~ N(0, 0.1^2) [C] and the
+    carried inputs init ~ N(0, 1) [b, C, width-1] (fp32), drawn in that order."""
+    gen = torch.Generator().manual_seed(seed + 104729)
+    x = torch.randn((batch, seqlen, channels), generator=gen).to(dtype)
+    w = torch.randn((channels, width), generator=gen) / width ** 0.5
+    bias = torch.randn((channels,), generator=gen) * 0.1
+    init = (torch.randn((batch, channels, max(width - 1, 0)), generator=gen)
+            if init_state and width > 1 else None)
+    return dict(x=x, weight=w, bias=bias, init_state=init)
+
+
 def nchunks(seqlen: int, chunk: int) -> int:
     return int(math.ceil(seqlen / chunk))

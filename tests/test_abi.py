@@ -104,3 +104,22 @@ def test_state_update_rejects_bad_args(lib):
     assert lib.ssd_state_update(ctypes.byref(a), None) == 2
     a.dstate, a.ngroups = 128, 3
     assert lib.ssd_state_update(ctypes.byref(a), None) == 1
+
+
+def test_conv1d_rejects_bad_args(lib):
+    import mamba_ssd_scan_b200 as ssd
+    a = ssd.SsdConv1dArgs()
+    a.batch, a.seqlen, a.channels, a.width, a.dtype, a.activation = 2, 64, 16, 4, 1, 1
+    assert lib.ssd_causal_conv1d(None, None) == 1
+    assert lib.ssd_causal_conv1d(ctypes.byref(a), None) == 1        # null pointers
+    a.width = 9
+    assert lib.ssd_causal_conv1d(ctypes.byref(a), None) == 2        # width beyond 8
+    a.width, a.channels = 4, 12
+    assert lib.ssd_causal_conv1d(ctypes.byref(a), None) == 2        # bf16 channels % 8
+    a.channels, a.seqlen = 16, 0
+    assert lib.ssd_causal_conv1d(ctypes.byref(a), None) == 1        # empty sequence
+    u = ssd.SsdConv1dUpdateArgs()
+    u.batch, u.channels, u.width, u.dtype = 2, 16, 4, 0
+    assert lib.ssd_conv1d_update(ctypes.byref(u), None) == 1        # null pointers
+    u.width = 0
+    assert lib.ssd_conv1d_update(ctypes.byref(u), None) == 1
