@@ -626,7 +626,91 @@ def other_workloads(ssd, synthetic, dev, flush, peaks, rank, world, barrier, ran
                      "achieved_gbs": step_bytes / (us * 1e-6) / 1e9,
                      "hbm_frac": step_bytes / (us * 1e-6) / (peaks["hbm_gbs"] * 1e9),
                      "bytes_per_step": step_bytes}
-    del g
+    del g, state, steps_in
+    torch.cuda.empty_cache()
+    out.update(conv_workloads(ssd, synthetic, dev, flush, peaks, rank, world, ranks_max))
+    return out
+
+
+def conv_workloads(ssd, synthetic, dev, flush, peaks, rank, world, ranks_max, steps=10):
+    """The causal depthwise convolution in front of the scan: the forward over
+    a sequence (L2 flushed before each launch) and the decode step (1024 steps
+    in one CUDA graph, cycling through several layers' carried states)."""
+    import torch
+    out = {}
+    stream = torch.cuda.current_stream()
+    cfg = synthetic.CONV_CONFIGS["conv1d_bf16_b8_L4096_C2304"]
+    inp = synthetic.make_conv_inputs(cfg.batch, cfg.seqlen, cfg.channels, cfg.width, cfg.dtype,
+                                     rank_seed(1234 + synthetic.SEED_OFFSET[cfg.name], rank))
+    d = {k: v.to(dev) for k, v in inp.items()}
+    y = torch.empty_like(d["x"])
+    fin = torch.empty_like(d["init_state"])
+
+    def step():
+        ssd.ssd_causal_conv1d(d["x"], d["weight"], d["bias"], d["init_state"], y=y,
+                              final_state=fin)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    for a, b_ in evs:
+        flush()
+        a.record(stream)
+        step()
+        b_.record(stream)
+    torch.cuda.synchronize()
+    ms = ranks_max(sum(a.elapsed_time(b_) for a, b_ in evs) / steps)
+    elt = 2 if cfg.dtype == torch.bfloat16 else 4
+    nbytes = 2 * cfg.batch * cfg.seqlen * cfg.channels * elt + \
+        2 * cfg.batch * cfg.channels * (cfg.width - 1) * 4 + cfg.channels * (cfg.width + 1) * 4
+    out[cfg.name] = {"tokens_per_s": job_throughput(cfg.batch * cfg.seqlen, world, ms), "ms": ms,
+                     "achieved_gbs": nbytes / (ms * 1e-3) / 1e9,
+                     "hbm_frac": nbytes / (ms * 1e-3) / (peaks["hbm_gbs"] * 1e9),
+                     "bytes": nbytes, "l2": "flushed"}
+    del d, y, fin
+
+    cfg = synthetic.CONV_CONFIGS["conv1d_update_b256_C7168"]
+    seed = rank_seed(1234 + synthetic.SEED_OFFSET[cfg.name], rank)
+    per = [synthetic.make_conv_inputs(cfg.batch, 16, cfg.channels, cfg.width, cfg.dtype,
+                                      seed + 97 * l) for l in range(cfg.layers)]
+    states = [p_["init_state"].to(dev) for p_ in per]
+    ws = [p_["weight"].to(dev) for p_ in per]
+    bs = [p_["bias"].to(dev) for p_ in per]
+    xs = [p_["x"][:, t].contiguous().to(dev) for p_ in per[:1] for t in range(16)]
+    yd = torch.empty((cfg.batch, cfg.channels), dtype=cfg.dtype, device=dev)
+    del per
+
+    def run(n):
+        for s in range(n):
+            l = s % cfg.layers
+            ssd.ssd_conv1d_update(states[l], xs[s % len(xs)], ws[l], bs[l], y=yd)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        run(3)
+    torch.cuda.current_stream().wait_stream(side)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        run(cfg.steps)
+    g.replay()
+    torch.cuda.synchronize()
+    a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    g.replay()
+    b_.record(stream)
+    torch.cuda.synchronize()
+    us = ranks_max(a.elapsed_time(b_) * 1e3 / cfg.steps)
+    step_bytes = 2 * cfg.batch * cfg.channels * (cfg.width - 1) * 4 + \
+        2 * cfg.batch * cfg.channels * elt + cfg.channels * (cfg.width + 1) * 4
+    out[cfg.name] = {"us_per_step": us, "steps": cfg.steps, "graph": True, "layers": cfg.layers,
+                     "achieved_gbs": step_bytes / (us * 1e-6) / 1e9,
+                     "hbm_frac": step_bytes / (us * 1e-6) / (peaks["hbm_gbs"] * 1e9),
+                     "bytes_per_step": step_bytes}
+    del g, states
+    torch.cuda.empty_cache()
     return out
 
 

@@ -227,7 +227,9 @@ ssd_status ssd_state_update(const ssd_state_update_args* args, void* stream);
  *   channels, width - 1] fp32, the inputs before token 0 / the last width - 1
  *   inputs, oldest first; NULL = zeros / not returned.
  * Supported: 1 <= width <= 8; channels a multiple of 8 (bf16) or 4 (fp32);
- *   x and y 16-byte aligned.  Errors as for ssd_fwd. */
+ *   batch <= 65535; x and y 16-byte aligned (else SSD_ERR_UNSUPPORTED /
+ *   SSD_ERR_INVALID_ARG).  Errors as for ssd_fwd; a kernel that gave up on a
+ *   wait is reported by ssd_conv1d_check_status. */
 typedef struct {
     int64_t batch, seqlen, channels, width;
     int32_t dtype;
@@ -241,6 +243,11 @@ typedef struct {
 } ssd_conv1d_args;
 
 ssd_status ssd_causal_conv1d(const ssd_conv1d_args* args, void* stream);
+
+/* Synchronises `stream` and returns SSD_ERR_TIMEOUT if a ssd_causal_conv1d
+ * launch on this device timed out on an internal wait since the last check
+ * (the flag is cleared), else SSD_OK. */
+ssd_status ssd_conv1d_check_status(void* stream);
 
 /* One decode step of the same convolution (its half of the Mamba2Cache):
  * state [batch, channels, width - 1] fp32 holds the previous width - 1 inputs,

@@ -19,6 +19,7 @@ __all__ = [
     "ssd_fwd_tensor_core_steps", "tensor_core_steps", "ssd_chunk_cumsum", "ssd_chunk_state",
     "ssd_state_passing", "ssd_chunk_scan", "ssd_state_update", "ssd_status_string",
     "ssd_version", "lib_path", "load_library", "SSD_FLAG_CUDA_CORES", "SSD_FLAG_WHOLE_GROUPS",
+    "ssd_causal_conv1d", "ssd_conv1d_update", "ssd_conv1d_check_status",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -109,6 +110,12 @@ def load_library():
     lib.ssd_chunk_scan.argtypes = [F, _vp, _vp, _vp, _vp]
     lib.ssd_state_update.restype = ctypes.c_int
     lib.ssd_state_update.argtypes = [ctypes.POINTER(SsdStateUpdateArgs), _vp]
+    lib.ssd_causal_conv1d.restype = ctypes.c_int
+    lib.ssd_causal_conv1d.argtypes = [ctypes.POINTER(SsdConv1dArgs), _vp]
+    lib.ssd_conv1d_update.restype = ctypes.c_int
+    lib.ssd_conv1d_update.argtypes = [ctypes.POINTER(SsdConv1dUpdateArgs), _vp]
+    lib.ssd_conv1d_check_status.restype = ctypes.c_int
+    lib.ssd_conv1d_check_status.argtypes = [_vp]
     lib.ssd_status_string.restype = ctypes.c_char_p
     lib.ssd_status_string.argtypes = [ctypes.c_int]
     lib.ssd_last_cuda_error.restype = ctypes.c_char_p
@@ -374,6 +381,12 @@ def ssd_causal_conv1d(x, weight, bias=None, init_state=None, *, activation: bool
     if return_final_state:
         return y, final_state
     return y
+
+
+def ssd_conv1d_check_status(stream=None) -> int:
+    """Synchronises the stream; SSD_ERR_TIMEOUT if a forward convolution on
+    this device gave up on an internal wait since the last check, else 0."""
+    return int(load_library().ssd_conv1d_check_status(_stream_ptr(stream)))
 
 
 def ssd_conv1d_update(state, x, weight, bias=None, *, activation: bool = True, y=None,

@@ -280,7 +280,7 @@ ssd_status ssd_causal_conv1d(const ssd_conv1d_args* a, void* stream) {
     if (a->batch <= 0 || a->seqlen <= 0 || a->channels <= 0 || a->width <= 0)
         return SSD_ERR_INVALID_ARG;
     if (a->dtype != SSD_F32 && a->dtype != SSD_BF16) return SSD_ERR_INVALID_ARG;
-    if (a->width > 8 || a->channels % (a->dtype == SSD_BF16 ? 8 : 4) != 0)
+    if (a->width > 8 || a->channels % (a->dtype == SSD_BF16 ? 8 : 4) != 0 || a->batch > 65535)
         return SSD_ERR_UNSUPPORTED;
     if (!check_ptr(a->x, false, true) || !check_ptr(a->weight, false, false) ||
         !check_ptr(a->bias, true, false) || !check_ptr(a->init_state, true, false) ||
@@ -302,6 +302,13 @@ ssd_status ssd_causal_conv1d(const ssd_conv1d_args* a, void* stream) {
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     return to_status(a->dtype == SSD_BF16 ? ssd::launch_conv1d<__nv_bfloat16>(p, false, s)
                                           : ssd::launch_conv1d<float>(p, false, s));
+}
+
+ssd_status ssd_conv1d_check_status(void* stream) {
+    int v = 0;
+    if (ssd::conv1d_take_status(&v, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return SSD_ERR_CUDA;
+    return v == 0 ? SSD_OK : static_cast<ssd_status>(v);
 }
 
 ssd_status ssd_conv1d_update(const ssd_conv1d_update_args* a, void* stream) {

@@ -62,16 +62,6 @@ __device__ __forceinline__ uint4 scale_bf16x8(uint4 v, float w) {
     return make_uint4(out[0], out[1], out[2], out[3]);
 }
 
-// Bounded mbarrier wait that also gives up when another role has aborted.
-__device__ __forceinline__ bool wait_or_abort(uint32_t mbar, uint32_t parity, volatile int* abort) {
-    for (uint32_t i = 0; i < kSpinLimit; ++i) {
-        if (mbar_try_wait_hint(mbar, parity, 200)) return true;
-        if ((i & 63) == 63 && *abort) return false;
-    }
-    *abort = 1;
-    return false;
-}
-
 template <int NST, int PD>
 __global__ void __launch_bounds__(NTHR, NST == 256 ? 2 : 3)  // CTAs per SM that fit
     chunk_state_tc_kernel(const __grid_constant__ FwdParams p,

@@ -6,116 +6,253 @@
 //   out[t, c] = bias[c] + sum_{k<K} w[c, k] xin[t - (K-1) + k, c];  y = silu(out)
 //
 // xin extends x backwards with the carried inputs (init_state, oldest first).
-// Bandwidth-bound: x is read once (plus a K-1 token halo per strip) and y
-// written once.  A thread owns one 16-byte vector of channels (8 bf16 or 4
-// fp32) and a strip of TS consecutive tokens; consecutive threads take
-// consecutive channel vectors of the same strip, so a warp's loads and stores
-// are contiguous.  The previous K-1 inputs of its channels live in registers
-// as a sliding window; the thread holding the last strip writes the final
-// window as the carried state.  The decode step keeps the same state
-// [batch, channels, K-1] and shifts it by one token.
+// Bandwidth-bound: x is read once (plus a K-1 token halo per sequence
+// segment) and y written once.  A CTA owns a block of channels (rows of at
+// most 2 KB) over a segment of the sequence.  Its producer warp streams the
+// segment's token rows into a ring of shared-memory tiles with bulk copies
+// (one row per lane, completing on the tile's "full" mbarrier); the consumer
+// warps take 4 channels per thread, keep the previous K-1 inputs in registers
+// as a sliding window, compute with packed fp32x2 arithmetic, store their
+// outputs directly and release the tile on its "empty" mbarrier.  The decode
+// step keeps the same state [batch, channels, K-1] and shifts it by one token.
 #include "internal.cuh"
+#include "tcgen05.cuh"
+#include "tma.cuh"
 
 namespace ssd {
 namespace {
 
-constexpr int TS = 32;  // tokens per thread strip
+constexpr int TT = 8;          // token rows per shared-memory tile
+constexpr int NSTAGE = 4;      // tiles in flight per CTA
+constexpr int MAXROWB = 2048;  // bytes of one tile row (the CTA's channel block)
+constexpr int CPT = 4;         // channels per consumer thread
+template <typename T> constexpr int kMaxConsumers = MAXROWB / (CPT * static_cast<int>(sizeof(T)));
 
-template <typename T> struct Vec;
-template <> struct Vec<float> {
-    static constexpr int V = 4;
-    static __device__ __forceinline__ void load(const float* p, float (&v)[4]) {
-        const float4 q = __ldg(reinterpret_cast<const float4*>(p));
-        v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+// SSD_ERR_TIMEOUT once a forward launch gave up on a wait; read and cleared
+// by ssd_conv1d_check_status.
+__device__ int g_conv_status;
+
+// Four consecutive channels of one token, widened to fp32 pairs.
+template <typename T> struct Quad;
+template <> struct Quad<float> {
+    static __device__ __forceinline__ void load(const uint8_t* s, float2& lo, float2& hi) {
+        const float4 v = *reinterpret_cast<const float4*>(s);
+        lo = make_float2(v.x, v.y);
+        hi = make_float2(v.z, v.w);
     }
-    static __device__ __forceinline__ void store(float* p, const float (&v)[4]) {
-        *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+    static __device__ __forceinline__ void store(float* p, float2 lo, float2 hi) {
+        *reinterpret_cast<float4*>(p) = make_float4(lo.x, lo.y, hi.x, hi.y);
     }
 };
-template <> struct Vec<__nv_bfloat16> {
-    static constexpr int V = 8;
-    static __device__ __forceinline__ void load(const __nv_bfloat16* p, float (&v)[8]) {
-        const uint4 q = __ldg(reinterpret_cast<const uint4*>(p));
-        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[i]));
-            v[2 * i] = f.x;
-            v[2 * i + 1] = f.y;
-        }
+template <> struct Quad<__nv_bfloat16> {
+    static __device__ __forceinline__ void load(const uint8_t* s, float2& lo, float2& hi) {
+        const uint2 v = *reinterpret_cast<const uint2*>(s);
+        lo = make_float2(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u));
+        hi = make_float2(__uint_as_float(v.y << 16), __uint_as_float(v.y & 0xffff0000u));
     }
-    static __device__ __forceinline__ void store(__nv_bfloat16* p, const float (&v)[8]) {
-        uint32_t w[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const __nv_bfloat162 t = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
-            w[i] = *reinterpret_cast<const uint32_t*>(&t);
-        }
-        *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+    static __device__ __forceinline__ void store(__nv_bfloat16* p, float2 lo, float2 hi) {
+        const __nv_bfloat162 a = __floats2bfloat162_rn(lo.x, lo.y);
+        const __nv_bfloat162 b = __floats2bfloat162_rn(hi.x, hi.y);
+        *reinterpret_cast<uint2*>(p) = make_uint2(*reinterpret_cast<const uint32_t*>(&a),
+                                                  *reinterpret_cast<const uint32_t*>(&b));
     }
 };
 
+__device__ __forceinline__ float ex2_approx(float v) {
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(v));
+    return r;
+}
+__device__ __forceinline__ float rcp_approx(float v) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(v));
+    return r;
+}
+
+// silu(z) = z / (1 + e^-z) on a pair, e^-z = 2^(-z log2 e); a very negative z
+// gives 1 + e^-z = inf and 1/inf = 0.
+__device__ __forceinline__ float2 silu2(float2 z) {
+    constexpr float kNegLog2e = -1.4426950408889634f;
+    const float2 t = __fmul2_rn(z, make_float2(kNegLog2e, kNegLog2e));
+    const float2 d = __fadd2_rn(make_float2(ex2_approx(t.x), ex2_approx(t.y)),
+                                make_float2(1.0f, 1.0f));
+    return __fmul2_rn(z, make_float2(rcp_approx(d.x), rcp_approx(d.y)));
+}
+
+// xin[i] for channel c: x[i] for i >= 0, the carried input init[K-1+i] (zero
+// without one) for i < 0.
 template <typename T, int K>
-__global__ void __launch_bounds__(256) conv1d_kernel(ConvParams p) {
-    constexpr int V = Vec<T>::V;
-    constexpr int KM = K > 1 ? K - 1 : 1;
-    const int64_t L = p.seqlen, Cn = p.channels, ncv = Cn / V;
-    const int64_t nstrips = (L + TS - 1) / TS;
-    const int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    const int64_t b = blockIdx.y;
-    if (g >= ncv * nstrips) return;
-    const int64_t cv = g % ncv, strip = g / ncv;
-    const int64_t c0 = cv * V, t0 = strip * TS;
+__device__ __forceinline__ float xin_at(const ConvParams& p, const T* xb, int64_t b, int64_t c,
+                                        int64_t i) {
+    if (i >= 0) return to_f32(xb[i * p.channels + c]);
+    return p.init_state ? p.init_state[(b * p.channels + c) * (K - 1) + (K - 1 + i)] : 0.0f;
+}
 
-    float w[V][K], bias[V];
+template <typename T, int K, bool ACT>
+__global__ void __launch_bounds__(kMaxConsumers<T> + 32) conv1d_kernel(ConvParams p, int64_t seg) {
+    using namespace tc;
+    constexpr int KM = K > 1 ? K - 1 : 1;
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ __align__(8) uint64_t full[NSTAGE], empty[NSTAGE];
+    __shared__ int abort_flag, issued;
+
+    const int NT = blockDim.x - 32;  // consumer threads; the last warp is the producer
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t L = p.seqlen, Cn = p.channels, ncq = Cn / CPT;
+    const int64_t cqb = static_cast<int64_t>(blockIdx.x) * NT;  // first channel quad
+    const int nv = static_cast<int>(ncq - cqb < NT ? ncq - cqb : NT);
+    const uint32_t rowb = static_cast<uint32_t>(NT) * CPT * sizeof(T);
+    const uint32_t rb = static_cast<uint32_t>(nv) * CPT * sizeof(T);
+    const int64_t b = blockIdx.z;
+    const int64_t ta = static_cast<int64_t>(blockIdx.y) * seg;  // < L by the grid
+    const int64_t te = (ta + seg < L) ? ta + seg : L;
+    const int ntiles = static_cast<int>((te - ta + TT - 1) / TT);
+
+    if (tid == 0) {
 #pragma unroll
-    for (int v = 0; v < V; ++v) {
-#pragma unroll
-        for (int k = 0; k < K; ++k) w[v][k] = p.weight[(c0 + v) * K + k];
-        bias[v] = p.bias ? p.bias[c0 + v] : 0.0f;
+        for (int st = 0; st < NSTAGE; ++st) {
+            mbar_init(smem_u32(&full[st]), 1);
+            mbar_init(smem_u32(&empty[st]), static_cast<uint32_t>(NT / 32));
+        }
+        fence_mbar_init();
+        abort_flag = 0;
+        issued = 0;
     }
-    // window[j] = xin[t - (K-1) + j] for the next output token t
-    float win[KM][V];
-    const T* x = static_cast<const T*>(p.x) + b * L * Cn + c0;
+    __syncthreads();
+
+    if (warp == NT / 32) {
+        // ----- producer: tile j (TT token rows of this channel block) into stage j % NSTAGE
+        const char* xt = static_cast<const char*>(p.x) + ((b * L + ta) * Cn + cqb * CPT) * sizeof(T);
+        const int64_t xs = Cn * static_cast<int64_t>(sizeof(T));
+        const uint32_t sbase = smem_u32(smem);
+        int j = 0;
+        for (; j < ntiles; ++j) {
+            const int st = j % NSTAGE, use = j / NSTAGE;
+            bool ok = true;
+            if (use > 0 && lane == 0) ok = wait_or_abort(smem_u32(&empty[st]), (use - 1) & 1, &abort_flag);
+            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+            const int64_t left = te - ta - static_cast<int64_t>(j) * TT;
+            const int rows = left < TT ? static_cast<int>(left) : TT;
+            const uint32_t bar = smem_u32(&full[st]);
+            if (lane == 0) mbar_expect_tx(bar, static_cast<uint32_t>(rows) * rb);
+            __syncwarp();
+            if (lane < rows)
+                bulk_load_1d(sbase + static_cast<uint32_t>(st * TT + lane) * rowb,
+                             xt + (static_cast<int64_t>(j) * TT + lane) * xs, rb, bar);
+        }
+        if (lane == 0) issued = j;
+    } else {
+        // ----- consumers: channels c0..c0+3 of every token of the segment
+        const bool active = tid < nv;
+        const int64_t c0 = (cqb + tid) * CPT;
+        float2 w[K][2], bias[2];
 #pragma unroll
-    for (int j = 0; j < K - 1; ++j) {
-        const int64_t i = t0 - (K - 1) + j;
-        if (i >= 0) {
-            Vec<T>::load(x + i * Cn, win[j]);
-        } else {
+        for (int h = 0; h < 2; ++h) {
+            const int64_t c = c0 + 2 * h;
 #pragma unroll
-            for (int v = 0; v < V; ++v)
-                win[j][v] = p.init_state ? p.init_state[((b * Cn) + c0 + v) * (K - 1) + (K - 1 + i)] : 0.0f;
+            for (int k = 0; k < K; ++k)
+                w[k][h] = active ? make_float2(p.weight[c * K + k], p.weight[(c + 1) * K + k])
+                                 : make_float2(0.0f, 0.0f);
+            bias[h] = (active && p.bias) ? make_float2(p.bias[c], p.bias[c + 1])
+                                         : make_float2(0.0f, 0.0f);
+        }
+        const T* xb = static_cast<const T*>(p.x) + b * L * Cn;
+        T* y = static_cast<T*>(p.y) + b * L * Cn + c0;
+
+        // The first K-1 tokens of a sequence reach back into the carried
+        // inputs (fp32): a scalar pass over them, then the window holds x only.
+        const int64_t ts = (ta == 0 && K > 1) ? ((K - 1 < te) ? K - 1 : te) : ta;
+        if (active) {
+            for (int64_t t = ta; t < ts; ++t) {
+                float o[CPT];
+#pragma unroll
+                for (int v = 0; v < CPT; ++v) {
+                    float acc = (v & 1) ? bias[v >> 1].y : bias[v >> 1].x;
+#pragma unroll
+                    for (int k = 0; k < K; ++k) {
+                        const float wk = (v & 1) ? w[k][v >> 1].y : w[k][v >> 1].x;
+                        acc = fmaf(wk, xin_at<T, K>(p, xb, b, c0 + v, t - (K - 1) + k), acc);
+                    }
+                    o[v] = ACT ? silu_f32(acc) : acc;
+                }
+                Quad<T>::store(y + t * Cn, make_float2(o[0], o[1]), make_float2(o[2], o[3]));
+            }
+        }
+        // win[j] = x[t - (K-1) + j] for the next output token t (indices >= 0:
+        // a segment after the first starts at least TT >= K-1 tokens in)
+        float2 win[KM][2];
+        if (active && ts < te) {
+#pragma unroll
+            for (int jj = 0; jj < K - 1; ++jj) {
+                const T* q = xb + (ts - (K - 1) + jj) * Cn + c0;
+                win[jj][0] = make_float2(to_f32(q[0]), to_f32(q[1]));
+                win[jj][1] = make_float2(to_f32(q[2]), to_f32(q[3]));
+            }
+        }
+        // one output token from the staged row at s (fp32x2 FMAs in tap order)
+        auto step = [&](const uint8_t* s, int64_t t) {
+            float2 lo, hi;
+            Quad<T>::load(s, lo, hi);
+            float2 a0 = bias[0], a1 = bias[1];
+#pragma unroll
+            for (int k = 0; k < K - 1; ++k) {
+                a0 = __ffma2_rn(w[k][0], win[k][0], a0);
+                a1 = __ffma2_rn(w[k][1], win[k][1], a1);
+            }
+            a0 = __ffma2_rn(w[K - 1][0], lo, a0);
+            a1 = __ffma2_rn(w[K - 1][1], hi, a1);
+            if (ACT) {
+                a0 = silu2(a0);
+                a1 = silu2(a1);
+            }
+            Quad<T>::store(y + t * Cn, a0, a1);
+#pragma unroll
+            for (int k = 0; k + 1 < K - 1; ++k) {
+                win[k][0] = win[k + 1][0];
+                win[k][1] = win[k + 1][1];
+            }
+            if (K > 1) {
+                win[KM - 1][0] = lo;
+                win[KM - 1][1] = hi;
+            }
+        };
+        for (int j = 0; j < ntiles; ++j) {
+            const int st = j % NSTAGE;
+            const bool ok = wait_or_abort(smem_u32(&full[st]), (j / NSTAGE) & 1, &abort_flag);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            if (active) {
+                const int64_t tb = ta + static_cast<int64_t>(j) * TT;
+                const uint8_t* row = smem + static_cast<uint32_t>(st * TT) * rowb + tid * CPT * sizeof(T);
+                if (tb >= ts && tb + TT <= te) {
+#pragma unroll
+                    for (int r = 0; r < TT; ++r) step(row + r * rowb, tb + r);
+                } else {
+#pragma unroll
+                    for (int r = 0; r < TT; ++r)
+                        if (tb + r >= ts && tb + r < te) step(row + r * rowb, tb + r);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&empty[st]));
+        }
+        // the carried inputs after the last token: xin[L-(K-1) .. L-1] (they
+        // reach into init_state when L < K-1)
+        if (active && p.final_state && te == L && K > 1 && !abort_flag) {
+#pragma unroll
+            for (int v = 0; v < CPT; ++v)
+#pragma unroll
+                for (int jj = 0; jj < K - 1; ++jj)
+                    p.final_state[((b * Cn) + c0 + v) * (K - 1) + jj] =
+                        xin_at<T, K>(p, xb, b, c0 + v, L - (K - 1) + jj);
         }
     }
-    T* y = static_cast<T*>(p.y) + b * L * Cn + c0;
-    const int64_t t1 = (t0 + TS < L) ? t0 + TS : L;
-    for (int64_t t = t0; t < t1; ++t) {
-        float cur[V], out[V];
-        Vec<T>::load(x + t * Cn, cur);
-#pragma unroll
-        for (int v = 0; v < V; ++v) {
-            float acc = bias[v];
-#pragma unroll
-            for (int k = 0; k < K - 1; ++k) acc = fmaf(w[v][k], win[k][v], acc);
-            acc = fmaf(w[v][K - 1], cur[v], acc);
-            out[v] = p.activation ? silu_f32(acc) : acc;
-        }
-        Vec<T>::store(y + t * Cn, out);
-#pragma unroll
-        for (int k = 0; k + 1 < K - 1; ++k)
-#pragma unroll
-            for (int v = 0; v < V; ++v) win[k][v] = win[k + 1][v];
-        if (K > 1) {
-#pragma unroll
-            for (int v = 0; v < V; ++v) win[KM - 1][v] = cur[v];
-        }
-    }
-    if (p.final_state && t1 == L && K > 1) {
-#pragma unroll
-        for (int v = 0; v < V; ++v)
-#pragma unroll
-            for (int j = 0; j < K - 1; ++j) p.final_state[((b * Cn) + c0 + v) * (K - 1) + j] = win[j][v];
+    __syncthreads();
+    if (abort_flag && tid == 0) {
+        // A wait gave up: let the copies still in flight land (bounded)
+        // before the CTA's shared memory goes away, and report it.
+        for (int jj = issued - NSTAGE < 0 ? 0 : issued - NSTAGE; jj < issued; ++jj)
+            mbar_wait(smem_u32(&full[jj % NSTAGE]), (jj / NSTAGE) & 1);
+        atomicExch(&g_conv_status, static_cast<int>(SSD_ERR_TIMEOUT));
     }
 }
 
@@ -141,16 +278,59 @@ __global__ void __launch_bounds__(256) conv1d_update_kernel(ConvParams p) {
     static_cast<T*>(p.y)[i] = from_f32<T>(p.activation ? silu_f32(acc) : acc);
 }
 
+int sm_count() {
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+        cudaGetLastError();
+        n = 148;
+    }
+    return n;
+}
+
+// Forward grid: channel blocks of at most kMaxConsumers quads split evenly (a
+// multiple of 32 consumer threads, plus the producer warp), and the sequence
+// cut into segments of whole tiles so that the CTAs of all batch rows fill
+// one wave of the SMs at the kernel's occupancy.
+template <typename T, int K, bool ACT>
+cudaError_t launch_fwd(const ConvParams& p, cudaStream_t s) {
+    constexpr int MAXNT = kMaxConsumers<T>;
+    const int64_t ncq = p.channels / CPT;
+    const int64_t nblk = (ncq + MAXNT - 1) / MAXNT;
+    const int nt = static_cast<int>(((ncq + nblk - 1) / nblk + 31) / 32 * 32);
+    const size_t smem = static_cast<size_t>(NSTAGE) * TT * nt * CPT * sizeof(T);
+    static int occ[MAXNT / 32 + 1];  // CTAs per SM by consumer count; benign race
+    int& per_sm = occ[nt / 32];
+    if (per_sm == 0) {
+        // a full ring (64 KB) exceeds the default 48 KB dynamic limit
+        cudaError_t e = cudaFuncSetAttribute(conv1d_kernel<T, K, ACT>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             NSTAGE * TT * MAXROWB);
+        if (e != cudaSuccess) return e;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, conv1d_kernel<T, K, ACT>,
+                                                          nt + 32, smem) != cudaSuccess ||
+            per_sm < 1) {
+            cudaGetLastError();
+            per_sm = 1;
+        }
+    }
+    const int64_t slots = static_cast<int64_t>(sm_count()) * per_sm;
+    const int64_t max_seg = (p.seqlen + TT - 1) / TT;
+    int64_t nseg = slots / (nblk * p.batch);
+    nseg = nseg < 1 ? 1 : (nseg > max_seg ? max_seg : nseg);
+    const int64_t seg = ((p.seqlen + nseg - 1) / nseg + TT - 1) / TT * TT;
+    nseg = (p.seqlen + seg - 1) / seg;
+    dim3 grid(static_cast<unsigned>(nblk), static_cast<unsigned>(nseg),
+              static_cast<unsigned>(p.batch));
+    conv1d_kernel<T, K, ACT><<<grid, nt + 32, smem, s>>>(p, seg);
+    return cudaGetLastError();
+}
+
 template <typename T, int K>
 cudaError_t launch_k(const ConvParams& p, bool update, cudaStream_t s) {
-    if (update) {
-        const int64_t n = p.batch * p.channels;
-        conv1d_update_kernel<T, K><<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(p);
-    } else {
-        const int64_t items = (p.channels / Vec<T>::V) * ((p.seqlen + TS - 1) / TS);
-        dim3 grid(static_cast<unsigned>((items + 255) / 256), static_cast<unsigned>(p.batch));
-        conv1d_kernel<T, K><<<grid, 256, 0, s>>>(p);
-    }
+    if (!update) return p.activation ? launch_fwd<T, K, true>(p, s) : launch_fwd<T, K, false>(p, s);
+    const int64_t n = p.batch * p.channels;
+    conv1d_update_kernel<T, K><<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(p);
     return cudaGetLastError();
 }
 
@@ -173,5 +353,15 @@ cudaError_t launch_conv1d(const ConvParams& p, bool update, cudaStream_t s) {
 
 template cudaError_t launch_conv1d<float>(const ConvParams&, bool, cudaStream_t);
 template cudaError_t launch_conv1d<__nv_bfloat16>(const ConvParams&, bool, cudaStream_t);
+
+cudaError_t conv1d_take_status(int* v, cudaStream_t s) {
+    int zero = 0;
+    cudaError_t e = cudaMemcpyFromSymbolAsync(v, g_conv_status, sizeof(int), 0,
+                                              cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess)
+        e = cudaMemcpyToSymbolAsync(g_conv_status, &zero, sizeof(int), 0, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    return e;
+}
 
 }  // namespace ssd

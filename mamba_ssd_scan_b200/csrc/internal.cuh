@@ -164,6 +164,8 @@ template <typename T> cudaError_t launch_state_passing(const FwdParams& p, cudaS
 template <typename T> cudaError_t launch_chunk_scan_ffma(const FwdParams& p, cudaStream_t s);
 template <typename T> cudaError_t launch_state_update(const DecodeParams& p, cudaStream_t s);
 template <typename T> cudaError_t launch_conv1d(const ConvParams& p, bool update, cudaStream_t s);
+// Copies the forward kernel's device status word to *v and clears it (synchronises s).
+cudaError_t conv1d_take_status(int* v, cudaStream_t s);
 
 // Tensor-core (tcgen05) variants for bf16 inputs, with their shape ranges.
 bool chunk_state_tc_supported(const FwdParams& p);

@@ -131,6 +131,16 @@ __device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity) {
     return false;
 }
 
+// Bounded mbarrier wait that also gives up when another role has aborted.
+__device__ __forceinline__ bool wait_or_abort(uint32_t mbar, uint32_t parity, volatile int* abort) {
+    for (uint32_t i = 0; i < kSpinLimit; ++i) {
+        if (mbar_try_wait_hint(mbar, parity, 200)) return true;
+        if ((i & 63) == 63 && *abort) return false;
+    }
+    *abort = 1;
+    return false;
+}
+
 __device__ __forceinline__ void fence_before_sync() {
     asm volatile("tcgen05.fence::before_thread_sync;" : : : "memory");
 }

@@ -50,6 +50,18 @@ __device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, uint32_t sr
         : "l"(reinterpret_cast<uint64_t>(map)), "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
         : "memory");
 }
+// One contiguous run of `bytes` from global into shared memory (both
+// addresses 16-byte aligned, bytes a multiple of 16); completes `bytes` on
+// mbar.  A plain bulk copy, never multicast.
+__device__ __forceinline__ void bulk_load_1d(uint32_t dst, const void* src, uint32_t bytes,
+                                             uint32_t mbar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        :
+        : "r"(dst), "l"(src), "r"(bytes), "r"(mbar)
+        : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit_group() {
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }

@@ -72,9 +72,32 @@ DECODE_CONFIGS = {
     "decode_b256_H80": DecodeConfig("decode_b256_H80", 256, 80, 64, 128, 8, 1024,
                                     torch.bfloat16),
 }
+@dataclasses.dataclass(frozen=True)
+class ConvConfig:
+    """The causal depthwise convolution over the concatenated x, B and C
+    channels of a Mamba-2 block: channels = nheads*headdim + 2*ngroups*dstate."""
+    name: str
+    batch: int
+    seqlen: int       # 1 for the decode step
+    channels: int
+    width: int
+    dtype: torch.dtype
+    steps: int = 0    # decode steps replayed (decode only)
+    layers: int = 1   # distinct carried states cycled through (decode only)
+
+
+CONV_CONFIGS = {
+    # the x, B, C channels of the b8 L4096 forward workload (32*64 + 2*128)
+    "conv1d_bf16_b8_L4096_C2304": ConvConfig("conv1d_bf16_b8_L4096_C2304", 8, 4096, 2304, 4,
+                                             torch.bfloat16),
+    # the decode workload's channels (80*64 + 2*8*128); 8 layers' states (176 MB) > L2
+    "conv1d_update_b256_C7168": ConvConfig("conv1d_update_b256_C7168", 256, 1, 7168, 4,
+                                           torch.bfloat16, steps=1024, layers=8),
+}
 # the seed offset of each workload (seed = 1234 + offset)
 SEED_OFFSET = {"fwd_f32_small": 0, "fwd_bf16_b4_L1024": 1, "fwd_bf16_b8_L4096_init": 2,
-               "fwd_bf16_b1_L65536_G8": 3, "decode_b256_H80": 4}
+               "fwd_bf16_b1_L65536_G8": 3, "decode_b256_H80": 4,
+               "conv1d_bf16_b8_L4096_C2304": 5, "conv1d_update_b256_C7168": 6}
 
 
 def _uniform(gen, shape, lo, hi):
