@@ -8,8 +8,10 @@ One step = one ssd_fwd call (chunk_cumsum -> chunk_state -> state_passing ->
 chunk_scan) over one batch of the headline workload, bf16 in / fp32 accumulate,
 batch 4 x seqlen 1024, 24 heads x headdim 64, dstate 64, 1 group, chunk 256.
 Inputs are seeded synthetic data already resident in HBM; the working set
-(26 MB) fits in L2, so a 256 MB buffer is rewritten before every timed step
-(outside the timed events) to flush it.  Each step is timed with CUDA events on
+(26 MB) fits in L2, so a 256 MB buffer is written and then read back before
+every timed step (outside the timed events) to flush it: the read makes the
+written lines leave L2 before the timed region, so their write-back is not
+charged to the step.  Each step is timed with CUDA events on
 the launching stream; ms_per_step is the mean over the K timed steps, the max
 over ranks.  Under torchrun every rank runs its own independent batch (weak
 scaling, no collective on the data path).
@@ -230,8 +232,15 @@ def main_ours(args):
     stream = torch.cuda.current_stream()
     flush_buf = torch.empty(args.flush_mb << 20, dtype=torch.uint8, device=dev)
 
+    flush_f = flush_buf.view(torch.float32)
+    flush_acc = torch.empty((), dtype=torch.float32, device=dev)
+
     def flush():
+        # write a buffer larger than L2, then read it back: the written lines
+        # are evicted (written back) here, outside the timed region, and L2
+        # holds none of the step's data
         flush_buf.fill_(1)
+        torch.sum(flush_f, dim=0, out=flush_acc)
 
     y = torch.empty_like(d["x"])
     fin = (torch.empty((cfg.batch, cfg.nheads, cfg.headdim, cfg.dstate), device=dev)
@@ -399,7 +408,8 @@ def main_ours(args):
                    "nheads": cfg.nheads, "headdim": cfg.headdim, "dstate": cfg.dstate,
                    "ngroups": cfg.ngroups, "chunk": cfg.chunk, "global_batch":
                    cfg.batch * world, "parallelism": f"dp{world}" if world > 1 else "single",
-                   "l2": f"flushed ({args.flush_mb} MB write) before every timed step"},
+                   "l2": f"flushed before every timed step ({args.flush_mb} MB write, then "
+                         "a read of it, so its write-back ends before the timed region)"},
         "roofline": roofline,
         "kernel_ms": kms,
         "e2e": e2e,

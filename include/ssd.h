@@ -253,7 +253,10 @@ ssd_status ssd_conv1d_check_status(void* stream);
  * state [batch, channels, width - 1] fp32 holds the previous width - 1 inputs,
  * oldest first, and is shifted in place to end with x;
  *   y[c] = silu(bias[c] + sum_{k<width-1} w[c, k] state[c, k] + w[c, width-1] x[c]).
- * x, y [batch, channels] dtype.  Supported: 1 <= width <= 8. */
+ * x, y [batch, channels] dtype; weight, bias as for ssd_causal_conv1d.
+ * Supported: 1 <= width <= 8; channels a multiple of 8 (bf16) or 4 (fp32)
+ *   (else SSD_ERR_UNSUPPORTED); every pointer 16-byte aligned (else
+ *   SSD_ERR_INVALID_ARG). */
 typedef struct {
     int64_t batch, channels, width;
     int32_t dtype;

@@ -315,10 +315,11 @@ ssd_status ssd_conv1d_update(const ssd_conv1d_update_args* a, void* stream) {
     if (!a) return SSD_ERR_INVALID_ARG;
     if (a->batch <= 0 || a->channels <= 0 || a->width <= 0) return SSD_ERR_INVALID_ARG;
     if (a->dtype != SSD_F32 && a->dtype != SSD_BF16) return SSD_ERR_INVALID_ARG;
-    if (a->width > 8) return SSD_ERR_UNSUPPORTED;
-    if (!check_ptr(a->state, a->width == 1, false) || !check_ptr(a->x, false, false) ||
-        !check_ptr(a->weight, false, false) || !check_ptr(a->bias, true, false) ||
-        !check_ptr(a->y, false, false))
+    if (a->width > 8 || a->channels % (a->dtype == SSD_BF16 ? 8 : 4) != 0)
+        return SSD_ERR_UNSUPPORTED;
+    if (!check_ptr(a->state, a->width == 1, true) || !check_ptr(a->x, false, true) ||
+        !check_ptr(a->weight, false, true) || !check_ptr(a->bias, true, true) ||
+        !check_ptr(a->y, false, true))
         return SSD_ERR_INVALID_ARG;
     ssd::ConvParams p;
     p.batch = a->batch;

@@ -256,26 +256,61 @@ __global__ void __launch_bounds__(kMaxConsumers<T> + 32) conv1d_kernel(ConvParam
     }
 }
 
+// Decode: one thread per (batch row, 4 channels); the carried state of the 4
+// channels (4 x (K-1) fp32, contiguous) moves as 16-byte vectors.
 template <typename T, int K>
 __global__ void __launch_bounds__(256) conv1d_update_kernel(ConvParams p) {
     constexpr int KM = K > 1 ? K - 1 : 1;
-    const int64_t Cn = p.channels;
+    const int64_t nq = p.channels / CPT;
     const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    if (i >= p.batch * Cn) return;
-    const int64_t c = i % Cn;
-    float* s = p.update_state + i * (K - 1);
-    float st[KM];
+    if (i >= p.batch * nq) return;
+    const int64_t c0 = (i % nq) * CPT;
+    // consecutive decode steps go out with programmatic dependent launch:
+    // wait for the previous step's state, then let the next step's CTAs in
+    grid_dep_wait();
+    grid_dep_launch();
+    float st[CPT * KM];
+    float4* s4 = reinterpret_cast<float4*>(p.update_state + i * CPT * (K - 1));
 #pragma unroll
-    for (int k = 0; k < K - 1; ++k) st[k] = s[k];
-    const float xv = to_f32(static_cast<const T*>(p.x)[i]);
-    float acc = p.bias ? p.bias[c] : 0.0f;
+    for (int q = 0; q < K - 1; ++q) {
+        const float4 v = s4[q];
+        st[4 * q] = v.x; st[4 * q + 1] = v.y; st[4 * q + 2] = v.z; st[4 * q + 3] = v.w;
+    }
+    float2 lo, hi;
+    Quad<T>::load(reinterpret_cast<const uint8_t*>(static_cast<const T*>(p.x) + i * CPT), lo, hi);
+    const float xv[CPT] = {lo.x, lo.y, hi.x, hi.y};
+    float wt[CPT * K];
+    const float4* w4 = reinterpret_cast<const float4*>(p.weight + c0 * K);
 #pragma unroll
-    for (int k = 0; k < K - 1; ++k) acc = fmaf(p.weight[c * K + k], st[k], acc);
-    acc = fmaf(p.weight[c * K + K - 1], xv, acc);
+    for (int q = 0; q < K; ++q) {
+        const float4 v = __ldg(w4 + q);
+        wt[4 * q] = v.x; wt[4 * q + 1] = v.y; wt[4 * q + 2] = v.z; wt[4 * q + 3] = v.w;
+    }
+    const float4 bv = p.bias ? __ldg(reinterpret_cast<const float4*>(p.bias + c0))
+                             : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    const float bias[CPT] = {bv.x, bv.y, bv.z, bv.w};
+    float o[CPT];
 #pragma unroll
-    for (int k = 0; k + 1 < K - 1; ++k) s[k] = st[k + 1];
-    if (K > 1) s[KM - 1] = xv;
-    static_cast<T*>(p.y)[i] = from_f32<T>(p.activation ? silu_f32(acc) : acc);
+    for (int v = 0; v < CPT; ++v) {
+        // channel v's taps are wt[v*K .. v*K+K-1], its state st[v*(K-1) ..]
+        float acc = bias[v];
+#pragma unroll
+        for (int k = 0; k < K - 1; ++k) acc = fmaf(wt[v * K + k], st[v * (K - 1) + k], acc);
+        acc = fmaf(wt[v * K + K - 1], xv[v], acc);
+        o[v] = p.activation ? silu_f32(acc) : acc;
+    }
+    // shift each channel's window by one token, the new input last
+    float ns[CPT * KM];
+#pragma unroll
+    for (int v = 0; v < CPT; ++v) {
+#pragma unroll
+        for (int k = 0; k + 1 < K - 1; ++k) ns[v * (K - 1) + k] = st[v * (K - 1) + k + 1];
+        if (K > 1) ns[v * (K - 1) + K - 2] = xv[v];
+    }
+#pragma unroll
+    for (int q = 0; q < K - 1; ++q)
+        s4[q] = make_float4(ns[4 * q], ns[4 * q + 1], ns[4 * q + 2], ns[4 * q + 3]);
+    Quad<T>::store(static_cast<T*>(p.y) + i * CPT, make_float2(o[0], o[1]), make_float2(o[2], o[3]));
 }
 
 int sm_count() {
@@ -329,9 +364,9 @@ cudaError_t launch_fwd(const ConvParams& p, cudaStream_t s) {
 template <typename T, int K>
 cudaError_t launch_k(const ConvParams& p, bool update, cudaStream_t s) {
     if (!update) return p.activation ? launch_fwd<T, K, true>(p, s) : launch_fwd<T, K, false>(p, s);
-    const int64_t n = p.batch * p.channels;
-    conv1d_update_kernel<T, K><<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(p);
-    return cudaGetLastError();
+    const int64_t n = p.batch * (p.channels / CPT);
+    return launch_kernel(conv1d_update_kernel<T, K>, dim3(static_cast<unsigned>((n + 255) / 256)),
+                         dim3(256), 0, s, true, p);
 }
 
 }  // namespace

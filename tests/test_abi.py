@@ -123,3 +123,7 @@ def test_conv1d_rejects_bad_args(lib):
     assert lib.ssd_conv1d_update(ctypes.byref(u), None) == 1        # null pointers
     u.width = 0
     assert lib.ssd_conv1d_update(ctypes.byref(u), None) == 1
+    u.width, u.channels = 4, 6
+    assert lib.ssd_conv1d_update(ctypes.byref(u), None) == 2        # fp32 channels % 4
+    u.width = 9
+    assert lib.ssd_conv1d_update(ctypes.byref(u), None) == 2        # width beyond 8
