@@ -53,6 +53,8 @@ def parse_args():
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--flush-mb", type=int, default=256)
+    ap.add_argument("--conv-only", action="store_true",
+                    help="time only the convolution workloads (one JSON line of them)")
     return ap.parse_args()
 
 
@@ -224,12 +226,6 @@ def main_ours(args):
 
     ssd.load_library()
     peaks = load_peaks()
-    cfg = synthetic.FWD_CONFIGS[args.workload]
-    seed = rank_seed(1234 + synthetic.SEED_OFFSET[cfg.name], rank)
-    inp = synthetic.make_config_inputs(cfg, seed)
-    d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
-    elt = d["x"].element_size()
-    stream = torch.cuda.current_stream()
     flush_buf = torch.empty(args.flush_mb << 20, dtype=torch.uint8, device=dev)
 
     flush_f = flush_buf.view(torch.float32)
@@ -241,6 +237,19 @@ def main_ours(args):
         # holds none of the step's data
         flush_buf.fill_(1)
         torch.sum(flush_f, dim=0, out=flush_acc)
+
+    if args.conv_only:
+        res = conv_workloads(ssd, synthetic, dev, flush, peaks, rank, world, ranks_max)
+        if rank == 0:
+            print(json.dumps({"workloads": res, "peaks_source": peaks["source"]}), flush=True)
+        return
+
+    cfg = synthetic.FWD_CONFIGS[args.workload]
+    seed = rank_seed(1234 + synthetic.SEED_OFFSET[cfg.name], rank)
+    inp = synthetic.make_config_inputs(cfg, seed)
+    d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
+    elt = d["x"].element_size()
+    stream = torch.cuda.current_stream()
 
     y = torch.empty_like(d["x"])
     fin = (torch.empty((cfg.batch, cfg.nheads, cfg.headdim, cfg.dstate), device=dev)
@@ -431,6 +440,8 @@ KERNEL_SOURCES = {
     "chunk_state": ["chunk_state_tc.cu", "tcgen05.cuh", "tma.cuh", "internal.cuh"],
     "state_passing": ["state_passing.cu", "internal.cuh"],
     "chunk_cumsum": ["chunk_cumsum.cu", "internal.cuh"],
+    "conv1d": ["conv1d.cu", "tcgen05.cuh", "tma.cuh", "internal.cuh"],
+    "conv1d_update": ["conv1d.cu", "tcgen05.cuh", "tma.cuh", "internal.cuh"],
 }
 
 
@@ -665,6 +676,7 @@ def conv_workloads(ssd, synthetic, dev, flush, peaks, rank, world, ranks_max, st
     torch.cuda.synchronize()
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(steps)]
+    gpu_head_start(2.0)
     for a, b_ in evs:
         flush()
         a.record(stream)
@@ -678,7 +690,8 @@ def conv_workloads(ssd, synthetic, dev, flush, peaks, rank, world, ranks_max, st
     out[cfg.name] = {"tokens_per_s": job_throughput(cfg.batch * cfg.seqlen, world, ms), "ms": ms,
                      "achieved_gbs": nbytes / (ms * 1e-3) / 1e9,
                      "hbm_frac": nbytes / (ms * 1e-3) / (peaks["hbm_gbs"] * 1e9),
-                     "bytes": nbytes, "l2": "flushed"}
+                     "bytes": nbytes, "traffic": measured_traffic("conv1d", cfg.name),
+                     "l2": "flushed"}
     del d, y, fin
 
     cfg = synthetic.CONV_CONFIGS["conv1d_update_b256_C7168"]
@@ -718,7 +731,8 @@ def conv_workloads(ssd, synthetic, dev, flush, peaks, rank, world, ranks_max, st
     out[cfg.name] = {"us_per_step": us, "steps": cfg.steps, "graph": True, "layers": cfg.layers,
                      "achieved_gbs": step_bytes / (us * 1e-6) / 1e9,
                      "hbm_frac": step_bytes / (us * 1e-6) / (peaks["hbm_gbs"] * 1e9),
-                     "bytes_per_step": step_bytes}
+                     "bytes_per_step": step_bytes,
+                     "traffic": measured_traffic("conv1d_update", cfg.name)}
     del g, states
     torch.cuda.empty_cache()
     return out
