@@ -64,6 +64,8 @@ class Oracle:
         lib.oracle_ssd_chunked.argtypes = [_i64] * 7 + [_dp] * 14
         lib.oracle_state_update.restype = None
         lib.oracle_state_update.argtypes = [_i64] * 5 + [_dp] * 9
+        lib.oracle_ssd_bwd.restype = None
+        lib.oracle_ssd_bwd.argtypes = [_i64] * 6 + [_dp] * 18
         lib.oracle_gate.restype = None
         lib.oracle_gate.argtypes = [_dp, _dp, _i64]
         lib.oracle_causal_conv1d.restype = None
@@ -123,6 +125,27 @@ class Oracle:
         if z is not None:
             y = self.gate(y, z)
         return y, fin
+
+    def ssd_bwd(self, x, dt, A, B, C, D=None, dt_bias=None, init_state=None, dy=None,
+                d_final=None):
+        """Gradients of J = sum dy.y + sum d_final*final_state with respect to
+        every input of ssd_fwd (float64).  Returns a dict with dx, ddt (with
+        respect to the raw dt), dA, dB, dC, dD, ddt_bias, d_init."""
+        x, dt, A, B, C = (self._f64(t) for t in (x, dt, A, B, C))
+        D, dt_bias, init = self._f64(D), self._f64(dt_bias), self._f64(init_state)
+        dy, dfin = self._f64(dy), self._f64(d_final)
+        b, L, H, P = x.shape
+        G, N = B.shape[2], B.shape[3]
+        assert dy.shape == x.shape
+        out = dict(dx=np.zeros_like(x), ddt=np.zeros_like(dt), dA=np.zeros(H),
+                   dB=np.zeros_like(B), dC=np.zeros_like(C), dD=np.zeros(H),
+                   ddt_bias=np.zeros(H), d_init=np.zeros((b, H, P, N)))
+        p = self._ptr
+        self.lib.oracle_ssd_bwd(b, L, H, P, N, G, p(x), p(dt), p(A), p(B), p(C), p(D),
+                                p(dt_bias), p(init), p(dy), p(dfin), p(out["dx"]),
+                                p(out["ddt"]), p(out["dA"]), p(out["dB"]), p(out["dC"]),
+                                p(out["dD"]), p(out["ddt_bias"]), p(out["d_init"]))
+        return out
 
     def ssd_chunked(self, x, dt, A, B, C, D=None, dt_bias=None, init_state=None,
                     chunk: int = 256, z=None):

@@ -40,6 +40,8 @@
  *                        body applied once; the page "MAMBA-2 Reference
  *                        Implementations Comparison", section 1.3, names the
  *                        Mamba2Cache this state lives in)
+ *   oracle_ssd_bwd       the gradients of oracle_ssd_fwd (reverse-mode
+ *                        differentiation of the recurrence, token by token)
  *
  * Pins (tests/, CPU only): the masked-attention (quadratic) dual form by brute
  * force, the A = 0 cumulative-sum closed form, chunk-size invariance, split /
@@ -183,6 +185,174 @@ void oracle_ssd_fwd(int64_t batch, int64_t L, int64_t H, int64_t P,
             memcpy(final_state + bh * P * N, S, sizeof(double) * (size_t)(P * N));
         free(S);
     }
+}
+
+/*
+ * The backward pass of oracle_ssd_fwd: the gradients of the scalar
+ *   J = sum_t dy_t . y_t + d_final : h_L
+ * with respect to every input, by reverse-mode differentiation of the
+ * recurrence one line at a time.  With g_t = dJ/dh_t (P x N), a_t = dt_t A_h
+ * the log decay and h_0 the initial state:
+ *   g_L = d_final + dy_L C_L^T,   g_t = e^{a_{t+1}} g_{t+1} + dy_t C_t^T
+ *   dC_t      = h_t^T dy_t                      (from y_t = C_t . h_t)
+ *   dx_t      = D_h dy_t + dt_t g_t B_t          (h_t receives dt_t x_t B_t^T)
+ *   dB_t      = dt_t g_t^T x_t
+ *   da_t      = e^{a_t} <g_t, h_{t-1}>           (h_t = e^{a_t} h_{t-1} + ...)
+ *   ddt_t     = x_t . (g_t B_t) + A_h da_t,   dA_h += dt_t da_t
+ *   ddt_raw_t = ddt_t sigmoid(dt_raw_t + dt_bias_h),   ddt_bias_h += ddt_raw_t
+ *   dD_h     += dy_t . x_t,   d_init = dJ/dh_0 = e^{a_1} g_1
+ * The recurrence is the one of "MAMBA-2 Reference Implementations
+ * Comparison", section 2.2; the pages list the gradients a backward pass must
+ * return ("MAMBA-2 Implementation Gaps") but not their formulas, which follow
+ * from the chain rule alone (softplus'(u) = sigmoid(u)).
+ *
+ * dy [b,L,H,P]; d_final [b,H,P,N] or NULL (zero).  Outputs shaped like the
+ * inputs: dx, ddt_raw, dB, dC (dB, dC summed over the heads of a group),
+ * d_init [b,H,P,N]; dA, dD, ddt_bias [H] summed over batch and time.  d_init,
+ * dD and ddt_bias may be NULL.  Sums over heads and batch rows are taken in a
+ * fixed order after the parallel part.
+ */
+void oracle_ssd_bwd(int64_t batch, int64_t L, int64_t H, int64_t P,
+                    int64_t N, int64_t G,
+                    const double* x, const double* dt_raw, const double* A,
+                    const double* B, const double* C, const double* D,
+                    const double* dt_bias, const double* init,
+                    const double* dy, const double* d_final,
+                    double* dx, double* ddt_raw, double* dA, double* dB,
+                    double* dC, double* dD, double* ddt_bias, double* d_init) {
+    const int64_t PN = P * N;
+    double* dBh = (double*)calloc((size_t)(batch * H * L * N), sizeof(double));
+    double* dCh = (double*)calloc((size_t)(batch * H * L * N), sizeof(double));
+    double* sums = (double*)calloc((size_t)(batch * H * 3), sizeof(double));
+    int64_t bh;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (bh = 0; bh < batch * H; ++bh) {
+        const int64_t b = bh / H, h = bh % H, g = group_of(h, H, G);
+        const double Dh = D ? D[h] : 0.0;
+        double* hs = (double*)malloc(sizeof(double) * (size_t)((L + 1) * PN));
+        double* gr = (double*)malloc(sizeof(double) * (size_t)PN);
+        double* dxs = (double*)malloc(sizeof(double) * (size_t)P);
+        /* forward, keeping every state: hs[t] = h_t, hs[0] = h_0 */
+        if (init)
+            memcpy(hs, init + bh * PN, sizeof(double) * (size_t)PN);
+        else
+            memset(hs, 0, sizeof(double) * (size_t)PN);
+        for (int64_t t = 0; t < L; ++t) {
+            const int64_t it = (b * L + t) * H + h;
+            const double dt = dt_of(dt_raw, dt_bias, it, h);
+            const double a = exp(dt * A[h]);
+            const double* xt = x + it * P;
+            const double* Bt = B + ((b * L + t) * G + g) * N;
+            const double* hp = hs + t * PN;
+            double* hn = hs + (t + 1) * PN;
+            for (int64_t p = 0; p < P; ++p)
+                for (int64_t n = 0; n < N; ++n)
+                    hn[p * N + n] = a * hp[p * N + n] + dt * xt[p] * Bt[n];
+        }
+        /* backward */
+        if (d_final)
+            memcpy(gr, d_final + bh * PN, sizeof(double) * (size_t)PN);
+        else
+            memset(gr, 0, sizeof(double) * (size_t)PN);
+        double sA = 0.0, sD = 0.0, sbias = 0.0;
+        for (int64_t t = L - 1; t >= 0; --t) {
+            const int64_t it = (b * L + t) * H + h;
+            const double u = dt_raw[it] + (dt_bias ? dt_bias[h] : 0.0);
+            const double dt = dt_of(dt_raw, dt_bias, it, h);
+            const double a = exp(dt * A[h]);
+            const double* xt = x + it * P;
+            const double* Bt = B + ((b * L + t) * G + g) * N;
+            const double* Ct = C + ((b * L + t) * G + g) * N;
+            const double* dyt = dy + it * P;
+            const double* ht = hs + (t + 1) * PN;
+            const double* hp = hs + t * PN;
+            double* dBt = dBh + (bh * L + t) * N;
+            double* dCt = dCh + (bh * L + t) * N;
+#if ORACLE_MUTANT != 17
+            for (int64_t p = 0; p < P; ++p)          /* g_t = ... + dy_t C_t^T */
+                for (int64_t n = 0; n < N; ++n) gr[p * N + n] += dyt[p] * Ct[n];
+#endif
+            for (int64_t n = 0; n < N; ++n) {
+                double acc = 0.0;
+                for (int64_t p = 0; p < P; ++p) acc += dyt[p] * ht[p * N + n];
+                dCt[n] = acc;
+            }
+            for (int64_t p = 0; p < P; ++p) {
+                double acc = 0.0;
+                for (int64_t n = 0; n < N; ++n) acc += gr[p * N + n] * Bt[n];
+                dxs[p] = acc;
+                dx[it * P + p] = Dh * dyt[p] + dt * acc;
+            }
+            for (int64_t n = 0; n < N; ++n) {
+                double acc = 0.0;
+                for (int64_t p = 0; p < P; ++p) acc += gr[p * N + n] * xt[p];
+                dBt[n] = dt * acc;
+            }
+            double gh = 0.0, xdxs = 0.0, dyx = 0.0;
+            for (int64_t k = 0; k < PN; ++k) gh += gr[k] * hp[k];
+            for (int64_t p = 0; p < P; ++p) {
+                xdxs += xt[p] * dxs[p];
+                dyx += dyt[p] * xt[p];
+            }
+            const double da = a * gh;
+#if ORACLE_MUTANT == 15
+            const double ddt = xdxs;
+#else
+            const double ddt = xdxs + A[h] * da;
+#endif
+            sA += dt * da;
+#if ORACLE_MUTANT == 16
+            const double dr = ddt;
+            (void)u;
+#else
+            const double dr = ddt / (1.0 + exp(-u));
+#endif
+            ddt_raw[it] = dr;
+            sbias += dr;
+            sD += dyx;
+#if ORACLE_MUTANT == 17
+            for (int64_t p = 0; p < P; ++p)
+                for (int64_t n = 0; n < N; ++n) gr[p * N + n] += dyt[p] * Ct[n];
+#endif
+#if ORACLE_MUTANT != 14
+            for (int64_t k = 0; k < PN; ++k) gr[k] *= a;   /* now dJ/dh_{t-1} */
+#endif
+        }
+        if (d_init) memcpy(d_init + bh * PN, gr, sizeof(double) * (size_t)PN);
+        sums[bh * 3 + 0] = sA;
+        sums[bh * 3 + 1] = sD;
+        sums[bh * 3 + 2] = sbias;
+        free(dxs);
+        free(gr);
+        free(hs);
+    }
+    for (int64_t h = 0; h < H; ++h) {
+        double sA = 0.0, sD = 0.0, sb = 0.0;
+        for (int64_t b = 0; b < batch; ++b) {
+            sA += sums[(b * H + h) * 3 + 0];
+            sD += sums[(b * H + h) * 3 + 1];
+            sb += sums[(b * H + h) * 3 + 2];
+        }
+        dA[h] = sA;
+        if (dD) dD[h] = sD;
+        if (ddt_bias) ddt_bias[h] = sb;
+    }
+    for (int64_t b = 0; b < batch; ++b)
+        for (int64_t t = 0; t < L; ++t)
+            for (int64_t g = 0; g < G; ++g)
+                for (int64_t n = 0; n < N; ++n) {
+                    double sb = 0.0, sc = 0.0;
+                    for (int64_t h = 0; h < H; ++h) {
+                        if (group_of(h, H, G) != g) continue;
+                        sb += dBh[((b * H + h) * L + t) * N + n];
+                        sc += dCh[((b * H + h) * L + t) * N + n];
+                    }
+                    dB[((b * L + t) * G + g) * N + n] = sb;
+                    dC[((b * L + t) * G + g) * N + n] = sc;
+                }
+    free(sums);
+    free(dCh);
+    free(dBh);
 }
 
 /*

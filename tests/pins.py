@@ -14,7 +14,9 @@ disagrees with something the pages or the mathematics fix independently:
 * special cases: C = 0, x = 0, full decay, L = 1, causality (the "no future
   leakage" test of "MAMBA-2 Implementation Gaps", Testing Strategy);
 * softplus values fixed by its definition;
-* a half-decay example worked by hand (tests/golden/half_decay_by_hand.json).
+* a half-decay example worked by hand (tests/golden/half_decay_by_hand.json);
+* the backward pass: central finite differences of the forward, and torch's
+  autodiff of the dual form.
 
 They are plain functions so that the mutant test can run every pin against
 deliberately wrong builds of the oracle and check that each one is caught.
@@ -293,6 +295,92 @@ def pin_conv1d(orc):
     _close(ya - yn, yl, 1e-13, "silu(u) - silu(-u) = u")
 
 
+def _bwd_loss(orc, case, dy, dfin):
+    y, fin = orc.ssd_fwd(**case)
+    return float(np.sum(dy * y) + np.sum(dfin * fin))
+
+
+def pin_bwd_finite_differences(orc):
+    """The backward pass against central finite differences of the forward
+    oracle: J = sum dy.y + sum d_final*final, dJ/dtheta ~ (J(theta + e) -
+    J(theta - e)) / 2e for every element of every input (x, raw dt, A, B, C,
+    D, dt_bias, initial state), groups shared by two heads.  The truncation
+    error is O(e^2) and the rounding error O(1e-16 |J| / e), both far below
+    the tolerance; any wrong term of the adjoint is O(1)."""
+    case = _rand_case(21, b=2, L=7, H=4, P=3, N=5, G=2)
+    rng = np.random.default_rng(22)
+    dy = rng.standard_normal(case["x"].shape)
+    dfin = rng.standard_normal(case["init_state"].shape)
+    gr = orc.ssd_bwd(**case, dy=dy, d_final=dfin)
+    names = {"x": "dx", "dt": "ddt", "A": "dA", "B": "dB", "C": "dC", "D": "dD",
+             "dt_bias": "ddt_bias", "init_state": "d_init"}
+    eps = 1e-6
+    for key, gname in names.items():
+        base = case[key]
+        fd = np.zeros_like(base)
+        for idx in np.ndindex(base.shape):
+            c = dict(case)
+            plus, minus = base.copy(), base.copy()
+            plus[idx] += eps
+            minus[idx] -= eps
+            c[key] = plus
+            jp = _bwd_loss(orc, c, dy, dfin)
+            c[key] = minus
+            jm = _bwd_loss(orc, c, dy, dfin)
+            fd[idx] = (jp - jm) / (2 * eps)
+        _close(gr[gname], fd, 1e-6, f"{gname} vs finite differences")
+
+
+def _quadratic_torch(x, dt, A, B, C, D, bias, h0):
+    """y and the final state in the masked-attention form (torch, fp64), for
+    autograd: y_t = sum_{s<=t} e^{S_t - S_s} (C_t.B_s) dt_s x_s + e^{S_t} h0 C_t
+    + D x_t and final = sum_s e^{S_L - S_s} dt_s x_s B_s^T + e^{S_L} h0, with
+    S_t = sum_{k<=t} dt_k A the cumulative log decay."""
+    import torch
+    b, L, H, P = x.shape
+    G = B.shape[2]
+    hpg = H // G
+    Bh = B.repeat_interleave(hpg, dim=2)                     # [b, L, H, N]
+    Ch = C.repeat_interleave(hpg, dim=2)
+    d = torch.nn.functional.softplus(dt + bias)               # [b, L, H]
+    S = torch.cumsum(d * A, dim=1)                            # [b, L, H]
+    seg = S.unsqueeze(2) - S.unsqueeze(1)                     # [b, t, s, H]
+    causal = torch.tril(torch.ones(L, L, dtype=torch.bool)).view(1, L, L, 1)
+    decay = torch.exp(torch.where(causal, seg, torch.full_like(seg, -math.inf)))
+    cb = torch.einsum("btgn,bsgn->btsg", Ch, Bh)              # C_t . B_s per head
+    w = decay * cb * d.unsqueeze(1)                           # [b, t, s, H]
+    y = torch.einsum("btsh,bshp->bthp", w, x)
+    y = y + torch.exp(S).unsqueeze(-1) * torch.einsum("bhpn,bthn->bthp", h0, Ch)
+    y = y + D.view(1, 1, H, 1) * x
+    wl = torch.exp(S[:, -1:, :] - S) * d                      # [b, s, H]
+    fin = torch.einsum("bsh,bshp,bshn->bhpn", wl, x, Bh)
+    fin = fin + torch.exp(S[:, -1, :]).view(b, H, 1, 1) * h0
+    return y, fin
+
+
+def pin_bwd_autograd(orc):
+    """The backward pass against torch's reverse-mode autodiff (fp64) of the
+    masked-attention dual form written above, an implementation that shares
+    nothing with the oracle's recurrence or its adjoint."""
+    import torch
+    case = _rand_case(31, b=2, L=11, H=4, P=3, N=5, G=2)
+    rng = np.random.default_rng(32)
+    dy = rng.standard_normal(case["x"].shape)
+    dfin = rng.standard_normal(case["init_state"].shape)
+    keys = ["x", "dt", "A", "B", "C", "D", "dt_bias", "init_state"]
+    t = {k: torch.tensor(case[k], dtype=torch.float64, requires_grad=True) for k in keys}
+    y, fin = _quadratic_torch(t["x"], t["dt"], t["A"], t["B"], t["C"], t["D"], t["dt_bias"],
+                              t["init_state"])
+    J = (y * torch.tensor(dy)).sum() + (fin * torch.tensor(dfin)).sum()
+    J.backward()
+    gr = orc.ssd_bwd(**case, dy=dy, d_final=dfin)
+    names = {"x": "dx", "dt": "ddt", "A": "dA", "B": "dB", "C": "dC", "D": "dD",
+             "dt_bias": "ddt_bias", "init_state": "d_init"}
+    for k, gname in names.items():
+        _close(gr[gname], t[k].grad.numpy(), 1e-11, f"{gname} vs autograd of the dual form")
+
+
 ALL_PINS = [pin_softplus, pin_quadratic_dual, pin_A_zero_cumsum, pin_chunk_invariance,
             pin_split_resume, pin_decode_equals_forward, pin_special_cases, pin_causality,
-            pin_half_decay_by_hand, pin_gate, pin_conv1d]
+            pin_half_decay_by_hand, pin_gate, pin_conv1d, pin_bwd_finite_differences,
+            pin_bwd_autograd]

@@ -7,14 +7,17 @@ dt_bias; 6 maps heads to groups round-robin instead of contiguously; 7 drops dt
 from the input term; 8 replaces softplus by exp; 9 ignores the initial state;
 10 gates with sigmoid(z) instead of silu(z); 11 reverses the convolution
 kernel; 12 shifts the convolution one token ahead; 13 ignores the carried
-convolution inputs.
+convolution inputs; in the backward pass, 14 drops the decay when the adjoint
+steps back a token; 15 drops the decay's share A*da of ddt; 16 drops the
+softplus derivative of ddt_raw; 17 adds dy_t C_t^T to the adjoint only after
+using it.
 """
 import pytest
 
 import oracle
 import pins
 
-MUTANTS = list(range(1, 14))
+MUTANTS = list(range(1, 18))
 
 
 @pytest.fixture(scope="module")
