@@ -185,6 +185,70 @@ ssd_status ssd_state_passing(const ssd_fwd_args* args, const float* cumA, void* 
 ssd_status ssd_chunk_scan(const ssd_fwd_args* args, const float* dt, const float* cumA,
                           const void* states, void* stream);
 
+/* ---- backward --------------------------------------------------------------- */
+/* The backward pass of ssd_fwd (without the output gate): the gradients of
+ *   J = sum_t dy_t . y_t + d_final : final_state
+ * with respect to every input, i.e. what reverse-mode differentiation of the
+ * recurrence of "MAMBA-2 Reference Implementations Comparison", section 2.2
+ * returns (the page "MAMBA-2 Implementation Gaps" lists dx, ddt, dA, dB, dC
+ * and dD as the gradients a backward pass provides; d_init and ddt_bias are
+ * the other two inputs).  The forward is recomputed inside the call (dt, the
+ * chunk states) from the same inputs.
+ *   sizes, dtype, x, dt, A, B, C, D, dt_bias, init_state: as ssd_fwd_args.
+ *   dy        [batch, seqlen, nheads, headdim] dtype: dJ/dy.
+ *   d_final   [batch, nheads, headdim, dstate] fp32, or NULL (= 0).
+ *   dx        [batch, seqlen, nheads, headdim] dtype.
+ *   ddt       [batch, seqlen, nheads] dtype: the gradient of the RAW dt.
+ *   dB, dC    [batch, seqlen, ngroups, dstate] dtype (summed over the heads of
+ *             a group).
+ *   dA [nheads] fp32; dD, ddt_bias [nheads] fp32 or NULL (not written); all
+ *             three summed over batch and time.
+ *   d_init    [batch, nheads, headdim, dstate] fp32, or NULL (not written).
+ * All gradients are accumulated in fp32 and rounded once to their dtype; sums
+ * over heads and batch rows run in a fixed order, so repeated calls give
+ * bitwise-identical results.
+ * Supported: as ssd_fwd, and chunk a multiple of 64, headdim and dstate at
+ * most 128 with the per-chunk tiles fitting the device's shared memory
+ * (else SSD_ERR_UNSUPPORTED); dy, d_final and d_init 16-byte aligned.
+ * Errors, stream ordering and the workspace rules as for ssd_fwd. */
+typedef struct {
+    int64_t batch, seqlen, nheads, headdim, dstate, ngroups, chunk;
+    int32_t dtype;
+    int32_t flags;          /* SSD_FLAG_* for the forward recompute */
+    const void* x;
+    const void* dt;
+    const float* A;
+    const void* B;
+    const void* C;
+    const float* D;
+    const float* dt_bias;
+    const float* init_state;
+    const void* dy;
+    const float* d_final;
+    void* dx;
+    void* ddt;
+    float* dA;
+    void* dB;
+    void* dC;
+    float* dD;
+    float* ddt_bias;
+    float* d_init;
+    void* workspace;        /* device scratch, >= ssd_bwd_workspace_size() */
+    size_t workspace_bytes;
+} ssd_bwd_args;
+
+/* Bytes of device workspace ssd_bwd needs for these sizes (0 on invalid or
+ * unsupported sizes).  Only sizes, dtype and flags are read. */
+size_t ssd_bwd_workspace_size(const ssd_bwd_args* args);
+
+/* The backward pass (see above).  Stream-ordered. */
+ssd_status ssd_bwd(const ssd_bwd_args* args, void* stream);
+
+/* Synchronises `stream` and returns the device status of the last ssd_bwd
+ * call that used this workspace: SSD_OK, or SSD_ERR_TIMEOUT when a kernel of
+ * its forward recompute gave up on a wait. */
+ssd_status ssd_bwd_check_status(const ssd_bwd_args* args, void* stream);
+
 /* ---- decode ------------------------------------------------------------- */
 /* One token per sequence against a carried state (the SSM half of the
  * Mamba2Cache the page "MAMBA-2 Reference Implementations Comparison",

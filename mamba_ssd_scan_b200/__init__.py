@@ -20,6 +20,7 @@ __all__ = [
     "ssd_state_passing", "ssd_chunk_scan", "ssd_state_update", "ssd_status_string",
     "ssd_version", "lib_path", "load_library", "SSD_FLAG_CUDA_CORES", "SSD_FLAG_WHOLE_GROUPS",
     "ssd_causal_conv1d", "ssd_conv1d_update", "ssd_conv1d_check_status",
+    "ssd_bwd", "ssd_bwd_workspace_size",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -41,6 +42,17 @@ class SsdFwdArgs(ctypes.Structure):
                 ("D", _vp), ("dt_bias", _vp), ("init_state", _vp), ("y", _vp),
                 ("final_state", _vp), ("workspace", _vp), ("workspace_bytes", _sz),
                 ("z", _vp)]
+
+
+class SsdBwdArgs(ctypes.Structure):
+    """Mirror of ssd_bwd_args."""
+    _fields_ = [("batch", _i64), ("seqlen", _i64), ("nheads", _i64), ("headdim", _i64),
+                ("dstate", _i64), ("ngroups", _i64), ("chunk", _i64), ("dtype", _i32),
+                ("flags", _i32), ("x", _vp), ("dt", _vp), ("A", _vp), ("B", _vp), ("C", _vp),
+                ("D", _vp), ("dt_bias", _vp), ("init_state", _vp), ("dy", _vp),
+                ("d_final", _vp), ("dx", _vp), ("ddt", _vp), ("dA", _vp), ("dB", _vp),
+                ("dC", _vp), ("dD", _vp), ("ddt_bias", _vp), ("d_init", _vp),
+                ("workspace", _vp), ("workspace_bytes", _sz)]
 
 
 class SsdStateUpdateArgs(ctypes.Structure):
@@ -110,6 +122,13 @@ def load_library():
     lib.ssd_chunk_scan.argtypes = [F, _vp, _vp, _vp, _vp]
     lib.ssd_state_update.restype = ctypes.c_int
     lib.ssd_state_update.argtypes = [ctypes.POINTER(SsdStateUpdateArgs), _vp]
+    BW = ctypes.POINTER(SsdBwdArgs)
+    lib.ssd_bwd_workspace_size.restype = _sz
+    lib.ssd_bwd_workspace_size.argtypes = [BW]
+    lib.ssd_bwd.restype = ctypes.c_int
+    lib.ssd_bwd.argtypes = [BW, _vp]
+    lib.ssd_bwd_check_status.restype = ctypes.c_int
+    lib.ssd_bwd_check_status.argtypes = [BW, _vp]
     lib.ssd_causal_conv1d.restype = ctypes.c_int
     lib.ssd_causal_conv1d.argtypes = [ctypes.POINTER(SsdConv1dArgs), _vp]
     lib.ssd_conv1d_update.restype = ctypes.c_int
@@ -237,6 +256,74 @@ def ssd_fwd(x, dt, A, B, C, D=None, dt_bias=None, chunk: int = 256, init_state=N
     if final_state is not None:
         return y, final_state
     return y
+
+
+def _bwd_args(x, dt, A, B, C, D, dt_bias, chunk, init_state, flags):
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    a = SsdBwdArgs()
+    a.batch, a.seqlen, a.nheads, a.headdim, a.dstate, a.ngroups, a.chunk = b, L, H, P, N, G, chunk
+    a.dtype = _dtype_code(x)
+    a.flags = int(flags)
+    for name, t in (("dt", dt), ("B", B), ("C", C)):
+        if t.dtype != x.dtype:
+            raise TypeError(f"{name} must have x's dtype {x.dtype}")
+    for name, t in (("A", A), ("D", D), ("dt_bias", dt_bias), ("init_state", init_state)):
+        if t is not None and t.dtype != torch.float32:
+            raise TypeError(f"{name} must be float32")
+    a.x, a.dt, a.A, a.B, a.C = _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C)
+    a.D, a.dt_bias, a.init_state = _ptr(D), _ptr(dt_bias), _ptr(init_state)
+    return a
+
+
+def ssd_bwd_workspace_size(batch, seqlen, nheads, headdim, dstate, ngroups, chunk,
+                           dtype=torch.bfloat16, flags: int = 0) -> int:
+    a = SsdBwdArgs()
+    a.batch, a.seqlen, a.nheads, a.headdim, a.dstate, a.ngroups, a.chunk = (
+        batch, seqlen, nheads, headdim, dstate, ngroups, chunk)
+    a.dtype = SSD_BF16 if dtype == torch.bfloat16 else SSD_F32
+    a.flags = flags
+    return int(load_library().ssd_bwd_workspace_size(ctypes.byref(a)))
+
+
+def ssd_bwd(x, dt, A, B, C, dy, D=None, dt_bias=None, chunk: int = 256, init_state=None,
+            d_final=None, *, out=None, workspace=None, flags: int = 0, stream=None) -> dict:
+    """The backward pass of ssd_fwd (no output gate): gradients of
+    sum(dy * y) + sum(d_final * final_state) with respect to every input.
+    dy has x's shape and dtype; d_final [b,H,P,N] float32 or None.  Returns a
+    dict dx, ddt (of the raw dt), dB, dC (input dtype), dA, dD, ddt_bias [H]
+    and d_init [b,H,P,N] (float32); ``out`` may hold preallocated tensors under
+    the same keys."""
+    lib = load_library()
+    b, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    if dy.dtype != x.dtype or tuple(dy.shape) != tuple(x.shape):
+        raise TypeError("dy must have x's shape and dtype")
+    if d_final is not None and d_final.dtype != torch.float32:
+        raise TypeError("d_final must be float32")
+    o = dict(out or {})
+    o.setdefault("dx", torch.empty_like(x))
+    o.setdefault("ddt", torch.empty_like(dt))
+    o.setdefault("dB", torch.empty_like(B))
+    o.setdefault("dC", torch.empty_like(C))
+    o.setdefault("dA", torch.empty(H, dtype=torch.float32, device=x.device))
+    o.setdefault("dD", torch.empty(H, dtype=torch.float32, device=x.device))
+    o.setdefault("ddt_bias", torch.empty(H, dtype=torch.float32, device=x.device))
+    o.setdefault("d_init", torch.empty((b, H, P, N), dtype=torch.float32, device=x.device))
+    a = _bwd_args(x, dt, A, B, C, D, dt_bias, chunk, init_state, flags)
+    a.dy, a.d_final = _ptr(dy), _ptr(d_final)
+    a.dx, a.ddt, a.dA, a.dB, a.dC = (_ptr(o["dx"]), _ptr(o["ddt"]), _ptr(o["dA"]), _ptr(o["dB"]),
+                                     _ptr(o["dC"]))
+    a.dD, a.ddt_bias, a.d_init = _ptr(o["dD"]), _ptr(o["ddt_bias"]), _ptr(o["d_init"])
+    need = int(lib.ssd_bwd_workspace_size(ctypes.byref(a)))
+    if need == 0:
+        raise SsdError(SSD_ERR_UNSUPPORTED, "ssd_bwd (sizes)")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    a.workspace = workspace.data_ptr()
+    a.workspace_bytes = workspace.numel() * workspace.element_size()
+    _check(lib.ssd_bwd(ctypes.byref(a), _stream_ptr(stream)), "ssd_bwd")
+    return o
 
 
 SSD_NO_ALLOC_SCRATCH_BYTES = 16 << 20

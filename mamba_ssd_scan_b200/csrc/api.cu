@@ -151,6 +151,80 @@ cudaError_t run_chunk_scan(const FwdParams& p, int dtype, int flags, cudaStream_
                              : ssd::launch_chunk_scan_ffma<float>(p, s);
 }
 
+// The forward's view of a backward call (the sizes, dtype and inputs).
+ssd_fwd_args fwd_view(const ssd_bwd_args* a) {
+    ssd_fwd_args f;
+    memset(&f, 0, sizeof(f));
+    f.batch = a->batch;
+    f.seqlen = a->seqlen;
+    f.nheads = a->nheads;
+    f.headdim = a->headdim;
+    f.dstate = a->dstate;
+    f.ngroups = a->ngroups;
+    f.chunk = a->chunk;
+    f.dtype = a->dtype;
+    f.flags = a->flags;
+    f.x = a->x;
+    f.dt = a->dt;
+    f.A = a->A;
+    f.B = a->B;
+    f.C = a->C;
+    f.D = a->D;
+    f.dt_bias = a->dt_bias;
+    f.init_state = a->init_state;
+    return f;
+}
+
+struct BwdWs {
+    size_t status, dt, cumA, states, dstates, xdxs, dyx, mterm, qterm, colw, roww, k4, partial, dBh,
+        dCh, total;
+};
+
+BwdWs bwd_layout(const ssd_bwd_args& a) {
+    const int64_t nc = (a.seqlen + a.chunk - 1) / a.chunk;
+    const size_t vec = (size_t)a.batch * a.nheads * nc * a.chunk * sizeof(float);
+    const size_t elt = a.dtype == SSD_BF16 ? 2 : 4;
+    const size_t pn = (size_t)a.headdim * a.dstate;
+    const size_t tok = (size_t)a.batch * a.nheads * a.seqlen * sizeof(float);
+    const size_t per_head = a.ngroups < a.nheads
+                                ? (size_t)a.batch * a.seqlen * a.nheads * a.dstate * sizeof(float)
+                                : 0;
+    BwdWs w;
+    w.status = 0;
+    w.dt = w.status + kAlign;
+    w.cumA = w.dt + round_up(vec);
+    w.states = w.cumA + round_up(vec);
+    w.dstates = w.states + round_up((size_t)a.batch * nc * a.nheads * pn * elt);
+    w.xdxs = w.dstates + round_up((size_t)a.batch * nc * a.nheads * pn * sizeof(float));
+    w.dyx = w.xdxs + round_up(tok);
+    w.mterm = w.dyx + round_up(tok);
+    w.qterm = w.mterm + round_up(tok);
+    w.colw = w.qterm + round_up(tok);
+    w.roww = w.colw + round_up(tok);
+    w.k4 = w.roww + round_up(tok * (size_t)(a.chunk / 64));
+    w.partial = w.k4 + round_up((size_t)a.batch * a.nheads * nc * sizeof(float));
+    w.dBh = w.partial + round_up((size_t)a.batch * a.nheads * 3 * sizeof(float));
+    w.dCh = w.dBh + round_up(per_head);
+    w.total = w.dCh + round_up(per_head);
+    return w;
+}
+
+// Largest opt-in shared memory per CTA on sm_100 (227 KB).
+constexpr size_t kMaxSmemOptin = 232448;
+
+ssd_status check_bwd_sizes(const ssd_bwd_args* a) {
+    if (!a) return SSD_ERR_INVALID_ARG;
+    const ssd_fwd_args f = fwd_view(a);
+    const ssd_status st = check_fwd_sizes(&f);
+    if (st != SSD_OK) return st;
+    const int64_t nc = (a->seqlen + a->chunk - 1) / a->chunk;
+    if (a->chunk % 64 != 0 || a->headdim > 128 || a->dstate > 128 || nc > 65535)
+        return SSD_ERR_UNSUPPORTED;
+    if (ssd::bwd_smem_bytes(a->headdim, a->dstate, a->chunk) > kMaxSmemOptin)
+        return SSD_ERR_UNSUPPORTED;
+    return SSD_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -207,6 +281,91 @@ ssd_status ssd_fwd_check_status(const ssd_fwd_args* a, void* stream) {
     ssd_status st = check_fwd_sizes(a);
     if (st != SSD_OK) return st;
     const WsLayout w = ws_layout(*a);
+    if (!a->workspace || a->workspace_bytes < w.total || !check_ptr(a->workspace, false, true))
+        return SSD_ERR_INVALID_ARG;
+    int v = 0;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(&v, static_cast<char*>(a->workspace) + w.status, sizeof(int),
+                        cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return SSD_ERR_CUDA;
+    return v == 0 ? SSD_OK : static_cast<ssd_status>(v);
+}
+
+size_t ssd_bwd_workspace_size(const ssd_bwd_args* args) {
+    if (check_bwd_sizes(args) != SSD_OK) return 0;
+    return bwd_layout(*args).total;
+}
+
+ssd_status ssd_bwd(const ssd_bwd_args* a, void* stream) {
+    ssd_status st = check_bwd_sizes(a);
+    if (st != SSD_OK) return st;
+    const ssd_fwd_args f = fwd_view(a);
+    if ((st = check_fwd_inputs(&f)) != SSD_OK) return st;
+    if (!check_ptr(a->dy, false, true) || !check_ptr(a->d_final, true, true) ||
+        !check_ptr(a->dx, false, false) || !check_ptr(a->ddt, false, false) ||
+        !check_ptr(a->dA, false, false) || !check_ptr(a->dB, false, false) ||
+        !check_ptr(a->dC, false, false) || !check_ptr(a->dD, true, false) ||
+        !check_ptr(a->ddt_bias, true, false) || !check_ptr(a->d_init, true, true))
+        return SSD_ERR_INVALID_ARG;
+    const BwdWs w = bwd_layout(*a);
+    if (!a->workspace || a->workspace_bytes < w.total || !check_ptr(a->workspace, false, true))
+        return SSD_ERR_INVALID_ARG;
+    char* ws = static_cast<char*>(a->workspace);
+    FwdParams p = make_params(&f);
+    p.dt = reinterpret_cast<float*>(ws + w.dt);
+    p.cumA = reinterpret_cast<float*>(ws + w.cumA);
+    p.states = ws + w.states;
+    p.status = reinterpret_cast<int*>(ws + w.status);
+    p.final_state = nullptr;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // the forward recompute: dt, cumA and the states entering each chunk
+    cudaError_t e = cudaSuccess;
+    const bool fused = use_tc(a->dtype, a->flags) && ssd::chunk_state_tc_supported(p);
+    if (!fused) {
+        e = run_cumsum(p, a->dtype, s);
+        p.pdl = 1;
+    } else {
+        p.fuse_cumsum = 1;
+    }
+    if (e == cudaSuccess) e = run_chunk_state(p, a->dtype, a->flags, s);
+    p.pdl = 1;
+    p.fuse_cumsum = 0;
+    if (e == cudaSuccess) e = run_state_passing(p, a->dtype, s);
+    if (e != cudaSuccess) return to_status(e);
+    ssd::BwdParams bp;
+    bp.f = p;
+    bp.f.pdl = 0;
+    bp.dy = a->dy;
+    bp.d_final = a->d_final;
+    bp.dx = a->dx;
+    bp.ddt = a->ddt;
+    bp.dA = a->dA;
+    bp.dB = a->dB;
+    bp.dC = a->dC;
+    bp.dD = a->dD;
+    bp.ddt_bias = a->ddt_bias;
+    bp.d_init = a->d_init;
+    bp.dstates = reinterpret_cast<float*>(ws + w.dstates);
+    const bool per_head = a->ngroups < a->nheads;
+    bp.dB_h = per_head ? reinterpret_cast<float*>(ws + w.dBh) : nullptr;
+    bp.dC_h = per_head ? reinterpret_cast<float*>(ws + w.dCh) : nullptr;
+    bp.xdxs = reinterpret_cast<float*>(ws + w.xdxs);
+    bp.dyx = reinterpret_cast<float*>(ws + w.dyx);
+    bp.mterm = reinterpret_cast<float*>(ws + w.mterm);
+    bp.qterm = reinterpret_cast<float*>(ws + w.qterm);
+    bp.colw = reinterpret_cast<float*>(ws + w.colw);
+    bp.roww = reinterpret_cast<float*>(ws + w.roww);
+    bp.k4 = reinterpret_cast<float*>(ws + w.k4);
+    bp.partial = reinterpret_cast<float*>(ws + w.partial);
+    return to_status(a->dtype == SSD_BF16 ? ssd::launch_ssd_bwd<__nv_bfloat16>(bp, s)
+                                          : ssd::launch_ssd_bwd<float>(bp, s));
+}
+
+ssd_status ssd_bwd_check_status(const ssd_bwd_args* a, void* stream) {
+    ssd_status st = check_bwd_sizes(a);
+    if (st != SSD_OK) return st;
+    const BwdWs w = bwd_layout(*a);
     if (!a->workspace || a->workspace_bytes < w.total || !check_ptr(a->workspace, false, true))
         return SSD_ERR_INVALID_ARG;
     int v = 0;

@@ -38,6 +38,35 @@ struct FwdParams {
     int* status;    // device status word (SSD_ERR_TIMEOUT on a timed-out wait); may be null
 };
 
+// One backward call: the forward's sizes and inputs (f, whose dt / cumA /
+// states / final_state point into the backward's workspace) plus the
+// incoming gradients, the outputs and the backward's own intermediates.
+struct BwdParams {
+    FwdParams f;
+    const void* dy;          // [b, L, H, P]
+    const float* d_final;    // [b, H, P, N] or null
+    void* dx;                // [b, L, H, P]
+    void* ddt;               // [b, L, H] (gradient of the raw dt)
+    float* dA;               // [H]
+    void* dB;                // [b, L, G, N]
+    void* dC;                // [b, L, G, N]
+    float* dD;               // [H] or null
+    float* ddt_bias;         // [H] or null
+    float* d_init;           // [b, H, P, N] or null
+    // workspace
+    float* dstates;          // [b, nc, H, P, N]: local adjoint, then dJ/d(state leaving chunk c)
+    float* dB_h;             // [b, L, H, N] per-head dB (when G < H), else null
+    float* dC_h;             // [b, L, H, N] per-head dC (when G < H), else null
+    float* xdxs;             // [b, H, L]: x_t . dxs_t
+    float* dyx;              // [b, H, L]: dy_t . x_t
+    float* mterm;            // [b, H, L]: dt_t x_t . (the dH part of dxs_t)
+    float* qterm;            // [b, H, L]: e^{cumA_t} dy_t . (H_c C_t)
+    float* colw;             // [b, H, L]: sum over later tokens s of the chunk of W[s, t]
+    float* roww;             // [b, H, Q/64, L]: per 64-token source block, sum over earlier r of W[t, r]
+    float* k4;               // [b, H, nc]: e^{cumA_c[last]} <dH_c, H_c>
+    float* partial;          // [b, H, 3]: per-row sums of dt*da, dy.x, ddt_raw
+};
+
 struct DecodeParams {
     int64_t batch, nheads, headdim, dstate, ngroups, heads_per_group;
     float* state;
@@ -164,6 +193,10 @@ template <typename T> cudaError_t launch_state_passing(const FwdParams& p, cudaS
 template <typename T> cudaError_t launch_chunk_scan_ffma(const FwdParams& p, cudaStream_t s);
 template <typename T> cudaError_t launch_state_update(const DecodeParams& p, cudaStream_t s);
 template <typename T> cudaError_t launch_conv1d(const ConvParams& p, bool update, cudaStream_t s);
+// The backward pass after the forward recompute (bwd.cu).
+template <typename T> cudaError_t launch_ssd_bwd(const BwdParams& p, cudaStream_t s);
+// Shared memory (bytes) the backward's per-chunk kernels need for a shape.
+size_t bwd_smem_bytes(int64_t headdim, int64_t dstate, int64_t chunk);
 // Copies the forward kernel's device status word to *v and clears it (synchronises s).
 cudaError_t conv1d_take_status(int* v, cudaStream_t s);
 

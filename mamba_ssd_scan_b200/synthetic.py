@@ -166,6 +166,15 @@ def make_gate(shape, dtype, seed: int) -> torch.Tensor:
     return torch.randn(tuple(shape), generator=gen, dtype=torch.float32).to(dtype)
 
 
+def make_bwd_grads(x_shape, state_shape, dtype, seed: int) -> dict:
+    """Incoming gradients of a backward call: dy ~ N(0,1) shaped like x (in
+    dtype) and d_final ~ N(0,1) shaped like the state (fp32)."""
+    gen = torch.Generator().manual_seed(seed + 7907)
+    dy = torch.randn(x_shape, generator=gen).to(dtype)
+    d_final = torch.randn(state_shape, generator=gen)
+    return dict(dy=dy, d_final=d_final)
+
+
 def make_conv_inputs(batch, seqlen, channels, width, dtype, seed: int,
                      init_state: bool = True) -> dict:
     """Inputs of the causal depthwise convolution: x ~ N(0, 1) [b, L, C] in

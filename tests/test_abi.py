@@ -127,3 +127,22 @@ def test_conv1d_rejects_bad_args(lib):
     assert lib.ssd_conv1d_update(ctypes.byref(u), None) == 2        # fp32 channels % 4
     u.width = 9
     assert lib.ssd_conv1d_update(ctypes.byref(u), None) == 2        # width beyond 8
+
+
+def test_bwd_rejects_bad_args(lib):
+    import mamba_ssd_scan_b200 as ssd
+    a = ssd.SsdBwdArgs()
+    a.batch, a.seqlen, a.nheads, a.headdim, a.dstate, a.ngroups, a.chunk = 1, 256, 4, 64, 64, 1, 256
+    a.dtype = 1
+    assert lib.ssd_bwd(None, None) == 1
+    assert lib.ssd_bwd_workspace_size(ctypes.byref(a)) > 0
+    assert lib.ssd_bwd(ctypes.byref(a), None) == 1               # null pointers
+    a.chunk = 100
+    assert lib.ssd_bwd_workspace_size(ctypes.byref(a)) == 0
+    assert lib.ssd_bwd(ctypes.byref(a), None) == 2               # chunk not a multiple of 64
+    a.chunk, a.headdim = 256, 256
+    assert lib.ssd_bwd(ctypes.byref(a), None) == 2               # headdim beyond 128
+    a.headdim, a.dstate = 128, 128
+    assert lib.ssd_bwd(ctypes.byref(a), None) == 2               # tiles beyond shared memory
+    a.dstate, a.ngroups = 64, 3
+    assert lib.ssd_bwd(ctypes.byref(a), None) == 1               # heads not divisible by groups
