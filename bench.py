@@ -55,6 +55,8 @@ def parse_args():
     ap.add_argument("--flush-mb", type=int, default=256)
     ap.add_argument("--conv-only", action="store_true",
                     help="time only the convolution workloads (one JSON line of them)")
+    ap.add_argument("--bwd-only", action="store_true",
+                    help="time only the backward-pass workloads (one JSON line of them)")
     return ap.parse_args()
 
 
@@ -238,8 +240,10 @@ def main_ours(args):
         flush_buf.fill_(1)
         torch.sum(flush_f, dim=0, out=flush_acc)
 
-    if args.conv_only:
-        res = conv_workloads(ssd, synthetic, dev, flush, peaks, rank, world, ranks_max)
+    if args.conv_only or args.bwd_only:
+        res = (conv_workloads(ssd, synthetic, dev, flush, peaks, rank, world, ranks_max)
+               if args.conv_only else bwd_workloads(ssd, synthetic, dev, flush, rank, world,
+                                                   ranks_max))
         if rank == 0:
             print(json.dumps({"workloads": res, "peaks_source": peaks["source"]}), flush=True)
         return
@@ -650,6 +654,74 @@ def other_workloads(ssd, synthetic, dev, flush, peaks, rank, world, barrier, ran
     del g, state, steps_in
     torch.cuda.empty_cache()
     out.update(conv_workloads(ssd, synthetic, dev, flush, peaks, rank, world, ranks_max))
+    out.update(bwd_workloads(ssd, synthetic, dev, flush, rank, world, ranks_max))
+    return out
+
+
+# fp32 FMA peak of the CUDA cores: 148 SMs x 128 FMA lanes x 2 FLOP x 1.965 GHz
+FP32_FMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def bwd_flops(cfg):
+    """Algorithmic FLOP of one ssd_bwd call: per chunk and head the two causal
+    score matrices (C.B over N, dy.x over P), the three products with them
+    (dxs over P, dB and dC over N) and the four state products (dS, and the
+    dH / H_c terms of dxs, dB, dC), 2 FLOP per multiply-add."""
+    nc = (cfg.seqlen + cfg.chunk - 1) // cfg.chunk
+    Q, P, N = cfg.chunk, cfg.headdim, cfg.dstate
+    tri = Q * (Q + 1) // 2
+    per = tri * (N + P) + tri * (P + 2 * N) + 4 * Q * P * N
+    return 2.0 * per * nc * cfg.nheads * cfg.batch
+
+
+def bwd_workloads(ssd, synthetic, dev, flush, rank, world, ranks_max, steps=5):
+    """The backward pass (forward recompute included) on two forward
+    workloads' shapes, with an initial state and d_final, L2 flushed before
+    each call."""
+    import torch
+    out = {}
+    stream = torch.cuda.current_stream()
+    for name in ("fwd_bf16_b4_L1024", "fwd_bf16_b8_L4096_init"):
+        cfg = synthetic.FWD_CONFIGS[name]
+        seed = rank_seed(1234 + synthetic.SEED_OFFSET[name], rank)
+        inp = synthetic.make_fwd_inputs(cfg.batch, cfg.seqlen, cfg.nheads, cfg.headdim,
+                                        cfg.dstate, cfg.ngroups, cfg.dtype, seed, init_state=True)
+        gr = synthetic.make_bwd_grads((cfg.batch, cfg.seqlen, cfg.nheads, cfg.headdim),
+                                      (cfg.batch, cfg.nheads, cfg.headdim, cfg.dstate),
+                                      cfg.dtype, seed)
+        d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
+        dy, dfin = gr["dy"].to(dev), gr["d_final"].to(dev)
+        ws = torch.empty(ssd.ssd_bwd_workspace_size(cfg.batch, cfg.seqlen, cfg.nheads,
+                                                    cfg.headdim, cfg.dstate, cfg.ngroups,
+                                                    cfg.chunk, cfg.dtype),
+                         dtype=torch.uint8, device=dev)
+        res = {}
+
+        def step():
+            ssd.ssd_bwd(d["x"], d["dt"], d["A"], d["B"], d["C"], dy, D=d["D"],
+                        dt_bias=d["dt_bias"], chunk=cfg.chunk, init_state=d["init_state"],
+                        d_final=dfin, out=res, workspace=ws)
+
+        for _ in range(3):
+            step()
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)]
+        gpu_head_start(2.0)
+        for a, b_ in evs:
+            flush()
+            a.record(stream)
+            step()
+            b_.record(stream)
+        torch.cuda.synchronize()
+        ms = ranks_max(sum(a.elapsed_time(b_) for a, b_ in evs) / steps)
+        fl = bwd_flops(cfg)
+        out["bwd_" + name] = {"tokens_per_s": job_throughput(cfg.tokens, world, ms), "ms": ms,
+                              "tflops": fl / (ms * 1e-3) / 1e12, "flop": fl,
+                              "fp32_fma_frac": fl / (ms * 1e-3) / 1e12 / FP32_FMA_TFLOPS,
+                              "bound": "alu", "l2": "flushed"}
+        del d, dy, dfin, ws, res
+        torch.cuda.empty_cache()
     return out
 
 

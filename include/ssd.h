@@ -190,9 +190,10 @@ ssd_status ssd_chunk_scan(const ssd_fwd_args* args, const float* dt, const float
  *   J = sum_t dy_t . y_t + d_final : final_state
  * with respect to every input, i.e. what reverse-mode differentiation of the
  * recurrence of "MAMBA-2 Reference Implementations Comparison", section 2.2
- * returns (the page "MAMBA-2 Implementation Gaps" lists dx, ddt, dA, dB, dC
- * and dD as the gradients a backward pass provides; d_init and ddt_bias are
- * the other two inputs).  The forward is recomputed inside the call (dt, the
+ * returns (the page "Agent 230: Comprehensive MAMBA-2 Implementation
+ * Comparison", section 6, Gradient Computation, takes the gradients of A, B,
+ * C and delta (dt); x, D, dt_bias and the initial state are the other
+ * inputs).  The forward is recomputed inside the call (dt, the
  * chunk states) from the same inputs.
  *   sizes, dtype, x, dt, A, B, C, D, dt_bias, init_state: as ssd_fwd_args.
  *   dy        [batch, seqlen, nheads, headdim] dtype: dJ/dy.

@@ -1,9 +1,10 @@
 // bwd.cu -- the backward pass of the chunked SSD scan: gradients of
 //   J = sum_t dy_t . y_t + d_final : h_L
 // with respect to x, the raw dt, A, B, C, D, dt_bias and the initial state.
-// The pages list the gradients a backward pass returns ("MAMBA-2
-// Implementation Gaps"); their form follows from the chain rule on the
-// chunked forward ("MAMBA-2 Reference Implementations Comparison", section
+// The page "Agent 230: Comprehensive MAMBA-2 Implementation Comparison",
+// section 6 (Gradient Computation), takes the gradients of A, B, C and delta
+// (dt) after its backward pass; it gives no formulas.  Theirs and the other
+// inputs' follow from the chain rule on the chunked forward ("MAMBA-2 Reference Implementations Comparison", section
 // 2.2; "MAMBA-2 Implementation Gaps", Gap 1).  Per (batch, head), with cumA
 // the in-chunk cumulative log decay, H_c the state entering chunk c and dH_c
 // the gradient with respect to the state leaving chunk c:

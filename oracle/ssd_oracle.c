@@ -202,9 +202,11 @@ void oracle_ssd_fwd(int64_t batch, int64_t L, int64_t H, int64_t P,
  *   ddt_raw_t = ddt_t sigmoid(dt_raw_t + dt_bias_h),   ddt_bias_h += ddt_raw_t
  *   dD_h     += dy_t . x_t,   d_init = dJ/dh_0 = e^{a_1} g_1
  * The recurrence is the one of "MAMBA-2 Reference Implementations
- * Comparison", section 2.2; the pages list the gradients a backward pass must
- * return ("MAMBA-2 Implementation Gaps") but not their formulas, which follow
- * from the chain rule alone (softplus'(u) = sigmoid(u)).
+ * Comparison", section 2.2; the page "Agent 230: Comprehensive MAMBA-2
+ * Implementation Comparison", section 6 (Gradient Computation), takes the
+ * gradients of A, B, C and delta (dt) after its backward pass but gives no
+ * formulas; all of them follow from the chain rule alone
+ * (softplus'(u) = sigmoid(u)).
  *
  * dy [b,L,H,P]; d_final [b,H,P,N] or NULL (zero).  Outputs shaped like the
  * inputs: dx, ddt_raw, dB, dC (dB, dC summed over the heads of a group),
