@@ -66,6 +66,10 @@ class Oracle:
         lib.oracle_state_update.argtypes = [_i64] * 5 + [_dp] * 9
         lib.oracle_ssd_bwd.restype = None
         lib.oracle_ssd_bwd.argtypes = [_i64] * 6 + [_dp] * 18
+        lib.oracle_selective_scan.restype = None
+        lib.oracle_selective_scan.argtypes = [_i64] * 4 + [_dp] * 10
+        lib.oracle_selective_state_update.restype = None
+        lib.oracle_selective_state_update.argtypes = [_i64] * 3 + [_dp] * 9
         lib.oracle_gate.restype = None
         lib.oracle_gate.argtypes = [_dp, _dp, _i64]
         lib.oracle_causal_conv1d.restype = None
@@ -125,6 +129,34 @@ class Oracle:
         if z is not None:
             y = self.gate(y, z)
         return y, fin
+
+    def selective_scan(self, x, dt, A, B, C, D=None, dt_bias=None, init_state=None):
+        """Diagonal-A selective scan.  x, dt [b,L,Dc]; A [Dc,N]; B, C [b,L,N];
+        D, dt_bias [Dc]; init_state [b,Dc,N].  Returns (y, final_state)."""
+        x, dt, A, B, C = (self._f64(t) for t in (x, dt, A, B, C))
+        D, dt_bias, init = self._f64(D), self._f64(dt_bias), self._f64(init_state)
+        b, L, Dc = x.shape
+        N = A.shape[1]
+        y = np.zeros((b, L, Dc))
+        fin = np.zeros((b, Dc, N))
+        p = self._ptr
+        self.lib.oracle_selective_scan(b, L, Dc, N, p(x), p(dt), p(A), p(B), p(C), p(D),
+                                       p(dt_bias), p(init), p(y), p(fin))
+        return y, fin
+
+    def selective_state_update(self, state, x, dt, A, B, C, D=None, dt_bias=None):
+        """One decode step: returns (new state, y); state [b,Dc,N], x/dt [b,Dc],
+        B/C [b,N]."""
+        st = self._f64(state).copy()
+        x, dt, A, B, C = (self._f64(t) for t in (x, dt, A, B, C))
+        D, dt_bias = self._f64(D), self._f64(dt_bias)
+        b, Dc = x.shape
+        N = A.shape[1]
+        y = np.zeros((b, Dc))
+        p = self._ptr
+        self.lib.oracle_selective_state_update(b, Dc, N, p(st), p(x), p(dt), p(A), p(B), p(C),
+                                               p(D), p(dt_bias), p(y))
+        return st, y
 
     def ssd_bwd(self, x, dt, A, B, C, D=None, dt_bias=None, init_state=None, dy=None,
                 d_final=None):

@@ -42,6 +42,9 @@
  *                        Mamba2Cache this state lives in)
  *   oracle_ssd_bwd       the gradients of oracle_ssd_fwd (reverse-mode
  *                        differentiation of the recurrence, token by token)
+ *   oracle_selective_scan, oracle_selective_state_update
+ *                        the diagonal-A (per channel and state) selective
+ *                        scan and its decode step
  *
  * Pins (tests/, CPU only): the masked-attention (quadratic) dual form by brute
  * force, the A = 0 cumulative-sum closed form, chunk-size invariance, split /
@@ -355,6 +358,77 @@ void oracle_ssd_bwd(int64_t batch, int64_t L, int64_t H, int64_t P,
     free(sums);
     free(dCh);
     free(dBh);
+}
+
+/*
+ * The selective scan with a diagonal A per channel (the Mamba-1 form the pages
+ * set beside SSD: "MAMBA-2 Reference Implementations Comparison", section 2.3,
+ * Mamba-1 vs SSD; A_log of shape [d_inner, d_state] in the block's parameter
+ * list of section 1.3, and dt per channel from dt_proj with B * dt as the
+ * input term in "MAMBA-2 Implementation Gaps", Gap 3).  Per channel d and state n:
+ *   dt_t[d]   = softplus(dt_raw_t[d] + dt_bias[d])
+ *   h_t[d,n]  = exp(dt_t[d] A[d,n]) h_{t-1}[d,n] + dt_t[d] B_t[n] x_t[d]
+ *   y_t[d]    = sum_n C_t[n] h_t[d,n] + D[d] x_t[d]
+ * Layouts: x, dt_raw, y [b, L, Dc]; A [Dc, N]; B, C [b, L, N]; D, dt_bias
+ * [Dc]; state [b, Dc, N].  init, D, dt_bias, final_state may be NULL.
+ */
+void oracle_selective_scan(int64_t batch, int64_t L, int64_t Dc, int64_t N,
+                           const double* x, const double* dt_raw, const double* A,
+                           const double* B, const double* C, const double* D,
+                           const double* dt_bias, const double* init,
+                           double* y, double* final_state) {
+    int64_t bd;
+#pragma omp parallel for schedule(dynamic, 16)
+    for (bd = 0; bd < batch * Dc; ++bd) {
+        const int64_t b = bd / Dc, d = bd % Dc;
+        double* h = (double*)malloc(sizeof(double) * (size_t)N);
+        for (int64_t n = 0; n < N; ++n) h[n] = init ? init[bd * N + n] : 0.0;
+        for (int64_t t = 0; t < L; ++t) {
+            const int64_t it = (b * L + t) * Dc + d;
+            const double dt = oracle_softplus(dt_raw[it] + (dt_bias ? dt_bias[d] : 0.0));
+#if ORACLE_MUTANT == 19
+            const double xt = x[(b * L + t) * Dc];
+#else
+            const double xt = x[it];
+#endif
+            const double* Bt = B + (b * L + t) * N;
+            const double* Ct = C + (b * L + t) * N;
+            double acc = 0.0;
+            for (int64_t n = 0; n < N; ++n) {
+#if ORACLE_MUTANT == 18
+                const double a = exp(dt * A[d * N]);
+#else
+                const double a = exp(dt * A[d * N + n]);
+#endif
+                h[n] = a * h[n] + dt * Bt[n] * xt;
+                acc += Ct[n] * h[n];
+            }
+            y[it] = acc + (D ? D[d] : 0.0) * x[it];
+        }
+        if (final_state) memcpy(final_state + bd * N, h, sizeof(double) * (size_t)N);
+        free(h);
+    }
+}
+
+/* One decode step of oracle_selective_scan on a carried state [b, Dc, N]:
+ * x, dt_raw, y [b, Dc]; B, C [b, N]. */
+void oracle_selective_state_update(int64_t batch, int64_t Dc, int64_t N, double* state,
+                                   const double* x, const double* dt_raw, const double* A,
+                                   const double* B, const double* C, const double* D,
+                                   const double* dt_bias, double* y) {
+    int64_t bd;
+#pragma omp parallel for schedule(static)
+    for (bd = 0; bd < batch * Dc; ++bd) {
+        const int64_t b = bd / Dc, d = bd % Dc;
+        const double dt = oracle_softplus(dt_raw[bd] + (dt_bias ? dt_bias[d] : 0.0));
+        double acc = 0.0;
+        for (int64_t n = 0; n < N; ++n) {
+            double* h = state + bd * N + n;
+            *h = exp(dt * A[d * N + n]) * *h + dt * B[b * N + n] * x[bd];
+            acc += C[b * N + n] * *h;
+        }
+        y[bd] = acc + (D ? D[d] : 0.0) * x[bd];
+    }
 }
 
 /*

@@ -380,7 +380,83 @@ def pin_bwd_autograd(orc):
         _close(gr[gname], t[k].grad.numpy(), 1e-11, f"{gname} vs autograd of the dual form")
 
 
+def _sel_case(seed, b=2, L=9, Dc=6, N=4):
+    rng = np.random.default_rng(seed)
+    return dict(x=rng.standard_normal((b, L, Dc)), dt=rng.standard_normal((b, L, Dc)),
+                A=-rng.uniform(0.2, 2.0, (Dc, N)), B=rng.standard_normal((b, L, N)),
+                C=rng.standard_normal((b, L, N)), D=rng.standard_normal(Dc),
+                dt_bias=rng.uniform(-1.0, 0.5, Dc),
+                init_state=0.5 * rng.standard_normal((b, Dc, N)))
+
+
+def pin_selective_scan(orc):
+    """The diagonal-A selective scan against: the unrolled double sum written
+    out by brute force, y_t[d] = sum_n C_t[n] (sum_{s<=t} e^{A[d,n] sum_{k=s+1..t}
+    dt_k[d]} dt_s[d] B_s[n] x_s[d] + e^{A[d,n] sum_{k<=t} dt_k[d]} h0[d,n]) +
+    D[d] x_t[d]; the SSD scan (a pinned, separate function) when A is the same
+    for every state of a head and the head's channels share dt ("MAMBA-2
+    Reference Implementations Comparison", section 2.2: SSD is this scan with
+    A a scalar times the identity); the states' independence (A of a state
+    that receives no input and starts at zero leaves y bitwise unchanged);
+    split / resume and decode == forward."""
+    c = _sel_case(41)
+    y, fin = orc.selective_scan(**c)
+    b, L, Dc = c["x"].shape
+    N = c["A"].shape[1]
+    d_ = _softplus_np(c["dt"] + c["dt_bias"])
+    ref = np.zeros_like(y)
+    for bi in range(b):
+        for d in range(Dc):
+            for t in range(L):
+                acc = 0.0
+                for n in range(N):
+                    for s in range(t + 1):
+                        acc += (c["C"][bi, t, n] * math.exp(c["A"][d, n] * d_[bi, s + 1:t + 1, d].sum())
+                                * d_[bi, s, d] * c["B"][bi, s, n] * c["x"][bi, s, d])
+                    acc += (c["C"][bi, t, n] * math.exp(c["A"][d, n] * d_[bi, :t + 1, d].sum())
+                            * c["init_state"][bi, d, n])
+                ref[bi, t, d] = acc + c["D"][d] * c["x"][bi, t, d]
+    _close(y, ref, 1e-12, "selective scan vs unrolled sum")
+    # SSD as the special case: Dc = H * P channels, A and dt shared per head
+    H, P = 3, 2
+    s = _rand_case(43, b=2, L=8, H=H, P=P, N=N, G=1)
+    sel = dict(x=s["x"].reshape(2, 8, H * P), dt=np.repeat(s["dt"], P, axis=2),
+               A=np.repeat(s["A"], P)[:, None] * np.ones((1, N)), B=s["B"][:, :, 0],
+               C=s["C"][:, :, 0], D=np.repeat(s["D"], P), dt_bias=np.repeat(s["dt_bias"], P),
+               init_state=s["init_state"].reshape(2, H * P, N))
+    ys, fs = orc.selective_scan(**sel)
+    yd, fd = orc.ssd_fwd(**s)
+    _close(ys, yd.reshape(2, 8, H * P), 1e-12, "selective scan == SSD for scalar A per head")
+    _close(fs, fd.reshape(2, H * P, N), 1e-12, "final state == SSD's")
+    # a state with no input and no initial value does not depend on its A
+    c2 = dict(c)
+    c2["B"] = c["B"].copy()
+    c2["B"][:, :, 1] = 0.0
+    c2["init_state"] = c["init_state"].copy()
+    c2["init_state"][:, :, 1] = 0.0
+    y1, _ = orc.selective_scan(**c2)
+    c3 = dict(c2)
+    c3["A"] = c2["A"].copy()
+    c3["A"][:, 1] *= 7.0
+    y2, _ = orc.selective_scan(**c3)
+    assert np.array_equal(y1, y2), "an idle state's A changed y"
+    # split / resume, decode == forward
+    L1 = 4
+    ya, fa = orc.selective_scan(**{k: (v[:, :L1] if k in ("x", "dt", "B", "C") else v)
+                                   for k, v in c.items()})
+    yb, fb = orc.selective_scan(**{k: (v[:, L1:] if k in ("x", "dt", "B", "C") else v)
+                                   for k, v in c.items() if k != "init_state"}, init_state=fa)
+    _close(np.concatenate([ya, yb], 1), y, 1e-13, "selective scan split / resume")
+    _close(fb, fin, 1e-13, "selective scan final state after resume")
+    st = c["init_state"].copy()
+    for t in range(L):
+        st, yt = orc.selective_state_update(st, c["x"][:, t], c["dt"][:, t], c["A"], c["B"][:, t],
+                                            c["C"][:, t], c["D"], c["dt_bias"])
+        _close(yt, y[:, t], 1e-13, f"selective decode step {t}")
+    _close(st, fin, 1e-13, "selective decode state == forward final state")
+
+
 ALL_PINS = [pin_softplus, pin_quadratic_dual, pin_A_zero_cumsum, pin_chunk_invariance,
             pin_split_resume, pin_decode_equals_forward, pin_special_cases, pin_causality,
             pin_half_decay_by_hand, pin_gate, pin_conv1d, pin_bwd_finite_differences,
-            pin_bwd_autograd]
+            pin_bwd_autograd, pin_selective_scan]
