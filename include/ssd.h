@@ -250,6 +250,68 @@ ssd_status ssd_bwd(const ssd_bwd_args* args, void* stream);
  * its forward recompute gave up on a wait. */
 ssd_status ssd_bwd_check_status(const ssd_bwd_args* args, void* stream);
 
+/* ---- diagonal-A selective scan (Mamba-1 form) ------------------------------ */
+/* The selective scan with A diagonal per channel and state, the Mamba-1 form
+ * the page "MAMBA-2 Reference Implementations Comparison" sets beside SSD
+ * (section 2.3; A_log [d_inner, d_state] in the block parameter list of
+ * section 1.3; dt per channel and B * dt in "MAMBA-2 Implementation Gaps",
+ * Gap 3):
+ *   dt_t[d]  = softplus(dt_raw_t[d] + dt_bias[d])
+ *   h_t[d,n] = exp(dt_t[d] A[d,n]) h_{t-1}[d,n] + dt_t[d] B_t[n] x_t[d]
+ *   y_t[d]   = sum_n C_t[n] h_t[d,n] + D[d] x_t[d]
+ * Layouts: x, dt (raw), y [batch, seqlen, channels] dtype; A [channels,
+ * dstate] fp32 (the negative values themselves, i.e. -exp(A_log)); B, C
+ * [batch, seqlen, dstate] dtype (shared by all channels); D, dt_bias
+ * [channels] fp32 or NULL; init_state, final_state [batch, channels, dstate]
+ * fp32 or NULL.  `chunk` cuts the sequence for parallelism (the result does
+ * not depend on it beyond rounding).
+ * Supported: dstate a multiple of 4 up to 32; 1 <= chunk, chunk * dstate <=
+ * 4096; batch <= 65535 (else SSD_ERR_UNSUPPORTED); A, init_state,
+ * final_state and the workspace 16-byte aligned.  Errors and stream ordering
+ * as for ssd_fwd. */
+typedef struct {
+    int64_t batch, seqlen, channels, dstate, chunk;
+    int32_t dtype;
+    int32_t flags;          /* reserved, 0 */
+    const void* x;
+    const void* dt;
+    const float* A;
+    const void* B;
+    const void* C;
+    const float* D;
+    const float* dt_bias;
+    const float* init_state;
+    void* y;
+    float* final_state;
+    void* workspace;        /* device scratch, >= ssd_selective_scan_workspace_size() */
+    size_t workspace_bytes;
+} ssd_selective_scan_args;
+
+/* Bytes of workspace for these sizes (0 if invalid or unsupported). */
+size_t ssd_selective_scan_workspace_size(const ssd_selective_scan_args* args);
+
+ssd_status ssd_selective_scan(const ssd_selective_scan_args* args, void* stream);
+
+/* One decode step of the same scan on a carried state [batch, channels,
+ * dstate] fp32 (16-byte aligned), updated in place; x, dt, y [batch,
+ * channels] dtype; B, C [batch, dstate] dtype.  Supported dstate as above. */
+typedef struct {
+    int64_t batch, channels, dstate;
+    int32_t dtype;
+    int32_t flags;          /* reserved, 0 */
+    float* state;
+    const void* x;
+    const void* dt;
+    const float* A;
+    const void* B;
+    const void* C;
+    const float* D;
+    const float* dt_bias;
+    void* y;
+} ssd_selective_state_update_args;
+
+ssd_status ssd_selective_state_update(const ssd_selective_state_update_args* args, void* stream);
+
 /* ---- decode ------------------------------------------------------------- */
 /* One token per sequence against a carried state (the SSM half of the
  * Mamba2Cache the page "MAMBA-2 Reference Implementations Comparison",

@@ -20,7 +20,8 @@ __all__ = [
     "ssd_state_passing", "ssd_chunk_scan", "ssd_state_update", "ssd_status_string",
     "ssd_version", "lib_path", "load_library", "SSD_FLAG_CUDA_CORES", "SSD_FLAG_WHOLE_GROUPS",
     "ssd_causal_conv1d", "ssd_conv1d_update", "ssd_conv1d_check_status",
-    "ssd_bwd", "ssd_bwd_workspace_size",
+    "ssd_bwd", "ssd_bwd_workspace_size", "ssd_selective_scan", "ssd_selective_scan_workspace_size",
+    "ssd_selective_state_update",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -53,6 +54,22 @@ class SsdBwdArgs(ctypes.Structure):
                 ("d_final", _vp), ("dx", _vp), ("ddt", _vp), ("dA", _vp), ("dB", _vp),
                 ("dC", _vp), ("dD", _vp), ("ddt_bias", _vp), ("d_init", _vp),
                 ("workspace", _vp), ("workspace_bytes", _sz)]
+
+
+class SsdSelectiveScanArgs(ctypes.Structure):
+    """Mirror of ssd_selective_scan_args."""
+    _fields_ = [("batch", _i64), ("seqlen", _i64), ("channels", _i64), ("dstate", _i64),
+                ("chunk", _i64), ("dtype", _i32), ("flags", _i32), ("x", _vp), ("dt", _vp),
+                ("A", _vp), ("B", _vp), ("C", _vp), ("D", _vp), ("dt_bias", _vp),
+                ("init_state", _vp), ("y", _vp), ("final_state", _vp), ("workspace", _vp),
+                ("workspace_bytes", _sz)]
+
+
+class SsdSelectiveStateUpdateArgs(ctypes.Structure):
+    """Mirror of ssd_selective_state_update_args."""
+    _fields_ = [("batch", _i64), ("channels", _i64), ("dstate", _i64), ("dtype", _i32),
+                ("flags", _i32), ("state", _vp), ("x", _vp), ("dt", _vp), ("A", _vp),
+                ("B", _vp), ("C", _vp), ("D", _vp), ("dt_bias", _vp), ("y", _vp)]
 
 
 class SsdStateUpdateArgs(ctypes.Structure):
@@ -129,6 +146,13 @@ def load_library():
     lib.ssd_bwd.argtypes = [BW, _vp]
     lib.ssd_bwd_check_status.restype = ctypes.c_int
     lib.ssd_bwd_check_status.argtypes = [BW, _vp]
+    SA = ctypes.POINTER(SsdSelectiveScanArgs)
+    lib.ssd_selective_scan_workspace_size.restype = _sz
+    lib.ssd_selective_scan_workspace_size.argtypes = [SA]
+    lib.ssd_selective_scan.restype = ctypes.c_int
+    lib.ssd_selective_scan.argtypes = [SA, _vp]
+    lib.ssd_selective_state_update.restype = ctypes.c_int
+    lib.ssd_selective_state_update.argtypes = [ctypes.POINTER(SsdSelectiveStateUpdateArgs), _vp]
     lib.ssd_causal_conv1d.restype = ctypes.c_int
     lib.ssd_causal_conv1d.argtypes = [ctypes.POINTER(SsdConv1dArgs), _vp]
     lib.ssd_conv1d_update.restype = ctypes.c_int
@@ -467,6 +491,82 @@ def ssd_causal_conv1d(x, weight, bias=None, init_state=None, *, activation: bool
     _check(lib.ssd_causal_conv1d(ctypes.byref(a), _stream_ptr(stream)), "ssd_causal_conv1d")
     if return_final_state:
         return y, final_state
+    return y
+
+
+def _sel_args(x, dt, A, B, C, D, dt_bias, chunk, init_state, y, final_state):
+    b, L, Dc = x.shape
+    N = A.shape[1]
+    for name, t in (("dt", dt), ("B", B), ("C", C)):
+        if t.dtype != x.dtype:
+            raise TypeError(f"{name} must have x's dtype {x.dtype}")
+    for name, t in (("A", A), ("D", D), ("dt_bias", dt_bias), ("init_state", init_state),
+                    ("final_state", final_state)):
+        if t is not None and t.dtype != torch.float32:
+            raise TypeError(f"{name} must be float32")
+    a = SsdSelectiveScanArgs()
+    a.batch, a.seqlen, a.channels, a.dstate, a.chunk = b, L, Dc, N, chunk
+    a.dtype = _dtype_code(x)
+    a.flags = 0
+    a.x, a.dt, a.A, a.B, a.C = _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C)
+    a.D, a.dt_bias, a.init_state = _ptr(D), _ptr(dt_bias), _ptr(init_state)
+    a.y, a.final_state = _ptr(y), _ptr(final_state)
+    return a
+
+
+def ssd_selective_scan(x, dt, A, B, C, D=None, dt_bias=None, chunk: int = 64, init_state=None,
+                       *, y=None, final_state=None, return_final_state: bool = False,
+                       workspace=None, stream=None):
+    """The diagonal-A (Mamba-1 form) selective scan.  x, dt [b,L,Dc] and B, C
+    [b,L,N] in one dtype; A [Dc,N], D, dt_bias [Dc], init_state [b,Dc,N] fp32.
+    Returns y (and the final fp32 state when asked)."""
+    lib = load_library()
+    b, L, Dc = x.shape
+    N = A.shape[1]
+    y = y if y is not None else torch.empty_like(x)
+    if final_state is None and return_final_state:
+        final_state = torch.empty((b, Dc, N), dtype=torch.float32, device=x.device)
+    a = _sel_args(x, dt, A, B, C, D, dt_bias, chunk, init_state, y, final_state)
+    need = int(lib.ssd_selective_scan_workspace_size(ctypes.byref(a)))
+    if need == 0:
+        raise SsdError(SSD_ERR_UNSUPPORTED, "ssd_selective_scan (sizes)")
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    a.workspace = workspace.data_ptr()
+    a.workspace_bytes = workspace.numel() * workspace.element_size()
+    _check(lib.ssd_selective_scan(ctypes.byref(a), _stream_ptr(stream)), "ssd_selective_scan")
+    if final_state is not None:
+        return y, final_state
+    return y
+
+
+def ssd_selective_scan_workspace_size(batch, seqlen, channels, dstate, chunk,
+                                      dtype=torch.bfloat16) -> int:
+    a = SsdSelectiveScanArgs()
+    a.batch, a.seqlen, a.channels, a.dstate, a.chunk = batch, seqlen, channels, dstate, chunk
+    a.dtype = SSD_BF16 if dtype == torch.bfloat16 else SSD_F32
+    return int(load_library().ssd_selective_scan_workspace_size(ctypes.byref(a)))
+
+
+def ssd_selective_state_update(state, x, dt, A, B, C, D=None, dt_bias=None, *, y=None,
+                               stream=None):
+    """One decode step of the diagonal-A scan, in place on state [b,Dc,N] fp32;
+    x, dt [b,Dc] and B, C [b,N] in one dtype.  Returns y [b,Dc]."""
+    lib = load_library()
+    b, Dc = x.shape
+    N = A.shape[1]
+    if state.dtype != torch.float32:
+        raise TypeError("state must be float32")
+    y = y if y is not None else torch.empty_like(x)
+    a = SsdSelectiveStateUpdateArgs()
+    a.batch, a.channels, a.dstate = b, Dc, N
+    a.dtype = _dtype_code(x)
+    a.flags = 0
+    a.state, a.x, a.dt, a.A, a.B, a.C = (_ptr(state), _ptr(x), _ptr(dt), _ptr(A), _ptr(B),
+                                         _ptr(C))
+    a.D, a.dt_bias, a.y = _ptr(D), _ptr(dt_bias), _ptr(y)
+    _check(lib.ssd_selective_state_update(ctypes.byref(a), _stream_ptr(stream)),
+           "ssd_selective_state_update")
     return y
 
 

@@ -209,6 +209,31 @@ BwdWs bwd_layout(const ssd_bwd_args& a) {
     return w;
 }
 
+ssd_status check_sel_sizes(const ssd_selective_scan_args* a) {
+    if (!a) return SSD_ERR_INVALID_ARG;
+    if (a->batch <= 0 || a->seqlen <= 0 || a->channels <= 0 || a->dstate <= 0 || a->chunk <= 0)
+        return SSD_ERR_INVALID_ARG;
+    if (a->dtype != SSD_F32 && a->dtype != SSD_BF16) return SSD_ERR_INVALID_ARG;
+    if (a->dstate % 4 != 0 || a->dstate > 32 || a->chunk * a->dstate > 4096 || a->batch > 65535)
+        return SSD_ERR_UNSUPPORTED;
+    const int64_t nc = (a->seqlen + a->chunk - 1) / a->chunk;
+    if (nc > 65535 || (a->channels + 127) / 128 > 0x7fffffffLL) return SSD_ERR_UNSUPPORTED;
+    return SSD_OK;
+}
+
+struct SelWs {
+    size_t S, sdt, total;
+};
+
+SelWs sel_layout(const ssd_selective_scan_args& a) {
+    const int64_t nc = (a.seqlen + a.chunk - 1) / a.chunk;
+    SelWs w;
+    w.S = 0;
+    w.sdt = round_up((size_t)a.batch * nc * a.channels * a.dstate * sizeof(float));
+    w.total = w.sdt + round_up((size_t)a.batch * nc * a.channels * sizeof(float));
+    return w;
+}
+
 // Largest opt-in shared memory per CTA on sm_100 (227 KB).
 constexpr size_t kMaxSmemOptin = 232448;
 
@@ -375,6 +400,79 @@ ssd_status ssd_bwd_check_status(const ssd_bwd_args* a, void* stream) {
         cudaStreamSynchronize(s) != cudaSuccess)
         return SSD_ERR_CUDA;
     return v == 0 ? SSD_OK : static_cast<ssd_status>(v);
+}
+
+size_t ssd_selective_scan_workspace_size(const ssd_selective_scan_args* args) {
+    if (check_sel_sizes(args) != SSD_OK) return 0;
+    return sel_layout(*args).total;
+}
+
+ssd_status ssd_selective_scan(const ssd_selective_scan_args* a, void* stream) {
+    const ssd_status st = check_sel_sizes(a);
+    if (st != SSD_OK) return st;
+    if (!check_ptr(a->x, false, false) || !check_ptr(a->dt, false, false) ||
+        !check_ptr(a->A, false, true) || !check_ptr(a->B, false, false) ||
+        !check_ptr(a->C, false, false) || !check_ptr(a->D, true, false) ||
+        !check_ptr(a->dt_bias, true, false) || !check_ptr(a->init_state, true, true) ||
+        !check_ptr(a->y, false, false) || !check_ptr(a->final_state, true, true))
+        return SSD_ERR_INVALID_ARG;
+    const SelWs w = sel_layout(*a);
+    if (!a->workspace || a->workspace_bytes < w.total || !check_ptr(a->workspace, false, true))
+        return SSD_ERR_INVALID_ARG;
+    ssd::SelParams p;
+    p.batch = a->batch;
+    p.seqlen = a->seqlen;
+    p.channels = a->channels;
+    p.dstate = a->dstate;
+    p.chunk = a->chunk;
+    p.nchunks = (a->seqlen + a->chunk - 1) / a->chunk;
+    p.x = a->x;
+    p.dt_raw = a->dt;
+    p.A = a->A;
+    p.B = a->B;
+    p.C = a->C;
+    p.D = a->D;
+    p.dt_bias = a->dt_bias;
+    p.init_state = a->init_state;
+    p.y = a->y;
+    p.final_state = a->final_state;
+    char* ws = static_cast<char*>(a->workspace);
+    p.S = reinterpret_cast<float*>(ws + w.S);
+    p.sdt = reinterpret_cast<float*>(ws + w.sdt);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return to_status(a->dtype == SSD_BF16 ? ssd::launch_selective_scan<__nv_bfloat16>(p, false, s)
+                                          : ssd::launch_selective_scan<float>(p, false, s));
+}
+
+ssd_status ssd_selective_state_update(const ssd_selective_state_update_args* a, void* stream) {
+    if (!a) return SSD_ERR_INVALID_ARG;
+    if (a->batch <= 0 || a->channels <= 0 || a->dstate <= 0) return SSD_ERR_INVALID_ARG;
+    if (a->dtype != SSD_F32 && a->dtype != SSD_BF16) return SSD_ERR_INVALID_ARG;
+    if (a->dstate % 4 != 0 || a->dstate > 32) return SSD_ERR_UNSUPPORTED;
+    if (!check_ptr(a->state, false, true) || !check_ptr(a->x, false, false) ||
+        !check_ptr(a->dt, false, false) || !check_ptr(a->A, false, false) ||
+        !check_ptr(a->B, false, false) || !check_ptr(a->C, false, false) ||
+        !check_ptr(a->D, true, false) || !check_ptr(a->dt_bias, true, false) ||
+        !check_ptr(a->y, false, false))
+        return SSD_ERR_INVALID_ARG;
+    ssd::SelParams p;
+    memset(&p, 0, sizeof(p));
+    p.batch = a->batch;
+    p.seqlen = 1;
+    p.channels = a->channels;
+    p.dstate = a->dstate;
+    p.x = a->x;
+    p.dt_raw = a->dt;
+    p.A = a->A;
+    p.B = a->B;
+    p.C = a->C;
+    p.D = a->D;
+    p.dt_bias = a->dt_bias;
+    p.y = a->y;
+    p.S = a->state;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return to_status(a->dtype == SSD_BF16 ? ssd::launch_selective_scan<__nv_bfloat16>(p, true, s)
+                                          : ssd::launch_selective_scan<float>(p, true, s));
 }
 
 ssd_status ssd_chunk_cumsum(const ssd_fwd_args* a, float* dt_out, float* cumA_out,

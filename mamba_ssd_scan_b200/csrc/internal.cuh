@@ -67,6 +67,23 @@ struct BwdParams {
     float* partial;          // [b, H, 3]: per-row sums of dt*da, dy.x, ddt_raw
 };
 
+// The diagonal-A selective scan (forward and decode step).
+struct SelParams {
+    int64_t batch, seqlen, channels, dstate, chunk, nchunks;
+    const void* x;           // [b, L, Dc] (forward) or [b, Dc] (decode)
+    const void* dt_raw;      // like x
+    const float* A;          // [Dc, N]
+    const void* B;           // [b, L, N] (forward) or [b, N] (decode)
+    const void* C;           // like B
+    const float* D;          // [Dc] or null
+    const float* dt_bias;    // [Dc] or null
+    const float* init_state; // [b, Dc, N] or null (forward)
+    void* y;                 // like x
+    float* final_state;      // [b, Dc, N] or null (forward)
+    float* S;                // forward: workspace [b, nc, Dc, N]; decode: the carried state [b, Dc, N]
+    float* sdt;              // forward: workspace [b, nc, Dc], the sum of dt over each chunk
+};
+
 struct DecodeParams {
     int64_t batch, nheads, headdim, dstate, ngroups, heads_per_group;
     float* state;
@@ -193,6 +210,8 @@ template <typename T> cudaError_t launch_state_passing(const FwdParams& p, cudaS
 template <typename T> cudaError_t launch_chunk_scan_ffma(const FwdParams& p, cudaStream_t s);
 template <typename T> cudaError_t launch_state_update(const DecodeParams& p, cudaStream_t s);
 template <typename T> cudaError_t launch_conv1d(const ConvParams& p, bool update, cudaStream_t s);
+template <typename T>
+cudaError_t launch_selective_scan(const SelParams& p, bool update, cudaStream_t s);
 // The backward pass after the forward recompute (bwd.cu).
 template <typename T> cudaError_t launch_ssd_bwd(const BwdParams& p, cudaStream_t s);
 // Shared memory (bytes) the backward's per-chunk kernels need for a shape.

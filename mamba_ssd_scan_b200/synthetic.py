@@ -94,10 +94,34 @@ CONV_CONFIGS = {
     "conv1d_update_b256_C7168": ConvConfig("conv1d_update_b256_C7168", 256, 1, 7168, 4,
                                            torch.bfloat16, steps=1024, layers=8),
 }
+
+
+@dataclasses.dataclass(frozen=True)
+class SelConfig:
+    """The diagonal-A selective scan: channels = d_inner of the model."""
+    name: str
+    batch: int
+    seqlen: int
+    channels: int
+    dstate: int
+    chunk: int
+    dtype: torch.dtype
+    steps: int = 0    # decode steps replayed (decode only)
+    layers: int = 1   # distinct carried states cycled through (decode only)
+
+
+SEL_CONFIGS = {
+    # the headline model's d_inner (d_model 768, expand 2) with Mamba-1's dstate 16
+    "sel_bf16_b4_L1024_D1536_N16": SelConfig("sel_bf16_b4_L1024_D1536_N16", 4, 1024, 1536, 16,
+                                             64, torch.bfloat16),
+    "sel_update_b256_D1536_N16": SelConfig("sel_update_b256_D1536_N16", 256, 1, 1536, 16, 1,
+                                           torch.bfloat16, steps=1024, layers=8),
+}
 # the seed offset of each workload (seed = 1234 + offset)
 SEED_OFFSET = {"fwd_f32_small": 0, "fwd_bf16_b4_L1024": 1, "fwd_bf16_b8_L4096_init": 2,
                "fwd_bf16_b1_L65536_G8": 3, "decode_b256_H80": 4,
-               "conv1d_bf16_b8_L4096_C2304": 5, "conv1d_update_b256_C7168": 6}
+               "conv1d_bf16_b8_L4096_C2304": 5, "conv1d_update_b256_C7168": 6,
+               "sel_bf16_b4_L1024_D1536_N16": 7, "sel_update_b256_D1536_N16": 8}
 
 
 def _uniform(gen, shape, lo, hi):
@@ -173,6 +197,25 @@ def make_bwd_grads(x_shape, state_shape, dtype, seed: int) -> dict:
     dy = torch.randn(x_shape, generator=gen).to(dtype)
     d_final = torch.randn(state_shape, generator=gen)
     return dict(dy=dy, d_final=d_final)
+
+
+def make_selective_inputs(batch, seqlen, channels, dstate, dtype, seed: int,
+                          init_state: bool = False) -> dict:
+    """Inputs of the diagonal-A selective scan: x, dt_raw, B, C ~ N(0,1) in
+    dtype; A[d,n] = -exp(A_log) with A_log = log(n+1) + U[-0.5, 0.5] (the
+    log(1..N) initialisation, perturbed per channel); dt_bias =
+    softplus^-1(U[1e-3, 0.1]); D ~ N(0,1); init ~ N(0, 0.1^2) (fp32)."""
+    gen = torch.Generator().manual_seed(seed + 65537)
+    x = torch.randn((batch, seqlen, channels), generator=gen).to(dtype)
+    dt = torch.randn((batch, seqlen, channels), generator=gen).to(dtype)
+    B = torch.randn((batch, seqlen, dstate), generator=gen).to(dtype)
+    C = torch.randn((batch, seqlen, dstate), generator=gen).to(dtype)
+    a_log = torch.log(torch.arange(1, dstate + 1, dtype=torch.float32)).expand(channels, dstate)
+    A = -torch.exp(a_log + _uniform(gen, (channels, dstate), -0.5, 0.5))
+    dt_bias = _inv_softplus(_uniform(gen, (channels,), 1e-3, 0.1))
+    D = torch.randn((channels,), generator=gen)
+    init = torch.randn((batch, channels, dstate), generator=gen) * 0.1 if init_state else None
+    return dict(x=x, dt=dt, A=A.contiguous(), B=B, C=C, D=D, dt_bias=dt_bias, init_state=init)
 
 
 def make_conv_inputs(batch, seqlen, channels, width, dtype, seed: int,

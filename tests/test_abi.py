@@ -146,3 +146,23 @@ def test_bwd_rejects_bad_args(lib):
     assert lib.ssd_bwd(ctypes.byref(a), None) == 2               # tiles beyond shared memory
     a.dstate, a.ngroups = 64, 3
     assert lib.ssd_bwd(ctypes.byref(a), None) == 1               # heads not divisible by groups
+
+
+def test_selective_scan_rejects_bad_args(lib):
+    import mamba_ssd_scan_b200 as ssd
+    a = ssd.SsdSelectiveScanArgs()
+    a.batch, a.seqlen, a.channels, a.dstate, a.chunk, a.dtype = 1, 64, 32, 16, 64, 0
+    assert lib.ssd_selective_scan(None, None) == 1
+    assert lib.ssd_selective_scan_workspace_size(ctypes.byref(a)) > 0
+    assert lib.ssd_selective_scan(ctypes.byref(a), None) == 1     # null pointers
+    a.dstate = 6
+    assert lib.ssd_selective_scan(ctypes.byref(a), None) == 2     # dstate not a multiple of 4
+    a.dstate = 36
+    assert lib.ssd_selective_scan(ctypes.byref(a), None) == 2     # dstate beyond 32
+    a.dstate, a.chunk = 32, 256
+    assert lib.ssd_selective_scan_workspace_size(ctypes.byref(a)) == 0   # chunk * dstate > 4096
+    u = ssd.SsdSelectiveStateUpdateArgs()
+    u.batch, u.channels, u.dstate, u.dtype = 2, 32, 16, 1
+    assert lib.ssd_selective_state_update(ctypes.byref(u), None) == 1   # null pointers
+    u.dstate = 40
+    assert lib.ssd_selective_state_update(ctypes.byref(u), None) == 2
