@@ -57,6 +57,8 @@ def parse_args():
                     help="time only the convolution workloads (one JSON line of them)")
     ap.add_argument("--bwd-only", action="store_true",
                     help="time only the backward-pass workloads (one JSON line of them)")
+    ap.add_argument("--sel-only", action="store_true",
+                    help="time only the diagonal-A selective-scan workloads (one JSON line)")
     return ap.parse_args()
 
 
@@ -240,10 +242,13 @@ def main_ours(args):
         flush_buf.fill_(1)
         torch.sum(flush_f, dim=0, out=flush_acc)
 
-    if args.conv_only or args.bwd_only:
-        res = (conv_workloads(ssd, synthetic, dev, flush, peaks, rank, world, ranks_max)
-               if args.conv_only else bwd_workloads(ssd, synthetic, dev, flush, rank, world,
-                                                   ranks_max))
+    if args.conv_only or args.bwd_only or args.sel_only:
+        if args.conv_only:
+            res = conv_workloads(ssd, synthetic, dev, flush, peaks, rank, world, ranks_max)
+        elif args.bwd_only:
+            res = bwd_workloads(ssd, synthetic, dev, flush, rank, world, ranks_max)
+        else:
+            res = sel_workloads(ssd, synthetic, dev, flush, peaks, rank, world, ranks_max)
         if rank == 0:
             print(json.dumps({"workloads": res, "peaks_source": peaks["source"]}), flush=True)
         return
@@ -655,6 +660,106 @@ def other_workloads(ssd, synthetic, dev, flush, peaks, rank, world, barrier, ran
     torch.cuda.empty_cache()
     out.update(conv_workloads(ssd, synthetic, dev, flush, peaks, rank, world, ranks_max))
     out.update(bwd_workloads(ssd, synthetic, dev, flush, rank, world, ranks_max))
+    out.update(sel_workloads(ssd, synthetic, dev, flush, peaks, rank, world, ranks_max))
+    return out
+
+
+# MUFU (special-function) throughput: 16 results per clock per SM, 148 SMs, 1.965 GHz
+MUFU_TOPS = 148 * 16 * 1.965e9 / 1e12
+
+
+def sel_workloads(ssd, synthetic, dev, flush, peaks, rank, world, ranks_max, steps=10):
+    """The diagonal-A selective scan: the forward over a sequence (L2 flushed
+    before each call; bound by the exponential of every (token, channel,
+    state), reported against the MUFU rate) and the decode step (1024 steps in
+    one CUDA graph over 8 layers' states, against HBM)."""
+    import torch
+    out = {}
+    stream = torch.cuda.current_stream()
+    cfg = synthetic.SEL_CONFIGS["sel_bf16_b4_L1024_D1536_N16"]
+    seed = rank_seed(1234 + synthetic.SEED_OFFSET[cfg.name], rank)
+    inp = synthetic.make_selective_inputs(cfg.batch, cfg.seqlen, cfg.channels, cfg.dstate,
+                                          cfg.dtype, seed, init_state=True)
+    d = {k: v.to(dev) for k, v in inp.items()}
+    y = torch.empty_like(d["x"])
+    fin = torch.empty_like(d["init_state"])
+    ws = torch.empty(ssd.ssd_selective_scan_workspace_size(cfg.batch, cfg.seqlen, cfg.channels,
+                                                           cfg.dstate, cfg.chunk, cfg.dtype),
+                     dtype=torch.uint8, device=dev)
+
+    def step():
+        ssd.ssd_selective_scan(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["dt_bias"],
+                               chunk=cfg.chunk, init_state=d["init_state"], y=y,
+                               final_state=fin, workspace=ws)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    gpu_head_start(2.0)
+    for a, b_ in evs:
+        flush()
+        a.record(stream)
+        step()
+        b_.record(stream)
+    torch.cuda.synchronize()
+    ms = ranks_max(sum(a.elapsed_time(b_) for a, b_ in evs) / steps)
+    exps = cfg.batch * cfg.seqlen * cfg.channels * cfg.dstate  # one exp per (t, d, n)
+    nbytes = (3 * cfg.batch * cfg.seqlen * cfg.channels * 2 + 2 * cfg.batch * cfg.seqlen *
+              cfg.dstate * 2 + 2 * cfg.batch * cfg.channels * cfg.dstate * 4)
+    out[cfg.name] = {"tokens_per_s": job_throughput(cfg.batch * cfg.seqlen, world, ms), "ms": ms,
+                     "bound": "alu", "exp_per_s": exps / (ms * 1e-3),
+                     "mufu_frac": exps / (ms * 1e-3) / (MUFU_TOPS * 1e12),
+                     "hbm_frac": nbytes / (ms * 1e-3) / (peaks["hbm_gbs"] * 1e9),
+                     "l2": "flushed"}
+    del d, y, fin, ws
+
+    cfg = synthetic.SEL_CONFIGS["sel_update_b256_D1536_N16"]
+    seed = rank_seed(1234 + synthetic.SEED_OFFSET[cfg.name], rank)
+    per = [synthetic.make_selective_inputs(cfg.batch, 16, cfg.channels, cfg.dstate, cfg.dtype,
+                                           seed + 97 * l, init_state=True)
+           for l in range(cfg.layers)]
+    states = [p_["init_state"].to(dev) for p_ in per]
+    As = [p_["A"].to(dev) for p_ in per]
+    Ds = [p_["D"].to(dev) for p_ in per]
+    bs = [p_["dt_bias"].to(dev) for p_ in per]
+    tok = [{k: per[0][k][:, t].contiguous().to(dev) for k in ("x", "dt", "B", "C")}
+           for t in range(16)]
+    yd = torch.empty((cfg.batch, cfg.channels), dtype=cfg.dtype, device=dev)
+    del per
+
+    def run(n):
+        for s_ in range(n):
+            l = s_ % cfg.layers
+            tk = tok[s_ % len(tok)]
+            ssd.ssd_selective_state_update(states[l], tk["x"], tk["dt"], As[l], tk["B"], tk["C"],
+                                           Ds[l], bs[l], y=yd)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        run(3)
+    torch.cuda.current_stream().wait_stream(side)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        run(cfg.steps)
+    g.replay()
+    torch.cuda.synchronize()
+    a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    g.replay()
+    b_.record(stream)
+    torch.cuda.synchronize()
+    us = ranks_max(a.elapsed_time(b_) * 1e3 / cfg.steps)
+    step_bytes = (2 * cfg.batch * cfg.channels * cfg.dstate * 4 + 3 * cfg.batch * cfg.channels * 2
+                  + 2 * cfg.batch * cfg.dstate * 2 + cfg.channels * (cfg.dstate + 2) * 4)
+    out[cfg.name] = {"us_per_step": us, "steps": cfg.steps, "graph": True, "layers": cfg.layers,
+                     "achieved_gbs": step_bytes / (us * 1e-6) / 1e9,
+                     "hbm_frac": step_bytes / (us * 1e-6) / (peaks["hbm_gbs"] * 1e9),
+                     "bytes_per_step": step_bytes}
+    del g, states
+    torch.cuda.empty_cache()
     return out
 
 

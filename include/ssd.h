@@ -293,8 +293,10 @@ size_t ssd_selective_scan_workspace_size(const ssd_selective_scan_args* args);
 ssd_status ssd_selective_scan(const ssd_selective_scan_args* args, void* stream);
 
 /* One decode step of the same scan on a carried state [batch, channels,
- * dstate] fp32 (16-byte aligned), updated in place; x, dt, y [batch,
- * channels] dtype; B, C [batch, dstate] dtype.  Supported dstate as above. */
+ * dstate] fp32, updated in place; x, dt, y [batch, channels] dtype; B, C
+ * [batch, dstate] dtype.  state, A, B and C 16-byte aligned (else
+ * SSD_ERR_INVALID_ARG); dstate as above.  Consecutive calls on one stream go
+ * out with programmatic dependent launch. */
 typedef struct {
     int64_t batch, channels, dstate;
     int32_t dtype;

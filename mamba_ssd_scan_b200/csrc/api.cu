@@ -450,8 +450,8 @@ ssd_status ssd_selective_state_update(const ssd_selective_state_update_args* a, 
     if (a->dtype != SSD_F32 && a->dtype != SSD_BF16) return SSD_ERR_INVALID_ARG;
     if (a->dstate % 4 != 0 || a->dstate > 32) return SSD_ERR_UNSUPPORTED;
     if (!check_ptr(a->state, false, true) || !check_ptr(a->x, false, false) ||
-        !check_ptr(a->dt, false, false) || !check_ptr(a->A, false, false) ||
-        !check_ptr(a->B, false, false) || !check_ptr(a->C, false, false) ||
+        !check_ptr(a->dt, false, false) || !check_ptr(a->A, false, true) ||
+        !check_ptr(a->B, false, true) || !check_ptr(a->C, false, true) ||
         !check_ptr(a->D, true, false) || !check_ptr(a->dt_bias, true, false) ||
         !check_ptr(a->y, false, false))
         return SSD_ERR_INVALID_ARG;

@@ -24,7 +24,9 @@
 namespace ssd {
 namespace {
 
-constexpr int CT = 128;  // threads (channels) per CTA
+// threads (channels) per CTA; with dstate <= 16 at most 80 registers each keeps 6
+// CTAs (24 warps) per SM, which measured faster than fewer, larger-register CTAs
+constexpr int CT = 128;
 
 __device__ __forceinline__ float ex2f(float v) {
     float r;
@@ -33,9 +35,41 @@ __device__ __forceinline__ float ex2f(float v) {
 }
 
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr int TU = 4;  // tokens whose x and dt loads are in flight together
+
+// x and dt of one channel for TU tokens at a time: the next group's loads go
+// out when the current group is taken, so they overlap its arithmetic.
+template <typename T>
+struct TokenQueue {
+    const T* x;
+    const T* dt;
+    int64_t stride;
+    int n;
+    float nx[TU], nd[TU];
+    __device__ __forceinline__ TokenQueue(const T* x_, const T* dt_, int64_t stride_, int n_)
+        : x(x_), dt(dt_), stride(stride_), n(n_) {
+        load(0);
+    }
+    __device__ __forceinline__ void load(int t0) {
+#pragma unroll
+        for (int u = 0; u < TU; ++u) {
+            const bool ok = t0 + u < n;
+            nx[u] = ok ? to_f32(x[(t0 + u) * stride]) : 0.0f;
+            nd[u] = ok ? to_f32(dt[(t0 + u) * stride]) : 0.0f;
+        }
+    }
+    __device__ __forceinline__ void take(int t0, float (&xv)[TU], float (&dv)[TU]) {
+#pragma unroll
+        for (int u = 0; u < TU; ++u) {
+            xv[u] = nx[u];
+            dv[u] = nd[u];
+        }
+        if (t0 + TU < n) load(t0 + TU);
+    }
+};
 
 template <typename T, int N>
-__global__ void __launch_bounds__(CT) sel_local_kernel(SelParams p) {
+__global__ void __launch_bounds__(CT, N <= 16 ? 6 : 3) sel_local_kernel(SelParams p) {
     extern __shared__ __align__(16) float sb[];  // [chunk][N] B rows of the chunk
     const int64_t L = p.seqlen, Dc = p.channels, Q = p.chunk, nc = p.nchunks;
     const int64_t c = blockIdx.y, b = blockIdx.z, t0 = c * Q;
@@ -55,13 +89,22 @@ __global__ void __launch_bounds__(CT) sel_local_kernel(SelParams p) {
     const T* xg = static_cast<const T*>(p.x) + (b * L + t0) * Dc + d;
     const T* dg = static_cast<const T*>(p.dt_raw) + (b * L + t0) * Dc + d;
     float sdt = 0.0f;
-    for (int t = 0; t < Lc; ++t) {
-        const float dt = softplus_f32(to_f32(dg[t * Dc]) + bias);
-        const float dx = dt * to_f32(xg[t * Dc]);
-        sdt += dt;
-        const float* bt = sb + t * N;
+    TokenQueue<T> qx(xg, dg, Dc, Lc);
+    for (int t0g = 0; t0g < Lc; t0g += TU) {
+        float xv[TU], dv[TU];
+        qx.take(t0g, xv, dv);
 #pragma unroll
-        for (int n = 0; n < N; ++n) h[n] = fmaf(ex2f(dt * a2[n]), h[n], dx * bt[n]);
+        for (int u = 0; u < TU; ++u) {
+            const int t = t0g + u;
+            if (t < Lc) {
+                const float dt = softplus_f32(dv[u] + bias);
+                const float dx = dt * xv[u];
+                sdt += dt;
+                const float* bt = sb + t * N;
+#pragma unroll
+                for (int n = 0; n < N; ++n) h[n] = fmaf(ex2f(dt * a2[n]), h[n], dx * bt[n]);
+            }
+        }
     }
     float4* out = reinterpret_cast<float4*>(p.S + ((b * nc + c) * Dc + d) * N);
 #pragma unroll
@@ -70,7 +113,10 @@ __global__ void __launch_bounds__(CT) sel_local_kernel(SelParams p) {
 }
 
 // One thread per 4 states of one (b, d): H_{c} (entering chunk c) in place of
-// the local state S_c, the final state after the last chunk.
+// the local state S_c, the final state after the last chunk.  The loads of
+// CU chunks (independent of the carry) go out before their multiply-adds.
+constexpr int CU = 8;
+
 __global__ void __launch_bounds__(256) sel_carry_kernel(SelParams p) {
     const int64_t Dc = p.channels, N = p.dstate, nc = p.nchunks;
     const int64_t nv = N / 4;
@@ -80,21 +126,35 @@ __global__ void __launch_bounds__(256) sel_carry_kernel(SelParams p) {
     float4 carry = p.init_state ? reinterpret_cast<const float4*>(p.init_state)[e]
                                 : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
     const float4 a = reinterpret_cast<const float4*>(p.A + d * N)[q];
-    for (int64_t c = 0; c < nc; ++c) {
-        float4* sp = reinterpret_cast<float4*>(p.S + ((b * nc + c) * Dc + d) * N) + q;
-        const float4 s = *sp;
-        const float st = p.sdt[(b * nc + c) * Dc + d];
-        *sp = carry;
-        carry.x = fmaf(expf(a.x * st), carry.x, s.x);
-        carry.y = fmaf(expf(a.y * st), carry.y, s.y);
-        carry.z = fmaf(expf(a.z * st), carry.z, s.z);
-        carry.w = fmaf(expf(a.w * st), carry.w, s.w);
+    float4* sbase = reinterpret_cast<float4*>(p.S + (b * nc * Dc + d) * N) + q;
+    const int64_t cstride = Dc * nv;  // float4s between consecutive chunks
+    const float* sdt = p.sdt + b * nc * Dc + d;
+    for (int64_t c0 = 0; c0 < nc; c0 += CU) {
+        float4 sv[CU];
+        float st[CU];
+#pragma unroll
+        for (int u = 0; u < CU; ++u) {
+            if (c0 + u < nc) {
+                sv[u] = sbase[(c0 + u) * cstride];
+                st[u] = sdt[(c0 + u) * Dc];
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < CU; ++u) {
+            if (c0 + u < nc) {
+                sbase[(c0 + u) * cstride] = carry;
+                carry.x = fmaf(expf(a.x * st[u]), carry.x, sv[u].x);
+                carry.y = fmaf(expf(a.y * st[u]), carry.y, sv[u].y);
+                carry.z = fmaf(expf(a.z * st[u]), carry.z, sv[u].z);
+                carry.w = fmaf(expf(a.w * st[u]), carry.w, sv[u].w);
+            }
+        }
     }
     if (p.final_state) reinterpret_cast<float4*>(p.final_state)[e] = carry;
 }
 
 template <typename T, int N>
-__global__ void __launch_bounds__(CT) sel_output_kernel(SelParams p) {
+__global__ void __launch_bounds__(CT, N <= 16 ? 6 : 3) sel_output_kernel(SelParams p) {
     extern __shared__ __align__(16) float sbc[];  // [chunk][N] B rows, then [chunk][N] C rows
     const int64_t L = p.seqlen, Dc = p.channels, Q = p.chunk, nc = p.nchunks;
     const int64_t c = blockIdx.y, b = blockIdx.z, t0 = c * Q;
@@ -124,59 +184,99 @@ __global__ void __launch_bounds__(CT) sel_output_kernel(SelParams p) {
     const T* xg = static_cast<const T*>(p.x) + (b * L + t0) * Dc + d;
     const T* dg = static_cast<const T*>(p.dt_raw) + (b * L + t0) * Dc + d;
     T* yg = static_cast<T*>(p.y) + (b * L + t0) * Dc + d;
-    for (int t = 0; t < Lc; ++t) {
-        const float xv = to_f32(xg[t * Dc]);
-        const float dt = softplus_f32(to_f32(dg[t * Dc]) + bias);
-        const float dx = dt * xv;
-        const float* bt = sb + t * N;
-        const float* ct = sc + t * N;
-        float acc = 0.0f;
+    TokenQueue<T> qx(xg, dg, Dc, Lc);
+    for (int t0g = 0; t0g < Lc; t0g += TU) {
+        float xv[TU], dv[TU];
+        qx.take(t0g, xv, dv);
 #pragma unroll
-        for (int n = 0; n < N; ++n) {
-            h[n] = fmaf(ex2f(dt * a2[n]), h[n], dx * bt[n]);
-            acc = fmaf(ct[n], h[n], acc);
+        for (int u = 0; u < TU; ++u) {
+            const int t = t0g + u;
+            if (t < Lc) {
+                const float dt = softplus_f32(dv[u] + bias);
+                const float dx = dt * xv[u];
+                const float* bt = sb + t * N;
+                const float* ct = sc + t * N;
+                float acc = 0.0f;
+#pragma unroll
+                for (int n = 0; n < N; ++n) {
+                    h[n] = fmaf(ex2f(dt * a2[n]), h[n], dx * bt[n]);
+                    acc = fmaf(ct[n], h[n], acc);
+                }
+                yg[t * Dc] = from_f32<T>(fmaf(Dd, xv[u], acc));
+            }
         }
-        yg[t * Dc] = from_f32<T>(fmaf(Dd, xv, acc));
     }
 }
 
-// Decode: one thread per (b, d), its N states moved as 16-byte vectors.
+// Decode: one thread per (b, d), its N states and A row moved as 16-byte
+// vectors, B and C of the batch row as 4-element vectors.  Consecutive steps
+// go out with programmatic dependent launch (wait for the previous step's
+// state, then let the next step's CTAs in).
+template <typename T> struct Vec4;
+template <> struct Vec4<float> {
+    static __device__ __forceinline__ float4 load(const float* p) {
+        return __ldg(reinterpret_cast<const float4*>(p));
+    }
+};
+template <> struct Vec4<__nv_bfloat16> {
+    static __device__ __forceinline__ float4 load(const __nv_bfloat16* p) {
+        const uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
+        return make_float4(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u),
+                           __uint_as_float(v.y << 16), __uint_as_float(v.y & 0xffff0000u));
+    }
+};
+
 template <typename T, int N>
 __global__ void __launch_bounds__(256) sel_update_kernel(SelParams p) {
     const int64_t Dc = p.channels;
     const int64_t e = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (e >= p.batch * Dc) return;
     const int64_t b = e / Dc, d = e % Dc;
+    grid_dep_wait();
+    grid_dep_launch();
     float4* sp = reinterpret_cast<float4*>(p.S + e * N);
-    float h[N];
+    const float4* ap = reinterpret_cast<const float4*>(p.A + d * N);
+    const T* Bg = static_cast<const T*>(p.B) + b * N;
+    const T* Cg = static_cast<const T*>(p.C) + b * N;
+    // every load first (the stores below could alias them for the compiler),
+    // then the arithmetic, then the stores
+    float4 hv[N / 4], av[N / 4], bv[N / 4], cv[N / 4];
 #pragma unroll
-    for (int n = 0; n < N; n += 4) {
-        const float4 v = sp[n / 4];
-        h[n] = v.x; h[n + 1] = v.y; h[n + 2] = v.z; h[n + 3] = v.w;
+    for (int q = 0; q < N / 4; ++q) {
+        hv[q] = sp[q];
+        av[q] = __ldg(ap + q);
+        bv[q] = Vec4<T>::load(Bg + 4 * q);
+        cv[q] = Vec4<T>::load(Cg + 4 * q);
     }
     const float xv = to_f32(static_cast<const T*>(p.x)[e]);
     const float dt = softplus_f32(to_f32(static_cast<const T*>(p.dt_raw)[e]) +
                                   (p.dt_bias ? p.dt_bias[d] : 0.0f));
-    const float dx = dt * xv;
-    const T* Bg = static_cast<const T*>(p.B) + b * N;
-    const T* Cg = static_cast<const T*>(p.C) + b * N;
+    const float Dd = p.D ? p.D[d] : 0.0f;
+    const float dx = dt * xv, dl = dt * kLog2e;
     float acc = 0.0f;
 #pragma unroll
-    for (int n = 0; n < N; ++n) {
-        h[n] = fmaf(ex2f(dt * p.A[d * N + n] * kLog2e), h[n], dx * to_f32(Bg[n]));
-        acc = fmaf(to_f32(Cg[n]), h[n], acc);
+    for (int q = 0; q < N / 4; ++q) {
+        float4& h = hv[q];
+        h.x = fmaf(ex2f(dl * av[q].x), h.x, dx * bv[q].x);
+        h.y = fmaf(ex2f(dl * av[q].y), h.y, dx * bv[q].y);
+        h.z = fmaf(ex2f(dl * av[q].z), h.z, dx * bv[q].z);
+        h.w = fmaf(ex2f(dl * av[q].w), h.w, dx * bv[q].w);
+        acc = fmaf(cv[q].x, h.x, acc);
+        acc = fmaf(cv[q].y, h.y, acc);
+        acc = fmaf(cv[q].z, h.z, acc);
+        acc = fmaf(cv[q].w, h.w, acc);
     }
 #pragma unroll
-    for (int n = 0; n < N; n += 4) sp[n / 4] = make_float4(h[n], h[n + 1], h[n + 2], h[n + 3]);
-    static_cast<T*>(p.y)[e] = from_f32<T>(fmaf(p.D ? p.D[d] : 0.0f, xv, acc));
+    for (int q = 0; q < N / 4; ++q) sp[q] = hv[q];
+    static_cast<T*>(p.y)[e] = from_f32<T>(fmaf(Dd, xv, acc));
 }
 
 template <typename T, int N>
 cudaError_t launch_n(const SelParams& p, bool update, cudaStream_t s) {
     if (update) {
         const int64_t n = p.batch * p.channels;
-        sel_update_kernel<T, N><<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(p);
-        return cudaGetLastError();
+        return launch_kernel(sel_update_kernel<T, N>, dim3(static_cast<unsigned>((n + 255) / 256)),
+                             dim3(256), 0, s, true, p);
     }
     const dim3 grid(static_cast<unsigned>((p.channels + CT - 1) / CT),
                     static_cast<unsigned>(p.nchunks), static_cast<unsigned>(p.batch));

@@ -113,7 +113,7 @@ class SelConfig:
 SEL_CONFIGS = {
     # the headline model's d_inner (d_model 768, expand 2) with Mamba-1's dstate 16
     "sel_bf16_b4_L1024_D1536_N16": SelConfig("sel_bf16_b4_L1024_D1536_N16", 4, 1024, 1536, 16,
-                                             64, torch.bfloat16),
+                                             32, torch.bfloat16),
     "sel_update_b256_D1536_N16": SelConfig("sel_update_b256_D1536_N16", 256, 1, 1536, 16, 1,
                                            torch.bfloat16, steps=1024, layers=8),
 }
