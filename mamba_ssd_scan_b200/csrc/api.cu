@@ -383,6 +383,7 @@ ssd_status ssd_bwd(const ssd_bwd_args* a, void* stream) {
     bp.roww = reinterpret_cast<float*>(ws + w.roww);
     bp.k4 = reinterpret_cast<float*>(ws + w.k4);
     bp.partial = reinterpret_cast<float*>(ws + w.partial);
+    bp.rblk = (use_tc(a->dtype, a->flags) && ssd::bwd_tc_supported(p)) ? 128 : 64;
     return to_status(a->dtype == SSD_BF16 ? ssd::launch_ssd_bwd<__nv_bfloat16>(bp, s)
                                           : ssd::launch_ssd_bwd<float>(bp, s));
 }

@@ -545,7 +545,7 @@ __global__ void __launch_bounds__(DTW * 32) bwd_dt_kernel(BwdParams bp) {
     __shared__ float spre[DTW][256];  // exclusive prefix of m + colw - roww over the chunk
     const FwdParams& p = bp.f;
     const int64_t H = p.nheads, L = p.seqlen, Q = p.chunk, nc = p.nchunks;
-    const int NB = static_cast<int>(Q / BR);
+    const int RB = bp.rblk, NB = static_cast<int>(Q / RB);
     const int wi = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t w = static_cast<int64_t>(blockIdx.x) * DTW + wi;
     if (w >= p.batch * H) return;
@@ -572,7 +572,7 @@ __global__ void __launch_bounds__(DTW * 32) bwd_dt_kernel(BwdParams bp) {
             if (l < Lc) {
                 const int64_t t = t0 + l;
                 float rsum = 0.0f;
-                for (int i = 0; i <= l / BR; ++i) rsum += rw[i * L + t];
+                for (int i = 0; i <= l / RB; ++i) rsum += rw[i * L + t];
                 v = mt[t] + cw[t] - rsum;
             }
             float incl = v;
@@ -682,7 +682,9 @@ cudaError_t launch_ssd_bwd(const BwdParams& bp, cudaStream_t s) {
         bwd_state_passing_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(bp);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    {
+    if (bp.rblk == 128) {
+        if ((e = launch_bwd_tc(bp, s)) != cudaSuccess) return e;
+    } else {
         const size_t sa = static_cast<size_t>(smem_a_floats(P, N, p.chunk)) * sizeof(float);
         const size_t sb = static_cast<size_t>(smem_b_floats(P, N, p.chunk)) * sizeof(float);
         if ((e = cudaFuncSetAttribute(bwd_chunk_a_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,

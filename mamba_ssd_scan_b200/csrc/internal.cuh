@@ -62,7 +62,8 @@ struct BwdParams {
     float* mterm;            // [b, H, L]: dt_t x_t . (the dH part of dxs_t)
     float* qterm;            // [b, H, L]: e^{cumA_t} dy_t . (H_c C_t)
     float* colw;             // [b, H, L]: sum over later tokens s of the chunk of W[s, t]
-    float* roww;             // [b, H, Q/64, L]: per 64-token source block, sum over earlier r of W[t, r]
+    float* roww;             // [b, H, Q/rblk, L]: per source block of rblk tokens, sum over earlier r of W[t, r]
+    int32_t rblk;            // tokens per source block of roww (64: CUDA-core kernels, 128: tensor cores)
     float* k4;               // [b, H, nc]: e^{cumA_c[last]} <dH_c, H_c>
     float* partial;          // [b, H, 3]: per-row sums of dt*da, dy.x, ddt_raw
 };
@@ -214,6 +215,10 @@ template <typename T>
 cudaError_t launch_selective_scan(const SelParams& p, bool update, cudaStream_t s);
 // The backward pass after the forward recompute (bwd.cu).
 template <typename T> cudaError_t launch_ssd_bwd(const BwdParams& p, cudaStream_t s);
+// The backward's per-chunk kernels on the tensor cores (bf16, headdim 64,
+// dstate 64 or 128, chunk 128 or 256); false when the shape is outside that.
+bool bwd_tc_supported(const FwdParams& p);
+cudaError_t launch_bwd_tc(const BwdParams& p, cudaStream_t s);
 // Shared memory (bytes) the backward's per-chunk kernels need for a shape.
 size_t bwd_smem_bytes(int64_t headdim, int64_t dstate, int64_t chunk);
 // Copies the forward kernel's device status word to *v and clears it (synchronises s).
