@@ -203,7 +203,7 @@ BwdWs bwd_layout(const ssd_bwd_args& a) {
     w.roww = w.colw + round_up(tok);
     w.k4 = w.roww + round_up(tok * (size_t)(a.chunk / 64));
     w.partial = w.k4 + round_up((size_t)a.batch * a.nheads * nc * sizeof(float));
-    w.dBh = w.partial + round_up((size_t)a.batch * a.nheads * 3 * sizeof(float));
+    w.dBh = w.partial + round_up((size_t)a.batch * a.nheads * nc * 3 * sizeof(float));
     w.dCh = w.dBh + round_up(per_head);
     w.total = w.dCh + round_up(per_head);
     return w;

@@ -529,17 +529,18 @@ __global__ void __launch_bounds__(NT) bwd_chunk_b_kernel(BwdParams bp) {
 }
 
 // ---------------------------------------------------------------------------
-// One warp per (b, h), chunk by chunk: the gradient of the log decay a_t,
+// The gradient of the log decay a_t, one chunk per warp:
 //   da_t = e^{a_t} <g_t, h_{t-1}>
 //        = k4_c + sum_{s in c, s>=t} q_s + sum_{r in c, r<t} (m_r + colw_r - roww_r)
 // (g_t = dJ/dh_t; splitting g_t and h_{t-1} at the chunk's boundary gives the
 // dH_c . H_c constant, the H_c . dy_s C_s^T terms q, the dH_c . x_r B_r^T terms
 // m, and the pairs r < t <= s inside the chunk, W[s, r], whose sum over the
 // pairs straddling t is the prefix of column-minus-row sums of W), then ddt_t,
-// ddt_raw_t and the row's sums of dt da, dy.x and ddt_raw.  All sums run over
+// ddt_raw_t and the chunk's sums of dt da, dy.x and ddt_raw.  All sums run over
 // one chunk at most.
 constexpr int DTW = 8;  // warps per CTA of bwd_dt_kernel
 
+// One warp per (b, h, chunk): the chunk-local pieces make chunks independent.
 template <typename T>
 __global__ void __launch_bounds__(DTW * 32) bwd_dt_kernel(BwdParams bp) {
     __shared__ float spre[DTW][256];  // exclusive prefix of m + colw - roww over the chunk
@@ -547,69 +548,66 @@ __global__ void __launch_bounds__(DTW * 32) bwd_dt_kernel(BwdParams bp) {
     const int64_t H = p.nheads, L = p.seqlen, Q = p.chunk, nc = p.nchunks;
     const int RB = bp.rblk, NB = static_cast<int>(Q / RB);
     const int wi = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t w = static_cast<int64_t>(blockIdx.x) * DTW + wi;
-    if (w >= p.batch * H) return;
-    const int64_t b = w / H, h = w % H;
-    const float* xd = bp.xdxs + w * L;
-    const float* yx = bp.dyx + w * L;
-    const float* mt = bp.mterm + w * L;
-    const float* qt = bp.qterm + w * L;
-    const float* cw = bp.colw + w * L;
-    const float* rw = bp.roww + w * NB * L;
-    const float* dtw = p.dt + w * nc * Q;
+    const int64_t w = static_cast<int64_t>(blockIdx.x) * DTW + wi;  // (b * H + h) * nc + c
+    if (w >= p.batch * H * nc) return;
+    const int64_t bh = w / nc, c = w % nc, b = bh / H, h = bh % H;
+    const float* xd = bp.xdxs + bh * L;
+    const float* yx = bp.dyx + bh * L;
+    const float* mt = bp.mterm + bh * L;
+    const float* qt = bp.qterm + bh * L;
+    const float* cw = bp.colw + bh * L;
+    const float* rw = bp.roww + bh * NB * L;
+    const float* dtw = p.dt + bh * nc * Q;
     const float Ah = p.A[h], bias = p.dt_bias ? p.dt_bias[h] : 0.0f;
     const T* dtr = static_cast<const T*>(p.dt_raw);
     T* ddt = static_cast<T*>(bp.ddt);
     float* pre = spre[wi];
     float sA = 0.0f, sD = 0.0f, sb = 0.0f;
-    for (int64_t c = 0; c < nc; ++c) {
-        const int64_t t0 = c * Q;
-        const int Lc = static_cast<int>((L - t0 < Q) ? (L - t0) : Q);
-        float carry = 0.0f;
-        for (int l0 = 0; l0 < Lc; l0 += 32) {
-            const int l = l0 + lane;
-            float v = 0.0f;
-            if (l < Lc) {
-                const int64_t t = t0 + l;
-                float rsum = 0.0f;
-                for (int i = 0; i <= l / RB; ++i) rsum += rw[i * L + t];
-                v = mt[t] + cw[t] - rsum;
-            }
-            float incl = v;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const float o = __shfl_up_sync(0xffffffffu, incl, off);
-                if (lane >= off) incl += o;
-            }
-            if (l < Lc) pre[l] = carry + incl - v;
-            carry += __shfl_sync(0xffffffffu, incl, 31);
-        }
-        __syncwarp();
-        const float k4 = bp.k4[w * nc + c];
-        carry = 0.0f;
-        for (int l0 = ((Lc - 1) / 32) * 32; l0 >= 0; l0 -= 32) {
-            const int l = l0 + lane;
+    const int64_t t0 = c * Q;
+    const int Lc = static_cast<int>((L - t0 < Q) ? (L - t0) : Q);
+    float carry = 0.0f;
+    for (int l0 = 0; l0 < Lc; l0 += 32) {
+        const int l = l0 + lane;
+        float v = 0.0f;
+        if (l < Lc) {
             const int64_t t = t0 + l;
-            float v = (l < Lc) ? qt[t] : 0.0f;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const float o = __shfl_down_sync(0xffffffffu, v, off);
-                if (lane + off < 32) v += o;
-            }
-            if (l < Lc) {
-                const float da = k4 + carry + v + pre[l];
-                const float dtv = dtw[c * Q + l];
-                const float ddtv = fmaf(Ah, da, xd[t]);
-                const float u = to_f32(dtr[(b * L + t) * H + h]) + bias;
-                const float dr = ddtv / (1.0f + expf(-u));
-                ddt[(b * L + t) * H + h] = from_f32<T>(dr);
-                sA = fmaf(dtv, da, sA);
-                sD += yx[t];
-                sb += dr;
-            }
-            carry += __shfl_sync(0xffffffffu, v, 0);
+            float rsum = 0.0f;
+            for (int i = 0; i <= l / RB; ++i) rsum += rw[i * L + t];
+            v = mt[t] + cw[t] - rsum;
         }
-        __syncwarp();
+        float incl = v;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float o = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += o;
+        }
+        if (l < Lc) pre[l] = carry + incl - v;
+        carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    __syncwarp();
+    const float k4 = bp.k4[w];
+    carry = 0.0f;
+    for (int l0 = ((Lc - 1) / 32) * 32; l0 >= 0; l0 -= 32) {
+        const int l = l0 + lane;
+        const int64_t t = t0 + l;
+        float v = (l < Lc) ? qt[t] : 0.0f;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float o = __shfl_down_sync(0xffffffffu, v, off);
+            if (lane + off < 32) v += o;
+        }
+        if (l < Lc) {
+            const float da = k4 + carry + v + pre[l];
+            const float dtv = dtw[c * Q + l];
+            const float ddtv = fmaf(Ah, da, xd[t]);
+            const float u = to_f32(dtr[(b * L + t) * H + h]) + bias;
+            const float dr = ddtv / (1.0f + expf(-u));
+            ddt[(b * L + t) * H + h] = from_f32<T>(dr);
+            sA = fmaf(dtv, da, sA);
+            sD += yx[t];
+            sb += dr;
+        }
+        carry += __shfl_sync(0xffffffffu, v, 0);
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) {
@@ -633,11 +631,14 @@ __global__ void __launch_bounds__(256) bwd_finish_kernel(BwdParams bp) {
     const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (i < H) {
         float sA = 0.0f, sD = 0.0f, sb = 0.0f;
-        for (int64_t b = 0; b < p.batch; ++b) {
-            sA += bp.partial[(b * H + i) * 3 + 0];
-            sD += bp.partial[(b * H + i) * 3 + 1];
-            sb += bp.partial[(b * H + i) * 3 + 2];
-        }
+        const int64_t nc = p.nchunks;
+        for (int64_t b = 0; b < p.batch; ++b)
+            for (int64_t c = 0; c < nc; ++c) {
+                const float* pp = bp.partial + ((b * H + i) * nc + c) * 3;
+                sA += pp[0];
+                sD += pp[1];
+                sb += pp[2];
+            }
         bp.dA[i] = sA;
         if (bp.dD) bp.dD[i] = sD;
         if (bp.ddt_bias) bp.ddt_bias[i] = sb;
@@ -701,7 +702,7 @@ cudaError_t launch_ssd_bwd(const BwdParams& bp, cudaStream_t s) {
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     {
-        const int64_t warps = p.batch * H;
+        const int64_t warps = p.batch * H * nc;
         bwd_dt_kernel<T><<<static_cast<unsigned>((warps + DTW - 1) / DTW), DTW * 32, 0, s>>>(bp);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }

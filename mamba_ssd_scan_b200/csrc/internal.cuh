@@ -65,7 +65,7 @@ struct BwdParams {
     float* roww;             // [b, H, Q/rblk, L]: per source block of rblk tokens, sum over earlier r of W[t, r]
     int32_t rblk;            // tokens per source block of roww (64: CUDA-core kernels, 128: tensor cores)
     float* k4;               // [b, H, nc]: e^{cumA_c[last]} <dH_c, H_c>
-    float* partial;          // [b, H, 3]: per-row sums of dt*da, dy.x, ddt_raw
+    float* partial;          // [b, H, nc, 3]: per-chunk sums of dt*da, dy.x, ddt_raw
 };
 
 // The diagonal-A selective scan (forward and decode step).
