@@ -35,17 +35,28 @@ constexpr int BLK = R * 128;        // bytes of one 64-column SW128 block of a 1
 constexpr int TPB = 128;            // threads per CTA
 constexpr float kLog2eB = 1.4426950408889634f;
 
+// 16 bytes global -> shared without passing through registers; src_bytes 0
+// writes zeros (the source is not read)
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
 // rows [r0, r0 + R) x 64-column blocks of a bf16 matrix (row stride `stride`
-// elements, `ncol` columns) into SW128 blocks at dst; rows at or past `lim`
-// are zero
+// elements, `ncol` columns) into SW128 blocks at dst with asynchronous copies
+// (all in flight together); rows at or past `lim` are zero.  The caller waits
+// (cp_async_wait_all) before the barrier that publishes the tile.
 __device__ __forceinline__ void stage_tile(uint32_t dst, const __nv_bfloat16* src, int64_t stride,
                                            int ncol, int r0, int lim, int rows = R) {
     const int chunks = rows * (ncol / 8);  // 16-byte chunks
     for (int i = threadIdx.x; i < chunks; i += TPB) {
         const int r = i / (ncol / 8), c = i % (ncol / 8);
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (r0 + r < lim) v = ldg16(src + static_cast<int64_t>(r0 + r) * stride + c * 8);
-        st_shared_v4(dst + (c >> 3) * (rows * 128) + sw128(r, c & 7), v.x, v.y, v.z, v.w);
+        const bool ok = r0 + r < lim;
+        const __nv_bfloat16* g = src + static_cast<int64_t>(ok ? r0 + r : r0) * stride + c * 8;
+        cp_async16(dst + (c >> 3) * (rows * 128) + sw128(r, c & 7), g, ok ? 16u : 0u);
     }
 }
 
@@ -134,6 +145,7 @@ __global__ void __launch_bounds__(TPB, 1) bwd_tc_a_kernel(BwdParams bp) {
     }
     stage_tile(sB, Bb, bs, NST, s0, Lc);
     stage_tile(sX, xb, xs, PD, s0, Lc);
+    cp_async_wait_all();
     fence_smem_async();
     fence_before_sync();
     __syncthreads();
@@ -152,6 +164,7 @@ __global__ void __launch_bounds__(TPB, 1) bwd_tc_a_kernel(BwdParams bp) {
         if (r0 >= Lc) break;
         stage_tile(sC, Cb, bs, NST, r0, Lc);
         stage_tile(sY, dyb, xs, PD, r0, Lc);
+        cp_async_wait_all();
         fence_smem_async();
         fence_before_sync();
         __syncthreads();
@@ -446,6 +459,7 @@ __global__ void __launch_bounds__(TPB) bwd_tc_b_kernel(BwdParams bp) {
         const int s0 = is * R;
         stage_tile(sX, xb, xs, PD, s0, Lc);
         stage_tile(sB, Bb, bs, NST, s0, Lc);
+        cp_async_wait_all();
         fence_smem_async();
         fence_before_sync();
         __syncthreads();
@@ -508,6 +522,7 @@ __global__ void __launch_bounds__(TPB) bwd_tc_b_kernel(BwdParams bp) {
     if (!failed) {
         // the H_c term e^{cumA_t} dy_t H_c: A = dy_t (K-major, K = p), B = H_c (MN-major, N = n)
         stage_tile(sH, Hg, NST, NST, 0, PD, PD);
+        cp_async_wait_all();
         fence_smem_async();
         fence_before_sync();
         __syncthreads();
