@@ -32,7 +32,7 @@ using namespace tc;
 
 constexpr int R = 128;              // rows of a tile (tokens)
 constexpr int BLK = R * 128;        // bytes of one 64-column SW128 block of a 128-row tile
-constexpr int TPB = 128;            // threads per CTA
+constexpr int TPB = 256;            // threads per CTA: two warps per TMEM lane quarter
 constexpr float kLog2eB = 1.4426950408889634f;
 
 // 16 bytes global -> shared without passing through registers; src_bytes 0
@@ -91,7 +91,8 @@ struct ATile {
     static constexpr int DH_OFF = T2_OFF;              // after the loop: dH = hi + lo, bf16 [p][n] each
     static constexpr int COL_OFF = T2_OFF + 2 * BLK;   // [4][R] column sums of W
     static constexpr int CS_OFF = COL_OFF + 4 * R * 4;       // [256] cumA, then [256] dt
-    static constexpr int BAR_OFF = CS_OFF + 2 * 256 * 4;
+    static constexpr int ROW_OFF = CS_OFF + 2 * 256 * 4;     // [2][R] the halves' row sums of W
+    static constexpr int BAR_OFF = ROW_OFF + 2 * R * 4;
     static constexpr int BYTES = BAR_OFF + 64 + 1024;        // + alignment slack
     static_assert(2 * NBN * 64 * 128 <= 2 * BLK, "dH hi + lo must fit in the T2 tile");
     static_assert(BYTES <= 232448, "kernel A's shared memory exceeds 227 KB");
@@ -121,9 +122,11 @@ __global__ void __launch_bounds__(TPB, 1) bwd_tc_a_kernel(BwdParams bp) {
     float* scol = reinterpret_cast<float*>(smem + T::COL_OFF);
     float* scs = reinterpret_cast<float*>(smem + T::CS_OFF);
     float* sdt = scs + 256;
+    float* srow = reinterpret_cast<float*>(smem + T::ROW_OFF);
     uint64_t* bar = reinterpret_cast<uint64_t*>(smem + T::BAR_OFF);
     uint32_t* tslot = reinterpret_cast<uint32_t*>(bar + 1);
     volatile int* abort = reinterpret_cast<volatile int*>(tslot + 1);
+    const int quarter = warp & 3, half = warp >> 2;  // TMEM lanes 32 quarter.., column half
 
     const int64_t xs = H * PD, bs = G * NST;
     const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(p.x) + ((b * L + t0) * H + h) * PD;
@@ -151,12 +154,12 @@ __global__ void __launch_bounds__(TPB, 1) bwd_tc_a_kernel(BwdParams bp) {
     __syncthreads();
     fence_after_sync();
     const uint32_t tmem = *tslot;
-    const uint32_t lane_off = static_cast<uint32_t>(32 * warp) << 16;
+    const uint32_t lane_off = static_cast<uint32_t>(32 * quarter) << 16;
     const uint32_t T1A = tmem, T2A = tmem + 128, DXS = tmem + 256, DBA = tmem + 320;
     const uint32_t mbar = smem_u32(bar);
     uint32_t ph = 0;
     bool failed = false;
-    float colacc = 0.0f;  // thread tid: column (source token) s0 + tid
+    float colacc = 0.0f;  // thread tid < R: column (source token) s0 + tid
     const int64_t tok = (b * H + h) * L + t0;
 
     for (int it = is; it < NTT; ++it) {
@@ -189,12 +192,12 @@ __global__ void __launch_bounds__(TPB, 1) bwd_tc_a_kernel(BwdParams bp) {
             break;
         }
         fence_after_sync();
-        // row t of the scores: mask, decay, W sums, bf16 tiles
-        const int row = 32 * warp + lane, tl = r0 + row;
+        // row t of the scores, this warp's column half: mask, decay, W sums, bf16 tiles
+        const int row = 32 * quarter + lane, tl = r0 + row;
         const float cst = scs[tl];
         float rowp = 0.0f;
 #pragma unroll 1
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 2 * half; q < 2 * half + 2; ++q) {
             float v1[32], v2[32], wv[32];
             tmem_ld32x2(T1A + lane_off + q * 32, v1, T2A + lane_off + q * 32, v2);
 #pragma unroll
@@ -228,14 +231,17 @@ __global__ void __launch_bounds__(TPB, 1) bwd_tc_a_kernel(BwdParams bp) {
                              pack_bf16x2(v2[8 * cc + 4], v2[8 * cc + 5]),
                              pack_bf16x2(v2[8 * cc + 6], v2[8 * cc + 7]));
             }
-            scol[warp * R + q * 32 + lane] = transpose_reduce32(wv, lane);
+            scol[quarter * R + q * 32 + lane] = transpose_reduce32(wv, lane);
         }
-        if (tl < Lc) bp.roww[((b * H + h) * NTT + is) * L + t0 + tl] = rowp;
+        srow[half * R + row] = rowp;
         fence_smem_async();
         fence_before_sync();
         __syncthreads();
         fence_after_sync();
-        colacc += (scol[tid] + scol[R + tid]) + (scol[2 * R + tid] + scol[3 * R + tid]);
+        if (tid < R) {
+            colacc += (scol[tid] + scol[R + tid]) + (scol[2 * R + tid] + scol[3 * R + tid]);
+            if (r0 + tid < Lc) bp.roww[((b * H + h) * NTT + is) * L + t0 + r0 + tid] = srow[tid] + srow[R + tid];
+        }
         if (tid == 0) {
             // dxs += T1^T dy_t, dB += T2^T C_t: K = the target tile's 128 tokens
 #pragma unroll
@@ -305,79 +311,83 @@ __global__ void __launch_bounds__(TPB, 1) bwd_tc_a_kernel(BwdParams bp) {
         fence_after_sync();
     }
     if (!failed) {
-        // outputs of the source row s
-        const int row = tid, sl = s0 + row;
+        // outputs of the source row s: dx and its per-token pieces in the low
+        // half of the warps, dB in the high half
+        const int row = 32 * quarter + lane, sl = s0 + row;
         const bool valid = sl < Lc;
         const float dts = valid ? sdt[sl] : 0.0f;
         const float wsr = valid ? ex2((scs[Q - 1] - scs[sl]) * kLog2eB) : 0.0f;
-        const float Dh = p.D ? p.D[h] : 0.0f;
-        float xv[PD], dyv[PD];
+        if (half == 0) {
+            const float Dh = p.D ? p.D[h] : 0.0f;
+            float xv[PD], dyv[PD];
 #pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
-            const uint4 v = ld_shared_v4(sX + sw128(row, cc));
-            const uint4 u = valid ? ldg16(dyb + static_cast<int64_t>(sl) * xs + cc * 8)
-                                  : make_uint4(0u, 0u, 0u, 0u);
-            const uint32_t vw[4] = {v.x, v.y, v.z, v.w}, uw[4] = {u.x, u.y, u.z, u.w};
+            for (int cc = 0; cc < 8; ++cc) {
+                const uint4 v = ld_shared_v4(sX + sw128(row, cc));
+                const uint4 u = valid ? ldg16(dyb + static_cast<int64_t>(sl) * xs + cc * 8)
+                                      : make_uint4(0u, 0u, 0u, 0u);
+                const uint32_t vw[4] = {v.x, v.y, v.z, v.w}, uw[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                xv[cc * 8 + 2 * e] = __uint_as_float(vw[e] << 16);
-                xv[cc * 8 + 2 * e + 1] = __uint_as_float(vw[e] & 0xffff0000u);
-                dyv[cc * 8 + 2 * e] = __uint_as_float(uw[e] << 16);
-                dyv[cc * 8 + 2 * e + 1] = __uint_as_float(uw[e] & 0xffff0000u);
+                for (int e = 0; e < 4; ++e) {
+                    xv[cc * 8 + 2 * e] = __uint_as_float(vw[e] << 16);
+                    xv[cc * 8 + 2 * e + 1] = __uint_as_float(vw[e] & 0xffff0000u);
+                    dyv[cc * 8 + 2 * e] = __uint_as_float(uw[e] << 16);
+                    dyv[cc * 8 + 2 * e + 1] = __uint_as_float(uw[e] & 0xffff0000u);
+                }
             }
-        }
-        float pxd = 0.0f, pm = 0.0f, pyx = 0.0f;
-        __nv_bfloat16* dxo = static_cast<__nv_bfloat16*>(bp.dx) + ((b * L + t0) * H + h) * PD;
+            float pxd = 0.0f, pm = 0.0f, pyx = 0.0f;
+            __nv_bfloat16* dxo = static_cast<__nv_bfloat16*>(bp.dx) + ((b * L + t0) * H + h) * PD;
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            float vi[32], vs[32];
-            tmem_ld32x2(DXS + lane_off + half * 32, vi, T1A + lane_off + half * 32, vs);
-            uint32_t o[16];
+            for (int hp = 0; hp < 2; ++hp) {
+                float vi[32], vs[32];
+                tmem_ld32x2(DXS + lane_off + hp * 32, vi, T1A + lane_off + hp * 32, vs);
+                uint32_t o[16];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const int pp = half * 32 + j;
-                const float st = wsr * vs[j];
-                const float d = vi[j] + st;
-                pxd = fmaf(xv[pp], d, pxd);
-                pm = fmaf(xv[pp], st, pm);
-                pyx = fmaf(dyv[pp], xv[pp], pyx);
-                const float dxv = fmaf(dts, d, Dh * dyv[pp]);
-                if (j & 1) o[j >> 1] |= pack_bf16x2(0.0f, dxv) & 0xffff0000u;
-                else o[j >> 1] = pack_bf16x2(dxv, 0.0f) & 0x0000ffffu;
+                for (int j = 0; j < 32; j += 2) {
+                    const int pp = hp * 32 + j;
+                    const float st0 = wsr * vs[j], st1 = wsr * vs[j + 1];
+                    const float d0 = vi[j] + st0, d1 = vi[j + 1] + st1;
+                    pxd = fmaf(xv[pp], d0, fmaf(xv[pp + 1], d1, pxd));
+                    pm = fmaf(xv[pp], st0, fmaf(xv[pp + 1], st1, pm));
+                    pyx = fmaf(dyv[pp], xv[pp], fmaf(dyv[pp + 1], xv[pp + 1], pyx));
+                    o[j >> 1] = pack_bf16x2(fmaf(dts, d0, Dh * dyv[pp]), fmaf(dts, d1, Dh * dyv[pp + 1]));
+                }
+                if (valid) {
+                    uint4* dst = reinterpret_cast<uint4*>(dxo + static_cast<int64_t>(sl) * xs + hp * 32);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        dst[k] = make_uint4(o[4 * k], o[4 * k + 1], o[4 * k + 2], o[4 * k + 3]);
+                }
             }
             if (valid) {
-                uint4* dst = reinterpret_cast<uint4*>(dxo + static_cast<int64_t>(sl) * xs + half * 32);
-#pragma unroll
-                for (int k = 0; k < 4; ++k) dst[k] = make_uint4(o[4 * k], o[4 * k + 1], o[4 * k + 2], o[4 * k + 3]);
+                bp.xdxs[tok + sl] = pxd;
+                bp.dyx[tok + sl] = pyx;
+                bp.mterm[tok + sl] = dts * pm;
+                bp.colw[tok + sl] = colacc;  // row == tid in this half
             }
-        }
-        if (valid) {
-            bp.xdxs[tok + sl] = pxd;
-            bp.dyx[tok + sl] = pyx;
-            bp.mterm[tok + sl] = dts * pm;
-            bp.colw[tok + sl] = colacc;
-        }
+        } else {
 #pragma unroll
-        for (int q = 0; q < NST / 32; ++q) {
-            float vi[32], vs[32];
-            tmem_ld32x2(DBA + lane_off + q * 32, vi, T2A + lane_off + q * 32, vs);
-            if (valid) {
-                if (bp.dB_h) {
-                    float* dst = bp.dB_h + ((b * L + t0 + sl) * H + h) * NST + q * 32;
+            for (int q = 0; q < NST / 32; ++q) {
+                float vi[32], vs[32];
+                tmem_ld32x2(DBA + lane_off + q * 32, vi, T2A + lane_off + q * 32, vs);
+                if (valid) {
+                    if (bp.dB_h) {
+                        float* dst = bp.dB_h + ((b * L + t0 + sl) * H + h) * NST + q * 32;
 #pragma unroll
-                    for (int j = 0; j < 32; j += 4)
-                        *reinterpret_cast<float4*>(dst + j) =
-                            make_float4(dts * fmaf(wsr, vs[j], vi[j]), dts * fmaf(wsr, vs[j + 1], vi[j + 1]),
-                                        dts * fmaf(wsr, vs[j + 2], vi[j + 2]), dts * fmaf(wsr, vs[j + 3], vi[j + 3]));
-                } else {
-                    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(bp.dB) + ((b * L + t0 + sl) * G + g) * NST + q * 32;
+                        for (int j = 0; j < 32; j += 4)
+                            *reinterpret_cast<float4*>(dst + j) = make_float4(
+                                dts * fmaf(wsr, vs[j], vi[j]), dts * fmaf(wsr, vs[j + 1], vi[j + 1]),
+                                dts * fmaf(wsr, vs[j + 2], vi[j + 2]), dts * fmaf(wsr, vs[j + 3], vi[j + 3]));
+                    } else {
+                        __nv_bfloat16* dst =
+                            static_cast<__nv_bfloat16*>(bp.dB) + ((b * L + t0 + sl) * G + g) * NST + q * 32;
 #pragma unroll
-                    for (int j = 0; j < 32; j += 8)
-                        *reinterpret_cast<uint4*>(dst + j) = make_uint4(
-                            pack_bf16x2(dts * fmaf(wsr, vs[j], vi[j]), dts * fmaf(wsr, vs[j + 1], vi[j + 1])),
-                            pack_bf16x2(dts * fmaf(wsr, vs[j + 2], vi[j + 2]), dts * fmaf(wsr, vs[j + 3], vi[j + 3])),
-                            pack_bf16x2(dts * fmaf(wsr, vs[j + 4], vi[j + 4]), dts * fmaf(wsr, vs[j + 5], vi[j + 5])),
-                            pack_bf16x2(dts * fmaf(wsr, vs[j + 6], vi[j + 6]), dts * fmaf(wsr, vs[j + 7], vi[j + 7])));
+                        for (int j = 0; j < 32; j += 8)
+                            *reinterpret_cast<uint4*>(dst + j) = make_uint4(
+                                pack_bf16x2(dts * fmaf(wsr, vs[j], vi[j]), dts * fmaf(wsr, vs[j + 1], vi[j + 1])),
+                                pack_bf16x2(dts * fmaf(wsr, vs[j + 2], vi[j + 2]), dts * fmaf(wsr, vs[j + 3], vi[j + 3])),
+                                pack_bf16x2(dts * fmaf(wsr, vs[j + 4], vi[j + 4]), dts * fmaf(wsr, vs[j + 5], vi[j + 5])),
+                                pack_bf16x2(dts * fmaf(wsr, vs[j + 6], vi[j + 6]), dts * fmaf(wsr, vs[j + 7], vi[j + 7])));
+                    }
                 }
             }
         }
@@ -400,7 +410,8 @@ struct BTile {
     static constexpr int T_OFF = B_OFF + NBN * BLK;    // masked, decayed, dt-scaled dy_t . x_s, bf16 [t][s]
     static constexpr int H_OFF = T_OFF + 2 * BLK;      // H_c, bf16 [p][n]
     static constexpr int CS_OFF = H_OFF + NBN * 64 * 128;
-    static constexpr int BAR_OFF = CS_OFF + 2 * 256 * 4;
+    static constexpr int SQ_OFF = CS_OFF + 2 * 256 * 4;  // [2][R] the halves' q partials, then [8] sums
+    static constexpr int BAR_OFF = SQ_OFF + (2 * R + 8) * 4;
     static constexpr int BYTES = BAR_OFF + 64 + 1024;
 };
 
@@ -428,7 +439,9 @@ __global__ void __launch_bounds__(TPB) bwd_tc_b_kernel(BwdParams bp) {
     uint64_t* bar = reinterpret_cast<uint64_t*>(smem + T::BAR_OFF);
     uint32_t* tslot = reinterpret_cast<uint32_t*>(bar + 1);
     volatile int* abort = reinterpret_cast<volatile int*>(tslot + 1);
-    float* wsum = reinterpret_cast<float*>(tslot + 2);  // [4]
+    float* sq = reinterpret_cast<float*>(smem + T::SQ_OFF);
+    float* wsum = sq + 2 * R;  // [8]
+    const int quarter = warp & 3, half = warp >> 2;
 
     const int64_t xs = H * PD, bs = G * NST;
     const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(p.x) + ((b * L + t0) * H + h) * PD;
@@ -453,8 +466,8 @@ __global__ void __launch_bounds__(TPB) bwd_tc_b_kernel(BwdParams bp) {
     uint32_t ph = 0;
     bool failed = false;
     uint32_t tmem = 0;
-    const uint32_t lane_off = static_cast<uint32_t>(32 * warp) << 16;
-    const int row = tid, tl = r0 + row;
+    const uint32_t lane_off = static_cast<uint32_t>(32 * quarter) << 16;
+    const int row = 32 * quarter + lane, tl = r0 + row;
     for (int is = 0; is <= it; ++is) {
         const int s0 = is * R;
         stage_tile(sX, xb, xs, PD, s0, Lc);
@@ -481,7 +494,7 @@ __global__ void __launch_bounds__(TPB) bwd_tc_b_kernel(BwdParams bp) {
         fence_after_sync();
         const float cst = scs[tl];
 #pragma unroll 1
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 2 * half; q < 2 * half + 2; ++q) {
             float v[32];
             tmem_ld32(tmem + lane_off + q * 32, v);
 #pragma unroll
@@ -543,7 +556,7 @@ __global__ void __launch_bounds__(TPB) bwd_tc_b_kernel(BwdParams bp) {
         const float wt = valid ? ex2(scs[tl] * kLog2eB) : 0.0f;
         float pq = 0.0f;
 #pragma unroll
-        for (int q = 0; q < NST / 32; ++q) {
+        for (int q = half * (NST / 64); q < (half + 1) * (NST / 64); ++q) {
             float vi[32], vs[32];
             tmem_ld32x2(tmem + 128 + lane_off + q * 32, vi, tmem + lane_off + q * 32, vs);
             if (valid) {
@@ -579,7 +592,9 @@ __global__ void __launch_bounds__(TPB) bwd_tc_b_kernel(BwdParams bp) {
                 }
             }
         }
-        if (valid) bp.qterm[(b * H + h) * L + t0 + tl] = pq;
+        sq[half * R + row] = pq;
+        __syncthreads();
+        if (half == 0 && valid) bp.qterm[(b * H + h) * L + t0 + tl] = sq[row] + sq[R + row];
         if (it == 0) {
             // e^{cumA_last} <dH_c, H_c>, reduced in a fixed order
             const float* dHg = bp.dstates + ((b * nc + c) * H + h) * static_cast<int64_t>(PD) * NST;
@@ -590,7 +605,9 @@ __global__ void __launch_bounds__(TPB) bwd_tc_b_kernel(BwdParams bp) {
             if (lane == 0) wsum[warp] = v;
             __syncthreads();
             if (tid == 0)
-                bp.k4[(b * H + h) * nc + c] = ex2(scs[Q - 1] * kLog2eB) * ((wsum[0] + wsum[1]) + (wsum[2] + wsum[3]));
+                bp.k4[(b * H + h) * nc + c] = ex2(scs[Q - 1] * kLog2eB) *
+                                              (((wsum[0] + wsum[1]) + (wsum[2] + wsum[3])) +
+                                               ((wsum[4] + wsum[5]) + (wsum[6] + wsum[7])));
         }
     }
     fence_before_sync();
