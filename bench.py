@@ -246,7 +246,7 @@ def main_ours(args):
         if args.conv_only:
             res = conv_workloads(ssd, synthetic, dev, flush, peaks, rank, world, ranks_max)
         elif args.bwd_only:
-            res = bwd_workloads(ssd, synthetic, dev, flush, rank, world, ranks_max)
+            res = bwd_workloads(ssd, synthetic, dev, flush, peaks, rank, world, ranks_max)
         else:
             res = sel_workloads(ssd, synthetic, dev, flush, peaks, rank, world, ranks_max)
         if rank == 0:
@@ -659,7 +659,7 @@ def other_workloads(ssd, synthetic, dev, flush, peaks, rank, world, barrier, ran
     del g, state, steps_in
     torch.cuda.empty_cache()
     out.update(conv_workloads(ssd, synthetic, dev, flush, peaks, rank, world, ranks_max))
-    out.update(bwd_workloads(ssd, synthetic, dev, flush, rank, world, ranks_max))
+    out.update(bwd_workloads(ssd, synthetic, dev, flush, peaks, rank, world, ranks_max))
     out.update(sel_workloads(ssd, synthetic, dev, flush, peaks, rank, world, ranks_max))
     return out
 
@@ -779,7 +779,7 @@ def bwd_flops(cfg):
     return 2.0 * per * nc * cfg.nheads * cfg.batch
 
 
-def bwd_workloads(ssd, synthetic, dev, flush, rank, world, ranks_max, steps=5):
+def bwd_workloads(ssd, synthetic, dev, flush, peaks, rank, world, ranks_max, steps=5):
     """The backward pass (forward recompute included) on two forward
     workloads' shapes, with an initial state and d_final, L2 flushed before
     each call."""
@@ -821,10 +821,20 @@ def bwd_workloads(ssd, synthetic, dev, flush, rank, world, ranks_max, steps=5):
         torch.cuda.synchronize()
         ms = ranks_max(sum(a.elapsed_time(b_) for a, b_ in evs) / steps)
         fl = bwd_flops(cfg)
-        out["bwd_" + name] = {"tokens_per_s": job_throughput(cfg.tokens, world, ms), "ms": ms,
-                              "tflops": fl / (ms * 1e-3) / 1e12, "flop": fl,
-                              "fp32_fma_frac": fl / (ms * 1e-3) / 1e12 / FP32_FMA_TFLOPS,
-                              "bound": "alu", "l2": "flushed"}
+        tf = fl / (ms * 1e-3) / 1e12
+        # bf16 shapes in range run the per-chunk products on the tensor cores:
+        # their roofline is the bf16 tensor peak; the CUDA-core path's is the
+        # fp32 FMA peak
+        on_tc = (cfg.dtype == torch.bfloat16 and cfg.headdim == 64 and cfg.dstate in (64, 128)
+                 and cfg.chunk in (128, 256))
+        line = {"tokens_per_s": job_throughput(cfg.tokens, world, ms), "ms": ms, "tflops": tf,
+                "flop": fl, "l2": "flushed"}
+        if on_tc:
+            line.update(bound="tensor", peak_tflops=peaks["bf16_tflops"],
+                        tensor_frac=tf / peaks["bf16_tflops"])
+        else:
+            line.update(bound="alu", peak_tflops=FP32_FMA_TFLOPS, fp32_fma_frac=tf / FP32_FMA_TFLOPS)
+        out["bwd_" + name] = line
         del d, dy, dfin, ws, res
         torch.cuda.empty_cache()
     return out
