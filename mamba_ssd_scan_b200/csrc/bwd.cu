@@ -34,6 +34,7 @@
 // rows and over the heads of a group in a fixed order (no atomics: the result
 // is bitwise reproducible).
 #include "internal.cuh"
+#include "bwd_tc.h"
 
 namespace ssd {
 namespace {
@@ -672,7 +673,9 @@ cudaError_t launch_ssd_bwd(const BwdParams& bp, cudaStream_t s) {
     const FwdParams& p = bp.f;
     const int64_t H = p.nheads, P = p.headdim, N = p.dstate, nc = p.nchunks;
     cudaError_t e;
-    {
+    if (bp.rblk == 128) {
+        if ((e = launch_bwd_tc_dstate(bp, s)) != cudaSuccess) return e;
+    } else {
         const unsigned tiles = static_cast<unsigned>(((P + DP - 1) / DP) * ((N + DN - 1) / DN));
         dim3 grid(static_cast<unsigned>(nc * H), tiles, static_cast<unsigned>(p.batch));
         bwd_dstate_kernel<T><<<grid, 256, 0, s>>>(bp);

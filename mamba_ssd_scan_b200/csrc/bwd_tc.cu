@@ -23,6 +23,7 @@
 // the masked T tiles are written back as bf16 in the same layout.  All waits
 // are bounded; a timed-out wait stops the CTA and sets the call's status word.
 #include "internal.cuh"
+#include "bwd_tc.h"
 #include "tcgen05.cuh"
 
 namespace ssd {
@@ -619,6 +620,144 @@ __global__ void __launch_bounds__(TPB) bwd_tc_b_kernel(BwdParams bp) {
     if (failed && tid == 0 && p.status) atomicExch(p.status, static_cast<int>(SSD_ERR_TIMEOUT));
 }
 
+// The chunk-local adjoint dS_c = sum_t e^{cumA_t} dy_t C_t^T, as its transpose
+// dS^T[n][p] (M = the state index, zero-padded to 128 rows when dstate is 64;
+// K = the chunk's tokens; N = headdim) so that the A operand is C scaled per
+// token: e^{cumA_t} C_t enters as bf16 hi + lo (the scaling is not rounded to
+// 8 bits), dy_t as staged.  One CTA per (b, c, h); fp32 out, [p][n].
+template <int NST>
+struct DTile {
+    static constexpr int Y_OFF = 0;                  // dy_t, bf16 [t][p]
+    static constexpr int AH_OFF = Y_OFF + BLK;       // e^{cumA_t} C_t, hi: 2 blocks of 64 states
+    static constexpr int AL_OFF = AH_OFF + 2 * BLK;  // lo
+    static constexpr int CS_OFF = AL_OFF + 2 * BLK;
+    static constexpr int BAR_OFF = CS_OFF + 256 * 4;
+    static constexpr int BYTES = BAR_OFF + 64 + 1024;
+};
+
+template <int NST>
+__global__ void __launch_bounds__(TPB) bwd_tc_ds_kernel(BwdParams bp) {
+    using T = DTile<NST>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const FwdParams& p = bp.f;
+    const int64_t H = p.nheads, G = p.ngroups, L = p.seqlen, Q = p.chunk, nc = p.nchunks;
+    const int NTT = static_cast<int>(Q / R);
+    const int64_t h = blockIdx.x, c = blockIdx.y, b = blockIdx.z, g = h / p.heads_per_group;
+    const int64_t t0 = c * Q;
+    const int Lc = static_cast<int>((L - t0 < Q) ? (L - t0) : Q);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quarter = warp & 3, half = warp >> 2;
+    const uint32_t base = smem_u32(smem);
+    const uint32_t sY = base + T::Y_OFF, sAh = base + T::AH_OFF, sAl = base + T::AL_OFF;
+    float* scs = reinterpret_cast<float*>(smem + T::CS_OFF);
+    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + T::BAR_OFF);
+    uint32_t* tslot = reinterpret_cast<uint32_t*>(bar + 1);
+    volatile int* abort = reinterpret_cast<volatile int*>(tslot + 1);
+    const int64_t xs = H * PD, bs = G * NST;
+    const __nv_bfloat16* dyb = static_cast<const __nv_bfloat16*>(bp.dy) + ((b * L + t0) * H + h) * PD;
+    const __nv_bfloat16* Cb = static_cast<const __nv_bfloat16*>(p.C) + ((b * L + t0) * G + g) * NST;
+    const float* csc = p.cumA + ((b * H + h) * nc + c) * Q;
+
+    if (warp == 0) tmem_alloc(smem_u32(tslot), 64);
+    if (tid == 0) {
+        mbar_init(smem_u32(bar), 1);
+        *abort = 0;
+        fence_mbar_init();
+    }
+    for (int i = tid; i < Q; i += TPB) scs[i] = csc[i];
+    if (NST == 64) {  // the padding states 64..127 of A stay zero
+        for (int i = tid; i < R * 8; i += TPB) {
+            st_shared_v4(sAh + BLK + sw128(i >> 3, i & 7), 0u, 0u, 0u, 0u);
+            st_shared_v4(sAl + BLK + sw128(i >> 3, i & 7), 0u, 0u, 0u, 0u);
+        }
+    }
+    __syncthreads();
+    const uint32_t tmem = *tslot;
+    const uint32_t mbar = smem_u32(bar);
+    uint32_t ph = 0;
+    bool failed = false;
+    for (int it = 0; it < NTT; ++it) {
+        const int r0 = it * R;
+        if (r0 >= Lc) break;
+        stage_tile(sY, dyb, xs, PD, r0, Lc);
+        // e^{cumA_t} C_t as hi + lo, rows t, 16-byte chunks of 8 states
+        for (int i = tid; i < R * (NST / 8); i += TPB) {
+            const int r = i / (NST / 8), cc = i % (NST / 8);
+            uint32_t hi[4] = {0u, 0u, 0u, 0u}, lo[4] = {0u, 0u, 0u, 0u};
+            if (r0 + r < Lc) {
+                const float w = ex2(scs[r0 + r] * kLog2eB);
+                const uint4 u = ldg16(Cb + static_cast<int64_t>(r0 + r) * bs + cc * 8);
+                const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float a0 = w * __uint_as_float(uw[e] << 16);
+                    const float a1 = w * __uint_as_float(uw[e] & 0xffff0000u);
+                    hi[e] = pack_bf16x2(a0, a1);
+                    lo[e] = pack_bf16x2(a0 - __uint_as_float(hi[e] << 16),
+                                        a1 - __uint_as_float(hi[e] & 0xffff0000u));
+                }
+            }
+            const uint32_t o = (cc >> 3) * BLK + sw128(r, cc & 7);
+            st_shared_v4(sAh + o, hi[0], hi[1], hi[2], hi[3]);
+            st_shared_v4(sAl + o, lo[0], lo[1], lo[2], lo[3]);
+        }
+        cp_async_wait_all();
+        fence_smem_async();
+        fence_before_sync();
+        __syncthreads();
+        fence_after_sync();
+        if (tid == 0) {
+            // dS^T += (e^{cumA} C)^T dy: A MN-major (M = state, K = t), B MN-major (N = p, K = t)
+#pragma unroll
+            for (int k = 0; k < R / 16; ++k) {
+                mma_bf16(tmem, desc_sw128(sAh + k * 2048, BLK, 1024), desc_sw128(sY + k * 2048, BLK, 1024),
+                         idesc_bf16(128, PD, true, true), (it > 0 || k > 0) ? 1u : 0u);
+                mma_bf16(tmem, desc_sw128(sAl + k * 2048, BLK, 1024), desc_sw128(sY + k * 2048, BLK, 1024),
+                         idesc_bf16(128, PD, true, true), 1u);
+            }
+            mma_commit(mbar);
+        }
+        const bool ok = wait_or_abort(mbar, ph, abort);
+        ph ^= 1u;
+        if (__syncthreads_or(!ok)) {
+            failed = true;
+            break;
+        }
+        fence_after_sync();
+    }
+    if (!failed) {
+        // lane n of the accumulator holds dS^T[n][*]; this warp's half of the 64 columns
+        const int n = 32 * quarter + lane;
+        float v[32];
+        tmem_ld32(tmem + (static_cast<uint32_t>(32 * quarter) << 16) + half * 32, v);
+        if (n < NST) {
+            float* out = bp.dstates + ((b * nc + c) * H + h) * static_cast<int64_t>(PD) * NST + n;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) out[static_cast<int64_t>(half * 32 + j) * NST] = v[j];
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        fence_after_sync();
+        tmem_dealloc(tmem, 64);
+    }
+    if (failed && tid == 0 && p.status) atomicExch(p.status, static_cast<int>(SSD_ERR_TIMEOUT));
+}
+
+template <int NST>
+cudaError_t launch_ds(const BwdParams& bp, cudaStream_t s) {
+    const FwdParams& p = bp.f;
+    const int sd = DTile<NST>::BYTES;
+    cudaError_t e = cudaFuncSetAttribute(bwd_tc_ds_kernel<NST>, cudaFuncAttributeMaxDynamicSharedMemorySize, sd);
+    if (e != cudaSuccess) return e;
+    const dim3 grid(static_cast<unsigned>(p.nheads), static_cast<unsigned>(p.nchunks),
+                    static_cast<unsigned>(p.batch));
+    bwd_tc_ds_kernel<NST><<<grid, TPB, sd, s>>>(bp);
+    return cudaGetLastError();
+}
+
 template <int NST>
 cudaError_t launch_nst(const BwdParams& bp, cudaStream_t s) {
     const FwdParams& p = bp.f;
@@ -644,6 +783,10 @@ bool bwd_tc_supported(const FwdParams& p) {
 
 cudaError_t launch_bwd_tc(const BwdParams& bp, cudaStream_t s) {
     return bp.f.dstate == 64 ? launch_nst<64>(bp, s) : launch_nst<128>(bp, s);
+}
+
+cudaError_t launch_bwd_tc_dstate(const BwdParams& bp, cudaStream_t s) {
+    return bp.f.dstate == 64 ? launch_ds<64>(bp, s) : launch_ds<128>(bp, s);
 }
 
 }  // namespace ssd
