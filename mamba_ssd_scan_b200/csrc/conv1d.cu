@@ -15,6 +15,8 @@
 // as a sliding window, compute with packed fp32x2 arithmetic, store their
 // outputs directly and release the tile on its "empty" mbarrier.  The decode
 // step keeps the same state [batch, channels, K-1] and shifts it by one token.
+#include <stdlib.h>
+
 #include "internal.cuh"
 #include "tcgen05.cuh"
 #include "tma.cuh"
@@ -89,7 +91,11 @@ __device__ __forceinline__ float xin_at(const ConvParams& p, const T* xb, int64_
 }
 
 template <typename T, int K, bool ACT>
-__global__ void __launch_bounds__(kMaxConsumers<T> + 32) conv1d_kernel(ConvParams p, int64_t seg) {
+// `withhold` >= 0 makes the producer stop before that tile (a test of the
+// bounded waits: the consumers time out, every role stops, the copies in
+// flight land and the status word reads SSD_ERR_TIMEOUT); -1 in normal use.
+__global__ void __launch_bounds__(kMaxConsumers<T> + 32)
+    conv1d_kernel(ConvParams p, int64_t seg, int withhold) {
     using namespace tc;
     constexpr int KM = K > 1 ? K - 1 : 1;
     extern __shared__ __align__(128) uint8_t smem[];
@@ -127,6 +133,7 @@ __global__ void __launch_bounds__(kMaxConsumers<T> + 32) conv1d_kernel(ConvParam
         const uint32_t sbase = smem_u32(smem);
         int j = 0;
         for (; j < ntiles; ++j) {
+            if (j == withhold) break;
             const int st = j % NSTAGE, use = j / NSTAGE;
             bool ok = true;
             if (use > 0 && lane == 0) ok = wait_or_abort(smem_u32(&empty[st]), (use - 1) & 1, &abort_flag);
@@ -357,7 +364,9 @@ cudaError_t launch_fwd(const ConvParams& p, cudaStream_t s) {
     nseg = (p.seqlen + seg - 1) / seg;
     dim3 grid(static_cast<unsigned>(nblk), static_cast<unsigned>(nseg),
               static_cast<unsigned>(p.batch));
-    conv1d_kernel<T, K, ACT><<<grid, nt + 32, smem, s>>>(p, seg);
+    // SSD_DEBUG_WITHHOLD_TILE (tests only): the producer withholds that tile
+    const char* wh = getenv("SSD_DEBUG_WITHHOLD_TILE");
+    conv1d_kernel<T, K, ACT><<<grid, nt + 32, smem, s>>>(p, seg, wh ? atoi(wh) : -1);
     return cudaGetLastError();
 }
 
