@@ -70,6 +70,8 @@ class Oracle:
         lib.oracle_selective_scan.argtypes = [_i64] * 4 + [_dp] * 10
         lib.oracle_selective_state_update.restype = None
         lib.oracle_selective_state_update.argtypes = [_i64] * 3 + [_dp] * 9
+        lib.oracle_gated_rmsnorm.restype = None
+        lib.oracle_gated_rmsnorm.argtypes = [_i64, _i64, _i64, ctypes.c_double] + [_dp] * 4
         lib.oracle_gate.restype = None
         lib.oracle_gate.argtypes = [_dp, _dp, _i64]
         lib.oracle_causal_conv1d.restype = None
@@ -157,6 +159,21 @@ class Oracle:
         self.lib.oracle_selective_state_update(b, Dc, N, p(st), p(x), p(dt), p(A), p(B), p(C),
                                                p(D), p(dt_bias), p(y))
         return st, y
+
+    def gated_rmsnorm(self, y, z, weight, group: int, eps: float = 1e-5):
+        """RMSNorm of g = y * silu(z) (g = y without z) over each group of
+        `group` consecutive channels of the last axis, times weight."""
+        yy = self._f64(y)
+        shape = yy.shape
+        yy = yy.reshape(-1, shape[-1])
+        zz = self._f64(z)
+        zz = zz.reshape(yy.shape) if zz is not None else None
+        w = self._f64(weight)
+        out = np.zeros_like(yy)
+        p = self._ptr
+        self.lib.oracle_gated_rmsnorm(yy.shape[0], yy.shape[1], int(group), float(eps), p(yy), p(zz),
+                                      p(w), p(out))
+        return out.reshape(shape)
 
     def ssd_bwd(self, x, dt, A, B, C, D=None, dt_bias=None, init_state=None, dy=None,
                 d_final=None):

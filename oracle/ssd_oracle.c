@@ -45,6 +45,7 @@
  *   oracle_selective_scan, oracle_selective_state_update
  *                        the diagonal-A (per channel and state) selective
  *                        scan and its decode step
+ *   oracle_gated_rmsnorm the RMSNorm of y * silu(z) per channel group
  *
  * Pins (tests/, CPU only): the masked-attention (quadratic) dual form by brute
  * force, the A = 0 cumulative-sum closed form, chunk-size invariance, split /
@@ -428,6 +429,48 @@ void oracle_selective_state_update(int64_t batch, int64_t Dc, int64_t N, double*
             acc += C[b * N + n] * *h;
         }
         y[bd] = acc + (D ? D[d] : 0.0) * x[bd];
+    }
+}
+
+/*
+ * The gated RMSNorm after the scan ("MAMBA-2 Implementation Gaps" lists an
+ * RMSNorm before the final projection; the gated form normalises the gated
+ * output): for each row and each group of `group` consecutive channels,
+ *   g = y * silu(z)   (g = y when z is NULL)
+ *   out = g / sqrt(mean over the group of g^2 + eps) * weight
+ * y, z, out [rows, channels]; weight [channels].
+ */
+void oracle_gated_rmsnorm(int64_t rows, int64_t channels, int64_t group, double eps,
+                          const double* y, const double* z, const double* weight, double* out) {
+    int64_t r;
+#pragma omp parallel for schedule(static)
+    for (r = 0; r < rows; ++r) {
+        for (int64_t g0 = 0; g0 < channels; g0 += group) {
+            double ss = 0.0;
+            for (int64_t k = 0; k < group; ++k) {
+                const int64_t i = r * channels + g0 + k;
+#if ORACLE_MUTANT == 20
+                const double g = y[i];
+#else
+                const double g = z ? y[i] * (z[i] / (1.0 + exp(-z[i]))) : y[i];
+#endif
+                out[i] = g;
+                ss += g * g;
+            }
+#if ORACLE_MUTANT == 21
+            const double inv = 1.0 / sqrt(ss + eps);
+#else
+            const double inv = 1.0 / sqrt(ss / (double)group + eps);
+#endif
+            for (int64_t k = 0; k < group; ++k) {
+                const int64_t i = r * channels + g0 + k;
+#if ORACLE_MUTANT == 20
+                out[i] = out[i] * inv * (z ? z[i] / (1.0 + exp(-z[i])) : 1.0) * weight[g0 + k];
+#else
+                out[i] = out[i] * inv * weight[g0 + k];
+#endif
+            }
+        }
     }
 }
 

@@ -456,7 +456,33 @@ def pin_selective_scan(orc):
     _close(st, fin, 1e-13, "selective decode state == forward final state")
 
 
+def pin_gated_rmsnorm(orc):
+    """The gated RMSNorm against facts its definition fixes: with eps = 0 and
+    weight 1 every group's mean square is exactly 1; it is invariant under a
+    positive rescaling of y and odd in y; a one-channel group gives
+    sign(g) * weight; and a gate of 40 everywhere (silu(40) = 40 to double
+    precision) drops out by the scale invariance, which tells the norm after
+    the gate from the norm before it."""
+    rng = np.random.default_rng(51)
+    rows, ch, grp = 5, 24, 8
+    y = rng.standard_normal((rows, ch))
+    z = rng.standard_normal((rows, ch))
+    w1 = np.ones(ch)
+    out = orc.gated_rmsnorm(y, z, w1, grp, eps=0.0)
+    ms = (out.reshape(rows, ch // grp, grp) ** 2).mean(-1)
+    _close(ms, np.ones_like(ms), 1e-13, "group mean square")
+    w = rng.standard_normal(ch)
+    o1 = orc.gated_rmsnorm(y, z, w, grp, eps=0.0)
+    _close(orc.gated_rmsnorm(3.7 * y, z, w, grp, eps=0.0), o1, 1e-13, "scale invariance")
+    _close(orc.gated_rmsnorm(-y, z, w, grp, eps=0.0), -o1, 1e-14, "odd in y")
+    g = y * z / (1.0 + np.exp(-z))
+    _close(orc.gated_rmsnorm(y, z, w, 1, eps=0.0), np.sign(g) * w, 1e-14, "one-channel groups")
+    big = np.full_like(z, 40.0)
+    _close(orc.gated_rmsnorm(y, big, w, grp, eps=0.0), orc.gated_rmsnorm(y, None, w, grp, eps=0.0),
+           1e-12, "constant large gate drops out")
+
+
 ALL_PINS = [pin_softplus, pin_quadratic_dual, pin_A_zero_cumsum, pin_chunk_invariance,
             pin_split_resume, pin_decode_equals_forward, pin_special_cases, pin_causality,
             pin_half_decay_by_hand, pin_gate, pin_conv1d, pin_bwd_finite_differences,
-            pin_bwd_autograd, pin_selective_scan]
+            pin_bwd_autograd, pin_selective_scan, pin_gated_rmsnorm]

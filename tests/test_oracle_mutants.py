@@ -11,14 +11,16 @@ convolution inputs; in the backward pass, 14 drops the decay when the adjoint
 steps back a token; 15 drops the decay's share A*da of ddt; 16 drops the
 softplus derivative of ddt_raw; 17 adds dy_t C_t^T to the adjoint only after
 using it; in the diagonal-A selective scan, 18 decays every state with the
-channel's first A entry; 19 feeds channel 0's x to every channel.
+channel's first A entry; 19 feeds channel 0's x to every channel; in the
+gated RMSNorm, 20 normalises before the gate; 21 divides by the root of the
+sum of squares instead of their mean.
 """
 import pytest
 
 import oracle
 import pins
 
-MUTANTS = list(range(1, 20))
+MUTANTS = list(range(1, 22))
 
 
 @pytest.fixture(scope="module")
