@@ -59,6 +59,8 @@ def parse_args():
                     help="time only the backward-pass workloads (one JSON line of them)")
     ap.add_argument("--sel-only", action="store_true",
                     help="time only the diagonal-A selective-scan workloads (one JSON line)")
+    ap.add_argument("--norm-only", action="store_true",
+                    help="time only the gated RMSNorm workloads (one JSON line of them)")
     return ap.parse_args()
 
 
@@ -242,8 +244,10 @@ def main_ours(args):
         flush_buf.fill_(1)
         torch.sum(flush_f, dim=0, out=flush_acc)
 
-    if args.conv_only or args.bwd_only or args.sel_only:
-        if args.conv_only:
+    if args.conv_only or args.bwd_only or args.sel_only or args.norm_only:
+        if args.norm_only:
+            res = norm_workloads(ssd, synthetic, dev, flush, peaks, rank, world, ranks_max)
+        elif args.conv_only:
             res = conv_workloads(ssd, synthetic, dev, flush, peaks, rank, world, ranks_max)
         elif args.bwd_only:
             res = bwd_workloads(ssd, synthetic, dev, flush, peaks, rank, world, ranks_max)
@@ -661,6 +665,47 @@ def other_workloads(ssd, synthetic, dev, flush, peaks, rank, world, barrier, ran
     out.update(conv_workloads(ssd, synthetic, dev, flush, peaks, rank, world, ranks_max))
     out.update(bwd_workloads(ssd, synthetic, dev, flush, peaks, rank, world, ranks_max))
     out.update(sel_workloads(ssd, synthetic, dev, flush, peaks, rank, world, ranks_max))
+    out.update(norm_workloads(ssd, synthetic, dev, flush, peaks, rank, world, ranks_max))
+    return out
+
+
+def norm_workloads(ssd, synthetic, dev, flush, peaks, rank, world, ranks_max, steps=10):
+    """The gated RMSNorm over the scan output of the two forward workloads
+    (rows = batch * seqlen, channels = nheads * headdim, one group per row),
+    L2 flushed before each launch."""
+    import torch
+    out = {}
+    stream = torch.cuda.current_stream()
+    for fname in ("fwd_bf16_b4_L1024", "fwd_bf16_b8_L4096_init"):
+        f = synthetic.FWD_CONFIGS[fname]
+        rows, ch = f.batch * f.seqlen, f.nheads * f.headdim
+        name = f"gated_rmsnorm_bf16_b{f.batch}_L{f.seqlen}_C{ch}"
+        inp = synthetic.make_norm_inputs(rows, ch, f.dtype, rank_seed(1234 + 9, rank))
+        d = {k: v.to(dev) for k, v in inp.items()}
+        o = torch.empty_like(d["y"])
+
+        def step():
+            ssd.ssd_gated_rmsnorm(d["y"], d["z"], d["weight"], eps=1e-5, out=o)
+
+        for _ in range(3):
+            step()
+        torch.cuda.synchronize()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)]
+        for a, b_ in evs:
+            flush()
+            a.record(stream)
+            step()
+            b_.record(stream)
+        torch.cuda.synchronize()
+        ms = ranks_max(sum(a.elapsed_time(b_) for a, b_ in evs) / steps)
+        nbytes = 3 * rows * ch * d["y"].element_size() + ch * 4
+        out[name] = {"tokens_per_s": job_throughput(rows, world, ms), "ms": ms,
+                     "achieved_gbs": nbytes / (ms * 1e-3) / 1e9,
+                     "hbm_frac": nbytes / (ms * 1e-3) / (peaks["hbm_gbs"] * 1e9),
+                     "bytes": nbytes, "group": ch, "l2": "flushed"}
+        del d, o
+    torch.cuda.empty_cache()
     return out
 
 

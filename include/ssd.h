@@ -399,6 +399,33 @@ typedef struct {
 
 ssd_status ssd_conv1d_update(const ssd_conv1d_update_args* args, void* stream);
 
+/* ---- gated RMSNorm (after the scan) ------------------------------------- */
+/* The normalisation "MAMBA-2 Implementation Gaps" (section 7.3, items 9 and
+ * 11) puts between the scan and the output projection, with the output gate
+ * y * silu(z) applied inside it: for each row and each group of `group`
+ * consecutive channels,
+ *   g = y * silu(z)  (g = y when z is NULL),
+ *   out = g / sqrt(mean over the group of g^2 + eps) * weight.
+ * Use it on the ungated y of ssd_fwd (z = NULL there) with the same z here.
+ * Layouts: y, z, out [rows, channels] dtype (rows = batch * seqlen for the
+ *   scan's y viewed as [batch * seqlen, nheads * headdim]); weight [channels]
+ *   fp32.  out may be y (in place).  Arithmetic in fp32; out rounded to dtype.
+ * Supported: channels % group == 0; group a multiple of 8 (bf16) or 4 (fp32)
+ *   (else SSD_ERR_UNSUPPORTED); eps >= 0 and finite, sizes > 0, y, weight,
+ *   out non-NULL (else SSD_ERR_INVALID_ARG); every pointer 16-byte aligned
+ *   (else SSD_ERR_INVALID_ARG). */
+typedef struct {
+    int64_t rows, channels, group;
+    int32_t dtype;
+    float eps;
+    const void* y;
+    const void* z;           /* optional gate; NULL = none */
+    const float* weight;
+    void* out;
+} ssd_gated_rmsnorm_args;
+
+ssd_status ssd_gated_rmsnorm(const ssd_gated_rmsnorm_args* args, void* stream);
+
 /* ---- misc --------------------------------------------------------------- */
 /* Static, human-readable name of a status code. */
 const char* ssd_status_string(ssd_status status);

@@ -21,7 +21,7 @@ __all__ = [
     "ssd_version", "lib_path", "load_library", "SSD_FLAG_CUDA_CORES", "SSD_FLAG_WHOLE_GROUPS",
     "ssd_causal_conv1d", "ssd_conv1d_update", "ssd_conv1d_check_status",
     "ssd_bwd", "ssd_bwd_workspace_size", "ssd_selective_scan", "ssd_selective_scan_workspace_size",
-    "ssd_selective_state_update",
+    "ssd_selective_state_update", "ssd_gated_rmsnorm",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -94,6 +94,12 @@ class SsdConv1dUpdateArgs(ctypes.Structure):
                 ("bias", _vp), ("y", _vp)]
 
 
+class SsdGatedRmsnormArgs(ctypes.Structure):
+    """Mirror of ssd_gated_rmsnorm_args."""
+    _fields_ = [("rows", _i64), ("channels", _i64), ("group", _i64), ("dtype", _i32),
+                ("eps", ctypes.c_float), ("y", _vp), ("z", _vp), ("weight", _vp), ("out", _vp)]
+
+
 class SsdError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
@@ -157,6 +163,8 @@ def load_library():
     lib.ssd_causal_conv1d.argtypes = [ctypes.POINTER(SsdConv1dArgs), _vp]
     lib.ssd_conv1d_update.restype = ctypes.c_int
     lib.ssd_conv1d_update.argtypes = [ctypes.POINTER(SsdConv1dUpdateArgs), _vp]
+    lib.ssd_gated_rmsnorm.restype = ctypes.c_int
+    lib.ssd_gated_rmsnorm.argtypes = [ctypes.POINTER(SsdGatedRmsnormArgs), _vp]
     lib.ssd_conv1d_check_status.restype = ctypes.c_int
     lib.ssd_conv1d_check_status.argtypes = [_vp]
     lib.ssd_status_string.restype = ctypes.c_char_p
@@ -593,3 +601,26 @@ def ssd_conv1d_update(state, x, weight, bias=None, *, activation: bool = True, y
     a.state, a.x, a.weight, a.bias, a.y = _ptr(state), _ptr(x), _ptr(weight), _ptr(bias), _ptr(y)
     _check(lib.ssd_conv1d_update(ctypes.byref(a), _stream_ptr(stream)), "ssd_conv1d_update")
     return y
+
+
+def ssd_gated_rmsnorm(y, z, weight, *, group: int | None = None, eps: float = 1e-5, out=None,
+                      stream=None):
+    """RMSNorm of g = y * silu(z) (g = y when z is None) over each group of
+    ``group`` consecutive channels of the last axis (default: the whole last
+    axis), times weight [channels] float32.  y, z: [..., channels] in one
+    dtype.  ``out`` may be ``y`` (in place).  Returns out."""
+    lib = load_library()
+    channels = y.shape[-1]
+    rows = y.numel() // channels
+    if z is not None and (z.dtype != y.dtype or z.shape != y.shape):
+        raise TypeError("z must match y in dtype and shape")
+    if weight.dtype != torch.float32 or weight.numel() != channels:
+        raise TypeError("weight must be float32 with one entry per channel")
+    out = out if out is not None else torch.empty_like(y)
+    a = SsdGatedRmsnormArgs()
+    a.rows, a.channels, a.group = rows, channels, int(group if group is not None else channels)
+    a.dtype = _dtype_code(y)
+    a.eps = float(eps)
+    a.y, a.z, a.weight, a.out = _ptr(y), _ptr(z), _ptr(weight), _ptr(out)
+    _check(lib.ssd_gated_rmsnorm(ctypes.byref(a), _stream_ptr(stream)), "ssd_gated_rmsnorm")
+    return out

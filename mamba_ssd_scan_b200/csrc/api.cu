@@ -4,6 +4,7 @@
 #include <stdint.h>
 #include <string.h>
 
+#include "gated_rmsnorm.h"
 #include "internal.cuh"
 
 namespace {
@@ -595,6 +596,29 @@ ssd_status ssd_conv1d_update(const ssd_conv1d_update_args* a, void* stream) {
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     return to_status(a->dtype == SSD_BF16 ? ssd::launch_conv1d<__nv_bfloat16>(p, true, s)
                                           : ssd::launch_conv1d<float>(p, true, s));
+}
+
+ssd_status ssd_gated_rmsnorm(const ssd_gated_rmsnorm_args* a, void* stream) {
+    if (!a) return SSD_ERR_INVALID_ARG;
+    if (a->rows <= 0 || a->channels <= 0 || a->group <= 0) return SSD_ERR_INVALID_ARG;
+    if (a->dtype != SSD_F32 && a->dtype != SSD_BF16) return SSD_ERR_INVALID_ARG;
+    if (!(a->eps >= 0.0f) || !(a->eps <= 3.4e38f)) return SSD_ERR_INVALID_ARG;
+    if (a->channels % a->group != 0 || a->group % (a->dtype == SSD_BF16 ? 8 : 4) != 0)
+        return SSD_ERR_UNSUPPORTED;
+    if (!check_ptr(a->y, false, true) || !check_ptr(a->z, true, true) ||
+        !check_ptr(a->weight, false, true) || !check_ptr(a->out, false, true))
+        return SSD_ERR_INVALID_ARG;
+    ssd::NormParams p;
+    p.rows = a->rows;
+    p.channels = a->channels;
+    p.group = a->group;
+    p.eps = a->eps;
+    p.y = a->y;
+    p.z = a->z;
+    p.weight = a->weight;
+    p.out = a->out;
+    return to_status(ssd::launch_gated_rmsnorm(p, a->dtype == SSD_BF16,
+                                               static_cast<cudaStream_t>(stream)));
 }
 
 ssd_status ssd_state_update(const ssd_state_update_args* a, void* stream) {

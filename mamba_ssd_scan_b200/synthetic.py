@@ -190,6 +190,17 @@ def make_gate(shape, dtype, seed: int) -> torch.Tensor:
     return torch.randn(tuple(shape), generator=gen, dtype=torch.float32).to(dtype)
 
 
+def make_norm_inputs(rows: int, channels: int, dtype, seed: int, gate: bool = True) -> dict:
+    """Inputs of the gated RMSNorm: y, z ~ N(0, 1) [rows, channels] in dtype
+    (z None without the gate) and the weight ~ 1 + 0.1 N(0, 1) [channels]
+    fp32 (an RMSNorm weight starts at one)."""
+    gen = torch.Generator().manual_seed(seed + 7927)
+    y = torch.randn((rows, channels), generator=gen).to(dtype)
+    z = torch.randn((rows, channels), generator=gen).to(dtype) if gate else None
+    weight = 1.0 + 0.1 * torch.randn((channels,), generator=gen)
+    return {"y": y, "z": z, "weight": weight}
+
+
 def make_bwd_grads(x_shape, state_shape, dtype, seed: int) -> dict:
     """Incoming gradients of a backward call: dy ~ N(0,1) shaped like x (in
     dtype) and d_final ~ N(0,1) shaped like the state (fp32)."""

@@ -166,3 +166,21 @@ def test_selective_scan_rejects_bad_args(lib):
     assert lib.ssd_selective_state_update(ctypes.byref(u), None) == 1   # null pointers
     u.dstate = 40
     assert lib.ssd_selective_state_update(ctypes.byref(u), None) == 2
+
+
+def test_gated_rmsnorm_rejects_bad_args(lib):
+    import mamba_ssd_scan_b200 as ssd
+    a = ssd.SsdGatedRmsnormArgs()
+    a.rows, a.channels, a.group, a.dtype, a.eps = 4, 64, 32, 1, 1e-5
+    assert lib.ssd_gated_rmsnorm(None, None) == 1
+    assert lib.ssd_gated_rmsnorm(ctypes.byref(a), None) == 1      # null pointers
+    a.group = 48
+    assert lib.ssd_gated_rmsnorm(ctypes.byref(a), None) == 2      # channels % group
+    a.group = 4
+    assert lib.ssd_gated_rmsnorm(ctypes.byref(a), None) == 2      # bf16 group % 8
+    a.dtype = 0
+    assert lib.ssd_gated_rmsnorm(ctypes.byref(a), None) == 1      # fp32 group 4 fine: null pointers
+    a.group, a.eps = 32, -1.0
+    assert lib.ssd_gated_rmsnorm(ctypes.byref(a), None) == 1      # negative eps
+    a.eps, a.rows = 1e-5, 0
+    assert lib.ssd_gated_rmsnorm(ctypes.byref(a), None) == 1      # no rows
