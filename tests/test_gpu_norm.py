@@ -80,7 +80,10 @@ def test_scan_then_norm_full_size(orc, name):
     d = {k: (v.to(DEV) if v is not None else None) for k, v in inp.items()}
     y = ssd.ssd_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["dt_bias"], cfg.chunk,
                     d["init_state"])
-    out = ssd.ssd_gated_rmsnorm(y, z.to(DEV), weight.to(DEV), eps=1e-5)
+    # heads * headdim are the channels of a token
+    out = ssd.ssd_gated_rmsnorm(y.view(cfg.batch, cfg.seqlen, ch),
+                                z.reshape(cfg.batch, cfg.seqlen, ch).to(DEV), weight.to(DEV),
+                                eps=1e-5)
     torch.cuda.synchronize()
     ref = orc.gated_rmsnorm(y.float().cpu().reshape(-1, ch), z.reshape(-1, ch), weight, ch,
                             eps=1e-5)
