@@ -91,7 +91,18 @@ def test_scan_then_norm_full_size(orc, name):
     row0 = {k: (v[:1] if k in ("x", "dt", "B", "C", "init_state") and v is not None else v)
             for k, v in inp.items()}
     y0, _ = orc.ssd_fwd(**row0)
-    ref0 = orc.gated_rmsnorm(np.asarray(y0).reshape(-1, ch), z[:1].reshape(-1, ch), weight, ch,
-                             eps=1e-5)
-    assert_close(out[:1].reshape(-1, ch), ref0, cfg.dtype,
-                 "scan + norm against the oracle, batch row 0")
+    y0 = np.asarray(y0).reshape(-1, ch)
+    ref0 = orc.gated_rmsnorm(y0, z[:1].reshape(-1, ch), weight, ch, eps=1e-5)
+    # the chain's bound: the scan's own bf16 bound on y, carried through the
+    # norm's per-row scale (first order: the row's mean square averages over
+    # its channels, so inv moves far less than one element does), plus the
+    # norm's own bf16 bound
+    zz = z[:1].reshape(-1, ch).double().numpy()
+    gate = zz / (1.0 + np.exp(-zz))
+    inv = 1.0 / np.sqrt(np.mean((y0 * gate) ** 2, axis=1, keepdims=True) + 1e-5)
+    scale = inv * np.abs(gate * weight.double().numpy())
+    y_bound = 2e-2 * (np.abs(y0) + np.sqrt(np.mean(y0 * y0)))
+    bound = y_bound * scale + 2e-2 * (np.abs(ref0) + np.sqrt(np.mean(ref0 * ref0)))
+    got = out[:1].reshape(-1, ch).double().cpu().numpy()
+    bad = np.abs(got - ref0) > bound
+    assert not bad.any(), f"scan + norm, batch row 0: {int(bad.sum())} elements beyond the chain bound"
