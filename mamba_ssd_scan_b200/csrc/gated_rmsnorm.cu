@@ -12,9 +12,9 @@
 //
 // A unit is one (row, group) pair; its `group` elements are contiguous at
 // unit * group.  A unit is spread over LPU lanes (a power of two up to the
-// CTA's 256 threads, chosen so that each lane holds up to MAXV vectors), each
-// lane holding V 16-byte vectors of it (lane l takes vectors l, l + LPU, ...,
-// so the lanes of a unit read consecutive 16-byte pieces).  Up to MAXV vectors per lane are kept in registers between the sum
+// CTA's 256 threads, the smallest that leaves each lane at most MAXV
+// vectors), lane l taking vectors l, l + LPU, ... of the unit, so the lanes of
+// a unit read consecutive 16-byte pieces; the last round may be ragged.  Up to MAXV vectors per lane are kept in registers between the sum
 // of squares and the scaling; a longer unit re-reads its y and z (from L2) in
 // the second pass.  The sum of squares is a shuffle reduction over the unit's
 // lanes, plus a shared-memory step when the unit spans several warps.
@@ -85,7 +85,7 @@ template <int N> __device__ __forceinline__ void weights(const float* p, float* 
 }
 
 template <typename T>
-__global__ void __launch_bounds__(TPB) gated_rmsnorm_kernel(NormParams p, int lpu, int nvec) {
+__global__ void __launch_bounds__(TPB) gated_rmsnorm_kernel(NormParams p, int lpu, int nvec, int vecs) {
     constexpr int N = Vec<T>::N;
     __shared__ float red[TPB / 32];
     const T* y = static_cast<const T*>(p.y);
@@ -111,15 +111,18 @@ __global__ void __launch_bounds__(TPB) gated_rmsnorm_kernel(NormParams p, int lp
         if (live) {
 #pragma unroll
             for (int j = 0; j < MAXV; ++j) {
-                if (j < nvec) {
-                    gated(y, z, base + static_cast<int64_t>(lane_in_unit + j * lpu) * N, g[j]);
+                const int v = lane_in_unit + j * lpu;
+                if (j < nvec && v < vecs) {
+                    gated(y, z, base + static_cast<int64_t>(v) * N, g[j]);
 #pragma unroll
                     for (int i = 0; i < N; ++i) ss = fmaf(g[j][i], g[j][i], ss);
                 }
             }
             for (int j = MAXV; j < nvec; ++j) {
+                const int v = lane_in_unit + j * lpu;
+                if (v >= vecs) break;
                 float t[N];
-                gated(y, z, base + static_cast<int64_t>(lane_in_unit + j * lpu) * N, t);
+                gated(y, z, base + static_cast<int64_t>(v) * N, t);
 #pragma unroll
                 for (int i = 0; i < N; ++i) ss = fmaf(t[i], t[i], ss);
             }
@@ -141,8 +144,9 @@ __global__ void __launch_bounds__(TPB) gated_rmsnorm_kernel(NormParams p, int lp
         if (live) {
 #pragma unroll
             for (int j = 0; j < MAXV; ++j) {
-                if (j < nvec) {
-                    const int64_t c = static_cast<int64_t>(lane_in_unit + j * lpu) * N;
+                const int v = lane_in_unit + j * lpu;
+                if (j < nvec && v < vecs) {
+                    const int64_t c = static_cast<int64_t>(v) * N;
                     float w[N];
                     weights<N>(p.weight + wbase + c, w);
 #pragma unroll
@@ -151,7 +155,9 @@ __global__ void __launch_bounds__(TPB) gated_rmsnorm_kernel(NormParams p, int lp
                 }
             }
             for (int j = MAXV; j < nvec; ++j) {
-                const int64_t c = static_cast<int64_t>(lane_in_unit + j * lpu) * N;
+                const int v = lane_in_unit + j * lpu;
+                if (v >= vecs) break;
+                const int64_t c = static_cast<int64_t>(v) * N;
                 float t[N], w[N];
                 gated(y, z, base + c, t);
                 weights<N>(p.weight + wbase + c, w);
@@ -173,14 +179,13 @@ int device_sms() {
 template <typename T> cudaError_t launch(const NormParams& p, cudaStream_t s) {
     constexpr int N = Vec<T>::N;
     const int64_t vecs = p.group / N;                // 16-byte vectors per unit
-    // lanes per unit: the largest power of two that divides the unit's vectors
-    // (at most a CTA), then halved while each lane can hold twice as many
-    // vectors in registers (more bytes in flight per thread, fewer barriers)
+    // lanes per unit: the smallest power of two (at most a CTA) that leaves
+    // each lane at most MAXV vectors, so that a lane keeps as many bytes in
+    // flight as its registers hold; the last round of a unit may be ragged
+    if (vecs > (int64_t{1} << 30)) return cudaErrorInvalidValue;
     int lpu = 1;
-    while (lpu < TPB && vecs % (2 * lpu) == 0) lpu *= 2;
-    while (lpu > 1 && (vecs / lpu) * 2 <= MAXV) lpu /= 2;
-    const int64_t nvec = vecs / lpu;
-    if (nvec > (1 << 20)) return cudaErrorInvalidValue;
+    while (lpu < TPB && static_cast<int64_t>(lpu) * MAXV < vecs) lpu *= 2;
+    const int64_t nvec = (vecs + lpu - 1) / lpu;
     const int64_t units = p.rows * (p.channels / p.group);
     const int64_t upc = TPB / lpu;
     int per_sm = 0;
@@ -190,7 +195,8 @@ template <typename T> cudaError_t launch(const NormParams& p, cudaStream_t s) {
     const int64_t want = (units + upc - 1) / upc;
     const int64_t cap = static_cast<int64_t>(device_sms()) * per_sm;
     const unsigned grid = static_cast<unsigned>(want < cap ? want : cap);
-    gated_rmsnorm_kernel<T><<<grid, TPB, 0, s>>>(p, lpu, static_cast<int>(nvec));
+    gated_rmsnorm_kernel<T><<<grid, TPB, 0, s>>>(p, lpu, static_cast<int>(nvec),
+                                                 static_cast<int>(vecs));
     return cudaGetLastError();
 }
 

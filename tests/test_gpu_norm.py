@@ -1,6 +1,7 @@
 """Parity of the gated RMSNorm (through the C ABI) with the fp64 oracle, over
 every element: the unit shapes the kernel distinguishes (one lane to a whole
-CTA per group, groups held in registers or re-read), in place, extreme gates,
+CTA per group, groups held in registers or re-read, ragged last rounds), in
+place, extreme gates,
 and the norm after the scan at the benchmark's sizes."""
 import numpy as np
 import pytest
@@ -24,8 +25,10 @@ NORM_CASES = [
     (50, 1536, 1536, torch.bfloat16, True),   # 64 x 3: two warps per group
     (33, 2048, 2048, torch.bfloat16, False),  # 64 x 4, no gate
     (3, 8192, 8192, torch.bfloat16, True),    # 256 x 4: a whole CTA per group
-    (7, 4112, 2056, torch.bfloat16, True),    # 1 x 257: the re-read pass
+    (5, 40, 40, torch.bfloat16, True),        # 2 x 3, the last round ragged (5 vectors)
+    (7, 4112, 2056, torch.bfloat16, True),    # 128 x 3, ragged (257 vectors)
     (3, 16384, 16384, torch.float32, True),   # 256 x 16: a whole CTA, re-read pass
+    (4, 24024, 24024, torch.bfloat16, True),  # 256 x 12, re-read pass, ragged (3003 vectors)
 ]
 
 
