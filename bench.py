@@ -692,6 +692,7 @@ def norm_workloads(ssd, synthetic, dev, flush, peaks, rank, world, ranks_max, st
         torch.cuda.synchronize()
         evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(steps)]
+        gpu_head_start(2.0)
         for a, b_ in evs:
             flush()
             a.record(stream)

@@ -26,14 +26,14 @@ namespace {
 constexpr int TPB = 256;
 constexpr int MAXV = 4;   // 16-byte vectors per lane kept in registers
 
-// Eight (bf16) or four (fp32) consecutive elements, widened to fp32.  Plain
-// (coherent) loads: out may be y itself.
+// Eight (bf16) or four (fp32) consecutive elements as one 16-byte word, widened
+// to fp32.  Plain (coherent) loads: out may be y itself.
 template <typename T> struct Vec;
 template <> struct Vec<float> {
     static constexpr int N = 4;
-    static __device__ __forceinline__ void load(const float* p, float* v) {
-        const float4 a = *reinterpret_cast<const float4*>(p);
-        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    static __device__ __forceinline__ void widen(uint4 a, float* v) {
+        v[0] = __uint_as_float(a.x); v[1] = __uint_as_float(a.y);
+        v[2] = __uint_as_float(a.z); v[3] = __uint_as_float(a.w);
     }
     static __device__ __forceinline__ void store(float* p, const float* v) {
         *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
@@ -41,8 +41,7 @@ template <> struct Vec<float> {
 };
 template <> struct Vec<__nv_bfloat16> {
     static constexpr int N = 8;
-    static __device__ __forceinline__ void load(const __nv_bfloat16* p, float* v) {
-        const uint4 a = *reinterpret_cast<const uint4*>(p);
+    static __device__ __forceinline__ void widen(uint4 a, float* v) {
         const uint32_t w[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -61,14 +60,18 @@ template <> struct Vec<__nv_bfloat16> {
     }
 };
 
-// g = y * silu(z) for one vector (y alone when there is no gate).
-template <typename T>
-__device__ __forceinline__ void gated(const T* y, const T* z, int64_t off, float* g) {
+template <typename T> __device__ __forceinline__ uint4 ld16(const T* p) {
+    return *reinterpret_cast<const uint4*>(p);
+}
+
+// g = y * silu(z) from the raw words (y alone without the gate).
+template <typename T, bool GATED>
+__device__ __forceinline__ void gate_vec(uint4 ry, uint4 rz, float* g) {
     constexpr int N = Vec<T>::N;
-    Vec<T>::load(y + off, g);
-    if (z) {
+    Vec<T>::widen(ry, g);
+    if constexpr (GATED) {
         float zv[N];
-        Vec<T>::load(z + off, zv);
+        Vec<T>::widen(rz, zv);
 #pragma unroll
         for (int i = 0; i < N; ++i) g[i] *= silu_f32(zv[i]);
     }
@@ -84,8 +87,10 @@ template <int N> __device__ __forceinline__ void weights(const float* p, float* 
     }
 }
 
-template <typename T>
-__global__ void __launch_bounds__(TPB) gated_rmsnorm_kernel(NormParams p, int lpu, int nvec, int vecs) {
+// NV: vectors per lane held in registers (1..MAXV); a lane's vectors past
+// NV (nvec > NV) are re-read in the second pass.
+template <typename T, int NV, bool GATED>
+__global__ void __launch_bounds__(TPB, 4) gated_rmsnorm_kernel(NormParams p, int lpu, int nvec, int vecs) {
     constexpr int N = Vec<T>::N;
     __shared__ float red[TPB / 32];
     const T* y = static_cast<const T*>(p.y);
@@ -105,24 +110,36 @@ __global__ void __launch_bounds__(TPB) gated_rmsnorm_kernel(NormParams p, int lp
         const int64_t base = u * p.group;
         const int64_t wbase = (u % ngroups) * p.group;
 
-        // pass 1: g and the sum of its squares
-        float g[MAXV][N];
+        // pass 1: every raw load of the lane first (a ragged round's missing
+        // vectors read the lane's first one again and count as zero), then g
+        // and the sum of its squares
+        float g[NV][N];
         float ss = 0.0f;
         if (live) {
+            uint4 ry[NV], rz[NV];
 #pragma unroll
-            for (int j = 0; j < MAXV; ++j) {
+            for (int j = 0; j < NV; ++j) {
                 const int v = lane_in_unit + j * lpu;
-                if (j < nvec && v < vecs) {
-                    gated(y, z, base + static_cast<int64_t>(v) * N, g[j]);
+                const int64_t off = base + static_cast<int64_t>(v < vecs ? v : lane_in_unit) * N;
+                ry[j] = ld16(y + off);
+                if constexpr (GATED) rz[j] = ld16(z + off);
+            }
 #pragma unroll
-                    for (int i = 0; i < N; ++i) ss = fmaf(g[j][i], g[j][i], ss);
+            for (int j = 0; j < NV; ++j) {
+                gate_vec<T, GATED>(ry[j], rz[j], g[j]);
+                const bool in = lane_in_unit + j * lpu < vecs;
+#pragma unroll
+                for (int i = 0; i < N; ++i) {
+                    g[j][i] = in ? g[j][i] : 0.0f;
+                    ss = fmaf(g[j][i], g[j][i], ss);
                 }
             }
-            for (int j = MAXV; j < nvec; ++j) {
+            for (int j = NV; j < nvec; ++j) {
                 const int v = lane_in_unit + j * lpu;
                 if (v >= vecs) break;
+                const int64_t off = base + static_cast<int64_t>(v) * N;
                 float t[N];
-                gated(y, z, base + static_cast<int64_t>(v) * N, t);
+                gate_vec<T, GATED>(ld16(y + off), GATED ? ld16(z + off) : uint4{}, t);
 #pragma unroll
                 for (int i = 0; i < N; ++i) ss = fmaf(t[i], t[i], ss);
             }
@@ -143,9 +160,9 @@ __global__ void __launch_bounds__(TPB) gated_rmsnorm_kernel(NormParams p, int lp
         // pass 2: scale by inv and the weight, round, store
         if (live) {
 #pragma unroll
-            for (int j = 0; j < MAXV; ++j) {
+            for (int j = 0; j < NV; ++j) {
                 const int v = lane_in_unit + j * lpu;
-                if (j < nvec && v < vecs) {
+                if (v < vecs) {
                     const int64_t c = static_cast<int64_t>(v) * N;
                     float w[N];
                     weights<N>(p.weight + wbase + c, w);
@@ -154,12 +171,12 @@ __global__ void __launch_bounds__(TPB) gated_rmsnorm_kernel(NormParams p, int lp
                     Vec<T>::store(out + base + c, w);
                 }
             }
-            for (int j = MAXV; j < nvec; ++j) {
+            for (int j = NV; j < nvec; ++j) {
                 const int v = lane_in_unit + j * lpu;
                 if (v >= vecs) break;
                 const int64_t c = static_cast<int64_t>(v) * N;
                 float t[N], w[N];
-                gated(y, z, base + c, t);
+                gate_vec<T, GATED>(ld16(y + base + c), GATED ? ld16(z + base + c) : uint4{}, t);
                 weights<N>(p.weight + wbase + c, w);
 #pragma unroll
                 for (int i = 0; i < N; ++i) w[i] *= t[i] * inv;
@@ -171,12 +188,39 @@ __global__ void __launch_bounds__(TPB) gated_rmsnorm_kernel(NormParams p, int lp
 
 int device_sms() {
     int dev = 0, n = 148;
-    if (cudaGetDevice(&dev) == cudaSuccess)
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+        cudaGetLastError();
+        n = 148;
+    }
     return n;
 }
 
-template <typename T> cudaError_t launch(const NormParams& p, cudaStream_t s) {
+template <typename T, int NV, bool GATED>
+cudaError_t launch_nv(const NormParams& p, int lpu, int64_t nvec, int64_t vecs, cudaStream_t s) {
+    const auto kern = gated_rmsnorm_kernel<T, NV, GATED>;
+    const int64_t units = p.rows * (p.channels / p.group);
+    const int64_t upc = TPB / lpu;
+    static int occ;  // CTAs per SM of this instantiation (same on every B200); benign race
+    if (occ == 0) {
+        int n = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, TPB, 0) != cudaSuccess ||
+            n < 1) {
+            cudaGetLastError();
+            n = 1;
+        }
+        occ = n;
+    }
+    const int per_sm = occ;
+    const int64_t want = (units + upc - 1) / upc;
+    const int64_t cap = static_cast<int64_t>(device_sms()) * per_sm;
+    const unsigned grid = static_cast<unsigned>(want < cap ? want : cap);
+    kern<<<grid, TPB, 0, s>>>(p, lpu, static_cast<int>(nvec), static_cast<int>(vecs));
+    return cudaGetLastError();
+}
+
+template <typename T, bool GATED>
+cudaError_t launch(const NormParams& p, cudaStream_t s) {
     constexpr int N = Vec<T>::N;
     const int64_t vecs = p.group / N;                // 16-byte vectors per unit
     // lanes per unit: the smallest power of two (at most a CTA) that leaves
@@ -186,24 +230,19 @@ template <typename T> cudaError_t launch(const NormParams& p, cudaStream_t s) {
     int lpu = 1;
     while (lpu < TPB && static_cast<int64_t>(lpu) * MAXV < vecs) lpu *= 2;
     const int64_t nvec = (vecs + lpu - 1) / lpu;
-    const int64_t units = p.rows * (p.channels / p.group);
-    const int64_t upc = TPB / lpu;
-    int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gated_rmsnorm_kernel<T>, TPB, 0) !=
-            cudaSuccess || per_sm < 1)
-        per_sm = 1;
-    const int64_t want = (units + upc - 1) / upc;
-    const int64_t cap = static_cast<int64_t>(device_sms()) * per_sm;
-    const unsigned grid = static_cast<unsigned>(want < cap ? want : cap);
-    gated_rmsnorm_kernel<T><<<grid, TPB, 0, s>>>(p, lpu, static_cast<int>(nvec),
-                                                 static_cast<int>(vecs));
-    return cudaGetLastError();
+    switch (nvec) {
+        case 1: return launch_nv<T, 1, GATED>(p, lpu, nvec, vecs, s);
+        case 2: return launch_nv<T, 2, GATED>(p, lpu, nvec, vecs, s);
+        case 3: return launch_nv<T, 3, GATED>(p, lpu, nvec, vecs, s);
+        default: return launch_nv<T, MAXV, GATED>(p, lpu, nvec, vecs, s);
+    }
 }
 
 }  // namespace
 
 cudaError_t launch_gated_rmsnorm(const NormParams& p, bool bf16, cudaStream_t s) {
-    return bf16 ? launch<__nv_bfloat16>(p, s) : launch<float>(p, s);
+    if (bf16) return p.z ? launch<__nv_bfloat16, true>(p, s) : launch<__nv_bfloat16, false>(p, s);
+    return p.z ? launch<float, true>(p, s) : launch<float, false>(p, s);
 }
 
 }  // namespace ssd
