@@ -17,8 +17,9 @@
 // each chunk replayed from the state entering it (sel_output_kernel).  One
 // thread per channel, its N states in registers; the chunk's B and C rows
 // (shared by every channel) are staged in shared memory and read as
-// broadcasts.  The decode step (sel_update_kernel) applies the recurrence
-// once to a carried state [b, channels, N].
+// broadcasts.  The decode step (sel_update_split_kernel for N = 8, 16, 32,
+// sel_update_kernel otherwise) applies the recurrence once to a carried state
+// [b, channels, N].
 #include "internal.cuh"
 
 namespace ssd {
@@ -271,10 +272,61 @@ __global__ void __launch_bounds__(256) sel_update_kernel(SelParams p) {
     static_cast<T*>(p.y)[e] = from_f32<T>(fmaf(Dd, xv, acc));
 }
 
+// The decode step with a (batch, channel)'s N states split over N / 4 lanes
+// (N = 8, 16 or 32), one float4 of state each, so that a warp's state loads and
+// stores are contiguous and a step has N / 4 times as many threads to hide
+// their latency; the lanes' parts of C . h are summed by a shuffle.  Every
+// lane takes part in the shuffle; only live lanes load and store.
+template <typename T, int N>
+__global__ void __launch_bounds__(256) sel_update_split_kernel(SelParams p) {
+    constexpr int TPE = N / 4;                       // lanes per (batch, channel)
+    static_assert(TPE == 2 || TPE == 4 || TPE == 8, "power-of-two split");
+    const int64_t Dc = p.channels, n = p.batch * Dc;
+    const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int64_t e = tid / TPE;
+    const int j = static_cast<int>(tid % TPE);
+    const bool live = e < n;
+    const int64_t b = live ? e / Dc : 0, d = live ? e % Dc : 0;
+    grid_dep_wait();
+    grid_dep_launch();
+    float4* sp = reinterpret_cast<float4*>(p.S) + e * TPE + j;
+    float4 hv = make_float4(0.0f, 0.0f, 0.0f, 0.0f), av = hv, bv = hv, cv = hv;
+    float xv = 0.0f, dr = 0.0f, bias = 0.0f, Dd = 0.0f;
+    if (live) {
+        hv = *sp;
+        av = __ldg(reinterpret_cast<const float4*>(p.A + d * N) + j);
+        bv = Vec4<T>::load(static_cast<const T*>(p.B) + b * N + 4 * j);
+        cv = Vec4<T>::load(static_cast<const T*>(p.C) + b * N + 4 * j);
+        xv = to_f32(static_cast<const T*>(p.x)[e]);
+        dr = to_f32(static_cast<const T*>(p.dt_raw)[e]);
+        bias = p.dt_bias ? p.dt_bias[d] : 0.0f;
+        Dd = p.D ? p.D[d] : 0.0f;
+    }
+    const float dt = softplus_f32(dr + bias);
+    const float dx = dt * xv, dl = dt * kLog2e;
+    hv.x = fmaf(ex2f(dl * av.x), hv.x, dx * bv.x);
+    hv.y = fmaf(ex2f(dl * av.y), hv.y, dx * bv.y);
+    hv.z = fmaf(ex2f(dl * av.z), hv.z, dx * bv.z);
+    hv.w = fmaf(ex2f(dl * av.w), hv.w, dx * bv.w);
+    float acc = fmaf(cv.x, hv.x, fmaf(cv.y, hv.y, fmaf(cv.z, hv.z, cv.w * hv.w)));
+#pragma unroll
+    for (int o = TPE / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (live) {
+        *sp = hv;
+        if (j == 0) static_cast<T*>(p.y)[e] = from_f32<T>(fmaf(Dd, xv, acc));
+    }
+}
+
 template <typename T, int N>
 cudaError_t launch_n(const SelParams& p, bool update, cudaStream_t s) {
     if (update) {
         const int64_t n = p.batch * p.channels;
+        if constexpr (N == 8 || N == 16 || N == 32) {
+            const int64_t threads = n * (N / 4);
+            return launch_kernel(sel_update_split_kernel<T, N>,
+                                 dim3(static_cast<unsigned>((threads + 255) / 256)), dim3(256), 0, s,
+                                 true, p);
+        }
         return launch_kernel(sel_update_kernel<T, N>, dim3(static_cast<unsigned>((n + 255) / 256)),
                              dim3(256), 0, s, true, p);
     }

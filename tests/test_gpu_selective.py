@@ -70,3 +70,31 @@ def test_selective_without_optional_inputs(orc):
     torch.cuda.synchronize()
     yo, _ = orc.selective_scan(inp["x"], inp["dt"], inp["A"], inp["B"], inp["C"])
     assert_close(y, yo, torch.float32, "y without D, dt_bias, init")
+
+
+@pytest.mark.parametrize("N,dtype,opt", [(4, torch.float32, True), (8, torch.bfloat16, True),
+                                         (12, torch.float32, False), (16, torch.float32, False),
+                                         (32, torch.bfloat16, True), (32, torch.float32, False)],
+                         ids=lambda v: str(v).split(".")[-1])
+def test_selective_decode_dstates(orc, N, dtype, opt):
+    """The decode step at each kernel form (one lane per channel for dstate 4
+    and 12, the states split over 2, 4 or 8 lanes for 8, 16 and 32), over 37
+    channels x 5 batch rows so the last warp holds a partial group, with and
+    without D and dt_bias."""
+    b, T, Dc = 5, 3, 37
+    inp = synthetic.make_selective_inputs(b, T, Dc, N, dtype, seed=N + 11, init_state=True)
+    if not opt:
+        inp["D"], inp["dt_bias"] = None, None
+    d = _dev(inp)
+    state = d["init_state"].clone()
+    st_o = inp["init_state"]
+    for t in range(T):
+        y = ssd.ssd_selective_state_update(state, d["x"][:, t].contiguous(), d["dt"][:, t].contiguous(),
+                                           d["A"], d["B"][:, t].contiguous(), d["C"][:, t].contiguous(),
+                                           d["D"], d["dt_bias"])
+        torch.cuda.synchronize()
+        st_o, yo = orc.selective_state_update(st_o, inp["x"][:, t], inp["dt"][:, t], inp["A"],
+                                              inp["B"][:, t], inp["C"][:, t], inp["D"],
+                                              inp["dt_bias"])
+        assert_close(y, yo, dtype, f"decode y, step {t}")
+        assert_close(state, st_o, torch.float32, f"decode state, step {t}")
