@@ -14,9 +14,10 @@
 // unit * group.  A unit is spread over LPU lanes (a power of two up to the
 // CTA's 256 threads, the smallest that leaves each lane at most MAXV
 // vectors), lane l taking vectors l, l + LPU, ... of the unit, so the lanes of
-// a unit read consecutive 16-byte pieces; the last round may be ragged.  Up to MAXV vectors per lane are kept in registers between the sum
-// of squares and the scaling; a longer unit re-reads its y and z (from L2) in
-// the second pass.  The sum of squares is a shuffle reduction over the unit's
+// a unit read consecutive 16-byte pieces; the last round may be ragged.  Up
+// to MAXV vectors per lane are kept in registers between the sum of squares
+// and the scaling; a longer unit re-reads its y and z (from L2) in the second
+// pass.  The sum of squares is a shuffle reduction over the unit's
 // lanes, plus a shared-memory step when the unit spans several warps.
 #include "gated_rmsnorm.h"
 
