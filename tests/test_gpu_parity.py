@@ -130,18 +130,25 @@ def test_steps_against_chunked_oracle(orc, dtype, Q):
 
 # ---------------------------------------------------------------------------
 # the named workloads at full size
-def test_workload_fwd_f32_small(orc):
+# each small workload at its own seed and two more (the inputs' recipe
+# repeated with three seeds)
+SEED_SHIFTS = [0, 1000, 2000]
+
+
+@pytest.mark.parametrize("shift", SEED_SHIFTS, ids=lambda v: f"seed+{v}")
+def test_workload_fwd_f32_small(orc, shift):
     cfg = synthetic.FWD_CONFIGS["fwd_f32_small"]
-    inp = synthetic.make_config_inputs(cfg)
+    inp = synthetic.make_config_inputs(cfg, 1234 + synthetic.SEED_OFFSET[cfg.name] + shift)
     y, fin = run_fwd(inp, cfg.chunk)
     yo, fo = orc.ssd_fwd(**inp)
     assert_close(y, yo, cfg.dtype, "y")
     assert_close(fin, fo, cfg.dtype, "final")
 
 
-def test_workload_fwd_bf16_b4_L1024(orc):
+@pytest.mark.parametrize("shift", SEED_SHIFTS, ids=lambda v: f"seed+{v}")
+def test_workload_fwd_bf16_b4_L1024(orc, shift):
     cfg = synthetic.FWD_CONFIGS["fwd_bf16_b4_L1024"]
-    inp = synthetic.make_config_inputs(cfg)
+    inp = synthetic.make_config_inputs(cfg, 1234 + synthetic.SEED_OFFSET[cfg.name] + shift)
     y, fin = run_fwd(inp, cfg.chunk)
     yo, fo = orc.ssd_fwd(**inp)
     assert_close(y, yo, cfg.dtype, "y")
