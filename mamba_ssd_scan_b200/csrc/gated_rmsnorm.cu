@@ -17,8 +17,8 @@
 // a unit read consecutive 16-byte pieces; the last round may be ragged.  Up
 // to MAXV vectors per lane are kept in registers between the sum of squares
 // and the scaling; a longer unit re-reads its y and z (from L2) in the second
-// pass.  The sum of squares is a shuffle reduction over the unit's
-// lanes, plus a shared-memory step when the unit spans several warps.
+// pass.  The sum of squares is a shuffle reduction over the unit's lanes,
+// plus a shared-memory step when the unit spans several warps.
 #include "gated_rmsnorm.h"
 
 namespace ssd {
