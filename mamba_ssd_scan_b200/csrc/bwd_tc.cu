@@ -409,15 +409,20 @@ struct BTile {
     static constexpr int X_OFF = Y_OFF + BLK;          // x_s
     static constexpr int B_OFF = X_OFF + BLK;          // B_s
     static constexpr int T_OFF = B_OFF + NBN * BLK;    // masked, decayed, dt-scaled dy_t . x_s, bf16 [t][s]
-    static constexpr int H_OFF = T_OFF + 2 * BLK;      // H_c, bf16 [p][n]
-    static constexpr int CS_OFF = H_OFF + NBN * 64 * 128;
+    // H_c, bf16 [p][n], staged after the source loop into the x tile, which
+    // no MMA reads any more by then; the kernel stays under half an SM's
+    // shared memory, so two CTAs share an SM (TMEM: 256 columns each)
+    static constexpr int H_OFF = X_OFF;
+    static constexpr int CS_OFF = T_OFF + 2 * BLK;
     static constexpr int SQ_OFF = CS_OFF + 2 * 256 * 4;  // [2][R] the halves' q partials, then [8] sums
     static constexpr int BAR_OFF = SQ_OFF + (2 * R + 8) * 4;
     static constexpr int BYTES = BAR_OFF + 64 + 1024;
+    static_assert(NBN * 64 * 128 <= BLK, "H_c must fit in the x tile");
+    static_assert(2 * (BYTES + 1024) <= 233472, "two CTAs of kernel B per SM");
 };
 
 template <int NST>
-__global__ void __launch_bounds__(TPB) bwd_tc_b_kernel(BwdParams bp) {
+__global__ void __launch_bounds__(TPB, 2) bwd_tc_b_kernel(BwdParams bp) {
     using T = BTile<NST>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
