@@ -46,6 +46,13 @@ __device__ __forceinline__ void cp_async_wait_all() {
     asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
+// Bring the 128-byte line holding p into L2 (no register is written, nothing
+// waits on it): data a CTA stages only later in its serial chain of phases is
+// requested at its start, so the later copies hit L2.
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // rows [r0, r0 + R) x 64-column blocks of a bf16 matrix (row stride `stride`
 // elements, `ncol` columns) into SW128 blocks at dst with asynchronous copies
 // (all in flight together); rows at or past `lim` are zero.  The caller waits
@@ -146,6 +153,18 @@ __global__ void __launch_bounds__(TPB, 1) bwd_tc_a_kernel(BwdParams bp) {
     for (int i = tid; i < Q; i += TPB) {
         scs[i] = csc[i];
         sdt[i] = dtc[i];
+    }
+    // the later target tiles' C and dy rows and the chunk's dH, into L2
+    for (int it = is + 1; it < NTT; ++it) {
+        const int r = it * R + tid;
+        if (tid < R && r < Lc) {
+            for (int cb = 0; cb < NST * 2; cb += 128) prefetch_l2(reinterpret_cast<const char*>(Cb + r * bs) + cb);
+            prefetch_l2(dyb + r * xs);
+        }
+    }
+    {
+        const float* dHp = bp.dstates + ((b * nc + c) * H + h) * static_cast<int64_t>(PD) * NST;
+        for (int i = tid; i < PD * NST / 32; i += TPB) prefetch_l2(dHp + 32 * i);
     }
     stage_tile(sB, Bb, bs, NST, s0, Lc);
     stage_tile(sX, xb, xs, PD, s0, Lc);
@@ -468,6 +487,12 @@ __global__ void __launch_bounds__(TPB, 2) bwd_tc_b_kernel(BwdParams bp) {
         sdt[i] = dtc[i];
     }
     stage_tile(sY, dyb, xs, PD, r0, Lc);
+    // the chunk's H_c (staged after the source loop) into L2
+    {
+        const __nv_bfloat16* Hp = static_cast<const __nv_bfloat16*>(p.states) +
+                                  ((b * nc + c) * H + h) * static_cast<int64_t>(PD) * NST;
+        for (int i = tid; i < PD * NST / 64; i += TPB) prefetch_l2(Hp + 64 * i);
+    }
     const uint32_t mbar = smem_u32(bar);
     uint32_t ph = 0;
     bool failed = false;
