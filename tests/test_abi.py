@@ -184,3 +184,18 @@ def test_gated_rmsnorm_rejects_bad_args(lib):
     assert lib.ssd_gated_rmsnorm(ctypes.byref(a), None) == 1      # negative eps
     a.eps, a.rows = 1e-5, 0
     assert lib.ssd_gated_rmsnorm(ctypes.byref(a), None) == 1      # no rows
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    """With the shared library absent the binding raises on the first call;
+    no entry point falls back to another implementation."""
+    import torch
+    import mamba_ssd_scan_b200 as ssd
+    monkeypatch.setattr(ssd, "_lib", None)
+    monkeypatch.setattr(ssd, "_LIB_FILE", str(tmp_path / "libssd_b200.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        ssd.load_library()
+    x = torch.zeros((1, 8, 2, 16))
+    with pytest.raises(RuntimeError, match="missing"):
+        ssd.ssd_fwd(x, torch.zeros((1, 8, 2)), torch.zeros(2), torch.zeros((1, 8, 1, 16)),
+                    torch.zeros((1, 8, 1, 16)), chunk=8)
