@@ -153,7 +153,8 @@ def test_workload_fwd_f32_small(orc, shift):
 # in that sum: a model of that rounding alone, from the oracle's chunked
 # intermediates, puts the same element at 0.88 of the bound.  The GPU result
 # is bitwise deterministic, so the case is a strict expected failure until the
-# state term takes its operand as bf16 hi + lo.
+# local states are kept in fp32 and the state term takes its operand as bf16
+# hi + lo (the CPU model shows that neither change alone removes it).
 HEADLINE_SEED_CASES = [0, pytest.param(1000, marks=pytest.mark.xfail(
     strict=True, reason="bf16 chunk state in the state term under cancellation")), 2000]
 
