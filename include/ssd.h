@@ -13,8 +13,11 @@
  *
  * with A_h a scalar per head (normally negative), B_t, C_t shared by the heads
  * of a group (head h reads group h / (nheads / ngroups)).  The forward pass
- * computes this chunkwise: chunk_cumsum -> chunk_state -> state_passing ->
- * chunk_scan, the chunked SSD of "MAMBA-2 Implementation Gaps", Gap 1.
+ * computes this chunkwise, the chunked SSD of "MAMBA-2 Implementation Gaps",
+ * Gap 1: chunk_cumsum -> chunk_state -> state_passing -> chunk_scan.  For bf16
+ * inputs in its range the four steps run as one fused kernel (the carried
+ * state stays fp32 and crosses between chunks through a small ring in the
+ * workspace); otherwise as the four step kernels below.
  *
  * Layouts: row-major, innermost index last, densely packed (no strides):
  *   x, y          [batch, seqlen, nheads, headdim]     dtype
@@ -77,12 +80,13 @@ typedef enum { SSD_F32 = 0, SSD_BF16 = 1 } ssd_dtype;
  *                and 6.1), applied in the kernel that writes y.  The gate does
  *                not touch the carried state.
  * Supported: 1 <= chunk <= 256; dstate a multiple of 4, <= 256; headdim a
- * multiple of 4.  bf16 inputs run the contractions on the tensor cores
- * (tcgen05) where the shape allows -- chunk_state: headdim in {32, 64, 128},
- * dstate in {64, 128, 256}, 128/headdim dividing the heads per group;
- * chunk_scan: headdim 64, dstate in {64, 128}, chunk in {128, 256} -- and on
- * the CUDA cores (fp32 FFMA) otherwise; fp32 inputs always take the CUDA-core
- * path (its exact fp32 arithmetic is what the 1e-4 agreement needs). */
+ * multiple of 4.  bf16 inputs with headdim 64, dstate 64 or 128 and chunk 128
+ * or 256 run the whole forward as one tensor-core (tcgen05) kernel; other bf16
+ * shapes run the step kernels with chunk_state on the tensor cores where it
+ * applies (headdim in {32, 64, 128}, dstate in {64, 128, 256}, 128/headdim
+ * dividing the heads per group) and the rest in fp32 on the CUDA cores; fp32
+ * inputs always take the CUDA-core path (its exact fp32 arithmetic is what the
+ * 1e-4 agreement needs). */
 typedef struct {
     int64_t batch, seqlen, nheads, headdim, dstate, ngroups, chunk;
     int32_t dtype;          /* ssd_dtype of x, dt, B, C and y */
@@ -104,18 +108,31 @@ typedef struct {
 
 /* flags */
 #define SSD_FLAG_CUDA_CORES 1   /* force the CUDA-core (FFMA) path */
-#define SSD_FLAG_WHOLE_GROUPS 2 /* tensor-core chunk_scan: one CTA per whole group
-                                   of heads (fewest B/C reads, fewest CTAs) */
+#define SSD_FLAG_WHOLE_GROUPS 2 /* tensor-core chunk_scan (bf16-states mode): one CTA
+                                   per whole group of heads */
+#define SSD_FLAG_SPLIT_STEPS 4  /* bf16: run the forward as its separate step
+                                   kernels (chunk states in fp32 in the workspace)
+                                   instead of the single fused kernel; for
+                                   comparisons and the per-step checks */
+#define SSD_FLAG_BF16_STATES 8  /* bf16, opt-in: the split steps with the chunk
+                                   states stored in bf16 and the carried state
+                                   entering the tensor-core state term as one bf16
+                                   operand.  Faster than the split fp32 steps but
+                                   OUTSIDE the stated bf16 tolerance for some inputs
+                                   (the carried state's rounding under cancellation
+                                   in C . H); never the default */
 
 /* Bytes of device workspace ssd_fwd needs for these sizes (0 on invalid
  * sizes).  Only sizes, dtype and flags are read; pointers may be NULL. */
 size_t ssd_fwd_workspace_size(const ssd_fwd_args* args);
 
 /* Which steps of ssd_fwd run on the tensor cores for these sizes, dtype and
- * flags: bit 0 = chunk_state, bit 1 = chunk_scan (0 = all on CUDA cores, or
- * invalid sizes).  Host-only; pointers are not read. */
+ * flags: bit 0 = chunk_state, bit 1 = chunk_scan, bit 2 = the whole forward in
+ * one fused kernel (0 = all on CUDA cores, or invalid sizes).  Host-only;
+ * pointers are not read. */
 #define SSD_TC_CHUNK_STATE 1
 #define SSD_TC_CHUNK_SCAN 2
+#define SSD_TC_FUSED 4
 int ssd_fwd_tensor_core_steps(const ssd_fwd_args* args);
 
 /* The whole forward scan: y (and final_state) from x, dt, A, B, C, D,
@@ -150,16 +167,17 @@ ssd_status ssd_fwd_no_alloc(const ssd_fwd_args* args, void* stream);
 /* Synchronises `stream` and returns the device status of the last ssd_fwd
  * call that used this workspace: SSD_OK, or SSD_ERR_TIMEOUT when a kernel gave
  * up on a bounded wait (it then stops early and its outputs are invalid).
- * Each ssd_fwd call resets the status at its start. */
+ * Each ssd_fwd call resets the status at its start.  The status word is the
+ * workspace's first 4 bytes in every path. */
 ssd_status ssd_fwd_check_status(const ssd_fwd_args* args, void* stream);
 
 /* ---- the four steps of ssd_fwd, exported one by one -------------------- */
 /* Each reads the fields of `args` it needs and the intermediate buffers named
  * in its signature (device, caller-owned, 16-byte aligned):
  *   dt_out, cumA_out  [batch, nheads, nc, chunk]                 fp32
- *   states            [batch, nc, nheads, headdim, dstate]       in args->dtype
- * (chunk states are stored in the input dtype -- bf16 for bf16 inputs -- and
- * accumulated in fp32; the carry across chunks is fp32 in registers).
+ *   states            [batch, nc, nheads, headdim, dstate]       fp32
+ * (with SSD_FLAG_BF16_STATES and bf16 inputs, `states` is bf16 instead; the
+ * carry across chunks is fp32 in registers either way).
  */
 
 /* Step 1: dt = softplus(dt_raw + dt_bias) and the inclusive in-chunk

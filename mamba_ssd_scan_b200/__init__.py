@@ -19,6 +19,8 @@ __all__ = [
     "ssd_fwd_tensor_core_steps", "tensor_core_steps", "ssd_chunk_cumsum", "ssd_chunk_state",
     "ssd_state_passing", "ssd_chunk_scan", "ssd_state_update", "ssd_status_string",
     "ssd_version", "lib_path", "load_library", "SSD_FLAG_CUDA_CORES", "SSD_FLAG_WHOLE_GROUPS",
+    "SSD_FLAG_SPLIT_STEPS", "SSD_FLAG_BF16_STATES", "SSD_TC_CHUNK_STATE", "SSD_TC_CHUNK_SCAN",
+    "SSD_TC_FUSED",
     "ssd_causal_conv1d", "ssd_conv1d_update", "ssd_conv1d_check_status",
     "ssd_bwd", "ssd_bwd_workspace_size", "ssd_selective_scan", "ssd_selective_scan_workspace_size",
     "ssd_selective_state_update", "ssd_gated_rmsnorm",
@@ -31,6 +33,9 @@ SSD_OK, SSD_ERR_INVALID_ARG, SSD_ERR_UNSUPPORTED, SSD_ERR_CUDA, SSD_ERR_TIMEOUT 
 SSD_F32, SSD_BF16 = 0, 1
 SSD_FLAG_CUDA_CORES = 1
 SSD_FLAG_WHOLE_GROUPS = 2
+SSD_FLAG_SPLIT_STEPS = 4
+SSD_FLAG_BF16_STATES = 8
+SSD_TC_CHUNK_STATE, SSD_TC_CHUNK_SCAN, SSD_TC_FUSED = 1, 2, 4
 
 _i64, _i32, _vp, _sz = ctypes.c_int64, ctypes.c_int32, ctypes.c_void_p, ctypes.c_size_t
 
@@ -248,7 +253,7 @@ def ssd_fwd_workspace_size(batch, seqlen, nheads, headdim, dstate, ngroups, chun
 def ssd_fwd_tensor_core_steps(batch, seqlen, nheads, headdim, dstate, ngroups, chunk,
                               dtype=torch.bfloat16, flags: int = 0) -> int:
     """Bitmask of the ssd_fwd steps that run on the tensor cores for these sizes
-    (1 = chunk_state, 2 = chunk_scan)."""
+    (1 = chunk_state, 2 = chunk_scan, 4 = the whole forward as one fused kernel)."""
     a = SsdFwdArgs()
     a.batch, a.seqlen, a.nheads, a.headdim, a.dstate, a.ngroups, a.chunk = (
         batch, seqlen, nheads, headdim, dstate, ngroups, chunk)
@@ -262,7 +267,7 @@ def tensor_core_steps(batch, seqlen, nheads, headdim, dstate, ngroups, chunk,
     """Names of the ssd_fwd steps that run on the tensor cores for these sizes."""
     m = ssd_fwd_tensor_core_steps(batch, seqlen, nheads, headdim, dstate, ngroups, chunk,
                                   dtype, flags)
-    return {n for bit, n in ((1, "chunk_state"), (2, "chunk_scan")) if m & bit}
+    return {n for bit, n in ((1, "chunk_state"), (2, "chunk_scan"), (4, "fused")) if m & bit}
 
 
 def ssd_fwd(x, dt, A, B, C, D=None, dt_bias=None, chunk: int = 256, init_state=None, *,
@@ -399,6 +404,13 @@ def _intermediate_shapes(x, B, chunk):
     return (b, H, nc, chunk), (b, nc, H, P, N)
 
 
+def _states_dtype(x, flags):
+    """The chunk states are fp32, except bf16 inputs in the bf16-states mode."""
+    if x.dtype == torch.bfloat16 and flags & SSD_FLAG_BF16_STATES:
+        return torch.bfloat16
+    return torch.float32
+
+
 def ssd_chunk_cumsum(x, dt, A, B, C, dt_bias=None, chunk: int = 256, *, dt_out=None,
                      cumA_out=None, stream=None):
     """Step 1: returns (dt, cumA), each [b, H, nc, chunk] float32."""
@@ -414,37 +426,38 @@ def ssd_chunk_cumsum(x, dt, A, B, C, dt_bias=None, chunk: int = 256, *, dt_out=N
 
 
 def ssd_chunk_state(x, dt, A, B, C, dt_sp, cumA, chunk: int = 256, *, states=None,
-                    stream=None):
-    """Step 2: returns the chunk-local states [b, nc, H, P, N] in x's dtype.
-    ``dt_sp``/``cumA`` are step 1's outputs."""
+                    stream=None, flags: int = 0):
+    """Step 2: returns the chunk-local states [b, nc, H, P, N], fp32 (bf16 for
+    bf16 inputs with SSD_FLAG_BF16_STATES).  ``dt_sp``/``cumA`` are step 1's
+    outputs."""
     lib = load_library()
     _, sshape = _intermediate_shapes(x, B, chunk)
-    states = states if states is not None else torch.empty(sshape, dtype=x.dtype,
-                                                           device=x.device)
-    a = _fwd_args(x, dt, A, B, C, None, None, chunk, None, None, None, 0)
+    states = states if states is not None else torch.empty(
+        sshape, dtype=_states_dtype(x, flags), device=x.device)
+    a = _fwd_args(x, dt, A, B, C, None, None, chunk, None, None, None, flags)
     _check(lib.ssd_chunk_state(ctypes.byref(a), _ptr(dt_sp), _ptr(cumA), _ptr(states),
                                _stream_ptr(stream)), "ssd_chunk_state")
     return states
 
 
 def ssd_state_passing(x, dt, A, B, C, cumA, states, chunk: int = 256, init_state=None,
-                      final_state=None, stream=None):
+                      final_state=None, stream=None, flags: int = 0):
     """Step 3, in place: ``states`` goes from chunk-local states to the states
     entering each chunk.  Writes ``final_state`` if given.  Returns states."""
     lib = load_library()
-    a = _fwd_args(x, dt, A, B, C, None, None, chunk, init_state, None, final_state, 0)
+    a = _fwd_args(x, dt, A, B, C, None, None, chunk, init_state, None, final_state, flags)
     _check(lib.ssd_state_passing(ctypes.byref(a), _ptr(cumA), _ptr(states),
                                  _stream_ptr(stream)), "ssd_state_passing")
     return states
 
 
 def ssd_chunk_scan(x, dt, A, B, C, dt_sp, cumA, states, D=None, chunk: int = 256, *, y=None,
-                   stream=None, z=None):
+                   stream=None, z=None, flags: int = 0):
     """Step 4: y from the chunk's tokens and the states entering each chunk
     (times silu(z) when the gate z is given)."""
     lib = load_library()
     y = y if y is not None else torch.empty_like(x)
-    a = _fwd_args(x, dt, A, B, C, D, None, chunk, None, y, None, 0, z)
+    a = _fwd_args(x, dt, A, B, C, D, None, chunk, None, y, None, flags, z)
     _check(lib.ssd_chunk_scan(ctypes.byref(a), _ptr(dt_sp), _ptr(cumA), _ptr(states),
                               _stream_ptr(stream)), "ssd_chunk_scan")
     return y

@@ -45,10 +45,16 @@ struct WsLayout {
     size_t status, dt, cumA, states, total;
 };
 
+// Chunk states in the split-step path are fp32, except in the opt-in
+// bf16-states mode (bf16 inputs with SSD_FLAG_BF16_STATES).
+bool bf16_states(const ssd_fwd_args& a) {
+    return a.dtype == SSD_BF16 && (a.flags & SSD_FLAG_BF16_STATES) != 0;
+}
+
 WsLayout ws_layout(const ssd_fwd_args& a) {
     const int64_t nc = (a.seqlen + a.chunk - 1) / a.chunk;
     const size_t vec = (size_t)a.batch * a.nheads * nc * a.chunk * sizeof(float);
-    const size_t elt = a.dtype == SSD_BF16 ? 2 : 4;  // chunk states are kept in the input dtype
+    const size_t elt = bf16_states(a) ? 2 : 4;
     const size_t st = (size_t)a.batch * nc * a.nheads * a.headdim * a.dstate * elt;
     WsLayout w;
     w.status = 0;
@@ -100,6 +106,7 @@ FwdParams make_params(const ssd_fwd_args* a) {
     p.flags = a->flags;
     p.pdl = 0;
     p.fuse_cumsum = 0;
+    p.states_f32 = bf16_states(*a) ? 0 : 1;
     p.x = a->x;
     p.dt_raw = a->dt;
     p.A = a->A;
@@ -115,6 +122,14 @@ FwdParams make_params(const ssd_fwd_args* a) {
     p.states = nullptr;
     p.status = nullptr;
     return p;
+}
+
+// The whole forward in one kernel: bf16 inputs in its shape range, unless the
+// caller asks for the CUDA cores, the split steps or the bf16-states mode.
+bool use_fused(const ssd_fwd_args& a) {
+    if (a.dtype != SSD_BF16) return false;
+    if (a.flags & (SSD_FLAG_CUDA_CORES | SSD_FLAG_SPLIT_STEPS | SSD_FLAG_BF16_STATES)) return false;
+    return ssd::fused_fwd_supported(make_params(&a));
 }
 
 // the last CUDA error a call of this library saw, per host thread
@@ -135,9 +150,10 @@ cudaError_t run_cumsum(const FwdParams& p, int dtype, cudaStream_t s) {
 bool use_tc(int dtype, int flags) {
     return dtype == SSD_BF16 && (flags & SSD_FLAG_CUDA_CORES) == 0;
 }
+// state passing is templated on the type the states are stored in
 cudaError_t run_state_passing(const FwdParams& p, int dtype, cudaStream_t s) {
-    return dtype == SSD_BF16 ? ssd::launch_state_passing<__nv_bfloat16>(p, s)
-                             : ssd::launch_state_passing<float>(p, s);
+    return (dtype == SSD_BF16 && !p.states_f32) ? ssd::launch_state_passing<__nv_bfloat16>(p, s)
+                                                : ssd::launch_state_passing<float>(p, s);
 }
 cudaError_t run_chunk_state(const FwdParams& p, int dtype, int flags, cudaStream_t s) {
     if (use_tc(dtype, flags) && ssd::chunk_state_tc_supported(p))
@@ -145,8 +161,11 @@ cudaError_t run_chunk_state(const FwdParams& p, int dtype, int flags, cudaStream
     return dtype == SSD_BF16 ? ssd::launch_chunk_state_ffma<__nv_bfloat16>(p, s)
                              : ssd::launch_chunk_state_ffma<float>(p, s);
 }
+// The tensor-core chunk_scan takes its carried state as one bf16 operand, so
+// it runs only in the opt-in bf16-states mode; with fp32 states the CUDA-core
+// kernel forms the state term in fp32.
 cudaError_t run_chunk_scan(const FwdParams& p, int dtype, int flags, cudaStream_t s) {
-    if (use_tc(dtype, flags) && ssd::chunk_scan_tc_supported(p))
+    if (use_tc(dtype, flags) && !p.states_f32 && ssd::chunk_scan_tc_supported(p))
         return ssd::launch_chunk_scan_tc(p, s);
     return dtype == SSD_BF16 ? ssd::launch_chunk_scan_ffma<__nv_bfloat16>(p, s)
                              : ssd::launch_chunk_scan_ffma<float>(p, s);
@@ -257,14 +276,16 @@ extern "C" {
 
 size_t ssd_fwd_workspace_size(const ssd_fwd_args* args) {
     if (check_fwd_sizes(args) != SSD_OK) return 0;
+    if (use_fused(*args)) return ssd::fused_fwd_workspace_bytes(make_params(args));
     return ws_layout(*args).total;
 }
 
 int ssd_fwd_tensor_core_steps(const ssd_fwd_args* a) {
     if (check_fwd_sizes(a) != SSD_OK || !use_tc(a->dtype, a->flags)) return 0;
+    if (use_fused(*a)) return SSD_TC_CHUNK_STATE | SSD_TC_CHUNK_SCAN | SSD_TC_FUSED;
     const FwdParams p = make_params(a);
     return (ssd::chunk_state_tc_supported(p) ? SSD_TC_CHUNK_STATE : 0) |
-           (ssd::chunk_scan_tc_supported(p) ? SSD_TC_CHUNK_SCAN : 0);
+           ((!p.states_f32 && ssd::chunk_scan_tc_supported(p)) ? SSD_TC_CHUNK_SCAN : 0);
 }
 
 ssd_status ssd_fwd(const ssd_fwd_args* a, void* stream) {
@@ -273,6 +294,14 @@ ssd_status ssd_fwd(const ssd_fwd_args* a, void* stream) {
     if ((st = check_fwd_inputs(a)) != SSD_OK) return st;
     if (!check_ptr(a->y, false, true) || !check_ptr(a->final_state, true, true))
         return SSD_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (use_fused(*a)) {
+        FwdParams p = make_params(a);
+        if (!a->workspace || a->workspace_bytes < ssd::fused_fwd_workspace_bytes(p) ||
+            !check_ptr(a->workspace, false, true))
+            return SSD_ERR_INVALID_ARG;
+        return to_status(ssd::launch_fused_fwd(p, a->workspace, s));
+    }
     const WsLayout w = ws_layout(*a);
     if (!a->workspace || a->workspace_bytes < w.total || !check_ptr(a->workspace, false, true))
         return SSD_ERR_INVALID_ARG;
@@ -282,7 +311,6 @@ ssd_status ssd_fwd(const ssd_fwd_args* a, void* stream) {
     p.cumA = reinterpret_cast<float*>(ws + w.cumA);
     p.states = ws + w.states;
     p.status = reinterpret_cast<int*>(ws + w.status);
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
     // The first kernel is a plain launch (it waits for all earlier work on
     // the stream); the later ones go out with programmatic dependent launch,
     // so their set-up overlaps the previous kernel's tail.  The tensor-core
@@ -306,12 +334,13 @@ ssd_status ssd_fwd(const ssd_fwd_args* a, void* stream) {
 ssd_status ssd_fwd_check_status(const ssd_fwd_args* a, void* stream) {
     ssd_status st = check_fwd_sizes(a);
     if (st != SSD_OK) return st;
-    const WsLayout w = ws_layout(*a);
-    if (!a->workspace || a->workspace_bytes < w.total || !check_ptr(a->workspace, false, true))
+    // both layouts keep the status word at the start of the workspace
+    const size_t need = ssd_fwd_workspace_size(a);
+    if (!a->workspace || a->workspace_bytes < need || !check_ptr(a->workspace, false, true))
         return SSD_ERR_INVALID_ARG;
     int v = 0;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (cudaMemcpyAsync(&v, static_cast<char*>(a->workspace) + w.status, sizeof(int),
+    if (cudaMemcpyAsync(&v, static_cast<char*>(a->workspace), sizeof(int),
                         cudaMemcpyDeviceToHost, s) != cudaSuccess ||
         cudaStreamSynchronize(s) != cudaSuccess)
         return SSD_ERR_CUDA;
@@ -339,6 +368,7 @@ ssd_status ssd_bwd(const ssd_bwd_args* a, void* stream) {
         return SSD_ERR_INVALID_ARG;
     char* ws = static_cast<char*>(a->workspace);
     FwdParams p = make_params(&f);
+    p.states_f32 = 0;  // the recompute keeps its states in the input dtype
     p.dt = reinterpret_cast<float*>(ws + w.dt);
     p.cumA = reinterpret_cast<float*>(ws + w.cumA);
     p.states = ws + w.states;

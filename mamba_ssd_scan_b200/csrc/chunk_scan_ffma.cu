@@ -42,7 +42,11 @@ __global__ void __launch_bounds__(256) chunk_scan_ffma_kernel(FwdParams p) {
     const T* x = static_cast<const T*>(p.x);
     const T* Bm = static_cast<const T*>(p.B);
     const T* Cm = static_cast<const T*>(p.C);
-    const T* Hin = static_cast<const T*>(p.states) + ((b * nc + c) * H + h) * P * N;
+    // the state entering the chunk, fp32 or in the input dtype
+    const int64_t sbase = ((b * nc + c) * H + h) * P * N;
+    const float* Hin32 = static_cast<const float*>(p.states) + sbase;
+    const T* HinT = static_cast<const T*>(p.states) + sbase;
+    auto hin = [&](int64_t i) { return p.states_f32 ? Hin32[i] : to_f32(HinT[i]); };
     const int64_t SN = cs_stride(N);
 
     extern __shared__ float smem[];
@@ -68,7 +72,7 @@ __global__ void __launch_bounds__(256) chunk_scan_ffma_kernel(FwdParams p) {
         for (int i = tid; i < TJ * TPP; i += 256) {
             const int kk = i / TPP, pp = i % TPP;
             const int64_t n = n0 + kk, pi = p0 + pp;
-            Xs[kk * TPP + pp] = (n < N && pi < P) ? to_f32(Hin[pi * N + n]) : 0.0f;
+            Xs[kk * TPP + pp] = (n < N && pi < P) ? hin(pi * N + n) : 0.0f;
         }
         __syncthreads();
         const int64_t kmax = (N - n0 < TJ) ? (N - n0) : TJ;

@@ -75,13 +75,20 @@ __global__ void __launch_bounds__(256) chunk_state_ffma_kernel(FwdParams p) {
         }
         __syncthreads();
     }
-    T* out = static_cast<T*>(p.states) + ((b * nc + c) * H + h) * P * N;
+    const int64_t sbase = ((b * nc + c) * H + h) * P * N;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const int64_t pi = p0 + ty * 4 + i, nj = n0 + tx * 4;
         if (pi < P && nj < N) {
+            if (p.states_f32) {
+                float* out = static_cast<float*>(p.states) + sbase;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) out[pi * N + nj + j] = from_f32<T>(acc[i][j]);
+                for (int j = 0; j < 4; ++j) out[pi * N + nj + j] = acc[i][j];
+            } else {
+                T* out = static_cast<T*>(p.states) + sbase;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) out[pi * N + nj + j] = from_f32<T>(acc[i][j]);
+            }
         }
     }
 }

@@ -16,9 +16,9 @@
 // while the previous quarter is scaled and multiplied (mbarriers per slot:
 // loaded, scaled, free).  With 64 KB of shared memory (dstate 128) three CTAs
 // share an SM, so one CTA's loads overlap another's MMAs and epilogue.  The
-// epilogue moves the fp32
-// accumulator from TMEM to the states buffer in the input dtype (bf16), one
-// row of dstate per thread.  When the forward call fuses step 1, the first
+// epilogue moves the fp32 accumulator from TMEM to the states buffer, in fp32
+// (the forward's split-step path) or bf16 (the backward's recompute and the
+// opt-in bf16-states mode), one row of dstate per thread.  When the forward call fuses step 1, the first
 // 128/P warps first form dt and cumA of the CTA's heads with the same warp
 // scan as step 1 and store them for steps 3 and 4.
 #include "internal.cuh"
@@ -187,21 +187,27 @@ __global__ void __launch_bounds__(NTHR, NST == 256 ? 2 : 3)  // CTAs per SM that
             // warp w reads TMEM lanes 32*(w%4).. (rows m), warpgroup w/4 half the columns
             const int m = 32 * (warp & 3) + lane;
             const int64_t hh = m / PD, pp = m % PD;
-            __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.states) +
-                                 (((b * nc + c) * H + h0 + hh) * PD + pp) * NST;
+            const int64_t row = (((b * nc + c) * H + h0 + hh) * PD + pp) * NST;
             constexpr int HALF = NST / 2;
             const int cbeg = (warp >> 2) * HALF;
 #pragma unroll
             for (int col = 0; col < HALF; col += 32) {
                 float v[32];
                 tmem_ld32(tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + cbeg + col, v);
-                uint4* o = reinterpret_cast<uint4*>(out + cbeg + col);
+                if (p.states_f32) {  // fp32 states, as the forward keeps them
+                    float4* o = reinterpret_cast<float4*>(static_cast<float*>(p.states) + row + cbeg + col);
 #pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    o[k] = make_uint4(pack_bf16x2(v[8 * k], v[8 * k + 1]),
-                                      pack_bf16x2(v[8 * k + 2], v[8 * k + 3]),
-                                      pack_bf16x2(v[8 * k + 4], v[8 * k + 5]),
-                                      pack_bf16x2(v[8 * k + 6], v[8 * k + 7]));
+                    for (int k = 0; k < 8; ++k)
+                        o[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+                } else {
+                    uint4* o = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.states) + row + cbeg + col);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        o[k] = make_uint4(pack_bf16x2(v[8 * k], v[8 * k + 1]),
+                                          pack_bf16x2(v[8 * k + 2], v[8 * k + 3]),
+                                          pack_bf16x2(v[8 * k + 4], v[8 * k + 5]),
+                                          pack_bf16x2(v[8 * k + 6], v[8 * k + 7]));
+                }
             }
         }
     }

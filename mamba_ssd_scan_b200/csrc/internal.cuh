@@ -20,6 +20,9 @@ struct FwdParams {
     // chunk_state forms dt and cumA itself (fusing step 1)
     int32_t pdl;
     int32_t fuse_cumsum;
+    // chunk states (workspace and step entry points) in fp32 (1) or in the
+    // input dtype (0: the backward's recompute, and the opt-in bf16-states mode)
+    int32_t states_f32;
     const void* x;
     const void* dt_raw;
     const float* A;
@@ -34,7 +37,7 @@ struct FwdParams {
     // intermediates (workspace)
     float* dt;      // [b, H, nc, Q]
     float* cumA;    // [b, H, nc, Q]
-    void* states;   // [b, nc, H, P, N] in the input dtype (local states, then states entering each chunk)
+    void* states;   // [b, nc, H, P, N] in fp32 or the input dtype (states_f32): local states, then states entering each chunk
     int* status;    // device status word (SSD_ERR_TIMEOUT on a timed-out wait); may be null
 };
 
@@ -229,5 +232,11 @@ bool chunk_state_tc_supported(const FwdParams& p);
 cudaError_t launch_chunk_state_tc(const FwdParams& p, cudaStream_t s);
 bool chunk_scan_tc_supported(const FwdParams& p);
 cudaError_t launch_chunk_scan_tc(const FwdParams& p, cudaStream_t s);
+// The whole forward in one kernel (fused_fwd.cu): bf16, headdim 64, dstate 64
+// or 128, chunk 128 or 256.  The workspace is its own (fused_fwd_workspace_bytes,
+// 16-byte aligned) and is zeroed by the launch itself; status goes to its first word.
+bool fused_fwd_supported(const FwdParams& p);
+size_t fused_fwd_workspace_bytes(const FwdParams& p);
+cudaError_t launch_fused_fwd(const FwdParams& p, void* ws, cudaStream_t s);
 
 }  // namespace ssd

@@ -43,9 +43,19 @@ def test_tensor_core_dispatch_query(lib):
     import torch
 
     import mamba_ssd_scan_b200 as m
-    assert m.tensor_core_steps(4, 1024, 24, 64, 64, 1, 256) == {"chunk_state", "chunk_scan"}
+    # bf16 in the fused kernel's range: the whole forward in one tensor-core kernel
+    assert m.tensor_core_steps(4, 1024, 24, 64, 64, 1, 256) == {"chunk_state", "chunk_scan", "fused"}
+    assert m.tensor_core_steps(1, 65536, 80, 64, 128, 8, 256) == {"chunk_state", "chunk_scan", "fused"}
+    assert m.tensor_core_steps(1, 300, 4, 64, 128, 4, 128) == {"chunk_state", "chunk_scan", "fused"}
     assert m.tensor_core_steps(4, 1024, 24, 64, 64, 1, 256, torch.float32) == set()
     assert m.tensor_core_steps(4, 1024, 24, 64, 64, 1, 256, flags=m.SSD_FLAG_CUDA_CORES) == set()
+    # the split steps keep fp32 chunk states: chunk_state on the tensor cores, the
+    # state term of chunk_scan in fp32 on the CUDA cores
+    assert m.tensor_core_steps(4, 1024, 24, 64, 64, 1, 256, flags=m.SSD_FLAG_SPLIT_STEPS) == {
+        "chunk_state"}
+    # the opt-in bf16-states mode takes the tensor-core chunk_scan
+    assert m.tensor_core_steps(4, 1024, 24, 64, 64, 1, 256, flags=m.SSD_FLAG_BF16_STATES) == {
+        "chunk_state", "chunk_scan"}
     assert m.tensor_core_steps(1, 512, 2, 128, 256, 1, 256) == {"chunk_state"}
     assert m.tensor_core_steps(1, 512, 4, 64, 128, 4, 64) == set()  # 1 head per group, chunk 64
 
@@ -68,8 +78,14 @@ def _args(**kw):
 
 
 def test_workspace_size_is_host_only(lib):
-    a = _args()
-    # status word (256 B) + dt + cumA: 1*4*2*256 fp32 each + states 1*2*4*64*64 bf16
+    import mamba_ssd_scan_b200 as m
+    # fused kernel: header (256 B) + a two-slot ring of 1*4 states of 64*64 fp32
+    assert lib.ssd_fwd_workspace_size(ctypes.byref(_args())) == 256 + 2 * 4 * 64 * 64 * 4
+    # split steps: header + dt + cumA (1*4*2*256 fp32 each) + fp32 chunk states 1*2*4*64*64
+    a = _args(flags=m.SSD_FLAG_SPLIT_STEPS)
+    assert lib.ssd_fwd_workspace_size(ctypes.byref(a)) == 256 + 8192 + 8192 + 131072
+    # bf16-states mode: the chunk states in bf16
+    a = _args(flags=m.SSD_FLAG_BF16_STATES)
     assert lib.ssd_fwd_workspace_size(ctypes.byref(a)) == 256 + 8192 + 8192 + 65536
     assert lib.ssd_fwd_workspace_size(None) == 0
     assert lib.ssd_fwd_workspace_size(ctypes.byref(_args(nheads=3, ngroups=2))) == 0

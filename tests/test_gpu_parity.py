@@ -145,18 +145,12 @@ def test_workload_fwd_f32_small(orc, shift):
     assert_close(fin, fo, cfg.dtype, "final")
 
 
-# At seed+1000 three of the 6.3 M y elements (first tokens of a chunk, where y
-# is almost all of the state term e^{cumA} C . H_in) exceed the elementwise
-# bf16 bound by up to 14 %; the tensor-wide bound holds with a 15x margin.
-# The state entering a chunk is held in bf16 between the kernels and enters
-# the tensor-core state term as bf16, and its entries (up to ~67 here) cancel
-# in that sum: a model of that rounding alone, from the oracle's chunked
-# intermediates, puts the same element at 0.88 of the bound.  The GPU result
-# is bitwise deterministic, so the case is a strict expected failure until the
-# local states are kept in fp32 and the state term takes its operand as bf16
-# hi + lo (the CPU model shows that neither change alone removes it).
-HEADLINE_SEED_CASES = [0, pytest.param(1000, marks=pytest.mark.xfail(
-    strict=True, reason="bf16 chunk state in the state term under cancellation")), 2000]
+# Five seeds of the b4 L1024 workload, every element against the bf16 bound.
+# At seed+1000 the state term e^{cumA} C . H_in cancels strongly at a chunk's
+# first tokens (state entries up to ~67): the carried state must stay fp32 and
+# enter the tensor cores as bf16 hi + lo, and the intra-chunk mask needs more
+# than bf16's 8 bits, which the fused forward keeps.
+HEADLINE_SEED_CASES = [0, 1000, 2000, 3000, 4000]
 
 
 @pytest.mark.parametrize("shift", HEADLINE_SEED_CASES, ids=lambda v: f"seed+{v}")
@@ -169,13 +163,14 @@ def test_workload_fwd_bf16_b4_L1024(orc, shift):
     assert_close(fin, fo, cfg.dtype, "final")
 
 
+@pytest.mark.parametrize("shift", [0, 1000, 2000], ids=lambda v: f"seed+{v}")
 @pytest.mark.parametrize("name,heads,batches", [
     ("fwd_bf16_b8_L4096_init", [0, 13, 31], [0, 7]),
     ("fwd_bf16_b1_L65536_G8", [0, 9, 10, 47, 79], None),
 ])
-def test_workload_sampled_heads(orc, name, heads, batches):
+def test_workload_sampled_heads(orc, name, heads, batches, shift):
     cfg = synthetic.FWD_CONFIGS[name]
-    inp = synthetic.make_config_inputs(cfg)
+    inp = synthetic.make_config_inputs(cfg, 1234 + synthetic.SEED_OFFSET[cfg.name] + shift)
     y, fin = run_fwd(inp, cfg.chunk)
     yo, fo = oracle_heads(orc, inp, heads, batches)
     bsel = slice(None) if batches is None else batches
@@ -202,8 +197,8 @@ def test_decode_small(orc, N, dtype):
                                       prm["D"], prm["dt_bias"])
         torch.cuda.synchronize()
         assert_close(y, yo, dtype, f"y step {step}")
-        assert_close(st_gpu, st_ref, torch.float32 if dtype == torch.float32 else dtype,
-                     f"state step {step}")
+        # the state is fp32 arithmetic on exactly representable inputs: fp32 rule
+        assert_close(st_gpu, st_ref, torch.float32, f"state step {step}")
 
 
 def test_decode_workload_1024_steps_sampled(orc):
@@ -263,19 +258,37 @@ TC_CASES = [
 
 @pytest.mark.parametrize("case", TC_CASES, ids=lambda c: "b{}_L{}_H{}_P{}_N{}_G{}_Q{}".format(*c))
 def test_tensor_core_path(orc, case):
+    """The default bf16 path (the fused kernel where the shape allows), the
+    split steps with fp32 chunk states, and the CUDA cores, each against the
+    oracle."""
     b, L, H, P, N, G, Q = case
     inp = synthetic.make_fwd_inputs(b, L, H, P, N, G, torch.bfloat16, seed=L + N,
                                     init_state=True)
     y_tc, f_tc = run_fwd(inp, Q)
-    y_wg, f_wg = run_fwd(inp, Q, flags=ssd.SSD_FLAG_WHOLE_GROUPS)
+    y_sp, f_sp = run_fwd(inp, Q, flags=ssd.SSD_FLAG_SPLIT_STEPS)
     y_cc, f_cc = run_fwd(inp, Q, flags=ssd.SSD_FLAG_CUDA_CORES)
     yo, fo = orc.ssd_fwd(**inp)
-    assert_close(y_tc, yo, torch.bfloat16, "tensor-core y")
-    assert_close(f_tc, fo, torch.bfloat16, "tensor-core final")
-    assert_close(y_wg, yo, torch.bfloat16, "tensor-core y, whole groups per CTA")
-    assert torch.equal(f_wg, f_tc)  # the head blocking changes only chunk_scan
+    assert_close(y_tc, yo, torch.bfloat16, "default y")
+    assert_close(f_tc, fo, torch.bfloat16, "default final")
+    assert_close(y_sp, yo, torch.bfloat16, "split-step y")
+    assert_close(f_sp, fo, torch.bfloat16, "split-step final")
     assert_close(y_cc, yo, torch.bfloat16, "CUDA-core y")
     assert_close(f_cc, fo, torch.bfloat16, "CUDA-core final")
+
+
+@pytest.mark.parametrize("case", TC_CASES[:3], ids=lambda c: "b{}_L{}_H{}_P{}_N{}_G{}_Q{}".format(*c))
+def test_bf16_states_mode_runs(orc, case):
+    """The opt-in bf16-states mode (split steps, chunk states in bf16, the
+    tensor-core chunk_scan) is outside the stated tolerance for some inputs:
+    it is held here only to the tensor-wide form of the bound."""
+    b, L, H, P, N, G, Q = case
+    inp = synthetic.make_fwd_inputs(b, L, H, P, N, G, torch.bfloat16, seed=L + N,
+                                    init_state=True)
+    for flags in (ssd.SSD_FLAG_BF16_STATES, ssd.SSD_FLAG_BF16_STATES | ssd.SSD_FLAG_WHOLE_GROUPS):
+        y, f = run_fwd(inp, Q, flags=flags)
+        yo, fo = orc.ssd_fwd(**inp)
+        d = (y.double().cpu().numpy() - yo)
+        assert np.isfinite(d).all() and np.abs(d).max() <= 2e-2 * np.abs(yo).max()
 
 
 # ---------------------------------------------------------------------------
@@ -312,7 +325,7 @@ def test_gated_scan_step(orc):
     nc = synthetic.nchunks(L, Q)
     dt_sp = torch.empty((b, H, nc, Q), device=DEV)
     cumA = torch.empty_like(dt_sp)
-    states = torch.empty((b, nc, H, P, N), device=DEV, dtype=torch.bfloat16)
+    states = torch.empty((b, nc, H, P, N), device=DEV, dtype=torch.float32)
     ssd.ssd_chunk_cumsum(d["x"], d["dt"], d["A"], d["B"], d["C"], d["dt_bias"], Q,
                          dt_out=dt_sp, cumA_out=cumA)
     ssd.ssd_chunk_state(d["x"], d["dt"], d["A"], d["B"], d["C"], dt_sp, cumA, Q, states=states)
