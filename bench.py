@@ -36,7 +36,7 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-HEADLINE = "fwd_bf16_b4_L1024"
+HEADLINE = "fwd_bf16_b1_L65536_G8"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
                   "sm_max_mhz": 1965.0, "source": "fallback"}
 N_SM = 148
@@ -53,6 +53,11 @@ def parse_args():
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--flush-mb", type=int, default=256)
+    ap.add_argument("--e2e-steps", type=int, default=20,
+                    help="steps of the end-to-end (pinned host buffers) measurement")
+    ap.add_argument("--plumbing-only", action="store_true",
+                    help="run only the rank plumbing (launcher, process group, max over "
+                         "ranks) on CPU with gloo and print a JSON line without a metric")
     ap.add_argument("--conv-only", action="store_true",
                     help="time only the convolution workloads (one JSON line of them)")
     ap.add_argument("--bwd-only", action="store_true",
@@ -286,7 +291,7 @@ def main_ours(args):
     with clocks:
         barrier()
         torch.cuda.synchronize()
-        gpu_head_start(0.15 * args.steps)
+        gpu_head_start(min(50.0, 0.15 * args.steps))
         for k in range(args.steps):
             flush()
             ev[k][0].record(stream)
@@ -300,49 +305,27 @@ def main_ours(args):
     value = job_throughput(tokens, world, ms)
     tc = ssd.tensor_core_steps(cfg.batch, cfg.seqlen, cfg.nheads, cfg.headdim, cfg.dstate,
                                cfg.ngroups, cfg.chunk, cfg.dtype)
-    # ssd_fwd folds step 1 into the tensor-core chunk_state
-    launches_per_step = 3 if "chunk_state" in tc else 4
-
-    # ---- per-kernel durations over the same kind of timed steps ---------
-    nc = -(-cfg.seqlen // cfg.chunk)
-    dt_sp = torch.empty((cfg.batch, cfg.nheads, nc, cfg.chunk), device=dev)
-    cumA = torch.empty_like(dt_sp)
-    states = torch.empty((cfg.batch, nc, cfg.nheads, cfg.headdim, cfg.dstate), device=dev,
-                         dtype=cfg.dtype)
-    names = ["chunk_cumsum", "chunk_state", "state_passing", "chunk_scan"]
-
-    def step_split(evs):
-        evs[0].record(stream)
-        ssd.ssd_chunk_cumsum(d["x"], d["dt"], d["A"], d["B"], d["C"], d["dt_bias"], cfg.chunk,
-                             dt_out=dt_sp, cumA_out=cumA)
-        evs[1].record(stream)
-        ssd.ssd_chunk_state(d["x"], d["dt"], d["A"], d["B"], d["C"], dt_sp, cumA, cfg.chunk,
-                            states=states)
-        evs[2].record(stream)
-        ssd.ssd_state_passing(d["x"], d["dt"], d["A"], d["B"], d["C"], cumA, states, cfg.chunk,
-                              init_state=d["init_state"], final_state=fin)
-        evs[3].record(stream)
-        ssd.ssd_chunk_scan(d["x"], d["dt"], d["A"], d["B"], d["C"], dt_sp, cumA, states,
-                           d["D"], cfg.chunk, y=y)
-        evs[4].record(stream)
-
-    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
-    for _ in range(args.warmup):
-        flush()
-        step_split([torch.cuda.Event() for _ in range(5)])
-    barrier()
-    torch.cuda.synchronize()
-    gpu_head_start(0.2 * args.steps)
-    for k in range(args.steps):
-        flush()
-        step_split(kev[k])
-    torch.cuda.synchronize()
-    kms = {n: sum(e[i].elapsed_time(e[i + 1]) for e in kev) / args.steps
-           for i, n in enumerate(names)}
     cost = algorithmic_cost(cfg, elt)
-    top = max(names, key=lambda n: kms[n])
-    roofline = roofline_entry(top, cost[top], kms[top], peaks, clocks.summary(),
-                              top in tc, cfg.name)
+    if "fused" in tc:
+        # one kernel does the whole path: its bytes are the path's (inputs
+        # read once, y written once; no intermediate counted)
+        launches_per_step = 1
+        kms = {"fused_fwd": ms}
+        roofline = roofline_entry("fused_fwd", cost["path"], ms, peaks, clocks.summary(), True,
+                                  cfg.name)
+        roofline["duration_note"] = ("CUDA events around each ssd_fwd call: the kernel plus "
+                                     "the memset of its carry ring")
+    else:
+        # ssd_fwd folds step 1 into the tensor-core chunk_state
+        launches_per_step = 3 if "chunk_state" in tc else 4
+        kms = split_kernel_ms(ssd, cfg, d, y, fin, dev, flush, args.steps)
+        top = max(kms, key=lambda n: kms[n])
+        roofline = roofline_entry(top, cost[top], kms[top], peaks, clocks.summary(),
+                                  top in tc, cfg.name)
+    # the whole step against the path's algorithmic bytes, whatever the kernel split
+    path_bytes = cost["path"][0]
+    roofline["path_bytes"] = path_bytes
+    roofline["path_frac"] = path_bytes / (ms * 1e-3) / (peaks["hbm_gbs"] * 1e9)
 
     # ---- e2e through the public API from pinned host buffers ------------
     # Every step moves its own inputs host -> device and its y device -> host
@@ -350,13 +333,14 @@ def main_ours(args):
     # serving loop runs them: step k+1's inputs go over PCIe on one copy
     # stream while step k computes and its y comes back on another (the link
     # is full duplex); two device input / output sets alternate.
+    e2e_steps = max(2, min(args.steps, args.e2e_steps))
     host = {k: (v.pin_memory() if v is not None else None) for k, v in inp.items()}
     y_host = [torch.empty(y.shape, dtype=y.dtype, pin_memory=True) for _ in range(2)]
     h2d = sum(v.numel() * v.element_size() for v in host.values() if v is not None)
     d2h = y_host[0].numel() * y_host[0].element_size()
-    dev_in = [{k: (torch.empty_like(v, device=dev) if v is not None else None)
-               for k, v in host.items()} for _ in range(2)]
-    y_dev = [torch.empty_like(y) for _ in range(2)]
+    dev_in = [d] + [{k: (torch.empty_like(v, device=dev) if v is not None else None)
+                     for k, v in host.items()}]
+    y_dev = [y, torch.empty_like(y)]
     s_h2d, s_d2h = torch.cuda.Stream(), torch.cuda.Stream()
     ev_in = [torch.cuda.Event() for _ in range(2)]
     ev_done = [torch.cuda.Event() for _ in range(2)]
@@ -376,37 +360,40 @@ def main_ours(args):
             stream.wait_event(ev_out[i])  # step k-2's y has been read back
         dd = dev_in[i]
         ssd.ssd_fwd(dd["x"], dd["dt"], dd["A"], dd["B"], dd["C"], dd["D"], dd["dt_bias"],
-                    cfg.chunk, dd["init_state"], y=y_dev[i], workspace=ws)
+                    cfg.chunk, dd["init_state"], y=y_dev[i], final_state=fin, workspace=ws)
         ev_done[i].record(stream)
         with torch.cuda.stream(s_d2h):
             s_d2h.wait_event(ev_done[i])
             y_host[i].copy_(y_dev[i], non_blocking=True)
             ev_out[i].record(s_d2h)
 
-    for k in range(args.warmup):
+    for k in range(min(args.warmup, 3)):
         e2e_step(k)
     torch.cuda.synchronize()
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     s_h2d.wait_event(e0)
-    for k in range(args.steps):
+    for k in range(e2e_steps):
         e2e_step(k)
-    stream.wait_event(ev_out[(args.steps - 1) % 2])
-    if args.steps > 1:
-        stream.wait_event(ev_out[(args.steps - 2) % 2])
+    stream.wait_event(ev_out[(e2e_steps - 1) % 2])
+    stream.wait_event(ev_out[(e2e_steps - 2) % 2])
     e1.record(stream)
     torch.cuda.synchronize()
-    ems = ranks_max(e0.elapsed_time(e1) / args.steps)
+    ems = ranks_max(e0.elapsed_time(e1) / e2e_steps)
     e2e = {"value": job_throughput(tokens, world, ems), "unit": "tokens/s",
-           "ms_per_step": ems, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+           "ms_per_step": ems, "steps": e2e_steps, "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h,
            "pipelined": "2 streams: next step's inputs in while this step's y goes out"}
+    del host, y_host, dev_in, y_dev
+    d = y = None
+    torch.cuda.empty_cache()
 
     # ---- other workloads (rank-local, reported for context) --------------
     extra = {}
     if not args.no_extra:
         extra = other_workloads(ssd, synthetic, dev, flush, peaks, rank, world,
-                                barrier, ranks_max)
+                                barrier, ranks_max, skip=cfg.name)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -430,8 +417,9 @@ def main_ours(args):
                    "nheads": cfg.nheads, "headdim": cfg.headdim, "dstate": cfg.dstate,
                    "ngroups": cfg.ngroups, "chunk": cfg.chunk, "global_batch":
                    cfg.batch * world, "parallelism": f"dp{world}" if world > 1 else "single",
-                   "l2": f"flushed before every timed step ({args.flush_mb} MB write, then "
-                         "a read of it, so its write-back ends before the timed region)"},
+                   "l2": f"inputs {input_bytes(inp) / 1e6:.0f} MB; L2 flushed before every "
+                         f"timed step ({args.flush_mb} MB write, then a read of it, so its "
+                         "write-back ends before the timed region)"},
         "roofline": roofline,
         "kernel_ms": kms,
         "e2e": e2e,
@@ -448,7 +436,12 @@ def main_ours(args):
         dist.destroy_process_group()
 
 
+def input_bytes(inp) -> int:
+    return sum(v.numel() * v.element_size() for v in inp.values() if v is not None)
+
+
 KERNEL_SOURCES = {
+    "fused_fwd": ["fused_fwd.cu", "tcgen05.cuh", "tma.cuh", "internal.cuh"],
     "chunk_scan": ["chunk_scan_tc.cu", "tcgen05.cuh", "tma.cuh", "internal.cuh"],
     "chunk_state": ["chunk_state_tc.cu", "tcgen05.cuh", "tma.cuh", "internal.cuh"],
     "state_passing": ["state_passing.cu", "internal.cuh"],
@@ -574,14 +567,18 @@ def launch_timing(ssd, synthetic, dev, flush, name, rank, steps=200):
     return res
 
 
-def other_workloads(ssd, synthetic, dev, flush, peaks, rank, world, barrier, ranks_max):
+def other_workloads(ssd, synthetic, dev, flush, peaks, rank, world, barrier, ranks_max,
+                    skip=None):
     import torch
     out = {}
     stream = torch.cuda.current_stream()
     # launch-latency view of the two small workloads
     for name in ("fwd_f32_small", "fwd_bf16_b4_L1024"):
         out[name + "_launch"] = launch_timing(ssd, synthetic, dev, flush, name, rank)
-    for name, steps in (("fwd_bf16_b8_L4096_init", 10), ("fwd_bf16_b1_L65536_G8", 5)):
+    for name, steps in (("fwd_bf16_b4_L1024", 50), ("fwd_bf16_b8_L4096_init", 20),
+                        ("fwd_bf16_b1_L65536_G8", 5)):
+        if name == skip:
+            continue
         cfg = synthetic.FWD_CONFIGS[name]
         inp = synthetic.make_config_inputs(cfg, rank_seed(1234 + synthetic.SEED_OFFSET[name], rank))
         d = {k: (v.to(dev) if v is not None else None) for k, v in inp.items()}
@@ -612,10 +609,15 @@ def other_workloads(ssd, synthetic, dev, flush, peaks, rank, world, barrier, ran
         torch.cuda.synchronize()
         ms = ranks_max(sum(a.elapsed_time(b_) for a, b_ in evs) / steps)
         nbytes = algorithmic_cost(cfg, 2)["path"][0]
-        kms = split_kernel_ms(ssd, cfg, d, y, fin, dev, flush, steps)
-        out[name] = {"tokens_per_s": job_throughput(cfg.tokens, world, ms), "ms": ms,
-                     "hbm_frac_of_path_bytes": nbytes / (ms * 1e-3) / (peaks["hbm_gbs"] * 1e9),
-                     "kernel_ms": kms}
+        tc = ssd.tensor_core_steps(cfg.batch, cfg.seqlen, cfg.nheads, cfg.headdim, cfg.dstate,
+                                   cfg.ngroups, cfg.chunk, cfg.dtype)
+        ent = {"tokens_per_s": job_throughput(cfg.tokens, world, ms), "ms": ms,
+               "path_bytes": nbytes,
+               "hbm_frac_of_path_bytes": nbytes / (ms * 1e-3) / (peaks["hbm_gbs"] * 1e9),
+               "kernels": "fused_fwd" if "fused" in tc else "split"}
+        if "fused" not in tc:
+            ent["kernel_ms"] = split_kernel_ms(ssd, cfg, d, y, fin, dev, flush, steps)
+        out[name] = ent
         del d, y, fin, ws
         torch.cuda.empty_cache()
 
@@ -979,8 +981,9 @@ def split_kernel_ms(ssd, cfg, d, y, fin, dev, flush, steps):
     nc = -(-cfg.seqlen // cfg.chunk)
     dt_sp = torch.empty((cfg.batch, cfg.nheads, nc, cfg.chunk), device=dev)
     cumA = torch.empty_like(dt_sp)
+    # the step entry points keep fp32 chunk states (the default precision)
     states = torch.empty((cfg.batch, nc, cfg.nheads, cfg.headdim, cfg.dstate), device=dev,
-                         dtype=cfg.dtype)
+                         dtype=torch.float32)
     names = ["chunk_cumsum", "chunk_state", "state_passing", "chunk_scan"]
     tot = dict.fromkeys(names, 0.0)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps + 2)]
@@ -1010,37 +1013,71 @@ def split_kernel_ms(ssd, cfg, d, y, fin, dev, flush, steps):
     return {n: tot[n] / steps for n in names}
 
 
+def oracle_sample(cfg, inp, heads: int, tokens: int):
+    """Batch row 0, its first `heads` heads and first `tokens` tokens: the
+    bounded unit of oracle work the CPU timings use (the recurrence's work per
+    token is the same all along the sequence).  Head h reads its own group's B
+    and C, given to the oracle as one group column per head."""
+    hpg = cfg.nheads // cfg.ngroups
+    gsel = [h // hpg for h in range(heads)]
+    return {"x": inp["x"][:1, :tokens, :heads], "dt": inp["dt"][:1, :tokens, :heads],
+            "A": inp["A"][:heads], "B": inp["B"][:1, :tokens, gsel],
+            "C": inp["C"][:1, :tokens, gsel], "D": inp["D"][:heads],
+            "dt_bias": inp["dt_bias"][:heads],
+            "init_state": None if inp["init_state"] is None else inp["init_state"][:1, :heads]}
+
+
+def calibrated_sample(cfg, inp, orc, heads: int, seconds: float):
+    """The oracle sample (heads x tokens) whose one run takes about `seconds`:
+    a first run on up to 2048 tokens sets the rate; tokens are then scaled to
+    the target and rounded to a multiple of the chunk (at least one chunk, at
+    most the whole sequence)."""
+    t0_tokens = min(cfg.seqlen, 2048)
+    sub = oracle_sample(cfg, inp, heads, t0_tokens)
+    t0 = time.perf_counter()
+    orc.ssd_fwd(**sub)
+    dt = max(time.perf_counter() - t0, 1e-6)
+    tok = int(t0_tokens * seconds / dt) // cfg.chunk * cfg.chunk
+    tok = max(cfg.chunk, min(cfg.seqlen, tok))
+    return oracle_sample(cfg, inp, heads, tok), tok
+
+
 def cpu_baseline(cfg, inp, budget_s=12.0):
-    """The fp64 oracle, as it stands, on a bounded sample of the workload:
-    whole batch rows (all heads, full sequence), cycling over the batch, until
-    about budget_s seconds of work have been done, on all host threads; then
-    a shorter sample on one thread, and a few decode steps of the decode
-    workload on all threads."""
+    """The fp64 oracle, as it stands, on a bounded sample of the workload: batch
+    row 0, as many heads as host threads, the first tokens of the sequence (a
+    run of about 2 s), repeated until about budget_s seconds of work; then the
+    same on one thread and one head for a quarter of that, and a few decode
+    steps of the decode workload on all threads.  Throughput is in
+    token-equivalents: tokens x heads / nheads per run."""
     import oracle
     from mamba_ssd_scan_b200 import synthetic
     orc = oracle.load()
     threads = orc.num_threads()
+    heads = max(1, min(cfg.nheads, threads))
+    sub, tok = calibrated_sample(cfg, inp, orc, heads, 2.0)
+    tok_equiv = tok * heads / cfg.nheads
 
-    def fwd_rate(budget):
+    def fwd_rate(sample, budget):
         t0 = time.perf_counter()
-        rows = 0
+        runs = 0
         while time.perf_counter() - t0 < budget:
-            r = rows % cfg.batch
-            sub = {k: (v[r:r + 1] if (v is not None and k not in ("A", "D", "dt_bias"))
-                       else v) for k, v in inp.items()}
-            orc.ssd_fwd(**sub)
-            rows += 1
-        return rows, time.perf_counter() - t0
+            orc.ssd_fwd(**sample)
+            runs += 1
+        return runs, time.perf_counter() - t0
 
-    rows, dt = fwd_rate(budget_s)
-    out = {"value": rows * cfg.seqlen / dt, "unit": "tokens/s", "cores": threads,
-           "kind": "oracle", "sample": f"{rows} batch rows of {cfg.name} (all heads, full "
-                                       f"sequence each), {dt:.1f} s"}
+    runs, dt = fwd_rate(sub, budget_s)
+    out = {"value": runs * tok_equiv / dt, "unit": "tokens/s", "cores": threads,
+           "kind": "oracle", "sample": f"{runs} x (batch row 0, heads 0-{heads - 1} of "
+                                       f"{cfg.nheads}, tokens 0-{tok - 1} of {cfg.seqlen}) of "
+                                       f"{cfg.name}, {dt:.1f} s; token-equivalents = "
+                                       f"{tok} x {heads}/{cfg.nheads} per run"}
     orc.set_num_threads(1)
-    rows1, dt1 = fwd_rate(budget_s / 4)
+    sub1, tok1 = calibrated_sample(cfg, inp, orc, 1, 1.0)
+    runs1, dt1 = fwd_rate(sub1, budget_s / 4)
     orc.set_num_threads(threads)
-    out["one_core"] = {"value": rows1 * cfg.seqlen / dt1, "unit": "tokens/s",
-                       "sample": f"{rows1} batch rows, {dt1:.1f} s"}
+    out["one_core"] = {"value": runs1 * tok1 / cfg.nheads / dt1, "unit": "tokens/s",
+                       "sample": f"{runs1} x (batch row 0, head 0, tokens 0-{tok1 - 1}), "
+                                 f"{dt1:.1f} s"}
     # decode: a few steps on 8 of the 256 batch rows (the rows are independent),
     # scaled to the whole batch
     dcfg = synthetic.DECODE_CONFIGS["decode_b256_H80"]
@@ -1063,8 +1100,11 @@ def cpu_baseline(cfg, inp, budget_s=12.0):
 # ---------------------------------------------------------------------------
 def main_reference(args):
     """The reference arm: the fp64 CPU oracle on this arm's workload, each step a
-    bounded sample (one batch row, as many heads as host threads, full sequence)."""
+    bounded sample (batch row 0, as many heads as host threads, the first tokens
+    of the sequence) sized so that warm-up and timed steps together take about
+    two minutes.  Under torchrun only rank 0 runs it; the others exit at once."""
     rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
     if rank != 0:
         return
     import oracle
@@ -1072,24 +1112,20 @@ def main_reference(args):
     cfg = synthetic.FWD_CONFIGS[args.workload]
     inp = synthetic.make_config_inputs(cfg)
     orc = oracle.load()
-    heads = min(cfg.nheads, orc.num_threads())
-    hpg = cfg.nheads // cfg.ngroups
-    gsel = [h // hpg for h in range(heads)]
-    sub = {"x": inp["x"][:1, :, :heads], "dt": inp["dt"][:1, :, :heads], "A": inp["A"][:heads],
-           "B": inp["B"][:1, :, gsel], "C": inp["C"][:1, :, gsel], "D": inp["D"][:heads],
-           "dt_bias": inp["dt_bias"][:heads],
-           "init_state": None if inp["init_state"] is None else inp["init_state"][:1, :heads]}
+    heads = max(1, min(cfg.nheads, orc.num_threads()))
+    per_step = min(2.0, 120.0 / max(1, args.steps + args.warmup))
+    sub, tok = calibrated_sample(cfg, inp, orc, heads, per_step)
     for _ in range(args.warmup):
         orc.ssd_fwd(**sub)
     t0 = time.perf_counter()
     for _ in range(args.steps):
         orc.ssd_fwd(**sub)
     sec = (time.perf_counter() - t0) / args.steps
-    # one step covers heads/H of one batch row's tokens
-    tok_equiv = cfg.seqlen * heads / cfg.nheads
+    # one step covers tokens x heads / nheads of one batch row
+    tok_equiv = tok * heads / cfg.nheads
     value = tok_equiv / sec
     line = {"impl": "reference", "metric": "SSD fwd tokens/s", "value": value,
-            "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+            "unit": "tokens/s", "n_gpus": 0, "ranks": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": cfg.name, "batch": cfg.batch, "seqlen": cfg.seqlen,
@@ -1098,16 +1134,67 @@ def main_reference(args):
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": orc.num_threads(),
                              "kind": "oracle",
                              "sample": f"per step: batch row 0, heads 0-{heads - 1} of "
-                                       f"{cfg.nheads}, full sequence (token-equivalents = "
-                                       f"seqlen x {heads}/{cfg.nheads})"},
+                                       f"{cfg.nheads}, tokens 0-{tok - 1} of {cfg.seqlen} "
+                                       f"(token-equivalents = {tok} x {heads}/{cfg.nheads}); "
+                                       "runs on the host cores of rank 0 only, no GPU"},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
+def main_plumbing(args):
+    """The rank plumbing alone (no GPU, no metric): process group over gloo,
+    every rank's id gathered and a max over ranks of a per-rank number, so a
+    CPU test can check what `--gpus N` launches."""
+    import torch
+    import torch.distributed as dist
+    rank, world, local = rank_env()
+    if world > 1:
+        import datetime
+        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    seen = [rank]
+    if world > 1:
+        t = torch.tensor([rank], dtype=torch.int64)
+        out = [torch.zeros(1, dtype=torch.int64) for _ in range(world)]
+        dist.all_gather(out, t)
+        seen = [int(v.item()) for v in out]
+    ms = max_over_ranks(1.0 + rank, world, torch.device("cpu"))
+    if rank == 0:
+        print(json.dumps({"plumbing": True, "n_gpus": world, "ranks_seen": seen,
+                          "local_ranks_ok": local == rank, "ms_max_over_ranks": ms}),
+              flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def launch_ranks(args) -> int:
+    """`--gpus N` (N > 1) started without a rank environment: start N ranks of
+    this same command on this node (torch.distributed.run, rendezvous on
+    127.0.0.1) and return their exit status."""
+    import socket
+    import subprocess
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={args.gpus}", "--master-addr=127.0.0.1",
+           f"--master-port={port}", os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.call(cmd)
+
+
 if __name__ == "__main__":
     a = parse_args()
-    if a.impl == "reference":
+    if a.gpus < 1:
+        sys.exit("--gpus must be at least 1")
+    if "WORLD_SIZE" not in os.environ and a.gpus > 1:
+        sys.exit(launch_ranks(a))
+    if int(os.environ.get("WORLD_SIZE", "1")) != a.gpus:
+        sys.exit(f"--gpus {a.gpus} but WORLD_SIZE={os.environ.get('WORLD_SIZE')}: "
+                 "launch one rank per GPU")
+    if a.plumbing_only:
+        main_plumbing(a)
+    elif a.impl == "reference":
         main_reference(a)
     else:
         main_ours(a)

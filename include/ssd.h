@@ -147,14 +147,18 @@ ssd_status ssd_fwd(const ssd_fwd_args* args, void* stream);
  * latency-critical code that must not risk a cudaMalloc's device-wide
  * synchronisation.  This entry point ignores args->workspace and
  * args->workspace_bytes and takes the scratch from a buffer of
- * SSD_NO_ALLOC_SCRATCH_BYTES compiled into the library (every GPU that loads
- * the library holds it until the process exits).  It calls no cudaMalloc,
- * cudaFree or other allocating routine.
+ * SSD_NO_ALLOC_SCRATCH_BYTES compiled into the library.  It calls no
+ * cudaMalloc, cudaFree or other allocating routine.
  *   - Sizes whose ssd_fwd_workspace_size() exceeds the buffer are rejected
  *     with SSD_ERR_UNSUPPORTED before anything is launched.
- *   - The first call on each device looks up the buffer's device address
- *     (cudaGetSymbolAddress, that device current) and caches it; make that
- *     first call before any stream capture on the device.
+ *   - The buffer is reserved on a device when the library's device code is
+ *     loaded there and is held until the process exits.  Under CUDA's lazy
+ *     module loading (the default since CUDA 12.2) that happens at the first
+ *     call on the device, which can then fail with SSD_ERR_CUDA for lack of
+ *     device memory and may synchronise the device.  That first call also
+ *     looks up the buffer's device address (cudaGetSymbolAddress, that device
+ *     current) and caches it.  So make one call per device at initialisation,
+ *     before any stream capture and before the latency-critical phase.
  *   - All calls share the one buffer: calls that can overlap on the GPU (on
  *     different streams without ordering between them, or from different host
  *     threads) race and give wrong results; serialise them.  The buffer keeps
@@ -163,6 +167,18 @@ ssd_status ssd_fwd(const ssd_fwd_args* args, void* stream);
  * Everything else (arguments, layouts, errors, asynchrony) is as ssd_fwd. */
 #define SSD_NO_ALLOC_SCRATCH_BYTES (16u << 20)
 ssd_status ssd_fwd_no_alloc(const ssd_fwd_args* args, void* stream);
+
+/* SSD_NO_ALLOC_SCRATCH_BYTES as compiled into this library (bindings read the
+ * limit from here rather than repeating the constant). */
+size_t ssd_fwd_no_alloc_scratch_bytes(void);
+
+/* ssd_fwd_check_status for ssd_fwd_no_alloc: synchronises `stream` and returns
+ * the device status of the last ssd_fwd_no_alloc call on the current device
+ * (SSD_OK, or SSD_ERR_TIMEOUT when a kernel gave up on a bounded wait and the
+ * outputs are invalid).  Only sizes, dtype and flags of `args` are read; they
+ * must be those of that call.  SSD_ERR_UNSUPPORTED for sizes beyond the
+ * buffer, SSD_ERR_INVALID_ARG for invalid sizes. */
+ssd_status ssd_fwd_no_alloc_check_status(const ssd_fwd_args* args, void* stream);
 
 /* Synchronises `stream` and returns the device status of the last ssd_fwd
  * call that used this workspace: SSD_OK, or SSD_ERR_TIMEOUT when a kernel gave
@@ -454,6 +470,18 @@ const char* ssd_last_cuda_error(void);
 
 /* Library version string (static). */
 const char* ssd_version(void);
+
+/* Test hook for the failure paths, off by default: makes one producer withhold
+ * one hand-off, so the consumers' bounded waits run out and the kernel reports
+ * SSD_ERR_TIMEOUT through its status word instead of hanging (no fault, no
+ * trap).  `what` = SSD_DEBUG_CONV_TILE: the convolution's producer stops before
+ * tile `index`; SSD_DEBUG_FWD_CARRY: the fused forward does not publish the
+ * state leaving chunk `index` (so the next chunk's wait gives up after about a
+ * second).  index < 0 turns the hook off.  Process-wide; read on the host when
+ * a kernel is launched.  Other values of `what` are ignored. */
+#define SSD_DEBUG_CONV_TILE 0
+#define SSD_DEBUG_FWD_CARRY 1
+void ssd_debug_set_withhold(int what, int64_t index);
 
 #ifdef __cplusplus
 }

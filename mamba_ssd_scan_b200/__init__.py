@@ -16,6 +16,8 @@ import torch
 
 __all__ = [
     "SsdError", "ssd_fwd", "ssd_fwd_workspace_size", "ssd_fwd_check_status", "ssd_fwd_no_alloc",
+    "ssd_fwd_no_alloc_check_status", "ssd_fwd_no_alloc_scratch_bytes", "ssd_debug_set_withhold",
+    "SSD_DEBUG_CONV_TILE", "SSD_DEBUG_FWD_CARRY",
     "ssd_fwd_tensor_core_steps", "tensor_core_steps", "ssd_chunk_cumsum", "ssd_chunk_state",
     "ssd_state_passing", "ssd_chunk_scan", "ssd_state_update", "ssd_status_string",
     "ssd_version", "lib_path", "load_library", "SSD_FLAG_CUDA_CORES", "SSD_FLAG_WHOLE_GROUPS",
@@ -140,6 +142,12 @@ def load_library():
     lib.ssd_fwd_no_alloc.argtypes = [F, _vp]
     lib.ssd_fwd_check_status.restype = ctypes.c_int
     lib.ssd_fwd_check_status.argtypes = [F, _vp]
+    lib.ssd_fwd_no_alloc_check_status.restype = ctypes.c_int
+    lib.ssd_fwd_no_alloc_check_status.argtypes = [F, _vp]
+    lib.ssd_fwd_no_alloc_scratch_bytes.restype = _sz
+    lib.ssd_fwd_no_alloc_scratch_bytes.argtypes = []
+    lib.ssd_debug_set_withhold.restype = None
+    lib.ssd_debug_set_withhold.argtypes = [ctypes.c_int, ctypes.c_int64]
     lib.ssd_chunk_cumsum.restype = ctypes.c_int
     lib.ssd_chunk_cumsum.argtypes = [F, _vp, _vp, _vp]
     lib.ssd_chunk_state.restype = ctypes.c_int
@@ -363,7 +371,19 @@ def ssd_bwd(x, dt, A, B, C, dy, D=None, dt_bias=None, chunk: int = 256, init_sta
     return o
 
 
-SSD_NO_ALLOC_SCRATCH_BYTES = 16 << 20
+SSD_DEBUG_CONV_TILE = 0
+SSD_DEBUG_FWD_CARRY = 1
+
+
+def ssd_debug_set_withhold(what: int, index: int) -> None:
+    """Test hook (include/ssd.h): make one producer withhold one hand-off so
+    the consumers' bounded waits run out; index < 0 turns it off."""
+    load_library().ssd_debug_set_withhold(int(what), int(index))
+
+
+def ssd_fwd_no_alloc_scratch_bytes() -> int:
+    """The size of the library's built-in scratch buffer (bytes)."""
+    return int(load_library().ssd_fwd_no_alloc_scratch_bytes())
 
 
 def ssd_fwd_no_alloc(x, dt, A, B, C, D=None, dt_bias=None, chunk: int = 256, init_state=None,
@@ -371,16 +391,27 @@ def ssd_fwd_no_alloc(x, dt, A, B, C, D=None, dt_bias=None, chunk: int = 256, ini
     """ssd_fwd without a workspace, for callers that cannot allocate: the
     scratch comes from a fixed buffer inside the library (see ssd_fwd_no_alloc
     in include/ssd.h).  ``y`` (and ``final_state``, if wanted) are caller-owned
-    outputs; calls that can overlap on the GPU race and must be serialised."""
+    outputs; calls that can overlap on the GPU race and must be serialised.
+    Sizes beyond the buffer are rejected by the library (SsdError,
+    SSD_ERR_UNSUPPORTED) before anything is launched."""
     lib = load_library()
     a = _fwd_args(x, dt, A, B, C, D, dt_bias, chunk, init_state, y, final_state, flags, z)
-    need = int(lib.ssd_fwd_workspace_size(ctypes.byref(a)))
-    if need > SSD_NO_ALLOC_SCRATCH_BYTES:
-        raise SsdError(SSD_ERR_UNSUPPORTED,
-                       f"ssd_fwd_no_alloc: these sizes need {need} bytes of scratch, more than "
-                       f"the built-in {SSD_NO_ALLOC_SCRATCH_BYTES}")
     _check(lib.ssd_fwd_no_alloc(ctypes.byref(a), _stream_ptr(stream)), "ssd_fwd_no_alloc")
     return y
+
+
+def ssd_fwd_no_alloc_check_status(x, B, chunk: int, flags: int = 0, stream=None) -> int:
+    """Synchronise and return the device status of the last ssd_fwd_no_alloc
+    call on the current device with these sizes (SSD_OK = 0,
+    SSD_ERR_TIMEOUT = 4)."""
+    b, L, H, P = x.shape
+    a = SsdFwdArgs()
+    a.batch, a.seqlen, a.nheads, a.headdim, a.dstate, a.ngroups, a.chunk = (
+        b, L, H, P, B.shape[3], B.shape[2], chunk)
+    a.dtype = _dtype_code(x)
+    a.flags = flags
+    return int(load_library().ssd_fwd_no_alloc_check_status(ctypes.byref(a),
+                                                            _stream_ptr(stream)))
 
 
 def ssd_fwd_check_status(x, B, chunk: int, workspace, flags: int = 0, stream=None) -> int:

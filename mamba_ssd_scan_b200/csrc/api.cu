@@ -1,6 +1,7 @@
 // api.cu -- the extern "C" entry points of libssd_b200.so (declared and
 // documented in include/ssd.h): argument validation, workspace carving and
 // kernel dispatch.  Nothing here allocates memory or synchronises the host.
+#include <atomic>
 #include <stdint.h>
 #include <string.h>
 
@@ -271,6 +272,16 @@ ssd_status check_bwd_sizes(const ssd_bwd_args* a) {
 }
 
 }  // namespace
+
+namespace {
+std::atomic<int64_t> g_withhold[2] = {{-1}, {-1}};
+}  // namespace
+
+namespace ssd {
+int64_t debug_withhold(int what) {
+    return (what == 0 || what == 1) ? g_withhold[what].load(std::memory_order_relaxed) : -1;
+}
+}  // namespace ssd
 
 extern "C" {
 
@@ -702,6 +713,10 @@ const char* ssd_status_string(ssd_status s) {
 
 const char* ssd_last_cuda_error(void) {
     return g_last_cuda_error == cudaSuccess ? "no CUDA error" : cudaGetErrorString(g_last_cuda_error);
+}
+
+void ssd_debug_set_withhold(int what, int64_t index) {
+    if (what == 0 || what == 1) g_withhold[what].store(index < 0 ? -1 : index, std::memory_order_relaxed);
 }
 
 const char* ssd_version(void) { return "ssd_b200 0.1.0 (sm_100a)"; }

@@ -364,9 +364,9 @@ cudaError_t launch_fwd(const ConvParams& p, cudaStream_t s) {
     nseg = (p.seqlen + seg - 1) / seg;
     dim3 grid(static_cast<unsigned>(nblk), static_cast<unsigned>(nseg),
               static_cast<unsigned>(p.batch));
-    // SSD_DEBUG_WITHHOLD_TILE (tests only): the producer withholds that tile
-    const char* wh = getenv("SSD_DEBUG_WITHHOLD_TILE");
-    conv1d_kernel<T, K, ACT><<<grid, nt + 32, smem, s>>>(p, seg, wh ? atoi(wh) : -1);
+    // the test hook (ssd_debug_set_withhold): the producer withholds that tile
+    const int64_t wh = debug_withhold(SSD_DEBUG_CONV_TILE);
+    conv1d_kernel<T, K, ACT><<<grid, nt + 32, smem, s>>>(p, seg, static_cast<int>(wh));
     return cudaGetLastError();
 }
 

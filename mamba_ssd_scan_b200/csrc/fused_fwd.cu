@@ -394,7 +394,7 @@ template <int NST, bool GATED>
 __global__ void __launch_bounds__(NTHREADS, 1)
     fused_fwd_kernel(const __grid_constant__ FwdParams p, const __grid_constant__ CUtensorMap tm_c,
                      const __grid_constant__ CUtensorMap tm_b, const __grid_constant__ CUtensorMap tm_x,
-                     int hb_size, int64_t total_items, uint64_t* ring) {
+                     int hb_size, int64_t total_items, uint64_t* ring, int64_t withhold) {
     using T = FusedSmem<NST>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -951,7 +951,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
 #pragma unroll
                                 for (int k = 0; k < 32; ++k) fp[k * NST] = hmid[k];
                             }
-                        } else {
+                        } else if (it.c != withhold) {  // (the test hook withholds one chunk's)
                             uint64_t* dst = ring + ((it.c & 1) * Bsz + it.b) * H * kWordsPerState +
                                             h * kWordsPerState + n * (PD / 2) + 16 * hf;
                             const uint64_t tag = static_cast<uint64_t>((it.c + 1) & 0xFFFF) << 48;
@@ -1127,7 +1127,7 @@ cudaError_t launch_nd(const FwdParams& p, void* ws, cudaStream_t s) {
     q.status = static_cast<int*>(ws);
     uint64_t* ring = reinterpret_cast<uint64_t*>(static_cast<char*>(ws) + kHdrBytes);
     return launch_kernel(kern, dim3(grid), dim3(NTHREADS), T::SMEM, s, false, q, tc_, tb_, tx_, hb, items,
-                         ring);
+                         ring, debug_withhold(SSD_DEBUG_FWD_CARRY));
 }
 
 }  // namespace

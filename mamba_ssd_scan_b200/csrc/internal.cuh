@@ -235,6 +235,12 @@ cudaError_t launch_chunk_scan_tc(const FwdParams& p, cudaStream_t s);
 // The whole forward in one kernel (fused_fwd.cu): bf16, headdim 64, dstate 64
 // or 128, chunk 128 or 256.  The workspace is its own (fused_fwd_workspace_bytes,
 // 16-byte aligned) and is zeroed by the launch itself; status goes to its first word.
+// The test hook ssd_debug_set_withhold() sets: the index a kernel's producer
+// withholds (SSD_DEBUG_CONV_TILE: a convolution tile; SSD_DEBUG_FWD_CARRY: the
+// carry leaving a chunk of the fused forward), -1 when off.  Read on the host
+// at launch and passed to the kernel as an argument.
+int64_t debug_withhold(int what);
+
 bool fused_fwd_supported(const FwdParams& p);
 size_t fused_fwd_workspace_bytes(const FwdParams& p);
 cudaError_t launch_fused_fwd(const FwdParams& p, void* ws, cudaStream_t s);

@@ -8,10 +8,13 @@
 // variant takes it from a fixed buffer compiled into the library instead.
 //
 // The buffer is a file-scope __device__ array of SSD_NO_ALLOC_SCRATCH_BYTES.
-// Every GPU that loads the library holds it until the process exits.  Host
-// code cannot use the array's name as a device address, so the first call on
-// each device looks up the address with cudaGetSymbolAddress (that device
-// current) and caches it.
+// It is reserved on a device when the library's device code is loaded there:
+// under CUDA's lazy module loading (the default since 12.2) that is the first
+// call on the device, not library load, and it can fail for lack of memory.
+// Host code cannot use the array's name as a device address, so the first
+// call on each device looks up the address with cudaGetSymbolAddress (that
+// device current) and caches it.  The status word of the kernels that ran on
+// the buffer is its first 4 bytes, read by ssd_fwd_no_alloc_check_status.
 #include <mutex>
 
 #include "internal.cuh"
@@ -59,4 +62,19 @@ extern "C" ssd_status ssd_fwd_no_alloc(const ssd_fwd_args* args, void* stream) {
     a.workspace = scratch;
     a.workspace_bytes = kScratchBytes;
     return ssd_fwd(&a, stream);
+}
+
+extern "C" size_t ssd_fwd_no_alloc_scratch_bytes(void) { return kScratchBytes; }
+
+extern "C" ssd_status ssd_fwd_no_alloc_check_status(const ssd_fwd_args* args, void* stream) {
+    if (!args) return SSD_ERR_INVALID_ARG;
+    const size_t need = ssd_fwd_workspace_size(args);
+    if (need == 0) return SSD_ERR_INVALID_ARG;
+    if (need > kScratchBytes) return SSD_ERR_UNSUPPORTED;
+    void* scratch = scratch_address();
+    if (!scratch) return SSD_ERR_CUDA;
+    ssd_fwd_args a = *args;
+    a.workspace = scratch;
+    a.workspace_bytes = kScratchBytes;
+    return ssd_fwd_check_status(&a, stream);
 }

@@ -215,3 +215,22 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     with pytest.raises(RuntimeError, match="missing"):
         ssd.ssd_fwd(x, torch.zeros((1, 8, 2)), torch.zeros(2), torch.zeros((1, 8, 1, 16)),
                     torch.zeros((1, 8, 1, 16)), chunk=8)
+
+
+def test_no_alloc_scratch_size_matches_the_header(lib):
+    import mamba_ssd_scan_b200 as ssd
+    text = open(os.path.join(ROOT, "include", "ssd.h")).read()
+    m = re.search(r"#define SSD_NO_ALLOC_SCRATCH_BYTES \((\d+)u << (\d+)\)", text)
+    assert m, "SSD_NO_ALLOC_SCRATCH_BYTES not found in the header"
+    assert ssd.ssd_fwd_no_alloc_scratch_bytes() == int(m.group(1)) << int(m.group(2))
+
+
+def test_no_alloc_status_rejects_sizes_on_the_host(lib):
+    # beyond the built-in buffer, and invalid sizes: answered before any
+    # device access
+    a = _args(batch=8, seqlen=4096, nheads=32, headdim=64, dstate=128)
+    assert lib.ssd_fwd_no_alloc_check_status(ctypes.byref(a), None) == 2  # UNSUPPORTED
+    assert lib.ssd_fwd_no_alloc_check_status(ctypes.byref(_args(batch=0)), None) == 1
+    assert lib.ssd_fwd_no_alloc_check_status(None, None) == 1
+    # ssd_fwd_no_alloc itself rejects the oversize call before launching
+    assert lib.ssd_fwd_no_alloc(ctypes.byref(a), None) in (1, 2)

@@ -60,3 +60,36 @@ def test_single_rank_defaults(monkeypatch):
     assert bench.rank_env() == (0, 1, 0)
     assert bench.max_over_ranks(3.5, 1, torch.device("cpu")) == 3.5
     assert bench.job_throughput(100, 1, 10.0) == pytest.approx(1e4)
+
+
+def test_bench_launches_its_own_ranks():
+    """`bench.py --gpus 2` without a rank environment starts two ranks itself
+    (here with the gloo plumbing only: no GPU on this host) and reports both."""
+    import json
+    import subprocess
+    import sys
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "2",
+                        "--plumbing-only"], env=env, capture_output=True, text=True,
+                       timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    rec = json.loads(lines[0])
+    assert rec["n_gpus"] == 2
+    assert sorted(rec["ranks_seen"]) == [0, 1]
+    assert rec["ms_max_over_ranks"] == 2.0
+
+
+def test_bench_rejects_a_mismatched_world():
+    import subprocess
+    import sys
+    env = dict(os.environ, WORLD_SIZE="1", RANK="0", LOCAL_RANK="0")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "2",
+                        "--plumbing-only"], env=env, capture_output=True, text=True,
+                       timeout=120)
+    assert r.returncode != 0
+    assert "n_gpus" not in r.stdout
