@@ -80,9 +80,10 @@ typedef enum { SSD_F32 = 0, SSD_BF16 = 1 } ssd_dtype;
  *                and 6.1), applied in the kernel that writes y.  The gate does
  *                not touch the carried state.
  * Supported: 1 <= chunk <= 256; dstate a multiple of 4, <= 256; headdim a
- * multiple of 4.  bf16 inputs with headdim 64, dstate 64 or 128 and chunk 128
- * or 256 run the whole forward as one tensor-core (tcgen05) kernel; other bf16
- * shapes run the step kernels with chunk_state on the tensor cores where it
+ * multiple of 4.  bf16 inputs with headdim 64 and dstate 64 or 128 run the
+ * whole forward as one tensor-core (tcgen05) kernel (its tiling is its own:
+ * the result does not depend on `chunk`, which the chunked form leaves exact
+ * up to rounding); other bf16 shapes run the step kernels with chunk_state on the tensor cores where it
  * applies (headdim in {32, 64, 128}, dstate in {64, 128, 256}, 128/headdim
  * dividing the heads per group) and the rest in fp32 on the CUDA cores; fp32
  * inputs always take the CUDA-core path (its exact fp32 arithmetic is what the
@@ -476,8 +477,9 @@ const char* ssd_version(void);
  * SSD_ERR_TIMEOUT through its status word instead of hanging (no fault, no
  * trap).  `what` = SSD_DEBUG_CONV_TILE: the convolution's producer stops before
  * tile `index`; SSD_DEBUG_FWD_CARRY: the fused forward does not publish the
- * state leaving chunk `index` (so the next chunk's wait gives up after about a
- * second).  index < 0 turns the hook off.  Process-wide; read on the host when
+ * state leaving run `index` (a run is the group of up to four consecutive
+ * 128-token tiles one cluster of CTAs takes; the next run's wait gives up
+ * after about a second).  index < 0 turns the hook off.  Process-wide; read on the host when
  * a kernel is launched.  Other values of `what` are ignored. */
 #define SSD_DEBUG_CONV_TILE 0
 #define SSD_DEBUG_FWD_CARRY 1

@@ -57,7 +57,9 @@ def test_tensor_core_dispatch_query(lib):
     assert m.tensor_core_steps(4, 1024, 24, 64, 64, 1, 256, flags=m.SSD_FLAG_BF16_STATES) == {
         "chunk_state", "chunk_scan"}
     assert m.tensor_core_steps(1, 512, 2, 128, 256, 1, 256) == {"chunk_state"}
-    assert m.tensor_core_steps(1, 512, 4, 64, 128, 4, 64) == set()  # 1 head per group, chunk 64
+    # the fused kernel tiles the sequence its own way: any chunk
+    assert m.tensor_core_steps(1, 512, 4, 64, 128, 4, 64) == {"chunk_state", "chunk_scan", "fused"}
+    assert m.tensor_core_steps(1, 512, 4, 64, 128, 4, 64, flags=m.SSD_FLAG_SPLIT_STEPS) == set()
 
 
 def test_status_strings(lib):
@@ -79,8 +81,9 @@ def _args(**kw):
 
 def test_workspace_size_is_host_only(lib):
     import mamba_ssd_scan_b200 as m
-    # fused kernel: header (256 B) + a two-slot ring of 1*4 states of 64*64 fp32
-    assert lib.ssd_fwd_workspace_size(ctypes.byref(_args())) == 256 + 2 * 4 * 64 * 64 * 4
+    # fused kernel: header (256 B), the ring's reader counts (2*1*4 ints, in 256 B)
+    # and a two-slot ring of 1*4 states of 64*64 fp32
+    assert lib.ssd_fwd_workspace_size(ctypes.byref(_args())) == 256 + 256 + 2 * 4 * 64 * 64 * 4
     # split steps: header + dt + cumA (1*4*2*256 fp32 each) + fp32 chunk states 1*2*4*64*64
     a = _args(flags=m.SSD_FLAG_SPLIT_STEPS)
     assert lib.ssd_fwd_workspace_size(ctypes.byref(a)) == 256 + 8192 + 8192 + 131072

@@ -5,9 +5,9 @@ The library's test hook (ssd_debug_set_withhold, read by the host launcher)
 makes one producer withhold one hand-off:
   - the convolution's producer warp its first tile: the consumers' waits on
     that tile's mbarrier give up after their iteration limit;
-  - the fused forward the state leaving chunk 0: the CTAs of chunk 1 poll the
-    carry ring until their limit (about a second), raise the abort word, and
-    every CTA stops.
+  - the fused forward the state leaving its first run of tiles (512 tokens):
+    the CTA of the second run that waits for it polls the carry ring until its
+    limit (about a second), raises the abort word, and every CTA stops.
 The status call must then report SSD_ERR_TIMEOUT, and the same process runs
 the operation again with the hook off and checks it against the oracle.  Each
 case runs in a child process with a time limit."""
@@ -47,7 +47,7 @@ print("TIMEOUT-OK")
 
 # bf16, two chunks per sequence, two sequences: the fused path
 FWD = r"""
-b, L, H, P, N, G, Q = 2, 512, 4, 64, 64, 1, 256
+b, L, H, P, N, G, Q = 2, 1024, 4, 64, 64, 1, 256
 inp = synthetic.make_fwd_inputs(b, L, H, P, N, G, torch.bfloat16, seed=11, init_state=True)
 d = {k: (v.cuda() if v is not None else None) for k, v in inp.items()}
 assert "fused" in ssd.tensor_core_steps(b, L, H, P, N, G, Q, torch.bfloat16)
