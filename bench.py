@@ -156,7 +156,10 @@ def algorithmic_cost(cfg, elt):
     bc = tok * G * N * elt
     dtr = tok * H * elt
     vec = b * H * nc * Q * 4
-    states = b * nc * H * P * N * elt     # chunk states are kept in the input dtype
+    # chunk states: fp32 local states (chunk_state out, state passing in), and
+    # the entering states as a hi / lo bf16 pair (state passing out,
+    # chunk_scan in): 4 bytes per element either way
+    states = b * nc * H * P * N * 4
     init = b * H * P * N * 4 if cfg.init_state else 0
     fin = b * H * P * N * 4 if cfg.return_final else 0
     causal = Q * (Q + 1) / 2
@@ -167,7 +170,7 @@ def algorithmic_cost(cfg, elt):
     return {
         "chunk_cumsum": (dtr + 2 * vec, 0.0),
         "chunk_state": (x + bc + 2 * vec + states, flops_state),
-        "state_passing": (2 * states + b * H * nc * 4 + init + fin, 3.0 * states / 4),
+        "state_passing": (2 * states + b * H * nc * 4 + init + fin, 2.0 * states / 4),
         "chunk_scan": (x + 2 * bc + 2 * vec + states + x, flops_scan),
         "path": (x + 2 * bc + dtr + x + init + fin, flops_state + flops_scan),
     }
@@ -586,39 +589,50 @@ def other_workloads(ssd, synthetic, dev, flush, peaks, rank, world, barrier, ran
         y = torch.empty_like(d["x"])
         fin = torch.empty((cfg.batch, cfg.nheads, cfg.headdim, cfg.dstate), device=dev) \
             if cfg.return_final else None
-        ws = torch.empty(ssd.ssd_fwd_workspace_size(cfg.batch, cfg.seqlen, cfg.nheads,
-                                                    cfg.headdim, cfg.dstate, cfg.ngroups,
-                                                    cfg.chunk, cfg.dtype),
-                         dtype=torch.uint8, device=dev)
-
-        def step():
-            ssd.ssd_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["dt_bias"],
-                        cfg.chunk, d["init_state"], y=y, final_state=fin, workspace=ws)
-
-        for _ in range(3):
-            step()
-        torch.cuda.synchronize()
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(steps)]
-        gpu_head_start(2.0)
-        for a, b_ in evs:
-            flush()
-            a.record(stream)
-            step()
-            b_.record(stream)
-        torch.cuda.synchronize()
-        ms = ranks_max(sum(a.elapsed_time(b_) for a, b_ in evs) / steps)
         nbytes = algorithmic_cost(cfg, 2)["path"][0]
+
+        def timed_ms(flags):
+            ws = torch.empty(ssd.ssd_fwd_workspace_size(cfg.batch, cfg.seqlen, cfg.nheads,
+                                                        cfg.headdim, cfg.dstate, cfg.ngroups,
+                                                        cfg.chunk, cfg.dtype, flags=flags),
+                             dtype=torch.uint8, device=dev)
+
+            def step():
+                ssd.ssd_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["dt_bias"],
+                            cfg.chunk, d["init_state"], y=y, final_state=fin, workspace=ws,
+                            flags=flags)
+
+            for _ in range(3):
+                step()
+            torch.cuda.synchronize()
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(steps)]
+            gpu_head_start(2.0)
+            for a, b_ in evs:
+                flush()
+                a.record(stream)
+                step()
+                b_.record(stream)
+            torch.cuda.synchronize()
+            del ws
+            return ranks_max(sum(a.elapsed_time(b_) for a, b_ in evs) / steps)
+
+        ms = timed_ms(0)
         tc = ssd.tensor_core_steps(cfg.batch, cfg.seqlen, cfg.nheads, cfg.headdim, cfg.dstate,
                                    cfg.ngroups, cfg.chunk, cfg.dtype)
         ent = {"tokens_per_s": job_throughput(cfg.tokens, world, ms), "ms": ms,
                "path_bytes": nbytes,
                "hbm_frac_of_path_bytes": nbytes / (ms * 1e-3) / (peaks["hbm_gbs"] * 1e9),
-               "kernels": "fused_fwd" if "fused" in tc else "split"}
+               "kernels": "fused_fwd" if "fused" in tc else "three kernels"}
         if "fused" not in tc:
             ent["kernel_ms"] = split_kernel_ms(ssd, cfg, d, y, fin, dev, flush, steps)
+        # the opt-in single-pass kernel on the same workload, for comparison
+        ms1 = timed_ms(ssd.SSD_FLAG_SINGLE_PASS)
+        ent["single_pass"] = {"ms": ms1, "tokens_per_s": job_throughput(cfg.tokens, world, ms1),
+                              "hbm_frac_of_path_bytes":
+                                  nbytes / (ms1 * 1e-3) / (peaks["hbm_gbs"] * 1e9)}
         out[name] = ent
-        del d, y, fin, ws
+        del d, y, fin
         torch.cuda.empty_cache()
 
     # decode: 1024 successive steps captured in one CUDA graph
@@ -975,15 +989,21 @@ def conv_workloads(ssd, synthetic, dev, flush, peaks, rank, world, ranks_max, st
 
 def split_kernel_ms(ssd, cfg, d, y, fin, dev, flush, steps):
     """Mean duration of each of the four steps (CUDA events between the step
-    entry points, which launch the same kernels ssd_fwd does)."""
+    entry points, which launch the kernels ssd_fwd does: with bf16 on the
+    tensor cores, state passing and chunk_scan in their hi / lo form; ssd_fwd
+    also folds step 1 into chunk_state, which the entry points keep apart)."""
     import torch
     stream = torch.cuda.current_stream()
     nc = -(-cfg.seqlen // cfg.chunk)
     dt_sp = torch.empty((cfg.batch, cfg.nheads, nc, cfg.chunk), device=dev)
     cumA = torch.empty_like(dt_sp)
-    # the step entry points keep fp32 chunk states (the default precision)
+    # fp32 chunk states (the default precision)
     states = torch.empty((cfg.batch, nc, cfg.nheads, cfg.headdim, cfg.dstate), device=dev,
                          dtype=torch.float32)
+    hilo = "chunk_scan" in ssd.tensor_core_steps(cfg.batch, cfg.seqlen, cfg.nheads, cfg.headdim,
+                                                 cfg.dstate, cfg.ngroups, cfg.chunk, cfg.dtype)
+    states_hl = (torch.empty((2,) + tuple(states.shape), device=dev, dtype=torch.bfloat16)
+                 if hilo else None)
     names = ["chunk_cumsum", "chunk_state", "state_passing", "chunk_scan"]
     tot = dict.fromkeys(names, 0.0)
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(steps + 2)]
@@ -999,17 +1019,26 @@ def split_kernel_ms(ssd, cfg, d, y, fin, dev, flush, steps):
         ssd.ssd_chunk_state(d["x"], d["dt"], d["A"], d["B"], d["C"], dt_sp, cumA, cfg.chunk,
                             states=states)
         ev[2].record(stream)
-        ssd.ssd_state_passing(d["x"], d["dt"], d["A"], d["B"], d["C"], cumA, states, cfg.chunk,
-                              init_state=d["init_state"], final_state=fin)
+        if hilo:
+            ssd.ssd_state_passing_hilo(d["x"], d["dt"], d["A"], d["B"], d["C"], cumA, states,
+                                       cfg.chunk, init_state=d["init_state"], final_state=fin,
+                                       states_hl=states_hl)
+        else:
+            ssd.ssd_state_passing(d["x"], d["dt"], d["A"], d["B"], d["C"], cumA, states,
+                                  cfg.chunk, init_state=d["init_state"], final_state=fin)
         ev[3].record(stream)
-        ssd.ssd_chunk_scan(d["x"], d["dt"], d["A"], d["B"], d["C"], dt_sp, cumA, states,
-                           d["D"], cfg.chunk, y=y)
+        if hilo:
+            ssd.ssd_chunk_scan_hilo(d["x"], d["dt"], d["A"], d["B"], d["C"], dt_sp, cumA,
+                                    states_hl, d["D"], cfg.chunk, y=y)
+        else:
+            ssd.ssd_chunk_scan(d["x"], d["dt"], d["A"], d["B"], d["C"], dt_sp, cumA, states,
+                               d["D"], cfg.chunk, y=y)
         ev[4].record(stream)
     torch.cuda.synchronize()
     for ev in evs[2:]:
         for i, n in enumerate(names):
             tot[n] += ev[i].elapsed_time(ev[i + 1])
-    del dt_sp, cumA, states
+    del dt_sp, cumA, states, states_hl
     return {n: tot[n] / steps for n in names}
 
 

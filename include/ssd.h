@@ -80,14 +80,17 @@ typedef enum { SSD_F32 = 0, SSD_BF16 = 1 } ssd_dtype;
  *                and 6.1), applied in the kernel that writes y.  The gate does
  *                not touch the carried state.
  * Supported: 1 <= chunk <= 256; dstate a multiple of 4, <= 256; headdim a
- * multiple of 4.  bf16 inputs with headdim 64 and dstate 64 or 128 run the
- * whole forward as one tensor-core (tcgen05) kernel (its tiling is its own:
- * the result does not depend on `chunk`, which the chunked form leaves exact
- * up to rounding); other bf16 shapes run the step kernels with chunk_state on the tensor cores where it
- * applies (headdim in {32, 64, 128}, dstate in {64, 128, 256}, 128/headdim
- * dividing the heads per group) and the rest in fp32 on the CUDA cores; fp32
- * inputs always take the CUDA-core path (its exact fp32 arithmetic is what the
- * 1e-4 agreement needs). */
+ * multiple of 4.  bf16 inputs run the forward as three tensor-core (tcgen05)
+ * kernels where they apply: chunk_state (with step 1 folded in; headdim in
+ * {32, 64, 128}, dstate in {64, 128, 256}, 128/headdim dividing the heads per
+ * group), state passing, and chunk_scan (headdim 64, dstate 64 or 128, chunk
+ * 128 or 256); the chunk states stay fp32 and reach chunk_scan as hi / lo
+ * bf16 halves.  Steps outside those ranges run in fp32 on the CUDA cores.
+ * With SSD_FLAG_SINGLE_PASS, bf16 inputs with headdim 64 and dstate 64 or 128
+ * run the whole forward as one kernel instead (its tiling is its own: the
+ * result does not depend on `chunk`, which the chunked form leaves exact up
+ * to rounding).  fp32 inputs always take the CUDA-core path (its exact fp32
+ * arithmetic is what the 1e-4 agreement needs). */
 typedef struct {
     int64_t batch, seqlen, nheads, headdim, dstate, ngroups, chunk;
     int32_t dtype;          /* ssd_dtype of x, dt, B, C and y */
@@ -111,10 +114,8 @@ typedef struct {
 #define SSD_FLAG_CUDA_CORES 1   /* force the CUDA-core (FFMA) path */
 #define SSD_FLAG_WHOLE_GROUPS 2 /* tensor-core chunk_scan (bf16-states mode): one CTA
                                    per whole group of heads */
-#define SSD_FLAG_SPLIT_STEPS 4  /* bf16: run the forward as its separate step
-                                   kernels (chunk states in fp32 in the workspace)
-                                   instead of the single fused kernel; for
-                                   comparisons and the per-step checks */
+#define SSD_FLAG_SPLIT_STEPS 4  /* bf16: the forward as its separate step kernels
+                                   (the default; overrides SSD_FLAG_SINGLE_PASS) */
 #define SSD_FLAG_BF16_STATES 8  /* bf16, opt-in: the split steps with the chunk
                                    states stored in bf16 and the carried state
                                    entering the tensor-core state term as one bf16
@@ -122,6 +123,13 @@ typedef struct {
                                    OUTSIDE the stated bf16 tolerance for some inputs
                                    (the carried state's rounding under cancellation
                                    in C . H); never the default */
+#define SSD_FLAG_SINGLE_PASS 16 /* bf16, opt-in: the whole forward as one kernel
+                                   (headdim 64, dstate 64 or 128): tiles of 128
+                                   tokens, the carried state handed from tile to
+                                   tile through the workspace.  Within the same
+                                   tolerance as the default; measured slower on
+                                   B200 than the three kernels (its per-tile
+                                   pipeline is latency-bound) */
 
 /* Bytes of device workspace ssd_fwd needs for these sizes (0 on invalid
  * sizes).  Only sizes, dtype and flags are read; pointers may be NULL. */
@@ -129,8 +137,8 @@ size_t ssd_fwd_workspace_size(const ssd_fwd_args* args);
 
 /* Which steps of ssd_fwd run on the tensor cores for these sizes, dtype and
  * flags: bit 0 = chunk_state, bit 1 = chunk_scan, bit 2 = the whole forward in
- * one fused kernel (0 = all on CUDA cores, or invalid sizes).  Host-only;
- * pointers are not read. */
+ * one kernel (SSD_FLAG_SINGLE_PASS; bits 0 and 1 are then set too) (0 = all
+ * on CUDA cores, or invalid sizes).  Host-only; pointers are not read. */
 #define SSD_TC_CHUNK_STATE 1
 #define SSD_TC_CHUNK_SCAN 2
 #define SSD_TC_FUSED 4
@@ -216,9 +224,26 @@ ssd_status ssd_state_passing(const ssd_fwd_args* args, const float* cumA, void* 
 
 /* Step 4: y[l,p] = sum_{j<=l in chunk} exp(cumA[l]-cumA[j]) (C_l.B_j) dt[j] x[j,p]
  *                 + exp(cumA[l]) sum_n C_l[n] H_in[p,n] + D x[l,p],
- * with H_in the state entering the chunk (states after step 3). */
+ * with H_in the state entering the chunk (states after step 3).  With fp32
+ * states the state term is formed in fp32 on the CUDA cores; the tensor-core
+ * kernel takes the _hilo form below. */
 ssd_status ssd_chunk_scan(const ssd_fwd_args* args, const float* dt, const float* cumA,
                           const void* states, void* stream);
+
+/* Steps 3 and 4 as ssd_fwd runs them for bf16 inputs on the tensor cores
+ * (ssd_fwd_tensor_core_steps reports SSD_TC_CHUNK_SCAN; SSD_ERR_UNSUPPORTED
+ * otherwise).  The state entering each chunk goes to chunk_scan as two bf16
+ * halves, hi = bf16(H) and lo = bf16(H - hi), so that the tensor-core state
+ * term C . (hi + lo) carries the fp32 state to about 2^-17 of its size:
+ *   states_hl  [2][batch, nc, nheads, headdim, dstate] bf16 (hi, then lo),
+ *              device, caller-owned, 16-byte aligned.
+ * ssd_state_passing_hilo reads the fp32 local states of step 2 (`states`, not
+ * modified) and writes the entering states to states_hl (and final_state if
+ * given); ssd_chunk_scan_hilo writes y from states_hl. */
+ssd_status ssd_state_passing_hilo(const ssd_fwd_args* args, const float* cumA,
+                                  const float* states, void* states_hl, void* stream);
+ssd_status ssd_chunk_scan_hilo(const ssd_fwd_args* args, const float* dt, const float* cumA,
+                               const void* states_hl, void* stream);
 
 /* ---- backward --------------------------------------------------------------- */
 /* The backward pass of ssd_fwd (without the output gate): the gradients of
@@ -479,10 +504,14 @@ const char* ssd_version(void);
  * tile `index`; SSD_DEBUG_FWD_CARRY: the fused forward does not publish the
  * state leaving run `index` (a run is the group of up to four consecutive
  * 128-token tiles one cluster of CTAs takes; the next run's wait gives up
- * after about a second).  index < 0 turns the hook off.  Process-wide; read on the host when
- * a kernel is launched.  Other values of `what` are ignored. */
+ * after about a second; SSD_FLAG_SINGLE_PASS only); SSD_DEBUG_SCAN_DECAYS: the
+ * tensor-core chunk_scan does not hand the decays of the first head of chunk
+ * `index` to its workers, whose waits give up.  index < 0 turns the hook off.
+ * Process-wide; read on the host when a kernel is launched.  Other values of
+ * `what` are ignored. */
 #define SSD_DEBUG_CONV_TILE 0
 #define SSD_DEBUG_FWD_CARRY 1
+#define SSD_DEBUG_SCAN_DECAYS 2
 void ssd_debug_set_withhold(int what, int64_t index);
 
 #ifdef __cplusplus

@@ -17,11 +17,13 @@ import torch
 __all__ = [
     "SsdError", "ssd_fwd", "ssd_fwd_workspace_size", "ssd_fwd_check_status", "ssd_fwd_no_alloc",
     "ssd_fwd_no_alloc_check_status", "ssd_fwd_no_alloc_scratch_bytes", "ssd_debug_set_withhold",
-    "SSD_DEBUG_CONV_TILE", "SSD_DEBUG_FWD_CARRY",
+    "SSD_DEBUG_CONV_TILE", "SSD_DEBUG_FWD_CARRY", "SSD_DEBUG_SCAN_DECAYS",
     "ssd_fwd_tensor_core_steps", "tensor_core_steps", "ssd_chunk_cumsum", "ssd_chunk_state",
-    "ssd_state_passing", "ssd_chunk_scan", "ssd_state_update", "ssd_status_string",
+    "ssd_state_passing", "ssd_chunk_scan", "ssd_state_passing_hilo", "ssd_chunk_scan_hilo",
+    "ssd_state_update", "ssd_status_string",
     "ssd_version", "lib_path", "load_library", "SSD_FLAG_CUDA_CORES", "SSD_FLAG_WHOLE_GROUPS",
-    "SSD_FLAG_SPLIT_STEPS", "SSD_FLAG_BF16_STATES", "SSD_TC_CHUNK_STATE", "SSD_TC_CHUNK_SCAN",
+    "SSD_FLAG_SPLIT_STEPS", "SSD_FLAG_BF16_STATES", "SSD_FLAG_SINGLE_PASS", "SSD_TC_CHUNK_STATE",
+    "SSD_TC_CHUNK_SCAN",
     "SSD_TC_FUSED",
     "ssd_causal_conv1d", "ssd_conv1d_update", "ssd_conv1d_check_status",
     "ssd_bwd", "ssd_bwd_workspace_size", "ssd_selective_scan", "ssd_selective_scan_workspace_size",
@@ -37,6 +39,7 @@ SSD_FLAG_CUDA_CORES = 1
 SSD_FLAG_WHOLE_GROUPS = 2
 SSD_FLAG_SPLIT_STEPS = 4
 SSD_FLAG_BF16_STATES = 8
+SSD_FLAG_SINGLE_PASS = 16
 SSD_TC_CHUNK_STATE, SSD_TC_CHUNK_SCAN, SSD_TC_FUSED = 1, 2, 4
 
 _i64, _i32, _vp, _sz = ctypes.c_int64, ctypes.c_int32, ctypes.c_void_p, ctypes.c_size_t
@@ -156,6 +159,10 @@ def load_library():
     lib.ssd_state_passing.argtypes = [F, _vp, _vp, _vp]
     lib.ssd_chunk_scan.restype = ctypes.c_int
     lib.ssd_chunk_scan.argtypes = [F, _vp, _vp, _vp, _vp]
+    lib.ssd_state_passing_hilo.restype = ctypes.c_int
+    lib.ssd_state_passing_hilo.argtypes = [F, _vp, _vp, _vp, _vp]
+    lib.ssd_chunk_scan_hilo.restype = ctypes.c_int
+    lib.ssd_chunk_scan_hilo.argtypes = [F, _vp, _vp, _vp, _vp]
     lib.ssd_state_update.restype = ctypes.c_int
     lib.ssd_state_update.argtypes = [ctypes.POINTER(SsdStateUpdateArgs), _vp]
     BW = ctypes.POINTER(SsdBwdArgs)
@@ -261,7 +268,8 @@ def ssd_fwd_workspace_size(batch, seqlen, nheads, headdim, dstate, ngroups, chun
 def ssd_fwd_tensor_core_steps(batch, seqlen, nheads, headdim, dstate, ngroups, chunk,
                               dtype=torch.bfloat16, flags: int = 0) -> int:
     """Bitmask of the ssd_fwd steps that run on the tensor cores for these sizes
-    (1 = chunk_state, 2 = chunk_scan, 4 = the whole forward as one fused kernel)."""
+    (1 = chunk_state, 2 = chunk_scan, 4 = the whole forward as one kernel, with
+    SSD_FLAG_SINGLE_PASS)."""
     a = SsdFwdArgs()
     a.batch, a.seqlen, a.nheads, a.headdim, a.dstate, a.ngroups, a.chunk = (
         batch, seqlen, nheads, headdim, dstate, ngroups, chunk)
@@ -373,6 +381,7 @@ def ssd_bwd(x, dt, A, B, C, dy, D=None, dt_bias=None, chunk: int = 256, init_sta
 
 SSD_DEBUG_CONV_TILE = 0
 SSD_DEBUG_FWD_CARRY = 1
+SSD_DEBUG_SCAN_DECAYS = 2
 
 
 def ssd_debug_set_withhold(what: int, index: int) -> None:
@@ -491,6 +500,34 @@ def ssd_chunk_scan(x, dt, A, B, C, dt_sp, cumA, states, D=None, chunk: int = 256
     a = _fwd_args(x, dt, A, B, C, D, None, chunk, None, y, None, flags, z)
     _check(lib.ssd_chunk_scan(ctypes.byref(a), _ptr(dt_sp), _ptr(cumA), _ptr(states),
                               _stream_ptr(stream)), "ssd_chunk_scan")
+    return y
+
+
+def ssd_state_passing_hilo(x, dt, A, B, C, cumA, states, chunk: int = 256, init_state=None,
+                           final_state=None, *, states_hl=None, stream=None, flags: int = 0):
+    """Step 3 as ssd_fwd runs it for bf16 on the tensor cores: the fp32 local
+    ``states`` (not modified) -> the states entering each chunk as hi / lo bf16
+    halves, returned as ``states_hl`` [2, b, nc, H, P, N] (hi, then lo).
+    Writes ``final_state`` if given."""
+    lib = load_library()
+    _, sshape = _intermediate_shapes(x, B, chunk)
+    states_hl = states_hl if states_hl is not None else torch.empty(
+        (2,) + sshape, dtype=torch.bfloat16, device=x.device)
+    a = _fwd_args(x, dt, A, B, C, None, None, chunk, init_state, None, final_state, flags)
+    _check(lib.ssd_state_passing_hilo(ctypes.byref(a), _ptr(cumA), _ptr(states), _ptr(states_hl),
+                                      _stream_ptr(stream)), "ssd_state_passing_hilo")
+    return states_hl
+
+
+def ssd_chunk_scan_hilo(x, dt, A, B, C, dt_sp, cumA, states_hl, D=None, chunk: int = 256, *,
+                        y=None, stream=None, z=None, flags: int = 0):
+    """Step 4 on the tensor cores from the hi / lo entering states of
+    ssd_state_passing_hilo (times silu(z) when the gate z is given)."""
+    lib = load_library()
+    y = y if y is not None else torch.empty_like(x)
+    a = _fwd_args(x, dt, A, B, C, D, None, chunk, None, y, None, flags, z)
+    _check(lib.ssd_chunk_scan_hilo(ctypes.byref(a), _ptr(dt_sp), _ptr(cumA), _ptr(states_hl),
+                                   _stream_ptr(stream)), "ssd_chunk_scan_hilo")
     return y
 
 

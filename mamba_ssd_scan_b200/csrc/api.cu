@@ -43,8 +43,12 @@ bool check_ptr(const void* p, bool allow_null, bool need_align) {
 }
 
 struct WsLayout {
-    size_t status, dt, cumA, states, total;
+    size_t status, dt, cumA, states, states_hl, total;
 };
+
+bool use_tc(int dtype, int flags) {
+    return dtype == SSD_BF16 && (flags & SSD_FLAG_CUDA_CORES) == 0;
+}
 
 // Chunk states in the split-step path are fp32, except in the opt-in
 // bf16-states mode (bf16 inputs with SSD_FLAG_BF16_STATES).
@@ -52,17 +56,29 @@ bool bf16_states(const ssd_fwd_args& a) {
     return a.dtype == SSD_BF16 && (a.flags & SSD_FLAG_BF16_STATES) != 0;
 }
 
+// With fp32 states and the tensor-core chunk_scan, state passing also writes
+// the entering states as hi / lo bf16 halves, the operand that kernel takes.
+bool states_hilo(const ssd_fwd_args& a) {
+    if (!use_tc(a.dtype, a.flags) || bf16_states(a)) return false;
+    ssd::FwdParams q;
+    q.headdim = a.headdim;
+    q.dstate = a.dstate;
+    q.chunk = a.chunk;
+    return ssd::chunk_scan_tc_supported(q);
+}
+
 WsLayout ws_layout(const ssd_fwd_args& a) {
     const int64_t nc = (a.seqlen + a.chunk - 1) / a.chunk;
     const size_t vec = (size_t)a.batch * a.nheads * nc * a.chunk * sizeof(float);
+    const size_t n_st = (size_t)a.batch * nc * a.nheads * a.headdim * a.dstate;
     const size_t elt = bf16_states(a) ? 2 : 4;
-    const size_t st = (size_t)a.batch * nc * a.nheads * a.headdim * a.dstate * elt;
     WsLayout w;
     w.status = 0;
     w.dt = w.status + kAlign;
     w.cumA = w.dt + round_up(vec);
     w.states = w.cumA + round_up(vec);
-    w.total = w.states + round_up(st);
+    w.states_hl = w.states + round_up(n_st * elt);
+    w.total = w.states_hl + (states_hilo(a) ? round_up(2 * n_st * 2) : 0);
     return w;
 }
 
@@ -121,14 +137,16 @@ FwdParams make_params(const ssd_fwd_args* a) {
     p.z = a->z;
     p.dt = p.cumA = nullptr;
     p.states = nullptr;
+    p.states_hl = nullptr;
     p.status = nullptr;
     return p;
 }
 
-// The whole forward in one kernel: bf16 inputs in its shape range, unless the
-// caller asks for the CUDA cores, the split steps or the bf16-states mode.
+// The whole forward in one kernel: asked for with SSD_FLAG_SINGLE_PASS, for
+// bf16 inputs in its shape range, unless the caller also asks for the CUDA
+// cores, the split steps or the bf16-states mode.
 bool use_fused(const ssd_fwd_args& a) {
-    if (a.dtype != SSD_BF16) return false;
+    if (a.dtype != SSD_BF16 || !(a.flags & SSD_FLAG_SINGLE_PASS)) return false;
     if (a.flags & (SSD_FLAG_CUDA_CORES | SSD_FLAG_SPLIT_STEPS | SSD_FLAG_BF16_STATES)) return false;
     return ssd::fused_fwd_supported(make_params(&a));
 }
@@ -148,9 +166,6 @@ cudaError_t run_cumsum(const FwdParams& p, int dtype, cudaStream_t s) {
 }
 // The tensor-core kernels take bf16 inputs in their shape range unless the
 // caller forces the CUDA-core path; everything else runs on the FFMA kernels.
-bool use_tc(int dtype, int flags) {
-    return dtype == SSD_BF16 && (flags & SSD_FLAG_CUDA_CORES) == 0;
-}
 // state passing is templated on the type the states are stored in
 cudaError_t run_state_passing(const FwdParams& p, int dtype, cudaStream_t s) {
     return (dtype == SSD_BF16 && !p.states_f32) ? ssd::launch_state_passing<__nv_bfloat16>(p, s)
@@ -162,11 +177,13 @@ cudaError_t run_chunk_state(const FwdParams& p, int dtype, int flags, cudaStream
     return dtype == SSD_BF16 ? ssd::launch_chunk_state_ffma<__nv_bfloat16>(p, s)
                              : ssd::launch_chunk_state_ffma<float>(p, s);
 }
-// The tensor-core chunk_scan takes its carried state as one bf16 operand, so
-// it runs only in the opt-in bf16-states mode; with fp32 states the CUDA-core
-// kernel forms the state term in fp32.
+// The tensor-core chunk_scan takes the carried state as bf16 operands: the
+// hi / lo pair that state passing wrote from the fp32 states, or, in the
+// opt-in bf16-states mode, the bf16 states alone.  fp32 states without the
+// pair (the step entry point) go to the CUDA-core kernel, which forms the
+// state term in fp32.
 cudaError_t run_chunk_scan(const FwdParams& p, int dtype, int flags, cudaStream_t s) {
-    if (use_tc(dtype, flags) && !p.states_f32 && ssd::chunk_scan_tc_supported(p))
+    if (use_tc(dtype, flags) && (p.states_hl || !p.states_f32) && ssd::chunk_scan_tc_supported(p))
         return ssd::launch_chunk_scan_tc(p, s);
     return dtype == SSD_BF16 ? ssd::launch_chunk_scan_ffma<__nv_bfloat16>(p, s)
                              : ssd::launch_chunk_scan_ffma<float>(p, s);
@@ -274,12 +291,12 @@ ssd_status check_bwd_sizes(const ssd_bwd_args* a) {
 }  // namespace
 
 namespace {
-std::atomic<int64_t> g_withhold[2] = {{-1}, {-1}};
+std::atomic<int64_t> g_withhold[3] = {{-1}, {-1}, {-1}};
 }  // namespace
 
 namespace ssd {
 int64_t debug_withhold(int what) {
-    return (what == 0 || what == 1) ? g_withhold[what].load(std::memory_order_relaxed) : -1;
+    return (what >= 0 && what < 3) ? g_withhold[what].load(std::memory_order_relaxed) : -1;
 }
 }  // namespace ssd
 
@@ -296,7 +313,7 @@ int ssd_fwd_tensor_core_steps(const ssd_fwd_args* a) {
     if (use_fused(*a)) return SSD_TC_CHUNK_STATE | SSD_TC_CHUNK_SCAN | SSD_TC_FUSED;
     const FwdParams p = make_params(a);
     return (ssd::chunk_state_tc_supported(p) ? SSD_TC_CHUNK_STATE : 0) |
-           ((!p.states_f32 && ssd::chunk_scan_tc_supported(p)) ? SSD_TC_CHUNK_SCAN : 0);
+           ((states_hilo(*a) || bf16_states(*a)) && ssd::chunk_scan_tc_supported(p) ? SSD_TC_CHUNK_SCAN : 0);
 }
 
 ssd_status ssd_fwd(const ssd_fwd_args* a, void* stream) {
@@ -321,6 +338,7 @@ ssd_status ssd_fwd(const ssd_fwd_args* a, void* stream) {
     p.dt = reinterpret_cast<float*>(ws + w.dt);
     p.cumA = reinterpret_cast<float*>(ws + w.cumA);
     p.states = ws + w.states;
+    p.states_hl = states_hilo(*a) ? ws + w.states_hl : nullptr;
     p.status = reinterpret_cast<int*>(ws + w.status);
     // The first kernel is a plain launch (it waits for all earlier work on
     // the stream); the later ones go out with programmatic dependent launch,
@@ -575,6 +593,38 @@ ssd_status ssd_chunk_scan(const ssd_fwd_args* a, const float* dt, const float* c
     return to_status(run_chunk_scan(p, a->dtype, a->flags, static_cast<cudaStream_t>(stream)));
 }
 
+ssd_status ssd_state_passing_hilo(const ssd_fwd_args* a, const float* cumA, const float* states,
+                                  void* states_hl, void* stream) {
+    ssd_status st = check_fwd_sizes(a);
+    if (st != SSD_OK) return st;
+    if (!states_hilo(*a)) return SSD_ERR_UNSUPPORTED;
+    if (!check_ptr(cumA, false, true) || !check_ptr(states, false, true) ||
+        !check_ptr(states_hl, false, true) || !check_ptr(a->init_state, true, true) ||
+        !check_ptr(a->final_state, true, true))
+        return SSD_ERR_INVALID_ARG;
+    FwdParams p = make_params(a);
+    p.cumA = const_cast<float*>(cumA);
+    p.states = const_cast<float*>(states);
+    p.states_hl = states_hl;
+    return to_status(run_state_passing(p, a->dtype, static_cast<cudaStream_t>(stream)));
+}
+
+ssd_status ssd_chunk_scan_hilo(const ssd_fwd_args* a, const float* dt, const float* cumA,
+                               const void* states_hl, void* stream) {
+    ssd_status st = check_fwd_sizes(a);
+    if (st != SSD_OK) return st;
+    if (!states_hilo(*a)) return SSD_ERR_UNSUPPORTED;
+    if ((st = check_fwd_inputs(a)) != SSD_OK) return st;
+    if (!check_ptr(a->y, false, true) || !check_ptr(dt, false, true) ||
+        !check_ptr(cumA, false, true) || !check_ptr(states_hl, false, true))
+        return SSD_ERR_INVALID_ARG;
+    FwdParams p = make_params(a);
+    p.dt = const_cast<float*>(dt);
+    p.cumA = const_cast<float*>(cumA);
+    p.states_hl = const_cast<void*>(states_hl);
+    return to_status(run_chunk_scan(p, a->dtype, a->flags, static_cast<cudaStream_t>(stream)));
+}
+
 ssd_status ssd_causal_conv1d(const ssd_conv1d_args* a, void* stream) {
     if (!a) return SSD_ERR_INVALID_ARG;
     if (a->batch <= 0 || a->seqlen <= 0 || a->channels <= 0 || a->width <= 0)
@@ -716,7 +766,7 @@ const char* ssd_last_cuda_error(void) {
 }
 
 void ssd_debug_set_withhold(int what, int64_t index) {
-    if (what == 0 || what == 1) g_withhold[what].store(index < 0 ? -1 : index, std::memory_order_relaxed);
+    if (what >= 0 && what < 3) g_withhold[what].store(index < 0 ? -1 : index, std::memory_order_relaxed);
 }
 
 const char* ssd_version(void) { return "ssd_b200 0.1.0 (sm_100a)"; }

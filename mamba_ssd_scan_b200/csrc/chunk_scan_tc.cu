@@ -102,17 +102,22 @@ struct ScanTile {
     static constexpr int MK0_BYTES = 2 * 128 * 128;
     static constexpr int X_OFF = MK0_OFF + MK0_BYTES;
     static constexpr int X_BYTES = QMAX * 128;
+    // the entering state, in 64-wide K blocks of PD rows (8 KB): the hi
+    // blocks, then one slot for lo block 0 (with NST = 128, lo block 1 reuses
+    // hi block 0's slot once the MMAs that read it are done)
     static constexpr int H_OFF = X_OFF + X_BYTES;
-    static constexpr int H_BYTES = (NST / 64) * PD * 128;
+    static constexpr int H_SLOT = PD * 128;
+    static constexpr int H_BYTES = (NST / 64 + 1) * H_SLOT;
     // per-head decays, two buffers filled by the loader warp:
-    // [log2e * cumA (QMAX) | dt (QMAX) | D, padding (4)] fp32
+    // [log2e * cumA (QMAX) | dt (QMAX) | D, max dt, padding (4)] fp32
     static constexpr int DEC_FLOATS = 2 * QMAX + 4;
     static constexpr int DEC_OFF = H_OFF + H_BYTES;
     static constexpr int RINV_OFF = DEC_OFF + 2 * DEC_FLOATS * 4;  // per-row CB scale, 2 tiles
     static constexpr int CBD_OFF = RINV_OFF + 2 * 128 * 4;   // per-row C_l . B_l, 2 tiles
     static constexpr int NORM_OFF = CBD_OFF + 2 * 128 * 4;   // |C_r|^2 per row, max |B_j|^2 partials
     static constexpr int CTAB_OFF = NORM_OFF + (256 + 8) * 4;  // per worker warp: 32 column factors
-    static constexpr int BAR_OFF = CTAB_OFF + NWORK * 32 * 4;
+    static constexpr int XMAX_OFF = CTAB_OFF + NWORK * 32 * 4;  // [2][worker warp]: max |x| bits
+    static constexpr int BAR_OFF = XMAX_OFF + 2 * NWORK * 4;
     static constexpr int SMEM = BAR_OFF + 32 * 8 + 1024;
     static_assert(SMEM <= 232448, "shared memory budget");
 };
@@ -138,7 +143,7 @@ enum : int {
     B_CB_LOAD = 0, B_CB_DONE, B_CB_PACKED, B_X_FULL, B_H_FULL, B_H_FREE, B_X_FREE,
     B_MK_FULL, B_MK_EMPTY = B_MK_FULL + 2, B_ACC_FULL = B_MK_EMPTY + 2,
     B_ACC_EMPTY = B_ACC_FULL + 2, B_DEC_FULL = B_ACC_EMPTY + 2, B_DEC_FREE = B_DEC_FULL + 2,
-    B_Y_STAGED = B_DEC_FREE + 2, B_Y_READ, B_MK1A_FULL, B_COUNT
+    B_Y_STAGED = B_DEC_FREE + 2, B_Y_READ, B_MK1A_FULL, B_H0_FREE, B_H1_FULL, B_XCONV, B_COUNT
 };
 
 // Bounded wait that also gives up when another role has aborted: a few
@@ -157,21 +162,12 @@ __device__ __forceinline__ bool wait_bar(uint32_t mbar, uint32_t parity, volatil
     return false;
 }
 
-__device__ __forceinline__ void unpack_f16x32(const uint32_t (&r)[16], float (&v)[32]) {
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&r[i]));
-        v[2 * i] = f.x;
-        v[2 * i + 1] = f.y;
-    }
-}
-
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
     const __half2 v = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-// 32 bf16 values of one row (16 packed pairs) into the K-major SW128 operand
+// 32 fp16 values of one row (16 packed pairs) into the K-major SW128 operand
 __device__ __forceinline__ void store_group_packed(uint32_t mbase, uint32_t row, int j0,
                                                    const uint32_t (&o)[16]) {
     const uint32_t dst = mbase + (j0 >> 6) * (128 * 128);
@@ -181,15 +177,15 @@ __device__ __forceinline__ void store_group_packed(uint32_t mbase, uint32_t row,
         st_shared_v4(dst + sw128(row, c0 + i), o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
 }
 
-// 32 masked values of one row -> bf16, into the K-major SW128 operand
+// 32 masked values of one row -> fp16, into the K-major SW128 operand
 __device__ __forceinline__ void store_group(uint32_t mbase, uint32_t row, int j0, const float (&v)[32]) {
     const uint32_t dst = mbase + (j0 >> 6) * (128 * 128);
     const int c0 = (j0 & 63) >> 3;
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-        st_shared_v4(dst + sw128(row, c0 + i), pack_bf16x2(v[8 * i + 0], v[8 * i + 1]),
-                     pack_bf16x2(v[8 * i + 2], v[8 * i + 3]), pack_bf16x2(v[8 * i + 4], v[8 * i + 5]),
-                     pack_bf16x2(v[8 * i + 6], v[8 * i + 7]));
+        st_shared_v4(dst + sw128(row, c0 + i), pack_f16x2(v[8 * i + 0], v[8 * i + 1]),
+                     pack_f16x2(v[8 * i + 2], v[8 * i + 3]), pack_f16x2(v[8 * i + 4], v[8 * i + 5]),
+                     pack_f16x2(v[8 * i + 6], v[8 * i + 7]));
 }
 
 __device__ __forceinline__ void store_zero_group(uint32_t mbase, uint32_t row, int j0) {
@@ -205,11 +201,21 @@ __device__ __forceinline__ void store_zero_group(uint32_t mbase, uint32_t row, i
 // writes there).  cum2 holds log2(e) * cumA, so every decay is one exp2.  The
 // diagonal entry (j = l, decay 1) is left out of the operand: the epilogue
 // adds (C_l . B_l dt_l + D) x_l in fp32, so the term that is often the row's
-// largest, and the D skip, are not rounded to bf16.  cbd is the row's C_l . B_l
+// largest, and the D skip, are not rounded.  cbd is the row's C_l . B_l
 // (fp32, saved when CB was packed).
+//
+// The operand is fp16 (2^-11 relative rounding, against bf16's 2^-8), so each
+// row carries a power-of-two scale rs_l into fp16's range: row l holds
+// m[l,j] = CBp[l,j] k_j rs_l, CBp the packed CB (|CBp| < 2^14) and k_j =
+// 2^{ref - c_j} dt_j (fast) or 2^{c_l - c_j} dt_j (steep).  For j < l, c_j >=
+// c_l, so |m[l,j]| <= 2^14 2^{ref - c_l} dmax rs_l (2^0 for 2^{ref - c_l} when
+// steep), dmax the chunk's largest dt; rs_l brings that bound to 2^15, below
+// fp16's 65504, so nothing overflows and the row's largest entries keep every
+// bit.  The epilogue factor f_l undoes rs_l.
 struct RowPlan {
     float ref, cl, c_first;
     float f, w;      // the row's epilogue factor and diagonal weight
+    float rs;        // the row's power-of-two scale into fp16 range
     bool fast;       // factored decays (warp-uniform)
     int rb;          // 32-row block index of the rows
     uint32_t row;    // TMEM lane = Mk row
@@ -218,8 +224,8 @@ struct RowPlan {
 
 template <int TT>
 __device__ __forceinline__ RowPlan plan_rows(uint32_t tmem, const float* cum2, const float* dtv,
-                                             float rinv, float cbd, float Dh, int qd, int lane,
-                                             int Lc) {
+                                             float rinv, float cbd, float Dh, float dmax, int qd,
+                                             int lane, int Lc) {
     RowPlan r;
     const int lb = block_row(TT, qd);
     r.rb = lb >> 5;
@@ -232,7 +238,11 @@ __device__ __forceinline__ RowPlan plan_rows(uint32_t tmem, const float* cum2, c
     r.fast = (r.c_first - c_last) <= kFastSpan;
     r.ref = r.fast ? 0.5f * (r.c_first + c_last) : r.c_first;
     r.cl = cum2[lb + lane];
-    r.f = r.fast ? rinv * ex2(r.cl - r.ref) : rinv;
+    const float lg = (r.fast ? r.ref - r.cl : 0.0f) + __log2f(fmaxf(16384.0f * dmax, 1e-30f));
+    const int e = min(120, max(-120, 15 - static_cast<int>(ceilf(fminf(fmaxf(lg, -200.0f), 200.0f)))));
+    r.rs = __int_as_float((127 + e) << 23);
+    const float irs = __int_as_float((127 - e) << 23);
+    r.f = (r.fast ? rinv * ex2(r.cl - r.ref) : rinv) * irs;
     r.w = fmaf(cbd, dtv[lb + lane], Dh);
     return r;
 }
@@ -253,23 +263,29 @@ __device__ __forceinline__ void mask_group(const RowPlan& r, int g, uint32_t mba
     ctab[lane] = cj;
     __syncwarp();
     const float4* ct = reinterpret_cast<const float4*>(ctab);
+    const float2 rs2 = make_float2(r.rs, r.rs);
     if (g < r.rb && r.fast) {  // below the diagonal block: packed fp32x2 products
         uint32_t o[16];
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const float4 c = ct[i];
-            const float2 a0 = __half22float2(*reinterpret_cast<const __half2*>(&raw[2 * i]));
-            const float2 a1 = __half22float2(*reinterpret_cast<const __half2*>(&raw[2 * i + 1]));
+            const float2 a0 = __fmul2_rn(__half22float2(*reinterpret_cast<const __half2*>(&raw[2 * i])), rs2);
+            const float2 a1 = __fmul2_rn(__half22float2(*reinterpret_cast<const __half2*>(&raw[2 * i + 1])), rs2);
             const float2 m0 = __fmul2_rn(a0, make_float2(c.x, c.y));
             const float2 m1 = __fmul2_rn(a1, make_float2(c.z, c.w));
-            o[2 * i] = pack_bf16x2(m0.x, m0.y);
-            o[2 * i + 1] = pack_bf16x2(m1.x, m1.y);
+            o[2 * i] = pack_f16x2(m0.x, m0.y);
+            o[2 * i + 1] = pack_f16x2(m1.x, m1.y);
         }
         store_group_packed(mbase, r.row, j0, o);
         return;
     }
     float v[32];
-    unpack_f16x32(raw, v);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const float2 f = __fmul2_rn(__half22float2(*reinterpret_cast<const __half2*>(&raw[i])), rs2);
+        v[2 * i] = f.x;
+        v[2 * i + 1] = f.y;
+    }
     if (g < r.rb) {  // below the diagonal block, steep row block
         const float rr = ex2(r.cl - r.c_first);
 #pragma unroll
@@ -303,25 +319,34 @@ __device__ __forceinline__ void mask_group(const RowPlan& r, int g, uint32_t mba
 
 // Per-head MMAs, issued by the control thread.  Descriptors are built once;
 // each K step only advances their start-address field (address / 16).
-// State term of one tile: C_t (K-major, NST wide) x H_in^T (K-major).
-template <int NST>
-__device__ __forceinline__ void issue_state(uint32_t d_tmem, uint64_t dA, uint64_t dB) {
+// State term of one tile, one 64-wide K block: C_t's K block ka (K-major) x
+// the state block in slot hs (K-major); ACC: add to the accumulator.
+__device__ __forceinline__ void issue_state_kb(uint32_t d_tmem, uint64_t dA, uint64_t dB, int ka,
+                                               int hs, bool acc) {
 #pragma unroll
-    for (int k = 0; k < NST / 16; ++k) {
-        const uint32_t ka = ((k >> 2) * (QMAX * 128) + (k & 3) * 32) >> 4;
-        const uint32_t kb = ((k >> 2) * (PD * 128) + (k & 3) * 32) >> 4;
-        mma_bf16(d_tmem, dA + ka, dB + kb, idesc_bf16(128, PD, false, false), k > 0 ? 1u : 0u);
+    for (int k = 0; k < 4; ++k) {
+        const uint32_t oa = (ka * (QMAX * 128) + k * 32) >> 4;
+        const uint32_t ob = (hs * (PD * 128) + k * 32) >> 4;
+        mma_bf16(d_tmem, dA + oa, dB + ob, idesc_bf16(128, PD, false, false), (acc || k > 0) ? 1u : 0u);
     }
 }
-// Intra-chunk term of one tile: Mk_t (K-major) x x (MN-major), K steps
-// [K0, K1) of 16; FRESH: the first of them overwrites the accumulator.
+// The state term's K blocks that are resident when the head starts: every hi
+// block, then lo block 0 (when the state comes as a hi / lo pair).
+template <int NST>
+__device__ __forceinline__ void issue_state(uint32_t d_tmem, uint64_t dA, uint64_t dB, bool hl) {
+#pragma unroll
+    for (int kb = 0; kb < NST / 64; ++kb) issue_state_kb(d_tmem, dA, dB, kb, kb, kb > 0);
+    if (hl) issue_state_kb(d_tmem, dA, dB, 0, NST / 64, true);
+}
+// Intra-chunk term of one tile: Mk_t (K-major) x x (MN-major), both fp16, K
+// steps [K0, K1) of 16; FRESH: the first of them overwrites the accumulator.
 template <int K0, int K1, bool FRESH>
 __device__ __forceinline__ void issue_intra(uint32_t d_tmem, uint64_t dA, uint64_t dB) {
 #pragma unroll
     for (int k = K0; k < K1; ++k) {
         const uint32_t ka = ((k >> 2) * (128 * 128) + (k & 3) * 32) >> 4;
         const uint32_t kb = (k * 2048) >> 4;
-        mma_bf16(d_tmem, dA + ka, dB + kb, idesc_bf16(128, PD, false, true),
+        mma_bf16(d_tmem, dA + ka, dB + kb, idesc_f16(128, PD, false, true),
                  (FRESH && k == K0) ? 0u : 1u);
     }
 }
@@ -333,7 +358,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                          const __grid_constant__ CUtensorMap tm_x,
                          const __grid_constant__ CUtensorMap tm_h,
                          const __grid_constant__ CUtensorMap tm_y,
-                         const __grid_constant__ CUtensorMap tm_z, int hb_size) {
+                         const __grid_constant__ CUtensorMap tm_z, int hb_size, int64_t withhold) {
     using T = ScanTile<NST>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -355,6 +380,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t sC = smem_u32(smem + T::C_OFF), sB = smem_u32(smem + T::B_OFF);
     const uint32_t sM0 = smem_u32(smem + T::MK0_OFF), sM1 = sB;
     const uint32_t sX = smem_u32(smem + T::X_OFF), sH = smem_u32(smem + T::H_OFF);
+    // hi / lo state operand (else the bf16 states alone); with NST = 128 the
+    // second lo block is loaded while the head's MMAs run
+    const bool hl = p.states_hl != nullptr;
+    const bool late_lo = hl && NST == 128;
     // y of one head is staged in tile 1's mask buffer, in its K columns
     // 0-127 (rewritten for every head, never a zero group), between the MMA
     // that read that buffer and the next mask, and leaves by TMA
@@ -366,7 +395,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             uint32_t count = 1;
             if (i == B_CB_PACKED) count = NMASK;
             if (i == B_MK_FULL || i == B_MK_FULL + 1 || i == B_ACC_EMPTY || i == B_ACC_EMPTY + 1 ||
-                i == B_DEC_FREE || i == B_DEC_FREE + 1 || i == B_Y_STAGED || i == B_MK1A_FULL)
+                i == B_DEC_FREE || i == B_DEC_FREE + 1 || i == B_Y_STAGED || i == B_MK1A_FULL ||
+                i == B_XCONV)
                 count = NMASK;
             if (i == B_DEC_FULL || i == B_DEC_FULL + 1) count = 32;
             mbar_init(bar(i), count);
@@ -392,17 +422,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 mbar_expect_tx(bar(B_X_FULL), box);
                 tma_load_4d(sX, &tm_x, bar(B_X_FULL), 0, (int)h, (int)t0, (int)b);
             };
+            // rows of the state map: hi blocks at b * nc + c, lo blocks
+            // batch * nc further on
+            const int hi_row = (int)(b * nc + c), lo_row = (int)(p.batch * nc + b * nc + c);
             auto load_h = [&](int64_t h) {
-                mbar_expect_tx(bar(B_H_FULL), T::H_BYTES);
+                mbar_expect_tx(bar(B_H_FULL), (NST / 64 + (hl ? 1 : 0)) * T::H_SLOT);
                 for (int kb = 0; kb < NST / 64; ++kb)
-                    tma_load_4d(sH + kb * (PD * 128), &tm_h, bar(B_H_FULL), kb * 64, 0, (int)h,
-                                (int)(b * nc + c));
+                    tma_load_4d(sH + kb * T::H_SLOT, &tm_h, bar(B_H_FULL), kb * 64, 0, (int)h, hi_row);
+                if (hl)
+                    tma_load_4d(sH + (NST / 64) * T::H_SLOT, &tm_h, bar(B_H_FULL), 0, 0, (int)h, lo_row);
             };
             auto prefetch_head = [&](int64_t h) {
                 tma_prefetch_l2_4d(&tm_x, 0, (int)h, (int)t0, (int)b);
                 if (gated) tma_prefetch_l2_4d(&tm_z, 0, (int)h, (int)t0, (int)b);
-                for (int kb = 0; kb < NST / 64; ++kb)
-                    tma_prefetch_l2_4d(&tm_h, kb * 64, 0, (int)h, (int)(b * nc + c));
+                for (int kb = 0; kb < NST / 64; ++kb) {
+                    tma_prefetch_l2_4d(&tm_h, kb * 64, 0, (int)h, hi_row);
+                    if (hl) tma_prefetch_l2_4d(&tm_h, kb * 64, 0, (int)h, lo_row);
+                }
             };
             tma_prefetch_map(&tm_c);
             tma_prefetch_map(&tm_b);
@@ -457,13 +493,25 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     if (i > 0) ok = wait_bar(bar(B_ACC_EMPTY + t), (i - 1) & 1, abort);
                     if (!ok) break;
                     fence_after_sync();
-                    issue_state<NST>(tmem + st_col(t), t == 0 ? dC0 : dC1, dH);
-                    if (t == ntiles - 1) mma_commit(bar(B_H_FREE));
+                    issue_state<NST>(tmem + st_col(t), t == 0 ? dC0 : dC1, dH, hl);
+                    if (t == ntiles - 1) {
+                        if (!late_lo) {
+                            mma_commit(bar(B_H_FREE));
+                        } else {
+                            // lo block 1 into hi block 0's slot once every
+                            // tile's MMAs have read it
+                            mma_commit(bar(B_H0_FREE));
+                            ok = wait_bar(bar(B_H0_FREE), ph, abort);
+                            if (!ok) break;
+                            mbar_expect_tx(bar(B_H1_FULL), T::H_SLOT);
+                            tma_load_4d(sH, &tm_h, bar(B_H1_FULL), 64, 0, (int)(hfirst + i), lo_row);
+                        }
+                    }
                     SCAN_TRACE(9 + 8 * i + 3 * t);
                     // intra-chunk term of tile t, once its mask (and the head's x) is in
                     ok = wait_bar(bar(B_MK_FULL + t), ph, abort);
                     SCAN_TRACE(10 + 8 * i + 3 * t);
-                    if (ok && t == 0) ok = wait_bar(bar(B_X_FULL), ph, abort);
+                    if (ok && t == 0) ok = wait_bar(bar(B_XCONV), ph, abort);  // x in fp16
                     if (!ok) break;
                     fence_after_sync();
                     if (t == 0) {
@@ -477,9 +525,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         fence_after_sync();
                         issue_intra<0, 8, false>(tmem + in_col(1), dM1, dX);
                     }
-                    mma_commit(bar(B_ACC_FULL + t));
+                    if (!late_lo) mma_commit(bar(B_ACC_FULL + t));
                     mma_commit(bar(B_MK_EMPTY + t));
                     SCAN_TRACE(11 + 8 * i + 3 * t);
+                }
+                if (ok && late_lo) {
+                    // lo block 1 of every tile; the workers drain both tiles'
+                    // accumulators together, so they wait for no tile longer
+                    ok = wait_bar(bar(B_H1_FULL), ph, abort);
+                    if (!ok) break;
+                    for (int t = 0; t < ntiles; ++t)
+                        issue_state_kb(tmem + st_col(t), t == 0 ? dC0 : dC1, dH, 1, 0, true);
+                    for (int t = 0; t < ntiles; ++t) mma_commit(bar(B_ACC_FULL + t));
+                    mma_commit(bar(B_H_FREE));
                 }
                 if (!ok) break;
                 mma_commit(bar(B_X_FREE));
@@ -520,8 +578,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 dec[lane + 32 * k] = cv[k] * 1.4426950408889634f;
                 dec[QMAX + lane + 32 * k] = dv[k];
             }
-            if (lane == 0) dec[2 * QMAX] = p.D ? p.D[h] : 0.0f;
-            mbar_arrive(bar(B_DEC_FULL + bsel));
+            // the chunk's largest dt, for the masks' fp16 row scales
+            float dm = 0.0f;
+#pragma unroll
+            for (int k = 0; k < QMAX / 32; ++k) dm = fmaxf(dm, dv[k]);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) dm = fmaxf(dm, __shfl_xor_sync(0xffffffffu, dm, o));
+            if (lane == 0) {
+                dec[2 * QMAX] = p.D ? p.D[h] : 0.0f;
+                dec[2 * QMAX + 1] = dm;
+            }
+            // the test hook: the first head of chunk `withhold` never gets its
+            // decays, so the workers' bounded waits run out
+            if (i > 0 || c != withhold) mbar_arrive(bar(B_DEC_FULL + bsel));
         }
         if (!ok) *abort = 1;
     } else if (warp == STORE_WARP) {
@@ -705,18 +774,65 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             return true;
         };
 
-        // This warp's x rows of the resident x tile -> TMEM, for the diagonal
-        // term of the head's epilogue (x is overwritten by the next head once
-        // the last tile's MMA is done, which waits for this warp's mask).
-        auto stash_x = [&]() {
-            for (int t = 0; t < ntiles; ++t) {
+        // This warp's x entries of the resident x tile (its rows, 16 p
+        // columns): the bf16 values -> TMEM, for the diagonal term of the
+        // head's epilogue; then the tile in place as the fp16 operand of the
+        // intra MMAs, x 2^es with one power of two per head that takes the
+        // tile's largest |x| to [2^13, 2^14) (bf16 values are exact in fp16
+        // there; only entries below 2^-27 of that largest lose bits).
+        // Returns 2^-es.  x is overwritten by the next head once the last
+        // tile's MMA is done, which waits for this warp's mask.
+        // Every worker reaches the named barrier once per head (with `live`
+        // false it only takes part in it), so a warp whose wait failed cannot
+        // leave the others waiting there.  The partial maxima alternate
+        // between two buffers by head, so a warp that runs ahead cannot
+        // overwrite one that another warp has still to read.
+        auto stash_convert_x = [&](bool live, int par) -> float {
+            uint32_t* xmax_s = reinterpret_cast<uint32_t*>(smem + T::XMAX_OFF) + par * NWORK;
+            uint32_t w[2][8] = {};
+            uint32_t m2 = 0u;
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+                if (live && t < ntiles) {
+                    const int l = block_row(t, qd) + lane;
+                    const uint4 v0 = ld_shared_v4(sX + sw128(l, 2 * hf));
+                    const uint4 v1 = ld_shared_v4(sX + sw128(l, 2 * hf + 1));
+                    w[t][0] = v0.x; w[t][1] = v0.y; w[t][2] = v0.z; w[t][3] = v0.w;
+                    w[t][4] = v1.x; w[t][5] = v1.y; w[t][6] = v1.z; w[t][7] = v1.w;
+                    tmem_st8(tmem + lanes + stash_col(t, hf), w[t]);
+                    // max |x| as bf16 bit patterns (sign cleared; non-negative
+                    // floats order as their bits), both halves at once
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) m2 = __vmaxu2(m2, w[t][k] & 0x7FFF7FFFu);
+                }
+            }
+            uint32_t am = max(m2 & 0xFFFFu, m2 >> 16);
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) am = max(am, __shfl_xor_sync(0xffffffffu, am, o));
+            if (lane == 0) xmax_s[warp] = am;
+            named_sync(3, NMASK);
+#pragma unroll
+            for (int k = 0; k < NWORK; ++k) am = max(am, xmax_s[k]);
+            // bf16 bits -> exponent (the inputs are finite)
+            const int ex = am ? static_cast<int>((am >> 7) & 255) - 127 : 0;
+            const int es = min(100, max(-100, 13 - ex));
+            const float sc = __int_as_float((127 + es) << 23);
+            const float2 sc2 = make_float2(sc, sc);
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+                if (!live || t >= ntiles) continue;
                 const int l = block_row(t, qd) + lane;
-                const uint4 v0 = ld_shared_v4(sX + sw128(l, 2 * hf));
-                const uint4 v1 = ld_shared_v4(sX + sw128(l, 2 * hf + 1));
-                const uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-                tmem_st8(tmem + lanes + stash_col(t, hf), w);
+                uint32_t o[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const float2 f = __fmul2_rn(__bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[t][k])), sc2);
+                    o[k] = pack_f16x2(f.x, f.y);
+                }
+                st_shared_v4(sX + sw128(l, 2 * hf), o[0], o[1], o[2], o[3]);
+                st_shared_v4(sX + sw128(l, 2 * hf + 1), o[4], o[5], o[6], o[7]);
             }
             tmem_wait_st();
+            return __int_as_float((127 - es) << 23);
         };
 
         // Iteration i builds head i's tile-0 mask, drains head i-1's
@@ -731,7 +847,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const float* dec = reinterpret_cast<const float*>(smem + T::DEC_OFF) + bsel * T::DEC_FLOATS;
             float cl_cur[2] = {0.0f, 0.0f};
             float2 fw_cur[2] = {make_float2(1.0f, 0.0f), make_float2(1.0f, 0.0f)};
-            float Dh = 0.0f;
+            float Dh = 0.0f, dmax = 0.0f;
             if (mask_now && ok) {
                 ok = wait_bar(bar(B_DEC_FULL + bsel), (i >> 1) & 1, abort);
                 if (warp == 0 && lane == 0) SCAN_TRACE(82 + 5 * i);
@@ -739,13 +855,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     cl_cur[0] = dec[block_row(0, qd) + lane];
                     cl_cur[1] = dec[block_row(1, qd) + lane];
                     Dh = dec[2 * QMAX];
+                    dmax = dec[2 * QMAX + 1];
                 }
             }
             if (mask_now && ok) {
                 if (i > 0) ok = wait_bar(bar(B_MK_EMPTY), (i - 1) & 1, abort);
                 if (warp == 0 && lane == 0) SCAN_TRACE(83 + 5 * i);
                 if (ok) {
-                    const RowPlan r0 = plan_rows<0>(tmem, dec, dec + QMAX, rinv0, cbd0, Dh, qd, lane, Lc);
+                    const RowPlan r0 =
+                        plan_rows<0>(tmem, dec, dec + QMAX, rinv0, cbd0, Dh, dmax, qd, lane, Lc);
                     mask_group(r0, hf, sM0, dec, dec + QMAX, ctab, lane, i == 0);
                     fw_cur[0] = make_float2(r0.f, r0.w);
                     fence_smem_async();
@@ -769,17 +887,23 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             RowPlan r1;
             if (mask_now && ok && ntiles == 2) {
                 // tile 1, K columns 128-255 (clear of the y staging area)
-                r1 = plan_rows<1>(tmem, dec, dec + QMAX, rinv1, cbd1, Dh, qd, lane, Lc);
+                r1 = plan_rows<1>(tmem, dec, dec + QMAX, rinv1, cbd1, Dh, dmax, qd, lane, Lc);
                 mask_group(r1, hf + 4, sM1, dec, dec + QMAX, ctab, lane, i == 0);
                 fw_cur[1] = make_float2(r1.f, r1.w);
                 fence_smem_async();
                 mbar_arrive(bar(B_MK_FULL + 1));
                 if (warp == 0 && lane == 0 && i < 16) SCAN_TRACE(240 + i);
             }
-            if (mask_now && ok) {
-                ok = wait_bar(bar(B_X_FULL), i & 1, abort);
+            if (mask_now) {
+                if (ok) ok = wait_bar(bar(B_X_FULL), i & 1, abort);
                 if (warp == 0 && lane == 0) SCAN_TRACE(200 + 2 * i);
-                if (ok) stash_x();
+                const float ix = stash_convert_x(ok, i & 1);
+                if (ok) {
+                    fw_cur[0].x *= ix;
+                    fw_cur[1].x *= ix;
+                    fence_smem_async();
+                    mbar_arrive(bar(B_XCONV));
+                }
                 if (warp == 0 && lane == 0) SCAN_TRACE(201 + 2 * i);
                 if (ok && ntiles == 1) mbar_arrive(bar(B_MK_FULL));
             }
@@ -863,7 +987,8 @@ cudaError_t launch_n(const FwdParams& p, cudaStream_t s) {
     if (!make_tmap_bf16_4d(&tc_, p.C, NST, p.ngroups, p.seqlen, p.batch, 1, 32) ||
         !make_tmap_bf16_4d(&tb_, p.B, NST, p.ngroups, p.seqlen, p.batch, 1, rows) ||
         !make_tmap_bf16_4d(&tx_, p.x, PD, p.nheads, p.seqlen, p.batch, 1, rows) ||
-        !make_tmap_bf16_4d(&th_, p.states, NST, PD, p.nheads, p.batch * p.nchunks, PD, 1) ||
+        !make_tmap_bf16_4d(&th_, p.states_hl ? p.states_hl : p.states, NST, PD, p.nheads,
+                           (p.states_hl ? 2 : 1) * p.batch * p.nchunks, PD, 1) ||
         !make_tmap_bf16_4d(&ty_, p.y, PD, p.nheads, p.seqlen, p.batch, 1, rows) ||
         !make_tmap_bf16_4d(&tz_, p.z ? p.z : p.x, PD, p.nheads, p.seqlen, p.batch, 1, rows))
         return cudaErrorInvalidValue;
@@ -873,7 +998,8 @@ cudaError_t launch_n(const FwdParams& p, cudaStream_t s) {
     const int hb = heads_per_cta(p, sm_count());
     dim3 grid(static_cast<unsigned>(p.nchunks * p.ngroups * (p.heads_per_group / hb)),
               static_cast<unsigned>(p.batch));
-    return launch_kernel(kern, grid, dim3(NTHREADS), T::SMEM, s, p.pdl != 0, p, tc_, tb_, tx_, th_, ty_, tz_, hb);
+    return launch_kernel(kern, grid, dim3(NTHREADS), T::SMEM, s, p.pdl != 0, p, tc_, tb_, tx_, th_, ty_, tz_, hb,
+                         debug_withhold(SSD_DEBUG_SCAN_DECAYS));
 }
 
 }  // namespace

@@ -38,6 +38,9 @@ struct FwdParams {
     float* dt;      // [b, H, nc, Q]
     float* cumA;    // [b, H, nc, Q]
     void* states;   // [b, nc, H, P, N] in fp32 or the input dtype (states_f32): local states, then states entering each chunk
+    // [2][b, nc, H, P, N] bf16, or null: the states entering each chunk as hi
+    // and lo halves (hi + lo = the fp32 state), for the tensor-core chunk_scan
+    void* states_hl;
     int* status;    // device status word (SSD_ERR_TIMEOUT on a timed-out wait); may be null
 };
 

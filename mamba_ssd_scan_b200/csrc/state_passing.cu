@@ -7,11 +7,14 @@
 //
 // Sequential over chunks, parallel over batch x heads x headdim x dstate: each
 // thread carries one 16-byte vector of state elements (4 fp32 or 8 bf16) in
-// fp32 registers.  In place over `states` (stored in the input dtype): slot c
-// receives H_{c-1}, the state that enters chunk c; the final state H_{nc-1}
-// goes to final_state in fp32.  The loads of the next chunks' S do not depend
-// on the carry, so UNROLL chunks are loaded before their multiply-adds to keep
-// enough bytes in flight.
+// fp32 registers.  Slot c receives H_{c-1}, the state that enters chunk c,
+// either in place over `states` (in the dtype the states are kept in) or, for
+// the tensor-core chunk_scan, as a pair of bf16 arrays in states_hl: hi =
+// bf16(H) and lo = bf16(H - hi), so that hi + lo carries H to about 2^-17 of
+// its size through a bf16 operand.  The final state H_{nc-1} goes to
+// final_state in fp32.  The loads of the next chunks' S do not depend on the
+// carry, so UNROLL chunks are loaded before their multiply-adds to keep enough
+// bytes in flight.
 #include "internal.cuh"
 
 namespace ssd {
@@ -53,6 +56,16 @@ template <> struct Pack<__nv_bfloat16> {
     }
 };
 
+// E / 2 packed bf16 pairs (8 or 16 bytes) to global memory
+template <int W>
+__device__ __forceinline__ void store_half(__nv_bfloat16* dst, const uint32_t (&w)[W]) {
+    if constexpr (W == 2) {
+        *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
+    } else {
+        *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(256) state_passing_kernel(FwdParams p) {
     grid_dep_wait();  // the local states and cumA come from the previous steps
@@ -79,6 +92,14 @@ __global__ void __launch_bounds__(256) state_passing_kernel(FwdParams p) {
     uint4* base = reinterpret_cast<uint4*>(p.states) + (b * nc * H + h) * vecs_per_head + off;
     const int64_t cstride = H * vecs_per_head;  // vectors between consecutive chunks
     const float* cs = p.cumA + (b * H + h) * nc * Q + (Q - 1);
+    // hi / lo outputs: the same element order as `states`, E bf16 per thread
+    __nv_bfloat16* hl_hi = nullptr;
+    __nv_bfloat16* hl_lo = nullptr;
+    if (p.states_hl) {
+        const int64_t elems = p.batch * nc * H * p.headdim * p.dstate;
+        hl_hi = static_cast<__nv_bfloat16*>(p.states_hl) + ((b * nc * H + h) * vecs_per_head + off) * E;
+        hl_lo = hl_hi + elems;
+    }
     for (int64_t c = 0; c < nc; c += UNROLL) {
         uint4 s[UNROLL];
         float a[UNROLL];
@@ -94,7 +115,22 @@ __global__ void __launch_bounds__(256) state_passing_kernel(FwdParams p) {
             if (c + u < nc) {
                 float sv[E];
                 Pack<T>::unpack(s[u], sv);
-                base[(c + u) * cstride] = Pack<T>::pack(carry);
+                if (hl_hi) {
+                    uint32_t hw[E / 2], lw[E / 2];
+#pragma unroll
+                    for (int k = 0; k < E / 2; ++k) {
+                        const __nv_bfloat162 hb = __floats2bfloat162_rn(carry[2 * k], carry[2 * k + 1]);
+                        const float2 hf = __bfloat1622float2(hb);
+                        const __nv_bfloat162 lb =
+                            __floats2bfloat162_rn(carry[2 * k] - hf.x, carry[2 * k + 1] - hf.y);
+                        hw[k] = *reinterpret_cast<const uint32_t*>(&hb);
+                        lw[k] = *reinterpret_cast<const uint32_t*>(&lb);
+                    }
+                    store_half(hl_hi + (c + u) * cstride * E, hw);
+                    store_half(hl_lo + (c + u) * cstride * E, lw);
+                } else {
+                    base[(c + u) * cstride] = Pack<T>::pack(carry);
+                }
 #pragma unroll
                 for (int k = 0; k < E; ++k) carry[k] = fmaf(a[u], carry[k], sv[k]);
             }

@@ -29,7 +29,8 @@ def test_header_declares_entry_points():
     names = declared_functions()
     for required in ("ssd_fwd", "ssd_fwd_workspace_size", "ssd_state_update",
                      "ssd_status_string", "ssd_chunk_cumsum", "ssd_chunk_state",
-                     "ssd_state_passing", "ssd_chunk_scan", "ssd_fwd_check_status"):
+                     "ssd_state_passing", "ssd_chunk_scan", "ssd_fwd_check_status",
+                     "ssd_state_passing_hilo", "ssd_chunk_scan_hilo"):
         assert required in names
 
 
@@ -43,23 +44,32 @@ def test_tensor_core_dispatch_query(lib):
     import torch
 
     import mamba_ssd_scan_b200 as m
-    # bf16 in the fused kernel's range: the whole forward in one tensor-core kernel
-    assert m.tensor_core_steps(4, 1024, 24, 64, 64, 1, 256) == {"chunk_state", "chunk_scan", "fused"}
-    assert m.tensor_core_steps(1, 65536, 80, 64, 128, 8, 256) == {"chunk_state", "chunk_scan", "fused"}
-    assert m.tensor_core_steps(1, 300, 4, 64, 128, 4, 128) == {"chunk_state", "chunk_scan", "fused"}
+    # bf16: chunk_state and chunk_scan on the tensor cores (fp32 chunk states,
+    # entering chunk_scan as hi / lo bf16 halves)
+    assert m.tensor_core_steps(4, 1024, 24, 64, 64, 1, 256) == {"chunk_state", "chunk_scan"}
+    assert m.tensor_core_steps(1, 65536, 80, 64, 128, 8, 256) == {"chunk_state", "chunk_scan"}
+    assert m.tensor_core_steps(1, 300, 4, 64, 128, 2, 128) == {"chunk_state", "chunk_scan"}
+    # one head per group: chunk_state's tile takes 128 / headdim heads of a group
+    assert m.tensor_core_steps(1, 300, 4, 64, 128, 4, 128) == {"chunk_scan"}
     assert m.tensor_core_steps(4, 1024, 24, 64, 64, 1, 256, torch.float32) == set()
     assert m.tensor_core_steps(4, 1024, 24, 64, 64, 1, 256, flags=m.SSD_FLAG_CUDA_CORES) == set()
-    # the split steps keep fp32 chunk states: chunk_state on the tensor cores, the
-    # state term of chunk_scan in fp32 on the CUDA cores
     assert m.tensor_core_steps(4, 1024, 24, 64, 64, 1, 256, flags=m.SSD_FLAG_SPLIT_STEPS) == {
-        "chunk_state"}
-    # the opt-in bf16-states mode takes the tensor-core chunk_scan
+        "chunk_state", "chunk_scan"}
+    # the opt-in bf16-states mode also takes the tensor-core chunk_scan
     assert m.tensor_core_steps(4, 1024, 24, 64, 64, 1, 256, flags=m.SSD_FLAG_BF16_STATES) == {
         "chunk_state", "chunk_scan"}
+    # chunk_scan's tensor-core kernel takes headdim 64 and dstate 64 / 128 only
     assert m.tensor_core_steps(1, 512, 2, 128, 256, 1, 256) == {"chunk_state"}
-    # the fused kernel tiles the sequence its own way: any chunk
-    assert m.tensor_core_steps(1, 512, 4, 64, 128, 4, 64) == {"chunk_state", "chunk_scan", "fused"}
-    assert m.tensor_core_steps(1, 512, 4, 64, 128, 4, 64, flags=m.SSD_FLAG_SPLIT_STEPS) == set()
+    # chunk 64: neither tensor-core step kernel
+    assert m.tensor_core_steps(1, 512, 4, 64, 128, 4, 64) == set()
+    # the single-pass kernel (opt-in) tiles the sequence its own way: any chunk
+    sp = m.SSD_FLAG_SINGLE_PASS
+    assert m.tensor_core_steps(1, 512, 4, 64, 128, 4, 64, flags=sp) == {
+        "chunk_state", "chunk_scan", "fused"}
+    assert m.tensor_core_steps(4, 1024, 24, 64, 64, 1, 256, flags=sp) == {
+        "chunk_state", "chunk_scan", "fused"}
+    assert m.tensor_core_steps(1, 512, 4, 64, 128, 4, 64, flags=sp | m.SSD_FLAG_SPLIT_STEPS) == set()
+    assert m.tensor_core_steps(1, 512, 2, 128, 256, 1, 256, flags=sp) == {"chunk_state"}
 
 
 def test_status_strings(lib):
@@ -81,15 +91,21 @@ def _args(**kw):
 
 def test_workspace_size_is_host_only(lib):
     import mamba_ssd_scan_b200 as m
-    # fused kernel: header (256 B), the ring's reader counts (2*1*4 ints, in 256 B)
-    # and a two-slot ring of 1*4 states of 64*64 fp32
-    assert lib.ssd_fwd_workspace_size(ctypes.byref(_args())) == 256 + 256 + 2 * 4 * 64 * 64 * 4
-    # split steps: header + dt + cumA (1*4*2*256 fp32 each) + fp32 chunk states 1*2*4*64*64
+    # default (three kernels): header + dt + cumA (1*4*2*256 fp32 each) + fp32
+    # chunk states 1*2*4*64*64 + their hi / lo bf16 halves
+    assert lib.ssd_fwd_workspace_size(ctypes.byref(_args())) == 256 + 8192 + 8192 + 131072 + 131072
     a = _args(flags=m.SSD_FLAG_SPLIT_STEPS)
+    assert lib.ssd_fwd_workspace_size(ctypes.byref(a)) == 256 + 8192 + 8192 + 131072 + 131072
+    # the CUDA cores form the state term from the fp32 states: no halves
+    a = _args(flags=m.SSD_FLAG_SPLIT_STEPS | m.SSD_FLAG_CUDA_CORES)
     assert lib.ssd_fwd_workspace_size(ctypes.byref(a)) == 256 + 8192 + 8192 + 131072
-    # bf16-states mode: the chunk states in bf16
+    # bf16-states mode: the chunk states in bf16, no halves
     a = _args(flags=m.SSD_FLAG_BF16_STATES)
     assert lib.ssd_fwd_workspace_size(ctypes.byref(a)) == 256 + 8192 + 8192 + 65536
+    # single pass: header (256 B), the ring's reader counts (2*1*4 ints, in
+    # 256 B) and a two-slot ring of 1*4 states of 64*64 fp32
+    a = _args(flags=m.SSD_FLAG_SINGLE_PASS)
+    assert lib.ssd_fwd_workspace_size(ctypes.byref(a)) == 256 + 256 + 2 * 4 * 64 * 64 * 4
     assert lib.ssd_fwd_workspace_size(None) == 0
     assert lib.ssd_fwd_workspace_size(ctypes.byref(_args(nheads=3, ngroups=2))) == 0
 

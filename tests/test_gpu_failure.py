@@ -5,9 +5,12 @@ The library's test hook (ssd_debug_set_withhold, read by the host launcher)
 makes one producer withhold one hand-off:
   - the convolution's producer warp its first tile: the consumers' waits on
     that tile's mbarrier give up after their iteration limit;
-  - the fused forward the state leaving its first run of tiles (512 tokens):
-    the CTA of the second run that waits for it polls the carry ring until its
-    limit (about a second), raises the abort word, and every CTA stops.
+  - the forward's tensor-core chunk_scan the decays of the first head of its
+    second chunk: that CTA's workers give up their wait and the CTA stops;
+  - the single-pass forward (SSD_FLAG_SINGLE_PASS) the state leaving its first
+    run of tiles (512 tokens): the CTA of the second run that waits for it
+    polls the carry ring until its limit (about a second), raises the abort
+    word, and every CTA stops.
 The status call must then report SSD_ERR_TIMEOUT, and the same process runs
 the operation again with the hook off and checks it against the oracle.  Each
 case runs in a child process with a time limit."""
@@ -45,32 +48,37 @@ assert_close(y, yo, torch.float32, "after the timeout")
 print("TIMEOUT-OK")
 """
 
-# bf16, two chunks per sequence, two sequences: the fused path
+# bf16, four chunks per sequence, two sequences.  MODE: "workspace" or
+# "no_alloc" (the scratch inside the library) for the default three-kernel
+# path; "single_pass" for the one-kernel forward.
 FWD = r"""
 b, L, H, P, N, G, Q = 2, 1024, 4, 64, 64, 1, 256
 inp = synthetic.make_fwd_inputs(b, L, H, P, N, G, torch.bfloat16, seed=11, init_state=True)
 d = {k: (v.cuda() if v is not None else None) for k, v in inp.items()}
-assert "fused" in ssd.tensor_core_steps(b, L, H, P, N, G, Q, torch.bfloat16)
 NO_ALLOC = MODE == "no_alloc"
+FLAGS = ssd.SSD_FLAG_SINGLE_PASS if MODE == "single_pass" else 0
+HOOK = ssd.SSD_DEBUG_FWD_CARRY if MODE == "single_pass" else ssd.SSD_DEBUG_SCAN_DECAYS
+steps = ssd.tensor_core_steps(b, L, H, P, N, G, Q, torch.bfloat16, flags=FLAGS)
+assert ("fused" in steps) == (MODE == "single_pass") and "chunk_scan" in steps, steps
 
 def run():
     if NO_ALLOC:
         y = torch.empty_like(d["x"])
         ssd.ssd_fwd_no_alloc(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["dt_bias"], Q,
-                             d["init_state"], y=y)
-        return y, ssd.ssd_fwd_no_alloc_check_status(d["x"], d["B"], Q)
-    ws = torch.empty(ssd.ssd_fwd_workspace_size(b, L, H, P, N, G, Q, torch.bfloat16),
+                             d["init_state"], y=y, flags=FLAGS)
+        return y, ssd.ssd_fwd_no_alloc_check_status(d["x"], d["B"], Q, flags=FLAGS)
+    ws = torch.empty(ssd.ssd_fwd_workspace_size(b, L, H, P, N, G, Q, torch.bfloat16, flags=FLAGS),
                      dtype=torch.uint8, device="cuda")
     y = ssd.ssd_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["dt_bias"], Q,
-                    d["init_state"], workspace=ws)
-    return y, ssd.ssd_fwd_check_status(d["x"], d["B"], Q, ws)
+                    d["init_state"], workspace=ws, flags=FLAGS)
+    return y, ssd.ssd_fwd_check_status(d["x"], d["B"], Q, ws, flags=FLAGS)
 
 y, st = run()
 assert st == 0, f"clean run: status {st}"
-ssd.ssd_debug_set_withhold(ssd.SSD_DEBUG_FWD_CARRY, 0)
+ssd.ssd_debug_set_withhold(HOOK, 0 if MODE == "single_pass" else 1)
 y, st = run()
 assert st == 4, f"expected SSD_ERR_TIMEOUT (4), got {st}"
-ssd.ssd_debug_set_withhold(ssd.SSD_DEBUG_FWD_CARRY, -1)
+ssd.ssd_debug_set_withhold(HOOK, -1)
 y, st = run()
 assert st == 0, f"after the timeout: status {st}"
 yo, _ = oracle.load().ssd_fwd(**inp)
@@ -90,9 +98,13 @@ def test_withheld_tile_times_out_and_context_survives():
     _child(CONV)
 
 
-def test_withheld_carry_times_out_and_context_survives():
+def test_withheld_decays_time_out_and_context_survives():
     _child(FWD, "workspace")
 
 
 def test_no_alloc_reports_the_timeout():
     _child(FWD, "no_alloc")
+
+
+def test_single_pass_withheld_carry_times_out_and_context_survives():
+    _child(FWD, "single_pass")

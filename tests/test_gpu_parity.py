@@ -128,6 +128,41 @@ def test_steps_against_chunked_oracle(orc, dtype, Q):
     assert_close(y, ref["y"], dtype, "y")
 
 
+@pytest.mark.parametrize("N,Q", [(64, 256), (128, 256), (128, 128)])
+def test_hilo_steps_against_chunked_oracle(orc, N, Q):
+    """Steps 3 and 4 as the bf16 forward runs them on the tensor cores: the
+    entering states as hi / lo bf16 halves (hi + lo against the oracle's
+    entering states, hi alone being bf16(H)), then y from them."""
+    b, L, H, P, G = 2, 700, 4, 64, 2
+    inp = synthetic.make_fwd_inputs(b, L, H, P, N, G, torch.bfloat16, seed=23 + N + Q,
+                                    init_state=True)
+    ref = orc.ssd_chunked(**inp, chunk=Q)
+    d = dev(inp)
+    assert "chunk_scan" in ssd.tensor_core_steps(b, L, H, P, N, G, Q, torch.bfloat16)
+    dt_sp, cumA = ssd.ssd_chunk_cumsum(d["x"], d["dt"], d["A"], d["B"], d["C"], d["dt_bias"], Q)
+    states = ssd.ssd_chunk_state(d["x"], d["dt"], d["A"], d["B"], d["C"], dt_sp, cumA, Q)
+    before = states.clone()
+    # the fp32 entering states from the in-place step 3, for the exact check
+    h32 = states.clone()
+    ssd.ssd_state_passing(d["x"], d["dt"], d["A"], d["B"], d["C"], cumA, h32, Q,
+                          init_state=d["init_state"])
+    fin = torch.empty((b, H, P, N), dtype=torch.float32, device=DEV)
+    hl = ssd.ssd_state_passing_hilo(d["x"], d["dt"], d["A"], d["B"], d["C"], cumA, states, Q,
+                                    init_state=d["init_state"], final_state=fin)
+    torch.cuda.synchronize()
+    assert torch.equal(states, before), "the local states are read, not written"
+    hi, lo = hl[0].float(), hl[1].float()
+    # hi = bf16(H) and lo = bf16(H - hi), H the same fp32 carry (H - hi is exact)
+    assert torch.equal(hi, h32.bfloat16().float())
+    assert torch.equal(lo, (h32 - hi).bfloat16().float())
+    assert_close(hi + lo, ref["Hin"], torch.bfloat16, "hi + lo vs entering states")
+    assert_close(fin, ref["final_state"], torch.bfloat16, "final state")
+    y = ssd.ssd_chunk_scan_hilo(d["x"], d["dt"], d["A"], d["B"], d["C"], dt_sp, cumA, hl,
+                                d["D"], Q)
+    torch.cuda.synchronize()
+    assert_close(y, ref["y"], torch.bfloat16, "y from the hi / lo states")
+
+
 # ---------------------------------------------------------------------------
 # the named workloads at full size
 # each small workload at its own seed and two more (the inputs' recipe
@@ -145,33 +180,39 @@ def test_workload_fwd_f32_small(orc, shift):
     assert_close(fin, fo, cfg.dtype, "final")
 
 
-# Five seeds of the b4 L1024 workload, every element against the bf16 bound.
-# At seed+1000 the state term e^{cumA} C . H_in cancels strongly at a chunk's
+# Five seeds of the b4 L1024 workload, every element against the bf16 bound,
+# on the default three-kernel path and on the single-pass kernel.  At
+# seed+1000 the state term e^{cumA} C . H_in cancels strongly at a chunk's
 # first tokens (state entries up to ~67): the carried state must stay fp32 and
 # enter the tensor cores as bf16 hi + lo, and the intra-chunk mask needs more
-# than bf16's 8 bits, which the fused forward keeps.
+# than bf16's 8 bits (both paths keep it in fp16: a bf16 mask reached 1.03 of
+# the bound there).
 HEADLINE_SEED_CASES = [0, 1000, 2000, 3000, 4000]
+PATHS = {"three_kernels": 0, "single_pass": ssd.SSD_FLAG_SINGLE_PASS}
 
 
+@pytest.mark.parametrize("path", list(PATHS))
 @pytest.mark.parametrize("shift", HEADLINE_SEED_CASES, ids=lambda v: f"seed+{v}")
-def test_workload_fwd_bf16_b4_L1024(orc, shift):
+def test_workload_fwd_bf16_b4_L1024(orc, shift, path):
     cfg = synthetic.FWD_CONFIGS["fwd_bf16_b4_L1024"]
     inp = synthetic.make_config_inputs(cfg, 1234 + synthetic.SEED_OFFSET[cfg.name] + shift)
-    y, fin = run_fwd(inp, cfg.chunk)
+    y, fin = run_fwd(inp, cfg.chunk, flags=PATHS[path])
     yo, fo = orc.ssd_fwd(**inp)
     assert_close(y, yo, cfg.dtype, "y")
     assert_close(fin, fo, cfg.dtype, "final")
 
 
-@pytest.mark.parametrize("shift", [0, 1000, 2000], ids=lambda v: f"seed+{v}")
+@pytest.mark.parametrize("shift,path", [(0, "three_kernels"), (1000, "three_kernels"),
+                                        (2000, "three_kernels"), (0, "single_pass")],
+                         ids=lambda v: f"seed+{v}" if isinstance(v, int) else v)
 @pytest.mark.parametrize("name,heads,batches", [
     ("fwd_bf16_b8_L4096_init", [0, 13, 31], [0, 7]),
     ("fwd_bf16_b1_L65536_G8", [0, 9, 10, 47, 79], None),
 ])
-def test_workload_sampled_heads(orc, name, heads, batches, shift):
+def test_workload_sampled_heads(orc, name, heads, batches, shift, path):
     cfg = synthetic.FWD_CONFIGS[name]
     inp = synthetic.make_config_inputs(cfg, 1234 + synthetic.SEED_OFFSET[cfg.name] + shift)
-    y, fin = run_fwd(inp, cfg.chunk)
+    y, fin = run_fwd(inp, cfg.chunk, flags=PATHS[path])
     yo, fo = oracle_heads(orc, inp, heads, batches)
     bsel = slice(None) if batches is None else batches
     print(name, "y", report(y.cpu()[bsel][:, :, heads], yo))
@@ -258,20 +299,20 @@ TC_CASES = [
 
 @pytest.mark.parametrize("case", TC_CASES, ids=lambda c: "b{}_L{}_H{}_P{}_N{}_G{}_Q{}".format(*c))
 def test_tensor_core_path(orc, case):
-    """The default bf16 path (the fused kernel where the shape allows), the
-    split steps with fp32 chunk states, and the CUDA cores, each against the
-    oracle."""
+    """The default bf16 path (three tensor-core kernels where the shape allows,
+    fp32 chunk states), the single-pass kernel, and the CUDA cores, each
+    against the oracle."""
     b, L, H, P, N, G, Q = case
     inp = synthetic.make_fwd_inputs(b, L, H, P, N, G, torch.bfloat16, seed=L + N,
                                     init_state=True)
     y_tc, f_tc = run_fwd(inp, Q)
-    y_sp, f_sp = run_fwd(inp, Q, flags=ssd.SSD_FLAG_SPLIT_STEPS)
+    y_1p, f_1p = run_fwd(inp, Q, flags=ssd.SSD_FLAG_SINGLE_PASS)
     y_cc, f_cc = run_fwd(inp, Q, flags=ssd.SSD_FLAG_CUDA_CORES)
     yo, fo = orc.ssd_fwd(**inp)
     assert_close(y_tc, yo, torch.bfloat16, "default y")
     assert_close(f_tc, fo, torch.bfloat16, "default final")
-    assert_close(y_sp, yo, torch.bfloat16, "split-step y")
-    assert_close(f_sp, fo, torch.bfloat16, "split-step final")
+    assert_close(y_1p, yo, torch.bfloat16, "single-pass y")
+    assert_close(f_1p, fo, torch.bfloat16, "single-pass final")
     assert_close(y_cc, yo, torch.bfloat16, "CUDA-core y")
     assert_close(f_cc, fo, torch.bfloat16, "CUDA-core final")
 
@@ -299,6 +340,7 @@ GATE_CASES = [
     (2, 600, 4, 64, 64, 2, 256, torch.bfloat16, 0),        # tensor cores, ragged tail
     (1, 1024, 8, 64, 128, 1, 256, torch.bfloat16, 0),      # tensor cores, dstate 128
     (2, 600, 4, 64, 64, 2, 256, torch.bfloat16, ssd.SSD_FLAG_CUDA_CORES),
+    (1, 1024, 8, 64, 128, 1, 256, torch.bfloat16, ssd.SSD_FLAG_SINGLE_PASS),
 ]
 
 
