@@ -18,18 +18,20 @@
 // hand work to each other through mbarriers:
 //
 //   warps 0-15 "workers": per head and tile, read CB back, apply the causal
-//              decay mask below the diagonal and write Mk as a bf16 K-major
-//              operand to shared memory (one buffer per tile, refilled as soon
-//              as its MMA is done); then drain the previous head's accumulators
-//              for the same tile (y = f * intra + exp(cumA) * state, plus the
-//              diagonal term (C_l . B_l dt_l + D) x_l in fp32, bf16 staged
-//              for the storer).  The
-//              four warps of a TMEM lane quarter share its 32 rows and take
-//              one column group in four (and a quarter of the p columns in
-//              the epilogue);
+//              decay mask (with the diagonal and the D skip folded in) and
+//              write Mk as an fp16 operand: tile 0's (K = 128) into TMEM, the A
+//              operand of its MMA, tile 1's (K = 256) K-major into shared
+//              memory, each refilled as soon as its MMA is done; convert the
+//              head's x tile in place to fp16; then drain the previous head's
+//              accumulators (y = f * intra + exp(cumA) * state, bf16 staged
+//              for the storer).  The four warps of a TMEM lane quarter share
+//              its 32 rows and take one column group in four (and a quarter
+//              of the p columns in the epilogue);
 //   warp 16    "control": one lane issues every TMA load (C, B once; x and
 //              H_in per head) and every MMA (CB once; per head and tile the
-//              state term C_t H_in^T and Mk x);
+//              state term C_t H_in^T, bf16, and Mk x, fp16).  H_in comes as
+//              the bf16 halves hi + lo of the fp32 state (both resident: 2 x
+//              NST / 64 blocks of 8 KB), each against the same C;
 //   warp 17    "loader": stages each head's decays and D in shared memory
 //              (two buffers), so the mask phase never waits on a global load;
 //   warp 18    "storer": the workers stage each head's y tile in shared memory
@@ -49,7 +51,7 @@
 // by one lane, so each mask element costs one multiply.  M is the midpoint of
 // the block's cumA range, so neither factor exceeds 2^(span / 2), span the
 // block's log2 decay; blocks whose span exceeds kFastSpan (where such factors
-// would leave fp32 or bf16 range) use M = cumA_lb and one exp2 per diagonal
+// would leave fp32 range) use M = cumA_lb and one exp2 per diagonal
 // element instead, which is exact for any decay.  Every wait is bounded; a
 // timed-out role raises a shared abort flag that the others observe, and the
 // CTA still frees its TMEM.
@@ -57,7 +59,7 @@
 // TMEM columns: [0,64) tile 0's CB and [128,256) tile 1's CB as packed fp16
 // pairs (the fp32 CB sits in [0,128) and [256,512) until packed; the two tiles
 // are packed at the same time, so their source and destination columns never
-// overlap); [64,128) the workers' stash of the head's x rows (diagonal term);
+// overlap); [64,128) tile 0's mask (fp16 pairs, written once CB is packed);
 // [256,320)/[320,384) tile 0's state/intra accumulators, [384,448)/[448,512)
 // tile 1's.
 #include <stdlib.h>
@@ -77,7 +79,7 @@ constexpr int NWORK = 16;                        // worker warps
 constexpr int CTRL_WARP = NWORK, LOAD_WARP = NWORK + 1, STORE_WARP = NWORK + 2;
 constexpr int NTHREADS = (NWORK + 3) * 32;
 constexpr int NMASK = NWORK * 32;
-constexpr uint32_t CB0P = 0, CB1P = 128, CB1F = 256;
+constexpr uint32_t CB0P = 0, MK0T = 64, CB1P = 128, CB1F = 256;
 // largest log2 decay span of a 32-row block that takes the factored path:
 // factors stay within 2^90, so masked entries (|CB| scaled below 2^15) and
 // their 256-term sums stay far inside fp32 and bf16 range
@@ -85,8 +87,6 @@ constexpr float kFastSpan = 180.0f;
 constexpr float kMaxExp = 96.0f;
 __device__ __forceinline__ uint32_t st_col(int t) { return t == 0 ? 256u : 384u; }
 __device__ __forceinline__ uint32_t in_col(int t) { return t == 0 ? 320u : 448u; }
-// TMEM columns of worker hf's stash of tile t's x rows (16 bf16 per lane)
-__device__ __forceinline__ uint32_t stash_col(int t, int hf) { return 64u + 32u * t + 8u * hf; }
 // first chunk row of the 32-row block that TMEM lane quarter qd holds in tile t
 __device__ __forceinline__ int block_row(int t, int qd) { return t == 0 ? 32 * (3 - qd) : 128 + 32 * qd; }
 
@@ -98,23 +98,19 @@ struct ScanTile {
     static constexpr int B_OFF = C_OFF + C_BYTES;            // B, later tile 1's mask
     static constexpr int MK1_BYTES = 4 * 128 * 128;
     static constexpr int B_BYTES = C_BYTES > MK1_BYTES ? C_BYTES : MK1_BYTES;
-    static constexpr int MK0_OFF = B_OFF + B_BYTES;          // tile 0's mask
-    static constexpr int MK0_BYTES = 2 * 128 * 128;
-    static constexpr int X_OFF = MK0_OFF + MK0_BYTES;
+    static constexpr int X_OFF = B_OFF + B_BYTES;
     static constexpr int X_BYTES = QMAX * 128;
     // the entering state, in 64-wide K blocks of PD rows (8 KB): the hi
-    // blocks, then one slot for lo block 0 (with NST = 128, lo block 1 reuses
-    // hi block 0's slot once the MMAs that read it are done)
+    // blocks, then the lo blocks
     static constexpr int H_OFF = X_OFF + X_BYTES;
     static constexpr int H_SLOT = PD * 128;
-    static constexpr int H_BYTES = (NST / 64 + 1) * H_SLOT;
+    static constexpr int H_BYTES = 2 * (NST / 64) * H_SLOT;
     // per-head decays, two buffers filled by the loader warp:
     // [log2e * cumA (QMAX) | dt (QMAX) | D, max dt, padding (4)] fp32
     static constexpr int DEC_FLOATS = 2 * QMAX + 4;
     static constexpr int DEC_OFF = H_OFF + H_BYTES;
     static constexpr int RINV_OFF = DEC_OFF + 2 * DEC_FLOATS * 4;  // per-row CB scale, 2 tiles
-    static constexpr int CBD_OFF = RINV_OFF + 2 * 128 * 4;   // per-row C_l . B_l, 2 tiles
-    static constexpr int NORM_OFF = CBD_OFF + 2 * 128 * 4;   // |C_r|^2 per row, max |B_j|^2 partials
+    static constexpr int NORM_OFF = RINV_OFF + 2 * 128 * 4;  // |C_r|^2 per row, max |B_j|^2 partials
     static constexpr int CTAB_OFF = NORM_OFF + (256 + 8) * 4;  // per worker warp: 32 column factors
     static constexpr int XMAX_OFF = CTAB_OFF + NWORK * 32 * 4;  // [2][worker warp]: max |x| bits
     static constexpr int BAR_OFF = XMAX_OFF + 2 * NWORK * 4;
@@ -143,7 +139,7 @@ enum : int {
     B_CB_LOAD = 0, B_CB_DONE, B_CB_PACKED, B_X_FULL, B_H_FULL, B_H_FREE, B_X_FREE,
     B_MK_FULL, B_MK_EMPTY = B_MK_FULL + 2, B_ACC_FULL = B_MK_EMPTY + 2,
     B_ACC_EMPTY = B_ACC_FULL + 2, B_DEC_FULL = B_ACC_EMPTY + 2, B_DEC_FREE = B_DEC_FULL + 2,
-    B_Y_STAGED = B_DEC_FREE + 2, B_Y_READ, B_MK1A_FULL, B_H0_FREE, B_H1_FULL, B_XCONV, B_COUNT
+    B_Y_STAGED = B_DEC_FREE + 2, B_Y_READ, B_MK1A_FULL, B_XCONV, B_COUNT
 };
 
 // Bounded wait that also gives up when another role has aborted: a few
@@ -177,45 +173,39 @@ __device__ __forceinline__ void store_group_packed(uint32_t mbase, uint32_t row,
         st_shared_v4(dst + sw128(row, c0 + i), o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
 }
 
-// 32 masked values of one row -> fp16, into the K-major SW128 operand
-__device__ __forceinline__ void store_group(uint32_t mbase, uint32_t row, int j0, const float (&v)[32]) {
-    const uint32_t dst = mbase + (j0 >> 6) * (128 * 128);
-    const int c0 = (j0 & 63) >> 3;
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-        st_shared_v4(dst + sw128(row, c0 + i), pack_f16x2(v[8 * i + 0], v[8 * i + 1]),
-                     pack_f16x2(v[8 * i + 2], v[8 * i + 3]), pack_f16x2(v[8 * i + 4], v[8 * i + 5]),
-                     pack_f16x2(v[8 * i + 6], v[8 * i + 7]));
-}
-
-__device__ __forceinline__ void store_zero_group(uint32_t mbase, uint32_t row, int j0) {
-    const uint32_t dst = mbase + (j0 >> 6) * (128 * 128);
-    const int c0 = (j0 & 63) >> 3;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) st_shared_v4(dst + sw128(row, c0 + i), 0u, 0u, 0u, 0u);
+// One packed group of mask values to its operand: tile 0's in TMEM (16
+// columns of this warp's lanes at mk_t), tile 1's in shared memory.
+__device__ __forceinline__ void put_group(bool to_tmem, uint32_t mk_t, uint32_t mbase, uint32_t row, int j0,
+                                          const uint32_t (&o)[16]) {
+    if (to_tmem)
+        tmem_st16(mk_t, o);
+    else
+        store_group_packed(mbase, row, j0, o);
 }
 
 // Mask warp for tile TT: rows block_row(TT, qd) + lane (TMEM lane 32 qd + lane),
 // column groups hf + 4 k (k <= TT) of 32 columns.  Groups above the diagonal
 // block are zeros; they are written for the first head only (nothing else
-// writes there).  cum2 holds log2(e) * cumA, so every decay is one exp2.  The
-// diagonal entry (j = l, decay 1) is left out of the operand: the epilogue
-// adds (C_l . B_l dt_l + D) x_l in fp32, so the term that is often the row's
-// largest, and the D skip, are not rounded.  cbd is the row's C_l . B_l
-// (fp32, saved when CB was packed).
+// writes there).  cum2 holds log2(e) * cumA, so every decay is one exp2.
 //
 // The operand is fp16 (2^-11 relative rounding, against bf16's 2^-8), so each
 // row carries a power-of-two scale rs_l into fp16's range: row l holds
-// m[l,j] = CBp[l,j] k_j rs_l, CBp the packed CB (|CBp| < 2^14) and k_j =
-// 2^{ref - c_j} dt_j (fast) or 2^{c_l - c_j} dt_j (steep).  For j < l, c_j >=
-// c_l, so |m[l,j]| <= 2^14 2^{ref - c_l} dmax rs_l (2^0 for 2^{ref - c_l} when
-// steep), dmax the chunk's largest dt; rs_l brings that bound to 2^15, below
-// fp16's 65504, so nothing overflows and the row's largest entries keep every
-// bit.  The epilogue factor f_l undoes rs_l.
+// m[l,j] = CBp[l,j] k_j rs_l for j < l, CBp the packed CB (CB = rinv_l CBp,
+// |CBp| < 2^14) and k_j = 2^{ref - c_j} dt_j (fast) or 2^{c_l - c_j} dt_j
+// (steep), and on the diagonal m[l,l] = (CBp[l,l] dt_l + D / rinv_l) e_l rs_l
+// with e_l = 2^{ref - c_l} (fast) or 1 (steep), so that the epilogue factor
+// f_l = rinv_l / (e_l rs_l) gives the diagonal term (C_l . B_l dt_l + D) x_l
+// and the D skip with the rest of the row.  For j <= l, c_j >= c_l, so
+// |m[l,j]| <= (2^14 dmax + |D| / rinv_l) e_l rs_l, dmax the chunk's largest
+// dt; rs_l brings that bound to 2^15, below fp16's 65504, so nothing
+// overflows and the row's largest entries keep every bit.
 struct RowPlan {
     float ref, cl, c_first;
-    float f, w;      // the row's epilogue factor and diagonal weight
+    float f;         // the row's epilogue factor
     float rs;        // the row's power-of-two scale into fp16 range
+    float dtl;       // dt_l
+    float dadd;      // D / rinv_l * rs_l: the skip term in the mask's units
+    float de;        // e_l: the diagonal's decay factor
     bool fast;       // factored decays (warp-uniform)
     int rb;          // 32-row block index of the rows
     uint32_t row;    // TMEM lane = Mk row
@@ -224,8 +214,7 @@ struct RowPlan {
 
 template <int TT>
 __device__ __forceinline__ RowPlan plan_rows(uint32_t tmem, const float* cum2, const float* dtv,
-                                             float rinv, float cbd, float Dh, float dmax, int qd,
-                                             int lane, int Lc) {
+                                             float rinv, float Dh, float dmax, int qd, int lane, int Lc) {
     RowPlan r;
     const int lb = block_row(TT, qd);
     r.rb = lb >> 5;
@@ -238,21 +227,30 @@ __device__ __forceinline__ RowPlan plan_rows(uint32_t tmem, const float* cum2, c
     r.fast = (r.c_first - c_last) <= kFastSpan;
     r.ref = r.fast ? 0.5f * (r.c_first + c_last) : r.c_first;
     r.cl = cum2[lb + lane];
-    const float lg = (r.fast ? r.ref - r.cl : 0.0f) + __log2f(fmaxf(16384.0f * dmax, 1e-30f));
+    const float irinv = __int_as_float(254 * (1 << 23) - __float_as_int(rinv));  // 1 / rinv (a power of 2)
+    const float lg = (r.fast ? r.ref - r.cl : 0.0f) +
+                     __log2f(fmaxf(16384.0f * dmax + fabsf(Dh) * irinv, 1e-30f));
     const int e = min(120, max(-120, 15 - static_cast<int>(ceilf(fminf(fmaxf(lg, -200.0f), 200.0f)))));
     r.rs = __int_as_float((127 + e) << 23);
     const float irs = __int_as_float((127 - e) << 23);
     r.f = (r.fast ? rinv * ex2(r.cl - r.ref) : rinv) * irs;
-    r.w = fmaf(cbd, dtv[lb + lane], Dh);
+    r.dtl = dtv[lb + lane];
+    r.dadd = Dh * irinv * r.rs;
+    r.de = r.fast ? ex2(r.ref - r.cl) : 1.0f;
     return r;
 }
 
-// One 32-column group g of the plan's rows.
-__device__ __forceinline__ void mask_group(const RowPlan& r, int g, uint32_t mbase, const float* cum2,
-                                           const float* dtv, float* ctab, int lane, bool first) {
+// One 32-column group g of the plan's rows, to TMEM (mk_t: the group's 16
+// columns at this warp's lanes) or to the shared operand at mbase.
+__device__ __forceinline__ void mask_group(const RowPlan& r, int g, bool to_tmem, uint32_t mk_t, uint32_t mbase,
+                                           const float* cum2, const float* dtv, float* ctab, int lane,
+                                           bool first) {
     const int j0 = 32 * g;
     if (g > r.rb) {  // above the diagonal block: zeros, kept from the first head
-        if (first) store_zero_group(mbase, r.row, j0);
+        if (first) {
+            const uint32_t z[16] = {};
+            put_group(to_tmem, mk_t, mbase, r.row, j0, z);
+        }
         return;
     }
     uint32_t raw[16];
@@ -276,7 +274,7 @@ __device__ __forceinline__ void mask_group(const RowPlan& r, int g, uint32_t mba
             o[2 * i] = pack_f16x2(m0.x, m0.y);
             o[2 * i + 1] = pack_f16x2(m1.x, m1.y);
         }
-        store_group_packed(mbase, r.row, j0, o);
+        put_group(to_tmem, mk_t, mbase, r.row, j0, o);
         return;
     }
     float v[32];
@@ -296,7 +294,7 @@ __device__ __forceinline__ void mask_group(const RowPlan& r, int g, uint32_t mba
             v[4 * i + 2] *= rr * c.z;
             v[4 * i + 3] *= rr * c.w;
         }
-    } else if (r.fast) {  // the diagonal block, factored; j = l left to the epilogue
+    } else if (r.fast) {  // the diagonal block, factored; j = l carries dt_l and D
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const float4 c = ct[i];
@@ -304,17 +302,23 @@ __device__ __forceinline__ void mask_group(const RowPlan& r, int g, uint32_t mba
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int q = 4 * i + e;
-                v[q] = (q < lane) ? v[q] * cc[e] : 0.0f;
+                float m = v[q] * cc[e];
+                if (q == lane) m = fmaf(v[q], r.dtl, r.dadd) * r.de;
+                v[q] = (q <= lane) ? m : 0.0f;
             }
         }
     } else {  // the diagonal block of a steep block: one exp2 per element
 #pragma unroll
         for (int q = 0; q < 32; ++q) {
-            const float e = ex2(fminf(r.cl - cum2[j0 + q], 0.0f)) * dtv[j0 + q];
-            v[q] = (q < lane) ? v[q] * e : 0.0f;
+            float m = v[q] * ex2(fminf(r.cl - cum2[j0 + q], 0.0f)) * dtv[j0 + q];
+            if (q == lane) m = fmaf(v[q], r.dtl, r.dadd) * r.de;
+            v[q] = (q <= lane) ? m : 0.0f;
         }
     }
-    store_group(mbase, r.row, j0, v);
+    uint32_t o[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) o[i] = pack_f16x2(v[2 * i], v[2 * i + 1]);
+    put_group(to_tmem, mk_t, mbase, r.row, j0, o);
 }
 
 // Per-head MMAs, issued by the control thread.  Descriptors are built once;
@@ -330,15 +334,25 @@ __device__ __forceinline__ void issue_state_kb(uint32_t d_tmem, uint64_t dA, uin
         mma_bf16(d_tmem, dA + oa, dB + ob, idesc_bf16(128, PD, false, false), (acc || k > 0) ? 1u : 0u);
     }
 }
-// The state term's K blocks that are resident when the head starts: every hi
-// block, then lo block 0 (when the state comes as a hi / lo pair).
+// The whole state term of one tile: every hi block, then (when the state
+// comes as a hi / lo pair) every lo block against the same C blocks.
 template <int NST>
 __device__ __forceinline__ void issue_state(uint32_t d_tmem, uint64_t dA, uint64_t dB, bool hl) {
 #pragma unroll
     for (int kb = 0; kb < NST / 64; ++kb) issue_state_kb(d_tmem, dA, dB, kb, kb, kb > 0);
-    if (hl) issue_state_kb(d_tmem, dA, dB, 0, NST / 64, true);
+    if (hl)
+#pragma unroll
+        for (int kb = 0; kb < NST / 64; ++kb) issue_state_kb(d_tmem, dA, dB, kb, NST / 64 + kb, true);
 }
-// Intra-chunk term of one tile: Mk_t (K-major) x x (MN-major), both fp16, K
+// Intra-chunk term of tile 0: its mask in TMEM (128 lanes x 64 columns of fp16
+// pairs) x x (MN-major), K = 128 in steps of 16 (8 columns of A each).
+__device__ __forceinline__ void issue_intra_t0(uint32_t d_tmem, uint32_t a_tmem, uint64_t dB) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+        mma_ts(d_tmem, a_tmem + 8 * k, dB + ((k * 2048) >> 4), idesc_f16(128, PD, false, true),
+               k > 0 ? 1u : 0u);
+}
+// Intra-chunk term of tile 1: Mk_1 (K-major) x x (MN-major), both fp16, K
 // steps [K0, K1) of 16; FRESH: the first of them overwrites the accumulator.
 template <int K0, int K1, bool FRESH>
 __device__ __forceinline__ void issue_intra(uint32_t d_tmem, uint64_t dA, uint64_t dB) {
@@ -378,12 +392,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const int ntiles = (Lc + 127) / 128;
     constexpr bool gated = GATED;  // y *= silu(z): a separate instantiation
     const uint32_t sC = smem_u32(smem + T::C_OFF), sB = smem_u32(smem + T::B_OFF);
-    const uint32_t sM0 = smem_u32(smem + T::MK0_OFF), sM1 = sB;
+    const uint32_t sM1 = sB;
     const uint32_t sX = smem_u32(smem + T::X_OFF), sH = smem_u32(smem + T::H_OFF);
-    // hi / lo state operand (else the bf16 states alone); with NST = 128 the
-    // second lo block is loaded while the head's MMAs run
+    // hi / lo state operand (else the bf16 states alone)
     const bool hl = p.states_hl != nullptr;
-    const bool late_lo = hl && NST == 128;
     // y of one head is staged in tile 1's mask buffer, in its K columns
     // 0-127 (rewritten for every head, never a zero group), between the MMA
     // that read that buffer and the next mask, and leaves by TMA
@@ -426,11 +438,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             // batch * nc further on
             const int hi_row = (int)(b * nc + c), lo_row = (int)(p.batch * nc + b * nc + c);
             auto load_h = [&](int64_t h) {
-                mbar_expect_tx(bar(B_H_FULL), (NST / 64 + (hl ? 1 : 0)) * T::H_SLOT);
-                for (int kb = 0; kb < NST / 64; ++kb)
+                mbar_expect_tx(bar(B_H_FULL), (hl ? 2 : 1) * (NST / 64) * T::H_SLOT);
+                for (int kb = 0; kb < NST / 64; ++kb) {
                     tma_load_4d(sH + kb * T::H_SLOT, &tm_h, bar(B_H_FULL), kb * 64, 0, (int)h, hi_row);
-                if (hl)
-                    tma_load_4d(sH + (NST / 64) * T::H_SLOT, &tm_h, bar(B_H_FULL), 0, 0, (int)h, lo_row);
+                    if (hl)
+                        tma_load_4d(sH + (NST / 64 + kb) * T::H_SLOT, &tm_h, bar(B_H_FULL), kb * 64, 0,
+                                    (int)h, lo_row);
+                }
             };
             auto prefetch_head = [&](int64_t h) {
                 tma_prefetch_l2_4d(&tm_x, 0, (int)h, (int)t0, (int)b);
@@ -482,7 +496,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             const uint64_t dC0 = desc_sw128(sC, 16, 1024), dC1 = desc_sw128(sC + 128 * 128, 16, 1024);
             const uint64_t dH = desc_sw128(sH, 16, 1024), dX = desc_sw128(sX, QMAX * 128, 1024);
-            const uint64_t dM0 = desc_sw128(sM0, 16, 1024), dM1 = desc_sw128(sM1, 16, 1024);
+            const uint64_t dM1 = desc_sw128(sM1, 16, 1024);
             for (int i = 0; ok && i < hb_size; ++i) {
                 const uint32_t ph = i & 1;
                 if (i + 1 < hb_size) prefetch_head(hfirst + i + 1);  // next head's x, H_in into L2
@@ -494,28 +508,17 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     if (!ok) break;
                     fence_after_sync();
                     issue_state<NST>(tmem + st_col(t), t == 0 ? dC0 : dC1, dH, hl);
-                    if (t == ntiles - 1) {
-                        if (!late_lo) {
-                            mma_commit(bar(B_H_FREE));
-                        } else {
-                            // lo block 1 into hi block 0's slot once every
-                            // tile's MMAs have read it
-                            mma_commit(bar(B_H0_FREE));
-                            ok = wait_bar(bar(B_H0_FREE), ph, abort);
-                            if (!ok) break;
-                            mbar_expect_tx(bar(B_H1_FULL), T::H_SLOT);
-                            tma_load_4d(sH, &tm_h, bar(B_H1_FULL), 64, 0, (int)(hfirst + i), lo_row);
-                        }
-                    }
+                    if (t == ntiles - 1) mma_commit(bar(B_H_FREE));
                     SCAN_TRACE(9 + 8 * i + 3 * t);
                     // intra-chunk term of tile t, once its mask (and the head's x) is in
                     ok = wait_bar(bar(B_MK_FULL + t), ph, abort);
                     SCAN_TRACE(10 + 8 * i + 3 * t);
                     if (ok && t == 0) ok = wait_bar(bar(B_XCONV), ph, abort);  // x in fp16
+                    if (t == 0) SCAN_TRACE(192 + i);
                     if (!ok) break;
                     fence_after_sync();
                     if (t == 0) {
-                        issue_intra<0, 8, true>(tmem + in_col(0), dM0, dX);
+                        issue_intra_t0(tmem + in_col(0), tmem + MK0T, dX);
                     } else {
                         // tile 1's mask arrives in two halves: K columns
                         // 128-255 first, then 0-127
@@ -525,19 +528,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         fence_after_sync();
                         issue_intra<0, 8, false>(tmem + in_col(1), dM1, dX);
                     }
-                    if (!late_lo) mma_commit(bar(B_ACC_FULL + t));
+                    mma_commit(bar(B_ACC_FULL + t));
                     mma_commit(bar(B_MK_EMPTY + t));
                     SCAN_TRACE(11 + 8 * i + 3 * t);
-                }
-                if (ok && late_lo) {
-                    // lo block 1 of every tile; the workers drain both tiles'
-                    // accumulators together, so they wait for no tile longer
-                    ok = wait_bar(bar(B_H1_FULL), ph, abort);
-                    if (!ok) break;
-                    for (int t = 0; t < ntiles; ++t)
-                        issue_state_kb(tmem + st_col(t), t == 0 ? dC0 : dC1, dH, 1, 0, true);
-                    for (int t = 0; t < ntiles; ++t) mma_commit(bar(B_ACC_FULL + t));
-                    mma_commit(bar(B_H_FREE));
                 }
                 if (!ok) break;
                 mma_commit(bar(B_X_FREE));
@@ -612,7 +605,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // ------------------------------ workers ------------------------------
         const int qd = warp & 3, hf = warp >> 2;
         float* rinv_s = reinterpret_cast<float*>(smem + T::RINV_OFF);
-        float* cbd_s = reinterpret_cast<float*>(smem + T::CBD_OFF);
         float* ctab = reinterpret_cast<float*>(smem + T::CTAB_OFF) + warp * 32;
         const uint32_t lanes = static_cast<uint32_t>(32 * qd) << 16;
         // CB is repacked as fp16 pairs with a power-of-two scale per row,
@@ -672,19 +664,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (ok) {
             fence_after_sync();
             if (ntiles == 2) {
-                const int rb1 = block_row(1, qd) >> 5;
 #pragma unroll
                 for (int k = 0; k < 2; ++k) {
                     const int kk = hf + 4 * k;
                     float v[32];
                     uint32_t r1[16];
                     tmem_ld32(tmem + lanes + CB1F + 32 * kk, v);
-                    if (kk == rb1) {
-                        float dg = 0.0f;
-#pragma unroll
-                        for (int q = 0; q < 32; ++q) dg = (q == lane) ? v[q] : dg;
-                        cbd_s[128 + 32 * qd + lane] = dg;
-                    }
 #pragma unroll
                     for (int q = 0; q < 16; ++q) r1[q] = pack_f16x2(v[2 * q] * sc_t[1], v[2 * q + 1] * sc_t[1]);
                     tmem_st16(tmem + lanes + CB1P + 16 * kk, r1);
@@ -692,12 +677,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             float v[32];
             tmem_ld32(tmem + lanes + 32 * hf, v);
-            if (hf == (block_row(0, qd) >> 5)) {
-                float dg = 0.0f;
-#pragma unroll
-                for (int q = 0; q < 32; ++q) dg = (q == lane) ? v[q] : dg;
-                cbd_s[32 * qd + lane] = dg;
-            }
 #pragma unroll
             for (int q = 0; q < 16; ++q) r0[q] = pack_f16x2(v[2 * q] * sc_t[0], v[2 * q + 1] * sc_t[0]);
         }
@@ -715,21 +694,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         fence_after_sync();
         const float rinv0 = ok ? rinv_s[32 * qd + lane] : 1.0f;
         const float rinv1 = (ok && ntiles == 2) ? rinv_s[128 + 32 * qd + lane] : 1.0f;
-        const float cbd0 = ok ? cbd_s[32 * qd + lane] : 0.0f;
-        const float cbd1 = (ok && ntiles == 2) ? cbd_s[128 + 32 * qd + lane] : 0.0f;
 
         // The epilogue of head i, tile t, for this warp's rows and 16 p
-        // columns: y = f * intra + 2^cl * state + w x_l, w the diagonal weight
-        // (C_l . B_l dt_l + D).  x_l was stashed in TMEM while the head's x
-        // tile was resident, so the worker loop never waits on a global load.
-        auto epilogue = [&](int i, int t, float cl2, float2 fw) -> bool {
+        // columns: y = f * intra + 2^cl * state (the intra term carries the
+        // diagonal and the D skip), so the worker loop never waits on a global
+        // load.
+        auto epilogue = [&](int i, int t, float cl2, float fr) -> bool {
             const int l = block_row(t, qd) + lane;
             if (!wait_bar(bar(B_ACC_FULL + t), i & 1, abort)) return false;
             if (warp == 0 && lane == 0) SCAN_TRACE(140 + 4 * i + 2 * t);
             fence_after_sync();
             const uint32_t a[2] = {tmem + lanes + in_col(t) + 16 * hf, tmem + lanes + st_col(t) + 16 * hf};
-            uint32_t r[2][16], xw[8];
-            tmem_ld8(tmem + lanes + stash_col(t, hf), xw);
+            uint32_t r[2][16];
             tmem_ld16x2(a, r);
             fence_before_sync();
             mbar_arrive(bar(B_ACC_EMPTY + t));
@@ -746,19 +722,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     zw[4] = z1.x; zw[5] = z1.y; zw[6] = z1.z; zw[7] = z1.w;
                 }
                 const float s = ex2(cl2);
-                const float2 f2 = make_float2(fw.x, fw.x), s2 = make_float2(s, s);
-                const float2 w2 = make_float2(fw.y, fw.y);
+                const float2 f2 = make_float2(fr, fr), s2 = make_float2(s, s);
 #pragma unroll
                 for (int k4 = 0; k4 < 2; ++k4) {
                     uint32_t o[4];
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
                         const int e = 8 * k4 + 2 * k;
-                        const float2 xf =
-                            __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&xw[4 * k4 + k]));
                         const float2 vi = make_float2(__uint_as_float(r[0][e]), __uint_as_float(r[0][e + 1]));
                         const float2 vs = make_float2(__uint_as_float(r[1][e]), __uint_as_float(r[1][e + 1]));
-                        float2 yv = __ffma2_rn(w2, xf, __ffma2_rn(s2, vs, __fmul2_rn(f2, vi)));
+                        float2 yv = __ffma2_rn(s2, vs, __fmul2_rn(f2, vi));
                         if constexpr (gated) {
                             const float2 zf =
                                 __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&zw[4 * k4 + k]));
@@ -775,19 +748,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         };
 
         // This warp's x entries of the resident x tile (its rows, 16 p
-        // columns): the bf16 values -> TMEM, for the diagonal term of the
-        // head's epilogue; then the tile in place as the fp16 operand of the
-        // intra MMAs, x 2^es with one power of two per head that takes the
-        // tile's largest |x| to [2^13, 2^14) (bf16 values are exact in fp16
-        // there; only entries below 2^-27 of that largest lose bits).
-        // Returns 2^-es.  x is overwritten by the next head once the last
-        // tile's MMA is done, which waits for this warp's mask.
+        // columns), in place as the fp16 operand of the intra MMAs: x 2^es
+        // with one power of two per head that takes the tile's largest |x| to
+        // [2^13, 2^14) (bf16 values are exact in fp16 there; only entries
+        // below 2^-27 of that largest lose bits).  Returns 2^-es.  x is
+        // overwritten by the next head once the last tile's MMA is done, which
+        // waits for this warp's mask.
         // Every worker reaches the named barrier once per head (with `live`
         // false it only takes part in it), so a warp whose wait failed cannot
         // leave the others waiting there.  The partial maxima alternate
         // between two buffers by head, so a warp that runs ahead cannot
         // overwrite one that another warp has still to read.
-        auto stash_convert_x = [&](bool live, int par) -> float {
+        auto convert_x = [&](bool live, int par) -> float {
             uint32_t* xmax_s = reinterpret_cast<uint32_t*>(smem + T::XMAX_OFF) + par * NWORK;
             uint32_t w[2][8] = {};
             uint32_t m2 = 0u;
@@ -799,7 +771,6 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     const uint4 v1 = ld_shared_v4(sX + sw128(l, 2 * hf + 1));
                     w[t][0] = v0.x; w[t][1] = v0.y; w[t][2] = v0.z; w[t][3] = v0.w;
                     w[t][4] = v1.x; w[t][5] = v1.y; w[t][6] = v1.z; w[t][7] = v1.w;
-                    tmem_st8(tmem + lanes + stash_col(t, hf), w[t]);
                     // max |x| as bf16 bit patterns (sign cleared; non-negative
                     // floats order as their bits), both halves at once
 #pragma unroll
@@ -831,22 +802,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 st_shared_v4(sX + sw128(l, 2 * hf), o[0], o[1], o[2], o[3]);
                 st_shared_v4(sX + sw128(l, 2 * hf + 1), o[4], o[5], o[6], o[7]);
             }
-            tmem_wait_st();
             return __int_as_float((127 - es) << 23);
         };
 
-        // Iteration i builds head i's tile-0 mask, drains head i-1's
-        // accumulators, stashes head i's x rows and builds its tile-1 mask, so
+        // Iteration i builds head i's tile-0 mask (in TMEM), drains head i-1's
+        // accumulators, converts head i's x tile and builds its tile-1 mask, so
         // the tensor core works on one head while the CUDA cores finish the
         // previous one.
+        const uint32_t mk0 = tmem + lanes + MK0T + 16 * hf;  // this warp's tile-0 mask columns
         float cl_prev[2] = {0.0f, 0.0f};
-        float2 fw_prev[2] = {make_float2(1.0f, 0.0f), make_float2(1.0f, 0.0f)};
+        float f_prev[2] = {1.0f, 1.0f};
         for (int i = 0; i <= hb_size; ++i) {
             const bool mask_now = i < hb_size, epi_now = i > 0;
             const int bsel = i & 1;
             const float* dec = reinterpret_cast<const float*>(smem + T::DEC_OFF) + bsel * T::DEC_FLOATS;
             float cl_cur[2] = {0.0f, 0.0f};
-            float2 fw_cur[2] = {make_float2(1.0f, 0.0f), make_float2(1.0f, 0.0f)};
+            float f_cur[2] = {1.0f, 1.0f};
             float Dh = 0.0f, dmax = 0.0f;
             if (mask_now && ok) {
                 ok = wait_bar(bar(B_DEC_FULL + bsel), (i >> 1) & 1, abort);
@@ -862,13 +833,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (i > 0) ok = wait_bar(bar(B_MK_EMPTY), (i - 1) & 1, abort);
                 if (warp == 0 && lane == 0) SCAN_TRACE(83 + 5 * i);
                 if (ok) {
-                    const RowPlan r0 =
-                        plan_rows<0>(tmem, dec, dec + QMAX, rinv0, cbd0, Dh, dmax, qd, lane, Lc);
-                    mask_group(r0, hf, sM0, dec, dec + QMAX, ctab, lane, i == 0);
-                    fw_cur[0] = make_float2(r0.f, r0.w);
-                    fence_smem_async();
-                    // a single tile's mask is released only after the x stash
-                    if (ntiles == 2) mbar_arrive(bar(B_MK_FULL));
+                    const RowPlan r0 = plan_rows<0>(tmem, dec, dec + QMAX, rinv0, Dh, dmax, qd, lane, Lc);
+                    mask_group(r0, hf, true, mk0, 0u, dec, dec + QMAX, ctab, lane, i == 0);
+                    f_cur[0] = r0.f;
+                    tmem_wait_st();
+                    fence_before_sync();
+                    mbar_arrive(bar(B_MK_FULL));
                 }
                 if (warp == 0 && lane == 0) SCAN_TRACE(84 + 5 * i);
             }
@@ -878,7 +848,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 if (ntiles == 2) ok = wait_bar(bar(B_MK_EMPTY + 1), (i - 1) & 1, abort);
                 else if (i >= 2) ok = wait_bar(bar(B_Y_READ), (i - 2) & 1, abort);
                 for (int t = 0; t < ntiles; ++t)
-                    if (ok) ok = epilogue(i - 1, t, cl_prev[t], fw_prev[t]);
+                    if (ok) ok = epilogue(i - 1, t, cl_prev[t], f_prev[t]);
                 if (ok) {
                     fence_smem_async();
                     mbar_arrive(bar(B_Y_STAGED));
@@ -887,9 +857,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             RowPlan r1;
             if (mask_now && ok && ntiles == 2) {
                 // tile 1, K columns 128-255 (clear of the y staging area)
-                r1 = plan_rows<1>(tmem, dec, dec + QMAX, rinv1, cbd1, Dh, dmax, qd, lane, Lc);
-                mask_group(r1, hf + 4, sM1, dec, dec + QMAX, ctab, lane, i == 0);
-                fw_cur[1] = make_float2(r1.f, r1.w);
+                r1 = plan_rows<1>(tmem, dec, dec + QMAX, rinv1, Dh, dmax, qd, lane, Lc);
+                mask_group(r1, hf + 4, false, 0u, sM1, dec, dec + QMAX, ctab, lane, i == 0);
+                f_cur[1] = r1.f;
                 fence_smem_async();
                 mbar_arrive(bar(B_MK_FULL + 1));
                 if (warp == 0 && lane == 0 && i < 16) SCAN_TRACE(240 + i);
@@ -897,22 +867,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (mask_now) {
                 if (ok) ok = wait_bar(bar(B_X_FULL), i & 1, abort);
                 if (warp == 0 && lane == 0) SCAN_TRACE(200 + 2 * i);
-                const float ix = stash_convert_x(ok, i & 1);
+                const float ix = convert_x(ok, i & 1);
                 if (ok) {
-                    fw_cur[0].x *= ix;
-                    fw_cur[1].x *= ix;
+                    f_cur[0] *= ix;
+                    f_cur[1] *= ix;
                     fence_smem_async();
                     mbar_arrive(bar(B_XCONV));
                 }
                 if (warp == 0 && lane == 0) SCAN_TRACE(201 + 2 * i);
-                if (ok && ntiles == 1) mbar_arrive(bar(B_MK_FULL));
             }
             if (mask_now && ok && ntiles == 2) {
                 // tile 1, K columns 0-127, once the staged y has been stored
                 if (i > 0) ok = wait_bar(bar(B_Y_READ), (i - 1) & 1, abort);
                 if (warp == 0 && lane == 0) SCAN_TRACE(85 + 5 * i);
                 if (ok) {
-                    mask_group(r1, hf, sM1, dec, dec + QMAX, ctab, lane, i == 0);
+                    mask_group(r1, hf, false, 0u, sM1, dec, dec + QMAX, ctab, lane, i == 0);
                     fence_smem_async();
                     mbar_arrive(bar(B_MK1A_FULL));
                 }
@@ -921,8 +890,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (mask_now && ok) mbar_arrive(bar(B_DEC_FREE + bsel));  // this head's decays are used
             cl_prev[0] = cl_cur[0];
             cl_prev[1] = cl_cur[1];
-            fw_prev[0] = fw_cur[0];
-            fw_prev[1] = fw_cur[1];
+            f_prev[0] = f_cur[0];
+            f_prev[1] = f_cur[1];
         }
     }
     fence_before_sync();
