@@ -56,16 +56,6 @@ template <> struct Pack<__nv_bfloat16> {
     }
 };
 
-// E / 2 packed bf16 pairs (8 or 16 bytes) to global memory
-template <int W>
-__device__ __forceinline__ void store_half(__nv_bfloat16* dst, const uint32_t (&w)[W]) {
-    if constexpr (W == 2) {
-        *reinterpret_cast<uint2*>(dst) = make_uint2(w[0], w[1]);
-    } else {
-        *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-}
-
 template <typename T>
 __global__ void __launch_bounds__(256) state_passing_kernel(FwdParams p) {
     grid_dep_wait();  // the local states and cumA come from the previous steps
@@ -92,14 +82,6 @@ __global__ void __launch_bounds__(256) state_passing_kernel(FwdParams p) {
     uint4* base = reinterpret_cast<uint4*>(p.states) + (b * nc * H + h) * vecs_per_head + off;
     const int64_t cstride = H * vecs_per_head;  // vectors between consecutive chunks
     const float* cs = p.cumA + (b * H + h) * nc * Q + (Q - 1);
-    // hi / lo outputs: the same element order as `states`, E bf16 per thread
-    __nv_bfloat16* hl_hi = nullptr;
-    __nv_bfloat16* hl_lo = nullptr;
-    if (p.states_hl) {
-        const int64_t elems = p.batch * nc * H * p.headdim * p.dstate;
-        hl_hi = static_cast<__nv_bfloat16*>(p.states_hl) + ((b * nc * H + h) * vecs_per_head + off) * E;
-        hl_lo = hl_hi + elems;
-    }
     for (int64_t c = 0; c < nc; c += UNROLL) {
         uint4 s[UNROLL];
         float a[UNROLL];
@@ -115,22 +97,7 @@ __global__ void __launch_bounds__(256) state_passing_kernel(FwdParams p) {
             if (c + u < nc) {
                 float sv[E];
                 Pack<T>::unpack(s[u], sv);
-                if (hl_hi) {
-                    uint32_t hw[E / 2], lw[E / 2];
-#pragma unroll
-                    for (int k = 0; k < E / 2; ++k) {
-                        const __nv_bfloat162 hb = __floats2bfloat162_rn(carry[2 * k], carry[2 * k + 1]);
-                        const float2 hf = __bfloat1622float2(hb);
-                        const __nv_bfloat162 lb =
-                            __floats2bfloat162_rn(carry[2 * k] - hf.x, carry[2 * k + 1] - hf.y);
-                        hw[k] = *reinterpret_cast<const uint32_t*>(&hb);
-                        lw[k] = *reinterpret_cast<const uint32_t*>(&lb);
-                    }
-                    store_half(hl_hi + (c + u) * cstride * E, hw);
-                    store_half(hl_lo + (c + u) * cstride * E, lw);
-                } else {
-                    base[(c + u) * cstride] = Pack<T>::pack(carry);
-                }
+                base[(c + u) * cstride] = Pack<T>::pack(carry);
 #pragma unroll
                 for (int k = 0; k < E; ++k) carry[k] = fmaf(a[u], carry[k], sv[k]);
             }
@@ -144,10 +111,89 @@ __global__ void __launch_bounds__(256) state_passing_kernel(FwdParams p) {
     }
 }
 
+// The hi / lo form: fp32 local states in, each entering state out as two
+// bf16 arrays (hi = bf16(H), lo = bf16(H - hi); H - hi is exact in fp32).
+// Each thread carries 8 consecutive state elements: two 16-byte loads per
+// chunk, one 16-byte store of each half.
+constexpr int HL_UNROLL = 4;
+
+__device__ __forceinline__ void split_store(__nv_bfloat16* hi, __nv_bfloat16* lo, const float (&v)[8]) {
+    uint32_t hw[4], lw[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const __nv_bfloat162 hb = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
+        const float2 hf = __bfloat1622float2(hb);
+        const __nv_bfloat162 lb = __floats2bfloat162_rn(v[2 * k] - hf.x, v[2 * k + 1] - hf.y);
+        hw[k] = *reinterpret_cast<const uint32_t*>(&hb);
+        lw[k] = *reinterpret_cast<const uint32_t*>(&lb);
+    }
+    *reinterpret_cast<uint4*>(hi) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    *reinterpret_cast<uint4*>(lo) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+}
+
+__global__ void __launch_bounds__(256) state_passing_hl_kernel(FwdParams p) {
+    grid_dep_wait();  // the local states and cumA come from the previous steps
+    grid_dep_launch();
+    const int64_t H = p.nheads, nc = p.nchunks, Q = p.chunk;
+    const int64_t vecs_per_head = p.headdim * p.dstate / 8;
+    const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= p.batch * H * vecs_per_head) return;
+    const int64_t bh = e / vecs_per_head, off = e % vecs_per_head;
+    const int64_t b = bh / H, h = bh % H;
+    float carry[8];
+    if (p.init_state) {
+        const float4* ip = reinterpret_cast<const float4*>(p.init_state + e * 8);
+        const float4 v0 = ip[0], v1 = ip[1];
+        carry[0] = v0.x; carry[1] = v0.y; carry[2] = v0.z; carry[3] = v0.w;
+        carry[4] = v1.x; carry[5] = v1.y; carry[6] = v1.z; carry[7] = v1.w;
+    } else {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) carry[k] = 0.0f;
+    }
+    const int64_t first = ((b * nc * H + h) * vecs_per_head + off) * 8;  // element of chunk 0
+    const int64_t cstride = H * vecs_per_head * 8;                        // elements between chunks
+    const float* src = static_cast<const float*>(p.states) + first;
+    __nv_bfloat16* hi = static_cast<__nv_bfloat16*>(p.states_hl) + first;
+    __nv_bfloat16* lo = hi + p.batch * nc * H * p.headdim * p.dstate;
+    const float* cs = p.cumA + (b * H + h) * nc * Q + (Q - 1);
+    for (int64_t c = 0; c < nc; c += HL_UNROLL) {
+        float4 s0[HL_UNROLL], s1[HL_UNROLL];
+        float a[HL_UNROLL];
+#pragma unroll
+        for (int u = 0; u < HL_UNROLL; ++u) {
+            if (c + u < nc) {
+                const float4* sp = reinterpret_cast<const float4*>(src + (c + u) * cstride);
+                s0[u] = sp[0];
+                s1[u] = sp[1];
+                a[u] = expf(cs[(c + u) * Q]);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < HL_UNROLL; ++u) {
+            if (c + u < nc) {
+                split_store(hi + (c + u) * cstride, lo + (c + u) * cstride, carry);
+                const float sv[8] = {s0[u].x, s0[u].y, s0[u].z, s0[u].w, s1[u].x, s1[u].y, s1[u].z, s1[u].w};
+#pragma unroll
+                for (int k = 0; k < 8; ++k) carry[k] = fmaf(a[u], carry[k], sv[k]);
+            }
+        }
+    }
+    if (p.final_state) {
+        float4* fp = reinterpret_cast<float4*>(p.final_state + e * 8);
+        fp[0] = make_float4(carry[0], carry[1], carry[2], carry[3]);
+        fp[1] = make_float4(carry[4], carry[5], carry[6], carry[7]);
+    }
+}
+
 }  // namespace
 
 template <typename T>
 cudaError_t launch_state_passing(const FwdParams& p, cudaStream_t s) {
+    if (p.states_hl) {
+        const int64_t n = p.batch * p.nheads * p.headdim * p.dstate / 8;
+        return launch_kernel(state_passing_hl_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s,
+                             p.pdl != 0, p);
+    }
     const int64_t n = p.batch * p.nheads * p.headdim * p.dstate / Pack<T>::E;
     return launch_kernel(state_passing_kernel<T>, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s,
                          p.pdl != 0, p);
