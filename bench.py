@@ -51,6 +51,9 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=HEADLINE)
     ap.add_argument("--no-extra", action="store_true", help="skip the other workloads")
+    ap.add_argument("--single-pass", action="store_true",
+                    help="time the opt-in single-pass kernel (SSD_FLAG_SINGLE_PASS) instead of "
+                         "the default three-kernel forward")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--flush-mb", type=int, default=256)
     ap.add_argument("--e2e-steps", type=int, default=20,
@@ -275,13 +278,15 @@ def main_ours(args):
     y = torch.empty_like(d["x"])
     fin = (torch.empty((cfg.batch, cfg.nheads, cfg.headdim, cfg.dstate), device=dev)
            if cfg.return_final else None)
+    fwd_flags = ssd.SSD_FLAG_SINGLE_PASS if args.single_pass else 0
     ws = torch.empty(ssd.ssd_fwd_workspace_size(cfg.batch, cfg.seqlen, cfg.nheads, cfg.headdim,
                                                 cfg.dstate, cfg.ngroups, cfg.chunk,
-                                                cfg.dtype), dtype=torch.uint8, device=dev)
+                                                cfg.dtype, flags=fwd_flags),
+                     dtype=torch.uint8, device=dev)
 
     def step():
         ssd.ssd_fwd(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["dt_bias"], cfg.chunk,
-                    d["init_state"], y=y, final_state=fin, workspace=ws)
+                    d["init_state"], y=y, final_state=fin, workspace=ws, flags=fwd_flags)
 
     # ---- headline: K timed steps ----------------------------------------
     for _ in range(args.warmup):
@@ -307,7 +312,7 @@ def main_ours(args):
     tokens = cfg.tokens
     value = job_throughput(tokens, world, ms)
     tc = ssd.tensor_core_steps(cfg.batch, cfg.seqlen, cfg.nheads, cfg.headdim, cfg.dstate,
-                               cfg.ngroups, cfg.chunk, cfg.dtype)
+                               cfg.ngroups, cfg.chunk, cfg.dtype, flags=fwd_flags)
     cost = algorithmic_cost(cfg, elt)
     if "fused" in tc:
         # one kernel does the whole path: its bytes are the path's (inputs
@@ -363,7 +368,8 @@ def main_ours(args):
             stream.wait_event(ev_out[i])  # step k-2's y has been read back
         dd = dev_in[i]
         ssd.ssd_fwd(dd["x"], dd["dt"], dd["A"], dd["B"], dd["C"], dd["D"], dd["dt_bias"],
-                    cfg.chunk, dd["init_state"], y=y_dev[i], final_state=fin, workspace=ws)
+                    cfg.chunk, dd["init_state"], y=y_dev[i], final_state=fin, workspace=ws,
+                    flags=fwd_flags)
         ev_done[i].record(stream)
         with torch.cuda.stream(s_d2h):
             s_d2h.wait_event(ev_done[i])
@@ -418,7 +424,9 @@ def main_ours(args):
         "data": "synthetic",
         "config": {"workload": cfg.name, "batch": cfg.batch, "seqlen": cfg.seqlen,
                    "nheads": cfg.nheads, "headdim": cfg.headdim, "dstate": cfg.dstate,
-                   "ngroups": cfg.ngroups, "chunk": cfg.chunk, "global_batch":
+                   "ngroups": cfg.ngroups, "chunk": cfg.chunk,
+                   "kernels": "single pass" if "fused" in tc else "three kernels",
+                   "global_batch":
                    cfg.batch * world, "parallelism": f"dp{world}" if world > 1 else "single",
                    "l2": f"inputs {input_bytes(inp) / 1e6:.0f} MB; L2 flushed before every "
                          f"timed step ({args.flush_mb} MB write, then a read of it, so its "
