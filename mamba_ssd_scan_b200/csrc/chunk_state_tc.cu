@@ -66,7 +66,8 @@ template <int NST, int PD>
 __global__ void __launch_bounds__(NTHR, NST == 256 ? 2 : 3)  // CTAs per SM that fit
     chunk_state_tc_kernel(const __grid_constant__ FwdParams p,
                           const __grid_constant__ CUtensorMap tm_x,
-                          const __grid_constant__ CUtensorMap tm_b) {
+                          const __grid_constant__ CUtensorMap tm_b,
+                          const __grid_constant__ CUtensorMap tm_s, int tma_out) {
     using T = StateTile<NST, PD>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -143,22 +144,26 @@ __global__ void __launch_bounds__(NTHR, NST == 256 ? 2 : 3)  // CTAs per SM that
         // ----- scalers (warps 0-7): decay weights, x scaling, epilogue -----
         grid_dep_wait();  // dt and cumA are formed here (step 1 fused) or come from step 1
         if (p.fuse_cumsum) {
+            // step 1 here: warp hh forms head hh's dt and cumA, stores them
+            // for steps 3 and 4, and writes its decay weights into wtab
             if (warp < T::HPC) {
                 const int64_t off = ((b * H + h0 + warp) * nc + c) * Q;
-                chunk_cumsum_warp<__nv_bfloat16>(p, b, c, h0 + warp, p.dt + off, p.cumA + off, lane);
+                chunk_cumsum_warp<__nv_bfloat16>(p, b, c, h0 + warp, p.dt + off, p.cumA + off, lane,
+                                                 wtab + warp * QMAX);
             }
             if (blockIdx.x == 0 && blockIdx.y == 0 && tid == 0 && p.status) *p.status = 0;  // a new call
-            named_sync(1, NSCALE);
-        }
-        grid_dep_launch();
-        for (int i = tid; i < T::HPC * QMAX; i += NSCALE) {
-            const int hh = i / QMAX, l = i % QMAX;
-            float w = 0.0f;
-            if (l < Lc) {
-                const int64_t base = ((b * H + h0 + hh) * nc + c) * Q;
-                w = expf(p.cumA[base + Q - 1] - p.cumA[base + l]) * p.dt[base + l];
+            grid_dep_launch();
+        } else {
+            grid_dep_launch();
+            for (int i = tid; i < T::HPC * QMAX; i += NSCALE) {
+                const int hh = i / QMAX, l = i % QMAX;
+                float w = 0.0f;
+                if (l < Lc) {
+                    const int64_t base = ((b * H + h0 + hh) * nc + c) * Q;
+                    w = expf(p.cumA[base + Q - 1] - p.cumA[base + l]) * p.dt[base + l];
+                }
+                wtab[i] = w;
             }
-            wtab[i] = w;
         }
         named_sync(1, NSCALE);
         bool ok = true;
@@ -183,6 +188,9 @@ __global__ void __launch_bounds__(NTHR, NST == 256 ? 2 : 3)  // CTAs per SM that
         }
         if (ok) ok = wait_or_abort(bar(B_DONE), 0, abort);
         fence_after_sync();
+        // fp32 states with dstate <= 128: the 128 x NST tile is staged in the
+        // ring (free once every MMA is done) in 32-column SW128 boxes and
+        // leaves by TMA stores, instead of 16-byte stores from every thread
         if (ok) {
             // warp w reads TMEM lanes 32*(w%4).. (rows m), warpgroup w/4 half the columns
             const int m = 32 * (warp & 3) + lane;
@@ -194,7 +202,13 @@ __global__ void __launch_bounds__(NTHR, NST == 256 ? 2 : 3)  // CTAs per SM that
             for (int col = 0; col < HALF; col += 32) {
                 float v[32];
                 tmem_ld32(tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16) + cbeg + col, v);
-                if (p.states_f32) {  // fp32 states, as the forward keeps them
+                if (NST <= 128 && tma_out) {
+                    const uint32_t dst = s0 + ((cbeg + col) / 32) * (128 * 128);
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        st_shared_v4(dst + sw128(m, k), __float_as_uint(v[4 * k]), __float_as_uint(v[4 * k + 1]),
+                                     __float_as_uint(v[4 * k + 2]), __float_as_uint(v[4 * k + 3]));
+                } else if (p.states_f32) {  // fp32 states, as the forward keeps them
                     float4* o = reinterpret_cast<float4*>(static_cast<float*>(p.states) + row + cbeg + col);
 #pragma unroll
                     for (int k = 0; k < 8; ++k)
@@ -210,6 +224,17 @@ __global__ void __launch_bounds__(NTHR, NST == 256 ? 2 : 3)  // CTAs per SM that
                 }
             }
         }
+        if (NST <= 128 && tma_out) {
+            fence_smem_async();     // the staged tile is read by the TMA (async proxy)
+            named_sync(2, NSCALE);  // every row is staged
+            if (tid == 0 && ok && !*abort) {
+                const int row0 = static_cast<int>(((b * nc + c) * H + h0) * PD);
+                for (int box = 0; box < NST / 32; ++box)
+                    tma_store_2d(&tm_s, s0 + box * (128 * 128), box * 32, row0);
+                bulk_commit_group();
+                bulk_wait_all();  // written before the CTA ends (and its shared memory with it)
+            }
+        }
     }
     fence_before_sync();
     __syncthreads();
@@ -223,15 +248,24 @@ __global__ void __launch_bounds__(NTHR, NST == 256 ? 2 : 3)  // CTAs per SM that
 template <int NST, int PD>
 cudaError_t launch_nd(const FwdParams& p, cudaStream_t s) {
     using T = StateTile<NST, PD>;
-    CUtensorMap tx_, tb_;
+    CUtensorMap tx_, tb_, ts_;
     if (!make_tmap_bf16_4d(&tx_, p.x, 64, p.nheads * PD / 64, p.seqlen, p.batch, 1, KT) ||
         !make_tmap_bf16_4d(&tb_, p.B, NST, p.ngroups, p.seqlen, p.batch, 1, KT))
         return cudaErrorInvalidValue;
+    // the fp32 states as rows of NST: [batch * nchunks * nheads * headdim][NST]
+    // (row coordinates are 32-bit)
+    const int64_t srows = p.batch * p.nchunks * p.nheads * PD;
+    const int tma_out = (NST <= 128 && p.states_f32 && srows < (1ll << 31)) ? 1 : 0;
+    if (tma_out) {
+        if (!make_tmap_f32_2d(&ts_, p.states, NST, srows, 128)) return cudaErrorInvalidValue;
+    } else {
+        ts_ = tx_;  // not read
+    }
     auto kern = chunk_state_tc_kernel<NST, PD>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, T::SMEM);
     if (e != cudaSuccess) return e;
     dim3 grid(static_cast<unsigned>(p.nchunks * (p.nheads / T::HPC)), static_cast<unsigned>(p.batch));
-    return launch_kernel(kern, grid, dim3(NTHR), T::SMEM, s, p.pdl != 0, p, tx_, tb_);
+    return launch_kernel(kern, grid, dim3(NTHR), T::SMEM, s, p.pdl != 0, p, tx_, tb_, ts_, tma_out);
 }
 
 }  // namespace

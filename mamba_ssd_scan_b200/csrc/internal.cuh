@@ -170,8 +170,12 @@ cudaError_t launch_kernel(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t 
 // "MAMBA-2 Reference Implementations Comparison", section 3.2 (softplus
 // discretisation of dt and the exp(A dt) decays whose exponents this sums).
 template <typename T>
+// When wout is given (shared memory, 8 x 32 = 256 entries), the warp also writes
+// each token's decay weight e^{cumA[last] - cumA[l]} dt[l] there (0 past the end):
+// the chunk_state weights, without reading back what it just stored.
 __device__ __forceinline__ void chunk_cumsum_warp(const FwdParams& p, int64_t b, int64_t c, int64_t h,
-                                                  float* dt_out, float* cum_out, int lane) {
+                                                  float* dt_out, float* cum_out, int lane,
+                                                  float* wout = nullptr) {
     constexpr int MAXSEG = 8;  // chunk <= 256 tokens
     const int64_t Q = p.chunk, H = p.nheads, L = p.seqlen;
     const int64_t t0 = c * Q;
@@ -187,9 +191,12 @@ __device__ __forceinline__ void chunk_cumsum_warp(const FwdParams& p, int64_t b,
         u[s] = (s < nseg && l < Lc) ? to_f32(dtr[l * H]) : 0.0f;
     }
     float carry = 0.0f;
+    float dts[MAXSEG], cums[MAXSEG];
 #pragma unroll
     for (int s = 0; s < MAXSEG; ++s) {
-        if (s >= nseg) break;
+        dts[s] = 0.0f;
+        cums[s] = 0.0f;
+        if (s >= nseg) continue;
         const int64_t l = s * 32 + lane;
         float dt = 0.0f, v = 0.0f;
         if (l < Lc) {
@@ -206,7 +213,19 @@ __device__ __forceinline__ void chunk_cumsum_warp(const FwdParams& p, int64_t b,
             dt_out[l] = dt;
             cum_out[l] = v;
         }
+        dts[s] = dt;
+        cums[s] = v;
         carry = __shfl_sync(0xffffffffu, v, 31);
+    }
+    if (wout) {
+        // carry is now cumA[last] (entries past the end repeat it); every one
+        // of the QMAX entries is written, 0 past the chunk's end, since the
+        // weights are read in whole 64-token quarters
+#pragma unroll
+        for (int s = 0; s < MAXSEG; ++s) {
+            const int64_t l = s * 32 + lane;
+            wout[l] = (s < nseg && l < Lc) ? expf(carry - cums[s]) * dts[s] : 0.0f;
+        }
     }
 }
 

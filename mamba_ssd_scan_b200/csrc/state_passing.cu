@@ -114,7 +114,7 @@ __global__ void __launch_bounds__(256) state_passing_kernel(FwdParams p) {
 // The hi / lo form: fp32 local states in, each entering state out as two
 // bf16 arrays (hi = bf16(H), lo = bf16(H - hi); H - hi is exact in fp32).
 // Each thread carries 8 consecutive state elements: two 16-byte loads per
-// chunk, one 16-byte store of each half.
+// chunk (four chunks' loads in flight), one 16-byte store of each half.
 constexpr int HL_UNROLL = 4;
 
 __device__ __forceinline__ void split_store(__nv_bfloat16* hi, __nv_bfloat16* lo, const float (&v)[8]) {

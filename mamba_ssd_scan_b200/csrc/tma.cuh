@@ -18,6 +18,10 @@ namespace ssd {
 // rejects the arguments.
 bool make_tmap_bf16_4d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1,
                        uint64_t d2, uint64_t d3, uint32_t box1, uint32_t box2);
+// A 2-D fp32 tensor [d1][d0] (d0 innermost, a multiple of 4 elements) read or
+// written in boxes of {32, box1} elements with the 128-byte swizzle: box1
+// 128-byte rows in the SW128 layout.
+bool make_tmap_f32_2d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint32_t box1);
 
 namespace tc {
 
@@ -49,6 +53,14 @@ __device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, uint32_t sr
         :
         : "l"(reinterpret_cast<uint64_t>(map)), "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
         : "memory");
+}
+// One box from shared memory to a 2-D tensor in global memory (bulk async
+// group of the issuing thread).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int c0, int c1) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];"
+                 :
+                 : "l"(reinterpret_cast<uint64_t>(map)), "r"(src), "r"(c0), "r"(c1)
+                 : "memory");
 }
 // One contiguous run of `bytes` from global into shared memory (both
 // addresses 16-byte aligned, bytes a multiple of 16); completes `bytes` on

@@ -40,4 +40,16 @@ bool make_tmap_bf16_4d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t
            CUDA_SUCCESS;
 }
 
+bool make_tmap_f32_2d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint32_t box1) {
+    EncodeTiledFn fn = encoder();
+    if (!fn || box1 == 0 || box1 > 256 || d0 < 32 || d0 % 4 != 0) return false;
+    const cuuint64_t dims[2] = {d0, d1};
+    const cuuint64_t strides[1] = {d0 * 4};
+    const cuuint32_t box[2] = {32, box1};
+    const cuuint32_t estr[2] = {1, 1};
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace ssd
