@@ -425,12 +425,12 @@ def main_ours(args):
         "config": {"workload": cfg.name, "batch": cfg.batch, "seqlen": cfg.seqlen,
                    "nheads": cfg.nheads, "headdim": cfg.headdim, "dstate": cfg.dstate,
                    "ngroups": cfg.ngroups, "chunk": cfg.chunk,
-                   "kernels": "single pass" if "fused" in tc else "three kernels",
                    "global_batch":
                    cfg.batch * world, "parallelism": f"dp{world}" if world > 1 else "single",
                    "l2": f"inputs {input_bytes(inp) / 1e6:.0f} MB; L2 flushed before every "
                          f"timed step ({args.flush_mb} MB write, then a read of it, so its "
                          "write-back ends before the timed region)"},
+        "path": "single pass" if "fused" in tc else "three kernels",
         "roofline": roofline,
         "kernel_ms": kms,
         "e2e": e2e,
