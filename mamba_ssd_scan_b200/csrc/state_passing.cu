@@ -131,7 +131,12 @@ __device__ __forceinline__ void split_store(__nv_bfloat16* hi, __nv_bfloat16* lo
     *reinterpret_cast<uint4*>(lo) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
 }
 
-__global__ void __launch_bounds__(256) state_passing_hl_kernel(FwdParams p) {
+// 128-thread blocks, five per SM (<= 102 registers): at seqlen 65536 all 640
+// blocks are resident at once (with 256-thread blocks at 95 registers only
+// two fit an SM and the last 24 of 320 ran as a second wave).
+constexpr int HL_THREADS = 128;
+
+__global__ void __launch_bounds__(HL_THREADS, 5) state_passing_hl_kernel(FwdParams p) {
     grid_dep_wait();  // the local states and cumA come from the previous steps
     grid_dep_launch();
     const int64_t H = p.nheads, nc = p.nchunks, Q = p.chunk;
@@ -191,8 +196,8 @@ template <typename T>
 cudaError_t launch_state_passing(const FwdParams& p, cudaStream_t s) {
     if (p.states_hl) {
         const int64_t n = p.batch * p.nheads * p.headdim * p.dstate / 8;
-        return launch_kernel(state_passing_hl_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s,
-                             p.pdl != 0, p);
+        return launch_kernel(state_passing_hl_kernel, dim3((unsigned)((n + HL_THREADS - 1) / HL_THREADS)),
+                             dim3(HL_THREADS), 0, s, p.pdl != 0, p);
     }
     const int64_t n = p.batch * p.nheads * p.headdim * p.dstate / Pack<T>::E;
     return launch_kernel(state_passing_kernel<T>, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s,
