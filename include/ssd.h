@@ -15,9 +15,11 @@
  * of a group (head h reads group h / (nheads / ngroups)).  The forward pass
  * computes this chunkwise, the chunked SSD of "MAMBA-2 Implementation Gaps",
  * Gap 1: chunk_cumsum -> chunk_state -> state_passing -> chunk_scan.  For bf16
- * inputs in its range the four steps run as one fused kernel (the carried
- * state stays fp32 and crosses between chunks through a small ring in the
- * workspace); otherwise as the four step kernels below.
+ * inputs the first two steps run as one tensor-core kernel and the last as
+ * another, the chunk states staying fp32 in the workspace (they reach the
+ * tensor cores as bf16 hi + lo halves); SSD_FLAG_SINGLE_PASS runs all four as
+ * one kernel instead (the carried state stays fp32 and crosses between tiles
+ * on chip and through a small ring in the workspace).
  *
  * Layouts: row-major, innermost index last, densely packed (no strides):
  *   x, y          [batch, seqlen, nheads, headdim]     dtype
@@ -501,7 +503,7 @@ const char* ssd_version(void);
  * one hand-off, so the consumers' bounded waits run out and the kernel reports
  * SSD_ERR_TIMEOUT through its status word instead of hanging (no fault, no
  * trap).  `what` = SSD_DEBUG_CONV_TILE: the convolution's producer stops before
- * tile `index`; SSD_DEBUG_FWD_CARRY: the fused forward does not publish the
+ * tile `index`; SSD_DEBUG_FWD_CARRY: the single-pass forward does not publish the
  * state leaving run `index` (a run is the group of up to four consecutive
  * 128-token tiles one cluster of CTAs takes; the next run's wait gives up
  * after about a second; SSD_FLAG_SINGLE_PASS only); SSD_DEBUG_SCAN_DECAYS: the
