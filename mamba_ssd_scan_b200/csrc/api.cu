@@ -60,7 +60,7 @@ bool bf16_states(const ssd_fwd_args& a) {
 // the entering states as hi / lo bf16 halves, the operand that kernel takes.
 bool states_hilo(const ssd_fwd_args& a) {
     if (!use_tc(a.dtype, a.flags) || bf16_states(a)) return false;
-    ssd::FwdParams q;
+    ssd::FwdParams q{};  // only the sizes the support check reads
     q.headdim = a.headdim;
     q.dstate = a.dstate;
     q.chunk = a.chunk;
